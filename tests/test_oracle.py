@@ -1,0 +1,292 @@
+"""Pins of the float64 oracle against things other than itself.
+
+Each test checks the oracle against a library routine, a closed form, a
+hand-derived fixture or brute force, so that a plausible slip in it (a dropped
+term, a wrong sign or index, a swapped operand) fails at least one of them.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_token_b200 import workloads
+from _util import bf16_bits, read_cases
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+# ---------------------------------------------------------------- formats
+def test_e4m3_decode_matches_torch_for_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_to_f64(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan) and nan.sum() == 2
+    assert np.array_equal(ours[~nan], ref[~nan])
+
+
+def test_e4m3_decode_spec_points():
+    # OCP E4M3: 0x7E is the largest finite value 448, 0x01 the smallest
+    # subnormal 2^-9, 0x08 the smallest normal 2^-6, 0x38 is 1.0.
+    v = oracle.e4m3_to_f64(np.array([0x7E, 0x01, 0x08, 0x38, 0xB8, 0x00, 0x80], np.uint8))
+    assert list(v[:5]) == [448.0, 2.0 ** -9, 2.0 ** -6, 1.0, -1.0]
+    assert v[5] == 0.0 and v[6] == 0.0
+
+
+def test_bf16_widening_matches_torch():
+    x = torch.randn(4096, generator=torch.Generator().manual_seed(1)) * 7
+    b = x.to(torch.bfloat16)
+    ours = oracle.bf16_to_f64(b.view(torch.int16).numpy().view(np.uint16))
+    assert np.array_equal(ours, b.to(torch.float64).numpy())
+
+
+# ------------------------------------------------------ full attention
+def _sdpa(q, k, v, scale, mask=None):
+    """torch's scaled_dot_product_attention in float64: q [h, d], k/v [n, d]."""
+    out = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(k)[None], torch.from_numpy(v)[None],
+        attn_mask=None if mask is None else torch.from_numpy(mask)[None], scale=scale)
+    return out[0].numpy()
+
+
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+def test_full_attention_matches_library_sdpa_with_causal_queries(kv):
+    inp = workloads.make_inputs(2, 300, n_q=5, h_q=16, kv=kv, seed=3, lens=[300, 211])
+    bits = workloads.numpy_bits(inp)
+    res = oracle.full_attn_select(bits)
+    q = oracle.bf16_to_f64(bits["q"])
+    for b in range(2):
+        L = int(bits["lens"][b])
+        k = oracle.widen_cache(bits["k"][b, :L], kv, None if kv == "bf16" else bits["k_scale"][b, :L])
+        v = oracle.widen_cache(bits["v"][b, :L], kv, None if kv == "bf16" else bits["v_scale"][b, :L])
+        for i in range(5):
+            p = L - 5 + i
+            mask = np.zeros((16, L), dtype=bool)
+            mask[:, :p + 1] = True
+            ref = _sdpa(q[b, i], k, v, bits["sm_scale"], mask)
+            np.testing.assert_allclose(res["out"][b, i], ref, rtol=0, atol=1e-12)
+            s = bits["sm_scale"] * q[b, i] @ k[:p + 1].T
+            lse_ref = torch.logsumexp(torch.from_numpy(s), dim=1).numpy()
+            np.testing.assert_allclose(res["lse"][b, i], lse_ref, rtol=0, atol=1e-12)
+
+
+def test_softmax_rows_sum_to_one():
+    rng = np.random.default_rng(0)
+    q, k, v = rng.standard_normal((8, 128)), rng.standard_normal((500, 128)), rng.standard_normal((500, 128))
+    _, lse, P, _ = oracle.attend(q, k, v, 0.3)
+    np.testing.assert_allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    assert np.all(P > 0)
+
+
+def test_zero_query_gives_mean_value_and_log_length():
+    inp = workloads.make_inputs(1, 777, n_q=1, h_q=16, seed=5, q_zero=True)
+    bits = workloads.numpy_bits(inp)
+    res = oracle.full_attn_select(bits)
+    v = oracle.bf16_to_f64(bits["v"][0])
+    np.testing.assert_allclose(res["out"][0, 0], np.broadcast_to(v.mean(axis=0), (16, 128)), atol=1e-13)
+    np.testing.assert_allclose(res["lse"][0, 0], math.log(777), atol=1e-13)
+
+
+def test_identical_keys_give_uniform_attention():
+    inp = workloads.make_inputs(1, 400, n_q=1, h_q=16, seed=6, identical_keys=True)
+    bits = workloads.numpy_bits(inp)
+    res = oracle.full_attn_select(bits)
+    q = oracle.bf16_to_f64(bits["q"][0, 0])
+    k0 = oracle.bf16_to_f64(bits["k"][0, 0])
+    v = oracle.bf16_to_f64(bits["v"][0])
+    np.testing.assert_allclose(res["out"][0, 0], np.broadcast_to(v.mean(axis=0), (16, 128)), atol=1e-13)
+    np.testing.assert_allclose(res["lse"][0, 0], bits["sm_scale"] * q @ k0 + math.log(400), atol=1e-12)
+
+
+# ------------------------------------------------------------ selection
+def _bits_from_case(c):
+    L, W, K = c["len"][0], c["window"][0], c["k_sel"][0]
+    x, y = np.array(c["x"], float), np.array(c["y"], float)
+    q = np.zeros((1, 1, 2, 128), np.float32)
+    q[0, 0, 0, 0] = 2.0
+    q[0, 0, 1, 1] = 2.0
+    k = np.zeros((1, L, 128), np.float32)
+    k[0, :, 0], k[0, :, 1] = x, y
+    v = np.zeros((1, L, 128), np.float32)
+    v[0, np.arange(L), np.arange(L)] = 1.0
+    return dict(q=bf16_bits(q), k=bf16_bits(k), v=bf16_bits(v), k_scale=None, v_scale=None,
+                lens=np.array([L]), sm_scale=0.5, window=W, k_sel=K, kv="bf16",
+                q_layers=[])
+
+
+@pytest.mark.parametrize("case", read_cases("selection_cases.txt"), ids=lambda c: c["name"])
+def test_golden_selection_cases(case):
+    bits = _bits_from_case(case)
+    res = oracle.full_attn_select(bits)
+    assert res["idx"][0, 0].tolist() == case["expected_idx"]
+    # closed forms: y is a permutation of x, so both heads share lse = ln sum e^x,
+    # and with one-hot values out_h[j] = exp(s_hj - lse).
+    x, y = np.array(case["x"], float), np.array(case["y"], float)
+    lse = math.log(np.exp(x).sum())
+    np.testing.assert_allclose(res["lse"][0, 0], [lse, lse], atol=1e-14)
+    L = case["len"][0]
+    np.testing.assert_allclose(res["out"][0, 0, 0, :L], np.exp(x - lse), atol=1e-15)
+    np.testing.assert_allclose(res["out"][0, 0, 1, :L], np.exp(y - lse), atol=1e-15)
+
+
+def _brute_force_selection(q, k, sm_scale, p, W, K):
+    """Selection of one query by definition, on tiny inputs: probabilities from
+    torch.softmax (float64); key j is chosen iff fewer than K outside keys rank
+    strictly before it in (importance desc, position asc)."""
+    s = torch.from_numpy(sm_scale * q @ k[:p + 1].T)
+    P = torch.softmax(s, dim=1).numpy()
+    w_lo = max(0, p - W + 1)
+    imp = [max(P[h, j] for h in range(P.shape[0])) for j in range(w_lo)]
+    chosen = []
+    for j in range(w_lo):
+        rank = sum(1 for jj in range(w_lo) if imp[jj] > imp[j] or (imp[jj] == imp[j] and jj < j))
+        if rank < K:
+            chosen.append(j)
+    return sorted(set(chosen) | set(range(w_lo, p + 1)))
+
+
+@pytest.mark.parametrize("h", [1, 3, 16])
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_selection_matches_brute_force_on_tiny_inputs(h, seed):
+    W, K = 4, 8
+    L = [48, 13, 9][seed]
+    inp = workloads.make_inputs(1, 48, n_q=3, h_q=h, seed=20 + seed, lens=[L], window=W, k_sel=K)
+    bits = workloads.numpy_bits(inp)
+    res = oracle.full_attn_select(bits)
+    q = oracle.bf16_to_f64(bits["q"][0])
+    k = oracle.bf16_to_f64(bits["k"][0, :L])
+    for i in range(3):
+        p = L - 3 + i
+        want = _brute_force_selection(q[i], k, bits["sm_scale"], p, W, K)
+        got = res["idx"][0, i]
+        assert got[got >= 0].tolist() == want
+        assert np.all(got[len(want):] == -1)
+
+
+def test_single_head_selection_is_argsort_of_logits():
+    # With one head, lse is a common shift, so importance order = logit order.
+    inp = workloads.make_inputs(1, 3000, n_q=1, h_q=1, seed=8, window=128, k_sel=1024)
+    bits = workloads.numpy_bits(inp)
+    res = oracle.full_attn_select(bits)
+    q = oracle.bf16_to_f64(bits["q"][0, 0, 0])
+    k = oracle.bf16_to_f64(bits["k"][0])
+    s = k[:3000 - 128] @ q
+    top = np.argsort(-s, kind="stable")[:1024]
+    want = np.sort(np.concatenate([top, np.arange(3000 - 128, 3000)]))
+    assert np.array_equal(res["idx"][0, 0], want)
+
+
+def test_zero_query_ties_go_to_lowest_positions():
+    inp = workloads.make_inputs(1, 5000, n_q=2, h_q=16, seed=9, q_zero=True)
+    bits = workloads.numpy_bits(inp)
+    res = oracle.full_attn_select(bits)
+    for i in range(2):
+        p = 5000 - 2 + i
+        want = np.concatenate([np.arange(1024), np.arange(p - 127, p + 1)])
+        assert np.array_equal(res["idx"][0, i], want)
+
+
+def test_planted_needles_are_selected_and_window_present():
+    w = workloads.WORKLOADS[1]
+    inp = workloads.generate(w)
+    bits = workloads.numpy_bits(inp)
+    res = oracle.full_attn_select(bits)
+    idx = res["idx"][0, 0]
+    L = int(bits["lens"][0])
+    assert len(inp.needles[0]) == 8
+    for pos, _ in inp.needles[0]:
+        assert pos in idx
+    assert np.all(np.isin(np.arange(L - 128, L), idx))
+    assert np.count_nonzero(idx >= 0) == 1152 and np.all(np.diff(idx) > 0)
+
+
+@pytest.mark.parametrize("L", [1, 2, 127, 128, 129, 1151, 1152, 1153, 1300])
+def test_index_set_size_window_and_order(L):
+    inp = workloads.make_inputs(1, 1300, n_q=1, h_q=16, seed=10, lens=[L])
+    bits = workloads.numpy_bits(inp)
+    idx = oracle.full_attn_select(bits)["idx"][0, 0]
+    p = L - 1
+    nvalid = min(p + 1, 1152)
+    assert np.all(idx[:nvalid] >= 0) and np.all(idx[nvalid:] == -1)
+    assert np.all(np.diff(idx[:nvalid]) > 0) and idx[nvalid - 1] == p
+    assert np.all(np.isin(np.arange(max(0, p - 127), p + 1), idx))
+
+
+# ------------------------------------------------------------ sparse layers
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+def test_sparse_equals_full_when_budget_covers_context(kv):
+    inp = workloads.make_inputs(2, 1152, n_q=2, h_q=16, kv=kv, n_sparse=1, seed=11, lens=[1152, 700])
+    bits = workloads.numpy_bits(inp)
+    full = oracle.full_attn_select(bits)
+    # A sparse layer that reuses the full layer's own queries must reproduce it.
+    out = oracle.sparse_attn(bits, bits["q"], full["idx"])
+    np.testing.assert_allclose(out, full["out"], rtol=0, atol=1e-12)
+
+
+def test_sparse_matches_library_sdpa_on_gathered_rows():
+    inp = workloads.make_inputs(1, 6000, n_q=1, h_q=16, kv="fp8", n_sparse=1, seed=12)
+    bits = workloads.numpy_bits(inp)
+    full = oracle.full_attn_select(bits)
+    out = oracle.sparse_attn(bits, bits["q_layers"][0], full["idx"])
+    sel = full["idx"][0, 0]
+    sel = sel[sel >= 0]
+    k = oracle.e4m3_to_f64(bits["k"][0, sel]) * bits["k_scale"][0, sel].astype(np.float64)[:, None]
+    v = oracle.e4m3_to_f64(bits["v"][0, sel]) * bits["v_scale"][0, sel].astype(np.float64)[:, None]
+    ref = _sdpa(oracle.bf16_to_f64(bits["q_layers"][0][0, 0]), k, v, bits["sm_scale"])
+    np.testing.assert_allclose(out[0, 0], ref, rtol=0, atol=1e-12)
+
+
+# -------------------------------------------- the pins catch planted mistakes
+def _swap(monkeypatch, name, fn):
+    monkeypatch.setattr(oracle.hs2_oracle, name, fn)
+
+
+def test_pins_catch_min_over_heads(monkeypatch):
+    _swap(monkeypatch, "importance", lambda s, lse: np.exp(s - lse[:, None]).min(axis=0))
+    with pytest.raises(AssertionError):
+        test_selection_matches_brute_force_on_tiny_inputs(3, 0)
+
+
+def test_pins_catch_unnormalised_importance(monkeypatch):
+    _swap(monkeypatch, "importance", lambda s, lse: np.exp(s).max(axis=0))
+    with pytest.raises(AssertionError):
+        test_selection_matches_brute_force_on_tiny_inputs(16, 0)
+
+
+def test_pins_catch_reversed_tie_break(monkeypatch):
+    def bad(imp, k):
+        n = imp.shape[0]
+        return np.lexsort((-np.arange(n), -imp))[:min(k, n)]
+    _swap(monkeypatch, "select_top", bad)
+    with pytest.raises(AssertionError):
+        test_zero_query_ties_go_to_lowest_positions()
+
+
+def test_pins_catch_window_off_by_one(monkeypatch):
+    orig = oracle.hs2_oracle.index_set
+
+    def bad(p, imp, window, k_sel):
+        return orig(p, imp, window, k_sel) if p < window else np.concatenate(
+            [orig(p, imp, window, k_sel)[1:], [-1]])
+    _swap(monkeypatch, "index_set", bad)
+    with pytest.raises(AssertionError):
+        test_index_set_size_window_and_order(1300)
+
+
+def test_pins_catch_dropped_scale(monkeypatch):
+    orig = oracle.hs2_oracle.attend
+    _swap(monkeypatch, "attend", lambda q, k, v, sc: orig(q, k, v, 1.0))
+    with pytest.raises(AssertionError):
+        test_full_attention_matches_library_sdpa_with_causal_queries("bf16")
+
+
+def test_pins_catch_dropped_fp8_scale(monkeypatch):
+    def bad(rows, kv, scale=None):
+        return oracle.bf16_to_f64(rows) if kv == "bf16" else oracle.e4m3_to_f64(rows)
+    _swap(monkeypatch, "widen_cache", bad)
+    with pytest.raises(AssertionError):
+        test_sparse_matches_library_sdpa_on_gathered_rows()
