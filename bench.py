@@ -1,0 +1,371 @@
+"""Benchmark of the hybrid-block decode step (full layer + selection + sparse layers).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl hs2|reference]
+
+One step = hs2_full_attn (split-K flash-decode) + hs2_select (importance, exact
+top-k, window merge) + one hs2_sparse_attn per reusing layer, for every sequence
+of the batch, on device-resident synthetic inputs.  L2 is flushed (256 MiB write)
+before every timed step, outside the timed interval.  Rank 0 prints one JSON line.
+
+With N > 1 (torchrun), every rank runs an independent replica of the workload on
+its own GPU (the step has no exchange between sequences): weak scaling.
+``--impl reference`` times the float64 CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from long_context_token_b200 import workloads  # noqa: E402
+
+METRIC = "hybrid-block decode steps/s & HBM GB/s (full+select+sparse) at 128K-1M ctx"
+UNIT = "steps/s"
+FLUSH_BYTES = 256 << 20
+LAUNCHES_PER_STEP_FULL = 1      # split-K flash-decode (+ merge in its last CTA)
+LAUNCHES_PER_STEP_SELECT = 3    # importance+histogram, compaction, exact finish
+LAUNCHES_PER_SPARSE = 1
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def alg_bytes(w: workloads.Workload, lens) -> dict:
+    """Bytes the method must move per step (see the design notes): K and V of every
+    visible row once, each sparse layer's gathered rows, indices, queries, outputs."""
+    d = 128
+    elem = 1 if w.kv == "fp8" else 2
+    row = d * elem + (4 if w.kv == "fp8" else 0)      # one K (or V) row incl. its scale
+    ctx_rows = int(sum(int(L) for L in lens))
+    width = w.window + w.k_sel
+    sel_rows = sum(min(int(L) - w.n_q + i + 1, width) for L in lens for i in range(w.n_q))
+    q_bytes = w.batch * w.n_q * w.h_q * d * 2
+    out_bytes = w.batch * w.n_q * w.h_q * d * 4
+    full = 2 * ctx_rows * row + q_bytes + out_bytes
+    idx_bytes = w.batch * w.n_q * width * 4
+    sparse = 2 * sel_rows * row + idx_bytes + q_bytes + out_bytes
+    return dict(full=full, step=full + idx_bytes + w.n_sparse * sparse, sparse=sparse,
+                kv_once=2 * ctx_rows * row)
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed loop runs."""
+
+    def __init__(self, device: torch.device):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: report no clocks rather than guess
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        names = {
+            "hw_slowdown": getattr(nv, "nvmlClocksThrottleReasonHwSlowdown", 0x8),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksThrottleReasonSwThermalSlowdown", 0x20),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksThrottleReasonHwThermalSlowdown", 0x40),
+            "sw_power_cap": getattr(nv, "nvmlClocksThrottleReasonSwPowerCap", 0x4),
+            "hw_power_brake": getattr(nv, "nvmlClocksThrottleReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                for k, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            self._stop.wait(0.05)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def oracle_sample(inp: workloads.Inputs, w: workloads.Workload, budget_s: float):
+    """Time the float64 oracle on whole sequences of the workload until `budget_s`
+    has passed (at least one).  Returns (seconds, sequences done)."""
+    import oracle
+    bits = workloads.numpy_bits(inp)
+    t0 = time.perf_counter()
+    done = 0
+    while True:
+        b = done % w.batch
+        sub = dict(bits)
+        for key in ("q", "k", "v", "k_scale", "v_scale", "lens"):
+            if sub[key] is not None:
+                sub[key] = bits[key][b:b + 1]
+        sub["q_layers"] = [ql[b:b + 1] for ql in bits["q_layers"]]
+        oracle.hybrid_block_step(sub)
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    return time.perf_counter() - t0, done
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args, w):
+    """The reference arm: the float64 CPU oracle, each step one sequence of the batch."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    inp = workloads.generate(w)
+    for _ in range(args.warmup):
+        oracle_sample(inp, w, 0.0)
+    secs, seqs = 0.0, 0
+    for _ in range(args.steps):
+        s, n = oracle_sample(inp, w, 0.0)
+        secs += s
+        seqs += n
+    value = seqs / (secs * w.batch)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+                         "sample": f"{seqs} whole sequences of the batch, one per step, "
+                                   "full layer + selection + every sparse layer in float64"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w):
+    return {"workload": w.name, "batch": w.batch, "context": w.max_len,
+            "ragged_from": w.len_lo, "n_q": w.n_q, "h_q": w.h_q, "h_kv": 1, "head_dim": 128,
+            "kv_cache": w.kv, "window": w.window, "k_sel": w.k_sel, "sparse_layers": w.n_sparse,
+            "l2": "flushed before every timed step (256 MiB write)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=2, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="hs2", choices=["hs2", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0,
+                    help="seconds of oracle time for the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = workloads.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    from long_context_token_b200 import hs2
+    world, rank, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    inp = workloads.generate(w)
+    cache = hs2.Cache(inp.k.to(dev), inp.v.to(dev), inp.lens.to(dev),
+                      None if inp.k_scale is None else inp.k_scale.to(dev),
+                      None if inp.v_scale is None else inp.v_scale.to(dev))
+    q = inp.q.to(dev)
+    qls = [x.to(dev) for x in inp.q_layers]
+    B, n_q, h = w.batch, w.n_q, w.h_q
+    width = w.window + w.k_sel
+    ws = hs2.alloc_workspace(cache, n_q, h, w.window, w.k_sel)
+    out = torch.empty(B, n_q, h, 128, dtype=torch.float32, device=dev)
+    lse = torch.empty(B, n_q, h, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, n_q, width, dtype=torch.int32, device=dev)
+    outs = [torch.empty_like(out) for _ in qls]
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        hs2.full_attn(q, cache, w.window, w.k_sel, inp.sm_scale, ws, out=out, lse=lse)
+        if evs:
+            evs[1].record(stream)
+        hs2.select(q, cache, ws, w.window, w.k_sel, inp.sm_scale, idx=idx)
+        if evs:
+            evs[2].record(stream)
+        for ql, o in zip(qls, outs):
+            hs2.sparse_attn(ql, cache, idx, ws, inp.sm_scale, out=o)
+        if evs:
+            evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    if hs2.check_device_status(ws) != 0:
+        raise RuntimeError("device-side error during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    with ClockSampler(dev) as clk:
+        for k in range(args.steps):
+            flush.fill_(float(k))
+            step(evs[k])
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    wall = time.perf_counter() - wall0
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    full_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    sel_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    sp_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    status = hs2.check_device_status(ws)
+
+    # End to end through the public API: queries from pinned host memory in, outputs out.
+    e2e = None
+    if not args.no_e2e:
+        hq = inp.q.pin_memory()
+        hqls = [x.pin_memory() for x in inp.q_layers]
+        hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        hidx = torch.empty(idx.shape, dtype=torch.int32).pin_memory()
+        houts = [torch.empty(out.shape, dtype=torch.float32).pin_memory() for _ in qls]
+        h2d = hq.numel() * 2 + sum(x.numel() * 2 for x in hqls)
+        d2h = hout.numel() * 4 + hidx.numel() * 4 + sum(x.numel() * 4 for x in houts)
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            for d_, h_ in zip(qls, hqls):
+                d_.copy_(h_, non_blocking=True)
+            hs2.full_attn_select(q, cache, w.window, w.k_sel, inp.sm_scale, ws, out=out,
+                                 idx=idx, lse=lse)
+            for ql, o in zip(qls, outs):
+                hs2.sparse_attn(ql, cache, idx, ws, inp.sm_scale, out=o)
+            hout.copy_(out, non_blocking=True)
+            hidx.copy_(idx, non_blocking=True)
+            for h_, o in zip(houts, outs):
+                h_.copy_(o, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        e_ms = 0.0
+        for k in range(args.steps):
+            flush.fill_(float(k))
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            e2e_step()
+            b.record(stream)
+            b.synchronize()
+            e_ms += a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * args.steps / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    lens = inp.lens.tolist()
+    ab = alg_bytes(w, lens)
+    peaks, peak_kind = measured_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    full_avg = statistics.mean(full_ms) / 1e3
+    achieved = ab["full"] / full_avg / 1e9
+    value = world * args.steps / (total_ms / 1e3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.kv == "bf16" else "fp8-e4m3",
+        "data": "synthetic", "config": config_of(w),
+        "hbm_gbs": ab["step"] / (total_ms / args.steps / 1e3) / 1e9,
+        "alg_bytes_per_step": ab["step"],
+        "phase_ms": {"full_attn": statistics.mean(full_ms), "select": statistics.mean(sel_ms),
+                     "sparse_layers": statistics.mean(sp_ms),
+                     "step_p10": float(np.percentile(step_ms, 10)),
+                     "step_p50": float(np.percentile(step_ms, 50)),
+                     "step_p90": float(np.percentile(step_ms, 90))},
+        "roofline": {"bound": "hbm", "kernel": "full_attn (split-K flash-decode)",
+                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "peak_kind": peak_kind,
+                     "alg_bytes_per_launch": ab["full"], "traffic": None},
+        "gpu_launches": args.steps * (LAUNCHES_PER_STEP_FULL + LAUNCHES_PER_STEP_SELECT
+                                      + w.n_sparse * LAUNCHES_PER_SPARSE),
+        "clocks": clk.summary(),
+        "device_status": status,
+        "wall_s_timed_region": wall,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if not args.no_cpu_baseline:
+        secs, seqs = oracle_sample(inp, w, args.cpu_budget)
+        cv = seqs / (secs * w.batch)
+        line["cpu_baseline"] = {"value": cv, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+                                "sample": f"{seqs} of the {w.batch} sequences of one step "
+                                          f"({secs:.1f} s), float64 numpy oracle"}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

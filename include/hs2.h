@@ -1,0 +1,164 @@
+/*
+ * hs2.h -- C ABI of libhs2, the decode step of a HySparse2 Cross-Decoder hybrid
+ * block on NVIDIA B200 (sm_100a).
+ *
+ * The step (sources: web coverage of the HySparse2 architecture paper):
+ *   1. a full-attention layer with one shared K/V head and h_q query heads (MQA)
+ *      attends over the whole context and scores every key
+ *      (toolnavs article 2080, fr "Ce que fait HySparse2", KV Reuse paragraph;
+ *       "Les chiffres mesurés" for MQA);
+ *   2. token-level selection keeps the most recent `window` (128) positions and
+ *      the top `k_sel` (1024) positions outside that window
+ *      (same article, fr/ko, paragraph on selection granularity; "Luo Fuli Teases
+ *       Xiaomi MiMo-V3 Architecture: HySparse2 Enables Early Prefill Exit",
+ *       paragraph on token granularity);
+ *   3. each following sparse-attention layer, with its own queries, attends only
+ *      to those positions of the same KV cache (same article, KV Reuse paragraph).
+ * The pages give no importance formula.  This library takes a key's importance as
+ * max over query heads h of exp(s_hj - lse_h), the full layer's softmax
+ * probability, with ties going to the lower position.
+ *
+ * Conventions shared by every call
+ *   - Pointers named "device" point to device memory of the current CUDA device.
+ *     The caller owns all memory; the library allocates nothing and keeps no
+ *     pointer after a call returns.
+ *   - Every compute call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and enqueues only kernels and memsets, so it can be
+ *     captured in a CUDA graph.
+ *   - Host-side validation failures return an error before anything is enqueued.
+ *     Launch failures return HS2_ERR_CUDA.  Errors found by the kernels (a bad
+ *     length, an index out of range) are recorded in the workspace's status word
+ *     and read with hs2_check_device_status().
+ *   - head_dim must be 128.  h_q must be a multiple of 16 in [16, 128].
+ *     n_q (query tokens per sequence) is in [1, 64].  window >= 1, k_sel >= 1,
+ *     window + k_sel <= 4096.  Otherwise HS2_ERR_UNSUPPORTED.
+ *   - Query token i of sequence b sits at position p = lens[b] - n_q + i and sees
+ *     keys [0, p]; 1 <= n_q <= lens[b] <= max_len is required (checked on the
+ *     device: a violating sequence sets HS2_ERR_BAD_LENGTH and is clamped).
+ *   - All of q, k, v, out and the workspace must be 16-byte aligned; rows are
+ *     dense (strides are implied by the shapes given below).
+ */
+#ifndef HS2_H_
+#define HS2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define HS2_API __attribute__((visibility("default")))
+#else
+#define HS2_API
+#endif
+
+typedef struct CUstream_st* hs2_stream_t; /* identical to cudaStream_t */
+
+typedef enum hs2_status {
+  HS2_OK = 0,
+  HS2_ERR_INVALID_ARGUMENT = 1,    /* null pointer, bad size, misalignment        */
+  HS2_ERR_UNSUPPORTED = 2,         /* outside the supported ranges listed above    */
+  HS2_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes < hs2_workspace_bytes(...)          */
+  HS2_ERR_CUDA = 4,                /* a CUDA runtime call failed                   */
+  HS2_ERR_DEVICE_TIMEOUT = 5,      /* a bounded device-side wait gave up           */
+  HS2_ERR_INDEX_OUT_OF_RANGE = 6,  /* sparse index outside [0, lens[b]) and != -1  */
+  HS2_ERR_BAD_LENGTH = 7           /* lens[b] outside [n_q, max_len]               */
+} hs2_status;
+
+typedef enum hs2_kv_dtype {
+  HS2_KV_BF16 = 0,     /* K and V are bfloat16                                      */
+  HS2_KV_FP8_E4M3 = 1  /* K and V are OCP FP8 E4M3 ("fn") codes with per-token
+                          float32 scales: value = decode(code) * scale[b][j]        */
+} hs2_kv_dtype;
+
+/* The shared KV cache of one hybrid block (one K/V head: MQA).
+ *   k, v     device, [batch][max_len][head_dim], head_dim contiguous; element type
+ *            per `dtype` (2 bytes bf16 or 1 byte E4M3 code).  Only rows [0, lens[b])
+ *            are read; the rest may hold anything, NaN included.
+ *   k_scale, v_scale  device float32 [batch][max_len]; required for FP8, must be
+ *            NULL for bf16.
+ *   lens     device int32 [batch].                                                */
+typedef struct hs2_kv {
+  const void* k;
+  const void* v;
+  const float* k_scale;
+  const float* v_scale;
+  const int32_t* lens;
+  int32_t batch;
+  int32_t max_len;
+  int32_t head_dim;
+  int32_t dtype; /* hs2_kv_dtype */
+} hs2_kv;
+
+/* Bytes of workspace that the calls below need for these sizes (0 if the sizes are
+ * unsupported).  One workspace serves hs2_full_attn_select and every following
+ * hs2_sparse_attn of the same step.  It must be zero-filled once before first use;
+ * afterwards the library keeps it consistent itself.  Calls sharing a workspace
+ * must be ordered (same stream, or otherwise serialised). */
+HS2_API size_t hs2_workspace_bytes(int batch, int n_q, int h_q, int max_len, int window,
+                           int k_sel, int dtype);
+
+/* Full-attention layer + token selection (steps 1 and 2).
+ *   q        device bf16 [batch][n_q][h_q][128].
+ *   sm_scale softmax scale applied to q.k (normally 1/sqrt(128) as float32).
+ *   out      device float32 [batch][n_q][h_q][128]: softmax(s) @ V over keys [0, p].
+ *   idx      device int32 [batch][n_q][window + k_sel]: the ascending union of
+ *            [max(0, p-window+1), p] and the top-k_sel positions of [0, p-window]
+ *            by (importance desc, position asc); when p+1 <= window + k_sel it is
+ *            all of [0, p]; unused slots are -1.
+ *   lse      device float32 [batch][n_q][h_q] natural-log sum-exp of the logits,
+ *            or NULL.
+ * Equivalent to hs2_full_attn followed by hs2_select on the same workspace. */
+HS2_API hs2_status hs2_full_attn_select(const void* q, int n_q, int h_q, const hs2_kv* kv,
+                                int window, int k_sel, float sm_scale, float* out,
+                                int32_t* idx, float* lse, void* workspace,
+                                size_t ws_bytes, hs2_stream_t stream);
+
+/* Step 1 alone: split-K flash-decode over every visible key, writing `out` and
+ * (if non-NULL) `lse`, and leaving the per-head log-sum-exp in the workspace for
+ * hs2_select.  Arguments as above. */
+HS2_API hs2_status hs2_full_attn(const void* q, int n_q, int h_q, const hs2_kv* kv,
+                         int window, int k_sel, float sm_scale, float* out, float* lse,
+                         void* workspace, size_t ws_bytes, hs2_stream_t stream);
+
+/* Step 2 alone: importance of every key outside the window and the exact top-k_sel
+ * selection merged with the window, into `idx`.  Must follow hs2_full_attn with the
+ * same q, kv, sizes and workspace, on the same stream. */
+HS2_API hs2_status hs2_select(const void* q, int n_q, int h_q, const hs2_kv* kv, int window,
+                      int k_sel, float sm_scale, int32_t* idx, void* workspace,
+                      size_t ws_bytes, hs2_stream_t stream);
+
+/* One reusing sparse-attention layer (step 3).
+ *   q_layer   device bf16 [batch][n_q][h_q][128], this layer's queries.
+ *   idx       device int32 [batch][n_q][idx_width]: positions to attend to (any
+ *             order, duplicates counted as given); -1 entries are skipped.  An entry
+ *             outside [0, lens[b]) is skipped and sets HS2_ERR_INDEX_OUT_OF_RANGE.
+ *   out       device float32 [batch][n_q][h_q][128]; a row whose set is empty gets 0.
+ * idx_width in [1, 4096]; the workspace must come from hs2_workspace_bytes with
+ * window + k_sel >= idx_width. */
+HS2_API hs2_status hs2_sparse_attn(const void* q_layer, int n_q, int h_q, const hs2_kv* kv,
+                           const int32_t* idx, int idx_width, float sm_scale, float* out,
+                           void* workspace, size_t ws_bytes, hs2_stream_t stream);
+
+/* Synchronises `stream`, returns the first error recorded by the kernels since the
+ * last check (HS2_OK if none) and clears it. */
+HS2_API hs2_status hs2_check_device_status(void* workspace, hs2_stream_t stream);
+
+/* Static description of a status code (never NULL). */
+HS2_API const char* hs2_status_string(hs2_status status);
+
+/* Text of the last CUDA error seen by this thread's calls ("" if none). */
+HS2_API const char* hs2_last_cuda_error(void);
+
+/* ABI version of this header; bumped on any incompatible change. */
+HS2_API int hs2_abi_version(void);
+
+#define HS2_ABI_VERSION 1
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HS2_H_ */

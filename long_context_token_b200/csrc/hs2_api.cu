@@ -1,0 +1,327 @@
+// Host side of the libhs2 C ABI: argument validation, workspace layout and the
+// launch sequence of each call.  Nothing here allocates device memory.
+#include <stdio.h>
+#include <string.h>
+
+#include "hs2_internal.cuh"
+
+namespace hs2 {
+
+static thread_local char g_last_cuda_error[256] = "";
+
+static hs2_status cuda_fail(cudaError_t e, const char* what) {
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", what,
+           cudaGetErrorString(e));
+  return HS2_ERR_CUDA;
+}
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Target of ~4 CTAs per SM of a 148-SM B200 for the key-chunk kernels; fixed so
+// that the workspace layout does not depend on the device it runs on.
+constexpr int kTargetCtas = 4 * 148;
+constexpr int kMinChunk = 256;
+constexpr int kChunk3 = 8192;
+constexpr int kChunk4 = 64;
+
+int plan_splits1(int bq, int max_len, int /*num_sms*/) {
+  int splits = (kTargetCtas + bq - 1) / bq;
+  const int max_splits = (max_len + kMinChunk - 1) / kMinChunk;
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  return splits;
+}
+
+static int chunk_for(int max_len, int splits) {
+  int chunk = (max_len + splits - 1) / splits;
+  return (chunk + 31) / 32 * 32;
+}
+
+int plan_splits4(int idx_width) { return (idx_width + kChunk4 - 1) / kChunk4; }
+
+bool make_layout(int batch, int n_q, int h, int max_len, int window, int k_sel,
+                 WsLayout* L) {
+  WsLayout w;
+  w.bq = batch * n_q;
+  w.h = h;
+  w.max_len = max_len;
+  w.window = window;
+  w.k_sel = k_sel;
+  w.splits1 = plan_splits1(w.bq, max_len, kSmCountBound);
+  w.splits4 = plan_splits4(kMaxIdxWidth);  // capacity for any idx_width
+  const size_t bq = (size_t)w.bq, ml = (size_t)max_len, hh = (size_t)h;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  // Regions that depend only on (bq, h): status and the sparse-layer state.
+  w.status = take(sizeof(uint32_t));
+  w.tickets1 = take(bq * sizeof(uint32_t));
+  w.tickets4 = take(bq * sizeof(uint32_t));
+  w.part4_o = take(bq * w.splits4 * hh * kHeadDim * sizeof(float));
+  w.part4_ml = take(bq * w.splits4 * hh * 2 * sizeof(float));
+  // Regions of the full layer and the selection.
+  w.clear_begin = off;
+  w.hist = take(bq * kHistBins * sizeof(uint32_t));
+  w.counters = take(bq * 8 * sizeof(uint32_t));
+  w.clear_end = off;
+  w.selmeta = take(bq * 4 * sizeof(uint32_t));
+  w.part1_o = take(bq * w.splits1 * hh * kHeadDim * sizeof(float));
+  w.part1_ml = take(bq * w.splits1 * hh * 2 * sizeof(float));
+  w.lse64 = take(bq * hh * sizeof(double));
+  w.delta64 = take(bq * hh * sizeof(double));
+  w.delta32 = take(bq * hh * sizeof(float));
+  w.tbuf = take(bq * ml * sizeof(float));
+  w.direct = take(bq * (size_t)k_sel * sizeof(int32_t));
+  w.cand_t = take(bq * ml * sizeof(float));
+  w.cand_j = take(bq * ml * sizeof(int32_t));
+  w.band_t = take(bq * ml * sizeof(double));
+  w.band_j = take(bq * ml * sizeof(int32_t));
+  w.total = off;
+  *L = w;
+  return true;
+}
+
+// Bytes of the leading part of the workspace that a sparse layer uses.
+static size_t sparse_prefix_bytes(const WsLayout& w) { return w.clear_begin; }
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static hs2_status check_shape(int batch, int n_q, int h, int max_len, int window, int k_sel) {
+  if (batch < 1 || max_len < 1) return HS2_ERR_INVALID_ARGUMENT;
+  if (n_q < 1 || n_q > kMaxNq) return HS2_ERR_UNSUPPORTED;
+  if (h < 16 || h > kMaxHeads || (h % 16) != 0) return HS2_ERR_UNSUPPORTED;
+  if (window < 1 || k_sel < 1 || window + k_sel > kMaxIdxWidth) return HS2_ERR_UNSUPPORTED;
+  if (max_len < n_q) return HS2_ERR_INVALID_ARGUMENT;
+  if ((long long)batch * (long long)max_len >= (1ll << 31)) return HS2_ERR_UNSUPPORTED;
+  return HS2_OK;
+}
+
+static hs2_status check_kv(const hs2_kv* kv) {
+  if (!kv || !kv->k || !kv->v || !kv->lens) return HS2_ERR_INVALID_ARGUMENT;
+  if (kv->head_dim != kHeadDim) return HS2_ERR_UNSUPPORTED;
+  if (kv->dtype == HS2_KV_BF16) {
+    if (kv->k_scale || kv->v_scale) return HS2_ERR_INVALID_ARGUMENT;
+  } else if (kv->dtype == HS2_KV_FP8_E4M3) {
+    if (!kv->k_scale || !kv->v_scale) return HS2_ERR_INVALID_ARGUMENT;
+  } else {
+    return HS2_ERR_UNSUPPORTED;
+  }
+  if (!aligned16(kv->k) || !aligned16(kv->v)) return HS2_ERR_INVALID_ARGUMENT;
+  return HS2_OK;
+}
+
+static KvView view_of(const hs2_kv* kv) {
+  KvView v;
+  v.k = kv->k;
+  v.v = kv->v;
+  v.k_scale = kv->k_scale;
+  v.v_scale = kv->v_scale;
+  v.lens = kv->lens;
+  v.batch = kv->batch;
+  v.max_len = kv->max_len;
+  v.fp8 = kv->dtype == HS2_KV_FP8_E4M3;
+  return v;
+}
+
+struct Prepared {
+  WsLayout w;
+};
+
+static hs2_status prepare(const void* q, int n_q, int h, const hs2_kv* kv, int window,
+                          int k_sel, void* ws, size_t ws_bytes, Prepared* P) {
+  hs2_status st = check_kv(kv);
+  if (st != HS2_OK) return st;
+  st = check_shape(kv->batch, n_q, h, kv->max_len, window, k_sel);
+  if (st != HS2_OK) return st;
+  if (!q || !ws) return HS2_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(ws)) return HS2_ERR_INVALID_ARGUMENT;
+  make_layout(kv->batch, n_q, h, kv->max_len, window, k_sel, &P->w);
+  if (ws_bytes < P->w.total) return HS2_ERR_WORKSPACE_TOO_SMALL;
+  return HS2_OK;
+}
+
+static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int window,
+                           int k_sel, float sm_scale, float* out, float* lse, void* ws,
+                           const WsLayout& w, cudaStream_t s) {
+  FullParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.kv = view_of(kv);
+  p.n_q = n_q;
+  p.h = h;
+  p.window = window;
+  p.k_sel = k_sel;
+  p.sm_scale = sm_scale;
+  p.splits1 = w.splits1;
+  p.chunk1 = chunk_for(kv->max_len, w.splits1);
+  p.part_o = ws_ptr<float>(ws, w.part1_o);
+  p.part_ml = ws_ptr<float>(ws, w.part1_ml);
+  p.tickets = ws_ptr<uint32_t>(ws, w.tickets1);
+  p.out = out;
+  p.lse_out = lse;
+  p.lse64 = ws_ptr<double>(ws, w.lse64);
+  p.delta64 = ws_ptr<double>(ws, w.delta64);
+  p.delta32 = ws_ptr<float>(ws, w.delta32);
+  p.status = ws_ptr<uint32_t>(ws, w.status);
+  cudaError_t e = launch_full_attn(p, kv->batch, s);
+  return e == cudaSuccess ? HS2_OK : cuda_fail(e, "full-attention launch");
+}
+
+static hs2_status run_select(const void* q, int n_q, int h, const hs2_kv* kv, int window,
+                             int k_sel, float sm_scale, int32_t* idx, void* ws,
+                             const WsLayout& w, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(ws_ptr<char>(ws, w.clear_begin), 0,
+                                  w.clear_end - w.clear_begin, s);
+  if (e != cudaSuccess) return cuda_fail(e, "workspace clear");
+  SelectParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.kv = view_of(kv);
+  p.n_q = n_q;
+  p.h = h;
+  p.window = window;
+  p.k_sel = k_sel;
+  p.sm_scale = sm_scale;
+  p.splits2 = w.splits1;
+  p.chunk2 = chunk_for(kv->max_len, w.splits1);
+  p.chunk3 = kChunk3;
+  p.splits3 = (kv->max_len + kChunk3 - 1) / kChunk3;
+  p.delta64 = ws_ptr<double>(ws, w.delta64);
+  p.delta32 = ws_ptr<float>(ws, w.delta32);
+  p.tbuf = ws_ptr<float>(ws, w.tbuf);
+  p.hist = ws_ptr<uint32_t>(ws, w.hist);
+  p.counters = ws_ptr<uint32_t>(ws, w.counters);
+  p.selmeta = ws_ptr<uint32_t>(ws, w.selmeta);
+  p.direct = ws_ptr<int32_t>(ws, w.direct);
+  p.cand_t = ws_ptr<float>(ws, w.cand_t);
+  p.cand_j = ws_ptr<int32_t>(ws, w.cand_j);
+  p.band_t = ws_ptr<double>(ws, w.band_t);
+  p.band_j = ws_ptr<int32_t>(ws, w.band_j);
+  p.idx = idx;
+  p.status = ws_ptr<uint32_t>(ws, w.status);
+  e = launch_select(p, kv->batch, s);
+  return e == cudaSuccess ? HS2_OK : cuda_fail(e, "selection launch");
+}
+
+}  // namespace hs2
+
+using namespace hs2;
+
+extern "C" {
+
+size_t hs2_workspace_bytes(int batch, int n_q, int h_q, int max_len, int window, int k_sel,
+                           int dtype) {
+  if (dtype != HS2_KV_BF16 && dtype != HS2_KV_FP8_E4M3) return 0;
+  if (check_shape(batch, n_q, h_q, max_len, window, k_sel) != HS2_OK) return 0;
+  WsLayout w;
+  make_layout(batch, n_q, h_q, max_len, window, k_sel, &w);
+  return w.total;
+}
+
+hs2_status hs2_full_attn(const void* q, int n_q, int h_q, const hs2_kv* kv, int window,
+                         int k_sel, float sm_scale, float* out, float* lse, void* workspace,
+                         size_t ws_bytes, hs2_stream_t stream) {
+  Prepared P;
+  hs2_status st = prepare(q, n_q, h_q, kv, window, k_sel, workspace, ws_bytes, &P);
+  if (st != HS2_OK) return st;
+  if (!out || !aligned16(out)) return HS2_ERR_INVALID_ARGUMENT;
+  return run_full(q, n_q, h_q, kv, window, k_sel, sm_scale, out, lse, workspace, P.w,
+                  (cudaStream_t)stream);
+}
+
+hs2_status hs2_select(const void* q, int n_q, int h_q, const hs2_kv* kv, int window,
+                      int k_sel, float sm_scale, int32_t* idx, void* workspace,
+                      size_t ws_bytes, hs2_stream_t stream) {
+  Prepared P;
+  hs2_status st = prepare(q, n_q, h_q, kv, window, k_sel, workspace, ws_bytes, &P);
+  if (st != HS2_OK) return st;
+  if (!idx) return HS2_ERR_INVALID_ARGUMENT;
+  return run_select(q, n_q, h_q, kv, window, k_sel, sm_scale, idx, workspace, P.w,
+                    (cudaStream_t)stream);
+}
+
+hs2_status hs2_full_attn_select(const void* q, int n_q, int h_q, const hs2_kv* kv,
+                                int window, int k_sel, float sm_scale, float* out,
+                                int32_t* idx, float* lse, void* workspace, size_t ws_bytes,
+                                hs2_stream_t stream) {
+  Prepared P;
+  hs2_status st = prepare(q, n_q, h_q, kv, window, k_sel, workspace, ws_bytes, &P);
+  if (st != HS2_OK) return st;
+  if (!out || !aligned16(out) || !idx) return HS2_ERR_INVALID_ARGUMENT;
+  st = run_full(q, n_q, h_q, kv, window, k_sel, sm_scale, out, lse, workspace, P.w,
+                (cudaStream_t)stream);
+  if (st != HS2_OK) return st;
+  return run_select(q, n_q, h_q, kv, window, k_sel, sm_scale, idx, workspace, P.w,
+                    (cudaStream_t)stream);
+}
+
+hs2_status hs2_sparse_attn(const void* q_layer, int n_q, int h_q, const hs2_kv* kv,
+                           const int32_t* idx, int idx_width, float sm_scale, float* out,
+                           void* workspace, size_t ws_bytes, hs2_stream_t stream) {
+  hs2_status st = check_kv(kv);
+  if (st != HS2_OK) return st;
+  if (idx_width < 1 || idx_width > kMaxIdxWidth) return HS2_ERR_UNSUPPORTED;
+  st = check_shape(kv->batch, n_q, h_q, kv->max_len, 1, 1);
+  if (st != HS2_OK) return st;
+  if (!q_layer || !idx || !out || !workspace) return HS2_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q_layer) || !aligned16(out) || !aligned16(workspace))
+    return HS2_ERR_INVALID_ARGUMENT;
+  WsLayout w;
+  make_layout(kv->batch, n_q, h_q, kv->max_len, 1, 1, &w);
+  if (ws_bytes < sparse_prefix_bytes(w)) return HS2_ERR_WORKSPACE_TOO_SMALL;
+  SparseParams p;
+  p.q = static_cast<const uint16_t*>(q_layer);
+  p.kv = view_of(kv);
+  p.idx = idx;
+  p.n_q = n_q;
+  p.h = h_q;
+  p.idx_width = idx_width;
+  p.sm_scale = sm_scale;
+  p.splits4 = plan_splits4(idx_width);
+  p.chunk4 = kChunk4;
+  p.part_o = ws_ptr<float>(workspace, w.part4_o);
+  p.part_ml = ws_ptr<float>(workspace, w.part4_ml);
+  p.tickets = ws_ptr<uint32_t>(workspace, w.tickets4);
+  p.out = out;
+  p.status = ws_ptr<uint32_t>(workspace, w.status);
+  cudaError_t e = launch_sparse_attn(p, kv->batch, (cudaStream_t)stream);
+  return e == cudaSuccess ? HS2_OK : cuda_fail(e, "sparse-attention launch");
+}
+
+hs2_status hs2_check_device_status(void* workspace, hs2_stream_t stream) {
+  if (!workspace) return HS2_ERR_INVALID_ARGUMENT;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  uint32_t word = 0;
+  e = cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (word == 0) return HS2_OK;
+  e = cudaMemsetAsync(workspace, 0, sizeof(word), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  for (int c = 1; c < 32; ++c)
+    if (word & (1u << c)) return (hs2_status)c;
+  return HS2_OK;
+}
+
+const char* hs2_status_string(hs2_status s) {
+  switch (s) {
+    case HS2_OK: return "ok";
+    case HS2_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case HS2_ERR_UNSUPPORTED: return "unsupported size or type";
+    case HS2_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case HS2_ERR_CUDA: return "CUDA runtime error";
+    case HS2_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case HS2_ERR_INDEX_OUT_OF_RANGE: return "sparse index out of range";
+    case HS2_ERR_BAD_LENGTH: return "sequence length out of range";
+  }
+  return "unknown status";
+}
+
+const char* hs2_last_cuda_error(void) { return g_last_cuda_error; }
+
+int hs2_abi_version(void) { return HS2_ABI_VERSION; }
+
+}  // extern "C"

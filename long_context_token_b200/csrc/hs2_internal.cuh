@@ -1,0 +1,210 @@
+// Internal declarations shared by the libhs2 translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/hs2.h"
+
+namespace hs2 {
+
+constexpr int kHeadDim = 128;
+constexpr int kHistBins = 4096;         // first-level radix histogram: top 12 bits
+constexpr int kHistShift = 20;
+constexpr int kMaxIdxWidth = 4096;      // window + k_sel
+constexpr int kMaxNq = 64;
+constexpr int kMaxHeads = 128;
+constexpr int kSmCountBound = 160;      // workspace sizing assumes at most this many SMs
+
+// Status bits kept in the workspace's status word (one bit per hs2_status code).
+__host__ __device__ constexpr uint32_t status_bit(hs2_status s) { return 1u << (int)s; }
+
+// ---------------------------------------------------------------------------
+// Workspace layout.  Every region starts on a 256-byte boundary.
+// ---------------------------------------------------------------------------
+struct WsLayout {
+  int bq = 0, h = 0, max_len = 0, window = 0, k_sel = 0;
+  int splits1 = 0;   // key chunks per (sequence, query token) in the full layer
+  int splits4 = 0;   // index chunks per (sequence, query token) in a sparse layer
+  size_t status = 0;      // u32 status word; never cleared by a compute call
+  size_t clear_begin = 0; // [clear_begin, clear_end) is zeroed by every full-layer call
+  size_t hist = 0;        // u32 [bq][kHistBins]
+  size_t counters = 0;    // u32 [bq][8]: 0 direct, 1 cand, 2 band
+  size_t clear_end = 0;
+  size_t tickets1 = 0;    // u32 [bq], self-resetting
+  size_t tickets4 = 0;    // u32 [bq], self-resetting
+  size_t selmeta = 0;     // u32 [bq][4]: bin, eps bits, k_eff, n_c
+  size_t part1_o = 0;     // f32 [bq][splits1][h][128]
+  size_t part1_ml = 0;    // f32 [bq][splits1][h][2]
+  size_t lse64 = 0;       // f64 [bq][h]
+  size_t delta64 = 0;     // f64 [bq][h]
+  size_t delta32 = 0;     // f32 [bq][h]
+  size_t tbuf = 0;        // f32 [bq][max_len]  selection keys t_j
+  size_t direct = 0;      // i32 [bq][k_sel]
+  size_t cand_t = 0;      // f32 [bq][max_len]
+  size_t cand_j = 0;      // i32 [bq][max_len]
+  size_t band_t = 0;      // f64 [bq][max_len]
+  size_t band_j = 0;      // i32 [bq][max_len]
+  size_t part4_o = 0;     // f32 [bq][splits4][h][128]
+  size_t part4_ml = 0;    // f32 [bq][splits4][h][2]
+  size_t total = 0;
+};
+
+int plan_splits1(int bq, int max_len, int num_sms);
+int plan_splits4(int idx_width);
+bool make_layout(int batch, int n_q, int h, int max_len, int window, int k_sel,
+                 WsLayout* L);
+
+template <typename T>
+inline T* ws_ptr(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+// ---------------------------------------------------------------------------
+// Kernel parameter blocks.
+// ---------------------------------------------------------------------------
+struct KvView {
+  const void* k;
+  const void* v;
+  const float* k_scale;
+  const float* v_scale;
+  const int32_t* lens;
+  int batch, max_len;
+  int fp8;
+};
+
+struct FullParams {
+  const uint16_t* q;  // bf16 bits [B][n_q][h][128]
+  KvView kv;
+  int n_q, h, window, k_sel;
+  float sm_scale;
+  int splits1, chunk1;
+  float* part_o;
+  float* part_ml;
+  uint32_t* tickets;
+  float* out;
+  float* lse_out;  // may be null
+  double* lse64;
+  double* delta64;
+  float* delta32;
+  uint32_t* status;
+};
+
+struct SelectParams {
+  const uint16_t* q;
+  KvView kv;
+  int n_q, h, window, k_sel;
+  float sm_scale;
+  int splits2, chunk2;   // importance pass
+  int splits3, chunk3;   // compaction pass
+  const double* delta64;
+  const float* delta32;
+  float* tbuf;
+  uint32_t* hist;
+  uint32_t* counters;
+  uint32_t* selmeta;
+  int32_t* direct;
+  float* cand_t;
+  int32_t* cand_j;
+  double* band_t;
+  int32_t* band_j;
+  int32_t* idx;
+  uint32_t* status;
+};
+
+struct SparseParams {
+  const uint16_t* q;
+  KvView kv;
+  const int32_t* idx;
+  int n_q, h, idx_width;
+  float sm_scale;
+  int splits4, chunk4;
+  float* part_o;
+  float* part_ml;
+  uint32_t* tickets;
+  float* out;
+  uint32_t* status;
+};
+
+// Launchers (each returns the launch's cudaError_t).
+cudaError_t launch_full_attn(const FullParams& p, int batch, cudaStream_t s);
+cudaError_t launch_select(const SelectParams& p, int batch, cudaStream_t s);
+cudaError_t launch_sparse_attn(const SparseParams& p, int batch, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// Device helpers.
+// ---------------------------------------------------------------------------
+#ifdef __CUDACC__
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) {
+  return __uint_as_float(b << 16);
+}
+
+// OCP FP8 E4M3 ("fn") code -> float32, from the format: sign, 4-bit exponent with
+// bias 7, 3-bit mantissa, exponent 0 subnormal, S.1111.111 NaN.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
+  const uint32_t e = (c >> 3) & 0xFu, m = c & 0x7u;
+  float mag;
+  if (e == 0) {
+    mag = (float)m * 0.001953125f;  // m * 2^-9
+  } else {
+    mag = __uint_as_float(((e + 120u) << 23) | (m << 20));
+  }
+  if ((c & 0x7Fu) == 0x7Fu) mag = __int_as_float(0x7fc00000);
+  return (c & 0x80u) ? -mag : mag;
+}
+
+__device__ __forceinline__ double e4m3_to_f64(uint32_t c) {
+  return (double)e4m3_to_f32(c);  // every E4M3 value is exact in float32
+}
+
+// Monotone map float -> uint32 (larger float -> larger key); NaN excluded.
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+  const uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+  return __uint_as_float(u);
+}
+__device__ __forceinline__ unsigned long long ordered_key64(double f) {
+  const unsigned long long u = (unsigned long long)__double_as_longlong(f);
+  return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ void set_status(uint32_t* status, hs2_status s) {
+  atomicOr(status, status_bit(s));
+}
+
+// Valid length of sequence b, clamped to [n_q, max_len] (an out-of-range length
+// is recorded and clamped so that no access leaves the cache).
+__device__ __forceinline__ int seq_len(const KvView& kv, int b, int n_q, uint32_t* status,
+                                       bool report) {
+  int L = kv.lens[b];
+  if (L < n_q || L > kv.max_len) {
+    if (report) set_status(status, HS2_ERR_BAD_LENGTH);
+    L = L < n_q ? n_q : kv.max_len;
+  }
+  return L;
+}
+
+#endif  // __CUDACC__
+
+}  // namespace hs2

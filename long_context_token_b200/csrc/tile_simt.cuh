@@ -1,0 +1,248 @@
+// CUDA-core building blocks: 32-row K/V tiles staged as float32 in shared memory,
+// the QK^T tile, the online-softmax update and the P.V accumulation, plus the
+// split merge.  Used by the full layer (contiguous rows), the importance pass and
+// the sparse layers (gathered rows).
+#pragma once
+
+#include "hs2_internal.cuh"
+
+namespace hs2 {
+
+constexpr int kTile = 32;      // rows per tile
+constexpr int kThreads = 256;  // threads per CTA of the SIMT kernels
+constexpr int kKsLd = kHeadDim + 1;  // padded row stride of the staged K tile
+
+// Dynamic shared memory of a SIMT attention CTA with H heads.
+__host__ __device__ constexpr size_t simt_smem_bytes(int H) {
+  return sizeof(float) * ((size_t)H * kHeadDim      // q (pre-scaled)
+                          + kTile * kKsLd            // K tile
+                          + kTile * kHeadDim         // V tile
+                          + (size_t)H * kTile        // S / P tile
+                          + 3 * (size_t)H)           // m, l, alpha
+         + sizeof(int) * kTile;                      // row index of each tile row
+}
+
+struct SimtSmem {
+  float* qs;
+  float* ks;
+  float* vs;
+  float* S;
+  float* m_run;
+  float* l_run;
+  float* alpha;
+  int* rowidx;
+};
+
+__device__ __forceinline__ SimtSmem carve_simt(float* sm, int H) {
+  SimtSmem s;
+  s.qs = sm;
+  s.ks = s.qs + H * kHeadDim;
+  s.vs = s.ks + kTile * kKsLd;
+  s.S = s.vs + kTile * kHeadDim;
+  s.m_run = s.S + H * kTile;
+  s.l_run = s.m_run + H;
+  s.alpha = s.l_run + H;
+  s.rowidx = reinterpret_cast<int*>(s.alpha + H);
+  return s;
+}
+
+// q (bf16 bits) of one (sequence, token) -> shared float, times sm_scale.
+template <int H>
+__device__ __forceinline__ void load_q_scaled(float* qs, const uint16_t* q, float sm_scale) {
+  for (int e = threadIdx.x; e < H * kHeadDim; e += kThreads)
+    qs[e] = bf16_bits_to_f32(q[e]) * sm_scale;
+}
+
+// Stage kTile cache rows into shared float32 (row r of `dst` has stride ld).
+// rowidx[r] is the flat row (b * max_len + j) or -1 for an absent row (zeros).
+// FP8 rows are decoded and multiplied by their per-token scale.
+template <bool FP8>
+__device__ __forceinline__ void load_rows(float* dst, int ld, const void* base,
+                                          const float* scale, const int* rowidx) {
+  if (!FP8) {
+    const uint16_t* src = static_cast<const uint16_t*>(base);
+    for (int v = threadIdx.x; v < kTile * 16; v += kThreads) {
+      const int r = v >> 4, c = (v & 15) * 8;
+      const int row = rowidx[r];
+      float* d = dst + r * ld + c;
+      if (row >= 0) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4*>(src + (size_t)row * kHeadDim + c));
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          d[2 * e] = bf16_bits_to_f32(w[e] & 0xffffu);
+          d[2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) d[e] = 0.f;
+      }
+    }
+  } else {
+    const uint8_t* src = static_cast<const uint8_t*>(base);
+    for (int v = threadIdx.x; v < kTile * 8; v += kThreads) {
+      const int r = v >> 3, c = (v & 7) * 16;
+      const int row = rowidx[r];
+      float* d = dst + r * ld + c;
+      if (row >= 0) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4*>(src + (size_t)row * kHeadDim + c));
+        const float sc = __ldg(scale + row);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+#pragma unroll
+          for (int t = 0; t < 4; ++t) d[4 * e + t] = e4m3_to_f32((w[e] >> (8 * t)) & 0xffu) * sc;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) d[e] = 0.f;
+      }
+    }
+  }
+}
+
+// S[h][r] = qs[h] . ks[r] for every head and tile row; -inf for absent rows.
+template <int H>
+__device__ __forceinline__ void qk_tile(const SimtSmem& s) {
+  constexpr int R = H / 8;  // heads per thread
+  const int key = threadIdx.x & 31, hg = threadIdx.x >> 5;
+  float acc[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) acc[r] = 0.f;
+  const float* kr = s.ks + key * kKsLd;
+#pragma unroll 4
+  for (int c = 0; c < kHeadDim; ++c) {
+    const float kv = kr[c];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r] = fmaf(s.qs[(hg + 8 * r) * kHeadDim + c], kv, acc[r]);
+  }
+  const bool valid = s.rowidx[key] >= 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) s.S[(hg + 8 * r) * kTile + key] = valid ? acc[r] : -INFINITY;
+}
+
+// Online-softmax update of one tile: S <- exp(S - m_new), l and alpha updated.
+template <int H>
+__device__ __forceinline__ void softmax_tile(const SimtSmem& s) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int hd = w; hd < H; hd += kThreads / 32) {
+    const float x = s.S[hd * kTile + lane];
+    const float m_old = s.m_run[hd];
+    const float m_new = fmaxf(m_old, warp_max(x));
+    float pr = 0.f, al = 1.f;
+    if (m_new != -INFINITY) {
+      pr = expf(x - m_new);
+      al = expf(m_old - m_new);
+    }
+    const float sum = warp_sum(pr);
+    s.S[hd * kTile + lane] = pr;
+    __syncwarp();
+    if (lane == 0) {
+      s.alpha[hd] = al;
+      s.m_run[hd] = m_new;
+      s.l_run[hd] = s.l_run[hd] * al + sum;
+    }
+  }
+}
+
+// acc[r] (head hg2 + 2r, dimension d) = acc * alpha + sum_r P[h][r] V[r][d].
+template <int H>
+__device__ __forceinline__ void pv_tile(const SimtSmem& s, float* acc) {
+  const int d = threadIdx.x & (kHeadDim - 1), hg2 = threadIdx.x >> 7;
+#pragma unroll
+  for (int r = 0; r < H / 2; ++r) {
+    const int hd = hg2 + 2 * r;
+    float a = acc[r] * s.alpha[hd];
+    const float* pr = s.S + hd * kTile;
+#pragma unroll 8
+    for (int j = 0; j < kTile; ++j) a = fmaf(pr[j], s.vs[j * kHeadDim + d], a);
+    acc[r] = a;
+  }
+}
+
+// Write this split's partial state (m, l, unnormalised o).
+template <int H>
+__device__ __forceinline__ void write_partial(const SimtSmem& s, const float* acc,
+                                              float* part_o, float* part_ml) {
+  const int d = threadIdx.x & (kHeadDim - 1), hg2 = threadIdx.x >> 7;
+#pragma unroll
+  for (int r = 0; r < H / 2; ++r) part_o[(hg2 + 2 * r) * kHeadDim + d] = acc[r];
+  for (int hd = threadIdx.x; hd < H; hd += kThreads) {
+    part_ml[2 * hd] = s.m_run[hd];
+    part_ml[2 * hd + 1] = s.l_run[hd];
+  }
+}
+
+// Returns true in exactly one CTA of the `n` CTAs sharing `ticket`: the last one to
+// arrive after all of them wrote their partials.  That CTA resets the ticket.
+__device__ __forceinline__ bool arrive_last(uint32_t* ticket, int n) {
+  __shared__ int last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t prev = atomicAdd(ticket, 1u);
+    last = (prev == (uint32_t)(n - 1));
+    if (last) *ticket = 0u;
+  }
+  __syncthreads();
+  if (last) __threadfence();
+  return last != 0;
+}
+
+// Merge `splits` partials of H heads into out (normalised) and per-head lse.
+// lse_d (shared, H doubles) receives ln(sum) in float64; heads with no key get
+// lse = -inf and out = 0.  Uses `scratch` (shared, >= 32*H + 2*H floats).
+template <int H>
+__device__ void merge_partials(const float* part_o, const float* part_ml, int splits,
+                               float* out, double* lse_d, float* scratch) {
+  float* w = scratch;              // [32][H]
+  float* Mf = scratch + 32 * H;    // [H]
+  float* invL = Mf + H;            // [H]
+  for (int hd = threadIdx.x; hd < H; hd += kThreads) {
+    float M = -INFINITY;
+    for (int sp = 0; sp < splits; ++sp) M = fmaxf(M, __ldcg(part_ml + ((size_t)sp * H + hd) * 2));
+    double Ls = 0.0;
+    if (M != -INFINITY) {
+      for (int sp = 0; sp < splits; ++sp) {
+        const float m = __ldcg(part_ml + ((size_t)sp * H + hd) * 2);
+        const float l = __ldcg(part_ml + ((size_t)sp * H + hd) * 2 + 1);
+        if (l > 0.f) Ls += (double)l * exp((double)m - (double)M);
+      }
+    }
+    Mf[hd] = M;
+    invL[hd] = Ls > 0.0 ? (float)(1.0 / Ls) : 0.f;
+    lse_d[hd] = Ls > 0.0 ? (double)M + log(Ls) : -INFINITY;
+  }
+  __syncthreads();
+  const int d = threadIdx.x & (kHeadDim - 1), hg2 = threadIdx.x >> 7;
+  float acc[H / 2];
+#pragma unroll
+  for (int r = 0; r < H / 2; ++r) acc[r] = 0.f;
+  for (int sb = 0; sb < splits; sb += 32) {
+    for (int e = threadIdx.x; e < 32 * H; e += kThreads) {
+      const int sp = sb + e / H, hd = e % H;
+      float wt = 0.f;
+      if (sp < splits && Mf[hd] != -INFINITY) {
+        const float m = __ldcg(part_ml + ((size_t)sp * H + hd) * 2);
+        const float l = __ldcg(part_ml + ((size_t)sp * H + hd) * 2 + 1);
+        if (l > 0.f) wt = expf(m - Mf[hd]) * invL[hd];
+      }
+      w[e] = wt;
+    }
+    __syncthreads();
+    const int nsb = min(32, splits - sb);
+    for (int t = 0; t < nsb; ++t) {
+#pragma unroll
+      for (int r = 0; r < H / 2; ++r) {
+        const int hd = hg2 + 2 * r;
+        const float wt = w[t * H + hd];
+        if (wt != 0.f)
+          acc[r] = fmaf(wt, __ldcg(part_o + ((size_t)(sb + t) * H + hd) * kHeadDim + d), acc[r]);
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int r = 0; r < H / 2; ++r) out[(hg2 + 2 * r) * kHeadDim + d] = acc[r];
+}
+
+}  // namespace hs2

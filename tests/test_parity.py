@@ -1,0 +1,177 @@
+"""GPU parity: libhs2 (through its C ABI) against the float64 oracle.
+
+Index sets must equal the oracle's except inside the tie band (gap between the
+k-th and (k+1)-th importance below 1e-6 relative); outputs within max-abs 2e-3
+(bf16 cache) or 1e-2 (FP8 cache); lse within 1e-4.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_token_b200 import hs2, workloads
+from _util import check_index_set
+
+pytestmark = [pytest.mark.gpu, pytest.mark.filterwarnings("ignore::RuntimeWarning")]
+
+TOL = {"bf16": 2e-3, "fp8": 1e-2}
+LSE_TOL = 1e-4
+
+
+def run_gpu(inp: workloads.Inputs, twice: bool = False):
+    dev = torch.device("cuda:0")
+    cache = hs2.Cache(inp.k.to(dev), inp.v.to(dev), inp.lens.to(dev),
+                      None if inp.k_scale is None else inp.k_scale.to(dev),
+                      None if inp.v_scale is None else inp.v_scale.to(dev))
+    q = inp.q.to(dev)
+    ws = hs2.alloc_workspace(cache, inp.n_q, inp.h_q, inp.window, inp.k_sel)
+    runs = []
+    for _ in range(2 if twice else 1):
+        out, idx, lse = hs2.full_attn_select(q, cache, inp.window, inp.k_sel, inp.sm_scale, ws)
+        sp = [hs2.sparse_attn(ql.to(dev), cache, idx, ws, inp.sm_scale) for ql in inp.q_layers]
+        torch.cuda.synchronize()
+        runs.append(dict(out=out.cpu().numpy(), idx=idx.cpu().numpy(), lse=lse.cpu().numpy(),
+                         sparse=[s.cpu().numpy() for s in sp]))
+    status = hs2.check_device_status(ws)
+    return runs, status
+
+
+def compare(inp: workloads.Inputs, res: dict, sparse_full: bool = True):
+    bits = workloads.numpy_bits(inp)
+    ref = oracle.full_attn_select(bits, keep_importance=True)
+    tol = TOL[inp.kv]
+    err = np.abs(res["out"] - ref["out"]).max()
+    assert err < tol, f"full-layer output max-abs error {err}"
+    lerr = np.abs(res["lse"] - ref["lse"]).max()
+    assert lerr < LSE_TOL, f"lse error {lerr}"
+    B, n_q = inp.batch, inp.n_q
+    n_exact = 0
+    for b in range(B):
+        L = int(inp.lens[b])
+        for i in range(n_q):
+            p = L - n_q + i
+            msg = check_index_set(res["idx"][b, i], ref["idx"][b, i], ref["imp"][b * n_q + i],
+                                  p, inp.window, inp.k_sel)
+            assert msg is None, f"(b={b}, i={i}, p={p}): {msg}"
+            n_exact += int(np.array_equal(res["idx"][b, i], ref["idx"][b, i]))
+    # Sparse layers: fed the GPU's own index set (identical to the oracle's outside
+    # the tie band), compared with the oracle's sparse layer on that set.
+    for li, ql in enumerate(bits["q_layers"]):
+        want = oracle.sparse_attn(bits, ql, res["idx"] if sparse_full else ref["idx"])
+        e = np.abs(res["sparse"][li] - want).max()
+        assert e < tol, f"sparse layer {li} max-abs error {e}"
+    return n_exact
+
+
+SMALL = [
+    dict(id="b1-L4096-h16-bf16", batch=1, max_len=4096, n_q=1, h_q=16, kv="bf16", seed=101,
+         n_needles=8, needle_layout="uniform"),
+    dict(id="ragged-b3-bf16", batch=3, max_len=5000, n_q=1, h_q=16, kv="bf16", seed=102,
+         lens=[5000, 1200, 1153]),
+    dict(id="short-contexts", batch=5, max_len=1300, n_q=1, h_q=16, kv="bf16", seed=103,
+         lens=[1, 100, 128, 1152, 1153]),
+    dict(id="h64-fp8-ragged", batch=2, max_len=3000, n_q=1, h_q=64, kv="fp8", seed=104,
+         lens=[3000, 2901]),
+    dict(id="h32-append4", batch=1, max_len=2500, n_q=4, h_q=32, kv="bf16", seed=105),
+    dict(id="h128-bf16", batch=1, max_len=2000, n_q=1, h_q=128, kv="bf16", seed=106),
+    dict(id="h48-fp8", batch=2, max_len=1800, n_q=2, h_q=48, kv="fp8", seed=107,
+         lens=[1800, 1500]),
+    dict(id="tiny-window4-k8", batch=2, max_len=48, n_q=3, h_q=16, kv="bf16", seed=108,
+         lens=[48, 13], window=4, k_sel=8),
+    dict(id="window1-k1", batch=1, max_len=300, n_q=2, h_q=16, kv="fp8", seed=109,
+         window=1, k_sel=1),
+    dict(id="max-width-4096", batch=1, max_len=10000, n_q=1, h_q=16, kv="bf16", seed=110,
+         window=128, k_sel=3968),
+    dict(id="append64-fp8", batch=1, max_len=3000, n_q=64, h_q=16, kv="fp8", seed=111),
+    dict(id="ragged-tail-fp8", batch=3, max_len=9000, n_q=1, h_q=16, kv="fp8", seed=112,
+         lens=[8999, 4097, 1333]),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: c["id"])
+def test_small_cases_match_oracle(case):
+    kw = {k: v for k, v in case.items() if k != "id"}
+    inp = workloads.make_inputs(n_sparse=2, **kw)
+    runs, status = run_gpu(inp)
+    assert status == 0
+    compare(inp, runs[0])
+
+
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+def test_zero_query_ties_pick_lowest_positions(kv):
+    inp = workloads.make_inputs(2, 20000, n_q=1, h_q=16, kv=kv, seed=120, q_zero=True,
+                                lens=[20000, 7000])
+    runs, status = run_gpu(inp)
+    assert status == 0
+    for b, L in enumerate([20000, 7000]):
+        want = np.concatenate([np.arange(1024), np.arange(L - 128, L)])
+        assert np.array_equal(runs[0]["idx"][b, 0], want)
+    compare(inp, runs[0])
+
+
+def test_identical_keys_are_all_ties():
+    inp = workloads.make_inputs(1, 6000, n_q=2, h_q=16, seed=121, identical_keys=True)
+    runs, status = run_gpu(inp)
+    assert status == 0
+    for i in range(2):
+        p = 6000 - 2 + i
+        want = np.concatenate([np.arange(1024), np.arange(p - 127, p + 1)])
+        assert np.array_equal(runs[0]["idx"][0, i], want)
+    compare(inp, runs[0])
+
+
+def test_repeat_runs_are_bitwise_identical():
+    inp = workloads.make_inputs(2, 9000, n_q=1, h_q=16, kv="fp8", seed=122, n_sparse=1)
+    runs, _ = run_gpu(inp, twice=True)
+    a, b = runs
+    assert np.array_equal(a["idx"], b["idx"])
+    assert np.array_equal(a["out"], b["out"]) and np.array_equal(a["lse"], b["lse"])
+    assert np.array_equal(a["sparse"][0], b["sparse"][0])
+
+
+def test_device_status_reports_bad_index_and_length():
+    dev = torch.device("cuda:0")
+    inp = workloads.make_inputs(2, 600, n_q=1, h_q=16, seed=123, lens=[600, 300])
+    cache = hs2.Cache(inp.k.to(dev), inp.v.to(dev), inp.lens.to(dev))
+    ws = hs2.alloc_workspace(cache, 1, 16)
+    idx = torch.full((2, 1, 8), -1, dtype=torch.int32, device=dev)
+    idx[0, 0, :3] = torch.tensor([0, 5, 599])
+    idx[1, 0, 0] = 300                     # == lens[1]: out of range
+    hs2.sparse_attn(inp.q.to(dev), cache, idx, ws)
+    assert hs2.check_device_status(ws) == 6
+    assert hs2.check_device_status(ws) == 0          # cleared by the read
+    bad = hs2.Cache(inp.k.to(dev), inp.v.to(dev), torch.tensor([601, 300], dtype=torch.int32,
+                                                                device=dev))
+    hs2.full_attn_select(inp.q.to(dev), bad, workspace=ws)
+    assert hs2.check_device_status(ws) == 7
+
+
+def test_sparse_layer_skips_padding_and_empty_rows():
+    dev = torch.device("cuda:0")
+    inp = workloads.make_inputs(1, 500, n_q=2, h_q=16, seed=124, n_sparse=1)
+    cache = hs2.Cache(inp.k.to(dev), inp.v.to(dev), inp.lens.to(dev))
+    ws = hs2.alloc_workspace(cache, 2, 16)
+    idx = torch.full((1, 2, 300), -1, dtype=torch.int32, device=dev)
+    idx[0, 0, 7:200] = torch.arange(100, 293, dtype=torch.int32)
+    out = hs2.sparse_attn(inp.q_layers[0].to(dev), cache, idx, ws).cpu().numpy()
+    assert hs2.check_device_status(ws) == 0
+    bits = workloads.numpy_bits(inp)
+    want = oracle.sparse_attn(bits, bits["q_layers"][0][:, :1], idx[:, :1].cpu().numpy())
+    assert np.abs(out[:, :1] - want).max() < 2e-3
+    assert np.all(out[0, 1] == 0.0)          # an empty index row yields zeros
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("n", sorted(workloads.WORKLOADS))
+def test_full_size_workloads_match_oracle(n):
+    w = workloads.WORKLOADS[n]
+    inp = workloads.generate(w)
+    runs, status = run_gpu(inp)
+    assert status == 0
+    compare(inp, runs[0])
+    idx = runs[0]["idx"]
+    for b, needles in enumerate(inp.needles):
+        for pos, _ in needles:
+            assert pos in idx[b, w.n_q - 1], f"needle at {pos} not selected"
