@@ -29,7 +29,7 @@ STATUS = {
 
 EXPORTS = ("hs2_workspace_bytes", "hs2_full_attn_select", "hs2_full_attn", "hs2_select",
            "hs2_sparse_attn", "hs2_check_device_status", "hs2_status_string",
-           "hs2_last_cuda_error", "hs2_abi_version")
+           "hs2_last_cuda_error", "hs2_abi_version", "hs2_sparse_attn_noalloc")
 
 
 class Hs2Error(RuntimeError):
@@ -77,6 +77,8 @@ def lib():
     L.hs2_select.restype = i32
     L.hs2_sparse_attn.argtypes = [vp, i32, i32, kvp, vp, i32, f32, vp, vp, sz, vp]
     L.hs2_sparse_attn.restype = i32
+    L.hs2_sparse_attn_noalloc.argtypes = [vp, i32, i32, kvp, vp, i32, f32, vp, vp, vp]
+    L.hs2_sparse_attn_noalloc.restype = i32
     L.hs2_check_device_status.argtypes = [vp, vp]
     L.hs2_check_device_status.restype = i32
     L.hs2_status_string.argtypes = [i32]
