@@ -1,0 +1,463 @@
+// Full-attention layer on the 5th-generation tensor cores (bf16 cache, h_q <= 64).
+//
+// Split-K flash-decode of the hybrid block's full layer (toolnavs article 2080, fr
+// "Ce que fait HySparse2": the full layer attends over the whole context; MQA per
+// "Les chiffres mesurés").  One CTA per key chunk of one (sequence, query token):
+//
+//   warp 0      TMA producer: 128-key K and V tiles (two 64-column boxes each,
+//               128-byte swizzle) into an NS-stage ring, K and V on separate
+//               barriers;
+//   warp 1      TMEM allocator, MMA issuer:
+//                 S^T[128 keys x H] = K_tile . Q^T          (8 x K=16, TMEM ping-pong)
+//                 O^T[128 d x H]  += V_tile^T . (P_hi + P_lo)^T  (16 x K=16)
+//               the P.V of tile i-1 is issued after the Q.K of tile i;
+//   warps 2..5  softmax: thread t owns key t of the tile (TMEM lane t).  Logits go to
+//               the log2 domain, x = s * sm_scale * log2(e) - m_h; the per-head
+//               reference m_h only moves when some x exceeds 8 (then the tile max
+//               is taken across the 128 threads and O is rescaled in TMEM), so the
+//               common tile needs no cross-thread reduction.  p = 2^x is split into
+//               bf16 hi + lo so that P.V keeps ~16 bits of p; per-thread partial
+//               sums l_h are reduced once at the end of the chunk.
+// The last CTA of each (sequence, token) merges the chunk partials (ticket, no
+// spin-wait) into out, lse and the selection shift delta_h.
+#include <cuda_bf16.h>
+
+#include "hs2_internal.cuh"
+#include "sm100.cuh"
+#include "tc_common.cuh"
+#include "tile_simt.cuh"
+
+namespace hs2 {
+
+using namespace sm100;
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleAt = 8.0f;  // log2 units: move the reference when p would exceed 2^8
+
+template <int H>
+struct FullSmem {
+  static constexpr int kStages = H <= 16 ? 3 : 2;
+  static constexpr uint32_t kTile = kKTileBytesBf16;    // one K or V tile
+  static constexpr uint32_t kQBytes = H * kHeadDim * 2;
+  static constexpr uint32_t kPBytes = kKeyTile * H * 2;  // one of hi / lo
+  static constexpr uint32_t kKOff = 0;
+  static constexpr uint32_t kVOff = kStages * kTile;
+  static constexpr uint32_t kQOff = 2 * kStages * kTile;
+  static constexpr uint32_t kPOff = kQOff + kQBytes;        // [2 buffers][hi, lo]
+  static constexpr uint32_t kRedOff = kPOff + 4 * kPBytes;  // [4 warps][H] floats
+  static constexpr uint32_t kRefOff = kRedOff + 4 * H * 4;  // [H] reference, [H] alpha
+  static constexpr uint32_t kBarOff = kRefOff + 2 * H * 4;
+  static constexpr uint32_t kBars = 4 * kStages + 9;
+  static constexpr uint32_t kSlotOff = kBarOff + kBars * 8;
+  static constexpr uint32_t kBytes = kSlotOff + 16 + 1024;
+  static constexpr uint32_t kTmemCols = tmem_cols_pow2(3 * H);
+  static_assert(kBytes <= 227 * 1024, "shared memory budget");
+};
+
+template <int H>
+__device__ void merge_log2_partials(const FullParams& p, int bq, uint8_t* smem);
+
+// Largest value of v over the 128 softmax threads, per head (named barrier 1).
+template <int H>
+__device__ __forceinline__ void block_max_heads(const float (&v)[H], float* red, float* out,
+                                                int t) {
+  const int w = t >> 5, lane = t & 31;
+#pragma unroll
+  for (int h = 0; h < H; ++h) {
+    const float m = warp_max(v[h]);
+    if (lane == 0) red[w * H + h] = m;
+  }
+  named_bar_sync(1, 128);
+  if (t < H) out[t] = fmaxf(fmaxf(red[t], red[H + t]), fmaxf(red[2 * H + t], red[3 * H + t]));
+  named_bar_sync(1, 128);
+}
+
+template <int H>
+__global__ void __launch_bounds__(192, 1)
+    full_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                        const __grid_constant__ CUtensorMap tmap_v, FullParams p) {
+  using L = FullSmem<H>;
+  constexpr int NS = L::kStages;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* kst = smem + L::kKOff;
+  uint8_t* vst = smem + L::kVOff;
+  uint8_t* qs = smem + L::kQOff;
+  uint8_t* ps = smem + L::kPOff;
+  float* red = reinterpret_cast<float*>(smem + L::kRedOff);
+  float* mref_s = reinterpret_cast<float*>(smem + L::kRefOff);
+  float* alpha_s = mref_s + H;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* kfull = bars;
+  uint64_t* kempty = bars + NS;
+  uint64_t* vfull = bars + 2 * NS;
+  uint64_t* vempty = bars + 3 * NS;
+  uint64_t* s_full = bars + 4 * NS;      // [2]
+  uint64_t* s_free = s_full + 2;         // [2]
+  uint64_t* p_full = s_full + 4;         // [2]
+  uint64_t* p_free = s_full + 6;         // [2]
+  uint64_t* mma_done = s_full + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
+
+  const int warp = threadIdx.x >> 5;
+  const int split = blockIdx.x, bq = blockIdx.y;
+  const int b = bq / p.n_q, qi = bq % p.n_q;
+  const int Lb = seq_len(p.kv, b, p.n_q, p.status, split == 0 && qi == 0);
+  const int pos = Lb - p.n_q + qi;
+  const int k0 = split * p.chunk1;
+  const int k1 = min(k0 + p.chunk1, pos + 1);
+  const int n_tiles = k0 < k1 ? (k1 - k0 + kKeyTile - 1) / kKeyTile : 0;
+  const size_t pidx = (size_t)bq * p.splits1 + split;
+
+  if (n_tiles == 0) {
+    // Empty chunk: an empty partial (no key), then take part in the merge ticket.
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
+      p.part_ml[pidx * H * 2 + 2 * h] = -INFINITY;
+      p.part_ml[pidx * H * 2 + 2 * h + 1] = 0.f;
+    }
+  } else {
+    if (threadIdx.x == 0) {
+      for (int s = 0; s < NS; ++s) {
+        mbar_init(kfull + s, 1);
+        mbar_init(kempty + s, 1);
+        mbar_init(vfull + s, 1);
+        mbar_init(vempty + s, 1);
+      }
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(s_full + s, 1);
+        mbar_init(s_free + s, 128);
+        mbar_init(p_full + s, 128);
+        mbar_init(p_free + s, 1);
+      }
+      mbar_init(mma_done, 1);
+      fence_mbar_init();
+    }
+    if (warp == 1) {
+      tmem_alloc(tmem_slot, L::kTmemCols);
+      tmem_relinquish();
+    }
+    if (warp == 0 && lane_id() == 0) {
+      prefetch_tmap(&tmap_k);
+      prefetch_tmap(&tmap_v);
+    }
+    store_q_kmajor<H>(qs, p.q + (size_t)bq * H * kHeadDim, threadIdx.x, blockDim.x);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t tmem_o = tmem_base + 2 * H;
+    bool ok = true;
+
+    if (warp == 0) {
+      // ------------------------------------------------------------ TMA producer
+      if (elect_one()) {
+        const uint64_t pol = policy_evict_first();
+        const int row0 = b * p.kv.max_len + k0;
+        int issued = 0;
+        for (int i = 0; i < n_tiles && ok; ++i) {
+          const int s = i % NS;
+          const uint32_t ph = ((i / NS) & 1) ^ 1;
+          const int row = row0 + i * kKeyTile;
+          if (!mbar_wait(kempty + s, ph)) { ok = false; break; }
+          mbar_arrive_expect_tx(kfull + s, L::kTile);
+          tma_load_2d(kst + s * L::kTile, &tmap_k, kfull + s, 0, row, pol);
+          tma_load_2d(kst + s * L::kTile + kBoxBytes, &tmap_k, kfull + s, 64, row, pol);
+          if (!mbar_wait(vempty + s, ph)) { ok = false; break; }
+          mbar_arrive_expect_tx(vfull + s, L::kTile);
+          tma_load_2d(vst + s * L::kTile, &tmap_v, vfull + s, 0, row, pol);
+          tma_load_2d(vst + s * L::kTile + kBoxBytes, &tmap_v, vfull + s, 64, row, pol);
+          issued = i + 1;
+        }
+        for (int i = issued > NS ? issued - NS : 0; i < issued; ++i) {
+          if (!mbar_wait(kfull + (i % NS), (i / NS) & 1)) ok = false;
+          if (!mbar_wait(vfull + (i % NS), (i / NS) & 1)) ok = false;
+        }
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (elect_one()) {
+        const uint32_t id_qk = idesc_f16(128, H, true, false, false);
+        const uint32_t id_pv = idesc_f16(128, H, true, true, true);
+        const uint32_t q_addr = smem_u32(qs);
+        auto issue_pv = [&](int t) -> bool {
+          const int s = t % NS, pb = t & 1;
+          if (!mbar_wait(vfull + s, (t / NS) & 1)) return false;
+          if (!mbar_wait(p_full + pb, (t >> 1) & 1)) return false;
+          tc_fence_after();
+          const uint32_t v_addr = smem_u32(vst + s * L::kTile);
+          const uint32_t p_hi = smem_u32(ps + (2 * pb) * L::kPBytes);
+          const uint32_t p_lo = p_hi + L::kPBytes;
+#pragma unroll
+          for (int kk = 0; kk < kKeyTile / 16; ++kk)
+            mma_f16_ss(tmem_o, vt_mnmajor_sw128_desc(v_addr, kk), pt_mnmajor_desc(p_hi, kk),
+                       id_pv, (t > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < kKeyTile / 16; ++kk)
+            mma_f16_ss(tmem_o, vt_mnmajor_sw128_desc(v_addr, kk), pt_mnmajor_desc(p_lo, kk),
+                       id_pv, 1u);
+          mma_commit(p_free + pb);
+          mma_commit(vempty + s);
+          return true;
+        };
+        for (int i = 0; i < n_tiles && ok; ++i) {
+          const int s = i % NS, sb = i & 1;
+          if (!mbar_wait(kfull + s, (i / NS) & 1)) { ok = false; break; }
+          if (!mbar_wait(s_free + sb, ((i >> 1) & 1) ^ 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(kst + s * L::kTile);
+#pragma unroll
+          for (int kk = 0; kk < kHeadDim / 16; ++kk)
+            mma_f16_ss(tmem_base + sb * H, kmajor_sw128_desc(k_addr, kk),
+                       q_kmajor_desc<H>(q_addr, kk), id_qk, kk > 0 ? 1u : 0u);
+          mma_commit(s_full + sb);
+          mma_commit(kempty + s);
+          if (i > 0 && !issue_pv(i - 1)) { ok = false; break; }
+        }
+        if (ok && !issue_pv(n_tiles - 1)) ok = false;
+        mma_commit(mma_done);
+        if (!mbar_wait(mma_done, 0)) ok = false;
+      }
+    } else {
+      // ------------------------------------------------------------ softmax
+      const int lg = warp & 3;
+      const int t = lg * 32 + (int)lane_id();  // key of the tile == TMEM lane
+      const uint32_t lane_base = (uint32_t)(lg * 32) << 16;
+      const float c2 = p.sm_scale * kLog2e;
+      float l[H];
+#pragma unroll
+      for (int h = 0; h < H; ++h) l[h] = 0.f;
+      if (t < H) mref_s[t] = -INFINITY;
+      named_bar_sync(1, 128);
+      for (int i = 0; i < n_tiles; ++i) {
+        // A failed wait in any softmax thread stops the waits of all of them (they
+        // keep taking part in the named barriers, so none is left behind).
+        const int sb = i & 1;
+        if (ok && !mbar_wait(s_full + sb, (i >> 1) & 1)) ok = false;
+        if (named_bar_or(3, 128, !ok)) ok = false;
+        tc_fence_after();
+        float x[H];
+#pragma unroll
+        for (int c = 0; c < H; c += 16) {
+          uint32_t r[16];
+          tmem_ld16(tmem_base + lane_base + sb * H + c, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) x[c + e] = __uint_as_float(r[e]) * c2;
+        }
+        tc_fence_before();
+        mbar_arrive(s_free + sb);
+        const int j = k0 + i * kKeyTile + t;
+        const bool valid = j < k1;
+        bool over = false;
+#pragma unroll
+        for (int h = 0; h < H; ++h) {
+          if (!valid) x[h] = -INFINITY;
+          over |= x[h] - mref_s[h] > kRescaleAt;
+        }
+        if (named_bar_or(2, 128, over)) {
+          // New per-head reference: the larger of the old one and this tile's max.
+          block_max_heads<H>(x, red, alpha_s, t);
+          if (t < H) {
+            const float mnew = fmaxf(mref_s[t], alpha_s[t]);
+            alpha_s[t] = exp2f(mref_s[t] - mnew);  // 0 on the first tile
+            mref_s[t] = mnew;
+          }
+          named_bar_sync(1, 128);
+#pragma unroll
+          for (int h = 0; h < H; ++h) l[h] *= alpha_s[h];
+          if (i > 0) {
+            // O holds the P.V of tiles < i: wait for the last one, then rescale.
+            if (ok && !mbar_wait(p_free + ((i - 1) & 1), ((i - 1) >> 1) & 1)) ok = false;
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < H; c += 16) {
+              uint32_t r[16];
+              tmem_ld16(tmem_o + lane_base + c, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha_s[c + e]);
+              tmem_st16(tmem_o + lane_base + c, r);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+          }
+        }
+        // P for this tile into buffer sb (free once the P.V of tile i-2 is done).
+        if (ok && i >= 2 && !mbar_wait(p_free + sb, ((i >> 1) & 1) ^ 1)) ok = false;
+        uint8_t* phi = ps + (2 * sb) * L::kPBytes;
+        uint8_t* plo = phi + L::kPBytes;
+#pragma unroll
+        for (int c = 0; c < H / 8; ++c) {
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int h0 = c * 8 + 2 * e;
+            const float p0 = exp2f(x[h0] - mref_s[h0]);
+            const float p1 = exp2f(x[h0 + 1] - mref_s[h0 + 1]);
+            l[h0] += p0;
+            l[h0 + 1] += p1;
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
+            const float2 hf = __bfloat1622float2(hi);
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+            hw[e] = *reinterpret_cast<const uint32_t*>(&hi);
+            lw[e] = *reinterpret_cast<const uint32_t*>(&lo);
+          }
+          *reinterpret_cast<uint4*>(phi + c * (kKeyTile * 16) + t * 16) =
+              make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(plo + c * (kKeyTile * 16) + t * 16) =
+              make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+        if (!valid && i == n_tiles - 1) {
+          // Rows past the chunk end may hold anything (NaN included); 0 * NaN would
+          // poison P.V, so zero this key's V row once its tile has landed.
+          const int s = i % NS;
+          if (ok && !mbar_wait(vfull + s, (i / NS) & 1)) ok = false;
+          uint4* v0 = reinterpret_cast<uint4*>(vst + s * L::kTile + t * 128);
+          uint4* v1 = reinterpret_cast<uint4*>(vst + s * L::kTile + kBoxBytes + t * 128);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            v0[e] = make_uint4(0, 0, 0, 0);
+            v1[e] = make_uint4(0, 0, 0, 0);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(p_full + sb);
+      }
+      // Epilogue: O^T row t is dimension t of every head; l is reduced across threads.
+      const int last = n_tiles - 1;
+      if (ok && !mbar_wait(p_free + (last & 1), (last >> 1) & 1)) ok = false;
+      tc_fence_after();
+      float* po = p.part_o + pidx * H * kHeadDim;
+#pragma unroll
+      for (int c = 0; c < H; c += 16) {
+        uint32_t r[16];
+        tmem_ld16(tmem_o + lane_base + c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) po[(c + e) * kHeadDim + t] = __uint_as_float(r[e]);
+      }
+      tc_fence_before();
+#pragma unroll
+      for (int h = 0; h < H; ++h) {
+        const float s = warp_sum(l[h]);
+        if (lane_id() == 0) red[(warp & 3) * H + h] = s;
+      }
+      named_bar_sync(1, 128);
+      if (t < H) {
+        p.part_ml[pidx * H * 2 + 2 * t] = mref_s[t];
+        p.part_ml[pidx * H * 2 + 2 * t + 1] = red[t] + red[H + t] + red[2 * H + t] + red[3 * H + t];
+      }
+    }
+    if (!ok) set_status(p.status, HS2_ERR_DEVICE_TIMEOUT);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem_base, L::kTmemCols);
+    }
+  }
+
+  // Merge of the chunk partials by the last CTA of this (sequence, token).
+  if (!arrive_last(p.tickets + bq, p.splits1)) return;
+  merge_log2_partials<H>(p, bq, smem);
+}
+
+// Merge of the chunk partials (m in log2 units, l, unnormalised o) of one
+// (sequence, token): out = sum_s 2^(m_s - M) o_s / L, lse = (M + log2 L) ln 2,
+// delta_h = lse_h - min_h' lse_h'.  Run by one CTA (any thread count).
+template <int H>
+__device__ void merge_log2_partials(const FullParams& p, int bq, uint8_t* smem) {
+  const int S = p.splits1, nt = blockDim.x, tid = threadIdx.x;
+  const float* pml = p.part_ml + (size_t)bq * S * H * 2;
+  const float* po = p.part_o + (size_t)bq * S * H * kHeadDim;
+  double* lse_d = reinterpret_cast<double*>(smem);          // [H + 1]
+  float* Mf = reinterpret_cast<float*>(lse_d + H + 1);       // [H]
+  float* invL = Mf + H;                                      // [H]
+  float* w = invL + H;                                       // [32][H]
+  for (int h = tid; h < H; h += nt) {
+    float M = -INFINITY;
+    for (int sp = 0; sp < S; ++sp) M = fmaxf(M, __ldcg(pml + ((size_t)sp * H + h) * 2));
+    double Ls = 0.0;
+    if (M != -INFINITY)
+      for (int sp = 0; sp < S; ++sp) {
+        const float m = __ldcg(pml + ((size_t)sp * H + h) * 2);
+        const float l = __ldcg(pml + ((size_t)sp * H + h) * 2 + 1);
+        if (l > 0.f) Ls += (double)l * exp2((double)m - (double)M);
+      }
+    Mf[h] = M;
+    invL[h] = Ls > 0.0 ? (float)(1.0 / Ls) : 0.f;
+    lse_d[h] = Ls > 0.0 ? ((double)M + log2(Ls)) * 0.69314718055994530942 : -INFINITY;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    double mn = INFINITY;
+    for (int h = 0; h < H; ++h) mn = fmin(mn, lse_d[h]);
+    lse_d[H] = mn;
+  }
+  __syncthreads();
+  for (int h = tid; h < H; h += nt) {
+    const double l = lse_d[h], dl = l - lse_d[H];
+    p.lse64[(size_t)bq * H + h] = l;
+    p.delta64[(size_t)bq * H + h] = dl;
+    p.delta32[(size_t)bq * H + h] = (float)dl;
+    if (p.lse_out) p.lse_out[(size_t)bq * H + h] = (float)l;
+  }
+  float* out = p.out + (size_t)bq * H * kHeadDim;
+  for (int e0 = 0; e0 < H * kHeadDim; e0 += nt) {
+    const int e = e0 + tid;
+    float acc = 0.f;
+    for (int sb = 0; sb < S; sb += 32) {
+      __syncthreads();
+      for (int x = tid; x < 32 * H; x += nt) {
+        const int sp = sb + x / H, h = x % H;
+        float wt = 0.f;
+        if (sp < S && Mf[h] != -INFINITY) {
+          const float m = __ldcg(pml + ((size_t)sp * H + h) * 2);
+          const float l = __ldcg(pml + ((size_t)sp * H + h) * 2 + 1);
+          if (l > 0.f) wt = exp2f(m - Mf[h]) * invL[h];
+        }
+        w[x] = wt;
+      }
+      __syncthreads();
+      if (e < H * kHeadDim) {
+        const int h = e / kHeadDim;
+        const int ns = min(32, S - sb);
+        for (int t = 0; t < ns; ++t) {
+          const float wt = w[t * H + h];
+          if (wt != 0.f) acc = fmaf(wt, __ldcg(po + ((size_t)(sb + t) * H) * kHeadDim + e), acc);
+        }
+      }
+    }
+    if (e < H * kHeadDim) out[e] = acc;
+  }
+}
+
+template <int H>
+static cudaError_t launch_full_tc_t(const FullParams& p, const CUtensorMap& tk,
+                                    const CUtensorMap& tv, int bq, cudaStream_t st) {
+  using L = FullSmem<H>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(full_attn_tc_kernel<H>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  full_attn_tc_kernel<H><<<dim3(p.splits1, bq), 192, L::kBytes, st>>>(tk, tv, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_full_attn_tc(const FullParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                                int bq, cudaStream_t st) {
+  switch (p.h) {
+    case 16: return launch_full_tc_t<16>(p, tk, tv, bq, st);
+    case 32: return launch_full_tc_t<32>(p, tk, tv, bq, st);
+    case 48: return launch_full_tc_t<48>(p, tk, tv, bq, st);
+    case 64: return launch_full_tc_t<64>(p, tk, tv, bq, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace hs2

@@ -4,6 +4,7 @@
 #include <string.h>
 
 #include "hs2_internal.cuh"
+#include "tc_common.cuh"
 
 namespace hs2 {
 
@@ -165,7 +166,28 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
   p.delta64 = ws_ptr<double>(ws, w.delta64);
   p.delta32 = ws_ptr<float>(ws, w.delta32);
   p.status = ws_ptr<uint32_t>(ws, w.status);
-  cudaError_t e = launch_full_attn(p, kv->batch, s);
+  cudaError_t e;
+  if (kv->dtype == HS2_KV_BF16 && h <= 64) {
+    // Tensor-core flash-decode: about one CTA per SM, chunks of whole 128-key tiles.
+    CUtensorMap tk, tv;
+    const uint64_t rows = (uint64_t)kv->batch * kv->max_len;
+    if (!make_tmap_2d(&tk, kv->k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kHeadDim, rows,
+                      kHeadDim * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_2d(&tv, kv->v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kHeadDim, rows,
+                      kHeadDim * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cuda_fail(cudaErrorInvalidValue, "tensor maps of K/V");
+    const int bq = kv->batch * n_q;
+    int splits = device_sm_count() / bq;
+    if (splits > w.splits1) splits = w.splits1;
+    if (splits < 1) splits = 1;
+    int chunk = (kv->max_len + splits - 1) / splits;
+    chunk = (chunk + 127) / 128 * 128;
+    p.splits1 = (kv->max_len + chunk - 1) / chunk;
+    p.chunk1 = chunk;
+    e = launch_full_attn_tc(p, tk, tv, bq, s);
+  } else {
+    e = launch_full_attn(p, kv->batch, s);
+  }
   return e == cudaSuccess ? HS2_OK : cuda_fail(e, "full-attention launch");
 }
 
@@ -200,7 +222,26 @@ static hs2_status run_select(const void* q, int n_q, int h, const hs2_kv* kv, in
   p.band_j = ws_ptr<int32_t>(ws, w.band_j);
   p.idx = idx;
   p.status = ws_ptr<uint32_t>(ws, w.status);
-  e = launch_select(p, kv->batch, s);
+  const int bq = kv->batch * n_q;
+  if (kv->dtype == HS2_KV_BF16) {
+    // Tensor-core importance pass: one CTA per SM per key chunk (128-key multiples).
+    CUtensorMap tk;
+    if (!make_tmap_2d(&tk, kv->k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kHeadDim,
+                      (uint64_t)kv->batch * kv->max_len, kHeadDim * 2, 64, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+      return cuda_fail(cudaErrorInvalidValue, "tensor map of K");
+    int splits = device_sm_count() / bq;
+    if (splits < 1) splits = 1;
+    int chunk = (kv->max_len + splits - 1) / splits;
+    chunk = (chunk + 127) / 128 * 128;
+    p.splits2 = (kv->max_len + chunk - 1) / chunk;
+    p.chunk2 = chunk;
+    e = launch_importance_tc(p, tk, bq, s);
+    if (e != cudaSuccess) return cuda_fail(e, "importance launch");
+    e = launch_select_rest(p, kv->batch, s);
+  } else {
+    e = launch_select(p, kv->batch, s);
+  }
   return e == cudaSuccess ? HS2_OK : cuda_fail(e, "selection launch");
 }
 

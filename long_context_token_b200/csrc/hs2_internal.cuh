@@ -52,6 +52,7 @@ struct WsLayout {
 };
 
 int plan_splits1(int bq, int max_len, int num_sms);
+int device_sm_count();
 int plan_splits4(int idx_width);
 bool make_layout(int batch, int n_q, int h, int max_len, int window, int k_sel,
                  WsLayout* L);
@@ -130,6 +131,8 @@ struct SparseParams {
 // Launchers (each returns the launch's cudaError_t).
 cudaError_t launch_full_attn(const FullParams& p, int batch, cudaStream_t s);
 cudaError_t launch_select(const SelectParams& p, int batch, cudaStream_t s);
+// The selection after the importance pass (compaction + finish).
+cudaError_t launch_select_rest(const SelectParams& p, int batch, cudaStream_t s);
 cudaError_t launch_sparse_attn(const SparseParams& p, int batch, cudaStream_t s);
 
 // ---------------------------------------------------------------------------

@@ -377,6 +377,35 @@ static cudaError_t launch_select_t(const SelectParams& p, int batch, cudaStream_
   return cudaGetLastError();
 }
 
+template <int H, bool FP8>
+static cudaError_t launch_rest_t(const SelectParams& p, int batch, cudaStream_t st) {
+  const int bq = batch * p.n_q;
+  select_compact_kernel<<<dim3(p.splits3, bq), kThreads, 0, st>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  select_finish_kernel<H, FP8><<<bq, kFinThreads, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <bool FP8>
+static cudaError_t launch_rest_h(const SelectParams& p, int batch, cudaStream_t st) {
+  switch (p.h) {
+    case 16: return launch_rest_t<16, FP8>(p, batch, st);
+    case 32: return launch_rest_t<32, FP8>(p, batch, st);
+    case 48: return launch_rest_t<48, FP8>(p, batch, st);
+    case 64: return launch_rest_t<64, FP8>(p, batch, st);
+    case 80: return launch_rest_t<80, FP8>(p, batch, st);
+    case 96: return launch_rest_t<96, FP8>(p, batch, st);
+    case 112: return launch_rest_t<112, FP8>(p, batch, st);
+    case 128: return launch_rest_t<128, FP8>(p, batch, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_select_rest(const SelectParams& p, int batch, cudaStream_t st) {
+  return p.kv.fp8 ? launch_rest_h<true>(p, batch, st) : launch_rest_h<false>(p, batch, st);
+}
+
 template <bool FP8>
 static cudaError_t launch_select_h(const SelectParams& p, int batch, cudaStream_t st) {
   switch (p.h) {

@@ -1,0 +1,72 @@
+// Shared pieces of the tensor-core (tcgen05) kernels: tile geometry, shared-memory
+// layouts of the operands and their descriptors, and host-side TMA tensor maps.
+#pragma once
+
+#include <cuda.h>
+
+#include "hs2_internal.cuh"
+#include "sm100.cuh"
+
+namespace hs2 {
+
+constexpr int kKeyTile = 128;             // keys per MMA tile (the MMA's M)
+constexpr uint32_t kBoxBytes = 16384;     // 128 rows x 64 bf16 (one 128-byte-swizzled box)
+constexpr uint32_t kKTileBytesBf16 = 2 * kBoxBytes;  // 128 keys x 128 d x bf16
+
+__host__ __device__ constexpr uint32_t tmem_cols_pow2(int cols) {
+  return cols <= 32 ? 32u : cols <= 64 ? 64u : cols <= 128 ? 128u : cols <= 256 ? 256u : 512u;
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Q [H heads][128 d] bf16 -> shared memory as the K-major, unswizzled B operand of
+// S^T = K . Q^T: 16-byte chunk c of head h sits at c * (H * 16) + h * 16.
+template <int H>
+__device__ __forceinline__ void store_q_kmajor(uint8_t* qs, const uint16_t* q, int tid, int nt) {
+  for (int e = tid; e < H * (kHeadDim / 8); e += nt) {
+    const int h = e % H, c = e / H;
+    const uint4 v = *reinterpret_cast<const uint4*>(q + h * kHeadDim + c * 8);
+    *reinterpret_cast<uint4*>(qs + c * (H * 16) + h * 16) = v;
+  }
+}
+
+#ifdef __CUDACC__
+// A operand (K tile, K-major, 128-byte swizzle written by TMA): K step kk of 16 d.
+__device__ __forceinline__ uint64_t kmajor_sw128_desc(uint32_t tile_addr, int kk) {
+  const uint32_t start = tile_addr + (uint32_t)(kk >> 2) * kBoxBytes + (uint32_t)(kk & 3) * 32u;
+  return sm100::smem_desc(start, 16, 1024, sm100::kSwizzle128B);
+}
+
+// B operand Q (K-major, unswizzled): K step kk covers chunks 2kk and 2kk+1.
+template <int H>
+__device__ __forceinline__ uint64_t q_kmajor_desc(uint32_t q_addr, int kk) {
+  return sm100::smem_desc(q_addr + (uint32_t)kk * 2u * H * 16u, H * 16, 128, sm100::kSwizzleNone);
+}
+
+// A operand V^T (V tile is [128 keys][128 d] in two 128-byte-swizzled boxes, so V^T is
+// MN-major): K step kk covers keys [16kk, 16kk + 16).
+__device__ __forceinline__ uint64_t vt_mnmajor_sw128_desc(uint32_t tile_addr, int kk) {
+  return sm100::smem_desc(tile_addr + (uint32_t)kk * 16u * 128u, kBoxBytes, 1024,
+                          sm100::kSwizzle128B);
+}
+
+// B operand P^T (P stored [H/8 chunks][128 keys][8 heads], MN-major, unswizzled):
+// K step kk covers keys [16kk, 16kk + 16).
+__device__ __forceinline__ uint64_t pt_mnmajor_desc(uint32_t p_addr, int kk) {
+  return sm100::smem_desc(p_addr + (uint32_t)kk * 256u, 128, kKeyTile * 16, sm100::kSwizzleNone);
+}
+#endif
+
+// Host: 2-D tiled tensor map over a row-major [rows][inner] array.
+bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner,
+                  uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
+                  CUtensorMapSwizzle swizzle);
+
+cudaError_t launch_full_attn_tc(const FullParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                                int bq, cudaStream_t st);
+cudaError_t launch_importance_tc(const SelectParams& p, const CUtensorMap& tmap_k, int bq,
+                                 cudaStream_t st);
+
+}  // namespace hs2
