@@ -145,15 +145,15 @@ HS2_API hs2_status hs2_sparse_attn(const void* q_layer, int n_q, int h_q, const 
 /* One reusing sparse-attention layer for callers that cannot allocate device memory
  * (no counterpart in the paper; a deployment aid).  It computes exactly what
  * hs2_sparse_attn computes, with the same arguments except the workspace: its scratch
- * (split partials and merge tickets) lives in a fixed 4 MiB array inside the library,
+ * (the split partials) lives in a fixed 4 MiB array inside the library,
  * which every GPU that loads the library keeps until the process exits.  Callers that
  * hand out all device memory from their own pool, or that must not call cudaMalloc
  * mid-step (it can synchronise the device), use this entry point.
  *   device_status  device uint32 into which the kernels OR (1 << code) for each
  *                  device-side error (HS2_ERR_INDEX_OUT_OF_RANGE, HS2_ERR_BAD_LENGTH);
  *                  may be NULL to discard them.  The caller clears it.
- * Limit: 256 + 256*ceil(B*n_q*4/256) + B*n_q*ceil(idx_width/64)*h_q*520 bytes (rounded
- * to 256 per region) must fit in 4 MiB, e.g. B*n_q*h_q <= 384 at idx_width 1152;
+ * Limit: 256 + B*n_q*ceil(idx_width/64)*h_q*520 bytes (two regions, each rounded up to
+ * 256) must fit in 4 MiB, e.g. B*n_q*h_q <= 384 at idx_width 1152;
  * larger sizes return HS2_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress)
  * and should come before any stream capture on that device.  All calls on a device

@@ -5,10 +5,8 @@
 // the selection; MQA per "Les chiffres mesurés").
 //
 // Grid: (splits1, batch * n_q).  CTA (split, bq) owns keys
-// [split * chunk1, (split + 1) * chunk1) of its sequence, clipped to [0, p].
-// The last CTA of each (sequence, token) to finish merges all splits (ticket
-// counter, no spin-wait) and also derives delta_h = lse_h - min_h' lse_h', the
-// per-head shift used by the selection pass.
+// [split * chunk1, (split + 1) * chunk1) of its sequence, clipped to [0, p], and
+// writes that chunk's partial (m, l, o); merge.cu combines the chunks.
 #include "tile_simt.cuh"
 
 namespace hs2 {
@@ -54,29 +52,6 @@ __global__ void __launch_bounds__(kThreads) full_attn_simt_kernel(FullParams p) 
   const size_t pidx = (size_t)bq * p.splits1 + split;
   write_partial<H>(s, acc, p.part_o + pidx * H * kHeadDim, p.part_ml + pidx * H * 2);
 
-  if (!arrive_last(p.tickets + bq, p.splits1)) return;
-
-  // Merge (reuses the q/K staging area as scratch; q is no longer needed).
-  double* lse_d = reinterpret_cast<double*>(s.ks);  // H doubles (K tile area >= 16 KB)
-  float* scratch = s.vs;                            // >= 32*H + 2H floats needed
-  merge_partials<H>(p.part_o + (size_t)bq * p.splits1 * H * kHeadDim,
-                    p.part_ml + (size_t)bq * p.splits1 * H * 2, p.splits1,
-                    p.out + (size_t)bq * H * kHeadDim, lse_d, scratch);
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double mn = INFINITY;
-    for (int hd = 0; hd < H; ++hd) mn = fmin(mn, lse_d[hd]);
-    lse_d[H] = mn;
-  }
-  __syncthreads();
-  for (int hd = threadIdx.x; hd < H; hd += kThreads) {
-    const double l = lse_d[hd];
-    const double dl = l - lse_d[H];
-    p.lse64[(size_t)bq * H + hd] = l;
-    p.delta64[(size_t)bq * H + hd] = dl;
-    p.delta32[(size_t)bq * H + hd] = (float)dl;
-    if (p.lse_out) p.lse_out[(size_t)bq * H + hd] = (float)l;
-  }
 }
 
 template <int H, bool FP8>

@@ -18,14 +18,14 @@
 //               common tile needs no cross-thread reduction.  p = 2^x is split into
 //               bf16 hi + lo so that P.V keeps ~16 bits of p; per-thread partial
 //               sums l_h are reduced once at the end of the chunk.
-// The last CTA of each (sequence, token) merges the chunk partials (ticket, no
-// spin-wait) into out, lse and the selection shift delta_h.
+// Each CTA writes its chunk's partial (m in log2 units, l, unnormalised o); merge.cu
+// combines the chunks.
 #include <cuda_bf16.h>
+#include <string.h>
 
 #include "hs2_internal.cuh"
 #include "sm100.cuh"
 #include "tc_common.cuh"
-#include "tile_simt.cuh"
 
 namespace hs2 {
 
@@ -54,9 +54,6 @@ struct FullSmem {
   static_assert(kBytes <= 227 * 1024, "shared memory budget");
 };
 
-template <int H>
-__device__ void merge_log2_partials(const FullParams& p, int bq, uint8_t* smem);
-
 // Largest value of v over the 128 softmax threads, per head (named barrier 1).
 template <int H>
 __device__ __forceinline__ void block_max_heads(const float (&v)[H], float* red, float* out,
@@ -72,7 +69,7 @@ __device__ __forceinline__ void block_max_heads(const float (&v)[H], float* red,
   named_bar_sync(1, 128);
 }
 
-template <int H>
+template <int H, bool GATHER>
 __global__ void __launch_bounds__(192, 1)
     full_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v, FullParams p) {
@@ -104,13 +101,16 @@ __global__ void __launch_bounds__(192, 1)
   const int b = bq / p.n_q, qi = bq % p.n_q;
   const int Lb = seq_len(p.kv, b, p.n_q, p.status, split == 0 && qi == 0);
   const int pos = Lb - p.n_q + qi;
+  // Keys [k0, k1) of the sequence, or (gather mode) index entries [k0, k1) of the row.
   const int k0 = split * p.chunk1;
-  const int k1 = min(k0 + p.chunk1, pos + 1);
+  const int k1 = GATHER ? min(k0 + p.chunk1, p.idx_width) : min(k0 + p.chunk1, pos + 1);
+  const int32_t* idx_row = GATHER ? p.idx + (size_t)bq * p.idx_width : nullptr;
+  const size_t row_base = (size_t)b * p.kv.max_len;
   const int n_tiles = k0 < k1 ? (k1 - k0 + kKeyTile - 1) / kKeyTile : 0;
   const size_t pidx = (size_t)bq * p.splits1 + split;
 
   if (n_tiles == 0) {
-    // Empty chunk: an empty partial (no key), then take part in the merge ticket.
+    // Empty chunk: an empty partial (no key).
     for (int h = threadIdx.x; h < H; h += blockDim.x) {
       p.part_ml[pidx * H * 2 + 2 * h] = -INFINITY;
       p.part_ml[pidx * H * 2 + 2 * h + 1] = 0.f;
@@ -118,9 +118,9 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     if (threadIdx.x == 0) {
       for (int s = 0; s < NS; ++s) {
-        mbar_init(kfull + s, 1);
+        mbar_init(kfull + s, GATHER ? 32 : 1);
         mbar_init(kempty + s, 1);
-        mbar_init(vfull + s, 1);
+        mbar_init(vfull + s, GATHER ? 32 : 1);
         mbar_init(vempty + s, 1);
       }
       for (int s = 0; s < 2; ++s) {
@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(192, 1)
       tmem_alloc(tmem_slot, L::kTmemCols);
       tmem_relinquish();
     }
-    if (warp == 0 && lane_id() == 0) {
+    if (!GATHER && warp == 0 && lane_id() == 0) {
       prefetch_tmap(&tmap_k);
       prefetch_tmap(&tmap_v);
     }
@@ -149,7 +149,46 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tmem_o = tmem_base + 2 * H;
     bool ok = true;
 
-    if (warp == 0) {
+    if (GATHER && warp == 0) {
+      // ------------------------------------------------ gather producer (32 lanes)
+      // Rows named by the index row go to the same 128-byte-swizzled layout that TMA
+      // writes (16-byte chunk c of row r at chunk c ^ (r mod 8)); absent rows are
+      // zero-filled.  Each lane copies 4 rows, waits for its copies and arrives.
+      const int lane = (int)lane_id();
+      const uint8_t* kb = static_cast<const uint8_t*>(p.kv.k);
+      const uint8_t* vb = static_cast<const uint8_t*>(p.kv.v);
+      for (int i = 0; i < n_tiles; ++i) {
+        const int s = i % NS;
+        const uint32_t ph = ((i / NS) & 1) ^ 1;
+        if (ok && !mbar_wait(kempty + s, ph)) ok = false;
+        if (ok && !mbar_wait(vempty + s, ph)) ok = false;
+        const uint32_t kdst = smem_u32(kst + s * L::kTile), vdst = smem_u32(vst + s * L::kTile);
+        for (int rr = 0; rr < kKeyTile / 32; ++rr) {
+          const int r = lane + 32 * rr, e = k0 + i * kKeyTile + r;
+          int j = -1;
+          if (e < k1) {
+            j = __ldg(idx_row + e);
+            if (j < 0 || j >= Lb) {
+              if (j != -1) set_status(p.status, HS2_ERR_INDEX_OUT_OF_RANGE);
+              j = -1;
+            }
+          }
+          const size_t off = j >= 0 ? (row_base + j) * (kHeadDim * 2) : 0;
+          const uint32_t nb = j >= 0 ? 16u : 0u;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const uint32_t at = (uint32_t)(c >> 3) * kBoxBytes + r * 128 +
+                                ((uint32_t)((c & 7) ^ (r & 7)) << 4);
+            cp_async_16(kdst + at, kb + off + c * 16, nb);
+            cp_async_16(vdst + at, vb + off + c * 16, nb);
+          }
+        }
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        mbar_arrive(kfull + s);
+        mbar_arrive(vfull + s);
+      }
+    } else if (warp == 0) {
       // ------------------------------------------------------------ TMA producer
       if (elect_one()) {
         const uint64_t pol = policy_evict_first();
@@ -224,6 +263,7 @@ __global__ void __launch_bounds__(192, 1)
       const int t = lg * 32 + (int)lane_id();  // key of the tile == TMEM lane
       const uint32_t lane_base = (uint32_t)(lg * 32) << 16;
       const float c2 = p.sm_scale * kLog2e;
+      const uint64_t keep_policy = policy_evict_last();
       float l[H];
 #pragma unroll
       for (int h = 0; h < H; ++h) l[h] = 0.f;
@@ -242,13 +282,30 @@ __global__ void __launch_bounds__(192, 1)
           uint32_t r[16];
           tmem_ld16(tmem_base + lane_base + sb * H + c, r);
           tmem_wait_ld();
+          if (!GATHER && p.sbuf) {
+            // Raw float32 logits of keys outside the window, for the selection (kept in
+            // L2 with an evict-last policy; the selection reads them right after).
+            const int jj = k0 + i * kKeyTile + t;
+            if (jj < k1 && jj <= pos - p.window && pos - p.window + 1 > p.k_sel) {
+              float* dst = p.sbuf + ((size_t)bq * p.kv.max_len + jj) * H + c;
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                st_global_v4_hint(dst + 4 * e,
+                                  make_uint4(r[4 * e], r[4 * e + 1], r[4 * e + 2], r[4 * e + 3]),
+                                  keep_policy);
+            }
+          }
 #pragma unroll
           for (int e = 0; e < 16; ++e) x[c + e] = __uint_as_float(r[e]) * c2;
         }
         tc_fence_before();
         mbar_arrive(s_free + sb);
         const int j = k0 + i * kKeyTile + t;
-        const bool valid = j < k1;
+        bool valid = j < k1;
+        if (GATHER && valid) {
+          const int pj = __ldg(idx_row + j);
+          valid = pj >= 0 && pj < Lb;
+        }
         bool over = false;
 #pragma unroll
         for (int h = 0; h < H; ++h) {
@@ -309,7 +366,7 @@ __global__ void __launch_bounds__(192, 1)
           *reinterpret_cast<uint4*>(plo + c * (kKeyTile * 16) + t * 16) =
               make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
-        if (!valid && i == n_tiles - 1) {
+        if (!GATHER && !valid && i == n_tiles - 1) {
           // Rows past the chunk end may hold anything (NaN included); 0 * NaN would
           // poison P.V, so zero this key's V row once its tile has landed.
           const int s = i % NS;
@@ -359,105 +416,44 @@ __global__ void __launch_bounds__(192, 1)
     }
   }
 
-  // Merge of the chunk partials by the last CTA of this (sequence, token).
-  if (!arrive_last(p.tickets + bq, p.splits1)) return;
-  merge_log2_partials<H>(p, bq, smem);
 }
 
-// Merge of the chunk partials (m in log2 units, l, unnormalised o) of one
-// (sequence, token): out = sum_s 2^(m_s - M) o_s / L, lse = (M + log2 L) ln 2,
-// delta_h = lse_h - min_h' lse_h'.  Run by one CTA (any thread count).
-template <int H>
-__device__ void merge_log2_partials(const FullParams& p, int bq, uint8_t* smem) {
-  const int S = p.splits1, nt = blockDim.x, tid = threadIdx.x;
-  const float* pml = p.part_ml + (size_t)bq * S * H * 2;
-  const float* po = p.part_o + (size_t)bq * S * H * kHeadDim;
-  double* lse_d = reinterpret_cast<double*>(smem);          // [H + 1]
-  float* Mf = reinterpret_cast<float*>(lse_d + H + 1);       // [H]
-  float* invL = Mf + H;                                      // [H]
-  float* w = invL + H;                                       // [32][H]
-  for (int h = tid; h < H; h += nt) {
-    float M = -INFINITY;
-    for (int sp = 0; sp < S; ++sp) M = fmaxf(M, __ldcg(pml + ((size_t)sp * H + h) * 2));
-    double Ls = 0.0;
-    if (M != -INFINITY)
-      for (int sp = 0; sp < S; ++sp) {
-        const float m = __ldcg(pml + ((size_t)sp * H + h) * 2);
-        const float l = __ldcg(pml + ((size_t)sp * H + h) * 2 + 1);
-        if (l > 0.f) Ls += (double)l * exp2((double)m - (double)M);
-      }
-    Mf[h] = M;
-    invL[h] = Ls > 0.0 ? (float)(1.0 / Ls) : 0.f;
-    lse_d[h] = Ls > 0.0 ? ((double)M + log2(Ls)) * 0.69314718055994530942 : -INFINITY;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    double mn = INFINITY;
-    for (int h = 0; h < H; ++h) mn = fmin(mn, lse_d[h]);
-    lse_d[H] = mn;
-  }
-  __syncthreads();
-  for (int h = tid; h < H; h += nt) {
-    const double l = lse_d[h], dl = l - lse_d[H];
-    p.lse64[(size_t)bq * H + h] = l;
-    p.delta64[(size_t)bq * H + h] = dl;
-    p.delta32[(size_t)bq * H + h] = (float)dl;
-    if (p.lse_out) p.lse_out[(size_t)bq * H + h] = (float)l;
-  }
-  float* out = p.out + (size_t)bq * H * kHeadDim;
-  for (int e0 = 0; e0 < H * kHeadDim; e0 += nt) {
-    const int e = e0 + tid;
-    float acc = 0.f;
-    for (int sb = 0; sb < S; sb += 32) {
-      __syncthreads();
-      for (int x = tid; x < 32 * H; x += nt) {
-        const int sp = sb + x / H, h = x % H;
-        float wt = 0.f;
-        if (sp < S && Mf[h] != -INFINITY) {
-          const float m = __ldcg(pml + ((size_t)sp * H + h) * 2);
-          const float l = __ldcg(pml + ((size_t)sp * H + h) * 2 + 1);
-          if (l > 0.f) wt = exp2f(m - Mf[h]) * invL[h];
-        }
-        w[x] = wt;
-      }
-      __syncthreads();
-      if (e < H * kHeadDim) {
-        const int h = e / kHeadDim;
-        const int ns = min(32, S - sb);
-        for (int t = 0; t < ns; ++t) {
-          const float wt = w[t * H + h];
-          if (wt != 0.f) acc = fmaf(wt, __ldcg(po + ((size_t)(sb + t) * H) * kHeadDim + e), acc);
-        }
-      }
-    }
-    if (e < H * kHeadDim) out[e] = acc;
-  }
-}
-
-template <int H>
+template <int H, bool GATHER>
 static cudaError_t launch_full_tc_t(const FullParams& p, const CUtensorMap& tk,
                                     const CUtensorMap& tv, int bq, cudaStream_t st) {
   using L = FullSmem<H>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(full_attn_tc_kernel<H>,
+    cudaError_t e = cudaFuncSetAttribute(full_attn_tc_kernel<H, GATHER>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  full_attn_tc_kernel<H><<<dim3(p.splits1, bq), 192, L::kBytes, st>>>(tk, tv, p);
+  full_attn_tc_kernel<H, GATHER><<<dim3(p.splits1, bq), 192, L::kBytes, st>>>(tk, tv, p);
   return cudaGetLastError();
+}
+
+template <bool GATHER>
+static cudaError_t launch_full_tc_h(const FullParams& p, const CUtensorMap& tk,
+                                    const CUtensorMap& tv, int bq, cudaStream_t st) {
+  switch (p.h) {
+    case 16: return launch_full_tc_t<16, GATHER>(p, tk, tv, bq, st);
+    case 32: return launch_full_tc_t<32, GATHER>(p, tk, tv, bq, st);
+    case 48: return launch_full_tc_t<48, GATHER>(p, tk, tv, bq, st);
+    case 64: return launch_full_tc_t<64, GATHER>(p, tk, tv, bq, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_full_attn_tc(const FullParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                                 int bq, cudaStream_t st) {
-  switch (p.h) {
-    case 16: return launch_full_tc_t<16>(p, tk, tv, bq, st);
-    case 32: return launch_full_tc_t<32>(p, tk, tv, bq, st);
-    case 48: return launch_full_tc_t<48>(p, tk, tv, bq, st);
-    case 64: return launch_full_tc_t<64>(p, tk, tv, bq, st);
-    default: return cudaErrorInvalidValue;
-  }
+  return launch_full_tc_h<false>(p, tk, tv, bq, st);
+}
+
+cudaError_t launch_sparse_attn_tc(const FullParams& p, int bq, cudaStream_t st) {
+  CUtensorMap unused;
+  memset(&unused, 0, sizeof(unused));
+  return launch_full_tc_h<true>(p, unused, unused, bq, st);
 }
 
 }  // namespace hs2

@@ -40,7 +40,7 @@ static int chunk_for(int max_len, int splits) {
 
 int plan_splits4(int idx_width) { return (idx_width + kChunk4 - 1) / kChunk4; }
 
-bool make_layout(int batch, int n_q, int h, int max_len, int window, int k_sel,
+bool make_layout(int batch, int n_q, int h, int max_len, int window, int k_sel, int dtype,
                  WsLayout* L) {
   WsLayout w;
   w.bq = batch * n_q;
@@ -59,8 +59,6 @@ bool make_layout(int batch, int n_q, int h, int max_len, int window, int k_sel,
   };
   // Regions that depend only on (bq, h): status and the sparse-layer state.
   w.status = take(sizeof(uint32_t));
-  w.tickets1 = take(bq * sizeof(uint32_t));
-  w.tickets4 = take(bq * sizeof(uint32_t));
   w.part4_o = take(bq * w.splits4 * hh * kHeadDim * sizeof(float));
   w.part4_ml = take(bq * w.splits4 * hh * 2 * sizeof(float));
   // Regions of the full layer and the selection.
@@ -72,9 +70,9 @@ bool make_layout(int batch, int n_q, int h, int max_len, int window, int k_sel,
   w.part1_o = take(bq * w.splits1 * hh * kHeadDim * sizeof(float));
   w.part1_ml = take(bq * w.splits1 * hh * 2 * sizeof(float));
   w.lse64 = take(bq * hh * sizeof(double));
-  w.delta64 = take(bq * hh * sizeof(double));
-  w.delta32 = take(bq * hh * sizeof(float));
   w.tbuf = take(bq * ml * sizeof(float));
+  w.use_sbuf = sbuf_eligible(n_q, h, dtype);
+  w.sbuf = take(w.use_sbuf ? bq * ml * hh * sizeof(float) : 0);
   w.direct = take(bq * (size_t)k_sel * sizeof(int32_t));
   w.cand_t = take(bq * ml * sizeof(float));
   w.cand_j = take(bq * ml * sizeof(int32_t));
@@ -139,7 +137,7 @@ static hs2_status prepare(const void* q, int n_q, int h, const hs2_kv* kv, int w
   if (st != HS2_OK) return st;
   if (!q || !ws) return HS2_ERR_INVALID_ARGUMENT;
   if (!aligned16(q) || !aligned16(ws)) return HS2_ERR_INVALID_ARGUMENT;
-  make_layout(kv->batch, n_q, h, kv->max_len, window, k_sel, &P->w);
+  make_layout(kv->batch, n_q, h, kv->max_len, window, k_sel, kv->dtype, &P->w);
   if (ws_bytes < P->w.total) return HS2_ERR_WORKSPACE_TOO_SMALL;
   return HS2_OK;
 }
@@ -159,13 +157,8 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
   p.chunk1 = chunk_for(kv->max_len, w.splits1);
   p.part_o = ws_ptr<float>(ws, w.part1_o);
   p.part_ml = ws_ptr<float>(ws, w.part1_ml);
-  p.tickets = ws_ptr<uint32_t>(ws, w.tickets1);
-  p.out = out;
-  p.lse_out = lse;
-  p.lse64 = ws_ptr<double>(ws, w.lse64);
-  p.delta64 = ws_ptr<double>(ws, w.delta64);
-  p.delta32 = ws_ptr<float>(ws, w.delta32);
   p.status = ws_ptr<uint32_t>(ws, w.status);
+  bool log2_partials = false;
   cudaError_t e;
   if (kv->dtype == HS2_KV_BF16 && h <= 64) {
     // Tensor-core flash-decode: about one CTA per SM, chunks of whole 128-key tiles.
@@ -184,11 +177,23 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
     chunk = (chunk + 127) / 128 * 128;
     p.splits1 = (kv->max_len + chunk - 1) / chunk;
     p.chunk1 = chunk;
+    p.sbuf = w.use_sbuf ? ws_ptr<float>(ws, w.sbuf) : nullptr;
     e = launch_full_attn_tc(p, tk, tv, bq, s);
+    log2_partials = true;
   } else {
     e = launch_full_attn(p, kv->batch, s);
   }
-  return e == cudaSuccess ? HS2_OK : cuda_fail(e, "full-attention launch");
+  if (e != cudaSuccess) return cuda_fail(e, "full-attention launch");
+  MergeParams m;
+  m.part_o = p.part_o;
+  m.part_ml = p.part_ml;
+  m.splits = p.splits1;
+  m.h = h;
+  m.out = out;
+  m.lse_out = lse;
+  m.lse64 = ws_ptr<double>(ws, w.lse64);
+  e = launch_merge(m, kv->batch * n_q, log2_partials, s);
+  return e == cudaSuccess ? HS2_OK : cuda_fail(e, "full-attention merge launch");
 }
 
 static hs2_status run_select(const void* q, int n_q, int h, const hs2_kv* kv, int window,
@@ -209,8 +214,8 @@ static hs2_status run_select(const void* q, int n_q, int h, const hs2_kv* kv, in
   p.chunk2 = chunk_for(kv->max_len, w.splits1);
   p.chunk3 = kChunk3;
   p.splits3 = (kv->max_len + kChunk3 - 1) / kChunk3;
-  p.delta64 = ws_ptr<double>(ws, w.delta64);
-  p.delta32 = ws_ptr<float>(ws, w.delta32);
+  p.lse64 = ws_ptr<double>(ws, w.lse64);
+  p.sbuf = w.use_sbuf ? ws_ptr<float>(ws, w.sbuf) : nullptr;
   p.tbuf = ws_ptr<float>(ws, w.tbuf);
   p.hist = ws_ptr<uint32_t>(ws, w.hist);
   p.counters = ws_ptr<uint32_t>(ws, w.counters);
@@ -223,7 +228,11 @@ static hs2_status run_select(const void* q, int n_q, int h, const hs2_kv* kv, in
   p.idx = idx;
   p.status = ws_ptr<uint32_t>(ws, w.status);
   const int bq = kv->batch * n_q;
-  if (kv->dtype == HS2_KV_BF16) {
+  if (w.use_sbuf) {
+    e = launch_importance_sbuf(p, bq, s);
+    if (e != cudaSuccess) return cuda_fail(e, "importance launch");
+    e = launch_select_rest(p, kv->batch, s);
+  } else if (kv->dtype == HS2_KV_BF16) {
     // Tensor-core importance pass: one CTA per SM per key chunk (128-key multiples).
     CUtensorMap tk;
     if (!make_tmap_2d(&tk, kv->k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kHeadDim,
@@ -256,7 +265,7 @@ size_t hs2_workspace_bytes(int batch, int n_q, int h_q, int max_len, int window,
   if (dtype != HS2_KV_BF16 && dtype != HS2_KV_FP8_E4M3) return 0;
   if (check_shape(batch, n_q, h_q, max_len, window, k_sel) != HS2_OK) return 0;
   WsLayout w;
-  make_layout(batch, n_q, h_q, max_len, window, k_sel, &w);
+  make_layout(batch, n_q, h_q, max_len, window, k_sel, dtype, &w);
   return w.total;
 }
 
@@ -309,8 +318,38 @@ hs2_status hs2_sparse_attn(const void* q_layer, int n_q, int h_q, const hs2_kv* 
   if (!aligned16(q_layer) || !aligned16(out) || !aligned16(workspace))
     return HS2_ERR_INVALID_ARGUMENT;
   WsLayout w;
-  make_layout(kv->batch, n_q, h_q, kv->max_len, 1, 1, &w);
+  make_layout(kv->batch, n_q, h_q, kv->max_len, 1, 1, kv->dtype, &w);
   if (ws_bytes < sparse_prefix_bytes(w)) return HS2_ERR_WORKSPACE_TOO_SMALL;
+  if (kv->dtype == HS2_KV_BF16 && h_q <= 64) {
+    // Tensor-core gather attention: 128 index entries per CTA, log2-domain partials.
+    FullParams f;
+    f.q = static_cast<const uint16_t*>(q_layer);
+    f.kv = view_of(kv);
+    f.n_q = n_q;
+    f.h = h_q;
+    f.window = 0;
+    f.k_sel = 0;
+    f.sm_scale = sm_scale;
+    f.chunk1 = 128;
+    f.splits1 = (idx_width + 127) / 128;
+    f.part_o = ws_ptr<float>(workspace, w.part4_o);
+    f.part_ml = ws_ptr<float>(workspace, w.part4_ml);
+    f.status = ws_ptr<uint32_t>(workspace, w.status);
+    f.idx = idx;
+    f.idx_width = idx_width;
+    cudaError_t e = launch_sparse_attn_tc(f, kv->batch * n_q, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "sparse-attention launch");
+    MergeParams m;
+    m.part_o = f.part_o;
+    m.part_ml = f.part_ml;
+    m.splits = f.splits1;
+    m.h = h_q;
+    m.out = out;
+    m.lse_out = nullptr;
+    m.lse64 = nullptr;
+    e = launch_merge(m, kv->batch * n_q, true, (cudaStream_t)stream);
+    return e == cudaSuccess ? HS2_OK : cuda_fail(e, "sparse-attention merge launch");
+  }
   SparseParams p;
   p.q = static_cast<const uint16_t*>(q_layer);
   p.kv = view_of(kv);
@@ -323,11 +362,19 @@ hs2_status hs2_sparse_attn(const void* q_layer, int n_q, int h_q, const hs2_kv* 
   p.chunk4 = kChunk4;
   p.part_o = ws_ptr<float>(workspace, w.part4_o);
   p.part_ml = ws_ptr<float>(workspace, w.part4_ml);
-  p.tickets = ws_ptr<uint32_t>(workspace, w.tickets4);
-  p.out = out;
   p.status = ws_ptr<uint32_t>(workspace, w.status);
   cudaError_t e = launch_sparse_attn(p, kv->batch, (cudaStream_t)stream);
-  return e == cudaSuccess ? HS2_OK : cuda_fail(e, "sparse-attention launch");
+  if (e != cudaSuccess) return cuda_fail(e, "sparse-attention launch");
+  MergeParams m;
+  m.part_o = p.part_o;
+  m.part_ml = p.part_ml;
+  m.splits = p.splits4;
+  m.h = h_q;
+  m.out = out;
+  m.lse_out = nullptr;
+  m.lse64 = nullptr;
+  e = launch_merge(m, kv->batch * n_q, false, (cudaStream_t)stream);
+  return e == cudaSuccess ? HS2_OK : cuda_fail(e, "sparse-attention merge launch");
 }
 
 hs2_status hs2_check_device_status(void* workspace, hs2_stream_t stream) {

@@ -32,15 +32,13 @@ struct WsLayout {
   size_t hist = 0;        // u32 [bq][kHistBins]
   size_t counters = 0;    // u32 [bq][8]: 0 direct, 1 cand, 2 band
   size_t clear_end = 0;
-  size_t tickets1 = 0;    // u32 [bq], self-resetting
-  size_t tickets4 = 0;    // u32 [bq], self-resetting
   size_t selmeta = 0;     // u32 [bq][4]: bin, eps bits, k_eff, n_c
   size_t part1_o = 0;     // f32 [bq][splits1][h][128]
   size_t part1_ml = 0;    // f32 [bq][splits1][h][2]
   size_t lse64 = 0;       // f64 [bq][h]
-  size_t delta64 = 0;     // f64 [bq][h]
-  size_t delta32 = 0;     // f32 [bq][h]
   size_t tbuf = 0;        // f32 [bq][max_len]  selection keys t_j
+  size_t sbuf = 0;        // f32 [bq][max_len][h] raw logits (0 bytes when not used)
+  bool use_sbuf = false;
   size_t direct = 0;      // i32 [bq][k_sel]
   size_t cand_t = 0;      // f32 [bq][max_len]
   size_t cand_j = 0;      // i32 [bq][max_len]
@@ -54,7 +52,7 @@ struct WsLayout {
 int plan_splits1(int bq, int max_len, int num_sms);
 int device_sm_count();
 int plan_splits4(int idx_width);
-bool make_layout(int batch, int n_q, int h, int max_len, int window, int k_sel,
+bool make_layout(int batch, int n_q, int h, int max_len, int window, int k_sel, int dtype,
                  WsLayout* L);
 
 template <typename T>
@@ -81,15 +79,22 @@ struct FullParams {
   int n_q, h, window, k_sel;
   float sm_scale;
   int splits1, chunk1;
-  float* part_o;
-  float* part_ml;
-  uint32_t* tickets;
+  float* part_o;   // [bq][splits1][h][128] unnormalised
+  float* part_ml;  // [bq][splits1][h][2]: reference m, sum l
+  uint32_t* status;
+  const int32_t* idx = nullptr;  // gather mode (a sparse layer): [bq][idx_width] positions
+  int idx_width = 0;
+  float* sbuf = nullptr;          // if set: raw float32 logits of the keys outside the window
+};
+
+// Split merge (full layer: log2-domain partials; sparse layers: natural-log ones).
+struct MergeParams {
+  const float* part_o;
+  const float* part_ml;
+  int splits, h;
   float* out;
   float* lse_out;  // may be null
-  double* lse64;
-  double* delta64;
-  float* delta32;
-  uint32_t* status;
+  double* lse64;   // may be null
 };
 
 struct SelectParams {
@@ -99,8 +104,8 @@ struct SelectParams {
   float sm_scale;
   int splits2, chunk2;   // importance pass
   int splits3, chunk3;   // compaction pass
-  const double* delta64;
-  const float* delta32;
+  const double* lse64;  // per-head lse of the full layer, [bq][h]
+  const float* sbuf;     // raw float32 logits written by the full layer, or null
   float* tbuf;
   uint32_t* hist;
   uint32_t* counters;
@@ -123,8 +128,6 @@ struct SparseParams {
   int splits4, chunk4;
   float* part_o;
   float* part_ml;
-  uint32_t* tickets;
-  float* out;
   uint32_t* status;
 };
 
@@ -133,7 +136,15 @@ cudaError_t launch_full_attn(const FullParams& p, int batch, cudaStream_t s);
 cudaError_t launch_select(const SelectParams& p, int batch, cudaStream_t s);
 // The selection after the importance pass (compaction + finish).
 cudaError_t launch_select_rest(const SelectParams& p, int batch, cudaStream_t s);
+// Importance from the full layer's stored float32 logits.
+cudaError_t launch_importance_sbuf(const SelectParams& p, int bq, cudaStream_t s);
+// The stored-logit path applies to single-token decode with 16 heads on a bf16 cache:
+// 64 bytes of logits per key instead of re-reading its 256-byte K row.
+inline bool sbuf_eligible(int n_q, int h, int dtype) {
+  return n_q == 1 && h == 16 && dtype == HS2_KV_BF16;
+}
 cudaError_t launch_sparse_attn(const SparseParams& p, int batch, cudaStream_t s);
+cudaError_t launch_merge(const MergeParams& p, int bq, bool log2_domain, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // Device helpers.

@@ -17,6 +17,7 @@
 #include "hs2_internal.cuh"
 #include "sm100.cuh"
 #include "tc_common.cuh"
+#include "tile_simt.cuh"
 
 namespace hs2 {
 
@@ -89,7 +90,7 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0 && lane_id() == 0) prefetch_tmap(&tmap_k);
   store_q_kmajor<H>(qs, p.q + (size_t)bq * H * kHeadDim, threadIdx.x, blockDim.x);
   for (int e = threadIdx.x; e < kHistBins; e += blockDim.x) hist_s[e] = 0u;
-  for (int e = threadIdx.x; e < H; e += blockDim.x) delta_s[e] = p.delta32[(size_t)bq * H + e];
+  load_delta(p.lse64 + (size_t)bq * H, H, delta_s, nullptr);
   fence_proxy_async_smem();  // Q written by threads, read by the tensor cores
   tc_fence_before();
   __syncthreads();

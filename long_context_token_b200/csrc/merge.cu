@@ -1,0 +1,115 @@
+// Merge of split partials (m, l, unnormalised o) into the normalised output and the
+// per-head log-sum-exp, for the full layer and the sparse layers.
+//
+//   out_h = sum_s w_sh o_sh,  w_sh = e^(m_sh - M_h) / L_h,  L_h = sum_s l_sh e^(m_sh - M_h),
+//   lse_h = M_h + ln L_h
+// (base 2 instead of e when the partials were produced in the log2 domain).
+//
+// Grid (bq, h): one CTA per (sequence/token, head), 128 x G threads.  Warp 0 reduces
+// M and L over the splits (float64 sum) and stages the weights in shared memory;
+// thread (g, d) then sums dimension d over the splits s = g, g + G, ... with eight
+// independent loads in flight, and the G partial sums are added in shared memory.
+#include "hs2_internal.cuh"
+
+namespace hs2 {
+
+constexpr int kMergeMaxGroups = 8;
+
+template <bool LOG2>
+__global__ void __launch_bounds__(kHeadDim * kMergeMaxGroups) merge_splits_kernel(MergeParams p) {
+  extern __shared__ float w[];  // [splits] weights, then [G][128] partial sums
+  const int bq = blockIdx.x, h = blockIdx.y;
+  const int H = p.h, S = p.splits;
+  const int G = blockDim.x / kHeadDim;
+  float* acc_s = w + ((S + 3) & ~3);
+  __shared__ float Mh, invL;
+  const float* pml = p.part_ml + (size_t)bq * S * H * 2;
+  const float* po = p.part_o + (size_t)bq * S * H * kHeadDim;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    float M = -INFINITY;
+    for (int s = lane; s < S; s += 32) M = fmaxf(M, __ldcg(pml + ((size_t)s * H + h) * 2));
+    M = warp_max(M);
+    double Ls = 0.0;
+    if (M != -INFINITY) {
+      for (int s = lane; s < S; s += 32) {
+        const float m = __ldcg(pml + ((size_t)s * H + h) * 2);
+        const float l = __ldcg(pml + ((size_t)s * H + h) * 2 + 1);
+        if (l > 0.f) Ls += (double)l * (LOG2 ? exp2((double)m - M) : exp((double)m - M));
+      }
+    }
+    Ls = warp_sum_d(Ls);
+    const float il = Ls > 0.0 ? (float)(1.0 / Ls) : 0.f;
+    for (int s = lane; s < S; s += 32) {
+      float wt = 0.f;
+      if (M != -INFINITY) {
+        const float m = __ldcg(pml + ((size_t)s * H + h) * 2);
+        const float l = __ldcg(pml + ((size_t)s * H + h) * 2 + 1);
+        if (l > 0.f) wt = (LOG2 ? exp2f(m - M) : expf(m - M)) * il;
+      }
+      w[s] = wt;
+    }
+    if (lane == 0) {
+      Mh = M;
+      invL = il;
+      double lse = -INFINITY;
+      if (Ls > 0.0) lse = LOG2 ? ((double)M + log2(Ls)) * 0.69314718055994530942 : M + log(Ls);
+      if (p.lse64) p.lse64[(size_t)bq * H + h] = lse;
+      if (p.lse_out) p.lse_out[(size_t)bq * H + h] = (float)lse;
+    }
+  }
+  __syncthreads();
+  const int d = threadIdx.x % kHeadDim, g = threadIdx.x / kHeadDim;
+  const float* src = po + (size_t)h * kHeadDim + d;
+  const size_t stride = (size_t)H * kHeadDim;
+  float acc = 0.f;
+  int s = g;
+  for (; s + 7 * G < S; s += 8 * G) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (size_t)(s + u * G) * stride);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float wt = w[s + u * G];
+      if (wt != 0.f) acc = fmaf(wt, v[u], acc);
+    }
+  }
+  for (; s < S; s += G) {
+    const float wt = w[s];
+    if (wt != 0.f) acc = fmaf(wt, __ldcg(src + (size_t)s * stride), acc);
+  }
+  acc_s[g * kHeadDim + d] = acc;
+  __syncthreads();
+  if (g == 0) {
+    float t = 0.f;
+    for (int k = 0; k < G; ++k) t += acc_s[k * kHeadDim + d];
+    p.out[((size_t)bq * H + h) * kHeadDim + d] = t;
+  }
+}
+
+cudaError_t launch_merge(const MergeParams& p, int bq, bool log2_domain, cudaStream_t st) {
+  int G = (p.splits + 15) / 16;
+  if (G > kMergeMaxGroups) G = kMergeMaxGroups;
+  if (G < 1) G = 1;
+  const size_t smem = (((size_t)p.splits + 3) / 4 * 4 + (size_t)G * kHeadDim) * sizeof(float);
+  if (smem > 200 * 1024) return cudaErrorInvalidValue;
+  static size_t attr_set[2] = {0, 0};
+  const int which = log2_domain ? 1 : 0;
+  if (smem > 48 * 1024 && smem > attr_set[which]) {
+    cudaError_t e = log2_domain
+        ? cudaFuncSetAttribute(merge_splits_kernel<true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+        : cudaFuncSetAttribute(merge_splits_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set[which] = smem;
+  }
+  dim3 grid(bq, p.h);
+  if (log2_domain)
+    merge_splits_kernel<true><<<grid, kHeadDim * G, smem, st>>>(p);
+  else
+    merge_splits_kernel<false><<<grid, kHeadDim * G, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace hs2

@@ -17,11 +17,18 @@
 //      tau among the candidates; keys with |t - tau| <= eps are re-scored in float64
 //      from the stored inputs and ranked by (t desc, position asc); the result is
 //      merged with the window, sorted ascending and padded with -1.
-// The float32 pass is exact whenever its logits lie within eps/2 of the true ones,
-// eps = 1e-3 * max(1, |bin edges|).
+// The float32 pass is exact whenever its keys lie within eps/2 of the true ones,
+// eps = 1e-3 * max(1, |bin edges| + max_h delta_h).
 #include "tile_simt.cuh"
+#include "sm100.cuh"
 
 namespace hs2 {
+
+__device__ __forceinline__ uint64_t sm100_evict_first_policy() { return sm100::policy_evict_first(); }
+__device__ __forceinline__ uint4 sm100_ld_v4_hint(const void* p, uint64_t pol) {
+  return sm100::ld_global_v4_hint(p, pol);
+}
+
 
 constexpr float kEpsRel = 1e-3f;
 
@@ -45,7 +52,7 @@ __global__ void __launch_bounds__(kThreads) importance_simt_kernel(SelectParams 
   if (k0 >= k1) return;
 
   for (int e = threadIdx.x; e < kHistBins; e += kThreads) hist_s[e] = 0u;
-  for (int hd = threadIdx.x; hd < H; hd += kThreads) delta_s[hd] = p.delta32[(size_t)bq * H + hd];
+  load_delta(p.lse64 + (size_t)bq * H, H, delta_s, nullptr);
   load_q_scaled<H>(s.qs, p.q + (size_t)bq * H * kHeadDim, p.sm_scale);
   const size_t row_base = (size_t)b * p.kv.max_len;
   float* trow = p.tbuf + (size_t)bq * p.kv.max_len;
@@ -74,6 +81,58 @@ __global__ void __launch_bounds__(kThreads) importance_simt_kernel(SelectParams 
     if (hist_s[e]) atomicAdd(gh + e, hist_s[e]);
 }
 
+// 1'. importance from the full layer's stored float32 logits (single-token decode,
+//     16 heads): the same t_j and histogram without reading K again.
+constexpr int kSbufChunk = 4096;
+
+template <int H>
+__global__ void __launch_bounds__(kThreads) importance_sbuf_kernel(SelectParams p) {
+  __shared__ uint32_t hist_s[kHistBins];
+  __shared__ float delta_s[kMaxHeads];
+  const int split = blockIdx.x, bq = blockIdx.y;
+  const int b = bq / p.n_q, i = bq % p.n_q;
+  const int L = seq_len(p.kv, b, p.n_q, p.status, false);
+  const int pos = L - p.n_q + i;
+  const int n_c = pos - p.window + 1;
+  if (n_c <= p.k_sel) return;
+  const int k0 = split * kSbufChunk;
+  const int k1 = min(k0 + kSbufChunk, n_c);
+  if (k0 >= k1) return;
+  for (int e = threadIdx.x; e < kHistBins; e += kThreads) hist_s[e] = 0u;
+  load_delta(p.lse64 + (size_t)bq * H, H, delta_s, nullptr);
+  const uint64_t pol = sm100_evict_first_policy();
+  const float* src = p.sbuf + (size_t)bq * p.kv.max_len * H;
+  float* trow = p.tbuf + (size_t)bq * p.kv.max_len;
+  const float sc = p.sm_scale;
+#pragma unroll 4
+  for (int j = k0 + threadIdx.x; j < k1; j += kThreads) {
+    float t = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < H; c += 4) {
+      const uint4 v = sm100_ld_v4_hint(src + (size_t)j * H + c, pol);
+      t = fmaxf(t, __uint_as_float(v.x) * sc - delta_s[c]);
+      t = fmaxf(t, __uint_as_float(v.y) * sc - delta_s[c + 1]);
+      t = fmaxf(t, __uint_as_float(v.z) * sc - delta_s[c + 2]);
+      t = fmaxf(t, __uint_as_float(v.w) * sc - delta_s[c + 3]);
+    }
+    trow[j] = t;
+    atomicAdd(&hist_s[ordered_key(t) >> kHistShift], 1u);
+  }
+  __syncthreads();
+  uint32_t* gh = p.hist + (size_t)bq * kHistBins;
+  for (int e = threadIdx.x; e < kHistBins; e += kThreads)
+    if (hist_s[e]) atomicAdd(gh + e, hist_s[e]);
+}
+
+cudaError_t launch_importance_sbuf(const SelectParams& p, int bq, cudaStream_t st) {
+  const dim3 grid((p.kv.max_len + kSbufChunk - 1) / kSbufChunk, bq);
+  switch (p.h) {
+    case 16: importance_sbuf_kernel<16><<<grid, kThreads, 0, st>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 // ----------------------------------------------------------------------------
 // 2. compaction
 // ----------------------------------------------------------------------------
@@ -82,36 +141,55 @@ struct BoundaryBin {
   float lo, hi, eps;
 };
 
-// Every CTA of a bq finds the same boundary bin from the global histogram.
-__device__ BoundaryBin find_boundary_bin(const uint32_t* gh, int k_eff) {
-  __shared__ uint32_t part[kThreads];
-  __shared__ uint32_t above[kThreads];
+// Every CTA of a bq finds the same boundary bin from the global histogram: thread t
+// sums 16 bins, warp 0 turns the 256 sums into counts "above" (a prefix sum from the
+// top bin down), and the thread whose range holds the k-th largest scans its bins.
+__device__ BoundaryBin find_boundary_bin(const uint32_t* gh, int k_eff, float delta_max) {
+  __shared__ uint32_t part[kThreads];  // indexed from the top: part[255 - t]
   __shared__ uint32_t bin_s;
   constexpr int per = kHistBins / kThreads;  // 16 bins per thread
   if (threadIdx.x == 0) bin_s = 0u;
-  uint32_t loc = 0;
-  for (int e = 0; e < per; ++e) loc += __ldcg(gh + threadIdx.x * per + e);
-  part[threadIdx.x] = loc;
+  uint32_t c[per], loc = 0;
+#pragma unroll
+  for (int e = 0; e < per; ++e) {
+    c[e] = __ldcg(gh + threadIdx.x * per + e);
+    loc += c[e];
+  }
+  part[kThreads - 1 - threadIdx.x] = loc;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    uint32_t cum = 0;
-    for (int t = kThreads - 1; t >= 0; --t) {
-      above[t] = cum;
-      cum += part[t];
+  if (threadIdx.x < 32) {
+    // lane l owns part[8l .. 8l+7]; exclusive prefix from the top
+    uint32_t v[8], sum = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      v[u] = part[8 * threadIdx.x + u];
+      sum += v[u];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+      if ((int)threadIdx.x >= o) incl += x;
+    }
+    uint32_t run = incl - sum;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t here = v[u];
+      part[8 * threadIdx.x + u] = run;  // count strictly above this thread's range
+      run += here;
     }
   }
   __syncthreads();
-  const uint32_t a = above[threadIdx.x];
+  const uint32_t a = part[kThreads - 1 - threadIdx.x];
   if (a < (uint32_t)k_eff && (uint32_t)k_eff <= a + loc) {
     uint32_t cum = a;
+#pragma unroll
     for (int e = per - 1; e >= 0; --e) {
-      const uint32_t bin = threadIdx.x * per + e;
-      const uint32_t c = __ldcg(gh + bin);
-      if (cum + c >= (uint32_t)k_eff) {
-        bin_s = bin;
+      if (cum + c[e] >= (uint32_t)k_eff) {
+        bin_s = threadIdx.x * per + e;
         break;
       }
-      cum += c;
+      cum += c[e];
     }
   }
   __syncthreads();
@@ -119,7 +197,10 @@ __device__ BoundaryBin find_boundary_bin(const uint32_t* gh, int k_eff) {
   r.bin = bin_s;
   r.lo = key_to_float(r.bin << kHistShift);
   r.hi = key_to_float((r.bin << kHistShift) | ((1u << kHistShift) - 1u));
-  r.eps = kEpsRel * fmaxf(1.f, fmaxf(fabsf(r.lo), fabsf(r.hi)));
+  // Margin around the boundary bin: the float32 logits (tensor-core accumulation) and
+  // the float32 shift are far inside 1e-3 of |t| + max delta for any sane input.
+  const float edge = fmaxf(fabsf(r.lo), fabsf(r.hi));
+  r.eps = kEpsRel * fmaxf(1.f, edge + delta_max);
   return r;
 }
 
@@ -143,7 +224,18 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(SelectParams p
   const int n_c = pos - p.window + 1;
   if (n_c <= p.k_sel) return;
   const int k_eff = p.k_sel;
-  const BoundaryBin bb = find_boundary_bin(p.hist + (size_t)bq * kHistBins, k_eff);
+  __shared__ float dmax_s;
+  if (threadIdx.x == 0) {
+    double lo = INFINITY, hi = -INFINITY;
+    for (int h = 0; h < p.h; ++h) {
+      const double l = p.lse64[(size_t)bq * p.h + h];
+      lo = fmin(lo, l);
+      hi = fmax(hi, l);
+    }
+    dmax_s = (float)(hi - lo);
+  }
+  __syncthreads();
+  const BoundaryBin bb = find_boundary_bin(p.hist + (size_t)bq * kHistBins, k_eff, dmax_s);
   if (split == 0 && threadIdx.x == 0) {
     uint32_t* meta = p.selmeta + (size_t)bq * 4;
     meta[0] = bb.bin;
@@ -159,18 +251,38 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(SelectParams p
   int32_t* direct = p.direct + (size_t)bq * p.k_sel;
   float* ct = p.cand_t + (size_t)bq * p.kv.max_len;
   int32_t* cj = p.cand_j + (size_t)bq * p.kv.max_len;
-  // Uniform trip count per warp so that every lane takes part in the ballots.
-  for (int j0 = k0; j0 < k1; j0 += kThreads) {
-    const int j = j0 + threadIdx.x;
-    const float t = j < k1 ? __ldcg(trow + j) : -INFINITY;
-    const bool is_direct = j < k1 && t > hi_e;
-    const bool is_cand = j < k1 && !is_direct && t >= lo_e;
-    const int sd = warp_append(is_direct, cnt + 0);
-    if (sd >= 0 && sd < p.k_sel) direct[sd] = j;
-    const int sc = warp_append(is_cand, cnt + 1);
-    if (sc >= 0 && sc < p.kv.max_len) {
-      ct[sc] = t;
-      cj[sc] = j;
+  // Each thread takes 16 consecutive keys per round, loaded up front (four 16-byte
+  // loads in flight); the trip count is uniform so every lane joins the ballots.
+  constexpr int kPer = 16;
+  for (int base = k0; base < k1; base += kThreads * kPer) {
+    const int j0 = base + threadIdx.x * kPer;
+    float t[kPer];
+    if (j0 + kPer <= k1 && ((j0 & 3) == 0)) {
+#pragma unroll
+      for (int u = 0; u < kPer / 4; ++u) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(trow + j0) + u);
+        t[4 * u] = v.x;
+        t[4 * u + 1] = v.y;
+        t[4 * u + 2] = v.z;
+        t[4 * u + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) t[u] = j0 + u < k1 ? __ldcg(trow + j0 + u) : -INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int j = j0 + u;
+      const bool in = j < k1;
+      const bool is_direct = in && t[u] > hi_e;
+      const bool is_cand = in && !is_direct && t[u] >= lo_e;
+      const int sd = warp_append(is_direct, cnt + 0);
+      if (sd >= 0 && sd < p.k_sel) direct[sd] = j;
+      const int sc = warp_append(is_cand, cnt + 1);
+      if (sc >= 0 && sc < p.kv.max_len) {
+        ct[sc] = t[u];
+        cj[sc] = j;
+      }
     }
   }
 }
@@ -179,18 +291,30 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(SelectParams p
 // 3. finish: exact select + float64 refinement + window merge + sort
 // ----------------------------------------------------------------------------
 constexpr int kFinThreads = 1024;
+constexpr int kSmallBand = 1024;  // bands up to this size are ranked pairwise
+constexpr int kBuckets = 1024;    // counting-sort buckets of the final index set
+constexpr int kQLd = kHeadDim + 8;  // padded q row (bf16) in shared memory
+static_assert(kSmallBand * (sizeof(double) + sizeof(int)) <= kMaxIdxWidth * sizeof(int),
+              "band pairs must fit the scratch area");
 
 // Radix select over the elements e in [0, n) with pred(e): the r-th largest
 // (1-based) of key(e), a KeyT of KBITS bits, 8 bits per pass.  Returns the key;
-// *n_gt receives how many selected elements are strictly greater.
+// *n_gt receives how many selected elements are strictly greater.  Each pass builds a
+// 256-bin shared histogram of the current digit, then warp 0 finds the digit holding
+// the r-th element with a warp-wide prefix sum (lane l owns digits 255-8l .. 248-8l).
 template <typename KeyT, int KBITS, typename KeyFn, typename PredFn>
 __device__ KeyT block_kth_largest(int n, int r, KeyFn key, PredFn pred, uint32_t* n_gt) {
   __shared__ uint32_t hist[256];
-  __shared__ uint32_t sh_digit, sh_rem;
+  __shared__ uint32_t sh_digit, sh_rem, sh_gt;
   KeyT prefix = 0, mask = 0;
   uint32_t rem = (uint32_t)r, gt = 0;
   for (int shift = KBITS - 8; shift >= 0; shift -= 8) {
     for (int e = threadIdx.x; e < 256; e += blockDim.x) hist[e] = 0u;
+    if (threadIdx.x == 0) {
+      sh_digit = 0u;
+      sh_rem = rem;
+      sh_gt = 0u;
+    }
     __syncthreads();
     for (int e = threadIdx.x; e < n; e += blockDim.x) {
       if (!pred(e)) continue;
@@ -198,24 +322,43 @@ __device__ KeyT block_kth_largest(int n, int r, KeyFn key, PredFn pred, uint32_t
       if ((k & mask) == prefix) atomicAdd(&hist[(uint32_t)(k >> shift) & 255u], 1u);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      uint32_t cum = 0;
-      int dg = 255;
-      for (; dg > 0; --dg) {
-        if (cum + hist[dg] >= rem) break;
-        cum += hist[dg];
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      uint32_t c[8], s = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        c[u] = hist[255 - 8 * lane - u];
+        s += c[u];
       }
-      sh_digit = (uint32_t)dg;
-      sh_rem = rem - cum;
-      gt += cum;
+      uint32_t incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const uint32_t excl = incl - s;
+      if (excl < rem && rem <= incl) {
+        uint32_t cum = excl;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (cum + c[u] >= rem) {
+            sh_digit = (uint32_t)(255 - 8 * lane - u);
+            sh_rem = rem - cum;
+            sh_gt = cum;
+            break;
+          }
+          cum += c[u];
+        }
+      }
     }
     __syncthreads();
     prefix |= (KeyT)sh_digit << shift;
     mask |= (KeyT)255 << shift;
     rem = sh_rem;
+    gt += sh_gt;
     __syncthreads();
   }
-  if (threadIdx.x == 0) *n_gt = gt;  // greater-count accumulated by thread 0 only
+  if (threadIdx.x == 0) *n_gt = gt;
   __syncthreads();
   return prefix;
 }
@@ -223,7 +366,14 @@ __device__ KeyT block_kth_largest(int n, int r, KeyFn key, PredFn pred, uint32_t
 template <int H, bool FP8>
 __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams p) {
   __shared__ int sel[kMaxIdxWidth];
+  // One scratch area: the small band's (t, position) pairs, later the sort buffer.
+  __shared__ __align__(16) unsigned char scratch[kMaxIdxWidth * sizeof(int)];
+  double* band_ts = reinterpret_cast<double*>(scratch);                    // [kSmallBand]
+  int* band_js = reinterpret_cast<int*>(scratch + kSmallBand * sizeof(double));
+  int* tmp = reinterpret_cast<int*>(scratch);                              // [kMaxIdxWidth]
+  __shared__ uint32_t bucket[kBuckets], bucket_beg[kBuckets];
   __shared__ uint32_t n_sel, n_band_s, gt_s;
+  extern __shared__ __align__(16) uint16_t qsm[];  // [H][kQLd] bf16 q of this query
   __shared__ double dlt[H];
   const int bq = blockIdx.x;
   const int b = bq / p.n_q, i = bq % p.n_q;
@@ -270,48 +420,89 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
     if (t > hi_b) push(__ldcg(cj + e));
     else if (t >= lo_b) bj[atomicAdd(&n_band_s, 1u)] = __ldcg(cj + e);
   }
-  for (int hd = threadIdx.x; hd < H; hd += blockDim.x) dlt[hd] = p.delta64[(size_t)bq * H + hd];
+  __syncthreads();
+  load_delta(p.lse64 + (size_t)bq * H, H, nullptr, dlt);
+  for (int e = threadIdx.x; e < H * (kHeadDim / 8); e += blockDim.x) {
+    const int h = e / (kHeadDim / 8), c = (e % (kHeadDim / 8)) * 8;
+    *reinterpret_cast<uint4*>(qsm + h * kQLd + c) =
+        *reinterpret_cast<const uint4*>(p.q + ((size_t)bq * H + h) * kHeadDim + c);
+  }
   __syncthreads();
   const int n_band = (int)n_band_s;
   const int need2 = p.k_sel - (int)n_sel;  // taken from the band
 
   if (need2 > 0) {
-    // float64 re-scoring of the band: one warp per key, lanes split the dimension.
+    // float64 re-scoring of the band: one warp per key, lane l takes heads l, l+32, ...
+    // (q from shared memory, the key's row through L1: every lane reads the same row).
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const double scale = (double)p.sm_scale;
     for (int e = warp; e < n_band; e += blockDim.x / 32) {
       const int j = bj[e];
       const size_t row = (size_t)b * p.kv.max_len + j;
-      double kx[4];
-      if (FP8) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(
-            static_cast<const uint8_t*>(p.kv.k) + row * kHeadDim + lane * 4);
-        const double ks = (double)p.kv.k_scale[row];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) kx[t] = e4m3_to_f64((w >> (8 * t)) & 0xffu) * ks;
-      } else {
-        const uint2 w = *reinterpret_cast<const uint2*>(
-            static_cast<const uint16_t*>(p.kv.k) + row * kHeadDim + lane * 4);
-        kx[0] = bf16_bits_to_f32(w.x & 0xffffu);
-        kx[1] = bf16_bits_to_f32(w.x >> 16);
-        kx[2] = bf16_bits_to_f32(w.y & 0xffffu);
-        kx[3] = bf16_bits_to_f32(w.y >> 16);
-      }
       double best = -INFINITY;
-      for (int hd = 0; hd < H; ++hd) {
-        const uint2 qw = __ldg(reinterpret_cast<const uint2*>(
-            p.q + ((size_t)bq * H + hd) * kHeadDim + lane * 4));
-        double d = (double)bf16_bits_to_f32(qw.x & 0xffffu) * kx[0] +
-                   (double)bf16_bits_to_f32(qw.x >> 16) * kx[1] +
-                   (double)bf16_bits_to_f32(qw.y & 0xffffu) * kx[2] +
-                   (double)bf16_bits_to_f32(qw.y >> 16) * kx[3];
-        d = warp_sum_d(d);
-        best = fmax(best, scale * d - dlt[hd]);
+      for (int h = lane; h < H; h += 32) {
+        const uint16_t* qh = qsm + h * kQLd;
+        double dot = 0.0;
+        if (FP8) {
+          const uint8_t* kr = static_cast<const uint8_t*>(p.kv.k) + row * kHeadDim;
+#pragma unroll 2
+          for (int c = 0; c < kHeadDim; c += 16) {
+            const uint4 kv = __ldg(reinterpret_cast<const uint4*>(kr + c));
+            const uint4 qa = *reinterpret_cast<const uint4*>(qh + c);
+            const uint4 qb = *reinterpret_cast<const uint4*>(qh + c + 8);
+            const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+            const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              const uint32_t code = (kw[u >> 2] >> (8 * (u & 3))) & 0xffu;
+              const uint32_t qbits = (u & 1) ? (qw[u >> 1] >> 16) : (qw[u >> 1] & 0xffffu);
+              dot = fma((double)bf16_bits_to_f32(qbits), e4m3_to_f64(code), dot);
+            }
+          }
+          dot *= (double)p.kv.k_scale[row];
+        } else {
+          const uint16_t* kr = static_cast<const uint16_t*>(p.kv.k) + row * kHeadDim;
+#pragma unroll 2
+          for (int c = 0; c < kHeadDim; c += 8) {
+            const uint4 kv = __ldg(reinterpret_cast<const uint4*>(kr + c));
+            const uint4 qv = *reinterpret_cast<const uint4*>(qh + c);
+            const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              dot = fma((double)bf16_bits_to_f32(qw[u] & 0xffffu),
+                        (double)bf16_bits_to_f32(kw[u] & 0xffffu), dot);
+              dot = fma((double)bf16_bits_to_f32(qw[u] >> 16),
+                        (double)bf16_bits_to_f32(kw[u] >> 16), dot);
+            }
+          }
+        }
+        best = fmax(best, scale * dot - dlt[h]);
       }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) best = fmax(best, __shfl_xor_sync(0xffffffffu, best, o));
       if (lane == 0) bt[e] = best;
     }
     __threadfence_block();
     __syncthreads();
+    if (n_band <= kSmallBand) {
+      // Small band: rank every key by (t desc, position asc) against all the others.
+      for (int e = threadIdx.x; e < n_band; e += blockDim.x) {
+        band_ts[e] = bt[e];
+        band_js[e] = bj[e];
+      }
+      __syncthreads();
+      for (int e = threadIdx.x; e < n_band; e += blockDim.x) {
+        const double te = band_ts[e];
+        const int je = band_js[e];
+        int rank = 0;
+        for (int f = 0; f < n_band; ++f) {
+          const double tf = band_ts[f];
+          rank += (tf > te) || (tf == te && band_js[f] < je);
+        }
+        if (rank < need2) push(je);
+      }
+    } else {
     // Boundary value among the band, then the lowest positions among its ties.
     const unsigned long long vb = block_kth_largest<unsigned long long, 64>(
         n_band, need2, [&](int e) { return ordered_key64(bt[e]); }, [](int) { return true; },
@@ -326,36 +517,59 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
       const unsigned long long kk = ordered_key64(bt[e]);
       if (kk > vb || (kk == vb && bj[e] <= jb)) push(bj[e]);
     }
+    }
   }
   // The forced recent window [p - window + 1, p].
   for (int j = n_c + threadIdx.x; j <= pos; j += blockDim.x) push(j);
   __syncthreads();
-  // Bitonic sort of the selection (ascending), padded to a power of two.
+  // Ascending order of the n selected (distinct) positions: counting sort on the
+  // position's high bits into 1024 buckets, then each key's rank inside its bucket.
   const int n = (int)min(n_sel, (uint32_t)kMaxIdxWidth);
-  int np2 = 1;
-  while (np2 < n) np2 <<= 1;
-  for (int e = n + threadIdx.x; e < np2; e += blockDim.x) sel[e] = 0x7fffffff;
+  int shift = 0;
+  while ((pos >> shift) >= kBuckets) ++shift;
+  for (int e = threadIdx.x; e < kBuckets; e += blockDim.x) bucket[e] = 0u;
   __syncthreads();
-  for (int kk = 2; kk <= np2; kk <<= 1) {
-    for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-      for (int e = threadIdx.x; e < np2; e += blockDim.x) {
-        const int partner = e ^ jj;
-        if (partner > e) {
-          const bool up = (e & kk) == 0;
-          const int a = sel[e], c = sel[partner];
-          if ((a > c) == up) {
-            sel[e] = c;
-            sel[partner] = a;
-          }
-        }
-      }
-      __syncthreads();
+  for (int e = threadIdx.x; e < n; e += blockDim.x) atomicAdd(&bucket[sel[e] >> shift], 1u);
+  __syncthreads();
+  if (threadIdx.x < 32) {  // exclusive prefix over the buckets, 32 per lane
+    const int lane = threadIdx.x;
+    uint32_t sum = 0;
+    for (int u = 0; u < kBuckets / 32; ++u) sum += bucket[lane * (kBuckets / 32) + u];
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += x;
+    }
+    uint32_t run = incl - sum;
+    for (int u = 0; u < kBuckets / 32; ++u) {
+      const uint32_t c = bucket[lane * (kBuckets / 32) + u];
+      bucket[lane * (kBuckets / 32) + u] = run;
+      bucket_beg[lane * (kBuckets / 32) + u] = run;
+      run += c;
     }
   }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const int v = sel[e];
+    tmp[atomicAdd(&bucket[v >> shift], 1u)] = v;  // bucket[b] advances to b's end
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const int v = tmp[e];
+    const uint32_t beg = bucket_beg[v >> shift], end = bucket[v >> shift];
+    uint32_t rank = 0;
+    for (uint32_t x = beg; x < end; ++x) rank += tmp[x] < v;
+    sel[beg + rank] = v;
+  }
+  __syncthreads();
   for (int e = threadIdx.x; e < width; e += blockDim.x) out[e] = e < n ? sel[e] : -1;
 }
 
 // ----------------------------------------------------------------------------
+template <int H, bool FP8>
+static cudaError_t launch_rest_t(const SelectParams& p, int batch, cudaStream_t st);
+
 template <int H, bool FP8>
 static cudaError_t launch_select_t(const SelectParams& p, int batch, cudaStream_t st) {
   const size_t smem = simt_smem_bytes(H);
@@ -370,11 +584,7 @@ static cudaError_t launch_select_t(const SelectParams& p, int batch, cudaStream_
   importance_simt_kernel<H, FP8><<<dim3(p.splits2, bq), kThreads, smem, st>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  select_compact_kernel<<<dim3(p.splits3, bq), kThreads, 0, st>>>(p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  select_finish_kernel<H, FP8><<<bq, kFinThreads, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_rest_t<H, FP8>(p, batch, st);
 }
 
 template <int H, bool FP8>
@@ -383,7 +593,15 @@ static cudaError_t launch_rest_t(const SelectParams& p, int batch, cudaStream_t 
   select_compact_kernel<<<dim3(p.splits3, bq), kThreads, 0, st>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  select_finish_kernel<H, FP8><<<bq, kFinThreads, 0, st>>>(p);
+  const size_t qbytes = H * kQLd * sizeof(uint16_t);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(select_finish_kernel<H, FP8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qbytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  select_finish_kernel<H, FP8><<<bq, kFinThreads, qbytes, st>>>(p);
   return cudaGetLastError();
 }
 

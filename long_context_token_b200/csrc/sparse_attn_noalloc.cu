@@ -6,15 +6,15 @@
 // stray allocations, a plugin loaded into a host framework that owns the allocator,
 // or a plain C caller that keeps no buffer alive between calls.  cudaMalloc may also
 // synchronise the device, which such callers cannot afford in the middle of a step.
-// For them this entry point keeps the layer's scratch (the split partials and the
-// merge tickets) in a fixed array that lives in the library's own device memory:
+// For them this entry point keeps the layer's scratch (the split partials) in a fixed
+// array that lives in the library's own device memory:
 // every GPU that loads the library holds kNoAllocScratchBytes of it until the
 // process exits.  The caller still passes the inputs and the output.
 //
-// The array is shared by every call on a device and keeps what the last call left
-// in it; the merge tickets are cleared at the start of each call.  Two calls whose
-// kernels overlap on the GPU (different streams without ordering between them) race
-// on the array and give wrong results: serialise them.
+// The array is shared by every call on a device and keeps what the last call left in
+// it; every call rewrites all the partials it reads, so nothing needs clearing.  Two
+// calls whose kernels overlap on the GPU (different streams without ordering between
+// them) race on the array and give wrong results: serialise them.
 #include <mutex>
 
 #include "hs2_internal.cuh"
@@ -76,11 +76,10 @@ extern "C" HS2_API hs2_status hs2_sparse_attn_noalloc(const void* q_layer, int n
                           (uintptr_t)kv->v;
   if (align & 15u) return HS2_ERR_INVALID_ARGUMENT;
 
-  // Scratch layout: [status word][tickets][partial o][partial (m, l)].
+  // Scratch layout: [status word][partial o][partial (m, l)].
   const size_t bq = (size_t)kv->batch * n_q;
   const int splits = (idx_width + kChunkRows - 1) / kChunkRows;
-  const size_t off_tickets = 256;
-  const size_t off_o = off_tickets + round256(bq * sizeof(uint32_t));
+  const size_t off_o = 256;
   const size_t off_ml = off_o + round256(bq * splits * h_q * kHeadDim * sizeof(float));
   const size_t need = off_ml + round256(bq * splits * h_q * 2 * sizeof(float));
   if (need > kNoAllocScratchBytes) return HS2_ERR_WORKSPACE_TOO_SMALL;
@@ -89,8 +88,6 @@ extern "C" HS2_API hs2_status hs2_sparse_attn_noalloc(const void* q_layer, int n
   cudaError_t e = scratch_address(&base);
   if (e != cudaSuccess) return HS2_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
-  e = cudaMemsetAsync(static_cast<char*>(base) + off_tickets, 0, bq * sizeof(uint32_t), s);
-  if (e != cudaSuccess) return HS2_ERR_CUDA;
 
   SparseParams p;
   p.q = static_cast<const uint16_t*>(q_layer);
@@ -111,9 +108,17 @@ extern "C" HS2_API hs2_status hs2_sparse_attn_noalloc(const void* q_layer, int n
   p.chunk4 = kChunkRows;
   p.part_o = reinterpret_cast<float*>(static_cast<char*>(base) + off_o);
   p.part_ml = reinterpret_cast<float*>(static_cast<char*>(base) + off_ml);
-  p.tickets = reinterpret_cast<uint32_t*>(static_cast<char*>(base) + off_tickets);
-  p.out = out;
   p.status = device_status ? device_status : static_cast<uint32_t*>(base);
   e = launch_sparse_attn(p, kv->batch, s);
+  if (e != cudaSuccess) return HS2_ERR_CUDA;
+  MergeParams m;
+  m.part_o = p.part_o;
+  m.part_ml = p.part_ml;
+  m.splits = splits;
+  m.h = h_q;
+  m.out = out;
+  m.lse_out = nullptr;
+  m.lse64 = nullptr;
+  e = launch_merge(m, (int)bq, false, s);
   return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
 }

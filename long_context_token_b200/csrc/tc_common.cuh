@@ -66,6 +66,8 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint
 
 cudaError_t launch_full_attn_tc(const FullParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                                 int bq, cudaStream_t st);
+// Sparse layer through the same kernel in gather mode (p.idx, p.idx_width set).
+cudaError_t launch_sparse_attn_tc(const FullParams& p, int bq, cudaStream_t st);
 cudaError_t launch_importance_tc(const SelectParams& p, const CUtensorMap& tmap_k, int bq,
                                  cudaStream_t st);
 

@@ -1,6 +1,5 @@
 // CUDA-core building blocks: 32-row K/V tiles staged as float32 in shared memory,
-// the QK^T tile, the online-softmax update and the P.V accumulation, plus the
-// split merge.  Used by the full layer (contiguous rows), the importance pass and
+// the QK^T tile, the online-softmax update and the P.V accumulation.  Used by the full layer (contiguous rows), the importance pass and
 // the sparse layers (gathered rows).
 #pragma once
 
@@ -159,6 +158,24 @@ __device__ __forceinline__ void pv_tile(const SimtSmem& s, float* acc) {
   }
 }
 
+// Selection shift delta_h = lse_h - min_h' lse_h' of one (sequence, token), from the
+// full layer's float64 lse (every thread of the block calls this).
+__device__ __forceinline__ void load_delta(const double* lse64, int H, float* d32, double* d64) {
+  __shared__ double mn;
+  if (threadIdx.x == 0) {
+    double m = INFINITY;
+    for (int h = 0; h < H; ++h) m = fmin(m, lse64[h]);
+    mn = m;
+  }
+  __syncthreads();
+  for (int h = threadIdx.x; h < H; h += blockDim.x) {
+    const double d = lse64[h] - mn;
+    if (d32) d32[h] = (float)d;
+    if (d64) d64[h] = d;
+  }
+  __syncthreads();
+}
+
 // Write this split's partial state (m, l, unnormalised o).
 template <int H>
 __device__ __forceinline__ void write_partial(const SimtSmem& s, const float* acc,
@@ -170,79 +187,6 @@ __device__ __forceinline__ void write_partial(const SimtSmem& s, const float* ac
     part_ml[2 * hd] = s.m_run[hd];
     part_ml[2 * hd + 1] = s.l_run[hd];
   }
-}
-
-// Returns true in exactly one CTA of the `n` CTAs sharing `ticket`: the last one to
-// arrive after all of them wrote their partials.  That CTA resets the ticket.
-__device__ __forceinline__ bool arrive_last(uint32_t* ticket, int n) {
-  __shared__ int last;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const uint32_t prev = atomicAdd(ticket, 1u);
-    last = (prev == (uint32_t)(n - 1));
-    if (last) *ticket = 0u;
-  }
-  __syncthreads();
-  if (last) __threadfence();
-  return last != 0;
-}
-
-// Merge `splits` partials of H heads into out (normalised) and per-head lse.
-// lse_d (shared, H doubles) receives ln(sum) in float64; heads with no key get
-// lse = -inf and out = 0.  Uses `scratch` (shared, >= 32*H + 2*H floats).
-template <int H>
-__device__ void merge_partials(const float* part_o, const float* part_ml, int splits,
-                               float* out, double* lse_d, float* scratch) {
-  float* w = scratch;              // [32][H]
-  float* Mf = scratch + 32 * H;    // [H]
-  float* invL = Mf + H;            // [H]
-  for (int hd = threadIdx.x; hd < H; hd += kThreads) {
-    float M = -INFINITY;
-    for (int sp = 0; sp < splits; ++sp) M = fmaxf(M, __ldcg(part_ml + ((size_t)sp * H + hd) * 2));
-    double Ls = 0.0;
-    if (M != -INFINITY) {
-      for (int sp = 0; sp < splits; ++sp) {
-        const float m = __ldcg(part_ml + ((size_t)sp * H + hd) * 2);
-        const float l = __ldcg(part_ml + ((size_t)sp * H + hd) * 2 + 1);
-        if (l > 0.f) Ls += (double)l * exp((double)m - (double)M);
-      }
-    }
-    Mf[hd] = M;
-    invL[hd] = Ls > 0.0 ? (float)(1.0 / Ls) : 0.f;
-    lse_d[hd] = Ls > 0.0 ? (double)M + log(Ls) : -INFINITY;
-  }
-  __syncthreads();
-  const int d = threadIdx.x & (kHeadDim - 1), hg2 = threadIdx.x >> 7;
-  float acc[H / 2];
-#pragma unroll
-  for (int r = 0; r < H / 2; ++r) acc[r] = 0.f;
-  for (int sb = 0; sb < splits; sb += 32) {
-    for (int e = threadIdx.x; e < 32 * H; e += kThreads) {
-      const int sp = sb + e / H, hd = e % H;
-      float wt = 0.f;
-      if (sp < splits && Mf[hd] != -INFINITY) {
-        const float m = __ldcg(part_ml + ((size_t)sp * H + hd) * 2);
-        const float l = __ldcg(part_ml + ((size_t)sp * H + hd) * 2 + 1);
-        if (l > 0.f) wt = expf(m - Mf[hd]) * invL[hd];
-      }
-      w[e] = wt;
-    }
-    __syncthreads();
-    const int nsb = min(32, splits - sb);
-    for (int t = 0; t < nsb; ++t) {
-#pragma unroll
-      for (int r = 0; r < H / 2; ++r) {
-        const int hd = hg2 + 2 * r;
-        const float wt = w[t * H + hd];
-        if (wt != 0.f)
-          acc[r] = fmaf(wt, __ldcg(part_o + ((size_t)(sb + t) * H + hd) * kHeadDim + d), acc[r]);
-      }
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int r = 0; r < H / 2; ++r) out[(hg2 + 2 * r) * kHeadDim + d] = acc[r];
 }
 
 }  // namespace hs2
