@@ -160,7 +160,27 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
   p.status = ws_ptr<uint32_t>(ws, w.status);
   bool log2_partials = false;
   cudaError_t e;
-  if (kv->dtype == HS2_KV_BF16 && h <= 64) {
+  if (kv->dtype == HS2_KV_FP8_E4M3 && h <= 64) {
+    // Tensor-core flash-decode over E4M3 tiles widened to f16 in shared memory.
+    CUtensorMap tk, tv;
+    const uint64_t rows = (uint64_t)kv->batch * kv->max_len;
+    if (!make_tmap_2d(&tk, kv->k, CU_TENSOR_MAP_DATA_TYPE_UINT8, kHeadDim, rows, kHeadDim, 128,
+                      128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_2d(&tv, kv->v, CU_TENSOR_MAP_DATA_TYPE_UINT8, kHeadDim, rows, kHeadDim, 128,
+                      128, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cuda_fail(cudaErrorInvalidValue, "tensor maps of K/V");
+    const int bq = kv->batch * n_q;
+    int splits = device_sm_count() / bq;
+    if (splits > w.splits1) splits = w.splits1;
+    if (splits < 1) splits = 1;
+    int chunk = (kv->max_len + splits - 1) / splits;
+    chunk = (chunk + 127) / 128 * 128;
+    p.splits1 = (kv->max_len + chunk - 1) / chunk;
+    p.chunk1 = chunk;
+    p.sbuf = w.use_sbuf ? ws_ptr<float>(ws, w.sbuf) : nullptr;
+    e = launch_full_attn_fp8(p, tk, tv, bq, s);
+    log2_partials = true;
+  } else if (kv->dtype == HS2_KV_BF16 && h <= 64) {
     // Tensor-core flash-decode: about one CTA per SM, chunks of whole 128-key tiles.
     CUtensorMap tk, tv;
     const uint64_t rows = (uint64_t)kv->batch * kv->max_len;
@@ -320,7 +340,7 @@ hs2_status hs2_sparse_attn(const void* q_layer, int n_q, int h_q, const hs2_kv* 
   WsLayout w;
   make_layout(kv->batch, n_q, h_q, kv->max_len, 1, 1, kv->dtype, &w);
   if (ws_bytes < sparse_prefix_bytes(w)) return HS2_ERR_WORKSPACE_TOO_SMALL;
-  if (kv->dtype == HS2_KV_BF16 && h_q <= 64) {
+  if (h_q <= 64) {
     // Tensor-core gather attention: 128 index entries per CTA, log2-domain partials.
     FullParams f;
     f.q = static_cast<const uint16_t*>(q_layer);
@@ -337,7 +357,9 @@ hs2_status hs2_sparse_attn(const void* q_layer, int n_q, int h_q, const hs2_kv* 
     f.status = ws_ptr<uint32_t>(workspace, w.status);
     f.idx = idx;
     f.idx_width = idx_width;
-    cudaError_t e = launch_sparse_attn_tc(f, kv->batch * n_q, (cudaStream_t)stream);
+    cudaError_t e = kv->dtype == HS2_KV_FP8_E4M3
+                        ? launch_sparse_attn_fp8(f, kv->batch * n_q, (cudaStream_t)stream)
+                        : launch_sparse_attn_tc(f, kv->batch * n_q, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "sparse-attention launch");
     MergeParams m;
     m.part_o = f.part_o;

@@ -138,10 +138,10 @@ cudaError_t launch_select(const SelectParams& p, int batch, cudaStream_t s);
 cudaError_t launch_select_rest(const SelectParams& p, int batch, cudaStream_t s);
 // Importance from the full layer's stored float32 logits.
 cudaError_t launch_importance_sbuf(const SelectParams& p, int bq, cudaStream_t s);
-// The stored-logit path applies to single-token decode with 16 heads on a bf16 cache:
-// 64 bytes of logits per key instead of re-reading its 256-byte K row.
-inline bool sbuf_eligible(int n_q, int h, int dtype) {
-  return n_q == 1 && h == 16 && dtype == HS2_KV_BF16;
+// The stored-logit path applies to single-token decode with 16 heads: 64 bytes of
+// logits per key instead of re-reading its K row (256 bytes bf16, 132 bytes FP8).
+inline bool sbuf_eligible(int n_q, int h, int /*dtype*/) {
+  return n_q == 1 && h == 16;
 }
 cudaError_t launch_sparse_attn(const SparseParams& p, int batch, cudaStream_t s);
 cudaError_t launch_merge(const MergeParams& p, int bq, bool log2_domain, cudaStream_t s);

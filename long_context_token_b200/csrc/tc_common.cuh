@@ -68,6 +68,10 @@ cudaError_t launch_full_attn_tc(const FullParams& p, const CUtensorMap& tk, cons
                                 int bq, cudaStream_t st);
 // Sparse layer through the same kernel in gather mode (p.idx, p.idx_width set).
 cudaError_t launch_sparse_attn_tc(const FullParams& p, int bq, cudaStream_t st);
+// The same two kernels for an FP8 E4M3 cache (tensor maps over uint8 rows).
+cudaError_t launch_full_attn_fp8(const FullParams& p, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, int bq, cudaStream_t st);
+cudaError_t launch_sparse_attn_fp8(const FullParams& p, int bq, cudaStream_t st);
 cudaError_t launch_importance_tc(const SelectParams& p, const CUtensorMap& tmap_k, int bq,
                                  cudaStream_t st);
 
