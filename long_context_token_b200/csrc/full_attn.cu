@@ -15,6 +15,7 @@ template <int H, bool FP8>
 __global__ void __launch_bounds__(kThreads) full_attn_simt_kernel(FullParams p) {
   extern __shared__ __align__(16) float smem[];
   SimtSmem s = carve_simt(smem, H);
+  griddep_wait();
   const int split = blockIdx.x, bq = blockIdx.y;
   const int b = bq / p.n_q, i = bq % p.n_q;
   const int L = seq_len(p.kv, b, p.n_q, p.status, split == 0 && i == 0);
@@ -65,8 +66,7 @@ static cudaError_t launch_full_t(const FullParams& p, int batch, cudaStream_t st
     attr_set = true;
   }
   dim3 grid(p.splits1, batch * p.n_q);
-  full_attn_simt_kernel<H, FP8><<<grid, kThreads, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(full_attn_simt_kernel<H, FP8>, grid, dim3(kThreads), smem, st, p);
 }
 
 template <bool FP8>

@@ -145,30 +145,8 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
   const int warp = threadIdx.x >> 5;
   const int split = blockIdx.x, bq = blockIdx.y;
   const int b = bq / p.n_q, qi = bq % p.n_q;
-  const int Lb = seq_len(p.kv, b, p.n_q, p.status, !GATHER && split == 0 && qi == 0);
-  const int pos = Lb - p.n_q + qi;
-  const int k0 = split * p.chunk1;
-  const int k1 = GATHER ? min(k0 + p.chunk1, p.idx_width) : min(k0 + p.chunk1, pos + 1);
-  const int32_t* idx_row = GATHER ? p.idx + (size_t)bq * p.idx_width : nullptr;
-  const size_t row_base = (size_t)b * p.kv.max_len;
-  const int n_tiles = k0 < k1 ? (k1 - k0 + kKeyTile - 1) / kKeyTile : 0;
-  const size_t pidx = (size_t)bq * p.splits1 + split;
 
-  // Row of the cache behind tile entry e (or -1 for an absent / past-the-end entry).
-  auto entry_row = [&](int e) -> long long {
-    if (e >= k1) return -1;
-    if (!GATHER) return (long long)(row_base + e);
-    const int j = __ldg(idx_row + e);
-    return (j >= 0 && j < Lb) ? (long long)(row_base + j) : -1;
-  };
-
-  if (n_tiles == 0) {
-    for (int h = threadIdx.x; h < H; h += blockDim.x) {
-      p.part_ml[pidx * H * 2 + 2 * h] = -INFINITY;
-      p.part_ml[pidx * H * 2 + 2 * h + 1] = 0.f;
-    }
-    return;
-  }
+  // Set-up that touches no global memory, overlapping the previous kernel's tail.
   if (threadIdx.x == 0) {
     for (int s = 0; s < R; ++s) {
       mbar_init(kr_full + s, GATHER ? 32 : 1);
@@ -197,48 +175,41 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
     prefetch_tmap(&tmap_k);
     prefetch_tmap(&tmap_v);
   }
-  // Per-head power-of-two Q scale: largest |q| of head h lands in [2^14, 2^15).
-  const uint16_t* qg = p.q + (size_t)bq * H * kHeadDim;
-  for (int h = warp; h < H; h += kFp8Threads / 32) {
-    float m = 0.f;
-    for (int c = (int)lane_id(); c < kHeadDim; c += 32)
-      m = fmaxf(m, fabsf(bf16_bits_to_f32(qg[h * kHeadDim + c])));
-    m = warp_max(m);
-    if (lane_id() == 0) {
-      int e = 0;
-      if (m > 0.f) {
-        int ex;
-        frexpf(m, &ex);  // m = f * 2^ex, f in [0.5, 1)
-        e = 15 - ex;
-        e = e < -100 ? -100 : (e > 100 ? 100 : e);
-      }
-      const float up = __int_as_float((127 + e) << 23), down = __int_as_float((127 - e) << 23);
-      qinv_s[h] = down;
-      c2_s[h] = p.sm_scale * kLog2eF8 * down;
-      alpha_s[h] = up;  // scratch: the factor applied to q before rounding to f16
+  griddep_wait();
+
+  const int Lb = seq_len(p.kv, b, p.n_q, p.status, !GATHER && split == 0 && qi == 0);
+  const int pos = Lb - p.n_q + qi;
+  const int k0 = split * p.chunk1;
+  const int k1 = GATHER ? min(k0 + p.chunk1, p.idx_width) : min(k0 + p.chunk1, pos + 1);
+  const int32_t* idx_row = GATHER ? p.idx + (size_t)bq * p.idx_width : nullptr;
+  const size_t row_base = (size_t)b * p.kv.max_len;
+  const int n_tiles = k0 < k1 ? (k1 - k0 + kKeyTile - 1) / kKeyTile : 0;
+  const size_t pidx = (size_t)bq * p.splits1 + split;
+
+  // Row of the cache behind tile entry e (or -1 for an absent / past-the-end entry).
+  auto entry_row = [&](int e) -> long long {
+    if (e >= k1) return -1;
+    if (!GATHER) return (long long)(row_base + e);
+    const int j = __ldg(idx_row + e);
+    return (j >= 0 && j < Lb) ? (long long)(row_base + j) : -1;
+  };
+  bool ok = true;
+
+  if (n_tiles == 0) {
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
+      p.part_ml[pidx * H * 2 + 2 * h] = -INFINITY;
+      p.part_ml[pidx * H * 2 + 2 * h + 1] = 0.f;
     }
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < H * (kHeadDim / 8); e += blockDim.x) {
-    const int h = e % H, c = e / H;
-    const uint4 v = *reinterpret_cast<const uint4*>(qg + h * kHeadDim + c * 8);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const __half lo = __float2half_rn(bf16_bits_to_f32(w[u] & 0xffffu) * alpha_s[h]);
-      const __half hi = __float2half_rn(bf16_bits_to_f32(w[u] >> 16) * alpha_s[h]);
-      o[u] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
-    }
-    *reinterpret_cast<uint4*>(qs + c * (H * 16) + h * 16) = make_uint4(o[0], o[1], o[2], o[3]);
-  }
+  } else {
+  // Q in f16 under a per-head power-of-two scale; its inverse goes into the logits.
+  store_q_f16_scaled<H>(qs, p.q + (size_t)bq * H * kHeadDim, qinv_s, nullptr);
+  for (int h = threadIdx.x; h < H; h += blockDim.x) c2_s[h] = p.sm_scale * kLog2eF8 * qinv_s[h];
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t tmem_o = tmem_base + 2 * H;
-  bool ok = true;
 
   if (warp == 0) {
     if (GATHER) {
@@ -366,13 +337,27 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
     for (int h = 0; h < H; ++h) l[h] = 0.f;
     if (t < H) mref_s[t] = -INFINITY;
     named_bar_sync(1, 128);
+    // Per-key scales (and validity) are loaded two tiles ahead so that their memory
+    // latency overlaps the tiles in between instead of stalling each tile.
+    auto scales_of = [&](int i, float& ks, float& vs, bool& ok_row) {
+      const long long row = i < n_tiles ? entry_row(k0 + i * kKeyTile + t) : -1;
+      ok_row = row >= 0;
+      ks = ok_row ? __ldg(p.kv.k_scale + row) : 0.f;
+      vs = ok_row ? __ldg(p.kv.v_scale + row) : 0.f;
+    };
+    float ks_next, vs_next, ks_far, vs_far;
+    bool val_next, val_far;
+    scales_of(0, ks_next, vs_next, val_next);
+    scales_of(1, ks_far, vs_far, val_far);
     for (int i = 0; i < n_tiles; ++i) {
       const int sb = i & 1;
       const int j = k0 + i * kKeyTile + t;
-      const long long row = entry_row(j);
-      const bool valid = row >= 0;
-      const float ks = valid ? __ldg(p.kv.k_scale + row) : 0.f;
-      const float vs = valid ? __ldg(p.kv.v_scale + row) : 0.f;
+      const float ks = ks_next, vs = vs_next;
+      const bool valid = val_next;
+      ks_next = ks_far;
+      vs_next = vs_far;
+      val_next = val_far;
+      scales_of(i + 2, ks_far, vs_far, val_far);
       if (ok && !mbar_wait(s_full + sb, (i >> 1) & 1)) ok = false;
       if (named_bar_or(3, 128, !ok)) ok = false;
       tc_fence_after();
@@ -455,6 +440,7 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
       fence_proxy_async_smem();
       mbar_arrive(p_full + sb);
     }
+    griddep_launch_dependents();  // the merge may be scheduled; it waits for this grid
     const int last = n_tiles - 1;
     if (ok && !mbar_wait(p_free + (last & 1), (last >> 1) & 1)) ok = false;
     tc_fence_after();
@@ -479,12 +465,13 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
       p.part_ml[pidx * H * 2 + 2 * t + 1] = red[t] + red[H + t] + red[2 * H + t] + red[3 * H + t];
     }
   }
+  }
   if (!ok) set_status(p.status, HS2_ERR_DEVICE_TIMEOUT);
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, L::kTmemCols);
+    tmem_dealloc(*tmem_slot, L::kTmemCols);
   }
 }
 
@@ -499,8 +486,8 @@ static cudaError_t launch_fp8_t(const FullParams& p, const CUtensorMap& tk, cons
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  full_attn_fp8_kernel<H, GATHER><<<dim3(p.splits1, bq), kFp8Threads, L::kBytes, st>>>(tk, tv, p);
-  return cudaGetLastError();
+  return launch_pdl(full_attn_fp8_kernel<H, GATHER>, dim3(p.splits1, bq), dim3(kFp8Threads),
+                    L::kBytes, st, tk, tv, p);
 }
 
 template <bool GATHER>

@@ -99,7 +99,35 @@ __global__ void __launch_bounds__(192, 1)
   const int warp = threadIdx.x >> 5;
   const int split = blockIdx.x, bq = blockIdx.y;
   const int b = bq / p.n_q, qi = bq % p.n_q;
-  const int Lb = seq_len(p.kv, b, p.n_q, p.status, split == 0 && qi == 0);
+
+  // Set-up that touches no global memory, overlapping the previous kernel's tail.
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(kfull + s, GATHER ? 32 : 1);
+      mbar_init(kempty + s, 1);
+      mbar_init(vfull + s, GATHER ? 32 : 1);
+      mbar_init(vempty + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(s_full + s, 1);
+      mbar_init(s_free + s, 128);
+      mbar_init(p_full + s, 128);
+      mbar_init(p_free + s, 1);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  if (!GATHER && warp == 0 && lane_id() == 0) {
+    prefetch_tmap(&tmap_k);
+    prefetch_tmap(&tmap_v);
+  }
+  griddep_wait();
+
+  const int Lb = seq_len(p.kv, b, p.n_q, p.status, !GATHER && split == 0 && qi == 0);
   const int pos = Lb - p.n_q + qi;
   // Keys [k0, k1) of the sequence, or (gather mode) index entries [k0, k1) of the row.
   const int k0 = split * p.chunk1;
@@ -108,6 +136,7 @@ __global__ void __launch_bounds__(192, 1)
   const size_t row_base = (size_t)b * p.kv.max_len;
   const int n_tiles = k0 < k1 ? (k1 - k0 + kKeyTile - 1) / kKeyTile : 0;
   const size_t pidx = (size_t)bq * p.splits1 + split;
+  bool ok = true;
 
   if (n_tiles == 0) {
     // Empty chunk: an empty partial (no key).
@@ -116,30 +145,6 @@ __global__ void __launch_bounds__(192, 1)
       p.part_ml[pidx * H * 2 + 2 * h + 1] = 0.f;
     }
   } else {
-    if (threadIdx.x == 0) {
-      for (int s = 0; s < NS; ++s) {
-        mbar_init(kfull + s, GATHER ? 32 : 1);
-        mbar_init(kempty + s, 1);
-        mbar_init(vfull + s, GATHER ? 32 : 1);
-        mbar_init(vempty + s, 1);
-      }
-      for (int s = 0; s < 2; ++s) {
-        mbar_init(s_full + s, 1);
-        mbar_init(s_free + s, 128);
-        mbar_init(p_full + s, 128);
-        mbar_init(p_free + s, 1);
-      }
-      mbar_init(mma_done, 1);
-      fence_mbar_init();
-    }
-    if (warp == 1) {
-      tmem_alloc(tmem_slot, L::kTmemCols);
-      tmem_relinquish();
-    }
-    if (!GATHER && warp == 0 && lane_id() == 0) {
-      prefetch_tmap(&tmap_k);
-      prefetch_tmap(&tmap_v);
-    }
     store_q_kmajor<H>(qs, p.q + (size_t)bq * H * kHeadDim, threadIdx.x, blockDim.x);
     fence_proxy_async_smem();
     tc_fence_before();
@@ -147,7 +152,6 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const uint32_t tmem_o = tmem_base + 2 * H;
-    bool ok = true;
 
     if (GATHER && warp == 0) {
       // ------------------------------------------------ gather producer (32 lanes)
@@ -382,6 +386,7 @@ __global__ void __launch_bounds__(192, 1)
         fence_proxy_async_smem();
         mbar_arrive(p_full + sb);
       }
+      griddep_launch_dependents();  // the merge may be scheduled; it waits for this grid
       // Epilogue: O^T row t is dimension t of every head; l is reduced across threads.
       const int last = n_tiles - 1;
       if (ok && !mbar_wait(p_free + (last & 1), (last >> 1) & 1)) ok = false;
@@ -407,15 +412,14 @@ __global__ void __launch_bounds__(192, 1)
         p.part_ml[pidx * H * 2 + 2 * t + 1] = red[t] + red[H + t] + red[2 * H + t] + red[3 * H + t];
       }
     }
-    if (!ok) set_status(p.status, HS2_ERR_DEVICE_TIMEOUT);
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-      tc_fence_after();
-      tmem_dealloc(tmem_base, L::kTmemCols);
-    }
   }
-
+  if (!ok) set_status(p.status, HS2_ERR_DEVICE_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(*tmem_slot, L::kTmemCols);
+  }
 }
 
 template <int H, bool GATHER>
@@ -429,8 +433,8 @@ static cudaError_t launch_full_tc_t(const FullParams& p, const CUtensorMap& tk,
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  full_attn_tc_kernel<H, GATHER><<<dim3(p.splits1, bq), 192, L::kBytes, st>>>(tk, tv, p);
-  return cudaGetLastError();
+  return launch_pdl(full_attn_tc_kernel<H, GATHER>, dim3(p.splits1, bq), dim3(192), L::kBytes, st,
+                    tk, tv, p);
 }
 
 template <bool GATHER>

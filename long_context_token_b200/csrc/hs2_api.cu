@@ -219,9 +219,9 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
 static hs2_status run_select(const void* q, int n_q, int h, const hs2_kv* kv, int window,
                              int k_sel, float sm_scale, int32_t* idx, void* ws,
                              const WsLayout& w, cudaStream_t s) {
-  cudaError_t e = cudaMemsetAsync(ws_ptr<char>(ws, w.clear_begin), 0,
-                                  w.clear_end - w.clear_begin, s);
-  if (e != cudaSuccess) return cuda_fail(e, "workspace clear");
+  // The histogram and counters start at zero: the workspace is zero-filled before first
+  // use and every selection leaves them at zero when it finishes.
+  cudaError_t e = cudaSuccess;
   SelectParams p;
   p.q = static_cast<const uint16_t*>(q);
   p.kv = view_of(kv);
@@ -266,6 +266,21 @@ static hs2_status run_select(const void* q, int n_q, int h, const hs2_kv* kv, in
     p.splits2 = (kv->max_len + chunk - 1) / chunk;
     p.chunk2 = chunk;
     e = launch_importance_tc(p, tk, bq, s);
+    if (e != cudaSuccess) return cuda_fail(e, "importance launch");
+    e = launch_select_rest(p, kv->batch, s);
+  } else if (kv->dtype == HS2_KV_FP8_E4M3 && h <= 64) {
+    CUtensorMap tk;
+    if (!make_tmap_2d(&tk, kv->k, CU_TENSOR_MAP_DATA_TYPE_UINT8, kHeadDim,
+                      (uint64_t)kv->batch * kv->max_len, kHeadDim, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+      return cuda_fail(cudaErrorInvalidValue, "tensor map of K");
+    int splits = device_sm_count() / bq;
+    if (splits < 1) splits = 1;
+    int chunk = (kv->max_len + splits - 1) / splits;
+    chunk = (chunk + 127) / 128 * 128;
+    p.splits2 = (kv->max_len + chunk - 1) / chunk;
+    p.chunk2 = chunk;
+    e = launch_importance_fp8(p, tk, bq, s);
     if (e != cudaSuccess) return cuda_fail(e, "importance launch");
     e = launch_select_rest(p, kv->batch, s);
   } else {

@@ -131,6 +131,25 @@ struct SparseParams {
   uint32_t* status;
 };
 
+// Programmatic dependent launch: the kernel may be scheduled while the previous kernel
+// on the stream is finishing, so every kernel does only shared-memory / TMEM set-up
+// before griddep_wait() and touches global memory after it.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // Launchers (each returns the launch's cudaError_t).
 cudaError_t launch_full_attn(const FullParams& p, int batch, cudaStream_t s);
 cudaError_t launch_select(const SelectParams& p, int batch, cudaStream_t s);
@@ -150,6 +169,14 @@ cudaError_t launch_merge(const MergeParams& p, int bq, bool log2_domain, cudaStr
 // Device helpers.
 // ---------------------------------------------------------------------------
 #ifdef __CUDACC__
+
+// Wait until the previous kernel on the stream has completed and its writes are visible
+// (a no-op for a kernel launched without programmatic serialisation).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel on the stream be scheduled (it still waits for this grid's end).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) {
   return __uint_as_float(b << 16);

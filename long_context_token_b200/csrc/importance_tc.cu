@@ -14,6 +14,9 @@
 //               buffers;
 //   warps 2..5  epilogue: thread t owns TMEM lane t (= key t of the tile), loads
 //               its H logits, takes the max over heads, writes t_j and counts it.
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "hs2_internal.cuh"
 #include "sm100.cuh"
 #include "tc_common.cuh"
@@ -59,6 +62,7 @@ __global__ void __launch_bounds__(192, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlotOff);
 
   const int warp = threadIdx.x >> 5;
+  griddep_wait();
   const int split = blockIdx.x, bq = blockIdx.y;
   const int b = bq / p.n_q, qi = bq % p.n_q;
   const int Lb = seq_len(p.kv, b, p.n_q, p.status, false);
@@ -202,8 +206,7 @@ static cudaError_t launch_imp_t(const SelectParams& p, const CUtensorMap& tm, in
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  importance_tc_kernel<H><<<dim3(p.splits2, bq), 192, L::kBytes, st>>>(tm, p);
-  return cudaGetLastError();
+  return launch_pdl(importance_tc_kernel<H>, dim3(p.splits2, bq), dim3(192), L::kBytes, st, tm, p);
 }
 
 cudaError_t launch_importance_tc(const SelectParams& p, const CUtensorMap& tmap_k, int bq,
@@ -217,6 +220,259 @@ cudaError_t launch_importance_tc(const SelectParams& p, const CUtensorMap& tmap_
     case 96: return launch_imp_t<96>(p, tmap_k, bq, st);
     case 112: return launch_imp_t<112>(p, tmap_k, bq, st);
     case 128: return launch_imp_t<128>(p, tmap_k, bq, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+
+// ============================================================================
+// The same pass for an FP8 E4M3 cache: raw 128-key tiles by TMA, four conversion
+// warps widen them exactly to f16 (see the FP8 full layer), Q goes to f16 under a
+// per-head power-of-two scale, and each key's logits are multiplied by its k_scale.
+// ============================================================================
+namespace {
+
+constexpr int kImpF8Threads = 320;
+constexpr uint32_t kImpRawTile = 16384;
+constexpr uint32_t kImpConvTile = 32768;
+
+__device__ __forceinline__ uint32_t imp_e4m3x2_to_f16x2(uint32_t two_codes) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two_codes, __NV_E4M3);
+  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+__device__ __forceinline__ void imp_convert_row(const uint8_t* raw, uint8_t* conv, int r,
+                                                bool valid) {
+  const uint8_t* src = raw + r * 128;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 in = *reinterpret_cast<const uint4*>(src + (((c ^ r) & 7) << 4));
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      o[2 * u] = valid ? imp_e4m3x2_to_f16x2(w[u] & 0xffffu) : 0u;
+      o[2 * u + 1] = valid ? imp_e4m3x2_to_f16x2(w[u] >> 16) : 0u;
+    }
+    uint8_t* dst = conv + (c >> 2) * kBoxBytes + r * 128;
+    const int c0 = 2 * (c & 3);
+    *reinterpret_cast<uint4*>(dst + (((c0 ^ r) & 7) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(dst + ((((c0 + 1) ^ r) & 7) << 4)) =
+        make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+template <int H>
+struct ImpF8Smem {
+  static constexpr int R = 4;  // raw stages
+  static constexpr int C = 2;  // converted buffers
+  static constexpr uint32_t kQBytes = H * kHeadDim * 2;
+  static constexpr uint32_t kRawOff = 0;
+  static constexpr uint32_t kConvOff = R * kImpRawTile;
+  static constexpr uint32_t kQOff = kConvOff + C * kImpConvTile;
+  static constexpr uint32_t kHistOff = kQOff + kQBytes;
+  static constexpr uint32_t kDeltaOff = kHistOff + kHistBins * 4;
+  static constexpr uint32_t kQinvOff = kDeltaOff + H * 4;
+  static constexpr uint32_t kBarOff = kQinvOff + H * 4;
+  static constexpr uint32_t kBars = 2 * R + 2 * C + 4 + 1;
+  static constexpr uint32_t kSlotOff = kBarOff + kBars * 8;
+  static constexpr uint32_t kBytes = kSlotOff + 16 + 1024;
+  static constexpr uint32_t kTmemCols = tmem_cols_pow2(2 * H);
+  static_assert(kBytes <= 227 * 1024, "shared memory budget");
+};
+
+}  // namespace
+
+template <int H>
+__global__ void __launch_bounds__(kImpF8Threads, 1)
+    importance_fp8_kernel(const __grid_constant__ CUtensorMap tmap_k, SelectParams p) {
+  using L = ImpF8Smem<H>;
+  constexpr int R = L::R, C = L::C;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* raw = smem + L::kRawOff;
+  uint8_t* conv = smem + L::kConvOff;
+  uint8_t* qs = smem + L::kQOff;
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + L::kHistOff);
+  float* delta_s = reinterpret_cast<float*>(smem + L::kDeltaOff);
+  float* qinv_s = reinterpret_cast<float*>(smem + L::kQinvOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* r_full = bars;
+  uint64_t* r_empty = bars + R;
+  uint64_t* c_full = bars + 2 * R;
+  uint64_t* c_empty = bars + 2 * R + C;
+  uint64_t* s_full = bars + 2 * R + 2 * C;  // [2]
+  uint64_t* s_free = s_full + 2;            // [2]
+  uint64_t* mma_done = s_full + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
+
+  const int warp = threadIdx.x >> 5;
+  griddep_wait();
+  const int split = blockIdx.x, bq = blockIdx.y;
+  const int b = bq / p.n_q, qi = bq % p.n_q;
+  const int Lb = seq_len(p.kv, b, p.n_q, p.status, false);
+  const int pos = Lb - p.n_q + qi;
+  const int n_c = pos - p.window + 1;
+  if (n_c <= p.k_sel) return;
+  const int k0 = split * p.chunk2;
+  const int k1 = min(k0 + p.chunk2, n_c);
+  if (k0 >= k1) return;
+  const int n_tiles = (k1 - k0 + kKeyTile - 1) / kKeyTile;
+  const size_t row_base = (size_t)b * p.kv.max_len;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < R; ++s) {
+      mbar_init(r_full + s, 1);
+      mbar_init(r_empty + s, 128);
+    }
+    for (int s = 0; s < C; ++s) {
+      mbar_init(c_full + s, 128);
+      mbar_init(c_empty + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(s_full + s, 1);
+      mbar_init(s_free + s, 128);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane_id() == 0) prefetch_tmap(&tmap_k);
+  for (int e = threadIdx.x; e < kHistBins; e += blockDim.x) hist_s[e] = 0u;
+  load_delta(p.lse64 + (size_t)bq * H, H, delta_s, nullptr);
+  store_q_f16_scaled<H>(qs, p.q + (size_t)bq * H * kHeadDim, qinv_s, nullptr);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      const uint64_t pol = policy_evict_first();
+      const int row0 = (int)row_base + k0;
+      int issued = 0;
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        const int s = i % R;
+        if (!mbar_wait(r_empty + s, ((i / R) & 1) ^ 1)) { ok = false; break; }
+        mbar_arrive_expect_tx(r_full + s, kImpRawTile);
+        tma_load_2d(raw + s * kImpRawTile, &tmap_k, r_full + s, 0, row0 + i * kKeyTile, pol);
+        issued = i + 1;
+      }
+      for (int i = issued > R ? issued - R : 0; i < issued; ++i)
+        if (!mbar_wait(r_full + (i % R), (i / R) & 1)) ok = false;
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      const uint32_t idesc = idesc_f16(128, H, false, false, false);
+      const uint32_t q_addr = smem_u32(qs);
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        const int cb = i % C, sb = i & 1;
+        if (!mbar_wait(c_full + cb, (i / C) & 1)) { ok = false; break; }
+        if (!mbar_wait(s_free + sb, ((i >> 1) & 1) ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(conv + cb * kImpConvTile);
+#pragma unroll
+        for (int kk = 0; kk < kHeadDim / 16; ++kk)
+          mma_f16_ss(tmem_base + sb * H, kmajor_sw128_desc(a_addr, kk),
+                     q_kmajor_desc<H>(q_addr, kk), idesc, kk > 0 ? 1u : 0u);
+        mma_commit(s_full + sb);
+        mma_commit(c_empty + cb);
+      }
+      mma_commit(mma_done);
+      if (!mbar_wait(mma_done, 0)) ok = false;
+    }
+  } else if (warp >= 6) {
+    // conversion: thread t converts row t of each raw tile
+    const int t = threadIdx.x - 192;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int s = i % R, cb = i % C;
+      if (ok && !mbar_wait(r_full + s, (i / R) & 1)) ok = false;
+      if (ok && !mbar_wait(c_empty + cb, ((i / C) & 1) ^ 1)) ok = false;
+      imp_convert_row(raw + s * kImpRawTile, conv + cb * kImpConvTile, t,
+                      k0 + i * kKeyTile + t < k1);
+      fence_proxy_async_smem();
+      mbar_arrive(c_full + cb);
+      mbar_arrive(r_empty + s);
+    }
+  } else {
+    // epilogue: thread t owns key t of the tile
+    const int lg = warp & 3;
+    const int t = lg * 32 + (int)lane_id();
+    float* trow = p.tbuf + (size_t)bq * p.kv.max_len;
+    const float sc = p.sm_scale;
+    auto scale_of = [&](int i) {
+      const int j = k0 + i * kKeyTile + t;
+      return (i < n_tiles && j < k1) ? __ldg(p.kv.k_scale + row_base + j) : 0.f;
+    };
+    float ks_next = scale_of(0), ks_far = scale_of(1);
+    for (int i = 0; i < n_tiles; ++i) {
+      const int buf = i & 1;
+      const float ks = ks_next;
+      ks_next = ks_far;
+      ks_far = scale_of(i + 2);
+      if (ok && !mbar_wait(s_full + buf, (i >> 1) & 1)) ok = false;
+      tc_fence_after();
+      float best = -INFINITY;
+      const uint32_t taddr = tmem_base + ((uint32_t)(lg * 32) << 16) + buf * H;
+#pragma unroll
+      for (int c = 0; c < H; c += 16) {
+        uint32_t r[16];
+        tmem_ld16(taddr + c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          best = fmaxf(best, __uint_as_float(r[e]) * (qinv_s[c + e] * ks * sc) - delta_s[c + e]);
+      }
+      tc_fence_before();
+      mbar_arrive(s_free + buf);
+      const int j = k0 + i * kKeyTile + t;
+      const bool valid = j < k1;
+      if (valid) trow[j] = best;
+      const uint32_t bin = valid ? (ordered_key(best) >> kHistShift) : 0xFFFFFFFFu;
+      const unsigned grp = __match_any_sync(0xffffffffu, bin);
+      if (valid && (int)lane_id() == __ffs(grp) - 1) atomicAdd(hist_s + bin, __popc(grp));
+    }
+    named_bar_sync(1, 128);
+    uint32_t* gh = p.hist + (size_t)bq * kHistBins;
+    for (int e = t; e < kHistBins; e += 128)
+      if (hist_s[e]) atomicAdd(gh + e, hist_s[e]);
+  }
+  if (!ok) set_status(p.status, HS2_ERR_DEVICE_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+template <int H>
+static cudaError_t launch_imp_f8_t(const SelectParams& p, const CUtensorMap& tm, int bq,
+                                   cudaStream_t st) {
+  using L = ImpF8Smem<H>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(importance_fp8_kernel<H>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  return launch_pdl(importance_fp8_kernel<H>, dim3(p.splits2, bq), dim3(kImpF8Threads), L::kBytes,
+                    st, tm, p);
+}
+
+cudaError_t launch_importance_fp8(const SelectParams& p, const CUtensorMap& tmap_k, int bq,
+                                  cudaStream_t st) {
+  switch (p.h) {
+    case 16: return launch_imp_f8_t<16>(p, tmap_k, bq, st);
+    case 32: return launch_imp_f8_t<32>(p, tmap_k, bq, st);
+    case 48: return launch_imp_f8_t<48>(p, tmap_k, bq, st);
+    case 64: return launch_imp_f8_t<64>(p, tmap_k, bq, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -25,6 +25,7 @@ __global__ void __launch_bounds__(kHeadDim * kMergeMaxGroups) merge_splits_kerne
   __shared__ float Mh, invL;
   const float* pml = p.part_ml + (size_t)bq * S * H * 2;
   const float* po = p.part_o + (size_t)bq * S * H * kHeadDim;
+  griddep_wait();
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
     float M = -INFINITY;
@@ -105,11 +106,9 @@ cudaError_t launch_merge(const MergeParams& p, int bq, bool log2_domain, cudaStr
     attr_set[which] = smem;
   }
   dim3 grid(bq, p.h);
-  if (log2_domain)
-    merge_splits_kernel<true><<<grid, kHeadDim * G, smem, st>>>(p);
-  else
-    merge_splits_kernel<false><<<grid, kHeadDim * G, smem, st>>>(p);
-  return cudaGetLastError();
+  return log2_domain
+             ? launch_pdl(merge_splits_kernel<true>, grid, dim3(kHeadDim * G), smem, st, p)
+             : launch_pdl(merge_splits_kernel<false>, grid, dim3(kHeadDim * G), smem, st, p);
 }
 
 }  // namespace hs2

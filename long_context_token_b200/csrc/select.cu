@@ -39,8 +39,10 @@ template <int H, bool FP8>
 __global__ void __launch_bounds__(kThreads) importance_simt_kernel(SelectParams p) {
   extern __shared__ __align__(16) float smem[];
   SimtSmem s = carve_simt(smem, H);
+  griddep_wait();
   __shared__ uint32_t hist_s[kHistBins];
   __shared__ float delta_s[kMaxHeads];
+  griddep_wait();
   const int split = blockIdx.x, bq = blockIdx.y;
   const int b = bq / p.n_q, i = bq % p.n_q;
   const int L = seq_len(p.kv, b, p.n_q, p.status, false);
@@ -89,6 +91,7 @@ template <int H>
 __global__ void __launch_bounds__(kThreads) importance_sbuf_kernel(SelectParams p) {
   __shared__ uint32_t hist_s[kHistBins];
   __shared__ float delta_s[kMaxHeads];
+  griddep_wait();
   const int split = blockIdx.x, bq = blockIdx.y;
   const int b = bq / p.n_q, i = bq % p.n_q;
   const int L = seq_len(p.kv, b, p.n_q, p.status, false);
@@ -127,10 +130,9 @@ __global__ void __launch_bounds__(kThreads) importance_sbuf_kernel(SelectParams 
 cudaError_t launch_importance_sbuf(const SelectParams& p, int bq, cudaStream_t st) {
   const dim3 grid((p.kv.max_len + kSbufChunk - 1) / kSbufChunk, bq);
   switch (p.h) {
-    case 16: importance_sbuf_kernel<16><<<grid, kThreads, 0, st>>>(p); break;
+    case 16: return launch_pdl(importance_sbuf_kernel<16>, grid, dim3(kThreads), 0, st, p);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 // ----------------------------------------------------------------------------
@@ -217,6 +219,7 @@ __device__ __forceinline__ int warp_append(bool pred, uint32_t* counter) {
 }
 
 __global__ void __launch_bounds__(kThreads) select_compact_kernel(SelectParams p) {
+  griddep_wait();
   const int split = blockIdx.x, bq = blockIdx.y;
   const int b = bq / p.n_q, i = bq % p.n_q;
   const int L = seq_len(p.kv, b, p.n_q, p.status, false);
@@ -375,6 +378,7 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
   __shared__ uint32_t n_sel, n_band_s, gt_s;
   extern __shared__ __align__(16) uint16_t qsm[];  // [H][kQLd] bf16 q of this query
   __shared__ double dlt[H];
+  griddep_wait();
   const int bq = blockIdx.x;
   const int b = bq / p.n_q, i = bq % p.n_q;
   const int L = seq_len(p.kv, b, p.n_q, p.status, false);
@@ -564,6 +568,10 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
   }
   __syncthreads();
   for (int e = threadIdx.x; e < width; e += blockDim.x) out[e] = e < n ? sel[e] : -1;
+  // Leave this query's histogram and counters at zero for the next selection.
+  uint32_t* gh = p.hist + (size_t)bq * kHistBins;
+  for (int e = threadIdx.x; e < kHistBins; e += blockDim.x) gh[e] = 0u;
+  if (threadIdx.x < 8) p.counters[(size_t)bq * 8 + threadIdx.x] = 0u;
 }
 
 // ----------------------------------------------------------------------------
@@ -581,8 +589,8 @@ static cudaError_t launch_select_t(const SelectParams& p, int batch, cudaStream_
     attr_set = true;
   }
   const int bq = batch * p.n_q;
-  importance_simt_kernel<H, FP8><<<dim3(p.splits2, bq), kThreads, smem, st>>>(p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(importance_simt_kernel<H, FP8>, dim3(p.splits2, bq), dim3(kThreads),
+                             smem, st, p);
   if (e != cudaSuccess) return e;
   return launch_rest_t<H, FP8>(p, batch, st);
 }
@@ -590,8 +598,7 @@ static cudaError_t launch_select_t(const SelectParams& p, int batch, cudaStream_
 template <int H, bool FP8>
 static cudaError_t launch_rest_t(const SelectParams& p, int batch, cudaStream_t st) {
   const int bq = batch * p.n_q;
-  select_compact_kernel<<<dim3(p.splits3, bq), kThreads, 0, st>>>(p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(select_compact_kernel, dim3(p.splits3, bq), dim3(kThreads), 0, st, p);
   if (e != cudaSuccess) return e;
   const size_t qbytes = H * kQLd * sizeof(uint16_t);
   static bool attr_set = false;
@@ -601,8 +608,7 @@ static cudaError_t launch_rest_t(const SelectParams& p, int batch, cudaStream_t 
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  select_finish_kernel<H, FP8><<<bq, kFinThreads, qbytes, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(select_finish_kernel<H, FP8>, dim3(bq), dim3(kFinThreads), qbytes, st, p);
 }
 
 template <bool FP8>

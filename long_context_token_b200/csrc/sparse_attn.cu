@@ -30,6 +30,7 @@ __global__ void __launch_bounds__(kSpThreads) sparse_attn_kernel(SparseParams p)
   float* vs = ks + kSpRows * kSpKLd;         // [64][128]
   float* S = vs + kSpRows * kHeadDim;        // [H][64] logits, then probabilities
   int* rowidx = reinterpret_cast<int*>(S + H * kSpRows);
+  griddep_wait();
   const int tid = threadIdx.x;
   const int split = blockIdx.x, bq = blockIdx.y;
   const int b = bq / p.n_q;
@@ -188,8 +189,8 @@ static cudaError_t launch_sparse_t(const SparseParams& p, int batch, cudaStream_
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  sparse_attn_kernel<H, FP8><<<dim3(p.splits4, batch * p.n_q), kSpThreads, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(sparse_attn_kernel<H, FP8>, dim3(p.splits4, batch * p.n_q), dim3(kSpThreads),
+                    smem, st, p);
 }
 
 template <bool FP8>

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include "hs2_internal.cuh"
 #include "sm100.cuh"
@@ -33,6 +34,51 @@ __device__ __forceinline__ void store_q_kmajor(uint8_t* qs, const uint16_t* q, i
 }
 
 #ifdef __CUDACC__
+// Q [H][128] bf16 -> f16 in the same K-major layout as store_q_kmajor, each head scaled
+// by a power of two 2^e_h that puts its largest |q| in [2^14, 2^15) (f16 cannot then
+// overflow and only elements below 2^-10 of the largest lose bits).  qinv[h] = 2^-e_h;
+// c2[h] (if not null) = sm_scale * log2(e) * 2^-e_h must be filled by the caller.
+// Every thread of the block calls this; it ends with __syncthreads.
+template <int H>
+__device__ void store_q_f16_scaled(uint8_t* qs, const uint16_t* qg, float* qinv, float* up) {
+  __shared__ float up_s[kMaxHeads];
+  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5, lane = threadIdx.x & 31;
+  for (int h = warp; h < H; h += nw) {
+    float m = 0.f;
+    for (int c = lane; c < kHeadDim; c += 32)
+      m = fmaxf(m, fabsf(__uint_as_float((uint32_t)qg[h * kHeadDim + c] << 16)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) {
+      int e = 0;
+      if (m > 0.f) {
+        int ex;
+        frexpf(m, &ex);
+        e = 15 - ex;
+        e = e < -100 ? -100 : (e > 100 ? 100 : e);
+      }
+      up_s[h] = __int_as_float((127 + e) << 23);
+      qinv[h] = __int_as_float((127 - e) << 23);
+      if (up) up[h] = up_s[h];
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < H * (kHeadDim / 8); e += blockDim.x) {
+    const int h = e % H, c = e / H;
+    const uint4 v = *reinterpret_cast<const uint4*>(qg + h * kHeadDim + c * 8);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const __half lo = __float2half_rn(__uint_as_float((w[u] & 0xffffu) << 16) * up_s[h]);
+      const __half hi = __float2half_rn(__uint_as_float(w[u] & 0xffff0000u) * up_s[h]);
+      o[u] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+    }
+    *reinterpret_cast<uint4*>(qs + c * (H * 16) + h * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  __syncthreads();
+}
+
 // A operand (K tile, K-major, 128-byte swizzle written by TMA): K step kk of 16 d.
 __device__ __forceinline__ uint64_t kmajor_sw128_desc(uint32_t tile_addr, int kk) {
   const uint32_t start = tile_addr + (uint32_t)(kk >> 2) * kBoxBytes + (uint32_t)(kk & 3) * 32u;
@@ -74,5 +120,7 @@ cudaError_t launch_full_attn_fp8(const FullParams& p, const CUtensorMap& tk,
 cudaError_t launch_sparse_attn_fp8(const FullParams& p, int bq, cudaStream_t st);
 cudaError_t launch_importance_tc(const SelectParams& p, const CUtensorMap& tmap_k, int bq,
                                  cudaStream_t st);
+cudaError_t launch_importance_fp8(const SelectParams& p, const CUtensorMap& tmap_k, int bq,
+                                  cudaStream_t st);
 
 }  // namespace hs2
