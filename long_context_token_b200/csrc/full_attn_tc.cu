@@ -136,13 +136,20 @@ __global__ void __launch_bounds__(192, 1)
   const size_t row_base = (size_t)b * p.kv.max_len;
   const int n_tiles = k0 < k1 ? (k1 - k0 + kKeyTile - 1) / kKeyTile : 0;
   const size_t pidx = (size_t)bq * p.splits1 + split;
+  // Cluster mode keeps the partial in this CTA's shared memory (the K stages, idle by
+  // the time the partial is written) for the on-chip merge.
+  const bool on_chip = GATHER && p.out != nullptr;
+  float* part_o = on_chip ? reinterpret_cast<float*>(smem + kClusterOOff)
+                          : p.part_o + pidx * H * kHeadDim;
+  float* part_ml = on_chip ? reinterpret_cast<float*>(smem + kClusterMlOff)
+                           : p.part_ml + pidx * H * 2;
   bool ok = true;
 
   if (n_tiles == 0) {
     // Empty chunk: an empty partial (no key).
     for (int h = threadIdx.x; h < H; h += blockDim.x) {
-      p.part_ml[pidx * H * 2 + 2 * h] = -INFINITY;
-      p.part_ml[pidx * H * 2 + 2 * h + 1] = 0.f;
+      part_ml[2 * h] = -INFINITY;
+      part_ml[2 * h + 1] = 0.f;
     }
   } else {
     store_q_kmajor<H>(qs, p.q + (size_t)bq * H * kHeadDim, threadIdx.x, blockDim.x);
@@ -355,8 +362,10 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int h0 = c * 8 + 2 * e;
-            const float p0 = exp2f(x[h0] - mref_s[h0]);
-            const float p1 = exp2f(x[h0 + 1] - mref_s[h0 + 1]);
+            // A head whose reference is still -inf has seen no key: its p is 0 (not
+            // 2^(-inf - -inf)), so a leading all-padding tile leaves O and l at zero.
+            const float p0 = exp2f(x[h0] - finite_ref(mref_s[h0]));
+            const float p1 = exp2f(x[h0 + 1] - finite_ref(mref_s[h0 + 1]));
             l[h0] += p0;
             l[h0 + 1] += p1;
             const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
@@ -391,14 +400,13 @@ __global__ void __launch_bounds__(192, 1)
       const int last = n_tiles - 1;
       if (ok && !mbar_wait(p_free + (last & 1), (last >> 1) & 1)) ok = false;
       tc_fence_after();
-      float* po = p.part_o + pidx * H * kHeadDim;
 #pragma unroll
       for (int c = 0; c < H; c += 16) {
         uint32_t r[16];
         tmem_ld16(tmem_o + lane_base + c, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) po[(c + e) * kHeadDim + t] = __uint_as_float(r[e]);
+        for (int e = 0; e < 16; ++e) part_o[(c + e) * kHeadDim + t] = __uint_as_float(r[e]);
       }
       tc_fence_before();
 #pragma unroll
@@ -408,12 +416,21 @@ __global__ void __launch_bounds__(192, 1)
       }
       named_bar_sync(1, 128);
       if (t < H) {
-        p.part_ml[pidx * H * 2 + 2 * t] = mref_s[t];
-        p.part_ml[pidx * H * 2 + 2 * t + 1] = red[t] + red[H + t] + red[2 * H + t] + red[3 * H + t];
+        part_ml[2 * t] = mref_s[t];
+        part_ml[2 * t + 1] = red[t] + red[H + t] + red[2 * H + t] + red[3 * H + t];
       }
     }
   }
   if (!ok) set_status(p.status, HS2_ERR_DEVICE_TIMEOUT);
+  if (on_chip) {
+    // Every CTA of the cluster reaches both barriers (no early exit above); the second
+    // keeps each CTA's shared memory alive until the others have read it.
+    __syncwarp();
+    cluster_sync();
+    cluster_merge_row<H>(smem, p.splits1, p.out + (size_t)bq * H * kHeadDim);
+    __syncwarp();
+    cluster_sync();
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -423,18 +440,22 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 template <int H, bool GATHER>
-static cudaError_t launch_full_tc_t(const FullParams& p, const CUtensorMap& tk,
-                                    const CUtensorMap& tv, int bq, cudaStream_t st) {
+static cudaError_t launch_full_tc_t(FullParams p, const CUtensorMap& tk, const CUtensorMap& tv,
+                                    int bq, cudaStream_t st) {
   using L = FullSmem<H>;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(full_attn_tc_kernel<H, GATHER>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+  auto kernel = full_attn_tc_kernel<H, GATHER>;
+  static int max_cluster = 0;
+  if (!max_cluster) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e != cudaSuccess) return e;
-    attr = true;
+    max_cluster = GATHER ? largest_cluster(kernel, dim3(192), L::kBytes) : 1;
+    if (max_cluster < 1) return cudaErrorLaunchOutOfResources;
   }
-  return launch_pdl(full_attn_tc_kernel<H, GATHER>, dim3(p.splits1, bq), dim3(192), L::kBytes, st,
-                    tk, tv, p);
+  if (!GATHER) return launch_pdl(kernel, dim3(p.splits1, bq), dim3(192), L::kBytes, st, tk, tv, p);
+  plan_gather_cluster(p.idx_width, max_cluster, &p.splits1, &p.chunk1);
+  return launch_pdl_cluster(kernel, dim3(p.splits1, bq), dim3(192), L::kBytes, p.splits1, st, tk,
+                            tv, p);
 }
 
 template <bool GATHER>
@@ -454,7 +475,7 @@ cudaError_t launch_full_attn_tc(const FullParams& p, const CUtensorMap& tk, cons
   return launch_full_tc_h<false>(p, tk, tv, bq, st);
 }
 
-cudaError_t launch_sparse_attn_tc(const FullParams& p, int bq, cudaStream_t st) {
+cudaError_t launch_sparse_attn_tc(FullParams p, int bq, cudaStream_t st) {
   CUtensorMap unused;
   memset(&unused, 0, sizeof(unused));
   return launch_full_tc_h<true>(p, unused, unused, bq, st);

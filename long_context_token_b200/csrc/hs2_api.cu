@@ -22,7 +22,6 @@ static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // that the workspace layout does not depend on the device it runs on.
 constexpr int kTargetCtas = 4 * 148;
 constexpr int kMinChunk = 256;
-constexpr int kChunk3 = 8192;
 constexpr int kChunk4 = 64;
 
 int plan_splits1(int bq, int max_len, int /*num_sms*/) {
@@ -232,8 +231,8 @@ static hs2_status run_select(const void* q, int n_q, int h, const hs2_kv* kv, in
   p.sm_scale = sm_scale;
   p.splits2 = w.splits1;
   p.chunk2 = chunk_for(kv->max_len, w.splits1);
-  p.chunk3 = kChunk3;
-  p.splits3 = (kv->max_len + kChunk3 - 1) / kChunk3;
+  p.chunk3 = kChunk3Keys;
+  p.splits3 = (kv->max_len + kChunk3Keys - 1) / kChunk3Keys;
   p.lse64 = ws_ptr<double>(ws, w.lse64);
   p.sbuf = w.use_sbuf ? ws_ptr<float>(ws, w.sbuf) : nullptr;
   p.tbuf = ws_ptr<float>(ws, w.tbuf);
@@ -356,7 +355,8 @@ hs2_status hs2_sparse_attn(const void* q_layer, int n_q, int h_q, const hs2_kv* 
   make_layout(kv->batch, n_q, h_q, kv->max_len, 1, 1, kv->dtype, &w);
   if (ws_bytes < sparse_prefix_bytes(w)) return HS2_ERR_WORKSPACE_TOO_SMALL;
   if (h_q <= 64) {
-    // Tensor-core gather attention: 128 index entries per CTA, log2-domain partials.
+    // Tensor-core gather attention: the row's 128-entry tiles spread over one
+    // thread-block cluster, whose CTAs merge their partials on chip and write `out`.
     FullParams f;
     f.q = static_cast<const uint16_t*>(q_layer);
     f.kv = view_of(kv);
@@ -365,27 +365,18 @@ hs2_status hs2_sparse_attn(const void* q_layer, int n_q, int h_q, const hs2_kv* 
     f.window = 0;
     f.k_sel = 0;
     f.sm_scale = sm_scale;
-    f.chunk1 = 128;
-    f.splits1 = (idx_width + 127) / 128;
-    f.part_o = ws_ptr<float>(workspace, w.part4_o);
-    f.part_ml = ws_ptr<float>(workspace, w.part4_ml);
+    f.chunk1 = 0;   // planned by the launcher
+    f.splits1 = 0;
+    f.part_o = nullptr;
+    f.part_ml = nullptr;
     f.status = ws_ptr<uint32_t>(workspace, w.status);
     f.idx = idx;
     f.idx_width = idx_width;
+    f.out = out;
     cudaError_t e = kv->dtype == HS2_KV_FP8_E4M3
                         ? launch_sparse_attn_fp8(f, kv->batch * n_q, (cudaStream_t)stream)
                         : launch_sparse_attn_tc(f, kv->batch * n_q, (cudaStream_t)stream);
-    if (e != cudaSuccess) return cuda_fail(e, "sparse-attention launch");
-    MergeParams m;
-    m.part_o = f.part_o;
-    m.part_ml = f.part_ml;
-    m.splits = f.splits1;
-    m.h = h_q;
-    m.out = out;
-    m.lse_out = nullptr;
-    m.lse64 = nullptr;
-    e = launch_merge(m, kv->batch * n_q, true, (cudaStream_t)stream);
-    return e == cudaSuccess ? HS2_OK : cuda_fail(e, "sparse-attention merge launch");
+    return e == cudaSuccess ? HS2_OK : cuda_fail(e, "sparse-attention launch");
   }
   SparseParams p;
   p.q = static_cast<const uint16_t*>(q_layer);

@@ -12,6 +12,7 @@ namespace hs2 {
 constexpr int kHeadDim = 128;
 constexpr int kHistBins = 4096;         // first-level radix histogram: top 12 bits
 constexpr int kHistShift = 20;
+constexpr int kChunk3Keys = 8192;      // keys per CTA of the compaction pass
 constexpr int kMaxIdxWidth = 4096;      // window + k_sel
 constexpr int kMaxNq = 64;
 constexpr int kMaxHeads = 128;
@@ -85,6 +86,10 @@ struct FullParams {
   const int32_t* idx = nullptr;  // gather mode (a sparse layer): [bq][idx_width] positions
   int idx_width = 0;
   float* sbuf = nullptr;          // if set: raw float32 logits of the keys outside the window
+  // Gather mode only: if set, the splits1 CTAs of one row form a thread-block cluster,
+  // merge their partials through distributed shared memory and write the normalised
+  // output [bq][h][128] here (part_o / part_ml are then unused).
+  float* out = nullptr;
 };
 
 // Split merge (full layer: log2-domain partials; sparse layers: natural-log ones).
@@ -147,6 +152,29 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
+// The same, with the grid's x dimension grouped into thread-block clusters of
+// `cluster_x` CTAs (grid.x must be a multiple of it).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                                      size_t smem, int cluster_x, cudaStream_t st,
+                                      Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
 }
 

@@ -5,8 +5,9 @@
 //   lse_h = M_h + ln L_h
 // (base 2 instead of e when the partials were produced in the log2 domain).
 //
-// Grid (bq, h): one CTA per (sequence/token, head), 128 x G threads.  Warp 0 reduces
-// M and L over the splits (float64 sum) and stages the weights in shared memory;
+// Grid (bq, h): one CTA per (sequence/token, head), 128 x G threads.  Warp 0 loads the
+// (m, l) pairs once, reduces M and L over the splits (float64 sum) and stages the
+// weights in shared memory;
 // thread (g, d) then sums dimension d over the splits s = g, g + G, ... with eight
 // independent loads in flight, and the G partial sums are added in shared memory.
 #include "hs2_internal.cuh"
@@ -17,25 +18,31 @@ constexpr int kMergeMaxGroups = 8;
 
 template <bool LOG2>
 __global__ void __launch_bounds__(kHeadDim * kMergeMaxGroups) merge_splits_kernel(MergeParams p) {
-  extern __shared__ float w[];  // [splits] weights, then [G][128] partial sums
+  extern __shared__ float w[];  // [splits] weights, [G][128] partial sums, [splits][2] (m, l)
   const int bq = blockIdx.x, h = blockIdx.y;
   const int H = p.h, S = p.splits;
   const int G = blockDim.x / kHeadDim;
   float* acc_s = w + ((S + 3) & ~3);
-  __shared__ float Mh, invL;
+  float* ml_s = acc_s + G * kHeadDim;
   const float* pml = p.part_ml + (size_t)bq * S * H * 2;
   const float* po = p.part_o + (size_t)bq * S * H * kHeadDim;
   griddep_wait();
   if (threadIdx.x < 32) {
+    // One pass over the (m, l) pairs (a single memory round trip), kept in shared memory.
     const int lane = threadIdx.x;
     float M = -INFINITY;
-    for (int s = lane; s < S; s += 32) M = fmaxf(M, __ldcg(pml + ((size_t)s * H + h) * 2));
+#pragma unroll 4
+    for (int s = lane; s < S; s += 32) {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(pml + ((size_t)s * H + h) * 2));
+      ml_s[2 * s] = v.x;
+      ml_s[2 * s + 1] = v.y;
+      if (v.y > 0.f) M = fmaxf(M, v.x);
+    }
     M = warp_max(M);
     double Ls = 0.0;
     if (M != -INFINITY) {
       for (int s = lane; s < S; s += 32) {
-        const float m = __ldcg(pml + ((size_t)s * H + h) * 2);
-        const float l = __ldcg(pml + ((size_t)s * H + h) * 2 + 1);
+        const float m = ml_s[2 * s], l = ml_s[2 * s + 1];
         if (l > 0.f) Ls += (double)l * (LOG2 ? exp2((double)m - M) : exp((double)m - M));
       }
     }
@@ -43,16 +50,11 @@ __global__ void __launch_bounds__(kHeadDim * kMergeMaxGroups) merge_splits_kerne
     const float il = Ls > 0.0 ? (float)(1.0 / Ls) : 0.f;
     for (int s = lane; s < S; s += 32) {
       float wt = 0.f;
-      if (M != -INFINITY) {
-        const float m = __ldcg(pml + ((size_t)s * H + h) * 2);
-        const float l = __ldcg(pml + ((size_t)s * H + h) * 2 + 1);
-        if (l > 0.f) wt = (LOG2 ? exp2f(m - M) : expf(m - M)) * il;
-      }
+      const float m = ml_s[2 * s], l = ml_s[2 * s + 1];
+      if (M != -INFINITY && l > 0.f) wt = (LOG2 ? exp2f(m - M) : expf(m - M)) * il;
       w[s] = wt;
     }
     if (lane == 0) {
-      Mh = M;
-      invL = il;
       double lse = -INFINITY;
       if (Ls > 0.0) lse = LOG2 ? ((double)M + log2(Ls)) * 0.69314718055994530942 : M + log(Ls);
       if (p.lse64) p.lse64[(size_t)bq * H + h] = lse;
@@ -92,7 +94,8 @@ cudaError_t launch_merge(const MergeParams& p, int bq, bool log2_domain, cudaStr
   int G = (p.splits + 15) / 16;
   if (G > kMergeMaxGroups) G = kMergeMaxGroups;
   if (G < 1) G = 1;
-  const size_t smem = (((size_t)p.splits + 3) / 4 * 4 + (size_t)G * kHeadDim) * sizeof(float);
+  const size_t smem =
+      (((size_t)p.splits + 3) / 4 * 4 + (size_t)G * kHeadDim + 2 * (size_t)p.splits) * sizeof(float);
   if (smem > 200 * 1024) return cudaErrorInvalidValue;
   static size_t attr_set[2] = {0, 0};
   const int which = log2_domain ? 1 : 0;

@@ -104,22 +104,40 @@ __global__ void __launch_bounds__(kThreads) importance_sbuf_kernel(SelectParams 
   for (int e = threadIdx.x; e < kHistBins; e += kThreads) hist_s[e] = 0u;
   load_delta(p.lse64 + (size_t)bq * H, H, delta_s, nullptr);
   const uint64_t pol = sm100_evict_first_policy();
-  const float* src = p.sbuf + (size_t)bq * p.kv.max_len * H;
-  float* trow = p.tbuf + (size_t)bq * p.kv.max_len;
+  const float* __restrict__ src = p.sbuf + (size_t)bq * p.kv.max_len * H;
+  float* __restrict__ trow = p.tbuf + (size_t)bq * p.kv.max_len;
   const float sc = p.sm_scale;
-#pragma unroll 4
-  for (int j = k0 + threadIdx.x; j < k1; j += kThreads) {
-    float t = -INFINITY;
+  // Keys are loaded kBatch at a time, all before the first is used (kBatch x H
+  // floats in flight per thread): one memory round trip per kBatch keys.
+  constexpr int kPer = kSbufChunk / kThreads;
+  static_assert(kPer * kThreads == kSbufChunk, "chunk is a multiple of the block");
+  constexpr int kBatch = 4;
+#pragma unroll 1
+  for (int u0 = 0; u0 < kPer; u0 += kBatch) {
+    uint4 v[kBatch][H / 4];
 #pragma unroll
-    for (int c = 0; c < H; c += 4) {
-      const uint4 v = sm100_ld_v4_hint(src + (size_t)j * H + c, pol);
-      t = fmaxf(t, __uint_as_float(v.x) * sc - delta_s[c]);
-      t = fmaxf(t, __uint_as_float(v.y) * sc - delta_s[c + 1]);
-      t = fmaxf(t, __uint_as_float(v.z) * sc - delta_s[c + 2]);
-      t = fmaxf(t, __uint_as_float(v.w) * sc - delta_s[c + 3]);
+    for (int u = 0; u < kBatch; ++u) {
+      const int j = k0 + (u0 + u) * kThreads + threadIdx.x;
+#pragma unroll
+      for (int c = 0; c < H / 4; ++c)
+        v[u][c] = j < k1 ? sm100_ld_v4_hint(src + (size_t)j * H + 4 * c, pol)
+                         : make_uint4(0, 0, 0, 0);
     }
-    trow[j] = t;
-    atomicAdd(&hist_s[ordered_key(t) >> kHistShift], 1u);
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int j = k0 + (u0 + u) * kThreads + threadIdx.x;
+      if (j >= k1) continue;
+      float t = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < H / 4; ++c) {
+        t = fmaxf(t, __uint_as_float(v[u][c].x) * sc - delta_s[4 * c]);
+        t = fmaxf(t, __uint_as_float(v[u][c].y) * sc - delta_s[4 * c + 1]);
+        t = fmaxf(t, __uint_as_float(v[u][c].z) * sc - delta_s[4 * c + 2]);
+        t = fmaxf(t, __uint_as_float(v[u][c].w) * sc - delta_s[4 * c + 3]);
+      }
+      trow[j] = t;
+      atomicAdd(&hist_s[ordered_key(t) >> kHistShift], 1u);
+    }
   }
   __syncthreads();
   uint32_t* gh = p.hist + (size_t)bq * kHistBins;
@@ -206,19 +224,37 @@ __device__ BoundaryBin find_boundary_bin(const uint32_t* gh, int k_eff, float de
   return r;
 }
 
-// Warp-aggregated append of `pred` lanes to a list; returns the slot or -1.
-__device__ __forceinline__ int warp_append(bool pred, uint32_t* counter) {
-  const unsigned m = __ballot_sync(0xffffffffu, pred);
-  if (!m) return -1;
-  const int lane = threadIdx.x & 31;
-  const int leader = __ffs(m) - 1;
-  uint32_t base = 0;
-  if (lane == leader) base = atomicAdd(counter, (uint32_t)__popc(m));
-  base = __shfl_sync(0xffffffffu, base, leader);
-  return pred ? (int)(base + __popc(m & ((1u << lane) - 1u))) : -1;
+// Exclusive prefix sum over the block of one value per thread; *total gets the sum.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* total) {
+  __shared__ uint32_t warp_tot[kThreads / 32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  if (lane == 31) warp_tot[w] = incl;
+  __syncthreads();
+  uint32_t before = 0, all = 0;
+#pragma unroll
+  for (int k = 0; k < kThreads / 32; ++k) {
+    const uint32_t c = warp_tot[k];
+    before += k < w ? c : 0u;
+    all += c;
+  }
+  __syncthreads();  // warp_tot may be reused by the next call
+  *total = all;
+  return before + incl - v;
 }
 
+// Each CTA takes kChunk3Keys keys of one query: kPer consecutive keys per thread,
+// loaded (with the histogram) before the boundary bin is known.  Keys are sorted into
+// the direct list (clearly above the boundary bin) and the candidate list (inside it,
+// with the margin); the CTA counts both, reserves its ranges with one atomic per list
+// and writes them, so no key waits on a global atomic.
 __global__ void __launch_bounds__(kThreads) select_compact_kernel(SelectParams p) {
+  constexpr int kPer = kChunk3Keys / kThreads;
   griddep_wait();
   const int split = blockIdx.x, bq = blockIdx.y;
   const int b = bq / p.n_q, i = bq % p.n_q;
@@ -226,16 +262,40 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(SelectParams p
   const int pos = L - p.n_q + i;
   const int n_c = pos - p.window + 1;
   if (n_c <= p.k_sel) return;
+  const int k0 = split * kChunk3Keys;
+  const int k1 = min(k0 + kChunk3Keys, n_c);
+  if (k0 >= k1) return;
   const int k_eff = p.k_sel;
+  const float* __restrict__ trow = p.tbuf + (size_t)bq * p.kv.max_len;
+  const int j0 = k0 + threadIdx.x * kPer;
+  float t[kPer];
+  if (j0 + kPer <= k1 && (reinterpret_cast<uintptr_t>(trow + j0) & 15u) == 0) {
+#pragma unroll
+    for (int u = 0; u < kPer / 4; ++u) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(trow + j0) + u);
+      t[4 * u] = v.x;
+      t[4 * u + 1] = v.y;
+      t[4 * u + 2] = v.z;
+      t[4 * u + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) t[u] = j0 + u < k1 ? __ldcg(trow + j0 + u) : -INFINITY;
+  }
   __shared__ float dmax_s;
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < 32) {
     double lo = INFINITY, hi = -INFINITY;
-    for (int h = 0; h < p.h; ++h) {
-      const double l = p.lse64[(size_t)bq * p.h + h];
+    for (int h = threadIdx.x; h < p.h; h += 32) {
+      const double l = __ldcg(p.lse64 + (size_t)bq * p.h + h);
       lo = fmin(lo, l);
       hi = fmax(hi, l);
     }
-    dmax_s = (float)(hi - lo);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lo = fmin(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = fmax(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if (threadIdx.x == 0) dmax_s = (float)(hi - lo);
   }
   __syncthreads();
   const BoundaryBin bb = find_boundary_bin(p.hist + (size_t)bq * kHistBins, k_eff, dmax_s);
@@ -247,45 +307,38 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(SelectParams p
     meta[3] = (uint32_t)n_c;
   }
   const float hi_e = bb.hi + bb.eps, lo_e = bb.lo - bb.eps;
-  const int k0 = split * p.chunk3;
-  const int k1 = min(k0 + p.chunk3, n_c);
-  const float* trow = p.tbuf + (size_t)bq * p.kv.max_len;
+  uint32_t nd = 0, nc = 0;
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    nd += t[u] > hi_e;
+    nc += t[u] <= hi_e && t[u] >= lo_e;
+  }
+  uint32_t tot_d, tot_c;
+  uint32_t od = block_excl_scan(nd, &tot_d);
+  uint32_t oc = block_excl_scan(nc, &tot_c);
+  __shared__ uint32_t base_d, base_c;
   uint32_t* cnt = p.counters + (size_t)bq * 8;
+  if (threadIdx.x == 0) {
+    base_d = tot_d ? atomicAdd(cnt + 0, tot_d) : 0u;
+    base_c = tot_c ? atomicAdd(cnt + 1, tot_c) : 0u;
+  }
+  __syncthreads();
+  od += base_d;
+  oc += base_c;
   int32_t* direct = p.direct + (size_t)bq * p.k_sel;
   float* ct = p.cand_t + (size_t)bq * p.kv.max_len;
   int32_t* cj = p.cand_j + (size_t)bq * p.kv.max_len;
-  // Each thread takes 16 consecutive keys per round, loaded up front (four 16-byte
-  // loads in flight); the trip count is uniform so every lane joins the ballots.
-  constexpr int kPer = 16;
-  for (int base = k0; base < k1; base += kThreads * kPer) {
-    const int j0 = base + threadIdx.x * kPer;
-    float t[kPer];
-    if (j0 + kPer <= k1 && ((j0 & 3) == 0)) {
 #pragma unroll
-      for (int u = 0; u < kPer / 4; ++u) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(trow + j0) + u);
-        t[4 * u] = v.x;
-        t[4 * u + 1] = v.y;
-        t[4 * u + 2] = v.z;
-        t[4 * u + 3] = v.w;
+  for (int u = 0; u < kPer; ++u) {
+    if (t[u] > hi_e) {
+      if (od < (uint32_t)p.k_sel) direct[od] = j0 + u;
+      ++od;
+    } else if (t[u] >= lo_e) {
+      if (oc < (uint32_t)p.kv.max_len) {
+        ct[oc] = t[u];
+        cj[oc] = j0 + u;
       }
-    } else {
-#pragma unroll
-      for (int u = 0; u < kPer; ++u) t[u] = j0 + u < k1 ? __ldcg(trow + j0 + u) : -INFINITY;
-    }
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int j = j0 + u;
-      const bool in = j < k1;
-      const bool is_direct = in && t[u] > hi_e;
-      const bool is_cand = in && !is_direct && t[u] >= lo_e;
-      const int sd = warp_append(is_direct, cnt + 0);
-      if (sd >= 0 && sd < p.k_sel) direct[sd] = j;
-      const int sc = warp_append(is_cand, cnt + 1);
-      if (sc >= 0 && sc < p.kv.max_len) {
-        ct[sc] = t[u];
-        cj[sc] = j;
-      }
+      ++oc;
     }
   }
 }
@@ -294,11 +347,30 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(SelectParams p
 // 3. finish: exact select + float64 refinement + window merge + sort
 // ----------------------------------------------------------------------------
 constexpr int kFinThreads = 1024;
-constexpr int kSmallBand = 1024;  // bands up to this size are ranked pairwise
+constexpr int kSmallBand = 1024;  // bands up to this size are ranked pairwise in shared memory
 constexpr int kBuckets = 1024;    // counting-sort buckets of the final index set
 constexpr int kQLd = kHeadDim + 8;  // padded q row (bf16) in shared memory
+constexpr int kCandSmem = 4096;   // candidate lists up to this size are staged in shared memory
 static_assert(kSmallBand * (sizeof(double) + sizeof(int)) <= kMaxIdxWidth * sizeof(int),
               "band pairs must fit the scratch area");
+
+__host__ __device__ constexpr size_t finish_dyn_smem(int H) {
+  return (size_t)H * kQLd * sizeof(uint16_t) + (size_t)kCandSmem * (sizeof(float) + sizeof(int));
+}
+
+// Warp-aggregated append to a shared-memory counter: one atomic per warp; returns the
+// lane's slot (only meaningful where pred holds).
+__device__ __forceinline__ uint32_t warp_slot(bool pred, uint32_t* counter) {
+  const unsigned m = __ballot_sync(0xffffffffu, pred);
+  const int lane = threadIdx.x & 31;
+  uint32_t base = 0;
+  if (m) {
+    const int leader = __ffs(m) - 1;
+    if (lane == leader) base = atomicAdd(counter, (uint32_t)__popc(m));
+    base = __shfl_sync(0xffffffffu, base, leader);
+  }
+  return base + __popc(m & ((1u << lane) - 1u));
+}
 
 // Radix select over the elements e in [0, n) with pred(e): the r-th largest
 // (1-based) of key(e), a KeyT of KBITS bits, 8 bits per pass.  Returns the key;
@@ -376,7 +448,10 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
   int* tmp = reinterpret_cast<int*>(scratch);                              // [kMaxIdxWidth]
   __shared__ uint32_t bucket[kBuckets], bucket_beg[kBuckets];
   __shared__ uint32_t n_sel, n_band_s, gt_s;
-  extern __shared__ __align__(16) uint16_t qsm[];  // [H][kQLd] bf16 q of this query
+  extern __shared__ __align__(16) unsigned char fin_dyn[];
+  uint16_t* qsm = reinterpret_cast<uint16_t*>(fin_dyn);  // [H][kQLd] bf16 q of this query
+  float* cts = reinterpret_cast<float*>(fin_dyn + (size_t)H * kQLd * sizeof(uint16_t));
+  int* cjs = reinterpret_cast<int*>(cts + kCandSmem);
   __shared__ double dlt[H];
   griddep_wait();
   const int bq = blockIdx.x;
@@ -390,67 +465,91 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
     for (int e = threadIdx.x; e < width; e += blockDim.x) out[e] = e <= pos ? e : -1;
     return;
   }
+  // Loads that depend on nothing but the previous pass, issued together: the counts,
+  // the margin, this query's q and the per-head shifts.
   const uint32_t* cnt = p.counters + (size_t)bq * 8;
   const uint32_t n_direct = min(__ldcg(cnt + 0), (uint32_t)p.k_sel);
   const uint32_t n_cand = min(__ldcg(cnt + 1), (uint32_t)p.kv.max_len);
   const float eps = __uint_as_float(__ldcg(p.selmeta + (size_t)bq * 4 + 1));
-  const int need = p.k_sel - (int)n_direct;  // >= 1 by construction
-  const float* ct = p.cand_t + (size_t)bq * p.kv.max_len;
-  const int32_t* cj = p.cand_j + (size_t)bq * p.kv.max_len;
-  if (threadIdx.x == 0) {
-    n_sel = 0;
-    n_band_s = 0;
-  }
-  __syncthreads();
-
-  // tau: the need-th largest float32 key among the candidates.
-  const uint32_t tau_key = block_kth_largest<uint32_t, 32>(
-      (int)n_cand, need, [&](int e) { return ordered_key(__ldcg(ct + e)); },
-      [](int) { return true; }, &gt_s);
-  const float tau = key_to_float(tau_key);
-  const float hi_b = tau + eps, lo_b = tau - eps;
-
-  // Kept outright: the direct list and candidates above the band.  Band -> refine.
-  auto push = [&](int j) {
-    const uint32_t slot = atomicAdd(&n_sel, 1u);
-    if (slot < (uint32_t)kMaxIdxWidth) sel[slot] = j;
-  };
-  for (uint32_t e = threadIdx.x; e < n_direct; e += blockDim.x)
-    push(__ldcg(p.direct + (size_t)bq * p.k_sel + e));
-  int32_t* bj = p.band_j + (size_t)bq * p.kv.max_len;
-  double* bt = p.band_t + (size_t)bq * p.kv.max_len;
-  for (uint32_t e = threadIdx.x; e < n_cand; e += blockDim.x) {
-    const float t = __ldcg(ct + e);
-    if (t > hi_b) push(__ldcg(cj + e));
-    else if (t >= lo_b) bj[atomicAdd(&n_band_s, 1u)] = __ldcg(cj + e);
-  }
-  __syncthreads();
-  load_delta(p.lse64 + (size_t)bq * H, H, nullptr, dlt);
   for (int e = threadIdx.x; e < H * (kHeadDim / 8); e += blockDim.x) {
     const int h = e / (kHeadDim / 8), c = (e % (kHeadDim / 8)) * 8;
     *reinterpret_cast<uint4*>(qsm + h * kQLd + c) =
         *reinterpret_cast<const uint4*>(p.q + ((size_t)bq * H + h) * kHeadDim + c);
   }
+  load_delta(p.lse64 + (size_t)bq * H, H, nullptr, dlt);  // (synchronises the block)
+  const int need = p.k_sel - (int)n_direct;  // >= 1 by construction
+  const float* ct = p.cand_t + (size_t)bq * p.kv.max_len;
+  const int32_t* cj = p.cand_j + (size_t)bq * p.kv.max_len;
+  // The direct list goes to the front of the selection; the candidates are staged in
+  // shared memory when they fit.
+  const bool cand_smem = n_cand <= (uint32_t)kCandSmem;
+  for (uint32_t e = threadIdx.x; e < n_direct; e += blockDim.x)
+    sel[e] = __ldcg(p.direct + (size_t)bq * p.k_sel + e);
+  if (cand_smem)
+    for (uint32_t e = threadIdx.x; e < n_cand; e += blockDim.x) {
+      cts[e] = __ldcg(ct + e);
+      cjs[e] = __ldcg(cj + e);
+    }
+  if (threadIdx.x == 0) {
+    n_sel = n_direct;
+    n_band_s = 0;
+  }
+  __syncthreads();
+  auto cand_t = [&](uint32_t e) { return cand_smem ? cts[e] : __ldcg(ct + e); };
+  auto cand_j = [&](uint32_t e) { return cand_smem ? cjs[e] : __ldcg(cj + e); };
+
+  // tau: the need-th largest float32 key among the candidates.
+  const uint32_t tau_key = block_kth_largest<uint32_t, 32>(
+      (int)n_cand, need, [&](int e) { return ordered_key(cand_t((uint32_t)e)); },
+      [](int) { return true; }, &gt_s);
+  const float tau = key_to_float(tau_key);
+  const float hi_b = tau + eps, lo_b = tau - eps;
+
+  // Candidates above the band are kept; band keys are listed for re-scoring (in shared
+  // memory while the band is small, else in the workspace).
+  int32_t* bj = p.band_j + (size_t)bq * p.kv.max_len;
+  double* bt = p.band_t + (size_t)bq * p.kv.max_len;
+  const uint32_t n_cand_r = (n_cand + 31u) & ~31u;  // whole warps take part in the ballots
+  for (uint32_t e = threadIdx.x; e < n_cand_r; e += blockDim.x) {
+    const bool in = e < n_cand;
+    const float t = in ? cand_t(e) : -INFINITY;
+    const int j = in ? cand_j(e) : -1;
+    const bool keep = in && t > hi_b;
+    const bool band = in && !keep && t >= lo_b;
+    const uint32_t sk = warp_slot(keep, &n_sel);
+    if (keep && sk < (uint32_t)kMaxIdxWidth) sel[sk] = j;
+    const uint32_t sb = warp_slot(band, &n_band_s);
+    if (band) {
+      bj[sb] = j;
+      if (sb < (uint32_t)kSmallBand) band_js[sb] = j;
+    }
+  }
   __syncthreads();
   const int n_band = (int)n_band_s;
   const int need2 = p.k_sel - (int)n_sel;  // taken from the band
+  const bool band_smem = n_band <= kSmallBand;
 
   if (need2 > 0) {
-    // float64 re-scoring of the band: one warp per key, lane l takes heads l, l+32, ...
-    // (q from shared memory, the key's row through L1: every lane reads the same row).
+    // float64 re-scoring of the band: one warp per key; for H < 32 the lanes split each
+    // head's dot product into 32 / H parts (lane = part * H + head).
+    constexpr int kParts = H < 32 ? 32 / H : 1;
+    constexpr int kSpan = kHeadDim / kParts;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int part = kParts > 1 ? lane / H : 0;
     const double scale = (double)p.sm_scale;
     for (int e = warp; e < n_band; e += blockDim.x / 32) {
-      const int j = bj[e];
+      const int j = band_smem ? band_js[e] : __ldcg(bj + e);
       const size_t row = (size_t)b * p.kv.max_len + j;
       double best = -INFINITY;
-      for (int h = lane; h < H; h += 32) {
+      for (int h0 = 0; h0 < H; h0 += 32 / kParts) {
+        const int h = h0 + (kParts > 1 ? lane % H : lane);
+        if (h >= H) continue;
         const uint16_t* qh = qsm + h * kQLd;
         double dot = 0.0;
         if (FP8) {
           const uint8_t* kr = static_cast<const uint8_t*>(p.kv.k) + row * kHeadDim;
 #pragma unroll 2
-          for (int c = 0; c < kHeadDim; c += 16) {
+          for (int c = part * kSpan; c < (part + 1) * kSpan; c += 16) {
             const uint4 kv = __ldg(reinterpret_cast<const uint4*>(kr + c));
             const uint4 qa = *reinterpret_cast<const uint4*>(qh + c);
             const uint4 qb = *reinterpret_cast<const uint4*>(qh + c + 8);
@@ -463,11 +562,10 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
               dot = fma((double)bf16_bits_to_f32(qbits), e4m3_to_f64(code), dot);
             }
           }
-          dot *= (double)p.kv.k_scale[row];
         } else {
           const uint16_t* kr = static_cast<const uint16_t*>(p.kv.k) + row * kHeadDim;
 #pragma unroll 2
-          for (int c = 0; c < kHeadDim; c += 8) {
+          for (int c = part * kSpan; c < (part + 1) * kSpan; c += 8) {
             const uint4 kv = __ldg(reinterpret_cast<const uint4*>(kr + c));
             const uint4 qv = *reinterpret_cast<const uint4*>(qh + c);
             const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
@@ -481,21 +579,22 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
             }
           }
         }
+#pragma unroll
+        for (int o = 16; o >= 32 / kParts && kParts > 1; o >>= 1)
+          dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        if (FP8) dot *= (double)p.kv.k_scale[row];
         best = fmax(best, scale * dot - dlt[h]);
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) best = fmax(best, __shfl_xor_sync(0xffffffffu, best, o));
-      if (lane == 0) bt[e] = best;
-    }
-    __threadfence_block();
-    __syncthreads();
-    if (n_band <= kSmallBand) {
-      // Small band: rank every key by (t desc, position asc) against all the others.
-      for (int e = threadIdx.x; e < n_band; e += blockDim.x) {
-        band_ts[e] = bt[e];
-        band_js[e] = bj[e];
+      if (lane == 0) {
+        if (band_smem) band_ts[e] = best;
+        else bt[e] = best;
       }
-      __syncthreads();
+    }
+    __syncthreads();
+    if (band_smem) {
+      // Small band: rank every key by (t desc, position asc) against all the others.
       for (int e = threadIdx.x; e < n_band; e += blockDim.x) {
         const double te = band_ts[e];
         const int je = band_js[e];
@@ -504,31 +603,43 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
           const double tf = band_ts[f];
           rank += (tf > te) || (tf == te && band_js[f] < je);
         }
-        if (rank < need2) push(je);
+        if (rank < need2) {
+          const uint32_t slot = atomicAdd(&n_sel, 1u);
+          if (slot < (uint32_t)kMaxIdxWidth) sel[slot] = je;
+        }
       }
     } else {
-    // Boundary value among the band, then the lowest positions among its ties.
-    const unsigned long long vb = block_kth_largest<unsigned long long, 64>(
-        n_band, need2, [&](int e) { return ordered_key64(bt[e]); }, [](int) { return true; },
-        &gt_s);
-    const uint32_t n_gt = gt_s;
-    const int take_eq = need2 - (int)n_gt;
-    const uint32_t jb_inv = block_kth_largest<uint32_t, 32>(
-        n_band, take_eq, [&](int e) { return ~(uint32_t)bj[e]; },
-        [&](int e) { return ordered_key64(bt[e]) == vb; }, &gt_s);
-    const int jb = (int)~jb_inv;
-    for (int e = threadIdx.x; e < n_band; e += blockDim.x) {
-      const unsigned long long kk = ordered_key64(bt[e]);
-      if (kk > vb || (kk == vb && bj[e] <= jb)) push(bj[e]);
-    }
+      // Boundary value among the band, then the lowest positions among its ties.
+      const unsigned long long vb = block_kth_largest<unsigned long long, 64>(
+          n_band, need2, [&](int e) { return ordered_key64(__ldcg(bt + e)); },
+          [](int) { return true; }, &gt_s);
+      const uint32_t n_gt = gt_s;
+      const int take_eq = need2 - (int)n_gt;
+      const uint32_t jb_inv = block_kth_largest<uint32_t, 32>(
+          n_band, take_eq, [&](int e) { return ~(uint32_t)__ldcg(bj + e); },
+          [&](int e) { return ordered_key64(__ldcg(bt + e)) == vb; }, &gt_s);
+      const int jb = (int)~jb_inv;
+      for (int e = threadIdx.x; e < n_band; e += blockDim.x) {
+        const unsigned long long kk = ordered_key64(__ldcg(bt + e));
+        const int je = __ldcg(bj + e);
+        if (kk > vb || (kk == vb && je <= jb)) {
+          const uint32_t slot = atomicAdd(&n_sel, 1u);
+          if (slot < (uint32_t)kMaxIdxWidth) sel[slot] = je;
+        }
+      }
     }
   }
+  __syncthreads();
   // The forced recent window [p - window + 1, p].
-  for (int j = n_c + threadIdx.x; j <= pos; j += blockDim.x) push(j);
+  const uint32_t n_top = n_sel;
+  for (int j = n_c + threadIdx.x; j <= pos; j += blockDim.x) {
+    const uint32_t slot = n_top + (uint32_t)(j - n_c);
+    if (slot < (uint32_t)kMaxIdxWidth) sel[slot] = j;
+  }
   __syncthreads();
   // Ascending order of the n selected (distinct) positions: counting sort on the
   // position's high bits into 1024 buckets, then each key's rank inside its bucket.
-  const int n = (int)min(n_sel, (uint32_t)kMaxIdxWidth);
+  const int n = (int)min(n_top + (uint32_t)(pos - n_c + 1), (uint32_t)kMaxIdxWidth);
   int shift = 0;
   while ((pos >> shift) >= kBuckets) ++shift;
   for (int e = threadIdx.x; e < kBuckets; e += blockDim.x) bucket[e] = 0u;
@@ -600,15 +711,15 @@ static cudaError_t launch_rest_t(const SelectParams& p, int batch, cudaStream_t 
   const int bq = batch * p.n_q;
   cudaError_t e = launch_pdl(select_compact_kernel, dim3(p.splits3, bq), dim3(kThreads), 0, st, p);
   if (e != cudaSuccess) return e;
-  const size_t qbytes = H * kQLd * sizeof(uint16_t);
+  const size_t dyn = finish_dyn_smem(H);
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(select_finish_kernel<H, FP8>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qbytes);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  return launch_pdl(select_finish_kernel<H, FP8>, dim3(bq), dim3(kFinThreads), qbytes, st, p);
+  return launch_pdl(select_finish_kernel<H, FP8>, dim3(bq), dim3(kFinThreads), dyn, st, p);
 }
 
 template <bool FP8>

@@ -98,6 +98,63 @@ __device__ __forceinline__ uint64_t vt_mnmajor_sw128_desc(uint32_t tile_addr, in
                           sm100::kSwizzle128B);
 }
 
+// Softmax reference usable in 2^(x - m): a reference of -inf (no key seen yet, so
+// every x is -inf too) becomes 0, which gives p = 0 instead of NaN.
+__device__ __forceinline__ float finite_ref(float m) { return m == -INFINITY ? 0.f : m; }
+
+// ---- cluster merge of a gathered row (sparse layers)
+// Gather-mode CTAs of one row run as a thread-block cluster of ns <= kMaxClusterCtas
+// CTAs.  Each leaves its chunk's partial in its own shared memory -- o at offset
+// kClusterOOff as [H][128] floats (unnormalised, reference m in log2 units), (m, l)
+// at kClusterMlOff as [H][2] floats (l = 0: no key) -- and CTA r then combines heads
+// r, r + ns, ... from all ns CTAs through distributed shared memory:
+//   out_h = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s,  M = max over non-empty s.
+// A row with no key at all gets zeros.  Threads [0, 128) take part (d = thread).
+constexpr int kMaxClusterCtas = 16;
+constexpr uint32_t kClusterOOff = 0;
+constexpr uint32_t kClusterMlOff = 32768;  // o of up to 64 heads fits below
+
+template <int H>
+__device__ __forceinline__ void cluster_merge_row(const uint8_t* smem, int ns, float* out_row) {
+  static_assert(H * kHeadDim * 4 <= kClusterMlOff, "partial o must fit below (m, l)");
+  const int d = threadIdx.x;
+  if (d >= kHeadDim) return;
+  const uint32_t o_base = sm100::smem_u32(smem + kClusterOOff);
+  const uint32_t ml_base = sm100::smem_u32(smem + kClusterMlOff);
+  for (int h = (int)sm100::cluster_ctarank(); h < H; h += ns) {
+    float m[kMaxClusterCtas], l[kMaxClusterCtas], o[kMaxClusterCtas];
+#pragma unroll
+    for (int s = 0; s < kMaxClusterCtas; ++s) {
+      if (s < ns) {
+        const float2 v = sm100::ld_shared_cluster_f32x2(
+            sm100::mapa_shared(ml_base + (uint32_t)h * 8u, (uint32_t)s));
+        m[s] = v.x;
+        l[s] = v.y;
+        o[s] = sm100::ld_shared_cluster_f32(
+            sm100::mapa_shared(o_base + (uint32_t)(h * kHeadDim + d) * 4u, (uint32_t)s));
+      } else {
+        m[s] = -INFINITY;
+        l[s] = 0.f;
+        o[s] = 0.f;
+      }
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < kMaxClusterCtas; ++s)
+      if (l[s] > 0.f) M = fmaxf(M, m[s]);
+    float L = 0.f, acc = 0.f;
+#pragma unroll
+    for (int s = 0; s < kMaxClusterCtas; ++s) {
+      if (l[s] > 0.f) {  // an empty partial's o is never read into the sum
+        const float w = exp2f(m[s] - M);
+        L = fmaf(w, l[s], L);
+        acc = fmaf(w, o[s], acc);
+      }
+    }
+    out_row[h * kHeadDim + d] = L > 0.f ? acc / L : 0.f;
+  }
+}
+
 // B operand P^T (P stored [H/8 chunks][128 keys][8 heads], MN-major, unswizzled):
 // K step kk covers keys [16kk, 16kk + 16).
 __device__ __forceinline__ uint64_t pt_mnmajor_desc(uint32_t p_addr, int kk) {
@@ -112,12 +169,24 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint
 
 cudaError_t launch_full_attn_tc(const FullParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                                 int bq, cudaStream_t st);
-// Sparse layer through the same kernel in gather mode (p.idx, p.idx_width set).
-cudaError_t launch_sparse_attn_tc(const FullParams& p, int bq, cudaStream_t st);
+// Sparse layer through the same kernel in gather mode (p.idx, p.idx_width, p.out set):
+// one thread-block cluster per row merges its chunks on chip; the launcher chooses
+// p.splits1 (the cluster size) and p.chunk1.
+cudaError_t launch_sparse_attn_tc(FullParams p, int bq, cudaStream_t st);
 // The same two kernels for an FP8 E4M3 cache (tensor maps over uint8 rows).
 cudaError_t launch_full_attn_fp8(const FullParams& p, const CUtensorMap& tk,
                                  const CUtensorMap& tv, int bq, cudaStream_t st);
-cudaError_t launch_sparse_attn_fp8(const FullParams& p, int bq, cudaStream_t st);
+cudaError_t launch_sparse_attn_fp8(FullParams p, int bq, cudaStream_t st);
+// Chunking of a gathered row over a cluster of at most max_ctas CTAs: chunks of whole
+// 128-entry tiles, as many CTAs as tiles while they fit.
+void plan_gather_cluster(int idx_width, int max_ctas, int* ns, int* chunk);
+// Largest cluster size (16, 8, 4, 2 or 1; 0 if none) with which one cluster of the
+// kernel can be resident, given its block size and dynamic shared memory.
+int largest_cluster_of(const void* kernel, dim3 block, size_t smem);
+template <typename K>
+int largest_cluster(K* kernel, dim3 block, size_t smem) {
+  return largest_cluster_of(reinterpret_cast<const void*>(kernel), block, smem);
+}
 cudaError_t launch_importance_tc(const SelectParams& p, const CUtensorMap& tmap_k, int bq,
                                  cudaStream_t st);
 cudaError_t launch_importance_fp8(const SelectParams& p, const CUtensorMap& tmap_k, int bq,

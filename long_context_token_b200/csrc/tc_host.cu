@@ -52,4 +52,35 @@ int device_sm_count() {
   return cached[dev];
 }
 
+int largest_cluster_of(const void* kernel, dim3 block, size_t smem) {
+  // Non-portable sizes (above 8) need the kernel's opt-in; without it, stop at 8.
+  const bool wide = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                         1) == cudaSuccess;
+  (void)cudaGetLastError();
+  for (int c = wide ? kMaxClusterCtas : 8; c >= 1; c /= 2) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(c, 1, 1);
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)c;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess && n >= 1) return c;
+    (void)cudaGetLastError();
+  }
+  return 0;
+}
+
+void plan_gather_cluster(int idx_width, int max_ctas, int* ns, int* chunk) {
+  const int tiles = (idx_width + kKeyTile - 1) / kKeyTile;
+  const int per = (tiles + max_ctas - 1) / max_ctas;  // tiles per CTA
+  *chunk = per * kKeyTile;
+  *ns = (idx_width + *chunk - 1) / *chunk;
+}
+
 }  // namespace hs2

@@ -161,17 +161,28 @@ __device__ __forceinline__ void pv_tile(const SimtSmem& s, float* acc) {
 // Selection shift delta_h = lse_h - min_h' lse_h' of one (sequence, token), from the
 // full layer's float64 lse (every thread of the block calls this).
 __device__ __forceinline__ void load_delta(const double* lse64, int H, float* d32, double* d64) {
-  __shared__ double mn;
-  if (threadIdx.x == 0) {
+  // Warp 0 loads every head's lse at once (one memory round trip) and reduces the min.
+  if (threadIdx.x < 32) {
+    constexpr int kPerLane = kMaxHeads / 32;
+    double v[kPerLane];
     double m = INFINITY;
-    for (int h = 0; h < H; ++h) m = fmin(m, lse64[h]);
-    mn = m;
-  }
-  __syncthreads();
-  for (int h = threadIdx.x; h < H; h += blockDim.x) {
-    const double d = lse64[h] - mn;
-    if (d32) d32[h] = (float)d;
-    if (d64) d64[h] = d;
+#pragma unroll
+    for (int u = 0; u < kPerLane; ++u) {
+      const int h = (int)threadIdx.x + 32 * u;
+      v[u] = h < H ? __ldcg(lse64 + h) : INFINITY;
+      m = fmin(m, v[u]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmin(m, __shfl_xor_sync(0xffffffffu, m, o));
+#pragma unroll
+    for (int u = 0; u < kPerLane; ++u) {
+      const int h = (int)threadIdx.x + 32 * u;
+      if (h < H) {
+        const double d = v[u] - m;
+        if (d32) d32[h] = (float)d;
+        if (d64) d64[h] = d;
+      }
+    }
   }
   __syncthreads();
 }

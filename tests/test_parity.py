@@ -163,6 +163,40 @@ def test_sparse_layer_skips_padding_and_empty_rows():
     assert np.all(out[0, 1] == 0.0)          # an empty index row yields zeros
 
 
+@pytest.mark.parametrize("kv,h_q", [("bf16", 16), ("fp8", 64), ("bf16", 48)])
+@pytest.mark.parametrize("width", [1, 127, 129, 1152, 2049, 4096])
+def test_sparse_layer_widths(kv, h_q, width):
+    """Index rows of 1 to 32 tiles (one to several tiles per CTA of the merging
+    cluster), with padding slots and a row whose only valid entry is its last."""
+    dev = torch.device("cuda:0")
+    inp = workloads.make_inputs(2, 6000, n_q=2, h_q=h_q, kv=kv, seed=131 + width, n_sparse=1,
+                                lens=[6000, 4500])
+    cache = hs2.Cache(inp.k.to(dev), inp.v.to(dev), inp.lens.to(dev),
+                      None if inp.k_scale is None else inp.k_scale.to(dev),
+                      None if inp.v_scale is None else inp.v_scale.to(dev))
+    ws = hs2.alloc_workspace(cache, 2, h_q)
+    rng = np.random.default_rng(width)
+    idx = np.full((2, 2, width), -1, dtype=np.int32)
+    for b in range(2):
+        L = int(inp.lens[b])
+        for i in range(2):
+            n = width if (b, i) != (1, 1) else 1
+            pos = np.sort(rng.choice(L - 1, size=n, replace=False)).astype(np.int32)
+            if n == width and width > 4:
+                pos[rng.choice(width, size=width // 5, replace=False)] = -1   # padding slots
+            if n == 1:
+                idx[b, i, -1] = pos[0]
+            else:
+                idx[b, i] = pos
+    idx_t = torch.from_numpy(idx).to(dev)
+    out = hs2.sparse_attn(inp.q_layers[0].to(dev), cache, idx_t, ws, inp.sm_scale).cpu().numpy()
+    assert hs2.check_device_status(ws) == 0
+    bits = workloads.numpy_bits(inp)
+    want = oracle.sparse_attn(bits, bits["q_layers"][0], idx)
+    err = np.abs(out - want).max()
+    assert err < TOL[kv], f"max-abs error {err}"
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("n", sorted(workloads.WORKLOADS))
 def test_full_size_workloads_match_oracle(n):
