@@ -37,7 +37,6 @@ FLUSH_BYTES = 256 << 20
 LAUNCHES_PER_STEP_FULL = 2      # split-K flash-decode, split merge
 LAUNCHES_PER_STEP_SELECT = 3    # importance+histogram, compaction, exact finish
 LAUNCHES_PER_SPARSE = 1         # gather attention with the split merge on chip (cluster)
-# (each step also has one workspace memset node, not counted as a kernel)
 
 
 def dist_env():

@@ -24,8 +24,10 @@ constexpr int kTargetCtas = 4 * 148;
 constexpr int kMinChunk = 256;
 constexpr int kChunk4 = 64;
 
-int plan_splits1(int bq, int max_len, int /*num_sms*/) {
-  int splits = (kTargetCtas + bq - 1) / bq;
+// `row_ctas`: CTAs of one key chunk across the batch (one per (sequence, token) row,
+// or per group of G tokens in the several-token kernel).
+int plan_splits1(int row_ctas, int max_len, int /*num_sms*/) {
+  int splits = (kTargetCtas + row_ctas - 1) / row_ctas;
   const int max_splits = (max_len + kMinChunk - 1) / kMinChunk;
   if (splits > max_splits) splits = max_splits;
   if (splits < 1) splits = 1;
@@ -47,7 +49,10 @@ bool make_layout(int batch, int n_q, int h, int max_len, int window, int k_sel, 
   w.max_len = max_len;
   w.window = window;
   w.k_sel = k_sel;
-  w.splits1 = plan_splits1(w.bq, max_len, kSmCountBound);
+  const int row_ctas = dtype == HS2_KV_BF16 && mq_eligible(n_q, h)
+                           ? batch * ((n_q + mq_tokens_per_cta(h) - 1) / mq_tokens_per_cta(h))
+                           : w.bq;
+  w.splits1 = plan_splits1(row_ctas, max_len, kSmCountBound);
   w.splits4 = plan_splits4(kMaxIdxWidth);  // capacity for any idx_width
   const size_t bq = (size_t)w.bq, ml = (size_t)max_len, hh = (size_t)h;
   size_t off = 0;
@@ -178,6 +183,27 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
     p.chunk1 = chunk;
     p.sbuf = w.use_sbuf ? ws_ptr<float>(ws, w.sbuf) : nullptr;
     e = launch_full_attn_fp8(p, tk, tv, bq, s);
+    log2_partials = true;
+  } else if (kv->dtype == HS2_KV_BF16 && mq_eligible(n_q, h)) {
+    // Several new tokens (or 128 heads): 128 query rows of one sequence per CTA, so
+    // each K/V tile is read once for G = 128 / h tokens; chunks of 64-key tiles.
+    CUtensorMap tk, tv;
+    const uint64_t rows = (uint64_t)kv->batch * kv->max_len;
+    if (!make_tmap_2d(&tk, kv->k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kHeadDim, rows,
+                      kHeadDim * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_2d(&tv, kv->v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kHeadDim, rows,
+                      kHeadDim * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cuda_fail(cudaErrorInvalidValue, "tensor maps of K/V");
+    const int G = mq_tokens_per_cta(h);
+    const int ctas_per_split = kv->batch * ((n_q + G - 1) / G);
+    int splits = device_sm_count() / ctas_per_split;
+    if (splits > w.splits1) splits = w.splits1;
+    if (splits < 1) splits = 1;
+    int chunk = (kv->max_len + splits - 1) / splits;
+    chunk = (chunk + 63) / 64 * 64;
+    p.splits1 = (kv->max_len + chunk - 1) / chunk;
+    p.chunk1 = chunk;
+    e = launch_full_attn_mq(p, tk, tv, kv->batch, s);
     log2_partials = true;
   } else if (kv->dtype == HS2_KV_BF16 && h <= 64) {
     // Tensor-core flash-decode: about one CTA per SM, chunks of whole 128-key tiles.

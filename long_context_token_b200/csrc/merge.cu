@@ -5,11 +5,11 @@
 //   lse_h = M_h + ln L_h
 // (base 2 instead of e when the partials were produced in the log2 domain).
 //
-// Grid (bq, h): one CTA per (sequence/token, head), 128 x G threads.  Warp 0 loads the
-// (m, l) pairs once, reduces M and L over the splits (float64 sum) and stages the
-// weights in shared memory;
-// thread (g, d) then sums dimension d over the splits s = g, g + G, ... with eight
-// independent loads in flight, and the G partial sums are added in shared memory.
+// Grid (bq, h): one CTA per (sequence/token, head), 128 x G threads (G = ceil(S / 8),
+// at most 8).  Thread (g, d) first requests dimension d of the partials s = g, g + G,
+// ... (eight at once); meanwhile warp 0 loads the (m, l) pairs, reduces M and L over
+// the splits (float64 sum) and stages the weights in shared memory.  Each thread then
+// sums its partials and the G partial sums are added in shared memory.
 #include "hs2_internal.cuh"
 
 namespace hs2 {
@@ -27,6 +27,14 @@ __global__ void __launch_bounds__(kHeadDim * kMergeMaxGroups) merge_splits_kerne
   const float* pml = p.part_ml + (size_t)bq * S * H * 2;
   const float* po = p.part_o + (size_t)bq * S * H * kHeadDim;
   griddep_wait();
+  // The first eight partials of this thread's dimension are requested before the
+  // weights are known, so the (m, l) and o loads share one memory round trip.
+  const int d = threadIdx.x % kHeadDim, g = threadIdx.x / kHeadDim;
+  const float* src = po + (size_t)h * kHeadDim + d;
+  const size_t stride = (size_t)H * kHeadDim;
+  float v0[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) v0[u] = g + u * G < S ? __ldcg(src + (size_t)(g + u * G) * stride) : 0.f;
   if (threadIdx.x < 32) {
     // One pass over the (m, l) pairs (a single memory round trip), kept in shared memory.
     const int lane = threadIdx.x;
@@ -62,11 +70,16 @@ __global__ void __launch_bounds__(kHeadDim * kMergeMaxGroups) merge_splits_kerne
     }
   }
   __syncthreads();
-  const int d = threadIdx.x % kHeadDim, g = threadIdx.x / kHeadDim;
-  const float* src = po + (size_t)h * kHeadDim + d;
-  const size_t stride = (size_t)H * kHeadDim;
   float acc = 0.f;
-  int s = g;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int s = g + u * G;
+    if (s < S) {
+      const float wt = w[s];
+      if (wt != 0.f) acc = fmaf(wt, v0[u], acc);
+    }
+  }
+  int s = g + 8 * G;
   for (; s + 7 * G < S; s += 8 * G) {
     float v[8];
 #pragma unroll
@@ -91,7 +104,7 @@ __global__ void __launch_bounds__(kHeadDim * kMergeMaxGroups) merge_splits_kerne
 }
 
 cudaError_t launch_merge(const MergeParams& p, int bq, bool log2_domain, cudaStream_t st) {
-  int G = (p.splits + 15) / 16;
+  int G = (p.splits + 7) / 8;
   if (G > kMergeMaxGroups) G = kMergeMaxGroups;
   if (G < 1) G = 1;
   const size_t smem =

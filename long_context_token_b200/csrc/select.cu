@@ -355,7 +355,8 @@ static_assert(kSmallBand * (sizeof(double) + sizeof(int)) <= kMaxIdxWidth * size
               "band pairs must fit the scratch area");
 
 __host__ __device__ constexpr size_t finish_dyn_smem(int H) {
-  return (size_t)H * kQLd * sizeof(uint16_t) + (size_t)kCandSmem * (sizeof(float) + sizeof(int));
+  return (size_t)H * kQLd * sizeof(uint16_t) + (size_t)kCandSmem * (sizeof(float) + sizeof(int)) +
+         (size_t)(kFinThreads / 32) * kHeadDim * sizeof(double);
 }
 
 // Warp-aggregated append to a shared-memory counter: one atomic per warp; returns the
@@ -391,10 +392,21 @@ __device__ KeyT block_kth_largest(int n, int r, KeyFn key, PredFn pred, uint32_t
       sh_gt = 0u;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < n; e += blockDim.x) {
-      if (!pred(e)) continue;
-      const KeyT k = key(e);
-      if ((k & mask) == prefix) atomicAdd(&hist[(uint32_t)(k >> shift) & 255u], 1u);
+    // Keys of one pass share most of their digits (the candidates come from one bin),
+    // so lanes with the same digit are combined first: one shared atomic per distinct
+    // digit per warp instead of one per key on the same address.
+    const int n_r = (n + 31) & ~31;  // whole warps take part in the match
+    for (int e = threadIdx.x; e < n_r; e += blockDim.x) {
+      bool take = false;
+      uint32_t digit = 0;
+      if (e < n && pred(e)) {
+        const KeyT k = key(e);
+        take = (k & mask) == prefix;
+        digit = (uint32_t)(k >> shift) & 255u;
+      }
+      const uint32_t tag = take ? digit : 256u;
+      const unsigned same = __match_any_sync(0xffffffffu, tag);
+      if (take && (threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&hist[digit], __popc(same));
     }
     __syncthreads();
     if (threadIdx.x < 32) {
@@ -452,6 +464,7 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
   uint16_t* qsm = reinterpret_cast<uint16_t*>(fin_dyn);  // [H][kQLd] bf16 q of this query
   float* cts = reinterpret_cast<float*>(fin_dyn + (size_t)H * kQLd * sizeof(uint16_t));
   int* cjs = reinterpret_cast<int*>(cts + kCandSmem);
+  double* kdsm = reinterpret_cast<double*>(cjs + kCandSmem);  // [warps][128] widened K rows
   __shared__ double dlt[H];
   griddep_wait();
   const int bq = blockIdx.x;
@@ -530,60 +543,56 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
   const bool band_smem = n_band <= kSmallBand;
 
   if (need2 > 0) {
-    // float64 re-scoring of the band: one warp per key; for H < 32 the lanes split each
-    // head's dot product into 32 / H parts (lane = part * H + head).
+    // float64 re-scoring of the band, one warp per key: the warp first widens the key's
+    // row to float64 in shared memory (FP8: code x scale, exact), then each lane takes
+    // heads lane, lane + 32, ...; for H < 32 the lanes split each head's dot product
+    // into 32 / H parts (lane = part * H + head).
     constexpr int kParts = H < 32 ? 32 / H : 1;
     constexpr int kSpan = kHeadDim / kParts;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int part = kParts > 1 ? lane / H : 0;
     const double scale = (double)p.sm_scale;
+    double* kd = kdsm + warp * kHeadDim;
     for (int e = warp; e < n_band; e += blockDim.x / 32) {
       const int j = band_smem ? band_js[e] : __ldcg(bj + e);
       const size_t row = (size_t)b * p.kv.max_len + j;
+      if (FP8) {
+        const uint32_t w4 =
+            __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(p.kv.k) +
+                                                    row * kHeadDim) + lane);
+        const double ksc = (double)__ldg(p.kv.k_scale + row);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) kd[4 * lane + u] = e4m3_to_f64((w4 >> (8 * u)) & 0xffu) * ksc;
+      } else {
+        const uint2 w4 = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.kv.k) +
+                                                              row * kHeadDim) + lane);
+        kd[4 * lane] = (double)bf16_bits_to_f32(w4.x & 0xffffu);
+        kd[4 * lane + 1] = (double)bf16_bits_to_f32(w4.x >> 16);
+        kd[4 * lane + 2] = (double)bf16_bits_to_f32(w4.y & 0xffffu);
+        kd[4 * lane + 3] = (double)bf16_bits_to_f32(w4.y >> 16);
+      }
+      __syncwarp();
       double best = -INFINITY;
       for (int h0 = 0; h0 < H; h0 += 32 / kParts) {
         const int h = h0 + (kParts > 1 ? lane % H : lane);
-        if (h >= H) continue;
-        const uint16_t* qh = qsm + h * kQLd;
         double dot = 0.0;
-        if (FP8) {
-          const uint8_t* kr = static_cast<const uint8_t*>(p.kv.k) + row * kHeadDim;
-#pragma unroll 2
-          for (int c = part * kSpan; c < (part + 1) * kSpan; c += 16) {
-            const uint4 kv = __ldg(reinterpret_cast<const uint4*>(kr + c));
-            const uint4 qa = *reinterpret_cast<const uint4*>(qh + c);
-            const uint4 qb = *reinterpret_cast<const uint4*>(qh + c + 8);
-            const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
-            const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              const uint32_t code = (kw[u >> 2] >> (8 * (u & 3))) & 0xffu;
-              const uint32_t qbits = (u & 1) ? (qw[u >> 1] >> 16) : (qw[u >> 1] & 0xffffu);
-              dot = fma((double)bf16_bits_to_f32(qbits), e4m3_to_f64(code), dot);
-            }
-          }
-        } else {
-          const uint16_t* kr = static_cast<const uint16_t*>(p.kv.k) + row * kHeadDim;
-#pragma unroll 2
+        if (h < H) {
+          const uint16_t* qh = qsm + h * kQLd;
+#pragma unroll 4
           for (int c = part * kSpan; c < (part + 1) * kSpan; c += 8) {
-            const uint4 kv = __ldg(reinterpret_cast<const uint4*>(kr + c));
             const uint4 qv = *reinterpret_cast<const uint4*>(qh + c);
-            const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
             const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              dot = fma((double)bf16_bits_to_f32(qw[u] & 0xffffu),
-                        (double)bf16_bits_to_f32(kw[u] & 0xffffu), dot);
-              dot = fma((double)bf16_bits_to_f32(qw[u] >> 16),
-                        (double)bf16_bits_to_f32(kw[u] >> 16), dot);
+              dot = fma((double)bf16_bits_to_f32(qw[u] & 0xffffu), kd[c + 2 * u], dot);
+              dot = fma((double)bf16_bits_to_f32(qw[u] >> 16), kd[c + 2 * u + 1], dot);
             }
           }
         }
 #pragma unroll
         for (int o = 16; o >= 32 / kParts && kParts > 1; o >>= 1)
           dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        if (FP8) dot *= (double)p.kv.k_scale[row];
-        best = fmax(best, scale * dot - dlt[h]);
+        if (h < H) best = fmax(best, scale * dot - dlt[h]);
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) best = fmax(best, __shfl_xor_sync(0xffffffffu, best, o));
@@ -591,6 +600,7 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
         if (band_smem) band_ts[e] = best;
         else bt[e] = best;
       }
+      __syncwarp();  // the next key reuses kd
     }
     __syncthreads();
     if (band_smem) {

@@ -187,6 +187,15 @@ template <typename K>
 int largest_cluster(K* kernel, dim3 block, size_t smem) {
   return largest_cluster_of(reinterpret_cast<const void*>(kernel), block, smem);
 }
+// Full layer for several new tokens per sequence (or 128 heads), bf16 cache: 128 query
+// rows (G = 128 / h tokens x h heads) per CTA, 64-key tiles (tensor maps with 64 x 64
+// boxes).  Partials in the one-token kernel's layout.
+cudaError_t launch_full_attn_mq(const FullParams& p, const CUtensorMap& tk,
+                                const CUtensorMap& tv, int batch, cudaStream_t st);
+int mq_tokens_per_cta(int h);
+inline bool mq_eligible(int n_q, int h) {
+  return (h == 16 || h == 32 || h == 48 || h == 64 || h == 128) && (n_q >= 2 || h > 64);
+}
 cudaError_t launch_importance_tc(const SelectParams& p, const CUtensorMap& tmap_k, int bq,
                                  cudaStream_t st);
 cudaError_t launch_importance_fp8(const SelectParams& p, const CUtensorMap& tmap_k, int bq,

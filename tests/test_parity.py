@@ -87,6 +87,13 @@ SMALL = [
     dict(id="append64-fp8", batch=1, max_len=3000, n_q=64, h_q=16, kv="fp8", seed=111),
     dict(id="ragged-tail-fp8", batch=3, max_len=9000, n_q=1, h_q=16, kv="fp8", seed=112,
          lens=[8999, 4097, 1333]),
+    # several new tokens per sequence (bf16): 128 query rows per CTA, groups of 128 / h
+    # tokens, the last group partial; contexts whose chunks end inside a 64-key tile
+    dict(id="append13-h16-ragged", batch=2, max_len=7000, n_q=13, h_q=16, kv="bf16",
+         seed=113, lens=[7000, 2222]),
+    dict(id="append5-h48", batch=1, max_len=4321, n_q=5, h_q=48, kv="bf16", seed=114),
+    dict(id="append3-h64-short", batch=2, max_len=700, n_q=3, h_q=64, kv="bf16", seed=115,
+         lens=[700, 130]),
 ]
 
 
