@@ -40,10 +40,12 @@ constexpr int kFp8Threads = 320;
 constexpr uint32_t kRawTile = 16384;    // 128 keys x 128 E4M3 codes
 constexpr uint32_t kConvTile = 32768;   // 128 keys x 128 f16 (two 64-column boxes)
 
-template <int H>
+// Gather mode (a sparse layer) keeps one raw stage and one converted V buffer: its CTAs
+// mostly take a single tile, and the smaller footprint lets two CTAs share an SM.
+template <int H, bool GATHER>
 struct Fp8Smem {
-  static constexpr int R = H <= 16 ? 3 : 2;     // raw stages (K and V each)
-  static constexpr int kVConv = 2;              // converted V buffers
+  static constexpr int R = GATHER ? 1 : (H <= 16 ? 3 : 2);  // raw stages (K and V each)
+  static constexpr int kVConv = GATHER ? 1 : 2;              // converted V buffers
   static constexpr uint32_t kQBytes = H * kHeadDim * 2;
   static constexpr uint32_t kPBytes = kKeyTile * H * 2;
   static constexpr uint32_t kKRawOff = 0;
@@ -108,10 +110,10 @@ __device__ __forceinline__ void block_max_heads_f8(const float (&v)[H], float* r
 }  // namespace
 
 template <int H, bool GATHER>
-__global__ void __launch_bounds__(kFp8Threads, 1)
+__global__ void __launch_bounds__(kFp8Threads, (GATHER && H <= 16) ? 2 : 1)
     full_attn_fp8_kernel(const __grid_constant__ CUtensorMap tmap_k,
                          const __grid_constant__ CUtensorMap tmap_v, FullParams p) {
-  using L = Fp8Smem<H>;
+  using L = Fp8Smem<H, GATHER>;
   constexpr int R = L::R;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -208,8 +210,17 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
       part_ml[2 * h + 1] = 0.f;
     }
   } else {
+  if (GATHER) {
+    // The first tile's rows are gathered by every thread of the CTA; warp 0 gathers any
+    // later tiles.  (store_q_f16_scaled below synchronises the block.)
+    gather_tile_rows<8, kRawTile>(smem_u32(kraw), smem_u32(vraw),
+                                  static_cast<const uint8_t*>(p.kv.k),
+                                  static_cast<const uint8_t*>(p.kv.v), idx_row, k0, k1, Lb,
+                                  row_base, p.status, threadIdx.x, blockDim.x);
+  }
   // Q in f16 under a per-head power-of-two scale; its inverse goes into the logits.
   store_q_f16_scaled<H>(qs, p.q + (size_t)bq * H * kHeadDim, qinv_s, nullptr);
+  if (GATHER) cp_async_wait_all();
   for (int h = threadIdx.x; h < H; h += blockDim.x) c2_s[h] = p.sm_scale * kLog2eF8 * qinv_s[h];
   fence_proxy_async_smem();
   tc_fence_before();
@@ -222,33 +233,19 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
     if (GATHER) {
       // ---------------------------------------------- gather producer (32 lanes)
       const int lane = (int)lane_id();
-      const uint8_t* kb = static_cast<const uint8_t*>(p.kv.k);
-      const uint8_t* vb = static_cast<const uint8_t*>(p.kv.v);
       for (int i = 0; i < n_tiles; ++i) {
         const int s = i % R;
-        const uint32_t ph = ((i / R) & 1) ^ 1;
-        if (ok && !mbar_wait(kr_empty + s, ph)) ok = false;
-        if (ok && !mbar_wait(vr_empty + s, ph)) ok = false;
-        const uint32_t kd = smem_u32(kraw + s * kRawTile), vd = smem_u32(vraw + s * kRawTile);
-        for (int rr = 0; rr < kKeyTile / 32; ++rr) {
-          const int r = lane + 32 * rr, e = k0 + i * kKeyTile + r;
-          long long row = -1;
-          if (e < k1) {
-            const int j = __ldg(idx_row + e);
-            if (j >= 0 && j < Lb) row = (long long)(row_base + j);
-            else if (j != -1) set_status(p.status, HS2_ERR_INDEX_OUT_OF_RANGE);
-          }
-          const size_t off = row >= 0 ? (size_t)row * kHeadDim : 0;
-          const uint32_t nb = row >= 0 ? 16u : 0u;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint32_t at = r * 128 + ((uint32_t)((c ^ r) & 7) << 4);
-            cp_async_16(kd + at, kb + off + c * 16, nb);
-            cp_async_16(vd + at, vb + off + c * 16, nb);
-          }
+        if (i > 0) {  // tile 0 was gathered by the whole CTA above
+          const uint32_t ph = ((i / R) & 1) ^ 1;
+          if (ok && !mbar_wait(kr_empty + s, ph)) ok = false;
+          if (ok && !mbar_wait(vr_empty + s, ph)) ok = false;
+          gather_tile_rows<8, kRawTile>(
+              smem_u32(kraw + s * kRawTile), smem_u32(vraw + s * kRawTile),
+              static_cast<const uint8_t*>(p.kv.k), static_cast<const uint8_t*>(p.kv.v), idx_row,
+              k0 + i * kKeyTile, k1, Lb, row_base, p.status, lane, 32);
+          cp_async_wait_all();
+          fence_proxy_async_smem();
         }
-        cp_async_wait_all();
-        fence_proxy_async_smem();
         mbar_arrive(kr_full + s);
         mbar_arrive(vr_full + s);
       }
@@ -282,8 +279,8 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
       const uint32_t q_addr = smem_u32(qs);
       const uint32_t k_addr = smem_u32(kconv);
       auto issue_pv = [&](int t) -> bool {
-        const int vb = t & 1, pb = t & 1;
-        if (!mbar_wait(vc_full + vb, (t >> 1) & 1)) return false;
+        const int vb = t % L::kVConv, pb = t & 1;
+        if (!mbar_wait(vc_full + vb, (t / L::kVConv) & 1)) return false;
         if (!mbar_wait(p_full + pb, (t >> 1) & 1)) return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(vconv + vb * kConvTile);
@@ -325,9 +322,9 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
       fence_proxy_async_smem();
       mbar_arrive(kc_full);
       mbar_arrive(kr_empty + s);
-      const int vb = i & 1;
+      const int vb = i % L::kVConv;
       if (ok && !mbar_wait(vr_full + s, (i / R) & 1)) ok = false;
-      if (ok && !mbar_wait(vc_empty + vb, ((i >> 1) & 1) ^ 1)) ok = false;
+      if (ok && !mbar_wait(vc_empty + vb, ((i / L::kVConv) & 1) ^ 1)) ok = false;
       convert_row(vraw + s * kRawTile, vconv + vb * kConvTile, t, valid);
       fence_proxy_async_smem();
       mbar_arrive(vc_full + vb);
@@ -369,27 +366,29 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
       if (named_bar_or(3, 128, !ok)) ok = false;
       tc_fence_after();
       float x[H];
+      {
+        // Every chunk's load in flight before the one wait.
+        uint32_t r[H];
 #pragma unroll
-      for (int c = 0; c < H; c += 16) {
-        uint32_t r[16];
-        tmem_ld16(tmem_base + lane_base + sb * H + c, r);
+        for (int c = 0; c < H; c += 16)
+          tmem_ld16(tmem_base + lane_base + sb * H + c, *reinterpret_cast<uint32_t(*)[16]>(r + c));
         tmem_wait_ld();
         if (!GATHER && p.sbuf) {
           if (j < k1 && j <= pos - p.window && pos - p.window + 1 > p.k_sel) {
-            float* dst = p.sbuf + ((size_t)bq * p.kv.max_len + j) * H + c;
+            float* dst = p.sbuf + ((size_t)bq * p.kv.max_len + j) * H;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
+            for (int e = 0; e < H / 4; ++e) {
               uint4 v;
-              v.x = __float_as_uint(__uint_as_float(r[4 * e]) * qinv_s[c + 4 * e] * ks);
-              v.y = __float_as_uint(__uint_as_float(r[4 * e + 1]) * qinv_s[c + 4 * e + 1] * ks);
-              v.z = __float_as_uint(__uint_as_float(r[4 * e + 2]) * qinv_s[c + 4 * e + 2] * ks);
-              v.w = __float_as_uint(__uint_as_float(r[4 * e + 3]) * qinv_s[c + 4 * e + 3] * ks);
+              v.x = __float_as_uint(__uint_as_float(r[4 * e]) * qinv_s[4 * e] * ks);
+              v.y = __float_as_uint(__uint_as_float(r[4 * e + 1]) * qinv_s[4 * e + 1] * ks);
+              v.z = __float_as_uint(__uint_as_float(r[4 * e + 2]) * qinv_s[4 * e + 2] * ks);
+              v.w = __float_as_uint(__uint_as_float(r[4 * e + 3]) * qinv_s[4 * e + 3] * ks);
               st_global_v4_hint(dst + 4 * e, v, keep_policy);
             }
           }
         }
 #pragma unroll
-        for (int e = 0; e < 16; ++e) x[c + e] = __uint_as_float(r[e]) * (c2_s[c + e] * ks);
+        for (int e = 0; e < H; ++e) x[e] = __uint_as_float(r[e]) * (c2_s[e] * ks);
       }
       tc_fence_before();
       mbar_arrive(s_free + sb);
@@ -495,7 +494,7 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
 template <int H, bool GATHER>
 static cudaError_t launch_fp8_t(FullParams p, const CUtensorMap& tk, const CUtensorMap& tv,
                                 int bq, cudaStream_t st) {
-  using L = Fp8Smem<H>;
+  using L = Fp8Smem<H, GATHER>;
   auto kernel = full_attn_fp8_kernel<H, GATHER>;
   static int max_cluster = 0;
   if (!max_cluster) {

@@ -12,12 +12,15 @@
 //   O[128 rows x 128 d]   += (P_hi + P_lo) . V_tile       (2 x 4 x K=16)
 //
 //   warp 0      TMA producer: 64-key K and V tiles (two 64-column boxes, 128-byte
-//               swizzle) into a 4-stage ring;
+//               swizzle) into a 3-stage ring;
 //   warp 1      TMEM allocator, MMA issuer (the P.V of tile i-1 after the Q.K of i);
-//   warps 2..5  softmax: thread r owns query row r (TMEM lane r).  Logits go to the
-//               log2 domain; the row's reference only moves when a logit exceeds it
-//               by more than 8 (then the row of O is rescaled in TMEM); p = 2^(x - m)
-//               is split into bf16 hi + lo so that P.V keeps ~16 bits of p.
+//   warps 2..9  softmax: query row r (TMEM lane r) is owned by two threads, of warps
+//               w and w + 4, each taking 32 of the tile's 64 keys and half of the
+//               row of O; they exchange their tile maxima through shared memory.
+//               Logits go to the log2 domain; the row's reference only moves when a
+//               logit exceeds it by more than 8 (then the row of O is rescaled in
+//               TMEM); p = 2^(x - m) is split into bf16 hi + lo so that P.V keeps
+//               ~16 bits of p.
 // Each CTA writes the partial (m in log2 units, l, unnormalised o) of each of its rows
 // for its key chunk, in the layout of the one-token kernel; merge.cu combines them.
 #include <cuda_bf16.h>
@@ -40,15 +43,19 @@ constexpr int kMqKeys = 64;                   // keys per tile
 constexpr uint32_t kMqBox = kMqKeys * 128;    // 64 rows x 128 B: one swizzled box
 constexpr uint32_t kMqTile = 2 * kMqBox;      // 64 keys x 128 d x bf16
 
+constexpr int kMqSoftmax = 256;                 // softmax threads (two per query row)
+constexpr int kMqThreads = 64 + kMqSoftmax;
+
 struct MqSmem {
-  static constexpr int kStages = 4;
+  static constexpr int kStages = 3;
   static constexpr uint32_t kKOff = 0;
   static constexpr uint32_t kVOff = kStages * kMqTile;
   static constexpr uint32_t kQOff = 2 * kStages * kMqTile;
   static constexpr uint32_t kQBytes = kMqRows * kHeadDim * 2;
   static constexpr uint32_t kPBytes = kMqRows * kMqKeys * 2;  // one of hi / lo
   static constexpr uint32_t kPOff = kQOff + kQBytes;           // [2 buffers][hi, lo]
-  static constexpr uint32_t kBarOff = kPOff + 4 * kPBytes;
+  static constexpr uint32_t kRedOff = kPOff + 4 * kPBytes;     // [2 tiles][2 halves][128] f32
+  static constexpr uint32_t kBarOff = kRedOff + 2 * 2 * kMqRows * 4;
   static constexpr uint32_t kBars = 4 * kStages + 9;
   static constexpr uint32_t kSlotOff = kBarOff + kBars * 8;
   static constexpr uint32_t kBytes = kSlotOff + 16 + 1024;
@@ -75,7 +82,7 @@ __device__ __forceinline__ uint64_t vtile_mnmajor_desc(uint32_t tile, int kk) {
 }  // namespace
 
 template <int H>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kMqThreads, 1)
     full_attn_mq_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v, FullParams p, int n_groups) {
   using L = MqSmem;
@@ -87,6 +94,7 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* vst = smem + L::kVOff;
   uint8_t* qs = smem + L::kQOff;
   uint8_t* ps = smem + L::kPOff;
+  float* red = reinterpret_cast<float*>(smem + L::kRedOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* kfull = bars;
   uint64_t* kempty = bars + NS;
@@ -112,8 +120,8 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(s_full + s, 1);
-      mbar_init(s_free + s, 128);
-      mbar_init(p_full + s, 128);
+      mbar_init(s_free + s, kMqSoftmax);
+      mbar_init(p_full + s, kMqSoftmax);
       mbar_init(p_free + s, 1);
     }
     mbar_init(mma_done, 1);
@@ -236,38 +244,49 @@ __global__ void __launch_bounds__(192, 1)
       }
     } else {
       // ------------------------------------------------------------ softmax
-      const int lg = warp & 3;
+      const int lg = warp & 3;                 // TMEM lane quarter of this warp
+      const int half = (warp - 2) >> 2;        // which 32 keys of a tile (and half of O)
       const int r = lg * 32 + (int)lane_id();  // query row == TMEM lane
+      const int st = half * kMqRows + r;       // softmax thread index, 0 .. 255
       const uint32_t lane_base = (uint32_t)(lg * 32) << 16;
       const int g = r / H;
       const bool row_live = g < ntok;
       const int pos_r = pos0 + g;                // this row's token sees keys [0, pos_r]
       const int kend = row_live ? min(k1, pos_r + 1) : k0;  // its keys in this chunk
       const float c2 = p.sm_scale * kLog2eMq;
+      constexpr int KH = kMqKeys / 2;            // keys per thread per tile
       float mref = -INFINITY, l = 0.f;
       for (int i = 0; i < n_tiles; ++i) {
         const int sb = i & 1;
         if (ok && !mbar_wait(s_full + sb, (i >> 1) & 1)) ok = false;
-        if (named_bar_or(3, 128, !ok)) ok = false;
+        if (named_bar_or(3, kMqSoftmax, !ok)) ok = false;
         tc_fence_after();
-        float x[kMqKeys];
+        float x[KH];
+        {
+          uint32_t v[KH];
 #pragma unroll
-        for (int c = 0; c < kMqKeys; c += 16) {
-          uint32_t v[16];
-          tmem_ld16(tmem_base + lane_base + sb * kMqKeys + c, v);
+          for (int c = 0; c < KH; c += 16)
+            tmem_ld16(tmem_base + lane_base + sb * kMqKeys + half * KH + c,
+                      *reinterpret_cast<uint32_t(*)[16]>(v + c));
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) x[c + e] = __uint_as_float(v[e]) * c2;
+          for (int e = 0; e < KH; ++e) x[e] = __uint_as_float(v[e]) * c2;
         }
         tc_fence_before();
         mbar_arrive(s_free + sb);
-        const int jb = k0 + i * kMqKeys;
+        const int jb = k0 + i * kMqKeys + half * KH;
         float tmax = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < kMqKeys; ++c) {
+        for (int c = 0; c < KH; ++c) {
           if (jb + c >= kend) x[c] = -INFINITY;
           tmax = fmaxf(tmax, x[c]);
         }
+        // Row max over both halves (slots alternate by tile so that a fast thread
+        // cannot overwrite a value its partner has not read yet).
+        float* rt = red + (size_t)(i & 1) * 2 * kMqRows;
+        rt[half * kMqRows + r] = tmax;
+        named_bar_sync(1, kMqSoftmax);
+        tmax = fmaxf(rt[r], rt[kMqRows + r]);
         // Lazy reference: move it only when this tile would give p > 2^8.
         const bool move = tmax - mref > kRescaleAtMq;  // false while tmax is -inf
         float alpha = 1.f;
@@ -277,19 +296,21 @@ __global__ void __launch_bounds__(192, 1)
           l *= alpha;
         }
         if (__any_sync(0xffffffffu, move) && i > 0) {
-          // O holds the P.V of tiles < i: wait for the last one, then rescale the rows
-          // whose reference moved (the others multiply by 1).
+          // O holds the P.V of tiles < i: wait for the last one, then rescale this
+          // thread's half of the row (rows whose reference stayed multiply by 1).
           if (ok && !mbar_wait(p_free + ((i - 1) & 1), ((i - 1) >> 1) & 1)) ok = false;
           tc_fence_after();
+          uint32_t v[64];
 #pragma unroll
-          for (int c = 0; c < kHeadDim; c += 16) {
-            uint32_t v[16];
-            tmem_ld16(tmem_o + lane_base + c, v);
-            tmem_wait_ld();
+          for (int c = 0; c < 64; c += 16)
+            tmem_ld16(tmem_o + lane_base + half * 64 + c, *reinterpret_cast<uint32_t(*)[16]>(v + c));
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-            tmem_st16(tmem_o + lane_base + c, v);
-          }
+          for (int e = 0; e < 64; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+#pragma unroll
+          for (int c = 0; c < 64; c += 16)
+            tmem_st16(tmem_o + lane_base + half * 64 + c,
+                      *reinterpret_cast<const uint32_t(*)[16]>(v + c));
           tmem_wait_st();
           tc_fence_before();
         }
@@ -299,7 +320,7 @@ __global__ void __launch_bounds__(192, 1)
         uint8_t* plo = phi + L::kPBytes;
         const float mr = finite_ref(mref);
 #pragma unroll
-        for (int c = 0; c < kMqKeys / 8; ++c) {
+        for (int c = 0; c < KH / 8; ++c) {
           uint32_t hw[4], lw[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -312,12 +333,13 @@ __global__ void __launch_bounds__(192, 1)
             hw[e] = *reinterpret_cast<const uint32_t*>(&hi);
             lw[e] = *reinterpret_cast<const uint32_t*>(&lo);
           }
-          *reinterpret_cast<uint4*>(phi + c * (kMqRows * 16) + r * 16) =
+          const int chunk = half * (KH / 8) + c;  // 8-key chunk of the tile
+          *reinterpret_cast<uint4*>(phi + chunk * (kMqRows * 16) + r * 16) =
               make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(plo + c * (kMqRows * 16) + r * 16) =
+          *reinterpret_cast<uint4*>(plo + chunk * (kMqRows * 16) + r * 16) =
               make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
-        if (i == n_tiles - 1 && r < kMqKeys && jb + r >= k1) {
+        if (i == n_tiles - 1 && half == 0 && r < kMqKeys && k0 + i * kMqKeys + r >= k1) {
           // Rows past the chunk end may hold anything (NaN included); 0 * NaN would
           // poison P.V, so zero this key's V row once its tile has landed.
           const int s = i % NS;
@@ -334,29 +356,34 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive(p_full + sb);
       }
       griddep_launch_dependents();  // the merge may be scheduled; it waits for this grid
-      // Epilogue: row r of O is (token g, head h); partial (m, l, o) of its split.
+      // Epilogue: row r of O is (token g, head h); each thread writes its half of the
+      // row, the half-0 thread the row's (m, l) with l summed over both halves.
       const int last = n_tiles - 1;
       if (ok && !mbar_wait(p_free + (last & 1), (last >> 1) & 1)) ok = false;
       tc_fence_after();
       const size_t pi = part_index(row_live ? g : 0) * H + r % H;
-      float* po = p.part_o + pi * kHeadDim;
+      float* po = p.part_o + pi * kHeadDim + half * 64;
+      {
+        uint32_t v[64];
 #pragma unroll
-      for (int c = 0; c < kHeadDim; c += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem_o + lane_base + c, v);
+        for (int c = 0; c < 64; c += 16)
+          tmem_ld16(tmem_o + lane_base + half * 64 + c, *reinterpret_cast<uint32_t(*)[16]>(v + c));
         tmem_wait_ld();
         if (row_live) {
 #pragma unroll
-          for (int e = 0; e < 16; e += 4)
-            *reinterpret_cast<float4*>(po + c + e) =
+          for (int e = 0; e < 64; e += 4)
+            *reinterpret_cast<float4*>(po + e) =
                 make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
                             __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
         }
       }
       tc_fence_before();
-      if (row_live) {
+      named_bar_sync(1, kMqSoftmax);  // every thread is past its last use of red
+      red[st] = l;
+      named_bar_sync(1, kMqSoftmax);
+      if (row_live && half == 0) {
         p.part_ml[pi * 2] = mref;
-        p.part_ml[pi * 2 + 1] = l;
+        p.part_ml[pi * 2 + 1] = red[r] + red[kMqRows + r];
       }
     }
   }
@@ -380,8 +407,8 @@ static cudaError_t launch_mq_t(const FullParams& p, const CUtensorMap& tk, const
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  return launch_pdl(full_attn_mq_kernel<H>, dim3(p.splits1, batch * n_groups), dim3(192),
-                    L::kBytes, st, tk, tv, p, n_groups);
+  return launch_pdl(full_attn_mq_kernel<H>, dim3(p.splits1, batch * n_groups),
+                    dim3(kMqThreads), L::kBytes, st, tk, tv, p, n_groups);
 }
 
 int mq_tokens_per_cta(int h) { return h >= 16 && h <= kMqRows ? kMqRows / h : 0; }

@@ -34,9 +34,11 @@ using namespace sm100;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleAt = 8.0f;  // log2 units: move the reference when p would exceed 2^8
 
-template <int H>
+// Gather mode (a sparse layer) keeps one stage: its CTAs mostly take a single tile, and
+// the smaller footprint lets two CTAs share an SM.
+template <int H, bool GATHER>
 struct FullSmem {
-  static constexpr int kStages = H <= 16 ? 3 : 2;
+  static constexpr int kStages = GATHER ? 1 : (H <= 16 ? 3 : 2);
   static constexpr uint32_t kTile = kKTileBytesBf16;    // one K or V tile
   static constexpr uint32_t kQBytes = H * kHeadDim * 2;
   static constexpr uint32_t kPBytes = kKeyTile * H * 2;  // one of hi / lo
@@ -70,10 +72,10 @@ __device__ __forceinline__ void block_max_heads(const float (&v)[H], float* red,
 }
 
 template <int H, bool GATHER>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
     full_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v, FullParams p) {
-  using L = FullSmem<H>;
+  using L = FullSmem<H, GATHER>;
   constexpr int NS = L::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -152,7 +154,16 @@ __global__ void __launch_bounds__(192, 1)
       part_ml[2 * h + 1] = 0.f;
     }
   } else {
+    if (GATHER) {
+      // The first tile's rows are gathered by every thread of the CTA (the issue of
+      // 4096 16-byte copies is the gather's cost); warp 0 gathers any later tiles.
+      gather_tile_rows<16, kBoxBytes>(smem_u32(kst), smem_u32(vst),
+                                      static_cast<const uint8_t*>(p.kv.k),
+                                      static_cast<const uint8_t*>(p.kv.v), idx_row, k0, k1, Lb,
+                                      row_base, p.status, threadIdx.x, blockDim.x);
+    }
     store_q_kmajor<H>(qs, p.q + (size_t)bq * H * kHeadDim, threadIdx.x, blockDim.x);
+    if (GATHER) cp_async_wait_all();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -165,38 +176,31 @@ __global__ void __launch_bounds__(192, 1)
       // Rows named by the index row go to the same 128-byte-swizzled layout that TMA
       // writes (16-byte chunk c of row r at chunk c ^ (r mod 8)); absent rows are
       // zero-filled.  Each lane copies 4 rows, waits for its copies and arrives.
+      // K and V of a later tile are gathered on their own barriers: with one stage the
+      // P.V of tile i-1 (which frees V) is issued only after the Q.K of tile i.
       const int lane = (int)lane_id();
       const uint8_t* kb = static_cast<const uint8_t*>(p.kv.k);
       const uint8_t* vb = static_cast<const uint8_t*>(p.kv.v);
       for (int i = 0; i < n_tiles; ++i) {
         const int s = i % NS;
         const uint32_t ph = ((i / NS) & 1) ^ 1;
-        if (ok && !mbar_wait(kempty + s, ph)) ok = false;
-        if (ok && !mbar_wait(vempty + s, ph)) ok = false;
-        const uint32_t kdst = smem_u32(kst + s * L::kTile), vdst = smem_u32(vst + s * L::kTile);
-        for (int rr = 0; rr < kKeyTile / 32; ++rr) {
-          const int r = lane + 32 * rr, e = k0 + i * kKeyTile + r;
-          int j = -1;
-          if (e < k1) {
-            j = __ldg(idx_row + e);
-            if (j < 0 || j >= Lb) {
-              if (j != -1) set_status(p.status, HS2_ERR_INDEX_OUT_OF_RANGE);
-              j = -1;
-            }
-          }
-          const size_t off = j >= 0 ? (row_base + j) * (kHeadDim * 2) : 0;
-          const uint32_t nb = j >= 0 ? 16u : 0u;
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const uint32_t at = (uint32_t)(c >> 3) * kBoxBytes + r * 128 +
-                                ((uint32_t)((c & 7) ^ (r & 7)) << 4);
-            cp_async_16(kdst + at, kb + off + c * 16, nb);
-            cp_async_16(vdst + at, vb + off + c * 16, nb);
-          }
+        if (i > 0) {  // tile 0 was gathered by the whole CTA above
+          if (ok && !mbar_wait(kempty + s, ph)) ok = false;
+          gather_tile_rows<16, kBoxBytes>(smem_u32(kst + s * L::kTile), 0u, kb, nullptr, idx_row,
+                                          k0 + i * kKeyTile, k1, Lb, row_base, p.status, lane,
+                                          32);
+          cp_async_wait_all();
+          fence_proxy_async_smem();
         }
-        cp_async_wait_all();
-        fence_proxy_async_smem();
         mbar_arrive(kfull + s);
+        if (i > 0) {
+          if (ok && !mbar_wait(vempty + s, ph)) ok = false;
+          gather_tile_rows<16, kBoxBytes>(0u, smem_u32(vst + s * L::kTile), nullptr, vb, idx_row,
+                                          k0 + i * kKeyTile, k1, Lb, row_base, p.status, lane,
+                                          32);
+          cp_async_wait_all();
+          fence_proxy_async_smem();
+        }
         mbar_arrive(vfull + s);
       }
     } else if (warp == 0) {
@@ -288,26 +292,28 @@ __global__ void __launch_bounds__(192, 1)
         if (named_bar_or(3, 128, !ok)) ok = false;
         tc_fence_after();
         float x[H];
+        {
+          // Every chunk's load in flight before the one wait.
+          uint32_t r[H];
 #pragma unroll
-        for (int c = 0; c < H; c += 16) {
-          uint32_t r[16];
-          tmem_ld16(tmem_base + lane_base + sb * H + c, r);
+          for (int c = 0; c < H; c += 16)
+            tmem_ld16(tmem_base + lane_base + sb * H + c, *reinterpret_cast<uint32_t(*)[16]>(r + c));
           tmem_wait_ld();
           if (!GATHER && p.sbuf) {
             // Raw float32 logits of keys outside the window, for the selection (kept in
             // L2 with an evict-last policy; the selection reads them right after).
             const int jj = k0 + i * kKeyTile + t;
             if (jj < k1 && jj <= pos - p.window && pos - p.window + 1 > p.k_sel) {
-              float* dst = p.sbuf + ((size_t)bq * p.kv.max_len + jj) * H + c;
+              float* dst = p.sbuf + ((size_t)bq * p.kv.max_len + jj) * H;
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
+              for (int e = 0; e < H / 4; ++e)
                 st_global_v4_hint(dst + 4 * e,
                                   make_uint4(r[4 * e], r[4 * e + 1], r[4 * e + 2], r[4 * e + 3]),
                                   keep_policy);
             }
           }
 #pragma unroll
-          for (int e = 0; e < 16; ++e) x[c + e] = __uint_as_float(r[e]) * c2;
+          for (int e = 0; e < H; ++e) x[e] = __uint_as_float(r[e]) * c2;
         }
         tc_fence_before();
         mbar_arrive(s_free + sb);
@@ -442,7 +448,7 @@ __global__ void __launch_bounds__(192, 1)
 template <int H, bool GATHER>
 static cudaError_t launch_full_tc_t(FullParams p, const CUtensorMap& tk, const CUtensorMap& tv,
                                     int bq, cudaStream_t st) {
-  using L = FullSmem<H>;
+  using L = FullSmem<H, GATHER>;
   auto kernel = full_attn_tc_kernel<H, GATHER>;
   static int max_cluster = 0;
   if (!max_cluster) {

@@ -146,6 +146,20 @@ static hs2_status prepare(const void* q, int n_q, int h, const hs2_kv* kv, int w
   return HS2_OK;
 }
 
+// Key chunks of the one-token tensor-core full layer (bf16 or FP8): about one CTA per SM,
+// chunks of whole 128-key tiles, at most the workspace's split count.
+static void plan_decode_splits(const hs2_kv* kv, int n_q, const WsLayout& w, int* splits_out,
+                               int* chunk_out) {
+  const int bq = kv->batch * n_q;
+  int splits = device_sm_count() / bq;
+  if (splits > w.splits1) splits = w.splits1;
+  if (splits < 1) splits = 1;
+  int chunk = (kv->max_len + splits - 1) / splits;
+  chunk = (chunk + 127) / 128 * 128;
+  *splits_out = (kv->max_len + chunk - 1) / chunk;
+  *chunk_out = chunk;
+}
+
 static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int window,
                            int k_sel, float sm_scale, float* out, float* lse, void* ws,
                            const WsLayout& w, cudaStream_t s) {
@@ -174,13 +188,7 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
                       128, CU_TENSOR_MAP_SWIZZLE_128B))
       return cuda_fail(cudaErrorInvalidValue, "tensor maps of K/V");
     const int bq = kv->batch * n_q;
-    int splits = device_sm_count() / bq;
-    if (splits > w.splits1) splits = w.splits1;
-    if (splits < 1) splits = 1;
-    int chunk = (kv->max_len + splits - 1) / splits;
-    chunk = (chunk + 127) / 128 * 128;
-    p.splits1 = (kv->max_len + chunk - 1) / chunk;
-    p.chunk1 = chunk;
+    plan_decode_splits(kv, n_q, w, &p.splits1, &p.chunk1);
     p.sbuf = w.use_sbuf ? ws_ptr<float>(ws, w.sbuf) : nullptr;
     e = launch_full_attn_fp8(p, tk, tv, bq, s);
     log2_partials = true;
@@ -215,13 +223,7 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
                       kHeadDim * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
       return cuda_fail(cudaErrorInvalidValue, "tensor maps of K/V");
     const int bq = kv->batch * n_q;
-    int splits = device_sm_count() / bq;
-    if (splits > w.splits1) splits = w.splits1;
-    if (splits < 1) splits = 1;
-    int chunk = (kv->max_len + splits - 1) / splits;
-    chunk = (chunk + 127) / 128 * 128;
-    p.splits1 = (kv->max_len + chunk - 1) / chunk;
-    p.chunk1 = chunk;
+    plan_decode_splits(kv, n_q, w, &p.splits1, &p.chunk1);
     p.sbuf = w.use_sbuf ? ws_ptr<float>(ws, w.sbuf) : nullptr;
     e = launch_full_attn_tc(p, tk, tv, bq, s);
     log2_partials = true;
@@ -274,7 +276,30 @@ static hs2_status run_select(const void* q, int n_q, int h, const hs2_kv* kv, in
   p.status = ws_ptr<uint32_t>(ws, w.status);
   const int bq = kv->batch * n_q;
   if (w.use_sbuf) {
+    // The stored logits come from the one-token tensor-core full layer (h = 16 <= 64).
+    p.part1_ml = ws_ptr<float>(ws, w.part1_ml);
+    int chunk1 = 0;
+    plan_decode_splits(kv, n_q, w, &p.splits1, &chunk1);
     e = launch_importance_sbuf(p, bq, s);
+    if (e != cudaSuccess) return cuda_fail(e, "importance launch");
+    e = launch_select_rest(p, kv->batch, s);
+  } else if (kv->dtype == HS2_KV_BF16 && mq_eligible(n_q, h)) {
+    // Several tokens per CTA (128 query rows): each K tile is read once per group.
+    CUtensorMap tk;
+    if (!make_tmap_2d(&tk, kv->k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kHeadDim,
+                      (uint64_t)kv->batch * kv->max_len, kHeadDim * 2, 64, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+      return cuda_fail(cudaErrorInvalidValue, "tensor map of K");
+    const int G = mq_tokens_per_cta(h);
+    const int ctas_per_split = kv->batch * ((n_q + G - 1) / G);
+    int splits = device_sm_count() / ctas_per_split;
+    const int min_splits = (kv->max_len + 65535 - 1) / 65535 + 1;  // chunk below 65536
+    if (splits < min_splits) splits = min_splits;
+    int chunk = (kv->max_len + splits - 1) / splits;
+    chunk = (chunk + 127) / 128 * 128;
+    p.splits2 = (kv->max_len + chunk - 1) / chunk;
+    p.chunk2 = chunk;
+    e = launch_importance_mq(p, tk, kv->batch, s);
     if (e != cudaSuccess) return cuda_fail(e, "importance launch");
     e = launch_select_rest(p, kv->batch, s);
   } else if (kv->dtype == HS2_KV_BF16) {

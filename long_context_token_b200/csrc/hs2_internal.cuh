@@ -111,6 +111,10 @@ struct SelectParams {
   int splits3, chunk3;   // compaction pass
   const double* lse64;  // per-head lse of the full layer, [bq][h]
   const float* sbuf;     // raw float32 logits written by the full layer, or null
+  // With sbuf: the full layer's split partials (m in log2 units, l), from which the
+  // importance pass takes the per-head lse itself instead of waiting for the merge.
+  const float* part1_ml = nullptr;
+  int splits1 = 0;
   float* tbuf;
   uint32_t* hist;
   uint32_t* counters;

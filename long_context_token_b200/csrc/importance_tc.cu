@@ -164,13 +164,15 @@ __global__ void __launch_bounds__(192, 1)
       float best = -INFINITY;
       const uint32_t taddr = tmem_base + ((uint32_t)(lg * 32) << 16) + buf * H;
 #pragma unroll
-      for (int c = 0; c < H; c += 16) {
-        uint32_t r[16];
-        tmem_ld16(taddr + c, r);
+      for (int c0 = 0; c0 < H; c0 += 64) {  // up to four loads in flight per wait
+        uint32_t r[64];
+#pragma unroll
+        for (int c = 0; c < 64; c += 16)
+          if (c0 + c < H) tmem_ld16(taddr + c0 + c, *reinterpret_cast<uint32_t(*)[16]>(r + c));
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          best = fmaxf(best, __uint_as_float(r[e]) * sc - delta_s[c + e]);
+        for (int e = 0; e < 64; ++e)
+          if (c0 + e < H) best = fmaxf(best, __uint_as_float(r[e]) * sc - delta_s[c0 + e]);
       }
       tc_fence_before();
       mbar_arrive(s_free + buf);
@@ -224,6 +226,256 @@ cudaError_t launch_importance_tc(const SelectParams& p, const CUtensorMap& tmap_
   }
 }
 
+
+// ============================================================================
+// Several new tokens of one sequence per CTA (bf16 cache, the several-token full
+// layer's shapes): S^T[128 keys x N] = K_tile . Q^T with N = G tokens x H heads
+// (G = 128 / H), so each K tile is read once for G tokens.  Thread t (key t) takes,
+// per token, the max over that token's H heads; each token has its own histogram,
+// kept in shared memory as two 16-bit counters per word (a CTA's chunk is below
+// 65536 keys, so a counter cannot carry into its neighbour).
+// ============================================================================
+namespace {
+
+constexpr int kImpMqRows = 128;
+constexpr int kImpMqMaxChunk = 65535;
+
+template <int H>
+struct ImpMqSmem {
+  static constexpr int G = kImpMqRows / H;
+  static constexpr int N = G * H;                          // MMA N (query rows)
+  static constexpr int kStages = 3;
+  static constexpr uint32_t kTileBytes = kKTileBytesBf16;  // 32 KB
+  static constexpr uint32_t kQBytes = N * kHeadDim * 2;
+  static constexpr uint32_t kStageOff = 0;
+  static constexpr uint32_t kQOff = kStages * kTileBytes;
+  static constexpr uint32_t kHistOff = kQOff + kQBytes;     // [G][kHistBins / 2] words
+  static constexpr uint32_t kDeltaOff = kHistOff + G * (kHistBins / 2) * 4;
+  static constexpr uint32_t kBarOff = kDeltaOff + N * 4;
+  static constexpr uint32_t kBars = 2 * kStages + 5;
+  static constexpr uint32_t kTmemSlotOff = kBarOff + kBars * 8;
+  static constexpr uint32_t kBytes = kTmemSlotOff + 16 + 1024;
+  static constexpr uint32_t kTmemCols = tmem_cols_pow2(2 * N);
+  static_assert(kBytes <= 227 * 1024, "shared memory budget");
+};
+
+}  // namespace
+
+template <int H>
+__global__ void __launch_bounds__(192, 1)
+    importance_mq_kernel(const __grid_constant__ CUtensorMap tmap_k, SelectParams p,
+                         int n_groups) {
+  using L = ImpMqSmem<H>;
+  constexpr int G = L::G, N = L::N;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* stages = smem + L::kStageOff;
+  uint8_t* qs = smem + L::kQOff;
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + L::kHistOff);
+  float* delta_s = reinterpret_cast<float*>(smem + L::kDeltaOff);  // [G][H]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + L::kStages;
+  uint64_t* s_full = bars + 2 * L::kStages;
+  uint64_t* s_free = bars + 2 * L::kStages + 2;
+  uint64_t* mma_done = bars + 2 * L::kStages + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlotOff);
+
+  const int warp = threadIdx.x >> 5;
+  const int split = blockIdx.x;
+  const int grp = blockIdx.y % n_groups, b = blockIdx.y / n_groups;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(s_full + s, 1);
+      mbar_init(s_free + s, 128);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane_id() == 0) prefetch_tmap(&tmap_k);
+  griddep_wait();
+
+  const int t0 = grp * G;
+  const int ntok = min(G, p.n_q - t0);
+  const int Lb = seq_len(p.kv, b, p.n_q, p.status, false);
+  // Token g ranks the keys [0, n_c(g)), n_c(g) = p_g - window + 1; the group's last
+  // token has the longest range.  Tokens with n_c <= k_sel keep everything.
+  const int nc0 = Lb - p.n_q + t0 - p.window + 1;  // n_c of token t0
+  const int nc_last = nc0 + ntok - 1;
+  const int k0 = split * p.chunk2;
+  const int k1 = min(k0 + p.chunk2, nc_last);
+  const bool any_ranked = nc_last > p.k_sel && k0 < k1;
+  const int n_tiles = any_ranked ? (k1 - k0 + kKeyTile - 1) / kKeyTile : 0;
+
+  if (n_tiles > 0) {
+    // Q rows (token g, head h) at row g * H + h, K-major unswizzled; absent tokens zero.
+    for (int e = threadIdx.x; e < N * (kHeadDim / 8); e += blockDim.x) {
+      const int n = e % N, c = e / N;
+      const int g = n / H, h = n % H;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (g < ntok)
+        v = *reinterpret_cast<const uint4*>(
+            p.q + (((size_t)b * p.n_q + t0 + g) * H + h) * kHeadDim + c * 8);
+      *reinterpret_cast<uint4*>(qs + c * (N * 16) + n * 16) = v;
+    }
+    for (int e = threadIdx.x; e < G * (kHistBins / 2); e += blockDim.x) hist_s[e] = 0u;
+    for (int g = 0; g < G; ++g) {
+      if (g < ntok)
+        load_delta(p.lse64 + ((size_t)b * p.n_q + t0 + g) * H, H, delta_s + g * H, nullptr);
+      else
+        for (int h = threadIdx.x; h < H; h += blockDim.x) delta_s[g * H + h] = 0.f;
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  bool ok = true;
+
+  if (n_tiles == 0) {
+    // nothing to rank in this chunk
+  } else if (warp == 0) {
+    // ---------------- TMA producer
+    if (elect_one()) {
+      const uint64_t pol = policy_evict_last();  // the other groups read the same tiles
+      const int row0 = b * p.kv.max_len + k0;
+      int issued = 0;
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        const int s = i % L::kStages;
+        const uint32_t ph = (i / L::kStages) & 1;
+        if (!mbar_wait(empty + s, ph ^ 1)) { ok = false; break; }
+        mbar_arrive_expect_tx(full + s, L::kTileBytes);
+        uint8_t* dst = stages + s * L::kTileBytes;
+        tma_load_2d(dst, &tmap_k, full + s, 0, row0 + i * kKeyTile, pol);
+        tma_load_2d(dst + kBoxBytes, &tmap_k, full + s, 64, row0 + i * kKeyTile, pol);
+        issued = i + 1;
+      }
+      for (int i = issued > L::kStages ? issued - L::kStages : 0; i < issued; ++i)
+        if (!mbar_wait(full + (i % L::kStages), (i / L::kStages) & 1)) ok = false;
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (elect_one()) {
+      const uint32_t idesc = idesc_f16(128, N, true, false, false);
+      const uint32_t q_addr = smem_u32(qs);
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        const int s = i % L::kStages;
+        const uint32_t ph = (i / L::kStages) & 1;
+        const int buf = i & 1;
+        if (!mbar_wait(full + s, ph)) { ok = false; break; }
+        if (!mbar_wait(s_free + buf, ((i >> 1) & 1) ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(stages + s * L::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < kHeadDim / 16; ++kk)
+          mma_f16_ss(tmem_base + buf * N, kmajor_sw128_desc(a_addr, kk),
+                     q_kmajor_desc<N>(q_addr, kk), idesc, kk > 0 ? 1u : 0u);
+        mma_commit(s_full + buf);
+        mma_commit(empty + s);
+      }
+      mma_commit(mma_done);
+      if (!mbar_wait(mma_done, 0)) ok = false;
+    }
+  } else {
+    // ---------------- epilogue: 128 threads, one key each, G tokens per key
+    const int lg = warp & 3;
+    const int t = lg * 32 + (int)lane_id();
+    const float sc = p.sm_scale;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int buf = i & 1;
+      if (ok && !mbar_wait(s_full + buf, (i >> 1) & 1)) ok = false;
+      tc_fence_after();
+      float best[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) best[g] = -INFINITY;
+      const uint32_t taddr = tmem_base + ((uint32_t)(lg * 32) << 16) + buf * N;
+      // Four loads in flight per wait (64 columns at a time).
+#pragma unroll
+      for (int c0 = 0; c0 < N; c0 += 64) {
+        uint32_t r[64];
+#pragma unroll
+        for (int c = 0; c < 64; c += 16)
+          if (c0 + c < N) tmem_ld16(taddr + c0 + c, *reinterpret_cast<uint32_t(*)[16]>(r + c));
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 64; ++e)
+          if (c0 + e < N)
+            best[(c0 + e) / H] =
+                fmaxf(best[(c0 + e) / H], __uint_as_float(r[e]) * sc - delta_s[c0 + e]);
+      }
+      tc_fence_before();
+      mbar_arrive(s_free + buf);
+      const int j = k0 + i * kKeyTile + t;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const int nc_g = nc0 + g;
+        // Tokens past the group's end, or that keep all their keys, are not ranked.
+        const bool ranked = g < ntok && nc_g > p.k_sel;
+        const bool valid = ranked && j < nc_g;
+        if (valid) p.tbuf[((size_t)b * p.n_q + t0 + g) * p.kv.max_len + j] = best[g];
+        const uint32_t bin = valid ? (ordered_key(best[g]) >> kHistShift) : 0xFFFFFFFFu;
+        const unsigned same = __match_any_sync(0xffffffffu, bin);
+        if (valid && (int)lane_id() == __ffs(same) - 1)
+          atomicAdd(hist_s + g * (kHistBins / 2) + (bin >> 1), (uint32_t)__popc(same) << (16 * (bin & 1)));
+      }
+    }
+    named_bar_sync(1, 128);
+    for (int g = 0; g < ntok; ++g) {
+      uint32_t* gh = p.hist + ((size_t)b * p.n_q + t0 + g) * kHistBins;
+      for (int e = t; e < kHistBins / 2; e += 128) {
+        const uint32_t w = hist_s[g * (kHistBins / 2) + e];
+        if (w & 0xffffu) atomicAdd(gh + 2 * e, w & 0xffffu);
+        if (w >> 16) atomicAdd(gh + 2 * e + 1, w >> 16);
+      }
+    }
+  }
+  if (!ok) set_status(p.status, HS2_ERR_DEVICE_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+template <int H>
+static cudaError_t launch_imp_mq_t(const SelectParams& p, const CUtensorMap& tm, int batch,
+                                   int n_groups, cudaStream_t st) {
+  using L = ImpMqSmem<H>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(importance_mq_kernel<H>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  return launch_pdl(importance_mq_kernel<H>, dim3(p.splits2, batch * n_groups), dim3(192),
+                    L::kBytes, st, tm, p, n_groups);
+}
+
+cudaError_t launch_importance_mq(const SelectParams& p, const CUtensorMap& tmap_k, int batch,
+                                 cudaStream_t st) {
+  if (p.chunk2 > kImpMqMaxChunk || p.chunk2 % kKeyTile != 0) return cudaErrorInvalidValue;
+  const int G = kImpMqRows / p.h;
+  const int n_groups = (p.n_q + G - 1) / G;
+  switch (p.h) {
+    case 16: return launch_imp_mq_t<16>(p, tmap_k, batch, n_groups, st);
+    case 32: return launch_imp_mq_t<32>(p, tmap_k, batch, n_groups, st);
+    case 48: return launch_imp_mq_t<48>(p, tmap_k, batch, n_groups, st);
+    case 64: return launch_imp_mq_t<64>(p, tmap_k, batch, n_groups, st);
+    case 128: return launch_imp_mq_t<128>(p, tmap_k, batch, n_groups, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 // ============================================================================
 // The same pass for an FP8 E4M3 cache: raw 128-key tiles by TMA, four conversion
@@ -420,13 +672,16 @@ __global__ void __launch_bounds__(kImpF8Threads, 1)
       float best = -INFINITY;
       const uint32_t taddr = tmem_base + ((uint32_t)(lg * 32) << 16) + buf * H;
 #pragma unroll
-      for (int c = 0; c < H; c += 16) {
-        uint32_t r[16];
-        tmem_ld16(taddr + c, r);
+      for (int c0 = 0; c0 < H; c0 += 64) {  // up to four loads in flight per wait
+        uint32_t r[64];
+#pragma unroll
+        for (int c = 0; c < 64; c += 16)
+          if (c0 + c < H) tmem_ld16(taddr + c0 + c, *reinterpret_cast<uint32_t(*)[16]>(r + c));
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          best = fmaxf(best, __uint_as_float(r[e]) * (qinv_s[c + e] * ks * sc) - delta_s[c + e]);
+        for (int e = 0; e < 64; ++e)
+          if (c0 + e < H)
+            best = fmaxf(best, __uint_as_float(r[e]) * (qinv_s[c0 + e] * ks * sc) - delta_s[c0 + e]);
       }
       tc_fence_before();
       mbar_arrive(s_free + buf);

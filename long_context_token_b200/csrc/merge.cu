@@ -27,6 +27,9 @@ __global__ void __launch_bounds__(kHeadDim * kMergeMaxGroups) merge_splits_kerne
   const float* pml = p.part_ml + (size_t)bq * S * H * 2;
   const float* po = p.part_o + (size_t)bq * S * H * kHeadDim;
   griddep_wait();
+  // The importance pass that may follow takes nothing from this kernel until it exits,
+  // so it may start now.
+  griddep_launch_dependents();
   // The first eight partials of this thread's dimension are requested before the
   // weights are known, so the (m, l) and o loads share one memory round trip.
   const int d = threadIdx.x % kHeadDim, g = threadIdx.x / kHeadDim;

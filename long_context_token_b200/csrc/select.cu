@@ -25,8 +25,8 @@
 namespace hs2 {
 
 __device__ __forceinline__ uint64_t sm100_evict_first_policy() { return sm100::policy_evict_first(); }
-__device__ __forceinline__ uint4 sm100_ld_v4_hint(const void* p, uint64_t pol) {
-  return sm100::ld_global_v4_hint(p, pol);
+__device__ __forceinline__ uint4 sm100_ld_cg_v4_hint(const void* p, uint64_t pol) {
+  return sm100::ld_global_cg_v4_hint(p, pol);
 }
 
 
@@ -83,46 +83,90 @@ __global__ void __launch_bounds__(kThreads) importance_simt_kernel(SelectParams 
     if (hist_s[e]) atomicAdd(gh + e, hist_s[e]);
 }
 
+// Per-head shift delta_h = lse_h - min lse from the full layer's split partials (m in
+// log2 units, l), with the merge's arithmetic: M = max m over non-empty splits,
+// lse = (M + log2 sum_s l_s 2^(m_s - M)) ln 2 in float64.  Loads through L2 only.
+template <int H>
+__device__ __forceinline__ void delta_from_partials(const float* pml, int S, float* delta_s) {
+  __shared__ double lse_s[H];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int h = w; h < H; h += nw) {
+    float M = -INFINITY;
+    for (int s = lane; s < S; s += 32) {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(pml + ((size_t)s * H + h) * 2));
+      if (v.y > 0.f) M = fmaxf(M, v.x);
+    }
+    M = warp_max(M);
+    double Ls = 0.0;
+    if (M != -INFINITY)
+      for (int s = lane; s < S; s += 32) {
+        const float2 v = __ldcg(reinterpret_cast<const float2*>(pml + ((size_t)s * H + h) * 2));
+        if (v.y > 0.f) Ls += (double)v.y * exp2((double)v.x - M);
+      }
+    Ls = warp_sum_d(Ls);
+    if (lane == 0)
+      lse_s[h] = Ls > 0.0 ? ((double)M + log2(Ls)) * 0.69314718055994530942 : -INFINITY;
+  }
+  __syncthreads();
+  if (threadIdx.x < H) {
+    double mn = INFINITY;
+#pragma unroll
+    for (int h = 0; h < H; ++h) mn = fmin(mn, lse_s[h]);
+    delta_s[threadIdx.x] = (float)(lse_s[threadIdx.x] - mn);
+  }
+  __syncthreads();
+}
+
 // 1'. importance from the full layer's stored float32 logits (single-token decode,
-//     16 heads): the same t_j and histogram without reading K again.
+//     16 heads): the same t_j and histogram without reading K again.  This pass does
+//     not use the merge kernel's output (it takes the per-head lse from the partials), so
+//     it waits for the previous grid (the merge, which lets it start as soon as the full
+//     layer is done) only before it exits: the passes after it may read the merge's lse.
+//     Everything it reads was written by the full layer and is loaded through L2.
 constexpr int kSbufChunk = 4096;
 
 template <int H>
 __global__ void __launch_bounds__(kThreads) importance_sbuf_kernel(SelectParams p) {
   __shared__ uint32_t hist_s[kHistBins];
   __shared__ float delta_s[kMaxHeads];
-  griddep_wait();
   const int split = blockIdx.x, bq = blockIdx.y;
   const int b = bq / p.n_q, i = bq % p.n_q;
   const int L = seq_len(p.kv, b, p.n_q, p.status, false);
   const int pos = L - p.n_q + i;
   const int n_c = pos - p.window + 1;
-  if (n_c <= p.k_sel) return;
   const int k0 = split * kSbufChunk;
   const int k1 = min(k0 + kSbufChunk, n_c);
-  if (k0 >= k1) return;
+  if (n_c <= p.k_sel || k0 >= k1) {
+    griddep_wait();
+    return;
+  }
   for (int e = threadIdx.x; e < kHistBins; e += kThreads) hist_s[e] = 0u;
-  load_delta(p.lse64 + (size_t)bq * H, H, delta_s, nullptr);
   const uint64_t pol = sm100_evict_first_policy();
   const float* __restrict__ src = p.sbuf + (size_t)bq * p.kv.max_len * H;
   float* __restrict__ trow = p.tbuf + (size_t)bq * p.kv.max_len;
   const float sc = p.sm_scale;
   // Keys are loaded kBatch at a time, all before the first is used (kBatch x H
-  // floats in flight per thread): one memory round trip per kBatch keys.
+  // floats in flight per thread): one memory round trip per kBatch keys.  The first
+  // batch is requested before the shifts are computed.
   constexpr int kPer = kSbufChunk / kThreads;
   static_assert(kPer * kThreads == kSbufChunk, "chunk is a multiple of the block");
   constexpr int kBatch = 4;
-#pragma unroll 1
-  for (int u0 = 0; u0 < kPer; u0 += kBatch) {
-    uint4 v[kBatch][H / 4];
+  uint4 v[kBatch][H / 4];
+  auto load_batch = [&](int u0) {
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int j = k0 + (u0 + u) * kThreads + threadIdx.x;
 #pragma unroll
       for (int c = 0; c < H / 4; ++c)
-        v[u][c] = j < k1 ? sm100_ld_v4_hint(src + (size_t)j * H + 4 * c, pol)
+        v[u][c] = j < k1 ? sm100_ld_cg_v4_hint(src + (size_t)j * H + 4 * c, pol)
                          : make_uint4(0, 0, 0, 0);
     }
+  };
+  load_batch(0);
+  delta_from_partials<H>(p.part1_ml + (size_t)bq * p.splits1 * H * 2, p.splits1, delta_s);
+#pragma unroll 1
+  for (int u0 = 0; u0 < kPer; u0 += kBatch) {
+    if (u0 > 0) load_batch(u0);
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int j = k0 + (u0 + u) * kThreads + threadIdx.x;
@@ -136,13 +180,15 @@ __global__ void __launch_bounds__(kThreads) importance_sbuf_kernel(SelectParams 
         t = fmaxf(t, __uint_as_float(v[u][c].w) * sc - delta_s[4 * c + 3]);
       }
       trow[j] = t;
-      atomicAdd(&hist_s[ordered_key(t) >> kHistShift], 1u);
+      const uint32_t bin = ordered_key(t) >> kHistShift;
+      atomicAdd(&hist_s[bin], 1u);
     }
   }
   __syncthreads();
   uint32_t* gh = p.hist + (size_t)bq * kHistBins;
   for (int e = threadIdx.x; e < kHistBins; e += kThreads)
     if (hist_s[e]) atomicAdd(gh + e, hist_s[e]);
+  griddep_wait();
 }
 
 cudaError_t launch_importance_sbuf(const SelectParams& p, int bq, cudaStream_t st) {
@@ -164,17 +210,30 @@ struct BoundaryBin {
 // Every CTA of a bq finds the same boundary bin from the global histogram: thread t
 // sums 16 bins, warp 0 turns the 256 sums into counts "above" (a prefix sum from the
 // top bin down), and the thread whose range holds the k-th largest scans its bins.
-__device__ BoundaryBin find_boundary_bin(const uint32_t* gh, int k_eff, float delta_max) {
+constexpr int kBinsPerThread = kHistBins / kThreads;  // 16
+
+__device__ __forceinline__ void load_hist_slice(const uint32_t* gh, uint32_t (&c)[kBinsPerThread]) {
+  const uint4* src = reinterpret_cast<const uint4*>(gh + threadIdx.x * kBinsPerThread);
+#pragma unroll
+  for (int e = 0; e < kBinsPerThread / 4; ++e) {
+    const uint4 v = __ldcg(src + e);
+    c[4 * e] = v.x;
+    c[4 * e + 1] = v.y;
+    c[4 * e + 2] = v.z;
+    c[4 * e + 3] = v.w;
+  }
+}
+
+// c: this thread's 16 bins of the histogram (load_hist_slice), requested early.
+__device__ BoundaryBin find_boundary_bin(const uint32_t (&c)[kBinsPerThread], int k_eff,
+                                         float delta_max) {
   __shared__ uint32_t part[kThreads];  // indexed from the top: part[255 - t]
   __shared__ uint32_t bin_s;
-  constexpr int per = kHistBins / kThreads;  // 16 bins per thread
+  constexpr int per = kBinsPerThread;
   if (threadIdx.x == 0) bin_s = 0u;
-  uint32_t c[per], loc = 0;
+  uint32_t loc = 0;
 #pragma unroll
-  for (int e = 0; e < per; ++e) {
-    c[e] = __ldcg(gh + threadIdx.x * per + e);
-    loc += c[e];
-  }
+  for (int e = 0; e < per; ++e) loc += c[e];
   part[kThreads - 1 - threadIdx.x] = loc;
   __syncthreads();
   if (threadIdx.x < 32) {
@@ -282,6 +341,8 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(SelectParams p
 #pragma unroll
     for (int u = 0; u < kPer; ++u) t[u] = j0 + u < k1 ? __ldcg(trow + j0 + u) : -INFINITY;
   }
+  uint32_t hc[kBinsPerThread];
+  load_hist_slice(p.hist + (size_t)bq * kHistBins, hc);
   __shared__ float dmax_s;
   if (threadIdx.x < 32) {
     double lo = INFINITY, hi = -INFINITY;
@@ -298,7 +359,7 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(SelectParams p
     if (threadIdx.x == 0) dmax_s = (float)(hi - lo);
   }
   __syncthreads();
-  const BoundaryBin bb = find_boundary_bin(p.hist + (size_t)bq * kHistBins, k_eff, dmax_s);
+  const BoundaryBin bb = find_boundary_bin(hc, k_eff, dmax_s);
   if (split == 0 && threadIdx.x == 0) {
     uint32_t* meta = p.selmeta + (size_t)bq * 4;
     meta[0] = bb.bin;
@@ -378,13 +439,26 @@ __device__ __forceinline__ uint32_t warp_slot(bool pred, uint32_t* counter) {
 // *n_gt receives how many selected elements are strictly greater.  Each pass builds a
 // 256-bin shared histogram of the current digit, then warp 0 finds the digit holding
 // the r-th element with a warp-wide prefix sum (lane l owns digits 255-8l .. 248-8l).
+// Keys known to lie in [lo, hi] share the bits above the highest bit where lo and hi
+// differ: those digits are skipped (pass lo = 0, hi = all ones when nothing is known).
 template <typename KeyT, int KBITS, typename KeyFn, typename PredFn>
-__device__ KeyT block_kth_largest(int n, int r, KeyFn key, PredFn pred, uint32_t* n_gt) {
+__device__ KeyT block_kth_largest(int n, int r, KeyFn key, PredFn pred, uint32_t* n_gt,
+                                  KeyT lo = KeyT(0), KeyT hi = ~KeyT(0)) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t sh_digit, sh_rem, sh_gt;
-  KeyT prefix = 0, mask = 0;
+  const KeyT diff = lo ^ hi;
+  if (diff == 0) {  // every key equals lo
+    if (threadIdx.x == 0) *n_gt = 0u;
+    __syncthreads();
+    return lo;
+  }
+  int top = KBITS - 1;
+  while (!((diff >> top) & 1)) --top;
+  const int start = (top / 8) * 8;  // lowest bit of the highest digit that varies
+  KeyT mask = start + 8 >= KBITS ? KeyT(0) : ~((KeyT(1) << (start + 8)) - 1);
+  KeyT prefix = lo & mask;
   uint32_t rem = (uint32_t)r, gt = 0;
-  for (int shift = KBITS - 8; shift >= 0; shift -= 8) {
+  for (int shift = start; shift >= 0; shift -= 8) {
     for (int e = threadIdx.x; e < 256; e += blockDim.x) hist[e] = 0u;
     if (threadIdx.x == 0) {
       sh_digit = 0u;
@@ -511,10 +585,35 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
   auto cand_t = [&](uint32_t e) { return cand_smem ? cts[e] : __ldcg(ct + e); };
   auto cand_j = [&](uint32_t e) { return cand_smem ? cjs[e] : __ldcg(cj + e); };
 
-  // tau: the need-th largest float32 key among the candidates.
+  // tau: the need-th largest float32 key among the candidates (whose keys share their
+  // high bits: the radix passes start below the bits that min and max have in common).
+  __shared__ uint32_t kmin_s, kmax_s;
+  if (threadIdx.x == 0) {
+    kmin_s = 0xffffffffu;
+    kmax_s = 0u;
+  }
+  __syncthreads();
+  {
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (uint32_t e = threadIdx.x; e < n_cand; e += blockDim.x) {
+      const uint32_t k = ordered_key(cand_t(e));
+      lo = min(lo, k);
+      hi = max(hi, k);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if ((threadIdx.x & 31) == 0) {
+      atomicMin(&kmin_s, lo);
+      atomicMax(&kmax_s, hi);
+    }
+  }
+  __syncthreads();
   const uint32_t tau_key = block_kth_largest<uint32_t, 32>(
       (int)n_cand, need, [&](int e) { return ordered_key(cand_t((uint32_t)e)); },
-      [](int) { return true; }, &gt_s);
+      [](int) { return true; }, &gt_s, kmin_s, kmax_s);
   const float tau = key_to_float(tau_key);
   const float hi_b = tau + eps, lo_b = tau - eps;
 
@@ -640,21 +739,16 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
     }
   }
   __syncthreads();
-  // The forced recent window [p - window + 1, p].
-  const uint32_t n_top = n_sel;
-  for (int j = n_c + threadIdx.x; j <= pos; j += blockDim.x) {
-    const uint32_t slot = n_top + (uint32_t)(j - n_c);
-    if (slot < (uint32_t)kMaxIdxWidth) sel[slot] = j;
-  }
-  __syncthreads();
-  // Ascending order of the n selected (distinct) positions: counting sort on the
-  // position's high bits into 1024 buckets, then each key's rank inside its bucket.
-  const int n = (int)min(n_top + (uint32_t)(pos - n_c + 1), (uint32_t)kMaxIdxWidth);
-  int shift = 0;
-  while ((pos >> shift) >= kBuckets) ++shift;
+  // Every top key lies in [0, n_c) and the forced recent window [n_c, p] lies above
+  // them, already in order: only the top keys are sorted.  Counting sort on the bucket
+  // floor(position * kBuckets / n_c) (monotone; about one key per bucket), then each
+  // key's rank inside its bucket.
+  const int n = (int)min(n_sel, (uint32_t)kMaxIdxWidth);
+  const float bscale = (float)kBuckets / (float)n_c;
+  auto bucket_of = [&](int v) { return min(kBuckets - 1, (int)((float)v * bscale)); };
   for (int e = threadIdx.x; e < kBuckets; e += blockDim.x) bucket[e] = 0u;
   __syncthreads();
-  for (int e = threadIdx.x; e < n; e += blockDim.x) atomicAdd(&bucket[sel[e] >> shift], 1u);
+  for (int e = threadIdx.x; e < n; e += blockDim.x) atomicAdd(&bucket[bucket_of(sel[e])], 1u);
   __syncthreads();
   if (threadIdx.x < 32) {  // exclusive prefix over the buckets, 32 per lane
     const int lane = threadIdx.x;
@@ -677,18 +771,21 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
   __syncthreads();
   for (int e = threadIdx.x; e < n; e += blockDim.x) {
     const int v = sel[e];
-    tmp[atomicAdd(&bucket[v >> shift], 1u)] = v;  // bucket[b] advances to b's end
+    tmp[atomicAdd(&bucket[bucket_of(v)], 1u)] = v;  // bucket[b] advances to b's end
   }
   __syncthreads();
   for (int e = threadIdx.x; e < n; e += blockDim.x) {
     const int v = tmp[e];
-    const uint32_t beg = bucket_beg[v >> shift], end = bucket[v >> shift];
+    const int bk = bucket_of(v);
+    const uint32_t beg = bucket_beg[bk], end = bucket[bk];
     uint32_t rank = 0;
     for (uint32_t x = beg; x < end; ++x) rank += tmp[x] < v;
     sel[beg + rank] = v;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < width; e += blockDim.x) out[e] = e < n ? sel[e] : -1;
+  const int n_win = pos - n_c + 1;
+  for (int e = threadIdx.x; e < width; e += blockDim.x)
+    out[e] = e < n ? sel[e] : (e < n + n_win ? n_c + (e - n) : -1);
   // Leave this query's histogram and counters at zero for the next selection.
   uint32_t* gh = p.hist + (size_t)bq * kHistBins;
   for (int e = threadIdx.x; e < kHistBins; e += blockDim.x) gh[e] = 0u;

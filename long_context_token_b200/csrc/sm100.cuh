@@ -126,6 +126,15 @@ __device__ __forceinline__ void st_global_v4_hint(void* p, uint4 v, uint64_t pol
                : "memory");
 }
 // 16-byte global load with an L2 eviction-priority policy.
+// The same through L2 only (no L1 allocation): coherent with writes made by a grid that
+// completed before this one started, even without a grid-dependency wait.
+__device__ __forceinline__ uint4 ld_global_cg_v4_hint(const void* p, uint64_t policy) {
+  uint4 v;
+  asm volatile("ld.global.cg.L2::cache_hint.v4.b32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(policy));
+  return v;
+}
 __device__ __forceinline__ uint4 ld_global_v4_hint(const void* p, uint64_t policy) {
   uint4 v;
   asm volatile("ld.global.L2::cache_hint.v4.b32 {%0, %1, %2, %3}, [%4], %5;"

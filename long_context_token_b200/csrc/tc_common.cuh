@@ -98,6 +98,38 @@ __device__ __forceinline__ uint64_t vt_mnmajor_sw128_desc(uint32_t tile_addr, in
                           sm100::kSwizzle128B);
 }
 
+// Gather of one tile (index entries [e0, e0 + 128), those at or past e_end absent) into
+// the 128-byte-swizzled layout that TMA writes: 16-byte chunk c of row r at box c / 8,
+// byte r * 128 + ((c mod 8) xor (r mod 8)) * 16.  K and V rows by cp.async, absent or
+// out-of-range entries zero-filled (an out-of-range one also sets the status word).
+// The 128 x CHUNKS work items are spread over nthreads threads starting at tid; each
+// thread still has to wait for its copies (cp.async.wait_all).  A null kb (vb) skips
+// the K (V) rows.
+template <int CHUNKS, uint32_t BOX>
+__device__ __forceinline__ void gather_tile_rows(uint32_t kdst, uint32_t vdst, const uint8_t* kb,
+                                                 const uint8_t* vb, const int32_t* idx_row,
+                                                 int e0, int e_end, int Lb, size_t row_base,
+                                                 uint32_t* status, int tid, int nthreads) {
+  constexpr uint32_t kRowBytes = CHUNKS * 16;
+  for (int w = tid; w < kKeyTile * CHUNKS; w += nthreads) {
+    const int r = w / CHUNKS, c = w % CHUNKS, e = e0 + r;
+    int j = -1;
+    if (e < e_end) {
+      j = __ldg(idx_row + e);
+      if (j < 0 || j >= Lb) {
+        if (j != -1 && c == 0) set_status(status, HS2_ERR_INDEX_OUT_OF_RANGE);
+        j = -1;
+      }
+    }
+    const size_t off = j >= 0 ? (row_base + (size_t)j) * kRowBytes : 0;
+    const uint32_t nb = j >= 0 ? 16u : 0u;
+    const uint32_t at = (uint32_t)(c >> 3) * BOX + (uint32_t)r * 128u +
+                        ((uint32_t)((c & 7) ^ (r & 7)) << 4);
+    if (kb) sm100::cp_async_16(kdst + at, kb + off + c * 16, nb);
+    if (vb) sm100::cp_async_16(vdst + at, vb + off + c * 16, nb);
+  }
+}
+
 // Softmax reference usable in 2^(x - m): a reference of -inf (no key seen yet, so
 // every x is -inf too) becomes 0, which gives p = 0 instead of NaN.
 __device__ __forceinline__ float finite_ref(float m) { return m == -INFINITY ? 0.f : m; }
@@ -197,6 +229,10 @@ inline bool mq_eligible(int n_q, int h) {
   return (h == 16 || h == 32 || h == 48 || h == 64 || h == 128) && (n_q >= 2 || h > 64);
 }
 cudaError_t launch_importance_tc(const SelectParams& p, const CUtensorMap& tmap_k, int bq,
+                                 cudaStream_t st);
+// Importance pass for the several-token shapes (bf16): G = 128 / h tokens per CTA;
+// p.chunk2 a multiple of 128 below 65536.
+cudaError_t launch_importance_mq(const SelectParams& p, const CUtensorMap& tmap_k, int batch,
                                  cudaStream_t st);
 cudaError_t launch_importance_fp8(const SelectParams& p, const CUtensorMap& tmap_k, int bq,
                                   cudaStream_t st);
