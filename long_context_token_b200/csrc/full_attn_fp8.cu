@@ -435,8 +435,8 @@ __global__ void __launch_bounds__(kFp8Threads, (GATHER && H <= 16) ? 2 : 1)
           const int h0 = c * 8 + 2 * e;
           // A head whose reference is still -inf has seen no key: its p is 0 (not
           // 2^(-inf - -inf)), so a leading all-padding tile leaves O and l at zero.
-          const float p0 = exp2f(x[h0] - finite_ref(mref_s[h0]));
-          const float p1 = exp2f(x[h0 + 1] - finite_ref(mref_s[h0 + 1]));
+          const float p0 = ex2_ftz(x[h0] - finite_ref(mref_s[h0]));
+          const float p1 = ex2_ftz(x[h0 + 1] - finite_ref(mref_s[h0 + 1]));
           l[h0] += p0;
           l[h0 + 1] += p1;
           const __half2 v2 = __floats2half2_rn(p0 * vs, p1 * vs);

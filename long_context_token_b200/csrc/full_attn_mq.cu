@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kMqThreads, 1)
         if (ok && !mbar_wait(s_full + sb, (i >> 1) & 1)) ok = false;
         if (named_bar_or(3, kMqSoftmax, !ok)) ok = false;
         tc_fence_after();
-        float x[KH];
+        float x[KH];  // raw logits s (the log2-domain value is s * c2)
         {
           uint32_t v[KH];
 #pragma unroll
@@ -270,17 +270,20 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                       *reinterpret_cast<uint32_t(*)[16]>(v + c));
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < KH; ++e) x[e] = __uint_as_float(v[e]) * c2;
+          for (int e = 0; e < KH; ++e) x[e] = __uint_as_float(v[e]);
         }
         tc_fence_before();
         mbar_arrive(s_free + sb);
         const int jb = k0 + i * kMqKeys + half * KH;
+        if (jb + KH > kend) {  // only tiles at the chunk end or the causal edge are masked
+#pragma unroll
+          for (int c = 0; c < KH; ++c)
+            if (jb + c >= kend) x[c] = -INFINITY;
+        }
         float tmax = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < KH; ++c) {
-          if (jb + c >= kend) x[c] = -INFINITY;
-          tmax = fmaxf(tmax, x[c]);
-        }
+        for (int c = 0; c < KH; ++c) tmax = fmaxf(tmax, x[c]);
+        tmax *= c2;  // c2 > 0: the max of the scaled logits
         // Row max over both halves (slots alternate by tile so that a fast thread
         // cannot overwrite a value its partner has not read yet).
         float* rt = red + (size_t)(i & 1) * 2 * kMqRows;
@@ -318,20 +321,16 @@ __global__ void __launch_bounds__(kMqThreads, 1)
         if (ok && i >= 2 && !mbar_wait(p_free + sb, ((i >> 1) & 1) ^ 1)) ok = false;
         uint8_t* phi = ps + (2 * sb) * L::kPBytes;
         uint8_t* plo = phi + L::kPBytes;
-        const float mr = finite_ref(mref);
+        const float nmr = -finite_ref(mref);
 #pragma unroll
         for (int c = 0; c < KH / 8; ++c) {
           uint32_t hw[4], lw[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float p0 = exp2f(x[c * 8 + 2 * e] - mr);
-            const float p1 = exp2f(x[c * 8 + 2 * e + 1] - mr);
+            const float p0 = ex2_ftz(fmaf(x[c * 8 + 2 * e], c2, nmr));
+            const float p1 = ex2_ftz(fmaf(x[c * 8 + 2 * e + 1], c2, nmr));
             l += p0 + p1;
-            const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
-            const float2 hf = __bfloat1622float2(hi);
-            const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
-            hw[e] = *reinterpret_cast<const uint32_t*>(&hi);
-            lw[e] = *reinterpret_cast<const uint32_t*>(&lo);
+            split_bf16_hi_lo(p0, p1, hw[e], lw[e]);
           }
           const int chunk = half * (KH / 8) + c;  // 8-key chunk of the tile
           *reinterpret_cast<uint4*>(phi + chunk * (kMqRows * 16) + r * 16) =

@@ -370,15 +370,11 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
             const int h0 = c * 8 + 2 * e;
             // A head whose reference is still -inf has seen no key: its p is 0 (not
             // 2^(-inf - -inf)), so a leading all-padding tile leaves O and l at zero.
-            const float p0 = exp2f(x[h0] - finite_ref(mref_s[h0]));
-            const float p1 = exp2f(x[h0 + 1] - finite_ref(mref_s[h0 + 1]));
+            const float p0 = ex2_ftz(x[h0] - finite_ref(mref_s[h0]));
+            const float p1 = ex2_ftz(x[h0 + 1] - finite_ref(mref_s[h0 + 1]));
             l[h0] += p0;
             l[h0 + 1] += p1;
-            const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
-            const float2 hf = __bfloat1622float2(hi);
-            const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
-            hw[e] = *reinterpret_cast<const uint32_t*>(&hi);
-            lw[e] = *reinterpret_cast<const uint32_t*>(&lo);
+            split_bf16_hi_lo(p0, p1, hw[e], lw[e]);
           }
           *reinterpret_cast<uint4*>(phi + c * (kKeyTile * 16) + t * 16) =
               make_uint4(hw[0], hw[1], hw[2], hw[3]);

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include "hs2_internal.cuh"
@@ -128,6 +129,25 @@ __device__ __forceinline__ void gather_tile_rows(uint32_t kdst, uint32_t vdst, c
     if (kb) sm100::cp_async_16(kdst + at, kb + off + c * 16, nb);
     if (vb) sm100::cp_async_16(vdst + at, vb + off + c * 16, nb);
   }
+}
+
+// 2^x with the hardware approximation (relative error about 2^-22), results below the
+// normal range flushed to zero; 2^-inf = 0.
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// p0, p1 -> bf16 pairs hi, lo with hi + lo = p to about 16 bits: hi keeps the top 16
+// bits of each float (truncation: byte permute), lo = p - hi exactly in float32, then
+// rounded to bf16.  Element order as __floats2bfloat162_rn (p0 in the low half).
+__device__ __forceinline__ void split_bf16_hi_lo(float p0, float p1, uint32_t& hi, uint32_t& lo) {
+  const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+  hi = __byte_perm(b0, b1, 0x7632);
+  const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0 - __uint_as_float(b0 & 0xffff0000u),
+                                                  p1 - __uint_as_float(b1 & 0xffff0000u));
+  lo = *reinterpret_cast<const uint32_t*>(&l2);
 }
 
 // Softmax reference usable in 2^(x - m): a reference of -inf (no key seen yet, so
