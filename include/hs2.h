@@ -137,7 +137,13 @@ HS2_API hs2_status hs2_select(const void* q, int n_q, int h_q, const hs2_kv* kv,
  *             outside [0, lens[b]) is skipped and sets HS2_ERR_INDEX_OUT_OF_RANGE.
  *   out       device float32 [batch][n_q][h_q][128]; a row whose set is empty gets 0.
  * idx_width in [1, 4096]; the workspace must come from hs2_workspace_bytes with
- * window + k_sel >= idx_width. */
+ * window + k_sel >= idx_width.
+ * Overlap: the layer's kernel may start while the previous kernel on the stream is
+ * still finishing when that kernel is this library's (programmatic dependent launch);
+ * it reads q_layer, idx and the cache right away and waits for that kernel to end only
+ * before writing `out`.  No library call writes those inputs except hs2_select /
+ * hs2_full_attn_select, which complete the index set before the next kernel may start.
+ * After any other kernel (not this library's) the layer starts when it has ended. */
 HS2_API hs2_status hs2_sparse_attn(const void* q_layer, int n_q, int h_q, const hs2_kv* kv,
                            const int32_t* idx, int idx_width, float sm_scale, float* out,
                            void* workspace, size_t ws_bytes, hs2_stream_t stream);

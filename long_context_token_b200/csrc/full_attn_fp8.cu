@@ -177,7 +177,10 @@ __global__ void __launch_bounds__(kFp8Threads, (GATHER && H <= 16) ? 2 : 1)
     prefetch_tmap(&tmap_k);
     prefetch_tmap(&tmap_v);
   }
-  griddep_wait();
+  // A sparse layer waits for the previous grid only before writing its output (see the
+  // bf16 kernel: nothing it reads is written by the previous kernel of this library).
+  const bool defer_wait = GATHER && p.out != nullptr;
+  if (!defer_wait) griddep_wait();
 
   const int Lb = seq_len(p.kv, b, p.n_q, p.status, !GATHER && split == 0 && qi == 0);
   const int pos = Lb - p.n_q + qi;
@@ -192,7 +195,7 @@ __global__ void __launch_bounds__(kFp8Threads, (GATHER && H <= 16) ? 2 : 1)
   auto entry_row = [&](int e) -> long long {
     if (e >= k1) return -1;
     if (!GATHER) return (long long)(row_base + e);
-    const int j = __ldg(idx_row + e);
+    const int j = __ldcg(idx_row + e);  // through L2: may have been written by the previous grid
     return (j >= 0 && j < Lb) ? (long long)(row_base + j) : -1;
   };
   bool ok = true;
@@ -479,6 +482,7 @@ __global__ void __launch_bounds__(kFp8Threads, (GATHER && H <= 16) ? 2 : 1)
     // keeps each CTA's shared memory alive until the others have read it.
     __syncwarp();
     cluster_sync();
+    griddep_wait();  // the previous grid is done before this layer writes its output
     cluster_merge_row<H>(smem, p.splits1, p.out + (size_t)bq * H * kHeadDim);
     __syncwarp();
     cluster_sync();

@@ -127,7 +127,13 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
     prefetch_tmap(&tmap_k);
     prefetch_tmap(&tmap_v);
   }
-  griddep_wait();
+  // A sparse layer (gather mode with the on-chip merge) reads nothing that the previous
+  // kernel of this library writes before letting its dependents start (the selection
+  // publishes the index set first; a sparse layer writes only its own output): it waits
+  // for the previous grid only before writing its output, so its gathers overlap the
+  // previous kernel's tail.  Index entries are read through L2.
+  const bool defer_wait = GATHER && p.out != nullptr;
+  if (!defer_wait) griddep_wait();
 
   const int Lb = seq_len(p.kv, b, p.n_q, p.status, !GATHER && split == 0 && qi == 0);
   const int pos = Lb - p.n_q + qi;
@@ -320,7 +326,7 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
         const int j = k0 + i * kKeyTile + t;
         bool valid = j < k1;
         if (GATHER && valid) {
-          const int pj = __ldg(idx_row + j);
+          const int pj = __ldcg(idx_row + j);
           valid = pj >= 0 && pj < Lb;
         }
         bool over = false;
@@ -429,6 +435,7 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
     // keeps each CTA's shared memory alive until the others have read it.
     __syncwarp();
     cluster_sync();
+    griddep_wait();  // the previous grid is done before this layer writes its output
     cluster_merge_row<H>(smem, p.splits1, p.out + (size_t)bq * H * kHeadDim);
     __syncwarp();
     cluster_sync();

@@ -550,6 +550,7 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
   int32_t* out = p.idx + (size_t)bq * width;
   if (n_c <= p.k_sel) {
     for (int e = threadIdx.x; e < width; e += blockDim.x) out[e] = e <= pos ? e : -1;
+    __threadfence();  // visible before the CTA counts as done for the next kernel
     return;
   }
   // Loads that depend on nothing but the previous pass, issued together: the counts,
@@ -786,6 +787,11 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
   const int n_win = pos - n_c + 1;
   for (int e = threadIdx.x; e < width; e += blockDim.x)
     out[e] = e < n ? sel[e] : (e < n + n_win ? n_c + (e - n) : -1);
+  // The index set is complete and visible: the next kernel (a sparse layer, which reads
+  // it without waiting for this grid to end) may start.
+  __threadfence();
+  __syncthreads();
+  griddep_launch_dependents();
   // Leave this query's histogram and counters at zero for the next selection.
   uint32_t* gh = p.hist + (size_t)bq * kHistBins;
   for (int e = threadIdx.x; e < kHistBins; e += blockDim.x) gh[e] = 0u;

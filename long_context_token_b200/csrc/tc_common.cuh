@@ -116,7 +116,7 @@ __device__ __forceinline__ void gather_tile_rows(uint32_t kdst, uint32_t vdst, c
     const int r = w / CHUNKS, c = w % CHUNKS, e = e0 + r;
     int j = -1;
     if (e < e_end) {
-      j = __ldg(idx_row + e);
+      j = __ldcg(idx_row + e);  // through L2: may have been written by the previous grid
       if (j < 0 || j >= Lb) {
         if (j != -1 && c == 0) set_status(status, HS2_ERR_INDEX_OUT_OF_RANGE);
         j = -1;
