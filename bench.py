@@ -39,6 +39,31 @@ LAUNCHES_PER_STEP_SELECT = 3    # importance+histogram, compaction, exact finish
 LAUNCHES_PER_SPARSE = 1         # gather attention with the split merge on chip (cluster)
 
 
+# DRAM bytes (read + write) of one full-layer launch, from an ncu capture of the same
+# kernel (dram__bytes_read.sum + dram__bytes_write.sum) on the first 2 of the 8
+# sequences, scaled by sequences (the traffic is per sequence); see profiles/.
+NCU_TRAFFIC = {
+    2: {"bytes": 4 * (134_288_128 + 786_304), "kernel": "full_attn_tc_kernel<16, 0>",
+        "capture": "2 x 131072 keys, scaled x4"},
+}
+
+
+def roofline_of(w, ab, full_s, peaks, peak_kind) -> dict:
+    """Roofline of the dominant kernel (the full layer, measured with its split merge):
+    HBM-bound for one query token per sequence (16-64 flop per byte), tensor-bound for
+    several tokens per sequence (each K/V tile serves 128/h tokens)."""
+    if w.n_q > 1:
+        achieved = ab["full_flops"] / full_s / 1e12
+        peak = float(peaks["bf16_tflops"])
+        return {"bound": "tensor", "kernel": "full_attn_mq (several-token flash attention)",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_kind": peak_kind + " bf16 burst", "alg_flops_per_launch": ab["full_flops"]}
+    achieved = ab["full"] / full_s / 1e9
+    peak = float(peaks["hbm_gbs"])
+    return {"bound": "hbm", "kernel": "full_attn (split-K flash-decode)", "achieved": achieved,
+            "peak": peak, "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind}
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -86,8 +111,12 @@ def alg_bytes(w: workloads.Workload, lens) -> dict:
     full = 2 * ctx_rows * row + q_bytes + out_bytes
     idx_bytes = w.batch * w.n_q * width * 4
     sparse = 2 * sel_rows * row + idx_bytes + q_bytes + out_bytes
+    # Dense work of the full layer: Q.K^T and P.V over every visible (row, key) pair,
+    # 2 * 128 flops each (the several-token case is bound by these, not by bytes).
+    vis = sum(int(L) - w.n_q + i + 1 for L in lens for i in range(w.n_q))
+    full_flops = 2 * 2 * d * w.h_q * vis
     return dict(full=full, step=full + idx_bytes + w.n_sparse * sparse, sparse=sparse,
-                kv_once=2 * ctx_rows * row)
+                kv_once=2 * ctx_rows * row, full_flops=full_flops)
 
 
 class ClockSampler:
@@ -414,7 +443,6 @@ def main():
     peaks, peak_kind = measured_peaks()
     hbm_peak = float(peaks["hbm_gbs"])
     full_avg = statistics.mean(full_ms) / 1e3
-    achieved = ab["full"] / full_avg / 1e9
     value = whole_job_rate(world, args.steps, total_ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -429,10 +457,13 @@ def main():
                      "step_p10": float(np.percentile(replay_ms, 10)),
                      "step_p50": float(np.percentile(replay_ms, 50)),
                      "step_p90": float(np.percentile(replay_ms, 90))},
-        "roofline": {"bound": "hbm", "kernel": "full_attn (split-K flash-decode)",
-                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "peak_kind": peak_kind,
-                     "alg_bytes_per_launch": ab["full"], "traffic": None},
+        "roofline": roofline_of(w, ab, full_avg, peaks, peak_kind) | {
+                     "alg_bytes_per_launch": ab["full"],
+                     "traffic": (NCU_TRAFFIC[args.workload]["bytes"]
+                                 if args.workload in NCU_TRAFFIC and args.batch is None else None),
+                     "traffic_source": (NCU_TRAFFIC[args.workload]
+                                        if args.workload in NCU_TRAFFIC and args.batch is None
+                                        else None)},
         "gpu_launches": args.steps * (LAUNCHES_PER_STEP_FULL + LAUNCHES_PER_STEP_SELECT
                                       + w.n_sparse * LAUNCHES_PER_SPARSE),
         "clocks": clk.summary(),

@@ -36,7 +36,13 @@ namespace {
 
 constexpr float kLog2eF8 = 1.4426950408889634f;
 constexpr float kRescaleAtF8 = 8.0f;
-constexpr int kFp8Threads = 320;
+// Conversion warps: eight (four for K rows, four for V rows, converting in parallel on
+// their own barriers) up to 32 heads; four (each thread a K row, then a V row) above,
+// where the softmax registers leave no room for more threads.
+template <int H>
+__host__ __device__ constexpr int fp8_conv_warps() { return H <= 32 ? 8 : 4; }
+template <int H>
+__host__ __device__ constexpr int fp8_threads() { return 192 + 32 * fp8_conv_warps<H>(); }
 constexpr uint32_t kRawTile = 16384;    // 128 keys x 128 E4M3 codes
 constexpr uint32_t kConvTile = 32768;   // 128 keys x 128 f16 (two 64-column boxes)
 
@@ -110,7 +116,7 @@ __device__ __forceinline__ void block_max_heads_f8(const float (&v)[H], float* r
 }  // namespace
 
 template <int H, bool GATHER>
-__global__ void __launch_bounds__(kFp8Threads, (GATHER && H <= 16) ? 2 : 1)
+__global__ void __launch_bounds__(fp8_threads<H>(), 1)
     full_attn_fp8_kernel(const __grid_constant__ CUtensorMap tmap_k,
                          const __grid_constant__ CUtensorMap tmap_v, FullParams p) {
   using L = Fp8Smem<H, GATHER>;
@@ -315,23 +321,30 @@ __global__ void __launch_bounds__(kFp8Threads, (GATHER && H <= 16) ? 2 : 1)
     }
   } else if (warp >= 6) {
     // ------------------------------------------------------------ conversion
-    const int t = threadIdx.x - 192;  // row of the tile
+    const int ct = threadIdx.x - 192;
+    const int t = ct & (kKeyTile - 1);  // row of the tile
+    constexpr bool kSplit = fp8_conv_warps<H>() == 8;
+    const bool do_k = !kSplit || ct < kKeyTile, do_v = !kSplit || ct >= kKeyTile;
     for (int i = 0; i < n_tiles; ++i) {
       const int s = i % R;
       const bool valid = entry_row(k0 + i * kKeyTile + t) >= 0;
-      if (ok && !mbar_wait(kr_full + s, (i / R) & 1)) ok = false;
-      if (ok && !mbar_wait(kc_empty, (i & 1) ^ 1)) ok = false;
-      convert_row(kraw + s * kRawTile, kconv, t, valid);
-      fence_proxy_async_smem();
-      mbar_arrive(kc_full);
-      mbar_arrive(kr_empty + s);
-      const int vb = i % L::kVConv;
-      if (ok && !mbar_wait(vr_full + s, (i / R) & 1)) ok = false;
-      if (ok && !mbar_wait(vc_empty + vb, ((i / L::kVConv) & 1) ^ 1)) ok = false;
-      convert_row(vraw + s * kRawTile, vconv + vb * kConvTile, t, valid);
-      fence_proxy_async_smem();
-      mbar_arrive(vc_full + vb);
-      mbar_arrive(vr_empty + s);
+      if (do_k) {
+        if (ok && !mbar_wait(kr_full + s, (i / R) & 1)) ok = false;
+        if (ok && !mbar_wait(kc_empty, (i & 1) ^ 1)) ok = false;
+        convert_row(kraw + s * kRawTile, kconv, t, valid);
+        fence_proxy_async_smem();
+        mbar_arrive(kc_full);
+        mbar_arrive(kr_empty + s);
+      }
+      if (do_v) {
+        const int vb = i % L::kVConv;
+        if (ok && !mbar_wait(vr_full + s, (i / R) & 1)) ok = false;
+        if (ok && !mbar_wait(vc_empty + vb, ((i / L::kVConv) & 1) ^ 1)) ok = false;
+        convert_row(vraw + s * kRawTile, vconv + vb * kConvTile, t, valid);
+        fence_proxy_async_smem();
+        mbar_arrive(vc_full + vb);
+        mbar_arrive(vr_empty + s);
+      }
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -505,13 +518,14 @@ static cudaError_t launch_fp8_t(FullParams p, const CUtensorMap& tk, const CUten
     cudaError_t e =
         cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e != cudaSuccess) return e;
-    max_cluster = GATHER ? largest_cluster(kernel, dim3(kFp8Threads), L::kBytes) : 1;
+    max_cluster = GATHER ? largest_cluster(kernel, dim3(fp8_threads<H>()), L::kBytes) : 1;
     if (max_cluster < 1) return cudaErrorLaunchOutOfResources;
   }
   if (!GATHER)
-    return launch_pdl(kernel, dim3(p.splits1, bq), dim3(kFp8Threads), L::kBytes, st, tk, tv, p);
+    return launch_pdl(kernel, dim3(p.splits1, bq), dim3(fp8_threads<H>()), L::kBytes, st, tk, tv,
+                      p);
   plan_gather_cluster(p.idx_width, max_cluster, &p.splits1, &p.chunk1);
-  return launch_pdl_cluster(kernel, dim3(p.splits1, bq), dim3(kFp8Threads), L::kBytes, p.splits1,
+  return launch_pdl_cluster(kernel, dim3(p.splits1, bq), dim3(fp8_threads<H>()), L::kBytes, p.splits1,
                             st, tk, tv, p);
 }
 

@@ -278,6 +278,51 @@ __device__ __forceinline__ int seq_len(const KvView& kv, int b, int n_q, uint32_
   return L;
 }
 
+// Adds a CTA's shared-memory histogram of selection keys (kHistBins bins) to its query's
+// global one, skipping every bin below the bin of the CTA's own k-th largest key: the
+// k-th largest key over all of the query's CTAs is at least each CTA's, and the boundary
+// search only reads bins from the top down to the bin of that key.  (If the CTA holds
+// fewer than k keys every non-empty bin is added.)  Threads [tid0, tid0 + NT) call it
+// together; `sync` is a barrier over exactly those threads; `red` is NT + 1 words of
+// shared scratch.
+template <int NT, typename Sync>
+__device__ __forceinline__ void flush_hist_top(const uint32_t* hist_s, uint32_t* gh, int k,
+                                               int tid, uint32_t* red, Sync sync) {
+  constexpr int kPer = kHistBins / NT;  // bins per thread, thread i from the top
+  static_assert(kPer * NT == kHistBins && NT % 32 == 0, "whole warps, whole bins");
+  const int hi_bin = kHistBins - 1 - tid * kPer;  // this thread's bins: hi_bin down
+  uint32_t loc = 0;
+#pragma unroll 8
+  for (int u = 0; u < kPer; ++u) loc += hist_s[hi_bin - u];
+  // Exclusive prefix from the top over the threads: warp scan, then the warp totals.
+  const int lane = tid & 31, w = tid >> 5;
+  uint32_t incl = loc;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  if (lane == 31) red[w] = incl;
+  if (tid == 0) red[NT] = 0u;  // lowest bin to add (0: all)
+  sync();
+  uint32_t above = incl - loc;
+  for (int ww = 0; ww < w; ++ww) above += red[ww];
+  if (above < (uint32_t)k && (uint32_t)k <= above + loc) {
+    uint32_t cum = above;
+    for (int u = 0; u < kPer; ++u) {
+      cum += hist_s[hi_bin - u];
+      if (cum >= (uint32_t)k) {
+        red[NT] = (uint32_t)(hi_bin - u);
+        break;
+      }
+    }
+  }
+  sync();
+  const int lowest = (int)red[NT];
+  for (int e = lowest + tid; e < kHistBins; e += NT)
+    if (hist_s[e]) atomicAdd(gh + e, hist_s[e]);
+}
+
 #endif  // __CUDACC__
 
 }  // namespace hs2

@@ -184,9 +184,9 @@ __global__ void __launch_bounds__(192, 1)
       if (valid && (int)lane_id() == __ffs(grp) - 1) atomicAdd(hist_s + bin, __popc(grp));
     }
     named_bar_sync(1, 128);
-    uint32_t* gh = p.hist + (size_t)bq * kHistBins;
-    for (int e = t; e < kHistBins; e += 128)
-      if (hist_s[e]) atomicAdd(gh + e, hist_s[e]);
+    __shared__ uint32_t flush_red[128 + 1];
+    flush_hist_top<128>(hist_s, p.hist + (size_t)bq * kHistBins, p.k_sel, t, flush_red,
+                        [] { named_bar_sync(1, 128); });
   }
   if (!ok) set_status(p.status, HS2_ERR_DEVICE_TIMEOUT);
   tc_fence_before();
@@ -693,9 +693,9 @@ __global__ void __launch_bounds__(kImpF8Threads, 1)
       if (valid && (int)lane_id() == __ffs(grp) - 1) atomicAdd(hist_s + bin, __popc(grp));
     }
     named_bar_sync(1, 128);
-    uint32_t* gh = p.hist + (size_t)bq * kHistBins;
-    for (int e = t; e < kHistBins; e += 128)
-      if (hist_s[e]) atomicAdd(gh + e, hist_s[e]);
+    __shared__ uint32_t flush_red[128 + 1];
+    flush_hist_top<128>(hist_s, p.hist + (size_t)bq * kHistBins, p.k_sel, t, flush_red,
+                        [] { named_bar_sync(1, 128); });
   }
   if (!ok) set_status(p.status, HS2_ERR_DEVICE_TIMEOUT);
   tc_fence_before();

@@ -78,9 +78,9 @@ __global__ void __launch_bounds__(kThreads) importance_simt_kernel(SelectParams 
     }
   }
   __syncthreads();
-  uint32_t* gh = p.hist + (size_t)bq * kHistBins;
-  for (int e = threadIdx.x; e < kHistBins; e += kThreads)
-    if (hist_s[e]) atomicAdd(gh + e, hist_s[e]);
+  __shared__ uint32_t flush_red[kThreads + 1];
+  flush_hist_top<kThreads>(hist_s, p.hist + (size_t)bq * kHistBins, p.k_sel, threadIdx.x,
+                           flush_red, [] { __syncthreads(); });
 }
 
 // Per-head shift delta_h = lse_h - min lse from the full layer's split partials (m in
@@ -185,9 +185,9 @@ __global__ void __launch_bounds__(kThreads) importance_sbuf_kernel(SelectParams 
     }
   }
   __syncthreads();
-  uint32_t* gh = p.hist + (size_t)bq * kHistBins;
-  for (int e = threadIdx.x; e < kHistBins; e += kThreads)
-    if (hist_s[e]) atomicAdd(gh + e, hist_s[e]);
+  __shared__ uint32_t flush_red[kThreads + 1];
+  flush_hist_top<kThreads>(hist_s, p.hist + (size_t)bq * kHistBins, p.k_sel, threadIdx.x,
+                           flush_red, [] { __syncthreads(); });
   griddep_wait();
 }
 
@@ -412,6 +412,9 @@ constexpr int kSmallBand = 1024;  // bands up to this size are ranked pairwise i
 constexpr int kBuckets = 1024;    // counting-sort buckets of the final index set
 constexpr int kQLd = kHeadDim + 8;  // padded q row (bf16) in shared memory
 constexpr int kCandSmem = 4096;   // candidate lists up to this size are staged in shared memory
+// The final sort uses a bitmap of positions in the candidate staging area (8 bytes per
+// candidate slot, 32 positions per word) when the ranked range fits in it.
+constexpr int kBitmapKeys = kCandSmem * 2 * 32;
 static_assert(kSmallBand * (sizeof(double) + sizeof(int)) <= kMaxIdxWidth * sizeof(int),
               "band pairs must fit the scratch area");
 
@@ -741,52 +744,92 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
   }
   __syncthreads();
   // Every top key lies in [0, n_c) and the forced recent window [n_c, p] lies above
-  // them, already in order: only the top keys are sorted.  Counting sort on the bucket
-  // floor(position * kBuckets / n_c) (monotone; about one key per bucket), then each
-  // key's rank inside its bucket.
+  // them, already in order: only the top keys are sorted.
   const int n = (int)min(n_sel, (uint32_t)kMaxIdxWidth);
-  const float bscale = (float)kBuckets / (float)n_c;
-  auto bucket_of = [&](int v) { return min(kBuckets - 1, (int)((float)v * bscale)); };
-  for (int e = threadIdx.x; e < kBuckets; e += blockDim.x) bucket[e] = 0u;
-  __syncthreads();
-  for (int e = threadIdx.x; e < n; e += blockDim.x) atomicAdd(&bucket[bucket_of(sel[e])], 1u);
-  __syncthreads();
-  if (threadIdx.x < 32) {  // exclusive prefix over the buckets, 32 per lane
-    const int lane = threadIdx.x;
-    uint32_t sum = 0;
-    for (int u = 0; u < kBuckets / 32; ++u) sum += bucket[lane * (kBuckets / 32) + u];
-    uint32_t incl = sum;
+  const int n_win = pos - n_c + 1;
+  if (n_c <= kBitmapKeys) {
+    // Bitmap of the positions (in the candidate staging area, no longer needed): set
+    // one bit per key, then each thread walks its run of words in order, starting at
+    // the number of keys below the run (a block-wide prefix sum of popcounts).
+    uint32_t* bm = reinterpret_cast<uint32_t*>(cts);
+    const int nw = (n_c + 31) / 32;
+    const int per = (nw + (int)blockDim.x - 1) / (int)blockDim.x;
+    for (int e = threadIdx.x; e < nw; e += blockDim.x) bm[e] = 0u;
+    __syncthreads();
+    for (int e = threadIdx.x; e < n; e += blockDim.x)
+      atomicOr(&bm[sel[e] >> 5], 1u << (sel[e] & 31));
+    __syncthreads();
+    const int w0 = threadIdx.x * per, w1 = min(w0 + per, nw);
+    uint32_t cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
+    __shared__ uint32_t warp_cnt[kFinThreads / 32];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    uint32_t incl = cnt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += x;
     }
-    uint32_t run = incl - sum;
-    for (int u = 0; u < kBuckets / 32; ++u) {
-      const uint32_t c = bucket[lane * (kBuckets / 32) + u];
-      bucket[lane * (kBuckets / 32) + u] = run;
-      bucket_beg[lane * (kBuckets / 32) + u] = run;
-      run += c;
+    if (lane == 31) warp_cnt[wid] = incl;
+    __syncthreads();
+    uint32_t base = incl - cnt;
+    for (int k = 0; k < wid; ++k) base += warp_cnt[k];
+    for (int w = w0; w < w1; ++w) {
+      uint32_t bits = bm[w];
+      while (bits) {
+        const int bpos = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (base < (uint32_t)n) out[base] = w * 32 + bpos;
+        ++base;
+      }
     }
+    for (int e = n + threadIdx.x; e < width; e += blockDim.x)
+      out[e] = e < n + n_win ? n_c + (e - n) : -1;
+  } else {
+    // Counting sort on the bucket floor(position * kBuckets / n_c) (monotone; about one
+    // key per bucket), then each key's rank inside its bucket.
+    const float bscale = (float)kBuckets / (float)n_c;
+    auto bucket_of = [&](int v) { return min(kBuckets - 1, (int)((float)v * bscale)); };
+    for (int e = threadIdx.x; e < kBuckets; e += blockDim.x) bucket[e] = 0u;
+    __syncthreads();
+    for (int e = threadIdx.x; e < n; e += blockDim.x) atomicAdd(&bucket[bucket_of(sel[e])], 1u);
+    __syncthreads();
+    if (threadIdx.x < 32) {  // exclusive prefix over the buckets, 32 per lane
+      const int lane = threadIdx.x;
+      uint32_t sum = 0;
+      for (int u = 0; u < kBuckets / 32; ++u) sum += bucket[lane * (kBuckets / 32) + u];
+      uint32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
+      }
+      uint32_t run = incl - sum;
+      for (int u = 0; u < kBuckets / 32; ++u) {
+        const uint32_t c = bucket[lane * (kBuckets / 32) + u];
+        bucket[lane * (kBuckets / 32) + u] = run;
+        bucket_beg[lane * (kBuckets / 32) + u] = run;
+        run += c;
+      }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < n; e += blockDim.x) {
+      const int v = sel[e];
+      tmp[atomicAdd(&bucket[bucket_of(v)], 1u)] = v;  // bucket[b] advances to b's end
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < n; e += blockDim.x) {
+      const int v = tmp[e];
+      const int bk = bucket_of(v);
+      const uint32_t beg = bucket_beg[bk], end = bucket[bk];
+      uint32_t rank = 0;
+      for (uint32_t x = beg; x < end; ++x) rank += tmp[x] < v;
+      sel[beg + rank] = v;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < width; e += blockDim.x)
+      out[e] = e < n ? sel[e] : (e < n + n_win ? n_c + (e - n) : -1);
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < n; e += blockDim.x) {
-    const int v = sel[e];
-    tmp[atomicAdd(&bucket[bucket_of(v)], 1u)] = v;  // bucket[b] advances to b's end
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < n; e += blockDim.x) {
-    const int v = tmp[e];
-    const int bk = bucket_of(v);
-    const uint32_t beg = bucket_beg[bk], end = bucket[bk];
-    uint32_t rank = 0;
-    for (uint32_t x = beg; x < end; ++x) rank += tmp[x] < v;
-    sel[beg + rank] = v;
-  }
-  __syncthreads();
-  const int n_win = pos - n_c + 1;
-  for (int e = threadIdx.x; e < width; e += blockDim.x)
-    out[e] = e < n ? sel[e] : (e < n + n_win ? n_c + (e - n) : -1);
   // The index set is complete and visible: the next kernel (a sparse layer, which reads
   // it without waiting for this grid to end) may start.
   __threadfence();
