@@ -41,8 +41,14 @@ constexpr float kRescaleAtF8 = 8.0f;
 // where the softmax registers leave no room for more threads.
 template <int H>
 __host__ __device__ constexpr int fp8_conv_warps() { return H <= 32 ? 8 : 4; }
+// Softmax threads per key: two at 64 heads (each takes 32 of the key's heads, so that
+// its logits and running sums stay in registers), else one.
 template <int H>
-__host__ __device__ constexpr int fp8_threads() { return 192 + 32 * fp8_conv_warps<H>(); }
+__host__ __device__ constexpr int fp8_halves() { return H == 64 ? 2 : 1; }
+template <int H>
+__host__ __device__ constexpr int fp8_threads() {
+  return 64 + 128 * fp8_halves<H>() + 32 * fp8_conv_warps<H>();
+}
 constexpr uint32_t kRawTile = 16384;    // 128 keys x 128 E4M3 codes
 constexpr uint32_t kConvTile = 32768;   // 128 keys x 128 f16 (two 64-column boxes)
 
@@ -97,6 +103,34 @@ __device__ __forceinline__ void convert_row(const uint8_t* raw, uint8_t* conv, i
     *reinterpret_cast<uint4*>(dst + ((((c0 + 1) ^ r) & 7) << 4)) =
         make_uint4(o[4], o[5], o[6], o[7]);
   }
+}
+
+// Named barrier of head group `half` over its 128 threads, with compile-time ids (1, 2)
+// so that the kernel reserves only the barriers it names.
+__device__ __forceinline__ void group_bar_sync(int half) {
+  if (half) sm100::named_bar_sync(2, 128);
+  else sm100::named_bar_sync(1, 128);
+}
+__device__ __forceinline__ bool group_bar_or(int half, bool pred) {
+  return half ? sm100::named_bar_or(5, 128, pred) : sm100::named_bar_or(4, 128, pred);
+}
+
+// Largest value over the 128 softmax threads of one head group (heads [hoff, hoff + HH)),
+// per head (the group's named barrier).
+template <int HH, int H>
+__device__ __forceinline__ void block_max_group_f8(const float (&v)[HH], float* red, float* out,
+                                                   int t, int hoff, int half) {
+  const int w = t >> 5, lane = t & 31;
+#pragma unroll
+  for (int h = 0; h < HH; ++h) {
+    const float m = warp_max(v[h]);
+    if (lane == 0) red[w * H + hoff + h] = m;
+  }
+  group_bar_sync(half);
+  if (t < HH)
+    out[hoff + t] = fmaxf(fmaxf(red[hoff + t], red[H + hoff + t]),
+                          fmaxf(red[2 * H + hoff + t], red[3 * H + hoff + t]));
+  group_bar_sync(half);
 }
 
 template <int H>
@@ -168,8 +202,8 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
       mbar_init(vc_full + s, 128);
       mbar_init(vc_empty + s, 1);
       mbar_init(s_full + s, 1);
-      mbar_init(s_free + s, 128);
-      mbar_init(p_full + s, 128);
+      mbar_init(s_free + s, 128 * fp8_halves<H>());
+      mbar_init(p_full + s, 128 * fp8_halves<H>());
       mbar_init(p_free + s, 1);
     }
     mbar_init(mma_done, 1);
@@ -319,9 +353,9 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
       mma_commit(mma_done);
       if (!mbar_wait(mma_done, 0)) ok = false;
     }
-  } else if (warp >= 6) {
+  } else if (warp >= 2 + 4 * fp8_halves<H>()) {
     // ------------------------------------------------------------ conversion
-    const int ct = threadIdx.x - 192;
+    const int ct = threadIdx.x - (64 + 128 * fp8_halves<H>());
     const int t = ct & (kKeyTile - 1);  // row of the tile
     constexpr bool kSplit = fp8_conv_warps<H>() == 8;
     const bool do_k = !kSplit || ct < kKeyTile, do_v = !kSplit || ct >= kKeyTile;
@@ -348,15 +382,21 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
+    // Thread (t, half): key t of the tile (TMEM lane t), heads [hoff, hoff + HH).
+    constexpr int NHALF = fp8_halves<H>();
+    constexpr int HH = H / NHALF;
+    constexpr int NSOFT = 128 * NHALF;
     const int lg = warp & 3;
     const int t = lg * 32 + (int)lane_id();
+    const int half = (warp - 2) >> 2;
+    const int hoff = half * HH;
     const uint32_t lane_base = (uint32_t)(lg * 32) << 16;
     const uint64_t keep_policy = policy_evict_last();
-    float l[H];
+    float l[HH];
 #pragma unroll
-    for (int h = 0; h < H; ++h) l[h] = 0.f;
-    if (t < H) mref_s[t] = -INFINITY;
-    named_bar_sync(1, 128);
+    for (int h = 0; h < HH; ++h) l[h] = 0.f;
+    if (t < HH) mref_s[hoff + t] = -INFINITY;
+    group_bar_sync(half);
     // Per-key scales (and validity) are loaded two tiles ahead so that their memory
     // latency overlaps the tiles in between instead of stalling each tile.
     auto scales_of = [&](int i, float& ks, float& vs, bool& ok_row) {
@@ -379,63 +419,65 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
       val_next = val_far;
       scales_of(i + 2, ks_far, vs_far, val_far);
       if (ok && !mbar_wait(s_full + sb, (i >> 1) & 1)) ok = false;
-      if (named_bar_or(3, 128, !ok)) ok = false;
+      if (named_bar_or(3, NSOFT, !ok)) ok = false;
       tc_fence_after();
-      float x[H];
+      float x[HH];
       {
         // Every chunk's load in flight before the one wait.
-        uint32_t r[H];
+        uint32_t r[HH];
 #pragma unroll
-        for (int c = 0; c < H; c += 16)
-          tmem_ld16(tmem_base + lane_base + sb * H + c, *reinterpret_cast<uint32_t(*)[16]>(r + c));
+        for (int c = 0; c < HH; c += 16)
+          tmem_ld16(tmem_base + lane_base + sb * H + hoff + c,
+                    *reinterpret_cast<uint32_t(*)[16]>(r + c));
         tmem_wait_ld();
         if (!GATHER && p.sbuf) {
           if (j < k1 && j <= pos - p.window && pos - p.window + 1 > p.k_sel) {
-            float* dst = p.sbuf + ((size_t)bq * p.kv.max_len + j) * H;
+            float* dst = p.sbuf + ((size_t)bq * p.kv.max_len + j) * H + hoff;
 #pragma unroll
-            for (int e = 0; e < H / 4; ++e) {
+            for (int e = 0; e < HH / 4; ++e) {
               uint4 v;
-              v.x = __float_as_uint(__uint_as_float(r[4 * e]) * qinv_s[4 * e] * ks);
-              v.y = __float_as_uint(__uint_as_float(r[4 * e + 1]) * qinv_s[4 * e + 1] * ks);
-              v.z = __float_as_uint(__uint_as_float(r[4 * e + 2]) * qinv_s[4 * e + 2] * ks);
-              v.w = __float_as_uint(__uint_as_float(r[4 * e + 3]) * qinv_s[4 * e + 3] * ks);
+              v.x = __float_as_uint(__uint_as_float(r[4 * e]) * qinv_s[hoff + 4 * e] * ks);
+              v.y = __float_as_uint(__uint_as_float(r[4 * e + 1]) * qinv_s[hoff + 4 * e + 1] * ks);
+              v.z = __float_as_uint(__uint_as_float(r[4 * e + 2]) * qinv_s[hoff + 4 * e + 2] * ks);
+              v.w = __float_as_uint(__uint_as_float(r[4 * e + 3]) * qinv_s[hoff + 4 * e + 3] * ks);
               st_global_v4_hint(dst + 4 * e, v, keep_policy);
             }
           }
         }
 #pragma unroll
-        for (int e = 0; e < H; ++e) x[e] = __uint_as_float(r[e]) * (c2_s[e] * ks);
+        for (int e = 0; e < HH; ++e) x[e] = __uint_as_float(r[e]) * (c2_s[hoff + e] * ks);
       }
       tc_fence_before();
       mbar_arrive(s_free + sb);
       bool over = false;
 #pragma unroll
-      for (int h = 0; h < H; ++h) {
+      for (int h = 0; h < HH; ++h) {
         if (!valid) x[h] = -INFINITY;
-        over |= x[h] - mref_s[h] > kRescaleAtF8;
+        over |= x[h] - mref_s[hoff + h] > kRescaleAtF8;
       }
-      if (named_bar_or(2, 128, over)) {
-        block_max_heads_f8<H>(x, red, alpha_s, t);
-        if (t < H) {
-          const float mnew = fmaxf(mref_s[t], alpha_s[t]);
-          alpha_s[t] = exp2f(mref_s[t] - mnew);
-          mref_s[t] = mnew;
+      if (group_bar_or(half, over)) {
+        block_max_group_f8<HH, H>(x, red, alpha_s, t, hoff, half);
+        if (t < HH) {
+          const int h = hoff + t;
+          const float mnew = fmaxf(mref_s[h], alpha_s[h]);
+          alpha_s[h] = exp2f(mref_s[h] - mnew);
+          mref_s[h] = mnew;
         }
-        named_bar_sync(1, 128);
+        group_bar_sync(half);
 #pragma unroll
-        for (int h = 0; h < H; ++h) l[h] *= alpha_s[h];
+        for (int h = 0; h < HH; ++h) l[h] *= alpha_s[hoff + h];
         if (i > 0) {
           if (ok && !mbar_wait(p_free + ((i - 1) & 1), ((i - 1) >> 1) & 1)) ok = false;
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < H; c += 16) {
+          for (int c = 0; c < HH; c += 16) {
             uint32_t r[16];
-            tmem_ld16(tmem_o + lane_base + c, r);
+            tmem_ld16(tmem_o + lane_base + hoff + c, r);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 16; ++e)
-              r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha_s[c + e]);
-            tmem_st16(tmem_o + lane_base + c, r);
+              r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha_s[hoff + c + e]);
+            tmem_st16(tmem_o + lane_base + hoff + c, r);
           }
           tmem_wait_st();
           tc_fence_before();
@@ -444,21 +486,21 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
       if (ok && i >= 2 && !mbar_wait(p_free + sb, ((i >> 1) & 1) ^ 1)) ok = false;
       uint8_t* pb = ps + sb * L::kPBytes;
 #pragma unroll
-      for (int c = 0; c < H / 8; ++c) {
+      for (int c = 0; c < HH / 8; ++c) {
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int h0 = c * 8 + 2 * e;
           // A head whose reference is still -inf has seen no key: its p is 0 (not
           // 2^(-inf - -inf)), so a leading all-padding tile leaves O and l at zero.
-          const float p0 = ex2_ftz(x[h0] - finite_ref(mref_s[h0]));
-          const float p1 = ex2_ftz(x[h0 + 1] - finite_ref(mref_s[h0 + 1]));
+          const float p0 = ex2_ftz(x[h0] - finite_ref(mref_s[hoff + h0]));
+          const float p1 = ex2_ftz(x[h0 + 1] - finite_ref(mref_s[hoff + h0 + 1]));
           l[h0] += p0;
           l[h0 + 1] += p1;
           const __half2 v2 = __floats2half2_rn(p0 * vs, p1 * vs);
           w[e] = *reinterpret_cast<const uint32_t*>(&v2);
         }
-        *reinterpret_cast<uint4*>(pb + c * (kKeyTile * 16) + t * 16) =
+        *reinterpret_cast<uint4*>(pb + (hoff / 8 + c) * (kKeyTile * 16) + t * 16) =
             make_uint4(w[0], w[1], w[2], w[3]);
       }
       fence_proxy_async_smem();
@@ -469,23 +511,25 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     if (ok && !mbar_wait(p_free + (last & 1), (last >> 1) & 1)) ok = false;
     tc_fence_after();
 #pragma unroll
-    for (int c = 0; c < H; c += 16) {
+    for (int c = 0; c < HH; c += 16) {
       uint32_t r[16];
-      tmem_ld16(tmem_o + lane_base + c, r);
+      tmem_ld16(tmem_o + lane_base + hoff + c, r);
       tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) part_o[(c + e) * kHeadDim + t] = __uint_as_float(r[e]);
+      for (int e = 0; e < 16; ++e)
+        part_o[(hoff + c + e) * kHeadDim + t] = __uint_as_float(r[e]);
     }
     tc_fence_before();
 #pragma unroll
-    for (int h = 0; h < H; ++h) {
+    for (int h = 0; h < HH; ++h) {
       const float s = warp_sum(l[h]);
-      if (lane_id() == 0) red[(warp & 3) * H + h] = s;
+      if (lane_id() == 0) red[(warp & 3) * H + hoff + h] = s;
     }
-    named_bar_sync(1, 128);
-    if (t < H) {
-      part_ml[2 * t] = mref_s[t];
-      part_ml[2 * t + 1] = red[t] + red[H + t] + red[2 * H + t] + red[3 * H + t];
+    group_bar_sync(half);
+    if (t < HH) {
+      const int h = hoff + t;
+      part_ml[2 * h] = mref_s[h];
+      part_ml[2 * h + 1] = red[h] + red[H + h] + red[2 * H + h] + red[3 * H + h];
     }
   }
   }
