@@ -179,9 +179,7 @@ __global__ void __launch_bounds__(192, 1)
       const int j = k0 + i * kKeyTile + t;
       const bool valid = j < k1;
       if (valid) trow[j] = best;
-      const uint32_t bin = valid ? (ordered_key(best) >> kHistShift) : 0xFFFFFFFFu;
-      const unsigned grp = __match_any_sync(0xffffffffu, bin);
-      if (valid && (int)lane_id() == __ffs(grp) - 1) atomicAdd(hist_s + bin, __popc(grp));
+      if (valid) atomicAdd(hist_s + (ordered_key(best) >> kHistShift), 1u);
     }
     named_bar_sync(1, 128);
     __shared__ uint32_t flush_red[128 + 1];
@@ -415,17 +413,19 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(s_free + buf);
       const int j = k0 + i * kKeyTile + t;
+      // Per token: the key's t and one count in the token's packed histogram (plain
+      // shared-memory atomics: a key's G counts go to G different histograms, and the
+      // lanes of a warp spread over many bins).
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const int nc_g = nc0 + g;
         // Tokens past the group's end, or that keep all their keys, are not ranked.
-        const bool ranked = g < ntok && nc_g > p.k_sel;
-        const bool valid = ranked && j < nc_g;
-        if (valid) p.tbuf[((size_t)b * p.n_q + t0 + g) * p.kv.max_len + j] = best[g];
-        const uint32_t bin = valid ? (ordered_key(best[g]) >> kHistShift) : 0xFFFFFFFFu;
-        const unsigned same = __match_any_sync(0xffffffffu, bin);
-        if (valid && (int)lane_id() == __ffs(same) - 1)
-          atomicAdd(hist_s + g * (kHistBins / 2) + (bin >> 1), (uint32_t)__popc(same) << (16 * (bin & 1)));
+        const bool valid = g < ntok && nc_g > p.k_sel && j < nc_g;
+        if (valid) {
+          p.tbuf[((size_t)b * p.n_q + t0 + g) * p.kv.max_len + j] = best[g];
+          const uint32_t bin = ordered_key(best[g]) >> kHistShift;
+          atomicAdd(hist_s + g * (kHistBins / 2) + (bin >> 1), 1u << (16 * (bin & 1)));
+        }
       }
     }
     named_bar_sync(1, 128);
@@ -688,9 +688,7 @@ __global__ void __launch_bounds__(kImpF8Threads, 1)
       const int j = k0 + i * kKeyTile + t;
       const bool valid = j < k1;
       if (valid) trow[j] = best;
-      const uint32_t bin = valid ? (ordered_key(best) >> kHistShift) : 0xFFFFFFFFu;
-      const unsigned grp = __match_any_sync(0xffffffffu, bin);
-      if (valid && (int)lane_id() == __ffs(grp) - 1) atomicAdd(hist_s + bin, __popc(grp));
+      if (valid) atomicAdd(hist_s + (ordered_key(best) >> kHistShift), 1u);
     }
     named_bar_sync(1, 128);
     __shared__ uint32_t flush_red[128 + 1];
