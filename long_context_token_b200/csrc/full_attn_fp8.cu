@@ -409,6 +409,7 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     bool val_next, val_far;
     scales_of(0, ks_next, vs_next, val_next);
     scales_of(1, ks_far, vs_far, val_far);
+    const float c2 = c2_s[0];  // sm_scale * log2(e) / (the Q scale, common to all heads)
     for (int i = 0; i < n_tiles; ++i) {
       const int sb = i & 1;
       const int j = k0 + i * kKeyTile + t;
@@ -444,17 +445,24 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
             }
           }
         }
+        const float cks = c2 * ks;  // one Q scale for every head: one multiplier per key
 #pragma unroll
-        for (int e = 0; e < HH; ++e) x[e] = __uint_as_float(r[e]) * (c2_s[hoff + e] * ks);
+        for (int e = 0; e < HH; ++e) x[e] = valid ? __uint_as_float(r[e]) * cks : -INFINITY;
       }
       tc_fence_before();
       mbar_arrive(s_free + sb);
+      // This group's references: read once per tile into registers up to 16 heads per
+      // thread; above, from shared memory at each use (registers are the limit there).
+      constexpr bool kRefRegs = HH <= 16;
+      float mr[kRefRegs ? HH : 1];
+      if (kRefRegs) {
+#pragma unroll
+        for (int h = 0; h < HH; ++h) mr[h] = mref_s[hoff + h];
+      }
+      auto ref = [&](int h) { return kRefRegs ? mr[kRefRegs ? h : 0] : mref_s[hoff + h]; };
       bool over = false;
 #pragma unroll
-      for (int h = 0; h < HH; ++h) {
-        if (!valid) x[h] = -INFINITY;
-        over |= x[h] - mref_s[hoff + h] > kRescaleAtF8;
-      }
+      for (int h = 0; h < HH; ++h) over |= x[h] - ref(h) > kRescaleAtF8;
       if (group_bar_or(half, over)) {
         block_max_group_f8<HH, H>(x, red, alpha_s, t, hoff, half);
         if (t < HH) {
@@ -465,7 +473,10 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
         }
         group_bar_sync(half);
 #pragma unroll
-        for (int h = 0; h < HH; ++h) l[h] *= alpha_s[hoff + h];
+        for (int h = 0; h < HH; ++h) {
+          l[h] *= alpha_s[hoff + h];
+          if (kRefRegs) mr[kRefRegs ? h : 0] = mref_s[hoff + h];
+        }
         if (i > 0) {
           if (ok && !mbar_wait(p_free + ((i - 1) & 1), ((i - 1) >> 1) & 1)) ok = false;
           tc_fence_after();
@@ -493,8 +504,8 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
           const int h0 = c * 8 + 2 * e;
           // A head whose reference is still -inf has seen no key: its p is 0 (not
           // 2^(-inf - -inf)), so a leading all-padding tile leaves O and l at zero.
-          const float p0 = ex2_ftz(x[h0] - finite_ref(mref_s[hoff + h0]));
-          const float p1 = ex2_ftz(x[h0 + 1] - finite_ref(mref_s[hoff + h0 + 1]));
+          const float p0 = ex2_ftz(x[h0] - finite_ref(ref(h0)));
+          const float p1 = ex2_ftz(x[h0 + 1] - finite_ref(ref(h0 + 1)));
           l[h0] += p0;
           l[h0 + 1] += p1;
           const __half2 v2 = __floats2half2_rn(p0 * vs, p1 * vs);
