@@ -84,35 +84,51 @@ __global__ void __launch_bounds__(kThreads) importance_simt_kernel(SelectParams 
 }
 
 // Per-head shift delta_h = lse_h - min lse from the full layer's split partials (m in
-// log2 units, l), with the merge's arithmetic: M = max m over non-empty splits,
-// lse = (M + log2 sum_s l_s 2^(m_s - M)) ln 2 in float64.  Loads through L2 only.
+// log2 units, l): M = max m over non-empty splits, lse = (M + log2 sum_s l_s 2^(m_s - M))
+// ln 2, in float32 (the selection keys are float32 anyway and tolerate ~1e-6 here; the
+// exact re-scoring takes the float64 lse of the merge).  One load pass, through L2.
 template <int H>
 __device__ __forceinline__ void delta_from_partials(const float* pml, int S, float* delta_s) {
-  __shared__ double lse_s[H];
+  constexpr int kMaxS = 64;  // up to 64 splits per query (two per lane)
+  __shared__ float lse_s[H];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int h = w; h < H; h += nw) {
+    float2 v[kMaxS / 32];
+#pragma unroll
+    for (int u = 0; u < kMaxS / 32; ++u) {
+      const int sp = lane + 32 * u;
+      v[u] = sp < S ? __ldcg(reinterpret_cast<const float2*>(pml + ((size_t)sp * H + h) * 2))
+                    : make_float2(-INFINITY, 0.f);
+    }
     float M = -INFINITY;
-    for (int s = lane; s < S; s += 32) {
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(pml + ((size_t)s * H + h) * 2));
-      if (v.y > 0.f) M = fmaxf(M, v.x);
+#pragma unroll
+    for (int u = 0; u < kMaxS / 32; ++u)
+      if (v[u].y > 0.f) M = fmaxf(M, v[u].x);
+    for (int sp = lane + kMaxS; sp < S; sp += 32) {  // rare: more than 64 splits
+      const float2 x = __ldcg(reinterpret_cast<const float2*>(pml + ((size_t)sp * H + h) * 2));
+      if (x.y > 0.f) M = fmaxf(M, x.x);
     }
     M = warp_max(M);
-    double Ls = 0.0;
-    if (M != -INFINITY)
-      for (int s = lane; s < S; s += 32) {
-        const float2 v = __ldcg(reinterpret_cast<const float2*>(pml + ((size_t)s * H + h) * 2));
-        if (v.y > 0.f) Ls += (double)v.y * exp2((double)v.x - M);
+    float Ls = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int u = 0; u < kMaxS / 32; ++u)
+        if (v[u].y > 0.f) Ls += v[u].y * exp2f(v[u].x - M);
+      for (int sp = lane + kMaxS; sp < S; sp += 32) {
+        const float2 x = __ldcg(reinterpret_cast<const float2*>(pml + ((size_t)sp * H + h) * 2));
+        if (x.y > 0.f) Ls += x.y * exp2f(x.x - M);
       }
-    Ls = warp_sum_d(Ls);
-    if (lane == 0)
-      lse_s[h] = Ls > 0.0 ? ((double)M + log2(Ls)) * 0.69314718055994530942 : -INFINITY;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+    if (lane == 0) lse_s[h] = Ls > 0.f ? (M + __log2f(Ls)) * 0.6931471805599453f : -INFINITY;
   }
   __syncthreads();
   if (threadIdx.x < H) {
-    double mn = INFINITY;
+    float mn = INFINITY;
 #pragma unroll
-    for (int h = 0; h < H; ++h) mn = fmin(mn, lse_s[h]);
-    delta_s[threadIdx.x] = (float)(lse_s[threadIdx.x] - mn);
+    for (int h = 0; h < H; ++h) mn = fminf(mn, lse_s[h]);
+    delta_s[threadIdx.x] = lse_s[threadIdx.x] - mn;
   }
   __syncthreads();
 }
@@ -400,6 +416,12 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(SelectParams p
         cj[oc] = j0 + u;
       }
       ++oc;
+      // The finish re-scores the candidates near the boundary from their K rows: bring
+      // the row into L2 now (a hint only).
+      const size_t row = (size_t)b * p.kv.max_len + (size_t)(j0 + u);
+      const char* kr = static_cast<const char*>(p.kv.k) + row * (p.kv.fp8 ? kHeadDim : 2 * kHeadDim);
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(kr));
+      if (!p.kv.fp8) asm volatile("prefetch.global.L2 [%0];" ::"l"(kr + 128));
     }
   }
 }
