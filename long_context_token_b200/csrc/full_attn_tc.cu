@@ -134,6 +134,10 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
   // previous kernel's tail.  Index entries are read through L2.
   const bool defer_wait = GATHER && p.out != nullptr;
   if (!defer_wait) griddep_wait();
+  // A sparse layer lets the next kernel start at once: the next sparse layer needs
+  // nothing from this one and, like this one, waits before writing its output; every
+  // other kernel of the library waits for this grid to end before it reads anything.
+  if (defer_wait) griddep_launch_dependents();
 
   const int Lb = seq_len(p.kv, b, p.n_q, p.status, !GATHER && split == 0 && qi == 0);
   const int pos = Lb - p.n_q + qi;
