@@ -52,6 +52,7 @@ import numpy as np
 __all__ = [
     "bf16_to_f64", "e4m3_to_f64", "widen_cache", "attend", "importance",
     "select_top", "index_set", "full_attn_select", "sparse_attn", "hybrid_block_step",
+    "f32_to_e4m3", "quantize_row_e4m3", "kv_append",
 ]
 
 
@@ -192,6 +193,85 @@ def sparse_attn(bits: dict, q_layer_bits, idx) -> np.ndarray:
             sel = sel[sel >= 0]
             o, _, _, _ = attend(q_all[b, i], keys[sel], vals[sel], bits["sm_scale"])
             out[b, i] = o
+    return out
+
+
+# ----------------------------------------------------------------------------
+# Appending new tokens to the cache (the step before the full layer in a decode
+# loop), with FP8 quantisation of each new row.
+# ----------------------------------------------------------------------------
+def f32_to_e4m3(y) -> np.ndarray:
+    """float32 values -> OCP E4M3 ("fn") codes, round to nearest with ties to the even
+    code, magnitudes beyond the largest finite value (448) saturating to it.  From the
+    format's definition: a magnitude below 2^-6 is a subnormal with quantum 2^-9; in
+    [2^e, 2^(e+1)), -6 <= e <= 8, the quantum is 2^(e-3).  A magnitude that rounds up to
+    the next power of two moves to the next exponent (its code is the next one)."""
+    y = np.asarray(y, dtype=np.float32).astype(np.float64)
+    sign = (y < 0) | ((y == 0) & np.signbit(y))
+    a = np.abs(y)
+    # exponent of the binade holding a (frexp: a = f 2^x, f in [0.5, 1)), clamped to the
+    # subnormal range below 2^-6 and to the top binade
+    e = (np.frexp(np.where(a > 0, a, 1.0))[1] - 1).astype(np.float64)
+    e = np.clip(e, -6, 8)
+    q = np.exp2(e - 3.0)                      # quantum of that binade (2^-9 below 2^-6)
+    n = a / q                                 # exact: q is a power of two
+    r = np.floor(n)
+    frac = n - r
+    r = np.where((frac > 0.5) | ((frac == 0.5) & (np.fmod(r, 2.0) == 1.0)), r + 1.0, r)
+    mag = r * q                               # the rounded magnitude
+    mag = np.minimum(mag, 448.0)              # saturate
+    # encode the rounded magnitude: subnormal (exp field 0) or normal
+    sub = mag < 2.0 ** -6
+    code_sub = np.round(mag / 2.0 ** -9).astype(np.int64)       # 0..7 (8 would be normal)
+    en = (np.frexp(np.where(mag > 0, mag, 1.0))[1] - 1).astype(np.float64)
+    m = np.round((mag / np.exp2(en) - 1.0) * 8.0).astype(np.int64)
+    code_norm = ((en.astype(np.int64) + 7) << 3) | m
+    out = np.where(sub, code_sub, code_norm)
+    out = np.where(sign, out | 0x80, out)
+    return out.astype(np.uint8)
+
+
+def quantize_row_e4m3(row_bits):
+    """One new K or V row (bf16 bit patterns, [d]) -> (E4M3 codes [d], float32 scale)
+    by per-token absolute-maximum scaling: s = amax / 448 and code = E4M3(x / s), both
+    divisions in IEEE float32 (round to nearest even); an all-zero row gets s = 1.
+    (The pages say only that the cache may be FP8; per-token amax scaling is this
+    build's reading.)"""
+    x = bf16_to_f64(row_bits).astype(np.float32)
+    amax = np.float32(np.max(np.abs(x)))
+    s = np.float32(1.0) if amax == 0 else np.float32(amax / np.float32(448.0))
+    y = (x / s).astype(np.float32)
+    return f32_to_e4m3(y), s
+
+
+def kv_append(bits: dict, k_new_bits, v_new_bits) -> dict:
+    """Appends n_new tokens per sequence: token i of sequence b goes to row
+    lens[b] + i of K and V (FP8 caches store codes and per-token scales from
+    quantize_row_e4m3), and lens[b] grows by n_new.  Returns the new cache dict
+    (inputs unchanged)."""
+    out = dict(bits)
+    k_new = np.asarray(k_new_bits, dtype=np.uint16)
+    v_new = np.asarray(v_new_bits, dtype=np.uint16)
+    B, n_new, d = k_new.shape
+    lens = np.asarray(bits["lens"]).astype(np.int64).copy()
+    k = np.array(bits["k"], copy=True)
+    v = np.array(bits["v"], copy=True)
+    fp8 = bits["kv"] == "fp8"
+    ks = np.array(bits["k_scale"], copy=True) if fp8 else None
+    vs = np.array(bits["v_scale"], copy=True) if fp8 else None
+    for b in range(B):
+        for i in range(n_new):
+            r = int(lens[b]) + i
+            if fp8:
+                k[b, r], ks[b, r] = quantize_row_e4m3(k_new[b, i])
+                v[b, r], vs[b, r] = quantize_row_e4m3(v_new[b, i])
+            else:
+                k[b, r] = k_new[b, i]
+                v[b, r] = v_new[b, i]
+        lens[b] += n_new
+    out.update(k=k, v=v, lens=lens.astype(np.asarray(bits["lens"]).dtype))
+    if fp8:
+        out.update(k_scale=ks, v_scale=vs)
     return out
 
 

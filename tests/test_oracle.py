@@ -290,3 +290,103 @@ def test_pins_catch_dropped_fp8_scale(monkeypatch):
     _swap(monkeypatch, "widen_cache", bad)
     with pytest.raises(AssertionError):
         test_sparse_matches_library_sdpa_on_gathered_rows()
+
+
+# ----------------------------------------------------------------------------
+# Appending tokens: E4M3 encoding and per-token quantisation of the new rows.
+# ----------------------------------------------------------------------------
+def _to_bf16_bits(x) -> np.ndarray:
+    """float32 array -> bf16 bit patterns (round to nearest even, through torch)."""
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16) \
+        .view(torch.int16).numpy().view(np.uint16)
+
+
+def _torch_e4m3(y):
+    return torch.from_numpy(np.asarray(y, dtype=np.float32)).to(torch.float8_e4m3fn) \
+        .view(torch.uint8).numpy()
+
+
+def test_e4m3_encode_matches_torch_cast():
+    """Round to nearest, ties to even, against torch's float8_e4m3fn cast (in range)."""
+    rng = np.random.default_rng(7)
+    mags = rng.choice(np.array([1e-5, 1e-3, 0.1, 1.0, 30.0, 300.0], dtype=np.float32), 100000)
+    y = np.clip(rng.standard_normal(100000).astype(np.float32) * mags, -448, 448)
+    assert np.array_equal(oracle.f32_to_e4m3(y), _torch_e4m3(y))
+
+
+def test_e4m3_encode_inverts_decode_and_rounds_ties_to_even():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    vals = oracle.e4m3_to_f64(codes).astype(np.float32)
+    enc = oracle.f32_to_e4m3(vals)
+    # every finite code decodes and re-encodes to itself (0x80 is -0)
+    assert np.array_equal(enc, codes)
+    # midpoints between neighbours of the same sign go to the even code
+    pos = np.sort(oracle.e4m3_to_f64(np.arange(0, 0x7F, dtype=np.uint8)))
+    mids = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)
+    got = oracle.f32_to_e4m3(mids)
+    lo = np.arange(0, 0x7E, dtype=np.int64)
+    want = np.where(lo % 2 == 0, lo, lo + 1)
+    assert np.array_equal(got.astype(np.int64), want)
+    assert np.array_equal(got, _torch_e4m3(mids))
+
+
+def test_e4m3_encode_saturates_and_keeps_sign_of_zero():
+    assert oracle.f32_to_e4m3(np.float32(500.0)) == 0x7E        # 448
+    assert oracle.f32_to_e4m3(np.float32(-1e6)) == 0xFE
+    assert oracle.f32_to_e4m3(np.float32(-1e-12)) == 0x80       # rounds to -0
+    assert oracle.f32_to_e4m3(np.float32(2.0 ** -10)) == 0      # half of the smallest subnormal: even
+
+
+def test_row_quantisation_scale_and_error_bound():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal(128).astype(np.float32) * 3
+    bits = _to_bf16_bits(x)
+    codes, s = oracle.quantize_row_e4m3(bits)
+    xb = oracle.bf16_to_f64(bits)
+    amax = np.abs(xb).max()
+    assert np.float32(s) == np.float32(np.float32(amax) / np.float32(448.0))
+    assert np.abs(oracle.e4m3_to_f64(codes)).max() == 448.0       # the amax maps to 448
+    back = oracle.e4m3_to_f64(codes) * np.float64(s)
+    # E4M3 keeps 3 mantissa bits: half-ulp error 2^-4 relative for normals, and an
+    # absolute 2^-10 * s for subnormals
+    err = np.abs(back - xb)
+    assert np.all(err <= np.maximum(np.abs(xb) * 2.0 ** -4, 2.0 ** -10 * s) * (1 + 1e-9))
+    zc, zs = oracle.quantize_row_e4m3(np.zeros(128, dtype=np.uint16))
+    assert zs == np.float32(1.0) and not zc.any()
+
+
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+def test_kv_append_writes_rows_and_grows_lengths(kv):
+    inp = workloads.make_inputs(2, 600, n_q=1, h_q=16, kv=kv, seed=41, lens=[500, 321])
+    bits = workloads.numpy_bits(inp)
+    rng = np.random.default_rng(5)
+    new = [_to_bf16_bits(rng.standard_normal((2, 3, 128))) for _ in range(2)]
+    after = oracle.kv_append(bits, new[0], new[1])
+    assert list(after["lens"]) == [503, 324]
+    for b, L in enumerate([500, 321]):
+        for i in range(3):
+            for which, src in (("k", new[0]), ("v", new[1])):
+                sc = after[which + "_scale"][b:b + 1, L + i] if kv == "fp8" else None
+                got = oracle.widen_cache(after[which][b, L + i:L + i + 1], kv, sc)[0]
+                want = oracle.bf16_to_f64(src[b, i])
+                if kv == "bf16":
+                    assert np.array_equal(got, want)
+                else:
+                    assert np.allclose(got, want, rtol=2 ** -4, atol=np.abs(want).max() * 2.0 ** -12)
+        # rows before the old length are untouched
+        assert np.array_equal(after["k"][b, :L], bits["k"][b, :L])
+    assert np.array_equal(bits["lens"], [500, 321])                  # input unchanged
+
+
+def test_pins_catch_truncating_encoder(monkeypatch):
+    """A plausible mistake: rounding toward zero instead of to nearest-even."""
+    def trunc(y):
+        y = np.asarray(y, dtype=np.float32)
+        t = torch.from_numpy(y).to(torch.float8_e4m3fn).float().numpy()
+        over = np.abs(t) > np.abs(y)                   # rounded away from zero: step back
+        codes = _torch_e4m3(y).astype(np.int64)
+        codes = np.where(over & ((codes & 0x7F) > 0), codes - 1, codes)
+        return codes.astype(np.uint8)
+    monkeypatch.setattr(oracle, "f32_to_e4m3", trunc)
+    with pytest.raises(AssertionError):
+        test_e4m3_encode_inverts_decode_and_rounds_ties_to_even()
