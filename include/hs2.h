@@ -170,6 +170,25 @@ HS2_API hs2_status hs2_sparse_attn_noalloc(const void* q_layer, int n_q, int h_q
                                            int idx_width, float sm_scale, float* out,
                                            uint32_t* device_status, hs2_stream_t stream);
 
+/* Appends n_new tokens to every sequence of the cache: the step before the full layer in
+ * a decode loop.  (The pages say only that the KV cache may be FP8; per-token
+ * absolute-maximum scaling of the new rows is this library's reading.)
+ *   k_new, v_new  device bf16 [batch][n_new][128]: the new tokens' keys and values.
+ *   kv            the cache.  Rows lens[b] .. lens[b] + n_new - 1 of K and V (and, for
+ *                 FP8, of k_scale / v_scale) are written: the arrays behind kv change.
+ *   lens          device int32 [batch], the cache's lengths (the array kv->lens points
+ *                 to): read, then grown by n_new.
+ * FP8: each new row becomes E4M3 codes with its own float32 scale s = amax|row| / 448 and
+ * code = row / s rounded to nearest even, saturating at 448 (both divisions IEEE
+ * float32); an all-zero row gets s = 1.  bf16: the rows are copied.
+ * A sequence with lens[b] + n_new > max_len is left unchanged and sets
+ * HS2_ERR_BAD_LENGTH in the workspace's status word.  n_new in [1, 64]; k_new and v_new
+ * 16-byte aligned.  Like the other calls it may start while an earlier kernel of this
+ * library is finishing, but it waits for that kernel before reading or writing. */
+HS2_API hs2_status hs2_kv_append(const void* k_new, const void* v_new, int n_new,
+                                 const hs2_kv* kv, int32_t* lens, void* workspace,
+                                 size_t ws_bytes, hs2_stream_t stream);
+
 /* Synchronises `stream`, returns the first error recorded by the kernels since the
  * last check (HS2_OK if none) and clears it. */
 HS2_API hs2_status hs2_check_device_status(void* workspace, hs2_stream_t stream);

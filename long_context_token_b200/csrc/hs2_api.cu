@@ -491,4 +491,31 @@ const char* hs2_last_cuda_error(void) { return g_last_cuda_error; }
 
 int hs2_abi_version(void) { return HS2_ABI_VERSION; }
 
+hs2_status hs2_kv_append(const void* k_new, const void* v_new, int n_new, const hs2_kv* kv,
+                         int32_t* lens, void* workspace, size_t ws_bytes, hs2_stream_t stream) {
+  hs2_status st = check_kv(kv);
+  if (st != HS2_OK) return st;
+  if (!k_new || !v_new || !lens || !workspace) return HS2_ERR_INVALID_ARGUMENT;
+  if (n_new < 1 || n_new > kMaxNq) return HS2_ERR_UNSUPPORTED;
+  if (kv->batch < 1 || kv->max_len < 1) return HS2_ERR_INVALID_ARGUMENT;
+  if ((long long)kv->batch * kv->max_len >= (1ll << 31)) return HS2_ERR_UNSUPPORTED;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(workspace))
+    return HS2_ERR_INVALID_ARGUMENT;
+  if (ws_bytes < 256) return HS2_ERR_WORKSPACE_TOO_SMALL;  // the status word
+  AppendParams p;
+  p.k_new = static_cast<const uint16_t*>(k_new);
+  p.v_new = static_cast<const uint16_t*>(v_new);
+  p.k = const_cast<void*>(kv->k);
+  p.v = const_cast<void*>(kv->v);
+  p.k_scale = const_cast<float*>(kv->k_scale);
+  p.v_scale = const_cast<float*>(kv->v_scale);
+  p.lens = lens;
+  p.max_len = kv->max_len;
+  p.n_new = n_new;
+  p.fp8 = kv->dtype == HS2_KV_FP8_E4M3;
+  p.status = static_cast<uint32_t*>(workspace);
+  cudaError_t e = launch_kv_append(p, kv->batch, (cudaStream_t)stream);
+  return e == cudaSuccess ? HS2_OK : cuda_fail(e, "kv-append launch");
+}
+
 }  // extern "C"

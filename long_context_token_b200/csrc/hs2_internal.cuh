@@ -128,6 +128,20 @@ struct SelectParams {
   uint32_t* status;
 };
 
+// Appending new tokens (KV append with FP8 quantisation of the new rows).
+struct AppendParams {
+  const uint16_t* k_new;  // bf16 [B][n_new][128]
+  const uint16_t* v_new;
+  void* k;                 // the cache, [B][max_len][128] (bf16 or E4M3 codes)
+  void* v;
+  float* k_scale;          // [B][max_len] (FP8 only)
+  float* v_scale;
+  int32_t* lens;           // [B], read and grown by n_new
+  int max_len, n_new;
+  bool fp8;
+  uint32_t* status;
+};
+
 struct SparseParams {
   const uint16_t* q;
   KvView kv;
@@ -196,6 +210,7 @@ inline bool sbuf_eligible(int n_q, int h, int /*dtype*/) {
 }
 cudaError_t launch_sparse_attn(const SparseParams& p, int batch, cudaStream_t s);
 cudaError_t launch_merge(const MergeParams& p, int bq, bool log2_domain, cudaStream_t s);
+cudaError_t launch_kv_append(const AppendParams& p, int batch, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // Device helpers.

@@ -29,7 +29,7 @@ STATUS = {
 
 EXPORTS = ("hs2_workspace_bytes", "hs2_full_attn_select", "hs2_full_attn", "hs2_select",
            "hs2_sparse_attn", "hs2_check_device_status", "hs2_status_string",
-           "hs2_last_cuda_error", "hs2_abi_version", "hs2_sparse_attn_noalloc")
+           "hs2_last_cuda_error", "hs2_abi_version", "hs2_sparse_attn_noalloc", "hs2_kv_append")
 
 
 class Hs2Error(RuntimeError):
@@ -79,6 +79,8 @@ def lib():
     L.hs2_sparse_attn.restype = i32
     L.hs2_sparse_attn_noalloc.argtypes = [vp, i32, i32, kvp, vp, i32, f32, vp, vp, vp]
     L.hs2_sparse_attn_noalloc.restype = i32
+    L.hs2_kv_append.argtypes = [vp, vp, i32, kvp, vp, vp, sz, vp]
+    L.hs2_kv_append.restype = i32
     L.hs2_check_device_status.argtypes = [vp, vp]
     L.hs2_check_device_status.restype = i32
     L.hs2_status_string.argtypes = [i32]
@@ -245,6 +247,23 @@ def sparse_attn(q_layer: torch.Tensor, cache: Cache, idx: torch.Tensor,
                                  workspace.numel(), _stream(stream))
     _check(code, "hs2_sparse_attn")
     return out
+
+
+def kv_append(k_new: torch.Tensor, v_new: torch.Tensor, cache: Cache, workspace: torch.Tensor,
+              stream=None) -> None:
+    """Appends n_new tokens per sequence to ``cache`` (bf16 [B, n_new, 128] keys and
+    values; FP8 caches quantise each new row with its own scale) and grows
+    ``cache.lens`` in place."""
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 3 \
+                or t.shape[0] != cache.batch or t.shape[2] != 128:
+            raise ValueError(f"{name} must be contiguous bf16 [B, n_new, 128] on the device")
+    if k_new.shape != v_new.shape:
+        raise ValueError("k_new and v_new must have the same shape")
+    code = lib().hs2_kv_append(k_new.data_ptr(), v_new.data_ptr(), k_new.shape[1], cache.ref(),
+                               cache.lens.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                               _stream(stream))
+    _check(code, "hs2_kv_append")
 
 
 def check_device_status(workspace: torch.Tensor, stream=None) -> int:

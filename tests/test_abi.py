@@ -93,3 +93,18 @@ def test_sparse_attn_host_validation(L):
     assert L.hs2_sparse_attn(p, 1, 16, ctypes.byref(kv), None, 8, 0.088, p, p, 1 << 30, None) == 1
     assert L.hs2_sparse_attn(p, 1, 16, ctypes.byref(kv), p, 8, 0.088, p, p, 16, None) == 3
     assert L.hs2_check_device_status(None, None) == 1
+
+
+@pytest.mark.parametrize("kv,kn,nn,lens,ws,wsb,expect", [
+    (_kv(), 0, 1, 1 << 20, 1 << 20, 4096, 1),                 # null k_new
+    (_kv(), 1 << 20, 1, 0, 1 << 20, 4096, 1),                 # null lens
+    (_kv(), 1 << 20, 0, 1 << 20, 1 << 20, 4096, 2),           # n_new = 0
+    (_kv(), 1 << 20, 65, 1 << 20, 1 << 20, 4096, 2),          # n_new > 64
+    (_kv(), 1 << 20 | 8, 1, 1 << 20, 1 << 20, 4096, 1),       # misaligned k_new
+    (_kv(dtype=1), 1 << 20, 1, 1 << 20, 1 << 20, 4096, 1),    # fp8 cache without scales
+    (_kv(head_dim=64), 1 << 20, 1, 1 << 20, 1 << 20, 4096, 2),  # head_dim != 128
+    (_kv(), 1 << 20, 1, 1 << 20, 1 << 20, 64, 3),             # workspace too small
+])
+def test_kv_append_rejects_bad_arguments(L, kv, kn, nn, lens, ws, wsb, expect):
+    code = L.hs2_kv_append(kn, 1 << 20, nn, ctypes.byref(kv), lens, ws, wsb, None)
+    assert code == expect

@@ -39,21 +39,26 @@ def run_gpu(inp: workloads.Inputs, twice: bool = False):
 
 
 def compare(inp: workloads.Inputs, res: dict, sparse_full: bool = True):
-    bits = workloads.numpy_bits(inp)
+    return compare_bits(workloads.numpy_bits(inp), res, sparse_full)
+
+
+def compare_bits(bits: dict, res: dict, sparse_full: bool = True):
+    """Checks one GPU step against the oracle run on the cache ``bits``."""
     ref = oracle.full_attn_select(bits, keep_importance=True)
-    tol = TOL[inp.kv]
+    tol = TOL[bits["kv"]]
     err = np.abs(res["out"] - ref["out"]).max()
     assert err < tol, f"full-layer output max-abs error {err}"
     lerr = np.abs(res["lse"] - ref["lse"]).max()
     assert lerr < LSE_TOL, f"lse error {lerr}"
-    B, n_q = inp.batch, inp.n_q
+    B, n_q = bits["q"].shape[:2]
+    window, k_sel = bits["window"], bits["k_sel"]
     n_exact = 0
     for b in range(B):
-        L = int(inp.lens[b])
+        L = int(bits["lens"][b])
         for i in range(n_q):
             p = L - n_q + i
             msg = check_index_set(res["idx"][b, i], ref["idx"][b, i], ref["imp"][b * n_q + i],
-                                  p, inp.window, inp.k_sel)
+                                  p, window, k_sel)
             assert msg is None, f"(b={b}, i={i}, p={p}): {msg}"
             n_exact += int(np.array_equal(res["idx"][b, i], ref["idx"][b, i]))
     # Sparse layers: fed the GPU's own index set (identical to the oracle's outside
@@ -216,3 +221,88 @@ def test_full_size_workloads_match_oracle(n):
     for b, needles in enumerate(inp.needles):
         for pos, _ in needles:
             assert pos in idx[b, w.n_q - 1], f"needle at {pos} not selected"
+
+
+# A decode loop: every step appends n_new tokens per sequence (the new tokens' K/V),
+# then runs the full layer with selection and the sparse layers for those tokens as
+# queries.  Sequence 1 starts empty; sequence 0 ends exactly at max_len.
+DECODE_LOOP = [
+    dict(id="bf16-h16", kv="bf16", h_q=16, n_new=1, seed=141),
+    dict(id="fp8-h16", kv="fp8", h_q=16, n_new=1, seed=142),
+    dict(id="fp8-h64", kv="fp8", h_q=64, n_new=1, seed=143),
+    dict(id="fp8-h16-append3", kv="fp8", h_q=16, n_new=3, seed=144),
+    dict(id="bf16-h32-append4", kv="bf16", h_q=32, n_new=4, seed=145),
+]
+LOOP_STEPS = 3
+
+
+def _new_rows(gen: torch.Generator, batch: int, n_new: int) -> torch.Tensor:
+    """bf16 [B, n_new, 128]: Gaussian rows with per-token magnitudes spread over
+    e^[-3, 1], one all-zero row (scale 1) and one row of tiny entries under a
+    dominant +5 / -6 pair (its other codes fall into the E4M3 subnormals)."""
+    x = torch.randn(batch, n_new, 128, generator=gen)
+    x *= torch.exp(torch.rand(batch, n_new, 1, generator=gen) * 4 - 3)
+    x[0, 0] = 0
+    x[-1, -1] *= 1e-4
+    x[-1, -1, 7], x[-1, -1, 9] = 5.0, -6.0
+    return x.to(torch.bfloat16)
+
+
+def _bits_of(t: torch.Tensor) -> np.ndarray:
+    t = t.cpu()
+    return (t.view(torch.int16).numpy().view("uint16") if t.dtype == torch.bfloat16
+            else t.numpy())
+
+
+def _assert_cache_equal(cache: hs2.Cache, want: dict):
+    assert np.array_equal(cache.lens.cpu().numpy(), want["lens"])
+    assert np.array_equal(_bits_of(cache.k), want["k"]), "K rows differ"
+    assert np.array_equal(_bits_of(cache.v), want["v"]), "V rows differ"
+    if want["kv"] == "fp8":
+        for name in ("k_scale", "v_scale"):
+            got = getattr(cache, name).cpu().numpy().view(np.uint32)
+            assert np.array_equal(got, want[name].view(np.uint32)), f"{name} differs"
+
+
+@pytest.mark.parametrize("case", DECODE_LOOP, ids=lambda c: c["id"])
+def test_decode_loop_with_append_matches_oracle(case):
+    dev = torch.device("cuda:0")
+    n_new, h_q = case["n_new"], case["h_q"]
+    lens0 = [1500, 0]
+    max_len = lens0[0] + LOOP_STEPS * n_new
+    inp = workloads.make_inputs(2, max_len, n_q=n_new, h_q=h_q, kv=case["kv"],
+                                seed=case["seed"], lens=lens0, n_sparse=2)
+    bits = workloads.numpy_bits(inp)
+    cache = hs2.Cache(inp.k.to(dev), inp.v.to(dev), inp.lens.to(dev),
+                      None if inp.k_scale is None else inp.k_scale.to(dev),
+                      None if inp.v_scale is None else inp.v_scale.to(dev))
+    ws = hs2.alloc_workspace(cache, n_new, h_q)
+    gen = torch.Generator().manual_seed(case["seed"])
+    for step in range(LOOP_STEPS):
+        k_new, v_new = _new_rows(gen, 2, n_new), _new_rows(gen, 2, n_new)
+        hs2.kv_append(k_new.to(dev), v_new.to(dev), cache, ws)
+        bits = oracle.kv_append(bits, _bits_of(k_new), _bits_of(v_new))
+        q = torch.randn(2, n_new, h_q, 128, generator=gen).to(torch.bfloat16)
+        q_layers = [torch.randn(2, n_new, h_q, 128, generator=gen).to(torch.bfloat16)
+                    for _ in range(2)]
+        out, idx, lse = hs2.full_attn_select(q.to(dev), cache, inp.window, inp.k_sel,
+                                             inp.sm_scale, ws)
+        sp = [hs2.sparse_attn(ql.to(dev), cache, idx, ws, inp.sm_scale) for ql in q_layers]
+        assert hs2.check_device_status(ws) == 0, f"step {step}"
+        _assert_cache_equal(cache, bits)
+        bits = dict(bits, q=_bits_of(q), q_layers=[_bits_of(x) for x in q_layers])
+        compare_bits(bits, dict(out=out.cpu().numpy(), idx=idx.cpu().numpy(),
+                                lse=lse.cpu().numpy(), sparse=[s.cpu().numpy() for s in sp]))
+    # Sequence 0 is full: one more append reports a bad length and leaves it as it
+    # was, while sequence 1 still grows.
+    k_new, v_new = _new_rows(gen, 2, n_new), _new_rows(gen, 2, n_new)
+    hs2.kv_append(k_new.to(dev), v_new.to(dev), cache, ws)
+    assert hs2.STATUS[hs2.check_device_status(ws)] == "HS2_ERR_BAD_LENGTH"
+    want = oracle.kv_append(dict(bits, lens=bits["lens"][1:], k=bits["k"][1:], v=bits["v"][1:],
+                                 k_scale=None if bits["k_scale"] is None else bits["k_scale"][1:],
+                                 v_scale=None if bits["v_scale"] is None else bits["v_scale"][1:]),
+                            _bits_of(k_new)[1:], _bits_of(v_new)[1:])
+    for key in ("lens", "k", "v", "k_scale", "v_scale"):
+        if want[key] is not None:
+            want[key] = np.concatenate([bits[key][:1], want[key]])
+    _assert_cache_equal(cache, want)
