@@ -63,7 +63,6 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x >> 5;
   griddep_wait();
-  griddep_launch_dependents();  // the compaction waits for this grid before reading
   const int split = blockIdx.x, bq = blockIdx.y;
   const int b = bq / p.n_q, qi = bq % p.n_q;
   const int Lb = seq_len(p.kv, b, p.n_q, p.status, false);
@@ -301,7 +300,6 @@ __global__ void __launch_bounds__(192, 1)
   }
   if (warp == 0 && lane_id() == 0) prefetch_tmap(&tmap_k);
   griddep_wait();
-  griddep_launch_dependents();  // the compaction waits for this grid before reading
 
   const int t0 = grp * G;
   const int ntok = min(G, p.n_q - t0);
@@ -562,7 +560,6 @@ __global__ void __launch_bounds__(kImpF8Threads, 1)
 
   const int warp = threadIdx.x >> 5;
   griddep_wait();
-  griddep_launch_dependents();  // the compaction waits for this grid before reading
   const int split = blockIdx.x, bq = blockIdx.y;
   const int b = bq / p.n_q, qi = bq % p.n_q;
   const int Lb = seq_len(p.kv, b, p.n_q, p.status, false);

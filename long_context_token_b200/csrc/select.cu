@@ -145,7 +145,6 @@ template <int H>
 __global__ void __launch_bounds__(kThreads) importance_sbuf_kernel(SelectParams p) {
   __shared__ uint32_t hist_s[kHistBins];
   __shared__ float delta_s[kMaxHeads];
-  griddep_launch_dependents();  // the compaction waits for this grid before reading
   const int split = blockIdx.x, bq = blockIdx.y;
   const int b = bq / p.n_q, i = bq % p.n_q;
   const int L = seq_len(p.kv, b, p.n_q, p.status, false);
@@ -332,7 +331,6 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* total)
 __global__ void __launch_bounds__(kThreads) select_compact_kernel(SelectParams p) {
   constexpr int kPer = kChunk3Keys / kThreads;
   griddep_wait();
-  griddep_launch_dependents();  // the finish waits for this grid before reading
   const int split = blockIdx.x, bq = blockIdx.y;
   const int b = bq / p.n_q, i = bq % p.n_q;
   const int L = seq_len(p.kv, b, p.n_q, p.status, false);
