@@ -45,6 +45,12 @@ LAUNCHES_PER_SPARSE = 1         # gather attention with the split merge on chip 
 NCU_TRAFFIC = {
     2: {"bytes": 4 * (134_288_128 + 786_304), "kernel": "full_attn_tc_kernel<16, 0>",
         "capture": "2 x 131072 keys, scaled x4"},
+    # first sequence of the ragged batch, scaled by the launch's algorithmic bytes
+    3: {"bytes": round((56_976_384 + 505_088) * 245_681_880 / 56_903_232),
+        "kernel": "full_attn_fp8_kernel<16, 0>",
+        "capture": "first sequence (56.9 MB of K/V/scales), scaled to the 4-sequence launch"},
+    4: {"bytes": 276_952_064 + 5_307_392, "kernel": "full_attn_fp8_kernel<64, 0>",
+        "capture": "the whole launch"},
 }
 
 
@@ -476,8 +482,10 @@ def main():
         secs, seqs = oracle_sample(inp, w, args.cpu_budget)
         cv = seqs / (secs * w.batch)
         line["cpu_baseline"] = {"value": cv, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
-                                "sample": f"{seqs} of the {w.batch} sequences of one step "
-                                          f"({secs:.1f} s), float64 numpy oracle"}
+                                "sample": f"{seqs} one-sequence hybrid-block steps (sequences "
+                                          f"taken in turn from the {w.batch} of the batch) in "
+                                          f"{secs:.1f} s, float64 numpy oracle; steps/s = "
+                                          f"sequences/s / {w.batch}"}
     print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
