@@ -51,7 +51,7 @@ import numpy as np
 
 __all__ = [
     "bf16_to_f64", "e4m3_to_f64", "widen_cache", "attend", "importance",
-    "select_top", "index_set", "full_attn_select", "sparse_attn", "hybrid_block_step",
+    "select_top", "index_set", "block_index_set", "full_attn_select", "sparse_attn", "hybrid_block_step",
     "f32_to_e4m3", "quantize_row_e4m3", "kv_append",
 ]
 
@@ -136,14 +136,39 @@ def index_set(p: int, imp_outside, window: int, k_sel: int) -> np.ndarray:
     return out
 
 
+def block_index_set(p: int, imp_outside, window: int, k_sel: int, block: int = 64) -> np.ndarray:
+    """Block-level index set of query position p: the first-generation scheme that the
+    pages set token-level selection against ([SP] paragraph on block selection, where a
+    64-token block spends selection budget as a whole, and paragraph on the ablation at
+    the same attention budget; [RAT] paragraph on Block vs Token selection).
+    Positions [0, p-window] form aligned blocks [c*block, (c+1)*block), the last one cut
+    at p-window.  A block's score is the largest importance among its positions (the
+    pages do not say how a block is scored; this is the reading taken).  The
+    k_sel // block best blocks, ties to the lower block, are kept whole, plus the
+    forced window; ascending, padded with -1 to window + k_sel entries."""
+    w_lo = max(0, p - window + 1)
+    n_out = w_lo
+    assert imp_outside.shape[0] == n_out
+    n_blk = -(-n_out // block)
+    scores = np.array([imp_outside[c * block:(c + 1) * block].max() for c in range(n_blk)])
+    chosen = select_top(scores, k_sel // block) if n_blk else np.zeros(0, dtype=np.int64)
+    parts = [np.arange(c * block, min((c + 1) * block, n_out)) for c in chosen]
+    sel = np.union1d(np.concatenate(parts + [np.arange(w_lo, p + 1)]), [])
+    out = np.full(window + k_sel, -1, dtype=np.int64)
+    out[:sel.shape[0]] = np.sort(sel).astype(np.int64)
+    return out
+
+
 def _rows(bits: dict, b: int, hi: int, which: str):
     scale = bits.get(which + "_scale")
     sc = None if scale is None else scale[b, :hi]
     return widen_cache(bits[which][b, :hi], bits["kv"], sc)
 
 
-def full_attn_select(bits: dict, keep_importance: bool = False):
-    """The full-attention layer of the hybrid block plus its token selection.
+def full_attn_select(bits: dict, keep_importance: bool = False, block: int = 1):
+    """The full-attention layer of the hybrid block plus its selection: token level
+    (block = 1, the pages' scheme) or whole blocks of ``block`` positions (the
+    first-generation comparator, block_index_set).
 
     ``bits``: q uint16 [B, n_q, h, d]; k, v uint16 or uint8 [B, max_len, d];
     k_scale, v_scale float32 [B, max_len] or None; lens [B]; sm_scale; window;
@@ -167,7 +192,8 @@ def full_attn_select(bits: dict, keep_importance: bool = False):
             out[b, i], lse[b, i] = o, l
             w_lo = max(0, p - W + 1)
             imp = importance(s[:, :w_lo], l)
-            idx[b, i] = index_set(p, imp, W, K)
+            idx[b, i] = (index_set(p, imp, W, K) if block == 1
+                         else block_index_set(p, imp, W, K, block))
             if keep_importance:
                 imps.append(imp)
     res = dict(out=out, lse=lse, idx=idx)

@@ -240,6 +240,61 @@ def test_sparse_matches_library_sdpa_on_gathered_rows():
     np.testing.assert_allclose(out[0, 0], ref, rtol=0, atol=1e-12)
 
 
+# ------------------------------------------------------- block-level selection
+@pytest.mark.parametrize("case", read_cases("block_selection_cases.txt"), ids=lambda c: c["name"])
+def test_golden_block_selection_cases(case):
+    bits = _bits_from_case(case)
+    res = oracle.full_attn_select(bits, block=case["block"][0])
+    assert res["idx"][0, 0].tolist() == case["expected_idx"]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_block_size_one_is_token_selection(seed):
+    rng = np.random.default_rng(seed)
+    for p, W, K in ((300, 128, 64), (40, 4, 8), (9, 4, 8), (2000, 128, 1024)):
+        n = max(0, p - W + 1)
+        imp = rng.choice([0.1, 0.2, 0.3], size=n) * rng.integers(1, 4, size=n)  # many ties
+        assert np.array_equal(oracle.block_index_set(p, imp, W, K, 1),
+                              oracle.index_set(p, imp, W, K))
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_block_selection_keeps_whole_best_blocks(seed):
+    """Invariants of the block set on random importances with ties: the kept outside
+    positions are whole blocks (the cut last block counting whole), as many as the
+    budget allows; no dropped block scores above a kept one, and among equal scores
+    the kept blocks are the lower ones; the window is present; ascending; padded."""
+    rng = np.random.default_rng(100 + seed)
+    W, K, blk = 128, 1024, 64
+    for p in (127, 128, 1151, 1152, 1300, 5000, 20000):
+        w_lo = max(0, p - W + 1)
+        imp = rng.integers(0, 50, size=w_lo) / 50.0
+        got = oracle.block_index_set(p, imp, W, K, blk)
+        valid = got[got >= 0]
+        assert np.all(np.diff(valid) > 0) and np.all(got[valid.size:] == -1)
+        assert np.all(np.isin(np.arange(w_lo, p + 1), valid))
+        outside = valid[valid < w_lo]
+        n_blk = -(-w_lo // blk)
+        kept = np.unique(outside // blk)
+        assert kept.size == min(n_blk, K // blk)
+        for c in kept:
+            assert np.array_equal(outside[outside // blk == c], np.arange(c * blk, min((c + 1) * blk, w_lo)))
+        score = np.array([imp[c * blk:(c + 1) * blk].max() for c in range(n_blk)])
+        dropped = np.setdiff1d(np.arange(n_blk), kept)
+        if dropped.size and kept.size:
+            assert score[kept].min() >= score[dropped].max()
+            tie = score[kept].min()
+            assert not np.any((score[dropped] == tie) & (dropped < kept[score[kept] == tie].max()))
+
+
+def test_block_zero_query_keeps_lowest_blocks():
+    inp = workloads.make_inputs(1, 3000, n_q=1, h_q=16, seed=7, q_zero=True)
+    res = oracle.full_attn_select(workloads.numpy_bits(inp), block=64)
+    p = 2999
+    want = np.concatenate([np.arange(1024), np.arange(p - 127, p + 1)])
+    assert res["idx"][0, 0].tolist() == want.tolist()
+
+
 # -------------------------------------------- the pins catch planted mistakes
 def _swap(monkeypatch, name, fn):
     monkeypatch.setattr(oracle.hs2_oracle, name, fn)
@@ -390,3 +445,20 @@ def test_pins_catch_truncating_encoder(monkeypatch):
     monkeypatch.setattr(oracle, "f32_to_e4m3", trunc)
     with pytest.raises(AssertionError):
         test_e4m3_encode_inverts_decode_and_rounds_ties_to_even()
+
+
+def test_pins_catch_block_mean_score(monkeypatch):
+    def bad(p, imp_outside, window, k_sel, block=64):
+        w_lo = max(0, p - window + 1)
+        n_blk = -(-w_lo // block)
+        scores = np.array([imp_outside[c * block:(c + 1) * block].mean() for c in range(n_blk)])
+        chosen = oracle.select_top(scores, k_sel // block)
+        parts = [np.arange(c * block, min((c + 1) * block, w_lo)) for c in chosen]
+        sel = np.union1d(np.concatenate(parts + [np.arange(w_lo, p + 1)]), [])
+        out = np.full(window + k_sel, -1, dtype=np.int64)
+        out[:sel.shape[0]] = np.sort(sel).astype(np.int64)
+        return out
+    _swap(monkeypatch, "block_index_set", bad)
+    case = read_cases("block_selection_cases.txt")[0]
+    with pytest.raises(AssertionError):
+        test_golden_block_selection_cases(case)
