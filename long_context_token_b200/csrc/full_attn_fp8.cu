@@ -3,23 +3,28 @@
 // (web coverage of HySparse2: the 1M-token footprint is quoted with an FP8 KV cache;
 // "Luo Fuli Teases Xiaomi MiMo-V3 Architecture ...", paragraph on cost at 1M tokens).
 //
-// The MMA needs both operands in the same 16-bit type.  E4M3 values are exact in f16
-// (4 significant bits, exponents 2^-9 .. 2^8), so the codes are widened to f16 with no
-// rounding; the per-token scales stay out of the MMA: k_scale[j] multiplies key j's
-// logits and v_scale[j] multiplies its probability before P.V.  Q (bf16) becomes f16
-// after a per-head power-of-two scaling that puts its largest element in [2^14, 2^15),
-// so the conversion cannot overflow; the scale is divided out of the logits.
+// The cache's E4M3 codes feed the MMA as they are (kind::f8f6f4, both operands E4M3,
+// fp32 accumulation), straight from the tiles TMA writes; the per-token scales stay
+// out of it: k_scale[j] multiplies key j's logits and v_scale[j] its probability
+// before P.V.  The other two operands are sums of E4M3 terms:
+//   Q = 2^-e (Q_hi + Q_lo / 16), one power of two for all heads putting the largest
+//     |q| into [128, 256): a bf16 element (8 significant bits) whose scaled magnitude
+//     is at least 2^-6 is exact in the two terms, smaller ones to 2^-13 absolute;
+//   P' = p * v_scale * 2^-ev = P_hi + P_lo / 16 + P_lo2 / 256 (about 12 significant
+//     bits), ev a power of two at or above every |v_scale| the CTA has seen, moved
+//     with a rescale of O (like the softmax reference) when a larger one arrives.
+// So S^T [128 keys x 2H] = K . [Q_hi | Q_lo]^T and O^T [128 d x 3H] += V^T . [P_hi |
+// P_lo | P_lo2]^T; the softmax and the epilogue combine each head's columns.
 //
 // One CTA per key chunk (or per 128 index entries) of one (sequence, token):
 //   warp 0      producer: TMA of 128-row E4M3 tiles (128-byte rows, 128-byte
-//               swizzle) into an R-stage raw ring; in gather mode cp.async of the
-//               indexed rows into the same layout;
-//   warp 1      TMEM allocator and MMA issuer (kind::f16 with f16 inputs):
-//                 S^T[128 keys x H] = K16 . Q16^T,   O^T[128 d x H] += V16^T . P16^T;
-//   warps 2..5  softmax, as in the bf16 kernel (one key per thread, lazily moved
-//               per-head reference), P in f16;
-//   warps 6..9  conversion: raw K / V tiles -> f16 in the swizzled operand layout
-//               (rows past the chunk end or absent in the index are zeroed).
+//               swizzle) into an R-stage ring, K and V on their own barriers; in
+//               gather mode cp.async of the indexed rows into the same layout;
+//   warp 1      TMEM allocator and MMA issuer: K (K-major) and V^T (MN-major) are
+//               read from the ring, whose stages the MMA commits release;
+//   warps 2..   softmax: one key per thread (two threads per key at 64 heads, 32
+//               heads each), lazily moved per-head reference, P written as its three
+//               E4M3 terms.
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <string.h>
@@ -36,73 +41,142 @@ namespace {
 
 constexpr float kLog2eF8 = 1.4426950408889634f;
 constexpr float kRescaleAtF8 = 8.0f;
-// Conversion warps: eight (four for K rows, four for V rows, converting in parallel on
-// their own barriers) up to 32 heads; four (each thread a K row, then a V row) above,
-// where the softmax registers leave no room for more threads.
-template <int H>
-__host__ __device__ constexpr int fp8_conv_warps() { return H <= 32 ? 8 : 4; }
+constexpr int kNoScale = -1000;  // exponent of a CTA that has seen no V scale yet
 // Softmax threads per key: two at 64 heads (each takes 32 of the key's heads, so that
-// its logits and running sums stay in registers), else one.
+// its logits, references and running sums stay in registers), else one.
 template <int H>
 __host__ __device__ constexpr int fp8_halves() { return H == 64 ? 2 : 1; }
 template <int H>
-__host__ __device__ constexpr int fp8_threads() {
-  return 64 + 128 * fp8_halves<H>() + 32 * fp8_conv_warps<H>();
-}
+__host__ __device__ constexpr int fp8_threads() { return 64 + 128 * fp8_halves<H>(); }
 constexpr uint32_t kRawTile = 16384;    // 128 keys x 128 E4M3 codes
-constexpr uint32_t kConvTile = 32768;   // 128 keys x 128 f16 (two 64-column boxes)
 
-// Gather mode (a sparse layer) keeps one raw stage and one converted V buffer: its CTAs
-// mostly take a single tile, and the smaller footprint lets two CTAs share an SM.
 template <int H, bool GATHER>
 struct Fp8Smem {
-  static constexpr int R = GATHER ? 1 : (H <= 16 ? 3 : 2);  // raw stages (K and V each)
-  static constexpr int kVConv = GATHER ? 1 : 2;              // converted V buffers
-  static constexpr uint32_t kQBytes = H * kHeadDim * 2;
-  static constexpr uint32_t kPBytes = kKeyTile * H * 2;
+  static constexpr uint32_t kQBytes = 2 * H * kHeadDim;       // Q_hi, Q_lo rows
+  static constexpr uint32_t kPBytes = 3 * H * kKeyTile;       // P_hi, P_lo, P_lo2
+  static constexpr uint32_t kRedBytes = (4 * H + 8) * 4;      // [4 warps][H] + V-scale maxima
+  static constexpr uint32_t kRefBytes = (2 * H + 8) * 4;      // mref, alpha, scalars
+  static constexpr uint32_t kMaxBars = 4 * 6 + 9;
+  // (+ 1024 for alignment, + 1024 for the static shared memory of the Q staging)
+  static constexpr uint32_t kFixed =
+      kQBytes + 2 * kPBytes + kRedBytes + kRefBytes + kMaxBars * 8 + 16 + 2048;
+  // Raw stages (K and V each): as many as fit, up to six; gather mode keeps one (its
+  // CTAs mostly take a single tile).
+  static constexpr int kFit = (int)((227u * 1024u - kFixed) / (2 * kRawTile));
+  static constexpr int R = GATHER ? 1 : (kFit > 6 ? 6 : kFit);
   static constexpr uint32_t kKRawOff = 0;
   static constexpr uint32_t kVRawOff = R * kRawTile;
-  static constexpr uint32_t kKConvOff = 2 * R * kRawTile;
-  static constexpr uint32_t kVConvOff = kKConvOff + kConvTile;
-  static constexpr uint32_t kQOff = kVConvOff + kVConv * kConvTile;
+  static constexpr uint32_t kQOff = 2 * R * kRawTile;
   static constexpr uint32_t kPOff = kQOff + kQBytes;          // [2 buffers]
-  static constexpr uint32_t kRedOff = kPOff + 2 * kPBytes;    // [4 warps][H]
-  static constexpr uint32_t kRefOff = kRedOff + 4 * H * 4;    // mref, alpha, c2, qinv
-  static constexpr uint32_t kBarOff = kRefOff + 4 * H * 4;
-  static constexpr uint32_t kBars = 4 * R + 15;
+  static constexpr uint32_t kRedOff = kPOff + 2 * kPBytes;
+  static constexpr uint32_t kRefOff = kRedOff + kRedBytes;
+  static constexpr uint32_t kBarOff = kRefOff + kRefBytes;
+  static constexpr uint32_t kBars = 4 * R + 9;
   static constexpr uint32_t kSlotOff = kBarOff + kBars * 8;
   static constexpr uint32_t kBytes = kSlotOff + 16 + 1024;
-  static constexpr uint32_t kTmemCols = tmem_cols_pow2(3 * H);
-  static_assert(kBytes <= 227 * 1024, "shared memory budget");
+  static constexpr uint32_t kTmemCols = tmem_cols_pow2(7 * H);  // S: 2 x 2H, O: 3H
+  static_assert(R >= 1 && kBytes <= 227 * 1024, "shared memory budget");
+  static_assert(kQOff + kQBytes >= kClusterMlOff + 2 * H * 4, "cluster partial fits");
+  static_assert(kQOff % 1024 == 0 && kPOff % 16 == 0 && kBarOff % 8 == 0, "alignment");
 };
 
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two_codes, __NV_E4M3);
-  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+// Two floats -> their E4M3 codes (round to nearest even, saturating; y0 in the low
+// byte) and the values those codes stand for.
+__device__ __forceinline__ uint32_t e4m3_pair(float y0, float y1, float& v0, float& v1) {
+  const __nv_fp8x2_storage_t c =
+      __nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
+  const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(c, __NV_E4M3);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+  v0 = f.x;
+  v1 = f.y;
+  return (uint32_t)c;
+}
+__device__ __forceinline__ uint32_t e4m3_codes(float y0, float y1) {
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
 }
 
-// Raw tile (128 rows x 128 codes, 16-byte chunk c of row r at chunk c ^ (r & 7)) ->
-// f16 tile in two 64-column boxes with the same swizzle.  Thread t (0..127) converts
-// row t; rows with valid == false become zeros.
-__device__ __forceinline__ void convert_row(const uint8_t* raw, uint8_t* conv, int r, bool valid) {
-  const uint8_t* src = raw + r * 128;
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint4 in = *reinterpret_cast<const uint4*>(src + (((c ^ r) & 7) << 4));
-    uint32_t w[4] = {in.x, in.y, in.z, in.w};
-    uint32_t o[8];
+// Q [H][128] bf16 -> the B operand of S^T = K . [Q_hi | Q_lo]^T (K-major, unswizzled,
+// N = 2H rows: row h holds Q_hi of head h, row H + h its Q_lo): 16-byte chunk c (16 d)
+// of row n at c * (2H * 16) + n * 16.  y = q * 2^e with the largest |y| in [128, 256),
+// Q_hi = E4M3(y), Q_lo = E4M3(16 (y - Q_hi)) (y - Q_hi is exact in float32).
+// *qinv = 2^-e.  Every thread of the block calls this; it ends with __syncthreads.
+template <int H>
+__device__ void store_q_e4m3_split(uint8_t* qs, const uint16_t* qg, float* qinv) {
+  __shared__ float hmax_s[kMaxHeads];
+  __shared__ float up_s;
+  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5, lane = threadIdx.x & 31;
+  for (int h = warp; h < H; h += nw) {
+    float m = 0.f;
+    for (int c = lane; c < kHeadDim; c += 32)
+      m = fmaxf(m, fabsf(__uint_as_float((uint32_t)qg[h * kHeadDim + c] << 16)));
+    m = warp_max(m);
+    if (lane == 0) hmax_s[h] = m;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.f;
+    for (int h = 0; h < H; ++h) m = fmaxf(m, hmax_s[h]);
+    int e = 0;
+    if (m > 0.f) {
+      int ex;
+      frexpf(m, &ex);  // m in [2^(ex-1), 2^ex)
+      e = 8 - ex;
+      e = e < -100 ? -100 : (e > 100 ? 100 : e);
+    }
+    up_s = __int_as_float((127 + e) << 23);
+    *qinv = __int_as_float((127 - e) << 23);
+  }
+  __syncthreads();
+  const float sc = up_s;
+  for (int w = threadIdx.x; w < H * (kHeadDim / 16); w += blockDim.x) {
+    const int h = w % H, c = w / H;
+    const uint4 a = *reinterpret_cast<const uint4*>(qg + h * kHeadDim + c * 16);
+    const uint4 b = *reinterpret_cast<const uint4*>(qg + h * kHeadDim + c * 16 + 8);
+    const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t hi[4], lo[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      o[2 * u] = valid ? e4m3x2_to_f16x2(w[u] & 0xffffu) : 0u;
-      o[2 * u + 1] = valid ? e4m3x2_to_f16x2(w[u] >> 16) : 0u;
+      hi[u] = 0u;
+      lo[u] = 0u;
+#pragma unroll
+      for (int v = 0; v < 2; ++v) {
+        const uint32_t x = in[2 * u + v];
+        const float y0 = __uint_as_float(x << 16) * sc;
+        const float y1 = __uint_as_float(x & 0xffff0000u) * sc;
+        float a0, a1;
+        const uint32_t ch = e4m3_pair(y0, y1, a0, a1);
+        const uint32_t cl = e4m3_codes((y0 - a0) * 16.f, (y1 - a1) * 16.f);
+        hi[u] |= ch << (16 * v);
+        lo[u] |= cl << (16 * v);
+      }
     }
-    // f16 elements 16c .. 16c+15: box c >> 2, 16-byte chunks 2(c & 3) and 2(c & 3) + 1.
-    uint8_t* dst = conv + (c >> 2) * kBoxBytes + r * 128;
-    const int c0 = 2 * (c & 3);
-    *reinterpret_cast<uint4*>(dst + (((c0 ^ r) & 7) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-    *reinterpret_cast<uint4*>(dst + ((((c0 + 1) ^ r) & 7) << 4)) =
-        make_uint4(o[4], o[5], o[6], o[7]);
+    *reinterpret_cast<uint4*>(qs + c * (2 * H * 16) + h * 16) =
+        make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(qs + c * (2 * H * 16) + (H + h) * 16) =
+        make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
+  __syncthreads();
+}
+
+// A operand K (K-major, 128-byte swizzle, one 128-byte row per key): K step kk of 32 d.
+__device__ __forceinline__ uint64_t k_e4m3_desc(uint32_t tile, int kk) {
+  return smem_desc(tile + (uint32_t)kk * 32u, 16, 1024, kSwizzle128B);
+}
+// B operand [Q_hi | Q_lo] (K-major, unswizzled, N rows): K step kk of 32 d.
+template <int N>
+__device__ __forceinline__ uint64_t q_e4m3_desc(uint32_t q, int kk) {
+  return smem_desc(q + (uint32_t)kk * 2u * N * 16u, N * 16, 128, kSwizzleNone);
+}
+// A operand V^T: the V tile is [128 keys][128 codes] with 128-byte swizzle, so V^T is
+// MN-major with all 128 d inside one swizzle atom; K step kk of 32 keys (four atoms
+// of 8 keys, 1024 bytes apart).
+__device__ __forceinline__ uint64_t vt_e4m3_desc(uint32_t tile, int kk) {
+  return smem_desc(tile + (uint32_t)kk * 32u * 128u, kRawTile, 1024, kSwizzle128B);
+}
+// B operand P^T: P stored [3H / 16 chunks][128 keys][16 codes] (MN-major, unswizzled;
+// chunk (term * H + h) / 16 holds heads h..h+15 of one term); K step kk of 32 keys.
+__device__ __forceinline__ uint64_t pt_e4m3_desc(uint32_t p, int kk) {
+  return smem_desc(p + (uint32_t)kk * 32u * 16u, 128, kKeyTile * 16, kSwizzleNone);
 }
 
 // Named barrier of head group `half` over its 128 threads, with compile-time ids (1, 2)
@@ -133,20 +207,6 @@ __device__ __forceinline__ void block_max_group_f8(const float (&v)[HH], float* 
   group_bar_sync(half);
 }
 
-template <int H>
-__device__ __forceinline__ void block_max_heads_f8(const float (&v)[H], float* red, float* out,
-                                                   int t) {
-  const int w = t >> 5, lane = t & 31;
-#pragma unroll
-  for (int h = 0; h < H; ++h) {
-    const float m = warp_max(v[h]);
-    if (lane == 0) red[w * H + h] = m;
-  }
-  named_bar_sync(1, 128);
-  if (t < H) out[t] = fmaxf(fmaxf(red[t], red[H + t]), fmaxf(red[2 * H + t], red[3 * H + t]));
-  named_bar_sync(1, 128);
-}
-
 }  // namespace
 
 template <int H, bool GATHER>
@@ -159,29 +219,24 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
   uint8_t* smem = align1024(smem_raw);
   uint8_t* kraw = smem + L::kKRawOff;
   uint8_t* vraw = smem + L::kVRawOff;
-  uint8_t* kconv = smem + L::kKConvOff;
-  uint8_t* vconv = smem + L::kVConvOff;
   uint8_t* qs = smem + L::kQOff;
   uint8_t* ps = smem + L::kPOff;
-  float* red = reinterpret_cast<float*>(smem + L::kRedOff);
+  float* red = reinterpret_cast<float*>(smem + L::kRedOff);  // [4][H], then [2 groups][4]
   float* mref_s = reinterpret_cast<float*>(smem + L::kRefOff);
   float* alpha_s = mref_s + H;
-  float* c2_s = mref_s + 2 * H;    // sm_scale * log2(e) / (Q scale of head h)
-  float* qinv_s = mref_s + 3 * H;  // 1 / (Q scale of head h)
+  float* qsc_s = mref_s + 2 * H;  // [0]: 2^-e of Q
+  int* ev_s = reinterpret_cast<int*>(mref_s + 2 * H + 2);    // [2 groups]
+  float* beta_s = mref_s + 2 * H + 4;                         // [2 groups]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* kr_full = bars;
   uint64_t* kr_empty = bars + R;
   uint64_t* vr_full = bars + 2 * R;
   uint64_t* vr_empty = bars + 3 * R;
-  uint64_t* kc_full = bars + 4 * R;      // [1]
-  uint64_t* kc_empty = kc_full + 1;      // [1]
-  uint64_t* vc_full = kc_full + 2;       // [2]
-  uint64_t* vc_empty = kc_full + 4;      // [2]
-  uint64_t* s_full = kc_full + 6;        // [2]
-  uint64_t* s_free = kc_full + 8;        // [2]
-  uint64_t* p_full = kc_full + 10;       // [2]
-  uint64_t* p_free = kc_full + 12;       // [2]
-  uint64_t* mma_done = kc_full + 14;
+  uint64_t* s_full = bars + 4 * R;  // [2]
+  uint64_t* s_free = s_full + 2;    // [2]
+  uint64_t* p_full = s_full + 4;    // [2]
+  uint64_t* p_free = s_full + 6;    // [2]
+  uint64_t* mma_done = s_full + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
 
   const int warp = threadIdx.x >> 5;
@@ -192,19 +247,17 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < R; ++s) {
       mbar_init(kr_full + s, GATHER ? 32 : 1);
-      mbar_init(kr_empty + s, 128);
+      mbar_init(kr_empty + s, 1);
       mbar_init(vr_full + s, GATHER ? 32 : 1);
-      mbar_init(vr_empty + s, 128);
+      mbar_init(vr_empty + s, 1);
     }
-    mbar_init(kc_full, 128);
-    mbar_init(kc_empty, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(vc_full + s, 128);
-      mbar_init(vc_empty + s, 1);
       mbar_init(s_full + s, 1);
       mbar_init(s_free + s, 128 * fp8_halves<H>());
       mbar_init(p_full + s, 128 * fp8_halves<H>());
       mbar_init(p_free + s, 1);
+      ev_s[s] = kNoScale;
+      beta_s[s] = 0.f;
     }
     mbar_init(mma_done, 1);
     fence_mbar_init();
@@ -243,8 +296,8 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     return (j >= 0 && j < Lb) ? (long long)(row_base + j) : -1;
   };
   bool ok = true;
-  // Cluster mode keeps the partial in this CTA's shared memory (the raw stages, idle by
-  // the time the partial is written) for the on-chip merge.
+  // Cluster mode keeps the partial in this CTA's shared memory (the raw stages and the
+  // Q operand, idle by the time the partial is written) for the on-chip merge.
   const bool on_chip = GATHER && p.out != nullptr;
   float* part_o = on_chip ? reinterpret_cast<float*>(smem + kClusterOOff)
                           : p.part_o + pidx * H * kHeadDim;
@@ -258,23 +311,22 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     }
   } else {
   if (GATHER) {
-    // The first tile's rows are gathered by every thread of the CTA; warp 0 gathers any
-    // later tiles.  (store_q_f16_scaled below synchronises the block.)
+    // The first tile's rows are gathered by every thread of the CTA (absent entries
+    // zero-filled); warp 0 gathers any later tiles.  (store_q_e4m3_split below
+    // synchronises the block.)
     gather_tile_rows<8, kRawTile>(smem_u32(kraw), smem_u32(vraw),
                                   static_cast<const uint8_t*>(p.kv.k),
                                   static_cast<const uint8_t*>(p.kv.v), idx_row, k0, k1, Lb,
                                   row_base, p.status, threadIdx.x, blockDim.x);
   }
-  // Q in f16 under a per-head power-of-two scale; its inverse goes into the logits.
-  store_q_f16_scaled<H>(qs, p.q + (size_t)bq * H * kHeadDim, qinv_s, nullptr);
+  store_q_e4m3_split<H>(qs, p.q + (size_t)bq * H * kHeadDim, qsc_s);
   if (GATHER) cp_async_wait_all();
-  for (int h = threadIdx.x; h < H; h += blockDim.x) c2_s[h] = p.sm_scale * kLog2eF8 * qinv_s[h];
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t tmem_o = tmem_base + 2 * H;
+  const uint32_t tmem_o = tmem_base + 4 * H;
 
   if (warp == 0) {
     if (GATHER) {
@@ -282,18 +334,29 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
       const int lane = (int)lane_id();
       for (int i = 0; i < n_tiles; ++i) {
         const int s = i % R;
-        if (i > 0) {  // tile 0 was gathered by the whole CTA above
-          const uint32_t ph = ((i / R) & 1) ^ 1;
-          if (ok && !mbar_wait(kr_empty + s, ph)) ok = false;
-          if (ok && !mbar_wait(vr_empty + s, ph)) ok = false;
-          gather_tile_rows<8, kRawTile>(
-              smem_u32(kraw + s * kRawTile), smem_u32(vraw + s * kRawTile),
-              static_cast<const uint8_t*>(p.kv.k), static_cast<const uint8_t*>(p.kv.v), idx_row,
-              k0 + i * kKeyTile, k1, Lb, row_base, p.status, lane, 32);
-          cp_async_wait_all();
-          fence_proxy_async_smem();
+        if (i == 0) {  // tile 0 was gathered by the whole CTA above
+          mbar_arrive(kr_full + s);
+          mbar_arrive(vr_full + s);
+          continue;
         }
+        // K and V separately, each once its stage is released: with one stage, V's is
+        // released by P.V of the previous tile, which the MMA issues only after this
+        // tile's Q.K^T.
+        const uint32_t ph = ((i / R) & 1) ^ 1;
+        const int e0 = k0 + i * kKeyTile;
+        if (ok && !mbar_wait(kr_empty + s, ph)) ok = false;
+        gather_tile_rows<8, kRawTile>(smem_u32(kraw + s * kRawTile), 0,
+                                      static_cast<const uint8_t*>(p.kv.k), nullptr, idx_row, e0,
+                                      k1, Lb, row_base, p.status, lane, 32);
+        cp_async_wait_all();
+        fence_proxy_async_smem();
         mbar_arrive(kr_full + s);
+        if (ok && !mbar_wait(vr_empty + s, ph)) ok = false;
+        gather_tile_rows<8, kRawTile>(0, smem_u32(vraw + s * kRawTile), nullptr,
+                                      static_cast<const uint8_t*>(p.kv.v), idx_row, e0, k1, Lb,
+                                      row_base, p.status, lane, 32);
+        cp_async_wait_all();
+        fence_proxy_async_smem();
         mbar_arrive(vr_full + s);
       }
     } else if (elect_one()) {
@@ -321,68 +384,41 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
-      const uint32_t id_qk = idesc_f16(128, H, false, false, false);
-      const uint32_t id_pv = idesc_f16(128, H, false, true, true);
+      constexpr uint32_t id_qk = idesc_e4m3(128, 2 * H, false, false);
+      constexpr uint32_t id_pv = idesc_e4m3(128, 3 * H, true, true);
       const uint32_t q_addr = smem_u32(qs);
-      const uint32_t k_addr = smem_u32(kconv);
       auto issue_pv = [&](int t) -> bool {
-        const int vb = t % L::kVConv, pb = t & 1;
-        if (!mbar_wait(vc_full + vb, (t / L::kVConv) & 1)) return false;
+        const int s = t % R, pb = t & 1;
+        if (!mbar_wait(vr_full + s, (t / R) & 1)) return false;
         if (!mbar_wait(p_full + pb, (t >> 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(vconv + vb * kConvTile);
+        const uint32_t v_addr = smem_u32(vraw + s * kRawTile);
         const uint32_t p_addr = smem_u32(ps + pb * L::kPBytes);
 #pragma unroll
-        for (int kk = 0; kk < kKeyTile / 16; ++kk)
-          mma_f16_ss(tmem_o, vt_mnmajor_sw128_desc(v_addr, kk), pt_mnmajor_desc(p_addr, kk),
-                     id_pv, (t > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kKeyTile / 32; ++kk)
+          mma_e4m3_ss(tmem_o, vt_e4m3_desc(v_addr, kk), pt_e4m3_desc(p_addr, kk), id_pv,
+                      (t > 0 || kk > 0) ? 1u : 0u);
         mma_commit(p_free + pb);
-        mma_commit(vc_empty + vb);
+        mma_commit(vr_empty + s);
         return true;
       };
       for (int i = 0; i < n_tiles && ok; ++i) {
-        const int sb = i & 1;
-        if (!mbar_wait(kc_full, i & 1)) { ok = false; break; }
+        const int s = i % R, sb = i & 1;
+        if (!mbar_wait(kr_full + s, (i / R) & 1)) { ok = false; break; }
         if (!mbar_wait(s_free + sb, ((i >> 1) & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t k_addr = smem_u32(kraw + s * kRawTile);
 #pragma unroll
-        for (int kk = 0; kk < kHeadDim / 16; ++kk)
-          mma_f16_ss(tmem_base + sb * H, kmajor_sw128_desc(k_addr, kk),
-                     q_kmajor_desc<H>(q_addr, kk), id_qk, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < kHeadDim / 32; ++kk)
+          mma_e4m3_ss(tmem_base + sb * 2 * H, k_e4m3_desc(k_addr, kk),
+                      q_e4m3_desc<2 * H>(q_addr, kk), id_qk, kk > 0 ? 1u : 0u);
         mma_commit(s_full + sb);
-        mma_commit(kc_empty);
+        mma_commit(kr_empty + s);
         if (i > 0 && !issue_pv(i - 1)) { ok = false; break; }
       }
       if (ok && !issue_pv(n_tiles - 1)) ok = false;
       mma_commit(mma_done);
       if (!mbar_wait(mma_done, 0)) ok = false;
-    }
-  } else if (warp >= 2 + 4 * fp8_halves<H>()) {
-    // ------------------------------------------------------------ conversion
-    const int ct = threadIdx.x - (64 + 128 * fp8_halves<H>());
-    const int t = ct & (kKeyTile - 1);  // row of the tile
-    constexpr bool kSplit = fp8_conv_warps<H>() == 8;
-    const bool do_k = !kSplit || ct < kKeyTile, do_v = !kSplit || ct >= kKeyTile;
-    for (int i = 0; i < n_tiles; ++i) {
-      const int s = i % R;
-      const bool valid = entry_row(k0 + i * kKeyTile + t) >= 0;
-      if (do_k) {
-        if (ok && !mbar_wait(kr_full + s, (i / R) & 1)) ok = false;
-        if (ok && !mbar_wait(kc_empty, (i & 1) ^ 1)) ok = false;
-        convert_row(kraw + s * kRawTile, kconv, t, valid);
-        fence_proxy_async_smem();
-        mbar_arrive(kc_full);
-        mbar_arrive(kr_empty + s);
-      }
-      if (do_v) {
-        const int vb = i % L::kVConv;
-        if (ok && !mbar_wait(vr_full + s, (i / R) & 1)) ok = false;
-        if (ok && !mbar_wait(vc_empty + vb, ((i / L::kVConv) & 1) ^ 1)) ok = false;
-        convert_row(vraw + s * kRawTile, vconv + vb * kConvTile, t, valid);
-        fence_proxy_async_smem();
-        mbar_arrive(vc_full + vb);
-        mbar_arrive(vr_empty + s);
-      }
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -396,11 +432,17 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     const int hoff = half * HH;
     const uint32_t lane_base = (uint32_t)(lg * 32) << 16;
     const uint64_t keep_policy = policy_evict_last();
-    float l[HH];
+    float l[HH], mr[HH];
 #pragma unroll
-    for (int h = 0; h < HH; ++h) l[h] = 0.f;
+    for (int h = 0; h < HH; ++h) {
+      l[h] = 0.f;
+      mr[h] = -INFINITY;
+    }
     if (t < HH) mref_s[hoff + t] = -INFINITY;
     group_bar_sync(half);
+    // V scales: |v_scale| <= vlim = 2^ev for every key seen; P' = p * v_scale * 2^-ev.
+    int ev = kNoScale;
+    float vlim = 0.f, vmul = 0.f;
     // Per-key scales (and validity) are loaded two tiles ahead so that their memory
     // latency overlaps the tiles in between instead of stalling each tile.
     auto scales_of = [&](int i, float& ks, float& vs, bool& ok_row) {
@@ -413,7 +455,8 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     bool val_next, val_far;
     scales_of(0, ks_next, vs_next, val_next);
     scales_of(1, ks_far, vs_far, val_far);
-    const float c2 = c2_s[0];  // sm_scale * log2(e) / (the Q scale, common to all heads)
+    const float qinv = qsc_s[0];
+    const float c2 = p.sm_scale * kLog2eF8 * qinv;  // Q-scaled logit -> log2 units
     for (int i = 0; i < n_tiles; ++i) {
       const int sb = i & 1;
       const int j = k0 + i * kKeyTile + t;
@@ -428,46 +471,50 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
       tc_fence_after();
       float x[HH];
       {
-        // Every chunk's load in flight before the one wait.
-        uint32_t r[HH];
+        // Every chunk's load in flight before the one wait: the Q_hi columns, then Q_lo.
+        uint32_t r[2 * HH];
 #pragma unroll
-        for (int c = 0; c < HH; c += 16)
-          tmem_ld16(tmem_base + lane_base + sb * H + hoff + c,
+        for (int c = 0; c < HH; c += 16) {
+          tmem_ld16(tmem_base + lane_base + sb * 2 * H + hoff + c,
                     *reinterpret_cast<uint32_t(*)[16]>(r + c));
-        tmem_wait_ld();
-        if (!GATHER && p.sbuf) {
-          if (j < k1 && j <= pos - p.window && pos - p.window + 1 > p.k_sel) {
-            float* dst = p.sbuf + ((size_t)bq * p.kv.max_len + j) * H + hoff;
-#pragma unroll
-            for (int e = 0; e < HH / 4; ++e) {
-              uint4 v;
-              v.x = __float_as_uint(__uint_as_float(r[4 * e]) * qinv_s[hoff + 4 * e] * ks);
-              v.y = __float_as_uint(__uint_as_float(r[4 * e + 1]) * qinv_s[hoff + 4 * e + 1] * ks);
-              v.z = __float_as_uint(__uint_as_float(r[4 * e + 2]) * qinv_s[hoff + 4 * e + 2] * ks);
-              v.w = __float_as_uint(__uint_as_float(r[4 * e + 3]) * qinv_s[hoff + 4 * e + 3] * ks);
-              st_global_v4_hint(dst + 4 * e, v, keep_policy);
-            }
-          }
+          tmem_ld16(tmem_base + lane_base + sb * 2 * H + H + hoff + c,
+                    *reinterpret_cast<uint32_t(*)[16]>(r + HH + c));
         }
-        const float cks = c2 * ks;  // one Q scale for every head: one multiplier per key
+        tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < HH; ++e) x[e] = valid ? __uint_as_float(r[e]) * cks : -INFINITY;
+        for (int e = 0; e < HH; ++e)
+          x[e] = fmaf(__uint_as_float(r[HH + e]), 0.0625f, __uint_as_float(r[e]));
       }
       tc_fence_before();
       mbar_arrive(s_free + sb);
-      // This group's references: read once per tile into registers up to 16 heads per
-      // thread; above, from shared memory at each use (registers are the limit there).
-      constexpr bool kRefRegs = HH <= 16;
-      float mr[kRefRegs ? HH : 1];
-      if (kRefRegs) {
+      if (!GATHER && p.sbuf) {
+        if (j < k1 && j <= pos - p.window && pos - p.window + 1 > p.k_sel) {
+          const float qk = qinv * ks;  // the stored logit is q.k times the key's scale
+          float* dst = p.sbuf + ((size_t)bq * p.kv.max_len + j) * H + hoff;
 #pragma unroll
-        for (int h = 0; h < HH; ++h) mr[h] = mref_s[hoff + h];
+          for (int e = 0; e < HH / 4; ++e) {
+            uint4 v;
+            v.x = __float_as_uint(x[4 * e] * qk);
+            v.y = __float_as_uint(x[4 * e + 1] * qk);
+            v.z = __float_as_uint(x[4 * e + 2] * qk);
+            v.w = __float_as_uint(x[4 * e + 3] * qk);
+            st_global_v4_hint(dst + 4 * e, v, keep_policy);
+          }
+        }
       }
-      auto ref = [&](int h) { return kRefRegs ? mr[kRefRegs ? h : 0] : mref_s[hoff + h]; };
-      bool over = false;
+      const float cks = c2 * ks;  // one Q scale for every head: one multiplier per key
 #pragma unroll
-      for (int h = 0; h < HH; ++h) over |= x[h] - ref(h) > kRescaleAtF8;
+      for (int e = 0; e < HH; ++e) x[e] = valid ? x[e] * cks : -INFINITY;
+      bool over = valid && fabsf(vs) > vlim;
+#pragma unroll
+      for (int h = 0; h < HH; ++h) over |= x[h] - mr[h] > kRescaleAtF8;
       if (group_bar_or(half, over)) {
+        // Move the references to the tile maxima where these are higher, and the V
+        // exponent to cover the largest |v_scale| of the tile; rescale l and O.
+        {
+          const float vm = warp_max(valid ? fabsf(vs) : 0.f);
+          if (lane_id() == 0) red[4 * H + 4 * half + (t >> 5)] = vm;
+        }
         block_max_group_f8<HH, H>(x, red, alpha_s, t, hoff, half);
         if (t < HH) {
           const int h = hoff + t;
@@ -475,24 +522,45 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
           alpha_s[h] = exp2f(mref_s[h] - mnew);
           mref_s[h] = mnew;
         }
+        if (t == 0) {
+          const float* vr = red + 4 * H + 4 * half;
+          const float vmax = fmaxf(fmaxf(vr[0], vr[1]), fmaxf(vr[2], vr[3]));
+          const int e_old = ev_s[half];
+          int e_new = e_old;
+          if (vmax > 0.f) {
+            int ex;
+            frexpf(vmax, &ex);  // vmax < 2^ex
+            ex = ex < -126 ? -126 : ex;
+            if (ex > e_old) e_new = ex;
+          }
+          beta_s[half] = e_new == e_old ? 1.f : (e_old == kNoScale ? 0.f : ldexpf(1.f, e_old - e_new));
+          ev_s[half] = e_new;
+        }
         group_bar_sync(half);
+        const float beta = beta_s[half];
+        ev = ev_s[half];
+        vlim = ev == kNoScale ? 0.f : ldexpf(1.f, ev);
+        vmul = ev == kNoScale ? 0.f : ldexpf(1.f, -ev);
 #pragma unroll
         for (int h = 0; h < HH; ++h) {
           l[h] *= alpha_s[hoff + h];
-          if (kRefRegs) mr[kRefRegs ? h : 0] = mref_s[hoff + h];
+          mr[h] = mref_s[hoff + h];
         }
         if (i > 0) {
           if (ok && !mbar_wait(p_free + ((i - 1) & 1), ((i - 1) >> 1) & 1)) ok = false;
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < HH; c += 16) {
-            uint32_t r[16];
-            tmem_ld16(tmem_o + lane_base + hoff + c, r);
-            tmem_wait_ld();
+          for (int term = 0; term < 3; ++term) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha_s[hoff + c + e]);
-            tmem_st16(tmem_o + lane_base + hoff + c, r);
+            for (int c = 0; c < HH; c += 16) {
+              uint32_t r[16];
+              tmem_ld16(tmem_o + lane_base + term * H + hoff + c, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                r[e] = __float_as_uint(__uint_as_float(r[e]) * (alpha_s[hoff + c + e] * beta));
+              tmem_st16(tmem_o + lane_base + term * H + hoff + c, r);
+            }
           }
           tmem_wait_st();
           tc_fence_before();
@@ -500,23 +568,51 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
       }
       if (ok && i >= 2 && !mbar_wait(p_free + sb, ((i >> 1) & 1) ^ 1)) ok = false;
       uint8_t* pb = ps + sb * L::kPBytes;
+      const float vsc = valid ? vs * vmul : 0.f;
 #pragma unroll
-      for (int c = 0; c < HH / 8; ++c) {
-        uint32_t w[4];
+      for (int c = 0; c < HH / 16; ++c) {
+        uint32_t w0[4], w1[4], w2[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int h0 = c * 8 + 2 * e;
-          // A head whose reference is still -inf has seen no key: its p is 0 (not
-          // 2^(-inf - -inf)), so a leading all-padding tile leaves O and l at zero.
-          const float p0 = ex2_ftz(x[h0] - finite_ref(ref(h0)));
-          const float p1 = ex2_ftz(x[h0 + 1] - finite_ref(ref(h0 + 1)));
-          l[h0] += p0;
-          l[h0 + 1] += p1;
-          const __half2 v2 = __floats2half2_rn(p0 * vs, p1 * vs);
-          w[e] = *reinterpret_cast<const uint32_t*>(&v2);
+          w0[e] = 0u;
+          w1[e] = 0u;
+          w2[e] = 0u;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int h0 = c * 16 + 4 * e + 2 * u;
+            // A head whose reference is still -inf has seen no key: its p is 0 (not
+            // 2^(-inf - -inf)), so a leading all-padding tile leaves O and l at zero.
+            const float p0 = ex2_ftz(x[h0] - finite_ref(mr[h0]));
+            const float p1 = ex2_ftz(x[h0 + 1] - finite_ref(mr[h0 + 1]));
+            l[h0] += p0;
+            l[h0 + 1] += p1;
+            const float y0 = p0 * vsc, y1 = p1 * vsc;
+            float a0, a1, b0, b1;
+            const uint32_t ch = e4m3_pair(y0, y1, a0, a1);
+            const float r0 = (y0 - a0) * 16.f, r1 = (y1 - a1) * 16.f;
+            const uint32_t cl = e4m3_pair(r0, r1, b0, b1);
+            const uint32_t cl2 = e4m3_codes((r0 - b0) * 16.f, (r1 - b1) * 16.f);
+            w0[e] |= ch << (16 * u);
+            w1[e] |= cl << (16 * u);
+            w2[e] |= cl2 << (16 * u);
+          }
         }
-        *reinterpret_cast<uint4*>(pb + (hoff / 8 + c) * (kKeyTile * 16) + t * 16) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+        const int ch0 = (hoff >> 4) + c;  // chunk of this head group's 16 heads, term 0
+        *reinterpret_cast<uint4*>(pb + ch0 * (kKeyTile * 16) + t * 16) =
+            make_uint4(w0[0], w0[1], w0[2], w0[3]);
+        *reinterpret_cast<uint4*>(pb + (ch0 + H / 16) * (kKeyTile * 16) + t * 16) =
+            make_uint4(w1[0], w1[1], w1[2], w1[3]);
+        *reinterpret_cast<uint4*>(pb + (ch0 + 2 * (H / 16)) * (kKeyTile * 16) + t * 16) =
+            make_uint4(w2[0], w2[1], w2[2], w2[3]);
+      }
+      if (!GATHER && !valid && half == 0 && i == n_tiles - 1) {
+        // Rows past the chunk end may hold anything (NaN codes included); 0 * NaN would
+        // poison P.V, so zero this key's V row once its tile has landed.
+        const int s = i % R;
+        if (ok && !mbar_wait(vr_full + s, (i / R) & 1)) ok = false;
+        uint4* v0 = reinterpret_cast<uint4*>(vraw + s * kRawTile + t * 128);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v0[e] = make_uint4(0, 0, 0, 0);
       }
       fence_proxy_async_smem();
       mbar_arrive(p_full + sb);
@@ -525,14 +621,20 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     const int last = n_tiles - 1;
     if (ok && !mbar_wait(p_free + (last & 1), (last >> 1) & 1)) ok = false;
     tc_fence_after();
+    const float oscale = ev == kNoScale ? 0.f : ldexpf(1.f, ev);
 #pragma unroll
     for (int c = 0; c < HH; c += 16) {
-      uint32_t r[16];
-      tmem_ld16(tmem_o + lane_base + hoff + c, r);
+      uint32_t r0[16], r1[16], r2[16];
+      tmem_ld16(tmem_o + lane_base + hoff + c, r0);
+      tmem_ld16(tmem_o + lane_base + H + hoff + c, r1);
+      tmem_ld16(tmem_o + lane_base + 2 * H + hoff + c, r2);
       tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 16; ++e)
-        part_o[(hoff + c + e) * kHeadDim + t] = __uint_as_float(r[e]);
+      for (int e = 0; e < 16; ++e) {
+        const float o = fmaf(__uint_as_float(r2[e]), 0.00390625f,
+                             fmaf(__uint_as_float(r1[e]), 0.0625f, __uint_as_float(r0[e])));
+        part_o[(hoff + c + e) * kHeadDim + t] = o * oscale;
+      }
     }
     tc_fence_before();
 #pragma unroll

@@ -126,6 +126,7 @@ struct SelectParams {
   int32_t* band_j;
   int32_t* idx;
   uint32_t* status;
+  int block = 1;  // 1: token-level selection; > 1: whole blocks of this many positions
 };
 
 // Appending new tokens (KV append with FP8 quantisation of the new rows).
