@@ -36,6 +36,7 @@ UNIT = "steps/s"
 FLUSH_BYTES = 256 << 20
 LAUNCHES_PER_STEP_FULL = 2      # split-K flash-decode, split merge
 LAUNCHES_PER_STEP_SELECT = 3    # importance+histogram, compaction, exact finish
+LAUNCHES_PER_STEP_BLOCKS = 2    # importance, exact block selection
 LAUNCHES_PER_SPARSE = 1         # gather attention with the split merge on chip (cluster)
 
 
@@ -176,7 +177,8 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-def oracle_sample(inp: workloads.Inputs, w: workloads.Workload, budget_s: float):
+def oracle_sample(inp: workloads.Inputs, w: workloads.Workload, budget_s: float,
+                  block: int = 1):
     """Time the float64 oracle on whole sequences of the workload until `budget_s`
     has passed (at least one).  Returns (seconds, sequences done)."""
     import oracle
@@ -190,7 +192,7 @@ def oracle_sample(inp: workloads.Inputs, w: workloads.Workload, budget_s: float)
             if sub[key] is not None:
                 sub[key] = bits[key][b:b + 1]
         sub["q_layers"] = [ql[b:b + 1] for ql in bits["q_layers"]]
-        oracle.hybrid_block_step(sub)
+        oracle.hybrid_block_step(sub, block)
         done += 1
         if time.perf_counter() - t0 >= budget_s:
             break
@@ -211,10 +213,10 @@ def run_reference(args, w):
         return
     inp = workloads.generate(w)
     for _ in range(args.warmup):
-        oracle_sample(inp, w, 0.0)
+        oracle_sample(inp, w, 0.0, args.block)
     secs, seqs = 0.0, 0
     for _ in range(args.steps):
-        s, n = oracle_sample(inp, w, 0.0)
+        s, n = oracle_sample(inp, w, 0.0, args.block)
         secs += s
         seqs += n
     value = seqs / (secs * w.batch)
@@ -222,7 +224,7 @@ def run_reference(args, w):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_of(w),
+        "data": "synthetic", "config": config_of(w, args.block),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
                          "sample": f"{seqs} whole sequences of the batch, one per step, "
                                    "full layer + selection + every sparse layer in float64"},
@@ -231,8 +233,9 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-def config_of(w):
+def config_of(w, block: int = 1):
     return {"workload": w.name, "batch": w.batch, "context": w.max_len,
+            "selection": "token" if block == 1 else f"blocks of {block} positions",
             "ragged_from": w.len_lo, "n_q": w.n_q, "h_q": w.h_q, "h_kv": 1, "head_dim": 128,
             "kv_cache": w.kv, "window": w.window, "k_sel": w.k_sel, "sparse_layers": w.n_sparse,
             "l2": "flushed before every timed step (256 MiB write, then 256 MiB read of "
@@ -250,6 +253,9 @@ def main():
                     help="seconds of oracle time for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--block", type=int, default=1,
+                    help="1: token-level selection (the method); N > 1: whole blocks of N "
+                         "positions (the first-generation comparator)")
     ap.add_argument("--batch", type=int, default=None,
                     help="run fewer sequences of the workload (profiling captures only)")
     args = ap.parse_args()
@@ -315,7 +321,10 @@ def main():
         hs2.full_attn(q, cache, w.window, w.k_sel, inp.sm_scale, ws, out=out, lse=lse)
         if with_marks:
             mark(1)
-        hs2.select(q, cache, ws, w.window, w.k_sel, inp.sm_scale, idx=idx)
+        if args.block > 1:
+            hs2.select_blocks(q, cache, ws, w.window, w.k_sel, args.block, inp.sm_scale, idx=idx)
+        else:
+            hs2.select(q, cache, ws, w.window, w.k_sel, inp.sm_scale, idx=idx)
         if with_marks:
             mark(2)
         for ql, o in zip(qls, outs):
@@ -402,8 +411,12 @@ def main():
             q.copy_(hq, non_blocking=True)
             for d_, h_ in zip(qls, hqls):
                 d_.copy_(h_, non_blocking=True)
-            hs2.full_attn_select(q, cache, w.window, w.k_sel, inp.sm_scale, ws, out=out,
-                                 idx=idx, lse=lse)
+            if args.block > 1:
+                hs2.full_attn_select_blocks(q, cache, w.window, w.k_sel, args.block,
+                                            inp.sm_scale, ws, out=out, idx=idx, lse=lse)
+            else:
+                hs2.full_attn_select(q, cache, w.window, w.k_sel, inp.sm_scale, ws, out=out,
+                                     idx=idx, lse=lse)
             for ql, o in zip(qls, outs):
                 hs2.sparse_attn(ql, cache, idx, ws, inp.sm_scale, out=o)
             hout.copy_(out, non_blocking=True)
@@ -448,7 +461,7 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.kv == "bf16" else "fp8-e4m3",
-        "data": "synthetic", "config": config_of(w),
+        "data": "synthetic", "config": config_of(w, args.block),
         "hbm_gbs": ab["step"] / (total_ms / args.steps / 1e3) / 1e9,
         "alg_bytes_per_step": ab["step"],
         "phase_ms": {"full_attn": statistics.mean(full_ms), "select": statistics.mean(sel_ms),
@@ -464,7 +477,9 @@ def main():
                      "traffic_source": (NCU_TRAFFIC[args.workload]
                                         if args.workload in NCU_TRAFFIC and args.batch is None
                                         else None)},
-        "gpu_launches": args.steps * (LAUNCHES_PER_STEP_FULL + LAUNCHES_PER_STEP_SELECT
+        "gpu_launches": args.steps * (LAUNCHES_PER_STEP_FULL
+                                      + (LAUNCHES_PER_STEP_BLOCKS if args.block > 1
+                                         else LAUNCHES_PER_STEP_SELECT)
                                       + w.n_sparse * LAUNCHES_PER_SPARSE),
         "clocks": clk.summary(),
         "device_status": status,
@@ -473,7 +488,7 @@ def main():
     if e2e is not None:
         line["e2e"] = e2e
     if not args.no_cpu_baseline:
-        secs, seqs = oracle_sample(inp, w, args.cpu_budget)
+        secs, seqs = oracle_sample(inp, w, args.cpu_budget, args.block)
         cv = seqs / (secs * w.batch)
         line["cpu_baseline"] = {"value": cv, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
                                 "sample": f"{seqs} one-sequence hybrid-block steps (sequences "

@@ -130,6 +130,36 @@ HS2_API hs2_status hs2_select(const void* q, int n_q, int h_q, const hs2_kv* kv,
                       int k_sel, float sm_scale, int32_t* idx, void* workspace,
                       size_t ws_bytes, hs2_stream_t stream);
 
+/* Block-level selection, the first-generation scheme that the pages set token-level
+ * selection against ("Luo Fuli Teases Xiaomi MiMo-V3 Architecture ...", paragraphs on
+ * block selection with 64-token blocks and on the ablation at the same attention
+ * budget): a comparator, not the method's own step.
+ *   block    positions per block (the pages' blocks hold 64), >= 2; k_sel must be a
+ *            multiple of block and k_sel / block <= 1024.
+ *   idx      device int32 [batch][n_q][window + k_sel]: positions [0, p-window] form
+ *            aligned blocks [c*block, (c+1)*block), the last one cut at p-window; a
+ *            block scores the largest importance among its positions (a reading: the
+ *            pages give no block score); the k_sel / block best blocks, ties to the
+ *            lower block, are kept whole, in ascending order, then the window
+ *            [p-window+1, p], then -1.  With no more blocks than k_sel / block, all of
+ *            [0, p].
+ * Other arguments, workspace and ordering as hs2_full_attn_select / hs2_select.
+ * HS2_ERR_UNSUPPORTED for a block size outside these limits, or when the row's
+ * ceil(max_len / block) block keys do not fit the kernel's shared memory (about
+ * 40000 blocks at 16 heads). */
+HS2_API hs2_status hs2_full_attn_select_blocks(const void* q, int n_q, int h_q,
+                                               const hs2_kv* kv, int window, int k_sel,
+                                               int block, float sm_scale, float* out,
+                                               int32_t* idx, float* lse, void* workspace,
+                                               size_t ws_bytes, hs2_stream_t stream);
+
+/* Block-level selection alone; must follow hs2_full_attn with the same q, kv, sizes
+ * and workspace, on the same stream. */
+HS2_API hs2_status hs2_select_blocks(const void* q, int n_q, int h_q, const hs2_kv* kv,
+                                     int window, int k_sel, int block, float sm_scale,
+                                     int32_t* idx, void* workspace, size_t ws_bytes,
+                                     hs2_stream_t stream);
+
 /* One reusing sparse-attention layer (step 3).
  *   q_layer   device bf16 [batch][n_q][h_q][128], this layer's queries.
  *   idx       device int32 [batch][n_q][idx_width]: positions to attend to (any

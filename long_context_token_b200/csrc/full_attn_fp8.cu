@@ -432,12 +432,16 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     const int hoff = half * HH;
     const uint32_t lane_base = (uint32_t)(lg * 32) << 16;
     const uint64_t keep_policy = policy_evict_last();
-    float l[HH], mr[HH];
+    // This group's references: in registers up to 16 heads per thread; above, read
+    // from shared memory at each use (registers are the limit there).
+    constexpr bool kRefRegs = HH <= 16;
+    float l[HH], mr[kRefRegs ? HH : 1];
 #pragma unroll
     for (int h = 0; h < HH; ++h) {
       l[h] = 0.f;
-      mr[h] = -INFINITY;
+      if (kRefRegs) mr[kRefRegs ? h : 0] = -INFINITY;
     }
+    auto ref = [&](int h) { return kRefRegs ? mr[kRefRegs ? h : 0] : mref_s[hoff + h]; };
     if (t < HH) mref_s[hoff + t] = -INFINITY;
     group_bar_sync(half);
     // V scales: |v_scale| <= vlim = 2^ev for every key seen; P' = p * v_scale * 2^-ev.
@@ -507,7 +511,7 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
       for (int e = 0; e < HH; ++e) x[e] = valid ? x[e] * cks : -INFINITY;
       bool over = valid && fabsf(vs) > vlim;
 #pragma unroll
-      for (int h = 0; h < HH; ++h) over |= x[h] - mr[h] > kRescaleAtF8;
+      for (int h = 0; h < HH; ++h) over |= x[h] - ref(h) > kRescaleAtF8;
       if (group_bar_or(half, over)) {
         // Move the references to the tile maxima where these are higher, and the V
         // exponent to cover the largest |v_scale| of the tile; rescale l and O.
@@ -544,7 +548,7 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
 #pragma unroll
         for (int h = 0; h < HH; ++h) {
           l[h] *= alpha_s[hoff + h];
-          mr[h] = mref_s[hoff + h];
+          if (kRefRegs) mr[kRefRegs ? h : 0] = mref_s[hoff + h];
         }
         if (i > 0) {
           if (ok && !mbar_wait(p_free + ((i - 1) & 1), ((i - 1) >> 1) & 1)) ok = false;
@@ -582,8 +586,8 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
             const int h0 = c * 16 + 4 * e + 2 * u;
             // A head whose reference is still -inf has seen no key: its p is 0 (not
             // 2^(-inf - -inf)), so a leading all-padding tile leaves O and l at zero.
-            const float p0 = ex2_ftz(x[h0] - finite_ref(mr[h0]));
-            const float p1 = ex2_ftz(x[h0 + 1] - finite_ref(mr[h0 + 1]));
+            const float p0 = ex2_ftz(x[h0] - finite_ref(ref(h0)));
+            const float p1 = ex2_ftz(x[h0 + 1] - finite_ref(ref(h0 + 1)));
             l[h0] += p0;
             l[h0 + 1] += p1;
             const float y0 = p0 * vsc, y1 = p1 * vsc;

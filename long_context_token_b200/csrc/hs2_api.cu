@@ -245,7 +245,7 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
 
 static hs2_status run_select(const void* q, int n_q, int h, const hs2_kv* kv, int window,
                              int k_sel, float sm_scale, int32_t* idx, void* ws,
-                             const WsLayout& w, cudaStream_t s) {
+                             const WsLayout& w, cudaStream_t s, int block = 1) {
   // The histogram and counters start at zero: the workspace is zero-filled before first
   // use and every selection leaves them at zero when it finishes.
   cudaError_t e = cudaSuccess;
@@ -274,6 +274,7 @@ static hs2_status run_select(const void* q, int n_q, int h, const hs2_kv* kv, in
   p.band_j = ws_ptr<int32_t>(ws, w.band_j);
   p.idx = idx;
   p.status = ws_ptr<uint32_t>(ws, w.status);
+  p.block = block;
   const int bq = kv->batch * n_q;
   if (w.use_sbuf) {
     // The stored logits come from the one-token tensor-core full layer (h = 16 <= 64).
@@ -389,6 +390,45 @@ hs2_status hs2_full_attn_select(const void* q, int n_q, int h_q, const hs2_kv* k
   if (st != HS2_OK) return st;
   return run_select(q, n_q, h_q, kv, window, k_sel, sm_scale, idx, workspace, P.w,
                     (cudaStream_t)stream);
+}
+
+// Block-level selection: whole blocks of `block` positions, k_sel a multiple of block,
+// at most 1024 blocks kept, and the per-block keys of a row in the kernel's shared memory.
+static hs2_status check_blocks(const hs2_kv* kv, int h, int k_sel, int block) {
+  if (block < 2 || k_sel % block != 0) return HS2_ERR_UNSUPPORTED;
+  if (k_sel / block > 1024) return HS2_ERR_UNSUPPORTED;
+  if (select_blocks_smem(h, kv->max_len, block) > 200u * 1024u) return HS2_ERR_UNSUPPORTED;
+  return HS2_OK;
+}
+
+hs2_status hs2_select_blocks(const void* q, int n_q, int h_q, const hs2_kv* kv, int window,
+                             int k_sel, int block, float sm_scale, int32_t* idx,
+                             void* workspace, size_t ws_bytes, hs2_stream_t stream) {
+  Prepared P;
+  hs2_status st = prepare(q, n_q, h_q, kv, window, k_sel, workspace, ws_bytes, &P);
+  if (st != HS2_OK) return st;
+  st = check_blocks(kv, h_q, k_sel, block);
+  if (st != HS2_OK) return st;
+  if (!idx) return HS2_ERR_INVALID_ARGUMENT;
+  return run_select(q, n_q, h_q, kv, window, k_sel, sm_scale, idx, workspace, P.w,
+                    (cudaStream_t)stream, block);
+}
+
+hs2_status hs2_full_attn_select_blocks(const void* q, int n_q, int h_q, const hs2_kv* kv,
+                                       int window, int k_sel, int block, float sm_scale,
+                                       float* out, int32_t* idx, float* lse, void* workspace,
+                                       size_t ws_bytes, hs2_stream_t stream) {
+  Prepared P;
+  hs2_status st = prepare(q, n_q, h_q, kv, window, k_sel, workspace, ws_bytes, &P);
+  if (st != HS2_OK) return st;
+  st = check_blocks(kv, h_q, k_sel, block);
+  if (st != HS2_OK) return st;
+  if (!out || !aligned16(out) || !idx) return HS2_ERR_INVALID_ARGUMENT;
+  st = run_full(q, n_q, h_q, kv, window, k_sel, sm_scale, out, lse, workspace, P.w,
+                (cudaStream_t)stream);
+  if (st != HS2_OK) return st;
+  return run_select(q, n_q, h_q, kv, window, k_sel, sm_scale, idx, workspace, P.w,
+                    (cudaStream_t)stream, block);
 }
 
 hs2_status hs2_sparse_attn(const void* q_layer, int n_q, int h_q, const hs2_kv* kv,

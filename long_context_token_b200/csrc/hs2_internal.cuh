@@ -202,6 +202,7 @@ cudaError_t launch_full_attn(const FullParams& p, int batch, cudaStream_t s);
 cudaError_t launch_select(const SelectParams& p, int batch, cudaStream_t s);
 // The selection after the importance pass (compaction + finish).
 cudaError_t launch_select_rest(const SelectParams& p, int batch, cudaStream_t s);
+size_t select_blocks_smem(int h, int max_len, int block);
 // Importance from the full layer's stored float32 logits.
 cudaError_t launch_importance_sbuf(const SelectParams& p, int bq, cudaStream_t s);
 // The stored-logit path applies to single-token decode with 16 heads: 64 bytes of

@@ -864,6 +864,238 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
 }
 
 // ----------------------------------------------------------------------------
+// 4. block-level selection (the first-generation scheme, a comparator)
+// ----------------------------------------------------------------------------
+// Positions [0, n_c) form aligned blocks of p.block positions, the last one cut at
+// n_c.  A block's key is the largest float32 key t of its positions (t orders the
+// positions as their importance does, and the maximum commutes with that order).
+// The kb = k_sel / block best blocks are kept whole, ties to the lower block: tau is
+// the kb-th largest block key; blocks above tau + eps are kept, and the blocks inside
+// [tau - eps, tau + eps] get their exact score -- the float64 maximum over their
+// positions of max_h(s_hj - delta_h), re-scored from the stored inputs as in the finish
+// kernel -- and are ranked by (score desc, block asc).  Output: the kept blocks'
+// positions in order, then the window, then -1.
+constexpr int kBlkThreads = 1024;
+constexpr int kBlkSmallBand = 1024;  // bands up to this size are ranked in shared memory
+
+__host__ __device__ constexpr size_t blocks_dyn_smem(int H, int max_blocks) {
+  return (size_t)H * kQLd * sizeof(uint16_t) + (size_t)(kBlkThreads / 32) * kHeadDim * sizeof(double) +
+         (size_t)max_blocks * sizeof(float);
+}
+
+template <int H, bool FP8>
+__global__ void __launch_bounds__(kBlkThreads) select_blocks_kernel(SelectParams p) {
+  extern __shared__ __align__(16) unsigned char blk_dyn[];
+  uint16_t* qsm = reinterpret_cast<uint16_t*>(blk_dyn);  // [H][kQLd] bf16 q of this query
+  double* kdsm = reinterpret_cast<double*>(blk_dyn + (size_t)H * kQLd * sizeof(uint16_t));
+  float* bkey = reinterpret_cast<float*>(kdsm + (kBlkThreads / 32) * kHeadDim);  // [n_blk]
+  __shared__ double dlt[H];
+  __shared__ unsigned long long band_key[kBlkSmallBand];  // exact scores, ordered keys
+  __shared__ int band_blk[kBlkSmallBand];
+  __shared__ int chosen[kMaxIdxWidth / 2];
+  __shared__ uint32_t n_keep_s, n_band_s, gt_s;
+  griddep_wait();
+  const int bq = blockIdx.x;
+  const int b = bq / p.n_q, i = bq % p.n_q;
+  const int L = seq_len(p.kv, b, p.n_q, p.status, false);
+  const int pos = L - p.n_q + i;
+  const int width = p.window + p.k_sel;
+  const int n_c = pos - p.window + 1;
+  const int blk = p.block, kb = p.k_sel / p.block;
+  const int n_blk = n_c > 0 ? (n_c + blk - 1) / blk : 0;
+  int32_t* out = p.idx + (size_t)bq * width;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int kWarps = kBlkThreads / 32;
+  if (n_blk > kb) {
+    for (int e = threadIdx.x; e < H * (kHeadDim / 8); e += blockDim.x) {
+      const int h = e / (kHeadDim / 8), c = (e % (kHeadDim / 8)) * 8;
+      *reinterpret_cast<uint4*>(qsm + h * kQLd + c) =
+          *reinterpret_cast<const uint4*>(p.q + ((size_t)bq * H + h) * kHeadDim + c);
+    }
+    load_delta(p.lse64 + (size_t)bq * H, H, nullptr, dlt);  // (synchronises the block)
+    // Block keys: one thread per block, its positions read with independent 16-byte
+    // loads where the row is aligned (many loads in flight instead of one per warp).
+    const float* trow = p.tbuf + (size_t)bq * p.kv.max_len;
+    for (int c = threadIdx.x; c < n_blk; c += blockDim.x) {
+      const int j0 = c * blk, j1 = min(j0 + blk, n_c);
+      float m = -INFINITY;
+      int j = j0;
+      if ((reinterpret_cast<uintptr_t>(trow + j0) & 15u) == 0) {
+#pragma unroll 8
+        for (; j + 4 <= j1; j += 4) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(trow + j));
+          m = fmaxf(m, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+        }
+      }
+      for (; j < j1; ++j) m = fmaxf(m, __ldcg(trow + j));
+      bkey[c] = m;
+    }
+    if (threadIdx.x == 0) {
+      n_keep_s = 0u;
+      n_band_s = 0u;
+    }
+    __syncthreads();
+    const uint32_t tau_key = block_kth_largest<uint32_t, 32>(
+        n_blk, kb, [&](int e) { return ordered_key(bkey[e]); }, [](int) { return true; }, &gt_s);
+    const float tau = key_to_float(tau_key);
+    double dmax = 0.0;
+    for (int h = 0; h < H; ++h) dmax = fmax(dmax, dlt[h]);
+    const float eps = kEpsRel * fmaxf(1.f, fabsf(tau) + (float)dmax);
+    const float hi_b = tau + eps, lo_b = tau - eps;
+    // Blocks above the band are kept (fewer than kb: their keys exceed the kb-th);
+    // band blocks are listed for re-scoring (shared memory while the band is small,
+    // else the workspace).
+    int32_t* bj = p.band_j + (size_t)bq * p.kv.max_len;
+    unsigned long long* bk = reinterpret_cast<unsigned long long*>(p.band_t + (size_t)bq * p.kv.max_len);
+    const int n_blk_r = (n_blk + 31) & ~31;
+    for (int c = threadIdx.x; c < n_blk_r; c += blockDim.x) {
+      const bool in = c < n_blk;
+      const float t = in ? bkey[c] : -INFINITY;
+      const bool keep = in && t > hi_b;
+      const bool band = in && !keep && t >= lo_b;
+      const uint32_t sk = warp_slot(keep, &n_keep_s);
+      if (keep && sk < (uint32_t)(kMaxIdxWidth / 2)) chosen[sk] = c;
+      const uint32_t sb = warp_slot(band, &n_band_s);
+      if (band) {
+        bj[sb] = c;
+        bk[sb] = 0ull;
+        if (sb < (uint32_t)kBlkSmallBand) {
+          band_blk[sb] = c;
+          band_key[sb] = 0ull;
+        }
+      }
+    }
+    __syncthreads();
+    const int n_band = (int)n_band_s;
+    const bool band_smem = n_band <= kBlkSmallBand;
+    const int need2 = kb - (int)n_keep_s;  // >= 1: tau's own block is in the band
+    // float64 re-scoring of every position of the band blocks, one warp per position
+    // (row widened to float64 in shared memory, lanes over heads or head parts); each
+    // block's score is the maximum over its positions (atomic max on ordered keys).
+    constexpr int kParts = H < 32 ? 32 / H : 1;
+    constexpr int kSpan = kHeadDim / kParts;
+    const int part = kParts > 1 ? lane / H : 0;
+    const double scale = (double)p.sm_scale;
+    double* kd = kdsm + warp * kHeadDim;
+    const long long n_pos = (long long)n_band * blk;
+    for (long long f = warp; f < n_pos; f += kWarps) {
+      const int e = (int)(f / blk);
+      const int c = band_smem ? band_blk[e] : __ldcg(bj + e);
+      const int j = c * blk + (int)(f % blk);
+      // Past the cut last block, or a position that cannot hold the block's exact
+      // maximum: its float32 key is more than eps below the block's (each float32 key
+      // is within eps / 2 of the exact one).  Both uniform over the warp.
+      if (j >= n_c || __ldcg(trow + j) < bkey[c] - eps) continue;
+      const size_t row = (size_t)b * p.kv.max_len + j;
+      if (FP8) {
+        const uint32_t w4 =
+            __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(p.kv.k) +
+                                                    row * kHeadDim) + lane);
+        const double ksc = (double)__ldg(p.kv.k_scale + row);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) kd[4 * lane + u] = e4m3_to_f64((w4 >> (8 * u)) & 0xffu) * ksc;
+      } else {
+        const uint2 w4 = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.kv.k) +
+                                                              row * kHeadDim) + lane);
+        kd[4 * lane] = (double)bf16_bits_to_f32(w4.x & 0xffffu);
+        kd[4 * lane + 1] = (double)bf16_bits_to_f32(w4.x >> 16);
+        kd[4 * lane + 2] = (double)bf16_bits_to_f32(w4.y & 0xffffu);
+        kd[4 * lane + 3] = (double)bf16_bits_to_f32(w4.y >> 16);
+      }
+      __syncwarp();
+      double best = -INFINITY;
+      for (int h0 = 0; h0 < H; h0 += 32 / kParts) {
+        const int h = h0 + (kParts > 1 ? lane % H : lane);
+        double dot = 0.0;
+        if (h < H) {
+          const uint16_t* qh = qsm + h * kQLd;
+#pragma unroll 4
+          for (int cc = part * kSpan; cc < (part + 1) * kSpan; cc += 8) {
+            const uint4 qv = *reinterpret_cast<const uint4*>(qh + cc);
+            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              dot = fma((double)bf16_bits_to_f32(qw[u] & 0xffffu), kd[cc + 2 * u], dot);
+              dot = fma((double)bf16_bits_to_f32(qw[u] >> 16), kd[cc + 2 * u + 1], dot);
+            }
+          }
+        }
+#pragma unroll
+        for (int o = 16; o >= 32 / kParts && kParts > 1; o >>= 1)
+          dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        if (h < H) best = fmax(best, scale * dot - dlt[h]);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) best = fmax(best, __shfl_xor_sync(0xffffffffu, best, o));
+      if (lane == 0) {
+        if (band_smem) atomicMax(&band_key[e], ordered_key64(best));
+        else atomicMax(bk + e, ordered_key64(best));
+      }
+      __syncwarp();  // the next position reuses kd
+    }
+    __syncthreads();
+    if (band_smem) {
+      // Small band: rank every block by (score desc, block asc) against the others.
+      for (int e = threadIdx.x; e < n_band; e += blockDim.x) {
+        const unsigned long long ke = band_key[e];
+        const int ce = band_blk[e];
+        int rank = 0;
+        for (int f = 0; f < n_band; ++f) {
+          const unsigned long long kf = band_key[f];
+          rank += (kf > ke) || (kf == ke && band_blk[f] < ce);
+        }
+        if (rank < need2) chosen[atomicAdd(&n_keep_s, 1u)] = ce;
+      }
+    } else {
+      // Boundary score among the band, then the lowest blocks among its ties.
+      const unsigned long long vb = block_kth_largest<unsigned long long, 64>(
+          n_band, need2, [&](int e) { return __ldcg(bk + e); }, [](int) { return true; }, &gt_s);
+      const int take_eq = need2 - (int)gt_s;
+      const uint32_t cb_inv = block_kth_largest<uint32_t, 32>(
+          n_band, take_eq, [&](int e) { return ~(uint32_t)__ldcg(bj + e); },
+          [&](int e) { return __ldcg(bk + e) == vb; }, &gt_s);
+      const int cb = (int)~cb_inv;
+      for (int e = threadIdx.x; e < n_band; e += blockDim.x) {
+        const unsigned long long ke = __ldcg(bk + e);
+        const int ce = __ldcg(bj + e);
+        if (ke > vb || (ke == vb && ce <= cb)) chosen[atomicAdd(&n_keep_s, 1u)] = ce;
+      }
+    }
+    __syncthreads();
+    // kb blocks in ascending order (rank of each among the kept), then their positions:
+    // every kept block is whole except possibly the cut last block, which sorts last.
+    int* sorted = reinterpret_cast<int*>(band_blk);  // the band lists are no longer needed
+    for (int e = threadIdx.x; e < kb; e += blockDim.x) {
+      const int ce = chosen[e];
+      int rank = 0;
+      for (int f = 0; f < kb; ++f) rank += chosen[f] < ce;
+      sorted[rank] = ce;
+    }
+    __syncthreads();
+    const int last = sorted[kb - 1];
+    const int n_sel = (kb - 1) * blk + min(blk, n_c - last * blk);
+    const int n_win = pos - n_c + 1;
+    for (int e = threadIdx.x; e < width; e += blockDim.x) {
+      int v = -1;
+      if (e < n_sel) v = sorted[e / blk] * blk + e % blk;
+      else if (e < n_sel + n_win) v = n_c + (e - n_sel);
+      out[e] = v;
+    }
+  } else {
+    // No more blocks than the budget: every position of [0, pos] is kept.
+    for (int e = threadIdx.x; e < width; e += blockDim.x) out[e] = e <= pos ? e : -1;
+  }
+  // The index set is complete and visible: the next kernel may start.
+  __threadfence();
+  __syncthreads();
+  griddep_launch_dependents();
+  // Leave this query's histogram and counters at zero for the next selection.
+  uint32_t* gh = p.hist + (size_t)bq * kHistBins;
+  for (int e = threadIdx.x; e < kHistBins; e += blockDim.x) gh[e] = 0u;
+  if (threadIdx.x < 8) p.counters[(size_t)bq * 8 + threadIdx.x] = 0u;
+}
+
+// ----------------------------------------------------------------------------
 template <int H, bool FP8>
 static cudaError_t launch_rest_t(const SelectParams& p, int batch, cudaStream_t st);
 
@@ -887,6 +1119,18 @@ static cudaError_t launch_select_t(const SelectParams& p, int batch, cudaStream_
 template <int H, bool FP8>
 static cudaError_t launch_rest_t(const SelectParams& p, int batch, cudaStream_t st) {
   const int bq = batch * p.n_q;
+  if (p.block > 1) {
+    const int max_blocks = (p.kv.max_len + p.block - 1) / p.block;
+    const size_t dyn = blocks_dyn_smem(H, max_blocks);
+    static size_t attr_bytes = 0;
+    if (dyn > attr_bytes) {
+      cudaError_t e = cudaFuncSetAttribute(select_blocks_kernel<H, FP8>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+      if (e != cudaSuccess) return e;
+      attr_bytes = dyn;
+    }
+    return launch_pdl(select_blocks_kernel<H, FP8>, dim3(bq), dim3(kBlkThreads), dyn, st, p);
+  }
   cudaError_t e = launch_pdl(select_compact_kernel, dim3(p.splits3, bq), dim3(kThreads), 0, st, p);
   if (e != cudaSuccess) return e;
   const size_t dyn = finish_dyn_smem(H);
@@ -913,6 +1157,11 @@ static cudaError_t launch_rest_h(const SelectParams& p, int batch, cudaStream_t 
     case 128: return launch_rest_t<128, FP8>(p, batch, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+// Dynamic shared memory of the block-selection kernel for these sizes.
+size_t select_blocks_smem(int h, int max_len, int block) {
+  return blocks_dyn_smem(h, (max_len + block - 1) / block);
 }
 
 cudaError_t launch_select_rest(const SelectParams& p, int batch, cudaStream_t st) {

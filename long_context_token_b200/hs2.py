@@ -29,7 +29,8 @@ STATUS = {
 
 EXPORTS = ("hs2_workspace_bytes", "hs2_full_attn_select", "hs2_full_attn", "hs2_select",
            "hs2_sparse_attn", "hs2_check_device_status", "hs2_status_string",
-           "hs2_last_cuda_error", "hs2_abi_version", "hs2_sparse_attn_noalloc", "hs2_kv_append")
+           "hs2_last_cuda_error", "hs2_abi_version", "hs2_sparse_attn_noalloc", "hs2_kv_append",
+           "hs2_full_attn_select_blocks", "hs2_select_blocks")
 
 
 class Hs2Error(RuntimeError):
@@ -79,6 +80,11 @@ def lib():
     L.hs2_sparse_attn.restype = i32
     L.hs2_sparse_attn_noalloc.argtypes = [vp, i32, i32, kvp, vp, i32, f32, vp, vp, vp]
     L.hs2_sparse_attn_noalloc.restype = i32
+    L.hs2_full_attn_select_blocks.argtypes = [vp, i32, i32, kvp, i32, i32, i32, f32, vp, vp, vp,
+                                              vp, sz, vp]
+    L.hs2_full_attn_select_blocks.restype = i32
+    L.hs2_select_blocks.argtypes = [vp, i32, i32, kvp, i32, i32, i32, f32, vp, vp, sz, vp]
+    L.hs2_select_blocks.restype = i32
     L.hs2_kv_append.argtypes = [vp, vp, i32, kvp, vp, vp, sz, vp]
     L.hs2_kv_append.restype = i32
     L.hs2_check_device_status.argtypes = [vp, vp]
@@ -199,6 +205,47 @@ def full_attn_select(q: torch.Tensor, cache: Cache, window: int = 128, k_sel: in
                                       workspace.data_ptr(), workspace.numel(), _stream(stream))
     _check(code, "hs2_full_attn_select")
     return out, idx, lse
+
+
+def full_attn_select_blocks(q: torch.Tensor, cache: Cache, window: int = 128, k_sel: int = 1024,
+                            block: int = 64, sm_scale: Optional[float] = None,
+                            workspace: Optional[torch.Tensor] = None,
+                            out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                            lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+                            stream=None):
+    """Full-attention layer + block-level selection (whole blocks of ``block``
+    positions, the first-generation comparator).  Returns (out, idx, lse)."""
+    n_q, h = _check_q(q, cache)
+    B = cache.batch
+    sm_scale = default_scale() if sm_scale is None else sm_scale
+    if workspace is None:
+        workspace = alloc_workspace(cache, n_q, h, window, k_sel)
+    if out is None:
+        out = torch.empty(B, n_q, h, 128, dtype=torch.float32, device=q.device)
+    if idx is None:
+        idx = torch.empty(B, n_q, window + k_sel, dtype=torch.int32, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty(B, n_q, h, dtype=torch.float32, device=q.device)
+    code = lib().hs2_full_attn_select_blocks(q.data_ptr(), n_q, h, cache.ref(), window, k_sel,
+                                             block, sm_scale, out.data_ptr(), idx.data_ptr(),
+                                             _ptr(lse), workspace.data_ptr(), workspace.numel(),
+                                             _stream(stream))
+    _check(code, "hs2_full_attn_select_blocks")
+    return out, idx, lse
+
+
+def select_blocks(q, cache: Cache, workspace: torch.Tensor, window=128, k_sel=1024, block=64,
+                  sm_scale=None, idx=None, stream=None):
+    """Block-level selection alone; must follow full_attn on the same workspace."""
+    n_q, h = _check_q(q, cache)
+    sm_scale = default_scale() if sm_scale is None else sm_scale
+    if idx is None:
+        idx = torch.empty(cache.batch, n_q, window + k_sel, dtype=torch.int32, device=q.device)
+    code = lib().hs2_select_blocks(q.data_ptr(), n_q, h, cache.ref(), window, k_sel, block,
+                                   sm_scale, idx.data_ptr(), workspace.data_ptr(),
+                                   workspace.numel(), _stream(stream))
+    _check(code, "hs2_select_blocks")
+    return idx
 
 
 def full_attn(q, cache: Cache, window=128, k_sel=1024, sm_scale=None, workspace=None,

@@ -301,9 +301,10 @@ def kv_append(bits: dict, k_new_bits, v_new_bits) -> dict:
     return out
 
 
-def hybrid_block_step(bits: dict):
-    """One decode step of the hybrid block: full layer + selection, then every
-    reusing sparse layer in order.  Returns (full-layer dict, [sparse outputs])."""
-    full = full_attn_select(bits)
+def hybrid_block_step(bits: dict, block: int = 1):
+    """One decode step of the hybrid block: full layer + selection (token level, or
+    whole blocks of ``block`` positions), then every reusing sparse layer in order.
+    Returns (full-layer dict, [sparse outputs])."""
+    full = full_attn_select(bits, block=block)
     sparse = [sparse_attn(bits, ql, full["idx"]) for ql in bits["q_layers"]]
     return full, sparse

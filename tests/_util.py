@@ -76,3 +76,48 @@ def check_index_set(gpu_idx, ora_idx, imp, p: int, window: int, k_sel: int,
     if np.any(np.isin(below, chosen)):
         return "a key clearly below the k-th importance is present"
     return None
+
+
+def check_block_index_set(gpu_idx, ora_idx, imp, p: int, window: int, k_sel: int, block: int,
+                          rel_band: float = 1e-6):
+    """Compare one block-level index set with the oracle's under the tie band on
+    block scores (a block's score: the largest of the oracle's float64 importances
+    among its positions).  If the kb-th and (kb+1)-th block scores differ by at least
+    ``rel_band`` relative (kb = k_sel // block) the sets must be equal; otherwise
+    the GPU set must hold kb whole blocks, every block clearly above the kb-th score
+    and none clearly below.  Returns None on success, else a message."""
+    g = np.asarray(gpu_idx, dtype=np.int64)
+    o = np.asarray(ora_idx, dtype=np.int64)
+    gv = g[g >= 0]
+    if np.any(np.diff(gv) <= 0):
+        return "indices not strictly ascending"
+    if not np.all(g[gv.size:] == -1):
+        return "padding not at the end"
+    if np.array_equal(g, o):
+        return None
+    w_lo = max(0, p - window + 1)
+    if not np.all(np.isin(np.arange(w_lo, p + 1), gv)):
+        return "forced window missing"
+    n_blk = -(-w_lo // block)
+    kb = k_sel // block
+    if n_blk <= kb:
+        return "every position should be kept"
+    score = np.array([imp[c * block:(c + 1) * block].max() for c in range(n_blk)])
+    srt = np.sort(score)[::-1]
+    sk, sk1 = srt[kb - 1], srt[kb]
+    if sk - sk1 >= rel_band * sk:
+        return f"block sets differ outside the tie band at {np.setxor1d(g, o)[:8]}"
+    outside = gv[gv < w_lo]
+    kept = np.unique(outside // block)
+    if kept.size != kb:
+        return f"{kept.size} blocks kept, expected {kb}"
+    for c in kept:
+        if not np.array_equal(outside[outside // block == c],
+                              np.arange(c * block, min((c + 1) * block, w_lo))):
+            return f"block {c} not whole"
+    lo, hi = sk * (1 - rel_band), sk * (1 + rel_band)
+    if np.any(score[np.setdiff1d(np.arange(n_blk), kept)] > hi):
+        return "a block clearly above the boundary was dropped"
+    if np.any(score[kept] < lo):
+        return "a block clearly below the boundary was kept"
+    return None

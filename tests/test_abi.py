@@ -108,3 +108,22 @@ def test_sparse_attn_host_validation(L):
 def test_kv_append_rejects_bad_arguments(L, kv, kn, nn, lens, ws, wsb, expect):
     code = L.hs2_kv_append(kn, 1 << 20, nn, ctypes.byref(kv), lens, ws, wsb, None)
     assert code == expect
+
+
+@pytest.mark.parametrize("block,k_sel,idx,max_len,expect", [
+    (1, 1024, 1 << 20, 4096, 2),        # block < 2
+    (0, 1024, 1 << 20, 4096, 2),        # block < 2
+    (48, 1024, 1 << 20, 4096, 2),       # k_sel not a multiple of block
+    (2, 3968, 1 << 20, 4096, 2),        # more than 1024 blocks kept
+    (64, 1024, 1 << 20, 1 << 24, 2),    # 262144 block keys do not fit shared memory
+    (64, 1024, 0, 4096, 1),             # null idx
+])
+def test_block_selection_host_validation(L, block, k_sel, idx, max_len, expect):
+    base = 1 << 20
+    kv = hs2.KV(base, base + 4096, None, None, base, 1, max_len, 128, 0)
+    p = 1 << 20
+    huge = 1 << 60  # passes the workspace-size check; nothing is dereferenced on the host
+    assert L.hs2_full_attn_select_blocks(p, 1, 16, ctypes.byref(kv), 128, k_sel, block, 0.088,
+                                         p, idx, None, p, huge, None) == expect
+    assert L.hs2_select_blocks(p, 1, 16, ctypes.byref(kv), 128, k_sel, block, 0.088, idx, p,
+                               huge, None) == expect

@@ -12,7 +12,7 @@ import torch
 
 import oracle
 from long_context_token_b200 import hs2, workloads
-from _util import check_index_set
+from _util import check_block_index_set, check_index_set
 
 pytestmark = [pytest.mark.gpu, pytest.mark.filterwarnings("ignore::RuntimeWarning")]
 
@@ -306,3 +306,98 @@ def test_decode_loop_with_append_matches_oracle(case):
         if want[key] is not None:
             want[key] = np.concatenate([bits[key][:1], want[key]])
     _assert_cache_equal(cache, want)
+
+
+# Block-level selection (the first-generation comparator): the GPU's block sets
+# against the oracle's, and the sparse layers on the GPU's sets.
+BLOCK_CASES = [
+    dict(id="b1-L4096-h16-bf16", batch=1, max_len=4096, n_q=1, h_q=16, kv="bf16", seed=201,
+         n_needles=8, needle_layout="uniform"),
+    dict(id="ragged-b3-bf16", batch=3, max_len=5000, n_q=1, h_q=16, kv="bf16", seed=202,
+         lens=[5000, 1217, 1153]),
+    dict(id="h64-fp8-ragged", batch=2, max_len=3000, n_q=1, h_q=64, kv="fp8", seed=203,
+         lens=[3000, 2901]),
+    dict(id="h32-append4", batch=1, max_len=2500, n_q=4, h_q=32, kv="bf16", seed=204),
+    dict(id="append13-h16-ragged", batch=2, max_len=7000, n_q=13, h_q=16, kv="bf16", seed=205,
+         lens=[7000, 2222]),
+    dict(id="h48-fp8", batch=2, max_len=1800, n_q=2, h_q=48, kv="fp8", seed=206,
+         lens=[1800, 1500]),
+    dict(id="h128-bf16", batch=1, max_len=2000, n_q=1, h_q=128, kv="bf16", seed=207),
+    dict(id="tiny-window4-k8-block4", batch=2, max_len=48, n_q=3, h_q=16, kv="bf16", seed=208,
+         lens=[48, 13], window=4, k_sel=8, block=4),
+    dict(id="block16-fp8", batch=1, max_len=6000, n_q=1, h_q=16, kv="fp8", seed=209, block=16),
+    dict(id="short-contexts", batch=4, max_len=1300, n_q=1, h_q=16, kv="bf16", seed=210,
+         lens=[1, 1152, 1153, 1217]),
+]
+
+
+def run_gpu_blocks(inp: workloads.Inputs, block: int):
+    dev = torch.device("cuda:0")
+    cache = hs2.Cache(inp.k.to(dev), inp.v.to(dev), inp.lens.to(dev),
+                      None if inp.k_scale is None else inp.k_scale.to(dev),
+                      None if inp.v_scale is None else inp.v_scale.to(dev))
+    ws = hs2.alloc_workspace(cache, inp.n_q, inp.h_q, inp.window, inp.k_sel)
+    out, idx, lse = hs2.full_attn_select_blocks(inp.q.to(dev), cache, inp.window, inp.k_sel,
+                                                block, inp.sm_scale, ws)
+    sp = [hs2.sparse_attn(ql.to(dev), cache, idx, ws, inp.sm_scale) for ql in inp.q_layers]
+    status = hs2.check_device_status(ws)
+    return dict(out=out.cpu().numpy(), idx=idx.cpu().numpy(), lse=lse.cpu().numpy(),
+                sparse=[x.cpu().numpy() for x in sp]), status
+
+
+def compare_blocks(inp: workloads.Inputs, res: dict, block: int):
+    bits = workloads.numpy_bits(inp)
+    ref = oracle.full_attn_select(bits, keep_importance=True, block=block)
+    tol = TOL[inp.kv]
+    assert np.abs(res["out"] - ref["out"]).max() < tol
+    assert np.abs(res["lse"] - ref["lse"]).max() < LSE_TOL
+    n_exact = 0
+    for b in range(inp.batch):
+        L = int(inp.lens[b])
+        for i in range(inp.n_q):
+            p = L - inp.n_q + i
+            msg = check_block_index_set(res["idx"][b, i], ref["idx"][b, i],
+                                        ref["imp"][b * inp.n_q + i], p, inp.window, inp.k_sel,
+                                        block)
+            assert msg is None, f"(b={b}, i={i}, p={p}): {msg}"
+            n_exact += int(np.array_equal(res["idx"][b, i], ref["idx"][b, i]))
+    for li, ql in enumerate(bits["q_layers"]):
+        want = oracle.sparse_attn(bits, ql, res["idx"])
+        assert np.abs(res["sparse"][li] - want).max() < tol, f"sparse layer {li}"
+    return n_exact
+
+
+@pytest.mark.parametrize("case", BLOCK_CASES, ids=lambda c: c["id"])
+def test_block_selection_matches_oracle(case):
+    kw = {k: v for k, v in case.items() if k not in ("id", "block")}
+    block = case.get("block", 64)
+    inp = workloads.make_inputs(n_sparse=2, **kw)
+    res, status = run_gpu_blocks(inp, block)
+    assert status == 0
+    compare_blocks(inp, res, block)
+
+
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+def test_block_selection_zero_query_keeps_lowest_blocks(kv):
+    inp = workloads.make_inputs(1, 3000, n_q=1, h_q=16, kv=kv, seed=211, q_zero=True)
+    res, status = run_gpu_blocks(inp, 64)
+    assert status == 0
+    want = np.concatenate([np.arange(1024), np.arange(3000 - 128, 3000)])
+    assert res["idx"][0, 0].tolist() == want.tolist()
+
+
+def test_block_then_token_selection_share_a_workspace():
+    """Block mode leaves the selection state clean: a token-level call on the same
+    workspace right after it still matches the oracle."""
+    dev = torch.device("cuda:0")
+    inp = workloads.make_inputs(2, 5000, n_q=1, h_q=16, kv="bf16", seed=212, n_sparse=1,
+                                lens=[5000, 3000])
+    cache = hs2.Cache(inp.k.to(dev), inp.v.to(dev), inp.lens.to(dev))
+    ws = hs2.alloc_workspace(cache, 1, 16)
+    q = inp.q.to(dev)
+    hs2.full_attn_select_blocks(q, cache, 128, 1024, 64, inp.sm_scale, ws)
+    out, idx, lse = hs2.full_attn_select(q, cache, 128, 1024, inp.sm_scale, ws)
+    sp = [hs2.sparse_attn(inp.q_layers[0].to(dev), cache, idx, ws, inp.sm_scale)]
+    assert hs2.check_device_status(ws) == 0
+    compare(inp, dict(out=out.cpu().numpy(), idx=idx.cpu().numpy(), lse=lse.cpu().numpy(),
+                      sparse=[x.cpu().numpy() for x in sp]))
