@@ -46,6 +46,12 @@ LAUNCHES_PER_SPARSE = 1         # gather attention with the split merge on chip 
 NCU_TRAFFIC = {
     2: {"bytes": 4 * (134_288_128 + 786_304), "kernel": "full_attn_tc_kernel<16, 0>",
         "capture": "2 x 131072 keys, scaled x4"},
+    # first sequence of the ragged batch, scaled by the launch's algorithmic bytes
+    3: {"bytes": round((56_967_424 + 623_104) * 245_681_880 / 56_903_232),
+        "kernel": "full_attn_fp8_kernel<16, 0>",
+        "capture": "first sequence (56.9 MB of codes and scales), scaled to the 4-sequence launch"},
+    4: {"bytes": 276_918_528 + 5_604_608, "kernel": "full_attn_fp8_kernel<64, 0>",
+        "capture": "the whole launch"},
 }
 
 

@@ -10,9 +10,10 @@
 //   Q = 2^-e (Q_hi + Q_lo / 16), one power of two for all heads putting the largest
 //     |q| into [128, 256): a bf16 element (8 significant bits) whose scaled magnitude
 //     is at least 2^-6 is exact in the two terms, smaller ones to 2^-13 absolute;
-//   P' = p * v_scale * 2^-ev = P_hi + P_lo / 16 + P_lo2 / 256 (about 12 significant
-//     bits), ev a power of two at or above every |v_scale| the CTA has seen, moved
-//     with a rescale of O (like the softmax reference) when a larger one arrives.
+//   P' = p * v_scale * 2^-ev rounded to f16 (11 significant bits, as an f16 P would
+//     carry) = P_hi + P_lo / 16 + P_lo2 / 256 exactly, ev a power of two at or above
+//     every |v_scale| the CTA has seen, moved with a rescale of O (like the softmax
+//     reference) when a larger one arrives.
 // So S^T [128 keys x 2H] = K . [Q_hi | Q_lo]^T and O^T [128 d x 3H] += V^T . [P_hi |
 // P_lo | P_lo2]^T; the softmax and the epilogue combine each head's columns.
 //
@@ -93,6 +94,20 @@ __device__ __forceinline__ uint32_t e4m3_pair(float y0, float y1, float& v0, flo
 }
 __device__ __forceinline__ uint32_t e4m3_codes(float y0, float y1) {
   return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
+}
+
+// Two f16 values y (11 significant bits) -> three pairs of E4M3 codes with
+// y = hi + lo / 16 + lo2 / 256 exactly (4 + 4 + 3 bits; every step's difference and
+// scaling is exact in f16 for |y| <= 448).  Element 0 in the low byte of each pair.
+__device__ __forceinline__ void e4m3_split3(__half2 y, uint32_t& hi, uint32_t& lo, uint32_t& lo2) {
+  const __half2 k16 = __float2half2_rn(16.f);
+  hi = (uint32_t)__nv_cvt_halfraw2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
+  const __half2 a = __half2(__nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)hi, __NV_E4M3));
+  const __half2 r = __hmul2(__hsub2(y, a), k16);
+  lo = (uint32_t)__nv_cvt_halfraw2_to_fp8x2(r, __NV_SATFINITE, __NV_E4M3);
+  const __half2 b = __half2(__nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)lo, __NV_E4M3));
+  lo2 = (uint32_t)__nv_cvt_halfraw2_to_fp8x2(__hmul2(__hsub2(r, b), k16), __NV_SATFINITE,
+                                             __NV_E4M3);
 }
 
 // Q [H][128] bf16 -> the B operand of S^T = K . [Q_hi | Q_lo]^T (K-major, unswizzled,
@@ -590,12 +605,8 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
             const float p1 = ex2_ftz(x[h0 + 1] - finite_ref(ref(h0 + 1)));
             l[h0] += p0;
             l[h0 + 1] += p1;
-            const float y0 = p0 * vsc, y1 = p1 * vsc;
-            float a0, a1, b0, b1;
-            const uint32_t ch = e4m3_pair(y0, y1, a0, a1);
-            const float r0 = (y0 - a0) * 16.f, r1 = (y1 - a1) * 16.f;
-            const uint32_t cl = e4m3_pair(r0, r1, b0, b1);
-            const uint32_t cl2 = e4m3_codes((r0 - b0) * 16.f, (r1 - b1) * 16.f);
+            uint32_t ch, cl, cl2;
+            e4m3_split3(__floats2half2_rn(p0 * vsc, p1 * vsc), ch, cl, cl2);
             w0[e] |= ch << (16 * u);
             w1[e] |= cl << (16 * u);
             w2[e] |= cl2 << (16 * u);
