@@ -51,7 +51,7 @@ import numpy as np
 
 __all__ = [
     "bf16_to_f64", "e4m3_to_f64", "widen_cache", "attend", "importance",
-    "select_top", "index_set", "block_index_set", "full_attn_select", "sparse_attn", "hybrid_block_step",
+    "select_top", "index_set", "block_index_set", "full_attn_select", "prefill_attn", "sparse_attn", "hybrid_block_step",
     "f32_to_e4m3", "quantize_row_e4m3", "kv_append",
 ]
 
@@ -200,6 +200,27 @@ def full_attn_select(bits: dict, keep_importance: bool = False, block: int = 1):
     if keep_importance:
         res["imp"] = imps
     return res
+
+
+def prefill_attn(bits: dict):
+    """The full-attention layer over a chunk of n_q new tokens (chunked prefill of the
+    Cross-Decoder's full layer): the same attention as full_attn_select -- token i at
+    p = L - n_q + i sees keys [0, p] ([TNfr] "Ce que fait HySparse2": the full layer
+    attends over the whole context) -- without the selection.  Returns dict(out
+    [B, n_q, h, d], lse [B, n_q, h])."""
+    q_all = bf16_to_f64(bits["q"])
+    B, n_q, h, d = q_all.shape
+    out = np.zeros((B, n_q, h, d))
+    lse = np.zeros((B, n_q, h))
+    for b in range(B):
+        L = int(bits["lens"][b])
+        keys = _rows(bits, b, L, "k")
+        vals = _rows(bits, b, L, "v")
+        for i in range(n_q):
+            p = L - n_q + i
+            out[b, i], lse[b, i], _, _ = attend(q_all[b, i], keys[:p + 1], vals[:p + 1],
+                                                bits["sm_scale"])
+    return dict(out=out, lse=lse)
 
 
 def sparse_attn(bits: dict, q_layer_bits, idx) -> np.ndarray:

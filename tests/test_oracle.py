@@ -74,6 +74,28 @@ def test_full_attention_matches_library_sdpa_with_causal_queries(kv):
             np.testing.assert_allclose(res["lse"][b, i], lse_ref, rtol=0, atol=1e-12)
 
 
+def test_prefill_matches_library_sdpa_with_one_causal_mask():
+    """The chunk's tokens all at once: one float64 SDPA call over every (token, head)
+    row with the causal mask [row, key] = key <= position of the row's token."""
+    n_q, h = 40, 16
+    inp = workloads.make_inputs(2, 200, n_q=n_q, h_q=h, seed=31, lens=[200, 97])
+    bits = workloads.numpy_bits(inp)
+    res = oracle.prefill_attn(bits)
+    q = oracle.bf16_to_f64(bits["q"])
+    for b in range(2):
+        L = int(bits["lens"][b])
+        k = oracle.bf16_to_f64(bits["k"][b, :L])
+        v = oracle.bf16_to_f64(bits["v"][b, :L])
+        pos = np.repeat(L - n_q + np.arange(n_q), h)           # row = token * h + head
+        mask = np.arange(L)[None, :] <= pos[:, None]
+        ref = _sdpa(q[b].reshape(n_q * h, 128), k, v, bits["sm_scale"], mask)
+        np.testing.assert_allclose(res["out"][b].reshape(n_q * h, 128), ref, rtol=0, atol=1e-12)
+        s = bits["sm_scale"] * q[b].reshape(n_q * h, 128) @ k.T
+        s[~mask] = -np.inf
+        lse_ref = torch.logsumexp(torch.from_numpy(s), dim=1).numpy()
+        np.testing.assert_allclose(res["lse"][b].reshape(-1), lse_ref, rtol=0, atol=1e-12)
+
+
 def test_softmax_rows_sum_to_one():
     rng = np.random.default_rng(0)
     q, k, v = rng.standard_normal((8, 128)), rng.standard_normal((500, 128)), rng.standard_normal((500, 128))
