@@ -239,6 +239,141 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def run_prefill(args, w):
+    """Chunked prefill of the full layer (no selection): args.prefill new tokens per
+    sequence of the workload's cache, timed like the decode step (CUDA graph replays,
+    L2 flushed before each, CUDA events on the launching stream).  One GPU."""
+    from long_context_token_b200 import hs2
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("--prefill runs on one GPU")
+    if w.kv != "bf16":
+        raise SystemExit("--prefill needs a bf16 workload")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    n = args.prefill
+    inp = workloads.make_inputs(w.batch, w.max_len, n_q=n, h_q=w.h_q, kv="bf16", seed=w.seed,
+                                n_sparse=0)
+    cache = hs2.Cache(inp.k.to(dev), inp.v.to(dev), inp.lens.to(dev))
+    q = inp.q.to(dev)
+    ws = hs2.prefill_workspace(cache, n, w.h_q)
+    out = torch.empty(w.batch, n, w.h_q, 128, dtype=torch.float32, device=dev)
+    lse = torch.empty(w.batch, n, w.h_q, dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    drain = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    drain_out = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2(k):
+        flush.fill_(float(k))
+        torch.sum(drain, dim=0, out=drain_out)
+
+    def step():
+        hs2.prefill_attn(q, cache, inp.sm_scale, ws, out=out, lse=lse)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        flush_l2(1)
+        graph.replay()
+    torch.cuda.synchronize()
+    if hs2.check_device_status(ws) != 0:
+        raise RuntimeError("device-side error during warm-up")
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    replay_ms = []
+    wall0 = time.perf_counter()
+    with ClockSampler(dev) as clk:
+        for k in range(args.steps):
+            flush_l2(k)
+            start.record(stream)
+            graph.replay()
+            end.record(stream)
+            end.synchronize()
+            replay_ms.append(start.elapsed_time(end))
+    wall = time.perf_counter() - wall0
+    status = hs2.check_device_status(ws)
+    total_ms = sum(replay_ms)
+    tokens = w.batch * n
+    # Q.K^T and P.V over every visible (row, key) pair: 2 * 2 * 128 flops each.
+    vis = sum(int(L) - n + i + 1 for L in inp.lens.tolist() for i in range(n))
+    flops = 4 * 128 * w.h_q * vis
+    peaks, peak_kind = measured_peaks()
+    avg_s = total_ms / args.steps / 1e3
+    line = {
+        "metric": "chunked-prefill full layer tokens/s", "value": tokens * args.steps / (total_ms / 1e3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_of(w) | {"workload": f"prefill chunk {n} x h{w.h_q} vs "
+                                              f"{w.batch} x {w.max_len} bf16", "n_q": n,
+                                  "selection": "none (full layer only)"},
+        "roofline": {"bound": "tensor", "kernel": "full_attn_mq + split merge",
+                     "achieved": flops / avg_s / 1e12, "peak": float(peaks["bf16_tflops"]),
+                     "unit": "TFLOP/s", "frac": flops / avg_s / 1e12 / float(peaks["bf16_tflops"]),
+                     "peak_kind": peak_kind + " bf16 burst", "alg_flops_per_launch": flops,
+                     "traffic": None},
+        "gpu_launches": args.steps * 2,
+        "clocks": clk.summary(),
+        "device_status": status,
+        "wall_s_timed_region": wall,
+    }
+    if not args.no_e2e:
+        hq = inp.q.clone().pin_memory()
+        hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        hlse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            hs2.prefill_attn(q, cache, inp.sm_scale, ws, out=out, lse=lse)
+            hout.copy_(out, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2):
+            e2e_step()
+        e_ms = 0.0
+        for k in range(args.steps):
+            flush_l2(k)
+            start.record(stream)
+            g2.replay()
+            end.record(stream)
+            end.synchronize()
+            e_ms += start.elapsed_time(end)
+        line["e2e"] = {"value": tokens * args.steps / (e_ms / 1e3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": hq.numel() * 2,
+                       "d2h_bytes_per_step": hout.numel() * 4 + hlse.numel() * 4,
+                       "path": "hs2 C ABI via the Python binding, step replayed from a CUDA graph"}
+        del g2
+    del graph
+    if not args.no_cpu_baseline:
+        import oracle
+        bits = workloads.numpy_bits(inp)
+        k = 8  # the chunk's first tokens of the first sequence
+        sub = dict(bits, q=bits["q"][:1, :k], k=bits["k"][:1], v=bits["v"][:1],
+                   lens=(bits["lens"][:1] - (n - k)).astype(bits["lens"].dtype))
+        t0 = time.perf_counter()
+        done = 0
+        while True:
+            oracle.prefill_attn(sub)
+            done += k
+            if time.perf_counter() - t0 >= args.cpu_budget:
+                break
+        secs = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": done / secs, "unit": "tokens/s", "cores": host_cores(),
+                                "kind": "oracle",
+                                "sample": f"{done} tokens ({k} per call: the chunk's first {k} "
+                                          f"tokens of sequence 0, same positions) in {secs:.1f} s, "
+                                          "float64 numpy oracle"}
+    print(json.dumps(line), flush=True)
+
+
 def config_of(w, block: int = 1):
     return {"workload": w.name, "batch": w.batch, "context": w.max_len,
             "selection": "token" if block == 1 else f"blocks of {block} positions",
@@ -262,6 +397,9 @@ def main():
     ap.add_argument("--block", type=int, default=1,
                     help="1: token-level selection (the method); N > 1: whole blocks of N "
                          "positions (the first-generation comparator)")
+    ap.add_argument("--prefill", type=int, default=0,
+                    help="N > 0: time the chunked-prefill full layer for N new tokens per "
+                         "sequence of the workload's bf16 cache instead of the decode step")
     ap.add_argument("--batch", type=int, default=None,
                     help="run fewer sequences of the workload (profiling captures only)")
     args = ap.parse_args()
@@ -272,6 +410,8 @@ def main():
         w = dataclasses.replace(w, batch=args.batch, name=f"{w.name} (first {args.batch} seqs)")
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.prefill > 0:
+        return run_prefill(args, w)
 
     from long_context_token_b200 import hs2
     world, rank, local = dist_env()

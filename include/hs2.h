@@ -160,6 +160,25 @@ HS2_API hs2_status hs2_select_blocks(const void* q, int n_q, int h_q, const hs2_
                                      int32_t* idx, void* workspace, size_t ws_bytes,
                                      hs2_stream_t stream);
 
+/* Chunked prefill of the Cross-Decoder's full layer: the full-attention layer for a
+ * chunk of n_q new tokens per sequence (already appended to the cache), the same
+ * attention as hs2_full_attn (token i at p = lens[b] - n_q + i sees keys [0, p]), with
+ * no selection ("Luo Fuli Teases Xiaomi MiMo-V3 Architecture ..." and toolnavs
+ * article 2080: the full layers attend over the whole context).  Tensor cores: 128
+ * query rows (128 / h_q tokens x h_q heads) share each K/V tile.
+ *   q        device bf16 [batch][n_q][h_q][128];  n_q in [1, 65536], n_q <= max_len.
+ *   h_q      16, 32, 48, 64 or 128.  kv: bf16 caches only (else HS2_ERR_UNSUPPORTED).
+ *   out      device float32 [batch][n_q][h_q][128]; lse float32 [batch][n_q][h_q] or NULL.
+ *   workspace  at least hs2_prefill_workspace_bytes(batch, n_q, h_q, max_len, dtype)
+ *            bytes (split partials; zero-filled once, as for the decode calls).
+ * A sequence with lens[b] < n_q reports HS2_ERR_BAD_LENGTH through the workspace's
+ * status word (hs2_check_device_status). */
+HS2_API size_t hs2_prefill_workspace_bytes(int batch, int n_q, int h_q, int max_len,
+                                           int dtype);
+HS2_API hs2_status hs2_prefill_attn(const void* q, int n_q, int h_q, const hs2_kv* kv,
+                                    float sm_scale, float* out, float* lse, void* workspace,
+                                    size_t ws_bytes, hs2_stream_t stream);
+
 /* One reusing sparse-attention layer (step 3).
  *   q_layer   device bf16 [batch][n_q][h_q][128], this layer's queries.
  *   idx       device int32 [batch][n_q][idx_width]: positions to attend to (any

@@ -344,6 +344,48 @@ static hs2_status run_select(const void* q, int n_q, int h, const hs2_kv* kv, in
 
 using namespace hs2;
 
+// ---------------------------------------------------------------- chunked prefill
+// The several-token tensor-core full layer over a chunk of up to 65536 new tokens, with
+// a workspace of split partials only: [status][part_o][part_ml].  Splits are planned
+// from a fixed target of CTAs (so the workspace size does not depend on the device).
+constexpr int kMaxPrefillTokens = 65536;
+constexpr int kPrefillCtaTarget = 296;  // about two CTAs per SM of a 148-SM part
+constexpr int kMaxPrefillSplits = 32;
+
+static hs2_status check_prefill(int batch, int n_q, int h, int max_len, int dtype) {
+  if (batch < 1 || max_len < 1) return HS2_ERR_INVALID_ARGUMENT;
+  if (dtype != HS2_KV_BF16) return HS2_ERR_UNSUPPORTED;
+  if (h != 16 && h != 32 && h != 48 && h != 64 && h != 128) return HS2_ERR_UNSUPPORTED;
+  if (n_q < 1 || n_q > kMaxPrefillTokens || n_q > max_len) return HS2_ERR_UNSUPPORTED;
+  if ((long long)batch * max_len >= (1ll << 31)) return HS2_ERR_UNSUPPORTED;
+  return HS2_OK;
+}
+
+static int prefill_splits(int batch, int n_q, int h, int max_len) {
+  const int G = mq_tokens_per_cta(h);
+  const long long groups = (long long)batch * ((n_q + G - 1) / G);
+  long long sp = (kPrefillCtaTarget + groups - 1) / groups;
+  const long long by_len = ((long long)max_len + 63) / 64;
+  if (sp > by_len) sp = by_len;
+  if (sp > kMaxPrefillSplits) sp = kMaxPrefillSplits;
+  return sp < 1 ? 1 : (int)sp;
+}
+
+struct PrefillLayout {
+  int splits;
+  size_t part_o, part_ml, total;
+};
+
+static PrefillLayout prefill_layout(int batch, int n_q, int h, int max_len) {
+  PrefillLayout L;
+  L.splits = prefill_splits(batch, n_q, h, max_len);
+  const size_t rows = (size_t)batch * n_q * L.splits * h;
+  L.part_o = 256;  // after the status word
+  L.part_ml = align_up(L.part_o + rows * kHeadDim * sizeof(float), 256);
+  L.total = align_up(L.part_ml + rows * 2 * sizeof(float), 256);
+  return L;
+}
+
 extern "C" {
 
 size_t hs2_workspace_bytes(int batch, int n_q, int h_q, int max_len, int window, int k_sel,
@@ -556,6 +598,59 @@ hs2_status hs2_kv_append(const void* k_new, const void* v_new, int n_new, const 
   p.status = static_cast<uint32_t*>(workspace);
   cudaError_t e = launch_kv_append(p, kv->batch, (cudaStream_t)stream);
   return e == cudaSuccess ? HS2_OK : cuda_fail(e, "kv-append launch");
+}
+
+size_t hs2_prefill_workspace_bytes(int batch, int n_q, int h_q, int max_len, int dtype) {
+  if (check_prefill(batch, n_q, h_q, max_len, dtype) != HS2_OK) return 0;
+  return prefill_layout(batch, n_q, h_q, max_len).total;
+}
+
+hs2_status hs2_prefill_attn(const void* q, int n_q, int h_q, const hs2_kv* kv, float sm_scale,
+                            float* out, float* lse, void* workspace, size_t ws_bytes,
+                            hs2_stream_t stream) {
+  hs2_status st = check_kv(kv);
+  if (st != HS2_OK) return st;
+  st = check_prefill(kv->batch, n_q, h_q, kv->max_len, kv->dtype);
+  if (st != HS2_OK) return st;
+  if (!q || !out || !workspace) return HS2_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return HS2_ERR_INVALID_ARGUMENT;
+  const PrefillLayout W = prefill_layout(kv->batch, n_q, h_q, kv->max_len);
+  if (ws_bytes < W.total) return HS2_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = (cudaStream_t)stream;
+  FullParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.kv = view_of(kv);
+  p.n_q = n_q;
+  p.h = h_q;
+  p.window = 1;
+  p.k_sel = 1;
+  p.sm_scale = sm_scale;
+  int chunk = (kv->max_len + W.splits - 1) / W.splits;
+  chunk = (chunk + 63) / 64 * 64;
+  p.splits1 = (kv->max_len + chunk - 1) / chunk;
+  p.chunk1 = chunk;
+  p.part_o = ws_ptr<float>(workspace, W.part_o);
+  p.part_ml = ws_ptr<float>(workspace, W.part_ml);
+  p.status = ws_ptr<uint32_t>(workspace, 0);
+  CUtensorMap tk, tv;
+  const uint64_t rows = (uint64_t)kv->batch * kv->max_len;
+  if (!make_tmap_2d(&tk, kv->k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kHeadDim, rows, kHeadDim * 2,
+                    64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tv, kv->v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kHeadDim, rows, kHeadDim * 2,
+                    64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cuda_fail(cudaErrorInvalidValue, "tensor maps of K/V");
+  cudaError_t e = launch_full_attn_mq(p, tk, tv, kv->batch, s);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  MergeParams m;
+  m.part_o = p.part_o;
+  m.part_ml = p.part_ml;
+  m.splits = p.splits1;
+  m.h = h_q;
+  m.out = out;
+  m.lse_out = lse;
+  m.lse64 = nullptr;
+  e = launch_merge(m, kv->batch * n_q, true, s);
+  return e == cudaSuccess ? HS2_OK : cuda_fail(e, "prefill merge launch");
 }
 
 }  // extern "C"

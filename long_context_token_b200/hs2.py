@@ -30,7 +30,8 @@ STATUS = {
 EXPORTS = ("hs2_workspace_bytes", "hs2_full_attn_select", "hs2_full_attn", "hs2_select",
            "hs2_sparse_attn", "hs2_check_device_status", "hs2_status_string",
            "hs2_last_cuda_error", "hs2_abi_version", "hs2_sparse_attn_noalloc", "hs2_kv_append",
-           "hs2_full_attn_select_blocks", "hs2_select_blocks")
+           "hs2_full_attn_select_blocks", "hs2_select_blocks", "hs2_prefill_workspace_bytes",
+           "hs2_prefill_attn")
 
 
 class Hs2Error(RuntimeError):
@@ -85,6 +86,10 @@ def lib():
     L.hs2_full_attn_select_blocks.restype = i32
     L.hs2_select_blocks.argtypes = [vp, i32, i32, kvp, i32, i32, i32, f32, vp, vp, sz, vp]
     L.hs2_select_blocks.restype = i32
+    L.hs2_prefill_workspace_bytes.argtypes = [i32] * 5
+    L.hs2_prefill_workspace_bytes.restype = sz
+    L.hs2_prefill_attn.argtypes = [vp, i32, i32, kvp, f32, vp, vp, vp, sz, vp]
+    L.hs2_prefill_attn.restype = i32
     L.hs2_kv_append.argtypes = [vp, vp, i32, kvp, vp, vp, sz, vp]
     L.hs2_kv_append.restype = i32
     L.hs2_check_device_status.argtypes = [vp, vp]
@@ -246,6 +251,34 @@ def select_blocks(q, cache: Cache, workspace: torch.Tensor, window=128, k_sel=10
                                    workspace.numel(), _stream(stream))
     _check(code, "hs2_select_blocks")
     return idx
+
+
+def prefill_workspace(cache: Cache, n_q: int, h_q: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace (uint8 tensor) for prefill_attn at these sizes."""
+    n = lib().hs2_prefill_workspace_bytes(cache.batch, n_q, h_q, cache.max_len, cache.dtype)
+    if n == 0:
+        raise Hs2Error(2, "hs2_prefill_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device or cache.k.device)
+
+
+def prefill_attn(q: torch.Tensor, cache: Cache, sm_scale: Optional[float] = None,
+                 workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None, want_lse: bool = True, stream=None):
+    """Full-attention layer over a chunk of n_q new tokens per sequence (chunked
+    prefill; no selection).  Returns (out, lse)."""
+    n_q, h = _check_q(q, cache)
+    sm_scale = default_scale() if sm_scale is None else sm_scale
+    if workspace is None:
+        workspace = prefill_workspace(cache, n_q, h)
+    if out is None:
+        out = torch.empty(cache.batch, n_q, h, 128, dtype=torch.float32, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty(cache.batch, n_q, h, dtype=torch.float32, device=q.device)
+    code = lib().hs2_prefill_attn(q.data_ptr(), n_q, h, cache.ref(), sm_scale, out.data_ptr(),
+                                  _ptr(lse), workspace.data_ptr(), workspace.numel(),
+                                  _stream(stream))
+    _check(code, "hs2_prefill_attn")
+    return out, lse
 
 
 def full_attn(q, cache: Cache, window=128, k_sel=1024, sm_scale=None, workspace=None,

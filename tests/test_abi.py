@@ -127,3 +127,36 @@ def test_block_selection_host_validation(L, block, k_sel, idx, max_len, expect):
                                          p, idx, None, p, huge, None) == expect
     assert L.hs2_select_blocks(p, 1, 16, ctypes.byref(kv), 128, k_sel, block, 0.088, idx, p,
                                huge, None) == expect
+
+
+@pytest.mark.parametrize("args", [
+    (1, 512, 16, 4096, 1),        # FP8 cache
+    (1, 512, 24, 4096, 0),        # h_q not supported
+    (1, 0, 16, 4096, 0),          # empty chunk
+    (1, 5000, 16, 4096, 0),       # chunk longer than the cache
+    (1, 65537, 16, 1 << 20, 0),   # chunk above 65536 tokens
+    (0, 512, 16, 4096, 0),        # empty batch
+])
+def test_prefill_workspace_rejects_unsupported(L, args):
+    assert L.hs2_prefill_workspace_bytes(*args) == 0
+
+
+def test_prefill_workspace_holds_the_partials(L):
+    # 4096 tokens x h16 in groups of 8: 512 CTAs, one split; partials 4096 * 16 * 130 floats
+    n = L.hs2_prefill_workspace_bytes(1, 4096, 16, 131072, 0)
+    assert 4096 * 16 * 130 * 4 <= n < 4096 * 16 * 130 * 4 + 4096
+    # a short chunk (one CTA of rows) is split along the keys to fill the GPU, up to 32
+    # splits: 32 partials per row
+    assert L.hs2_prefill_workspace_bytes(1, 8, 16, 131072, 0) >= 8 * 16 * 130 * 4 * 32
+
+
+def test_prefill_host_validation(L):
+    base = 1 << 20
+    kv = hs2.KV(base, base + 4096, None, None, base, 1, 4096, 128, 0)
+    kv8 = hs2.KV(base, base + 4096, base, base, base, 1, 4096, 128, 1)
+    p = 1 << 20
+    assert L.hs2_prefill_attn(None, 64, 16, ctypes.byref(kv), 0.088, p, None, p, 1 << 30, None) == 1
+    assert L.hs2_prefill_attn(p, 64, 16, ctypes.byref(kv8), 0.088, p, None, p, 1 << 30, None) == 2
+    assert L.hs2_prefill_attn(p, 64, 24, ctypes.byref(kv), 0.088, p, None, p, 1 << 30, None) == 2
+    assert L.hs2_prefill_attn(p | 8, 64, 16, ctypes.byref(kv), 0.088, p, None, p, 1 << 30, None) == 1
+    assert L.hs2_prefill_attn(p, 64, 16, ctypes.byref(kv), 0.088, p, None, p, 64, None) == 3

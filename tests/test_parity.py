@@ -401,3 +401,40 @@ def test_block_then_token_selection_share_a_workspace():
     assert hs2.check_device_status(ws) == 0
     compare(inp, dict(out=out.cpu().numpy(), idx=idx.cpu().numpy(), lse=lse.cpu().numpy(),
                       sparse=[x.cpu().numpy() for x in sp]))
+
+
+# Chunked prefill of the full layer (no selection): many new tokens per sequence.
+PREFILL_CASES = [
+    dict(id="L4096-chunk512-h16", batch=1, max_len=4096, n_q=512, h_q=16, seed=301),
+    dict(id="ragged-chunk300-h32", batch=2, max_len=3000, n_q=300, h_q=32, seed=302,
+         lens=[3000, 1500]),
+    dict(id="whole-context-1024-h64", batch=1, max_len=1024, n_q=1024, h_q=64, seed=303),
+    dict(id="chunk37-h128", batch=1, max_len=1500, n_q=37, h_q=128, seed=304),
+    dict(id="chunk129-h16-ragged", batch=2, max_len=2000, n_q=129, h_q=16, seed=305,
+         lens=[2000, 129]),
+    dict(id="single-token-h48", batch=3, max_len=700, n_q=1, h_q=48, seed=306,
+         lens=[700, 1, 333]),
+]
+
+
+@pytest.mark.parametrize("case", PREFILL_CASES, ids=lambda c: c["id"])
+def test_prefill_matches_oracle(case):
+    kw = {k: v for k, v in case.items() if k != "id"}
+    inp = workloads.make_inputs(kv="bf16", n_sparse=0, **kw)
+    dev = torch.device("cuda:0")
+    cache = hs2.Cache(inp.k.to(dev), inp.v.to(dev), inp.lens.to(dev))
+    ws = hs2.prefill_workspace(cache, inp.n_q, inp.h_q)
+    out, lse = hs2.prefill_attn(inp.q.to(dev), cache, inp.sm_scale, ws)
+    assert hs2.check_device_status(ws) == 0
+    ref = oracle.prefill_attn(workloads.numpy_bits(inp))
+    assert np.abs(out.cpu().numpy() - ref["out"]).max() < TOL["bf16"]
+    assert np.abs(lse.cpu().numpy() - ref["lse"]).max() < LSE_TOL
+
+
+def test_prefill_reports_a_sequence_shorter_than_the_chunk():
+    inp = workloads.make_inputs(2, 200, n_q=64, h_q=16, seed=307, n_sparse=0, lens=[200, 50])
+    dev = torch.device("cuda:0")
+    cache = hs2.Cache(inp.k.to(dev), inp.v.to(dev), inp.lens.to(dev))
+    ws = hs2.prefill_workspace(cache, 64, 16)
+    hs2.prefill_attn(inp.q.to(dev), cache, inp.sm_scale, ws)
+    assert hs2.STATUS[hs2.check_device_status(ws)] == "HS2_ERR_BAD_LENGTH"
