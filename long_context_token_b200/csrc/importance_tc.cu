@@ -478,59 +478,32 @@ cudaError_t launch_importance_mq(const SelectParams& p, const CUtensorMap& tmap_
 }
 
 // ============================================================================
-// The same pass for an FP8 E4M3 cache: raw 128-key tiles by TMA, four conversion
-// warps widen them exactly to f16 (see the FP8 full layer), Q goes to f16 under a
-// per-head power-of-two scale, and each key's logits are multiplied by its k_scale.
+// The same pass for an FP8 E4M3 cache: raw 128-key tiles by TMA go straight into
+// kind::f8f6f4 MMAs (K-major, 128-byte swizzle) against Q as two E4M3 terms
+// (Q_hi + Q_lo / 16 after one power-of-two scale, exact for bf16 queries; the FP8
+// full layer does the same), and each key's logits are multiplied by its k_scale.
 // ============================================================================
 namespace {
 
-constexpr int kImpF8Threads = 320;
-constexpr uint32_t kImpRawTile = 16384;
-constexpr uint32_t kImpConvTile = 32768;
-
-__device__ __forceinline__ uint32_t imp_e4m3x2_to_f16x2(uint32_t two_codes) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two_codes, __NV_E4M3);
-  return (uint32_t)h.x | ((uint32_t)h.y << 16);
-}
-
-__device__ __forceinline__ void imp_convert_row(const uint8_t* raw, uint8_t* conv, int r,
-                                                bool valid) {
-  const uint8_t* src = raw + r * 128;
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const uint4 in = *reinterpret_cast<const uint4*>(src + (((c ^ r) & 7) << 4));
-    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
-    uint32_t o[8];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      o[2 * u] = valid ? imp_e4m3x2_to_f16x2(w[u] & 0xffffu) : 0u;
-      o[2 * u + 1] = valid ? imp_e4m3x2_to_f16x2(w[u] >> 16) : 0u;
-    }
-    uint8_t* dst = conv + (c >> 2) * kBoxBytes + r * 128;
-    const int c0 = 2 * (c & 3);
-    *reinterpret_cast<uint4*>(dst + (((c0 ^ r) & 7) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-    *reinterpret_cast<uint4*>(dst + ((((c0 + 1) ^ r) & 7) << 4)) =
-        make_uint4(o[4], o[5], o[6], o[7]);
-  }
-}
+constexpr int kImpF8Threads = 192;  // TMA, MMA, four epilogue warps (thread = key)
 
 template <int H>
 struct ImpF8Smem {
-  static constexpr int R = 4;  // raw stages
-  static constexpr int C = 2;  // converted buffers
-  static constexpr uint32_t kQBytes = H * kHeadDim * 2;
+  static constexpr int R = 8;  // raw K stages
+  static constexpr uint32_t kQBytes = 2 * H * kHeadDim;  // Q_hi, Q_lo rows
   static constexpr uint32_t kRawOff = 0;
-  static constexpr uint32_t kConvOff = R * kImpRawTile;
-  static constexpr uint32_t kQOff = kConvOff + C * kImpConvTile;
+  static constexpr uint32_t kQOff = R * kE4m3TileBytes;
   static constexpr uint32_t kHistOff = kQOff + kQBytes;
   static constexpr uint32_t kDeltaOff = kHistOff + kHistBins * 4;
   static constexpr uint32_t kQinvOff = kDeltaOff + H * 4;
-  static constexpr uint32_t kBarOff = kQinvOff + H * 4;
-  static constexpr uint32_t kBars = 2 * R + 2 * C + 4 + 1;
+  static constexpr uint32_t kBarOff = kQinvOff + 16;
+  static constexpr uint32_t kBars = 2 * R + 4 + 1;
   static constexpr uint32_t kSlotOff = kBarOff + kBars * 8;
   static constexpr uint32_t kBytes = kSlotOff + 16 + 1024;
-  static constexpr uint32_t kTmemCols = tmem_cols_pow2(2 * H);
-  static_assert(kBytes <= 227 * 1024, "shared memory budget");
+  static constexpr uint32_t kTmemCols = tmem_cols_pow2(4 * H);  // two S buffers of 2H
+  // (+ 2048 for the static shared memory of the Q staging and the histogram flush)
+  static_assert(kBytes + 2048 <= 227 * 1024, "shared memory budget");
+  static_assert(kQOff % 1024 == 0 && kBarOff % 8 == 0, "alignment");
 };
 
 }  // namespace
@@ -539,11 +512,10 @@ template <int H>
 __global__ void __launch_bounds__(kImpF8Threads, 1)
     importance_fp8_kernel(const __grid_constant__ CUtensorMap tmap_k, SelectParams p) {
   using L = ImpF8Smem<H>;
-  constexpr int R = L::R, C = L::C;
+  constexpr int R = L::R;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* raw = smem + L::kRawOff;
-  uint8_t* conv = smem + L::kConvOff;
   uint8_t* qs = smem + L::kQOff;
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + L::kHistOff);
   float* delta_s = reinterpret_cast<float*>(smem + L::kDeltaOff);
@@ -551,10 +523,8 @@ __global__ void __launch_bounds__(kImpF8Threads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* r_full = bars;
   uint64_t* r_empty = bars + R;
-  uint64_t* c_full = bars + 2 * R;
-  uint64_t* c_empty = bars + 2 * R + C;
-  uint64_t* s_full = bars + 2 * R + 2 * C;  // [2]
-  uint64_t* s_free = s_full + 2;            // [2]
+  uint64_t* s_full = bars + 2 * R;  // [2]
+  uint64_t* s_free = s_full + 2;    // [2]
   uint64_t* mma_done = s_full + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
 
@@ -575,11 +545,7 @@ __global__ void __launch_bounds__(kImpF8Threads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < R; ++s) {
       mbar_init(r_full + s, 1);
-      mbar_init(r_empty + s, 128);
-    }
-    for (int s = 0; s < C; ++s) {
-      mbar_init(c_full + s, 128);
-      mbar_init(c_empty + s, 1);
+      mbar_init(r_empty + s, 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(s_full + s, 1);
@@ -595,7 +561,7 @@ __global__ void __launch_bounds__(kImpF8Threads, 1)
   if (warp == 0 && lane_id() == 0) prefetch_tmap(&tmap_k);
   for (int e = threadIdx.x; e < kHistBins; e += blockDim.x) hist_s[e] = 0u;
   load_delta(p.lse64 + (size_t)bq * H, H, delta_s, nullptr);
-  store_q_f16_scaled<H>(qs, p.q + (size_t)bq * H * kHeadDim, qinv_s, nullptr);
+  store_q_e4m3_split<H>(qs, p.q + (size_t)bq * H * kHeadDim, qinv_s);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -611,8 +577,8 @@ __global__ void __launch_bounds__(kImpF8Threads, 1)
       for (int i = 0; i < n_tiles && ok; ++i) {
         const int s = i % R;
         if (!mbar_wait(r_empty + s, ((i / R) & 1) ^ 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(r_full + s, kImpRawTile);
-        tma_load_2d(raw + s * kImpRawTile, &tmap_k, r_full + s, 0, row0 + i * kKeyTile, pol);
+        mbar_arrive_expect_tx(r_full + s, kE4m3TileBytes);
+        tma_load_2d(raw + s * kE4m3TileBytes, &tmap_k, r_full + s, 0, row0 + i * kKeyTile, pol);
         issued = i + 1;
       }
       for (int i = issued > R ? issued - R : 0; i < issued; ++i)
@@ -620,43 +586,30 @@ __global__ void __launch_bounds__(kImpF8Threads, 1)
     }
   } else if (warp == 1) {
     if (elect_one()) {
-      const uint32_t idesc = idesc_f16(128, H, false, false, false);
+      constexpr uint32_t idesc = idesc_e4m3(128, 2 * H, false, false);
       const uint32_t q_addr = smem_u32(qs);
       for (int i = 0; i < n_tiles && ok; ++i) {
-        const int cb = i % C, sb = i & 1;
-        if (!mbar_wait(c_full + cb, (i / C) & 1)) { ok = false; break; }
+        const int s = i % R, sb = i & 1;
+        if (!mbar_wait(r_full + s, (i / R) & 1)) { ok = false; break; }
         if (!mbar_wait(s_free + sb, ((i >> 1) & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(conv + cb * kImpConvTile);
+        const uint32_t a_addr = smem_u32(raw + s * kE4m3TileBytes);
 #pragma unroll
-        for (int kk = 0; kk < kHeadDim / 16; ++kk)
-          mma_f16_ss(tmem_base + sb * H, kmajor_sw128_desc(a_addr, kk),
-                     q_kmajor_desc<H>(q_addr, kk), idesc, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < kHeadDim / 32; ++kk)
+          mma_e4m3_ss(tmem_base + sb * 2 * H, k_e4m3_desc(a_addr, kk),
+                      q_e4m3_desc<2 * H>(q_addr, kk), idesc, kk > 0 ? 1u : 0u);
         mma_commit(s_full + sb);
-        mma_commit(c_empty + cb);
+        mma_commit(r_empty + s);
       }
       mma_commit(mma_done);
       if (!mbar_wait(mma_done, 0)) ok = false;
-    }
-  } else if (warp >= 6) {
-    // conversion: thread t converts row t of each raw tile
-    const int t = threadIdx.x - 192;
-    for (int i = 0; i < n_tiles; ++i) {
-      const int s = i % R, cb = i % C;
-      if (ok && !mbar_wait(r_full + s, (i / R) & 1)) ok = false;
-      if (ok && !mbar_wait(c_empty + cb, ((i / C) & 1) ^ 1)) ok = false;
-      imp_convert_row(raw + s * kImpRawTile, conv + cb * kImpConvTile, t,
-                      k0 + i * kKeyTile + t < k1);
-      fence_proxy_async_smem();
-      mbar_arrive(c_full + cb);
-      mbar_arrive(r_empty + s);
     }
   } else {
     // epilogue: thread t owns key t of the tile
     const int lg = warp & 3;
     const int t = lg * 32 + (int)lane_id();
     float* trow = p.tbuf + (size_t)bq * p.kv.max_len;
-    const float sc = p.sm_scale;
+    const float qsc = qinv_s[0] * p.sm_scale;  // Q-scaled logit -> s (before k_scale)
     auto scale_of = [&](int i) {
       const int j = k0 + i * kKeyTile + t;
       return (i < n_tiles && j < k1) ? __ldg(p.kv.k_scale + row_base + j) : 0.f;
@@ -664,24 +617,29 @@ __global__ void __launch_bounds__(kImpF8Threads, 1)
     float ks_next = scale_of(0), ks_far = scale_of(1);
     for (int i = 0; i < n_tiles; ++i) {
       const int buf = i & 1;
-      const float ks = ks_next;
+      const float m = qsc * ks_next;
       ks_next = ks_far;
       ks_far = scale_of(i + 2);
       if (ok && !mbar_wait(s_full + buf, (i >> 1) & 1)) ok = false;
       tc_fence_after();
       float best = -INFINITY;
-      const uint32_t taddr = tmem_base + ((uint32_t)(lg * 32) << 16) + buf * H;
+      const uint32_t taddr = tmem_base + ((uint32_t)(lg * 32) << 16) + buf * 2 * H;
 #pragma unroll
-      for (int c0 = 0; c0 < H; c0 += 64) {  // up to four loads in flight per wait
+      for (int c0 = 0; c0 < H; c0 += 32) {  // hi and lo of 32 heads: four loads per wait
         uint32_t r[64];
 #pragma unroll
-        for (int c = 0; c < 64; c += 16)
-          if (c0 + c < H) tmem_ld16(taddr + c0 + c, *reinterpret_cast<uint32_t(*)[16]>(r + c));
+        for (int c = 0; c < 32; c += 16)
+          if (c0 + c < H) {
+            tmem_ld16(taddr + c0 + c, *reinterpret_cast<uint32_t(*)[16]>(r + c));
+            tmem_ld16(taddr + H + c0 + c, *reinterpret_cast<uint32_t(*)[16]>(r + 32 + c));
+          }
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 64; ++e)
-          if (c0 + e < H)
-            best = fmaxf(best, __uint_as_float(r[e]) * (qinv_s[c0 + e] * ks * sc) - delta_s[c0 + e]);
+        for (int e = 0; e < 32; ++e)
+          if (c0 + e < H) {
+            const float x = fmaf(__uint_as_float(r[32 + e]), 0.0625f, __uint_as_float(r[e]));
+            best = fmaxf(best, x * m - delta_s[c0 + e]);
+          }
       }
       tc_fence_before();
       mbar_arrive(s_free + buf);

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "hs2_internal.cuh"
 #include "sm100.cuh"
@@ -223,6 +224,112 @@ __device__ __forceinline__ void cluster_merge_row(const uint8_t* smem, int ns, f
 __device__ __forceinline__ uint64_t pt_mnmajor_desc(uint32_t p_addr, int kk) {
   return sm100::smem_desc(p_addr + (uint32_t)kk * 256u, 128, kKeyTile * 16, sm100::kSwizzleNone);
 }
+#endif
+
+#ifdef __CUDACC__
+// ---- E4M3 operands of the kind::f8f6f4 MMAs (FP8 cache)
+constexpr uint32_t kE4m3TileBytes = 16384;  // 128 keys x 128 E4M3 codes
+
+// Two floats -> their E4M3 codes (round to nearest even, saturating; y0 in the low
+// byte) and the values those codes stand for.
+__device__ __forceinline__ uint32_t e4m3_pair(float y0, float y1, float& v0, float& v1) {
+  const __nv_fp8x2_storage_t c =
+      __nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
+  const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(c, __NV_E4M3);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+  v0 = f.x;
+  v1 = f.y;
+  return (uint32_t)c;
+}
+__device__ __forceinline__ uint32_t e4m3_codes(float y0, float y1) {
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
+}
+
+// Q [H][128] bf16 -> the B operand of S^T = K . [Q_hi | Q_lo]^T (K-major, unswizzled,
+// N = 2H rows: row h holds Q_hi of head h, row H + h its Q_lo): 16-byte chunk c (16 d)
+// of row n at c * (2H * 16) + n * 16.  y = q * 2^e with the largest |y| in [128, 256),
+// Q_hi = E4M3(y), Q_lo = E4M3(16 (y - Q_hi)) (y - Q_hi is exact in float32).
+// *qinv = 2^-e.  Every thread of the block calls this; it ends with __syncthreads.
+template <int H>
+__device__ void store_q_e4m3_split(uint8_t* qs, const uint16_t* qg, float* qinv) {
+  __shared__ float hmax_s[kMaxHeads];
+  __shared__ float up_s;
+  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5, lane = threadIdx.x & 31;
+  for (int h = warp; h < H; h += nw) {
+    float m = 0.f;
+    for (int c = lane; c < kHeadDim; c += 32)
+      m = fmaxf(m, fabsf(__uint_as_float((uint32_t)qg[h * kHeadDim + c] << 16)));
+    m = warp_max(m);
+    if (lane == 0) hmax_s[h] = m;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.f;
+    for (int h = 0; h < H; ++h) m = fmaxf(m, hmax_s[h]);
+    int e = 0;
+    if (m > 0.f) {
+      int ex;
+      frexpf(m, &ex);  // m in [2^(ex-1), 2^ex)
+      e = 8 - ex;
+      e = e < -100 ? -100 : (e > 100 ? 100 : e);
+    }
+    up_s = __int_as_float((127 + e) << 23);
+    *qinv = __int_as_float((127 - e) << 23);
+  }
+  __syncthreads();
+  const float sc = up_s;
+  for (int w = threadIdx.x; w < H * (kHeadDim / 16); w += blockDim.x) {
+    const int h = w % H, c = w / H;
+    const uint4 a = *reinterpret_cast<const uint4*>(qg + h * kHeadDim + c * 16);
+    const uint4 b = *reinterpret_cast<const uint4*>(qg + h * kHeadDim + c * 16 + 8);
+    const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      hi[u] = 0u;
+      lo[u] = 0u;
+#pragma unroll
+      for (int v = 0; v < 2; ++v) {
+        const uint32_t x = in[2 * u + v];
+        const float y0 = __uint_as_float(x << 16) * sc;
+        const float y1 = __uint_as_float(x & 0xffff0000u) * sc;
+        float a0, a1;
+        const uint32_t ch = e4m3_pair(y0, y1, a0, a1);
+        const uint32_t cl = e4m3_codes((y0 - a0) * 16.f, (y1 - a1) * 16.f);
+        hi[u] |= ch << (16 * v);
+        lo[u] |= cl << (16 * v);
+      }
+    }
+    *reinterpret_cast<uint4*>(qs + c * (2 * H * 16) + h * 16) =
+        make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(qs + c * (2 * H * 16) + (H + h) * 16) =
+        make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+  __syncthreads();
+}
+
+// A operand K (K-major, 128-byte swizzle, one 128-byte row per key): K step kk of 32 d.
+__device__ __forceinline__ uint64_t k_e4m3_desc(uint32_t tile, int kk) {
+  return sm100::smem_desc(tile + (uint32_t)kk * 32u, 16, 1024, sm100::kSwizzle128B);
+}
+// B operand [Q_hi | Q_lo] (K-major, unswizzled, N rows): K step kk of 32 d.
+template <int N>
+__device__ __forceinline__ uint64_t q_e4m3_desc(uint32_t q, int kk) {
+  return sm100::smem_desc(q + (uint32_t)kk * 2u * N * 16u, N * 16, 128, sm100::kSwizzleNone);
+}
+// A operand V^T: the V tile is [128 keys][128 codes] with 128-byte swizzle, so V^T is
+// MN-major with all 128 d inside one swizzle atom; K step kk of 32 keys (four atoms
+// of 8 keys, 1024 bytes apart).
+__device__ __forceinline__ uint64_t vt_e4m3_desc(uint32_t tile, int kk) {
+  return sm100::smem_desc(tile + (uint32_t)kk * 32u * 128u, kE4m3TileBytes, 1024,
+                          sm100::kSwizzle128B);
+}
+// B operand P^T: P stored [3H / 16 chunks][128 keys][16 codes] (MN-major, unswizzled;
+// chunk (term * H + h) / 16 holds heads h..h+15 of one term); K step kk of 32 keys.
+__device__ __forceinline__ uint64_t pt_e4m3_desc(uint32_t p, int kk) {
+  return sm100::smem_desc(p + (uint32_t)kk * 32u * 16u, 128, kKeyTile * 16, sm100::kSwizzleNone);
+}
+
 #endif
 
 // Host: 2-D tiled tensor map over a row-major [rows][inner] array.
