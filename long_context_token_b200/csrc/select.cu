@@ -427,12 +427,72 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(SelectParams p
 }
 
 // ----------------------------------------------------------------------------
+// float64 selection key of one position, by one warp: max_h(sm_scale * q_h . k_j -
+// delta_h) from the stored inputs (K row widened exactly to float64 in the warp's
+// shared row kd -- FP8: code x scale -- then each lane takes heads lane, lane + 32, ...;
+// for H < 32 the lanes split each head's dot product into 32 / H parts, lane = part *
+// H + head).  q: the query's bf16 rows [H][kQLd] in shared memory; dlt: the float64
+// shifts.  Every lane returns the key.
+// ----------------------------------------------------------------------------
+constexpr int kQLd = kHeadDim + 8;  // padded q row (bf16) in shared memory
+
+template <int H, bool FP8>
+__device__ __forceinline__ double rescore_f64(const SelectParams& p, size_t row,
+                                              const uint16_t* qsm, const double* dlt,
+                                              double* kd, int lane) {
+  constexpr int kParts = H < 32 ? 32 / H : 1;
+  constexpr int kSpan = kHeadDim / kParts;
+  const int part = kParts > 1 ? lane / H : 0;
+  if (FP8) {
+    const uint32_t w4 = __ldg(reinterpret_cast<const uint32_t*>(
+                                  static_cast<const uint8_t*>(p.kv.k) + row * kHeadDim) + lane);
+    const double ksc = (double)__ldg(p.kv.k_scale + row);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) kd[4 * lane + u] = e4m3_to_f64((w4 >> (8 * u)) & 0xffu) * ksc;
+  } else {
+    const uint2 w4 = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.kv.k) +
+                                                          row * kHeadDim) + lane);
+    kd[4 * lane] = (double)bf16_bits_to_f32(w4.x & 0xffffu);
+    kd[4 * lane + 1] = (double)bf16_bits_to_f32(w4.x >> 16);
+    kd[4 * lane + 2] = (double)bf16_bits_to_f32(w4.y & 0xffffu);
+    kd[4 * lane + 3] = (double)bf16_bits_to_f32(w4.y >> 16);
+  }
+  __syncwarp();
+  const double scale = (double)p.sm_scale;
+  double best = -INFINITY;
+  for (int h0 = 0; h0 < H; h0 += 32 / kParts) {
+    const int h = h0 + (kParts > 1 ? lane % H : lane);
+    double dot = 0.0;
+    if (h < H) {
+      const uint16_t* qh = qsm + h * kQLd;
+#pragma unroll 4
+      for (int c = part * kSpan; c < (part + 1) * kSpan; c += 8) {
+        const uint4 qv = *reinterpret_cast<const uint4*>(qh + c);
+        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          dot = fma((double)bf16_bits_to_f32(qw[u] & 0xffffu), kd[c + 2 * u], dot);
+          dot = fma((double)bf16_bits_to_f32(qw[u] >> 16), kd[c + 2 * u + 1], dot);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o >= 32 / kParts && kParts > 1; o >>= 1)
+      dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    if (h < H) best = fmax(best, scale * dot - dlt[h]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) best = fmax(best, __shfl_xor_sync(0xffffffffu, best, o));
+  __syncwarp();  // the warp's next position reuses kd
+  return best;
+}
+
+// ----------------------------------------------------------------------------
 // 3. finish: exact select + float64 refinement + window merge + sort
 // ----------------------------------------------------------------------------
 constexpr int kFinThreads = 1024;
 constexpr int kSmallBand = 1024;  // bands up to this size are ranked pairwise in shared memory
 constexpr int kBuckets = 1024;    // counting-sort buckets of the final index set
-constexpr int kQLd = kHeadDim + 8;  // padded q row (bf16) in shared memory
 constexpr int kCandSmem = 4096;   // candidate lists up to this size are staged in shared memory
 // The final sort uses a bitmap of positions in the candidate staging area (8 bytes per
 // candidate slot, 32 positions per word) when the ranked range fits in it.
@@ -668,64 +728,17 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
   const bool band_smem = n_band <= kSmallBand;
 
   if (need2 > 0) {
-    // float64 re-scoring of the band, one warp per key: the warp first widens the key's
-    // row to float64 in shared memory (FP8: code x scale, exact), then each lane takes
-    // heads lane, lane + 32, ...; for H < 32 the lanes split each head's dot product
-    // into 32 / H parts (lane = part * H + head).
-    constexpr int kParts = H < 32 ? 32 / H : 1;
-    constexpr int kSpan = kHeadDim / kParts;
+    // float64 re-scoring of the band, one warp per key.
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int part = kParts > 1 ? lane / H : 0;
-    const double scale = (double)p.sm_scale;
     double* kd = kdsm + warp * kHeadDim;
     for (int e = warp; e < n_band; e += blockDim.x / 32) {
       const int j = band_smem ? band_js[e] : __ldcg(bj + e);
-      const size_t row = (size_t)b * p.kv.max_len + j;
-      if (FP8) {
-        const uint32_t w4 =
-            __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(p.kv.k) +
-                                                    row * kHeadDim) + lane);
-        const double ksc = (double)__ldg(p.kv.k_scale + row);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) kd[4 * lane + u] = e4m3_to_f64((w4 >> (8 * u)) & 0xffu) * ksc;
-      } else {
-        const uint2 w4 = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.kv.k) +
-                                                              row * kHeadDim) + lane);
-        kd[4 * lane] = (double)bf16_bits_to_f32(w4.x & 0xffffu);
-        kd[4 * lane + 1] = (double)bf16_bits_to_f32(w4.x >> 16);
-        kd[4 * lane + 2] = (double)bf16_bits_to_f32(w4.y & 0xffffu);
-        kd[4 * lane + 3] = (double)bf16_bits_to_f32(w4.y >> 16);
-      }
-      __syncwarp();
-      double best = -INFINITY;
-      for (int h0 = 0; h0 < H; h0 += 32 / kParts) {
-        const int h = h0 + (kParts > 1 ? lane % H : lane);
-        double dot = 0.0;
-        if (h < H) {
-          const uint16_t* qh = qsm + h * kQLd;
-#pragma unroll 4
-          for (int c = part * kSpan; c < (part + 1) * kSpan; c += 8) {
-            const uint4 qv = *reinterpret_cast<const uint4*>(qh + c);
-            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              dot = fma((double)bf16_bits_to_f32(qw[u] & 0xffffu), kd[c + 2 * u], dot);
-              dot = fma((double)bf16_bits_to_f32(qw[u] >> 16), kd[c + 2 * u + 1], dot);
-            }
-          }
-        }
-#pragma unroll
-        for (int o = 16; o >= 32 / kParts && kParts > 1; o >>= 1)
-          dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        if (h < H) best = fmax(best, scale * dot - dlt[h]);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) best = fmax(best, __shfl_xor_sync(0xffffffffu, best, o));
+      const double best =
+          rescore_f64<H, FP8>(p, (size_t)b * p.kv.max_len + j, qsm, dlt, kd, lane);
       if (lane == 0) {
         if (band_smem) band_ts[e] = best;
         else bt[e] = best;
       }
-      __syncwarp();  // the next key reuses kd
     }
     __syncthreads();
     if (band_smem) {
@@ -969,13 +982,8 @@ __global__ void __launch_bounds__(kBlkThreads) select_blocks_kernel(SelectParams
     const int n_band = (int)n_band_s;
     const bool band_smem = n_band <= kBlkSmallBand;
     const int need2 = kb - (int)n_keep_s;  // >= 1: tau's own block is in the band
-    // float64 re-scoring of every position of the band blocks, one warp per position
-    // (row widened to float64 in shared memory, lanes over heads or head parts); each
+    // float64 re-scoring of the band blocks' positions, one warp per position; each
     // block's score is the maximum over its positions (atomic max on ordered keys).
-    constexpr int kParts = H < 32 ? 32 / H : 1;
-    constexpr int kSpan = kHeadDim / kParts;
-    const int part = kParts > 1 ? lane / H : 0;
-    const double scale = (double)p.sm_scale;
     double* kd = kdsm + warp * kHeadDim;
     const long long n_pos = (long long)n_band * blk;
     for (long long f = warp; f < n_pos; f += kWarps) {
@@ -986,52 +994,12 @@ __global__ void __launch_bounds__(kBlkThreads) select_blocks_kernel(SelectParams
       // maximum: its float32 key is more than eps below the block's (each float32 key
       // is within eps / 2 of the exact one).  Both uniform over the warp.
       if (j >= n_c || __ldcg(trow + j) < bkey[c] - eps) continue;
-      const size_t row = (size_t)b * p.kv.max_len + j;
-      if (FP8) {
-        const uint32_t w4 =
-            __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(p.kv.k) +
-                                                    row * kHeadDim) + lane);
-        const double ksc = (double)__ldg(p.kv.k_scale + row);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) kd[4 * lane + u] = e4m3_to_f64((w4 >> (8 * u)) & 0xffu) * ksc;
-      } else {
-        const uint2 w4 = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.kv.k) +
-                                                              row * kHeadDim) + lane);
-        kd[4 * lane] = (double)bf16_bits_to_f32(w4.x & 0xffffu);
-        kd[4 * lane + 1] = (double)bf16_bits_to_f32(w4.x >> 16);
-        kd[4 * lane + 2] = (double)bf16_bits_to_f32(w4.y & 0xffffu);
-        kd[4 * lane + 3] = (double)bf16_bits_to_f32(w4.y >> 16);
-      }
-      __syncwarp();
-      double best = -INFINITY;
-      for (int h0 = 0; h0 < H; h0 += 32 / kParts) {
-        const int h = h0 + (kParts > 1 ? lane % H : lane);
-        double dot = 0.0;
-        if (h < H) {
-          const uint16_t* qh = qsm + h * kQLd;
-#pragma unroll 4
-          for (int cc = part * kSpan; cc < (part + 1) * kSpan; cc += 8) {
-            const uint4 qv = *reinterpret_cast<const uint4*>(qh + cc);
-            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              dot = fma((double)bf16_bits_to_f32(qw[u] & 0xffffu), kd[cc + 2 * u], dot);
-              dot = fma((double)bf16_bits_to_f32(qw[u] >> 16), kd[cc + 2 * u + 1], dot);
-            }
-          }
-        }
-#pragma unroll
-        for (int o = 16; o >= 32 / kParts && kParts > 1; o >>= 1)
-          dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        if (h < H) best = fmax(best, scale * dot - dlt[h]);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) best = fmax(best, __shfl_xor_sync(0xffffffffu, best, o));
+      const double best =
+          rescore_f64<H, FP8>(p, (size_t)b * p.kv.max_len + j, qsm, dlt, kd, lane);
       if (lane == 0) {
         if (band_smem) atomicMax(&band_key[e], ordered_key64(best));
         else atomicMax(bk + e, ordered_key64(best));
       }
-      __syncwarp();  // the next position reuses kd
     }
     __syncthreads();
     if (band_smem) {
