@@ -14,6 +14,11 @@
  *       paragraph on token granularity);
  *   3. each following sparse-attention layer, with its own queries, attends only
  *      to those positions of the same KV cache (same article, KV Reuse paragraph).
+ * Around the step: hs2_kv_append writes the new tokens' K and V rows before it (E4M3
+ * with a per-token scale for an FP8 cache); hs2_prefill_attn runs the full layer over
+ * a chunk of new tokens (chunked prefill, no selection); hs2_full_attn_select_blocks
+ * keeps whole 64-token blocks instead of tokens (the first-generation scheme the
+ * pages compare against).
  * The pages give no importance formula.  This library takes a key's importance as
  * max over query heads h of exp(s_hj - lse_h), the full layer's softmax
  * probability, with ties going to the lower position.
@@ -30,7 +35,8 @@
  *     length, an index out of range) are recorded in the workspace's status word
  *     and read with hs2_check_device_status().
  *   - head_dim must be 128.  h_q must be a multiple of 16 in [16, 128].
- *     n_q (query tokens per sequence) is in [1, 64].  window >= 1, k_sel >= 1,
+ *     n_q (query tokens per sequence) is in [1, 64] (hs2_prefill_attn: [1, 65536]).
+ *     window >= 1, k_sel >= 1,
  *     window + k_sel <= 4096.  Otherwise HS2_ERR_UNSUPPORTED.
  *   - Query token i of sequence b sits at position p = lens[b] - n_q + i and sees
  *     keys [0, p]; 1 <= n_q <= lens[b] <= max_len is required (checked on the

@@ -179,7 +179,7 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
   bool log2_partials = false;
   cudaError_t e;
   if (kv->dtype == HS2_KV_FP8_E4M3 && h <= 64) {
-    // Tensor-core flash-decode over E4M3 tiles widened to f16 in shared memory.
+    // Tensor-core flash-decode: the E4M3 tiles go straight into kind::f8f6f4 MMAs.
     CUtensorMap tk, tv;
     const uint64_t rows = (uint64_t)kv->batch * kv->max_len;
     if (!make_tmap_2d(&tk, kv->k, CU_TENSOR_MAP_DATA_TYPE_UINT8, kHeadDim, rows, kHeadDim, 128,

@@ -1,8 +1,14 @@
 """ctypes binding of libhs2 (argument marshalling only; every step runs in the CUDA
 library).  PyTorch provides device memory and the current stream.
 
-    out, idx, lse = full_attn_select(q, k, v, lens)            # full layer + selection
-    out_l = sparse_attn(q_layer, k, v, lens, idx, workspace=ws) # one reusing layer
+    cache = Cache(k, v, lens)                        # FP8: Cache(k, v, lens, k_scale, v_scale)
+    ws = alloc_workspace(cache, n_q, h_q)
+    kv_append(k_new, v_new, cache, ws)               # the new tokens' K/V rows; lens grows
+    out, idx, lse = full_attn_select(q, cache, workspace=ws)    # full layer + selection
+    out_l = sparse_attn(q_layer, cache, idx, ws)     # one reusing sparse layer
+    # comparators and neighbours of the step:
+    out, idx, lse = full_attn_select_blocks(q, cache, block=64, workspace=ws)
+    out, lse = prefill_attn(q_chunk, cache)          # full layer over a chunk of new tokens
 
 The library is loaded from ``long_context_token_b200/_lib/libhs2.so``.  There is no
 fallback: if the library is missing or no CUDA device is present, calls raise.
