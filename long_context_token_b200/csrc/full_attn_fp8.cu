@@ -11,7 +11,8 @@
 //     |q| into [128, 256): a bf16 element (8 significant bits) whose scaled magnitude
 //     is at least 2^-6 is exact in the two terms, smaller ones to 2^-13 absolute;
 //   P' = p * v_scale * 2^-ev rounded to f16 (11 significant bits, as an f16 P would
-//     carry) = P_hi + P_lo / 16 + P_lo2 / 256 exactly, ev a power of two at or above
+//     carry) = P_hi + P_lo / 16 + P_lo2 / 256 (exact for P' >= 2^-6; below, within
+//     2^-18 absolute, 2^-26 of the largest P' of 256), ev a power of two at or above
 //     every |v_scale| the CTA has seen, moved with a rescale of O (like the softmax
 //     reference) when a larger one arrives.
 // So S^T [128 keys x 2H] = K . [Q_hi | Q_lo]^T and O^T [128 d x 3H] += V^T . [P_hi |
@@ -81,9 +82,10 @@ struct Fp8Smem {
   static_assert(kQOff % 1024 == 0 && kPOff % 16 == 0 && kBarOff % 8 == 0, "alignment");
 };
 
-// Two f16 values y (11 significant bits) -> three pairs of E4M3 codes with
-// y = hi + lo / 16 + lo2 / 256 exactly (4 + 4 + 3 bits; every step's difference and
-// scaling is exact in f16 for |y| <= 448).  Element 0 in the low byte of each pair.
+// Two f16 values y (11 significant bits, |y| <= 448) -> three pairs of E4M3 codes with
+// y = hi + lo / 16 + lo2 / 256 (4 + 4 + 3 bits; every difference and scaling below is
+// exact in f16): exactly for |y| >= 2^-6, to 2^-18 absolute below (E4M3 subnormals).
+// Element 0 in the low byte of each pair.
 __device__ __forceinline__ void e4m3_split3(__half2 y, uint32_t& hi, uint32_t& lo, uint32_t& lo2) {
   const __half2 k16 = __float2half2_rn(16.f);
   hi = (uint32_t)__nv_cvt_halfraw2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
