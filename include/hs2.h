@@ -35,7 +35,8 @@
  *     length, an index out of range) are recorded in the workspace's status word
  *     and read with hs2_check_device_status().
  *   - head_dim must be 128.  h_q must be a multiple of 16 in [16, 128].
- *     n_q (query tokens per sequence) is in [1, 64] (hs2_prefill_attn: [1, 65536]).
+ *     n_q (query tokens per sequence) is in [1, 64] (hs2_prefill_attn: [1, 65536]);
+ *     batch * n_q <= 65535 (hs2_prefill_attn: batch * ceil(n_q * h_q / 128) <= 65535).
  *     window >= 1, k_sel >= 1,
  *     window + k_sel <= 4096.  Otherwise HS2_ERR_UNSUPPORTED.
  *   - Query token i of sequence b sits at position p = lens[b] - n_q + i and sees

@@ -92,6 +92,8 @@ static size_t sparse_prefix_bytes(const WsLayout& w) { return w.clear_begin; }
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+constexpr long long kMaxGridY = 65535;
+
 static hs2_status check_shape(int batch, int n_q, int h, int max_len, int window, int k_sel) {
   if (batch < 1 || max_len < 1) return HS2_ERR_INVALID_ARGUMENT;
   if (n_q < 1 || n_q > kMaxNq) return HS2_ERR_UNSUPPORTED;
@@ -99,6 +101,8 @@ static hs2_status check_shape(int batch, int n_q, int h, int max_len, int window
   if (window < 1 || k_sel < 1 || window + k_sel > kMaxIdxWidth) return HS2_ERR_UNSUPPORTED;
   if (max_len < n_q) return HS2_ERR_INVALID_ARGUMENT;
   if ((long long)batch * (long long)max_len >= (1ll << 31)) return HS2_ERR_UNSUPPORTED;
+  // One grid row per (sequence, token): the grid's y extent.
+  if ((long long)batch * n_q > kMaxGridY) return HS2_ERR_UNSUPPORTED;
   return HS2_OK;
 }
 
@@ -358,6 +362,9 @@ static hs2_status check_prefill(int batch, int n_q, int h, int max_len, int dtyp
   if (h != 16 && h != 32 && h != 48 && h != 64 && h != 128) return HS2_ERR_UNSUPPORTED;
   if (n_q < 1 || n_q > kMaxPrefillTokens || n_q > max_len) return HS2_ERR_UNSUPPORTED;
   if ((long long)batch * max_len >= (1ll << 31)) return HS2_ERR_UNSUPPORTED;
+  // One grid row per group of 128 / h tokens of a sequence: the grid's y extent.
+  const int G = mq_tokens_per_cta(h);
+  if ((long long)batch * ((n_q + G - 1) / G) > kMaxGridY) return HS2_ERR_UNSUPPORTED;
   return HS2_OK;
 }
 

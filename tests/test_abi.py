@@ -58,6 +58,7 @@ def test_workspace_sizes_for_every_workload(L, n):
     (1, 1, 16, 4096, 0, 1024, 0),      # empty window
     (1, 1, 16, 4096, 128, 1024, 2),    # unknown KV type
     (0, 1, 16, 4096, 128, 1024, 0),    # empty batch
+    (2048, 64, 16, 4096, 128, 1024, 0),  # 131072 (sequence, token) rows: above the grid's 65535
 ])
 def test_workspace_bytes_rejects_unsupported(L, args):
     assert L.hs2_workspace_bytes(*args) == 0
@@ -136,9 +137,15 @@ def test_block_selection_host_validation(L, block, k_sel, idx, max_len, expect):
     (1, 5000, 16, 4096, 0),       # chunk longer than the cache
     (1, 65537, 16, 1 << 20, 0),   # chunk above 65536 tokens
     (0, 512, 16, 4096, 0),        # empty batch
+    (1, 65536, 128, 65536, 0),    # 65536 row groups of one token: above the grid's 65535
 ])
 def test_prefill_workspace_rejects_unsupported(L, args):
     assert L.hs2_prefill_workspace_bytes(*args) == 0
+
+
+def test_prefill_accepts_the_largest_chunk(L):
+    # 65536 tokens at 16 heads: 8192 groups of 8 tokens
+    assert L.hs2_prefill_workspace_bytes(1, 65536, 16, 65536, 0) > 0
 
 
 def test_prefill_workspace_holds_the_partials(L):
