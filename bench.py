@@ -34,9 +34,11 @@ from long_context_token_b200 import workloads  # noqa: E402
 METRIC = "hybrid-block decode steps/s & HBM GB/s (full+select+sparse) at 128K-1M ctx"
 UNIT = "steps/s"
 FLUSH_BYTES = 256 << 20
-LAUNCHES_PER_STEP_FULL = 2      # split-K flash-decode, split merge
+LAUNCHES_PER_STEP_FUSED = 1     # full layer with the split merge and selection in its tail
+LAUNCHES_PER_STEP_FULL = 2      # split-K flash-decode, split merge (other shapes)
 LAUNCHES_PER_STEP_SELECT = 3    # importance+histogram, compaction, exact finish
 LAUNCHES_PER_STEP_BLOCKS = 2    # importance, exact block selection
+LAUNCHES_PER_FULL_FUSED = 1     # full layer merging its own split partials (block mode)
 LAUNCHES_PER_SPARSE = 1         # gather attention with the split merge on chip (cluster)
 
 
@@ -45,13 +47,14 @@ LAUNCHES_PER_SPARSE = 1         # gather attention with the split merge on chip 
 # sequences, scaled by sequences (the traffic is per sequence); see profiles/.
 NCU_TRAFFIC = {
     2: {"bytes": 4 * (134_288_128 + 786_304), "kernel": "full_attn_tc_kernel<16, 0>",
-        "capture": "2 x 131072 keys, scaled x4"},
+        "capture": "2 x 131072 keys, scaled x4", "fused": False},
     # first sequence of the ragged batch, scaled by the launch's algorithmic bytes
     3: {"bytes": round((56_967_424 + 623_104) * 245_681_880 / 56_903_232),
         "kernel": "full_attn_fp8_kernel<16, 0>",
-        "capture": "first sequence (56.9 MB of codes and scales), scaled to the 4-sequence launch"},
+        "capture": "first sequence (56.9 MB of codes and scales), scaled to the 4-sequence launch",
+        "fused": False},
     4: {"bytes": 276_918_528 + 5_604_608, "kernel": "full_attn_fp8_kernel<64, 0>",
-        "capture": "the whole launch"},
+        "capture": "the whole launch", "fused": False},
 }
 
 
@@ -163,7 +166,7 @@ class ClockSampler:
                         self.reasons.add(k)
             except Exception:
                 pass
-            self._stop.wait(0.01)
+            self._stop.wait(0.001)
 
     def __enter__(self):
         if self.nv is not None:
@@ -213,7 +216,10 @@ def host_cores():
 
 
 def run_reference(args, w):
-    """The reference arm: the float64 CPU oracle, each step one sequence of the batch."""
+    """The reference arm: the float64 CPU oracle.  Each of its steps is a bounded sample
+    of the workload, one sequence of the batch (1/B of a whole step); `value` is in
+    whole-workload steps/s (sequences/s divided by B) and `ms_per_step` is the measured
+    time of one such sample, so that steps x ms_per_step is the time spent."""
     ws, rank, _ = dist_env()
     if rank != 0:
         return
@@ -228,7 +234,10 @@ def run_reference(args, w):
     value = seqs / (secs * w.batch)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "step": f"one sequence of the batch of {w.batch} (1/{w.batch} of a whole step); "
+                "value = sequences/s / batch",
+        "sequences_timed": seqs, "seconds_timed": secs,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(w, args.block),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
@@ -427,15 +436,30 @@ def main():
     cache = hs2.Cache(inp.k.to(dev), inp.v.to(dev), inp.lens.to(dev),
                       None if inp.k_scale is None else inp.k_scale.to(dev),
                       None if inp.v_scale is None else inp.v_scale.to(dev))
-    q = inp.q.to(dev)
-    qls = [x.to(dev) for x in inp.q_layers]
     B, n_q, h = w.batch, w.n_q, w.h_q
     width = w.window + w.k_sel
+    n_layers = len(inp.q_layers)
     ws = hs2.alloc_workspace(cache, n_q, h, w.window, w.k_sel)
-    out = torch.empty(B, n_q, h, 128, dtype=torch.float32, device=dev)
+    fused = args.block == 1 and hs2.select_fused(cache, n_q, h)
+    # Every input of a step (the full layer's queries, then each sparse layer's) sits in
+    # one device buffer, and every result (the full layer's output, each sparse layer's
+    # output, then the index set) in another, so that the end-to-end leg moves each with
+    # a single copy.  Offsets are multiples of 16 bytes.
+    q_elems = B * n_q * h * 128
+    din = torch.empty((1 + n_layers) * q_elems, dtype=torch.bfloat16, device=dev)
+    q = din[:q_elems].view(B, n_q, h, 128)
+    qls = [din[(1 + i) * q_elems:(2 + i) * q_elems].view(B, n_q, h, 128) for i in range(n_layers)]
+    q.copy_(inp.q)
+    for d_, h_ in zip(qls, inp.q_layers):
+        d_.copy_(h_)
+    o_bytes = q_elems * 4
+    idx_bytes = B * n_q * width * 4
+    dout = torch.empty((1 + n_layers) * o_bytes + idx_bytes, dtype=torch.uint8, device=dev)
+    out = dout[:o_bytes].view(torch.float32).view(B, n_q, h, 128)
+    outs = [dout[(1 + i) * o_bytes:(2 + i) * o_bytes].view(torch.float32).view(B, n_q, h, 128)
+            for i in range(n_layers)]
+    idx = dout[(1 + n_layers) * o_bytes:].view(torch.int32).view(B, n_q, width)
     lse = torch.empty(B, n_q, h, dtype=torch.float32, device=dev)
-    idx = torch.empty(B, n_q, width, dtype=torch.int32, device=dev)
-    outs = [torch.empty_like(out) for _ in qls]
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     drain = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     drain_out = torch.empty((), dtype=torch.float32, device=dev)
@@ -454,23 +478,38 @@ def main():
         return res[1] if isinstance(res, tuple) and len(res) > 1 else None
 
     # Phase marks recorded from inside the captured graph (external event-record nodes),
-    # so the per-kernel durations come from the same replays that are timed.
+    # so the per-phase durations come from replays of the same step.
     marks = [cuda_ok(cudart.cudaEventCreate()) for _ in range(4)]
 
     def mark(k):
         cuda_ok(cudart.cudaEventRecordWithFlags(marks[k], stream.cuda_stream,
                                                 cudart.cudaEventRecordExternal))
 
+    def first_layer(with_marks=False):
+        """The full layer and the selection: one call (hs2_full_attn_select) for the token
+        selection, as a user makes it; the full layer and the block selection for the
+        comparator.  The marked capture splits the token path into its two calls where
+        they are separate kernels anyway, to time the full layer alone."""
+        if args.block > 1:
+            hs2.full_attn(q, cache, w.window, w.k_sel, inp.sm_scale, ws, out=out, lse=lse)
+            if with_marks:
+                mark(1)
+            hs2.select_blocks(q, cache, ws, w.window, w.k_sel, args.block, inp.sm_scale, idx=idx)
+        elif fused or not with_marks:
+            hs2.full_attn_select(q, cache, w.window, w.k_sel, inp.sm_scale, ws, out=out, idx=idx,
+                                 lse=lse)
+            if with_marks:
+                mark(1)
+        else:
+            hs2.full_attn(q, cache, w.window, w.k_sel, inp.sm_scale, ws, out=out, lse=lse)
+            if with_marks:
+                mark(1)
+            hs2.select(q, cache, ws, w.window, w.k_sel, inp.sm_scale, idx=idx)
+
     def step(with_marks=False):
         if with_marks:
             mark(0)
-        hs2.full_attn(q, cache, w.window, w.k_sel, inp.sm_scale, ws, out=out, lse=lse)
-        if with_marks:
-            mark(1)
-        if args.block > 1:
-            hs2.select_blocks(q, cache, ws, w.window, w.k_sel, args.block, inp.sm_scale, idx=idx)
-        else:
-            hs2.select(q, cache, ws, w.window, w.k_sel, inp.sm_scale, idx=idx)
+        first_layer(with_marks)
         if with_marks:
             mark(2)
         for ql, o in zip(qls, outs):
@@ -513,7 +552,7 @@ def main():
         torch.distributed.barrier()
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
-    step_ms, full_ms, sel_ms, sp_ms, replay_ms = [], [], [], [], []
+    step_ms, first_ms, full_ms, sel_ms, sp_ms, replay_ms = [], [], [], [], [], []
     with ClockSampler(dev) as clk:
         for k in range(args.steps):
             flush_l2(k)
@@ -531,6 +570,7 @@ def main():
             end.record(stream)
             end.synchronize()
             step_ms.append(elapsed(0, 3))
+            first_ms.append(elapsed(0, 2))
             full_ms.append(elapsed(0, 1))
             sel_ms.append(elapsed(1, 2))
             sp_ms.append(elapsed(2, 3))
@@ -540,23 +580,17 @@ def main():
     status = hs2.check_device_status(ws)
 
     # End to end through the public API: each step copies its queries from pinned host
-    # memory, runs the full layer + selection + sparse layers and copies every output
-    # (outputs and the index set) back; the step is replayed from a CUDA graph, as a
-    # serving loop would.  The KV cache is device-resident model state.
+    # memory in one copy, runs the full layer + selection + sparse layers and copies every
+    # result (the outputs and the index set) back in one copy; the step is replayed from
+    # a CUDA graph, as a serving loop would.  The KV cache is device-resident model state.
     e2e = None
     if not args.no_e2e:
-        hq = inp.q.pin_memory()
-        hqls = [x.pin_memory() for x in inp.q_layers]
-        hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-        hidx = torch.empty(idx.shape, dtype=torch.int32).pin_memory()
-        houts = [torch.empty(out.shape, dtype=torch.float32).pin_memory() for _ in qls]
-        h2d = hq.numel() * 2 + sum(x.numel() * 2 for x in hqls)
-        d2h = hout.numel() * 4 + hidx.numel() * 4 + sum(x.numel() * 4 for x in houts)
+        hin = torch.empty(din.shape, dtype=din.dtype).pin_memory()
+        hin.copy_(din.cpu())
+        hout = torch.empty(dout.shape, dtype=dout.dtype).pin_memory()
 
         def e2e_step():
-            q.copy_(hq, non_blocking=True)
-            for d_, h_ in zip(qls, hqls):
-                d_.copy_(h_, non_blocking=True)
+            din.copy_(hin, non_blocking=True)
             if args.block > 1:
                 hs2.full_attn_select_blocks(q, cache, w.window, w.k_sel, args.block,
                                             inp.sm_scale, ws, out=out, idx=idx, lse=lse)
@@ -565,10 +599,7 @@ def main():
                                      idx=idx, lse=lse)
             for ql, o in zip(qls, outs):
                 hs2.sparse_attn(ql, cache, idx, ws, inp.sm_scale, out=o)
-            hout.copy_(out, non_blocking=True)
-            hidx.copy_(idx, non_blocking=True)
-            for h_, o in zip(houts, outs):
-                h_.copy_(o, non_blocking=True)
+            hout.copy_(dout, non_blocking=True)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -588,7 +619,9 @@ def main():
             e_ms += start.elapsed_time(end)
         e_ms = max_over_ranks(e_ms, dev)
         e2e = {"value": whole_job_rate(world, args.steps, e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "h2d_bytes_per_step": int(hin.numel() * hin.element_size()),
+               "d2h_bytes_per_step": int(hout.numel()),
+               "copies_per_step": {"h2d": 1, "d2h": 1},
                "path": "hs2 C ABI via the Python binding, step replayed from a CUDA graph"}
         del g2
     del graph, graph_marked
@@ -600,9 +633,21 @@ def main():
     lens = inp.lens.tolist()
     ab = alg_bytes(w, lens)
     peaks, peak_kind = measured_peaks()
-    hbm_peak = float(peaks["hbm_gbs"])
-    full_avg = statistics.mean(full_ms) / 1e3
+    first_avg = statistics.mean(first_ms if fused else full_ms) / 1e3
     value = whole_job_rate(world, args.steps, total_ms)
+    if args.block > 1:
+        phases = {"full_attn": statistics.mean(full_ms), "select": statistics.mean(sel_ms)}
+        launches = LAUNCHES_PER_FULL_FUSED + LAUNCHES_PER_STEP_BLOCKS
+    elif fused:
+        phases = {"full_attn_select": statistics.mean(first_ms)}
+        launches = LAUNCHES_PER_STEP_FUSED
+    else:
+        phases = {"full_attn": statistics.mean(full_ms), "select": statistics.mean(sel_ms)}
+        launches = LAUNCHES_PER_STEP_FULL + LAUNCHES_PER_STEP_SELECT
+    roof = roofline_of(w, ab, first_avg, peaks, peak_kind)
+    if fused:
+        roof["kernel"] = ("full layer with the split merge and the token selection in its "
+                          "tail (one launch)")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -610,23 +655,21 @@ def main():
         "data": "synthetic", "config": config_of(w, args.block),
         "hbm_gbs": ab["step"] / (total_ms / args.steps / 1e3) / 1e9,
         "alg_bytes_per_step": ab["step"],
-        "phase_ms": {"full_attn": statistics.mean(full_ms), "select": statistics.mean(sel_ms),
-                     "sparse_layers": statistics.mean(sp_ms),
-                     "step_with_phase_marks": statistics.mean(step_ms),
-                     "step_p10": float(np.percentile(replay_ms, 10)),
-                     "step_p50": float(np.percentile(replay_ms, 50)),
-                     "step_p90": float(np.percentile(replay_ms, 90))},
-        "roofline": roofline_of(w, ab, full_avg, peaks, peak_kind) | {
+        "phase_ms": phases | {"sparse_layers": statistics.mean(sp_ms),
+                              "step_with_phase_marks": statistics.mean(step_ms),
+                              "step_p10": float(np.percentile(replay_ms, 10)),
+                              "step_p50": float(np.percentile(replay_ms, 50)),
+                              "step_p90": float(np.percentile(replay_ms, 90))},
+        "roofline": roof | {
                      "alg_bytes_per_launch": ab["full"],
                      "traffic": (NCU_TRAFFIC[args.workload]["bytes"]
-                                 if args.workload in NCU_TRAFFIC and args.batch is None else None),
+                                 if args.workload in NCU_TRAFFIC and args.batch is None
+                                 and NCU_TRAFFIC[args.workload]["fused"] == fused else None),
                      "traffic_source": (NCU_TRAFFIC[args.workload]
                                         if args.workload in NCU_TRAFFIC and args.batch is None
+                                        and NCU_TRAFFIC[args.workload]["fused"] == fused
                                         else None)},
-        "gpu_launches": args.steps * (LAUNCHES_PER_STEP_FULL
-                                      + (LAUNCHES_PER_STEP_BLOCKS if args.block > 1
-                                         else LAUNCHES_PER_STEP_SELECT)
-                                      + w.n_sparse * LAUNCHES_PER_SPARSE),
+        "gpu_launches": args.steps * (launches + w.n_sparse * LAUNCHES_PER_SPARSE),
         "clocks": clk.summary(),
         "device_status": status,
         "wall_s_timed_region": wall,

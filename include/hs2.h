@@ -252,6 +252,12 @@ HS2_API hs2_status hs2_check_device_status(void* workspace, hs2_stream_t stream)
 /* Static description of a status code (never NULL). */
 HS2_API const char* hs2_status_string(hs2_status status);
 
+/* 1 if hs2_full_attn_select runs as a single kernel for these sizes (the one-token
+ * tensor-core full layer, which merges its split partials and selects the tokens in its
+ * own tail), 0 if it runs as the full layer, the split merge and separate selection
+ * kernels.  The results are the same either way; only the launches differ. */
+HS2_API int hs2_select_fused(int n_q, int h_q, int dtype);
+
 /* Text of the last CUDA error seen by this thread's calls ("" if none). */
 HS2_API const char* hs2_last_cuda_error(void);
 

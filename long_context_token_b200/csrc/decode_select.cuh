@@ -1,0 +1,864 @@
+// Fused tail of the one-token full layer: after streaming their key chunks, the CTAs
+// of one (sequence, token) row merge their split partials and select the row's tokens
+// together, so that the step needs no separate merge, importance or selection kernels.
+//
+// The selection (web coverage of HySparse2: toolnavs article 2080, fr "Ce que fait
+// HySparse2", paragraph on selection granularity -- the last `window` positions, plus
+// the top `k_sel` positions outside the window ranked by the full layer's own scores)
+// ranks key j by t_j = max_h (x_hj - D_h), x_hj = s_hj log2(e) its logit in log2 units
+// and D_h = lse2_h - min_h' lse2_h' (log2 units): the same order as max_h exp(s_hj -
+// lse_h).  The lse is only known once every chunk of the row is done, so during the
+// stream each key records only the bound
+//     u_j = max_h x_hj,     u_j - W <= t_j <= u_j,     W = max_h D_h,
+// and counts u_j in a shared-memory histogram, linear in u.  Then, per row (CTA r of the
+// row owns the positions [r chunk, (r + 1) chunk) for the selection):
+//   1. every CTA publishes its histogram and arrives at the row's first barrier (its own
+//      bounds already on their way into shared memory), then computes the row's lse from
+//      the split partials;
+//   2. the bin holding the k_sel-th largest u gives a lower edge lo; no key with
+//      u_j < lo - W - 2 eps can be among the top k_sel (the k_sel-th largest t, T, is at
+//      least lo - W), so only the other keys of its chunk -- the candidates, a few per
+//      thousand -- get their exact float32 t_j, from their K rows gathered again through
+//      the tensor cores, and go to the row's candidate list;
+//   3. after the second barrier every CTA reads the whole candidate list (a few thousand
+//      entries) and takes the same decisions from it: the fine histogram of t over
+//      [lo - W - 2 eps, hi] (which holds T) gives the bin B of the k_sel-th largest t; with
+//      m bins of width at least eps around it, keys of bins >= B + m are in, keys of bins
+//      < B - m are out, and the band between is re-scored in float64 and ranked by (key
+//      desc, position asc);
+//   4. each CTA writes the selected positions of its own chunk, in order, from the slot
+//      after the selected positions below its chunk; the first CTA appends the window.
+//      Then the CTA lets the next kernel start and merges its share of the row's output.
+// The float32 keys are within eps / 2 of the exact ones, eps = 1e-3 max(1, |bin edge| +
+// W) (as in the separate selection kernels), so the chosen set is the float64
+// definition's up to the tie band.
+//
+// The CTAs of a row wait for one another at the barriers: the kernel is launched
+// cooperatively (all CTAs resident) whenever a row has more than one CTA, and every
+// wait gives up after a bounded number of cycles, recording HS2_ERR_DEVICE_TIMEOUT.
+#pragma once
+
+#include "hs2_internal.cuh"
+#include "select_common.cuh"
+#include "sm100.cuh"
+
+namespace hs2 {
+
+constexpr int kUBins = 2048;         // bins of the u histogram and of the fine t histogram
+constexpr float kUScale = 16.f;      // u bins per log2 unit
+constexpr float kUOrigin = -64.f;    // lower edge of u bin 1 is kUOrigin + 1/16
+constexpr float kSelEps = 1e-3f;
+constexpr long long kRowSpinCycles = 4000000000ll;
+constexpr int kBandSmem = 512;       // bands up to this size are ranked pairwise on chip
+constexpr int kTailTiles = 2;        // candidate tiles (128 keys) gathered at a time
+static_assert(kUBins <= kHistBins, "the u histogram lives in the histogram region");
+
+// Slots of a row's synchronisation words (the first two belong to the separate selection
+// kernels).
+enum : int { kRowNBand = 2, kRowArrive1 = 3, kRowArrive2 = 4, kRowArrive3 = 5, kRowDone = 6,
+             kRowNcand = 7 };
+
+// Histogram bin of a bound u: monotone in u, u below -64 + 1/16 in bin 0 and u at or above
+// 64 - 1/16 in the last bin (a NaN goes to bin 0).
+__device__ __forceinline__ int ubin(float u) {
+  float y = (u - kUOrigin) * kUScale;
+  y = fminf(fmaxf(y, 0.f), (float)(kUBins - 1));
+  return (int)y;
+}
+// Nominal lower edge of bin b.
+__device__ __forceinline__ float ubin_edge(int b) { return (float)b / kUScale + kUOrigin; }
+// A value at or below every u whose bin is b or higher: the edge less the rounding of
+// u - kUOrigin (at most 2^-18 below 128) and of this subtraction.
+__device__ __forceinline__ float ubin_floor(int b) {
+  return b <= 0 ? -INFINITY : ubin_edge(b) - 3e-5f;
+}
+
+// The fine histogram of t over [lo, lo + kUBins / inv_w): monotone, clamped at both ends.
+struct FineBins {
+  float lo, inv_w;
+  __device__ __forceinline__ int bin(float t) const {
+    float y = (t - lo) * inv_w;
+    y = fminf(fmaxf(y, 0.f), (float)(kUBins - 1));
+    return (int)y;
+  }
+};
+
+// Shared-memory histograms keep four padding words after every 64 bins: 16-byte chunks
+// stay aligned (cp.async copies them in), and the 32 lanes scanning 64 consecutive bins
+// each (kth_bin_from_top) meet at most 4-way bank conflicts.
+constexpr int kUBinsPadded = kUBins + kUBins / 16;
+__device__ __forceinline__ int ubin_slot(int b) { return b + ((b >> 6) << 2); }
+
+// ---- row barriers: every CTA of a row arrives once per counter and call, then waits
+// until `target` have.  Arrival: a block barrier, then a release reduction by thread 0
+// (the CTA's earlier writes, ordered by the block barrier, become visible to whoever
+// acquires the counter).  Waiting: thread 0 spins on an acquire load (a bounded number of
+// cycles), then a block barrier.
+__device__ __forceinline__ void row_arrive(uint32_t* counter) {
+  __syncthreads();
+  if (threadIdx.x == 0) sm100::red_release_gpu_add(counter, 1u);
+}
+static __device__ __noinline__ bool row_wait(uint32_t* counter, uint32_t target) {
+  __shared__ uint32_t ok_s;
+  if (threadIdx.x == 0) {
+    uint32_t ok = 1;
+    if (sm100::ld_acquire_gpu_u32(counter) < target) {
+      const long long t0 = clock64();
+      while (sm100::ld_acquire_gpu_u32(counter) < target) {
+        if (clock64() - t0 > kRowSpinCycles) {
+          ok = 0;
+          break;
+        }
+        __nanosleep(100);  // leave the counter's L2 slice to the others
+      }
+    }
+    ok_s = ok;
+  }
+  __syncthreads();
+  return ok_s != 0;
+}
+
+// Warp 0 scans a padded shared-memory histogram (ubin_slot) from the top: lane l owns
+// bins [kUBins - 64(l + 1), kUBins - 64 l).  Returns (to every thread) the bin holding the
+// k-th largest element, or 0 if there are fewer than k.  All threads call.
+__device__ __forceinline__ int kth_bin_from_top(int k, const uint32_t* hs) {
+  static_assert(kUBins == 32 * 64, "64 bins per lane");
+  __shared__ int bin_s;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int base = kUBins - 64 * (lane + 1);
+    const uint4* row = reinterpret_cast<const uint4*>(hs + ubin_slot(base));  // contiguous
+    uint4 c[16];
+    uint32_t sum = 0;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      c[u] = row[u];
+      sum += c[u].x + c[u].y + c[u].z + c[u].w;
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += x;
+    }
+    if (lane == 0) bin_s = 0;
+    __syncwarp();
+    const uint32_t above = incl - sum;
+    if (above < (uint32_t)k && (uint32_t)k <= incl) {
+      uint32_t cum = above;
+      int bin = base;
+      bool found = false;
+#pragma unroll
+      for (int u = 15; u >= 0; --u) {
+        const uint32_t v[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+#pragma unroll
+        for (int q = 3; q >= 0; --q) {
+          cum += v[q];
+          if (!found && cum >= (uint32_t)k) {
+            found = true;
+            bin = base + 4 * u + q;
+          }
+        }
+      }
+      bin_s = bin;
+    }
+  }
+  __syncthreads();
+  return bin_s;
+}
+
+// Warp 0 (all 32 lanes) reads a global kUBins histogram straight into registers (lane l
+// holds bins [kUBins - 64(l + 1), kUBins - 64 l)) and finds the bin B holding the k-th
+// largest element (0 if there are fewer than k).  With mb > 0 it also sums the bins >= B +
+// mb (`above`) and the bins [B - mb, B + mb) (`near`).  Results in lane 0.
+struct BinScan {
+  int bin;
+  uint32_t above, near;
+};
+__device__ __forceinline__ BinScan scan_global_bins(const uint32_t* gh, int k, int mb) {
+  static_assert(kUBins == 32 * 64, "64 bins per lane");
+  const int lane = threadIdx.x & 31;
+  const int base = kUBins - 64 * (lane + 1);
+  uint4 c[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) c[u] = __ldcg(reinterpret_cast<const uint4*>(gh + base) + u);
+  uint32_t sum = 0;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) sum += c[u].x + c[u].y + c[u].z + c[u].w;
+  uint32_t incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  const uint32_t before = incl - sum;  // in the bins above this lane's
+  int bin = -1;
+  if (before < (uint32_t)k && (uint32_t)k <= incl) {
+    uint32_t cum = before;
+#pragma unroll
+    for (int u = 15; u >= 0; --u) {
+      const uint32_t v[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+#pragma unroll
+      for (int q = 3; q >= 0; --q) {
+        cum += v[q];
+        if (bin < 0 && cum >= (uint32_t)k) bin = base + 4 * u + q;
+      }
+    }
+  }
+  const unsigned found = __ballot_sync(0xffffffffu, bin >= 0);
+  const int B = found ? __shfl_sync(0xffffffffu, bin, __ffs(found) - 1) : 0;
+  BinScan r;
+  r.bin = B;
+  r.above = 0;
+  r.near = 0;
+  if (mb > 0) {
+    uint32_t above = 0, near = 0;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const uint32_t v[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int e = base + 4 * u + q;
+        above += e >= B + mb ? v[q] : 0u;
+        near += (e >= B - mb && e < B + mb) ? v[q] : 0u;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      above += __shfl_xor_sync(0xffffffffu, above, o);
+      near += __shfl_xor_sync(0xffffffffu, near, o);
+    }
+    r.above = above;
+    r.near = near;
+  }
+  return r;
+}
+
+// Adds a padded shared-memory histogram to a global one: every non-empty bin at or above
+// `low`.  All threads call.
+__device__ __forceinline__ void add_bins(const uint32_t* hs, uint32_t* gh, int low) {
+  for (int e = low + (int)threadIdx.x; e < kUBins; e += blockDim.x) {
+    const uint32_t c = hs[ubin_slot(e)];
+    if (c) atomicAdd(gh + e, c);
+  }
+}
+
+// Asynchronous copies (cp.async, waited for with cp_async_wait_all) by all threads:
+// a global histogram into a padded shared-memory copy, and n 4-byte words.
+__device__ __forceinline__ void async_bins(uint32_t* hs, const uint32_t* gh) {
+  for (int v = threadIdx.x; v < kUBins / 4; v += blockDim.x)
+    sm100::cp_async_16(sm100::smem_u32(hs + ubin_slot(4 * v)), gh + 4 * v, 16u);
+}
+__device__ __forceinline__ void async_words(void* dst, const void* src, int n) {
+  const int nv = (n + 3) / 4;
+  for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+    const int left = n - 4 * v;
+    sm100::cp_async_16(sm100::smem_u32(static_cast<uint8_t*>(dst) + 16 * v),
+                       static_cast<const uint8_t*>(src) + 16 * v, left >= 4 ? 16u : 4u * left);
+  }
+}
+
+// Block-wide ordered compaction: the indices e of [0, m) with pred(e), in increasing
+// order, as val(e) into out[0, count); returns count to every thread.  Each thread takes a
+// contiguous run of up to 64 indices (independent loads, a bit mask), then one block-wide
+// exclusive scan of the counts places the runs: no atomics on a shared counter, whose
+// round trips would serialise a loop run by a handful of warps.  All threads call.
+template <typename Pred, typename Val>
+__device__ __forceinline__ int block_compact(int m, Pred pred, Val val, int* out) {
+  __shared__ uint32_t wsum[32];
+  const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = nt >> 5;
+  int total = 0;
+  for (int c0 = 0; c0 < m; c0 += 64 * nt) {
+    const int cm = min(64 * nt, m - c0);
+    const int R = (cm + nt - 1) / nt;
+    const int e0 = c0 + tid * R, e1 = min(e0 + R, c0 + cm);
+    unsigned long long mask = 0ull;
+#pragma unroll 8
+    for (int e = e0; e < e1; ++e)
+      if (pred(e)) mask |= 1ull << (e - e0);
+    const uint32_t cnt = (uint32_t)__popcll(mask);
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += x;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    uint32_t before = 0, all = 0;
+    for (int w = 0; w < nw; ++w) {
+      const uint32_t c = wsum[w];
+      before += w < warp ? c : 0u;
+      all += c;
+    }
+    uint32_t at = (uint32_t)total + before + incl - cnt;
+    while (mask) {
+      const int r = __ffsll(mask) - 1;
+      mask &= mask - 1;
+      out[at++] = val(e0 + r);
+    }
+    total += (int)all;
+    __syncthreads();  // wsum is reused by the next chunk or call
+  }
+  return total;
+}
+
+// The row's log-sum-exp per head, from its split partials.
+template <int H>
+struct RowLse {
+  float M[H];      // largest reference m over the non-empty splits (log2 units)
+  float invL[H];   // 1 / sum_s l_s 2^(m_s - M)
+  double lse2[H];  // M + log2 sum_s l_s 2^(m_s - M)  (log2 units)
+  double dl[H];    // (lse2 - min_h lse2) ln 2: the float64 shifts of the re-scoring
+  float D[H];      // lse2 - min_h lse2 (log2 units, float32)
+  float W;         // max_h D
+};
+
+// Every thread calls this; pml: the row's partials [S][H][2] (m in log2 units, l).  Head h
+// is taken by tph consecutive threads (the largest power of two, at most 32, with
+// H * tph <= blockDim), each over the splits sub, sub + tph, ...: the largest reference M
+// over the non-empty splits, then L = sum_s l_s 2^(m_s - M) with each weight in float32
+// (relative error below 2^-22, well under that of the partial sums l) summed without loss
+// (two-sum, also across the threads of the head).  log2 L is taken on the mantissa of its
+// leading float (log2f of a value in [0.5, 1), absolute error about 2^-24) plus the
+// exponent and the first-order term of the trailing float, and assembled with M in
+// float64: lse2 carries about 2^-23 absolute, well inside the 1e-6 tie band of the
+// selection.  The shifts D and dl are taken from C, a common value just below the
+// smallest lse2 (the ranking does not depend on which).
+template <int H>
+__device__ __forceinline__ void row_lse(const float* __restrict__ pml, int S, RowLse<H>& r) {
+  const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31;
+  int tph = 1;
+  while (tph < 32 && 2 * tph * H <= nt) tph *= 2;
+  const int h = tid / tph, sub = tid % tph;
+  const bool mine = h < H;
+  float M = -INFINITY;
+  if (mine) {
+#pragma unroll 8
+    for (int s = sub; s < S; s += tph) {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(pml + ((size_t)s * H + h) * 2));
+      if (v.y > 0.f) M = fmaxf(M, v.x);
+    }
+  }
+  for (int o = 1; o < tph; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float ls = 0.f, le = 0.f;
+  if (mine && M != -INFINITY) {
+#pragma unroll 8
+    for (int s = sub; s < S; s += tph) {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(pml + ((size_t)s * H + h) * 2));
+      if (v.y > 0.f) two_sum_acc(ls, le, v.y * exp2f(v.x - M));
+    }
+  }
+  for (int o = 1; o < tph; o <<= 1) {
+    const float os = __shfl_xor_sync(0xffffffffu, ls, o);
+    const float oe = __shfl_xor_sync(0xffffffffu, le, o);
+    le += oe;
+    two_sum_acc(ls, le, os);
+  }
+  if (mine && sub == 0) {
+    const float lh = ls + le;            // leading float of L
+    const float ll = (ls - lh) + le;     // and the rest
+    r.M[h] = M;
+    if (lh > 0.f) {
+      int ex;
+      const float mant = frexpf(lh, &ex);  // lh = mant 2^ex, mant in [0.5, 1)
+      r.invL[h] = 1.f / lh;
+      r.lse2[h] = (double)M + (double)ex + (double)log2f(mant) +
+                  (double)(ll / lh * 1.4426950408889634f);
+    } else {
+      r.invL[h] = 0.f;
+      r.lse2[h] = -INFINITY;
+    }
+  }
+  __syncthreads();
+  if (tid < 32) {
+    float mn = INFINITY, mx = -INFINITY;
+    for (int hh = lane; hh < H; hh += 32) {
+      mn = fminf(mn, (float)r.lse2[hh]);
+      mx = fmaxf(mx, (float)r.lse2[hh]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    const double c = (double)mn - 1e-5 * fmax(1.0, fabs((double)mn));  // at or below every lse2
+    float w = 0.f;
+    for (int hh = lane; hh < H; hh += 32) {
+      const double d = r.lse2[hh] - c;
+      r.D[hh] = (float)d;
+      r.dl[hh] = d * 0.69314718055994530942;
+      w = fmaxf(w, (float)d);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, o));
+    if (lane == 0) r.W = w * (1.f + 1e-6f);  // covers the rounding of D to float
+    (void)mx;
+  }
+  __syncthreads();
+}
+
+// This CTA's share of the row's merged output: outputs (h, d) of the row taken in turn
+// by the row's S CTAs; out_h = sum_s 2^(m_s - M) o_s / L.  The thread holding d = 0 of a
+// head writes its lse (natural log) to lse64 and lse_out.
+template <int H>
+__device__ __forceinline__ void row_merge(const FullParams& p, int bq, int split, int S,
+                                          const RowLse<H>& r) {
+  const float* po = p.part_o + (size_t)bq * S * H * kHeadDim;
+  const float* pml = p.part_ml + (size_t)bq * S * H * 2;
+  constexpr int kOut = H * kHeadDim;
+  constexpr int kB = 8;  // splits whose loads are in flight together
+  for (int o = split * (int)blockDim.x + (int)threadIdx.x; o < kOut; o += S * (int)blockDim.x) {
+    const int h = o / kHeadDim, d = o % kHeadDim;
+    const float M = r.M[h], il = r.invL[h];
+    float acc = 0.f;
+    for (int s0 = 0; s0 < S; s0 += kB) {
+      float2 ml[kB];
+      float v[kB];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int s = s0 + u;
+        ml[u] = s < S ? __ldcg(reinterpret_cast<const float2*>(pml + ((size_t)s * H + h) * 2))
+                      : make_float2(0.f, 0.f);
+        v[u] = s < S ? __ldcg(po + ((size_t)s * H + h) * kHeadDim + d) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kB; ++u)
+        if (ml[u].y > 0.f) acc = fmaf(exp2f(ml[u].x - M) * il, v[u], acc);
+    }
+    p.out[(size_t)bq * kOut + o] = acc;
+    if (d == 0) {
+      const double lse = r.lse2[h] * 0.69314718055994530942;
+      if (p.lse64) p.lse64[(size_t)bq * H + h] = lse;
+      if (p.lse_out) p.lse_out[(size_t)bq * H + h] = (float)lse;
+    }
+  }
+}
+
+// Index row of a row that keeps every position (no more than k_sel positions outside the
+// window): [0, pos], then -1.
+__device__ __forceinline__ void write_all_positions(int32_t* out_row, int width, int pos) {
+  for (int e = threadIdx.x; e < width; e += blockDim.x) out_row[e] = e <= pos ? e : -1;
+}
+
+// Where the tail finds the query for the float64 re-scoring (byte strides of heads and of
+// 8-element chunks, as rescore_f64 takes them).
+struct QView {
+  const uint8_t* base;
+  int hstride, cstride;
+};
+
+// Steps 2 to 4 of the selection (see the top of this file), after the row's first barrier
+// and lse, with this CTA's first `first` bounds already in `us`.  All threads of every CTA
+// of the row call it.  `recompute(list, m, t2, round, D)` (all threads) gathers the K rows
+// of the positions list[0, m) (m <= kTailTiles * 128), runs them through the stream's S =
+// K Q^T MMA and stores t = max_h (x_h - D[h]) of each into t2[0, m), ending with a block
+// barrier; it returns false if a wait gave up.  Returns false if a wait gave up.
+template <int H, bool FP8, typename Recompute>
+__device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* stage,
+                                           uint32_t stage_bytes, uint32_t tile_bytes, float* us,
+                                           int* cl, float* t2s, int piece, int bq, int b,
+                                           int split, int S, int k0, int c_hi, int n_c, int pos,
+                                           int bk, const RowLse<H>& rl, const QView& qv,
+                                           Recompute&& recompute) {
+  __shared__ uint32_t slot_s, ncand_s, nband_s, sure_s, below_s, base_s;
+  __shared__ float eps_s;
+  __shared__ FineBins fb_s;
+  __shared__ int mb_s;
+  __shared__ unsigned long long vb_s;
+  __shared__ int jb_s;
+  __shared__ uint32_t warp_cnt[32];
+  const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = nt >> 5;
+  const int width = p.window + p.k_sel;
+  int32_t* out_row = p.sel_idx + (size_t)bq * width;
+  const size_t rowoff = (size_t)bq * p.kv.max_len;
+  uint32_t* rs = p.rowsync + (size_t)bq * 8;
+  float* gct = p.cand_t + (size_t)bq * p.ld_u;  // the row's candidate list (16-byte aligned)
+  int32_t* gcj = p.cand_j + (size_t)bq * p.ld_u;
+  bool ok = true;
+
+  if (tid == 0) {
+    const float edge = fmaxf(fabsf(ubin_edge(bk)), fabsf(ubin_edge(bk + 1)));
+    const float eps = kSelEps * fmaxf(1.f, edge + rl.W);
+    // T (the k_sel-th largest t) lies in [floor(bk) - W, edge(bk + 1)]: the fine bins
+    // span that with a margin; keys outside fall into the end bins.
+    const float lo = bk <= 0 ? kUOrigin - 64.f - rl.W : ubin_floor(bk) - rl.W - 2.f * eps;
+    const float hi = bk >= kUBins - 1 ? lo + 2.f * rl.W + 64.f : ubin_edge(bk + 1) + 3e-5f;
+    FineBins fb;
+    fb.lo = lo;
+    fb.inv_w = (float)kUBins / fmaxf(hi - lo, 1e-6f);
+    fb_s = fb;
+    eps_s = eps;
+    // mb bins of the fine histogram cover eps, with a spare bin for rounding.
+    mb_s = (int)ceilf(eps * fb.inv_w) + 2;
+  }
+  __syncthreads();
+  const float eps = eps_s;
+  const float theta = ubin_floor(bk) - rl.W - 2.f * eps;
+
+  // ---- 2. this chunk's candidates, a piece at a time, through the tensor cores in rounds
+  // of kTailTiles tiles; their keys go to the row's candidate list.
+  uint32_t round = 0;
+  for (int pc = k0; pc < c_hi; pc += piece) {
+    const int m = min(piece, c_hi - pc);
+    if (pc != k0) {  // later pieces (long chunks only) are staged here
+      __syncthreads();
+      async_words(us, p.ubuf + (size_t)bq * p.ld_u + pc, m);
+      sm100::cp_async_wait_all();
+    }
+    __syncthreads();
+    const int ncl = block_compact(
+        m, [&](int e) { return us[e] >= theta; }, [&](int e) { return pc + e; }, cl);
+    uint32_t base = 0;
+    if (tid == 0 && ncl > 0) base = atomicAdd(rs + kRowNcand, (uint32_t)ncl);  // in flight
+    for (int r0 = 0; r0 < ncl; r0 += kTailTiles * 128, ++round) {
+      const int mm = min(kTailTiles * 128, ncl - r0);
+      if (!recompute(cl + r0, mm, t2s, round, rl.D)) ok = false;
+      if (tid == 0 && r0 == 0) slot_s = base;
+      __syncthreads();
+      const uint32_t at = slot_s + (uint32_t)r0;
+      for (int e = tid; e < mm; e += nt) {
+        gct[at + e] = t2s[e];
+        gcj[at + e] = cl[r0 + e];
+      }
+      __syncthreads();
+    }
+  }
+  row_arrive(rs + kRowArrive2);
+  if (!row_wait(rs + kRowArrive2, (uint32_t)S)) ok = false;
+  // Every CTA of the row has its copy of the u histogram by now (each copied it before
+  // arriving): clear this CTA's share for the next call.
+  uint32_t* gu = p.uhist + (size_t)bq * kHistBins;
+  for (int e = split * nt + tid; e < kUBins; e += S * nt) gu[e] = 0u;
+
+  // ---- 3. every CTA reads the row's candidate list and takes the same decisions
+  // Each thread holds kRegCand entries of the list in registers per pass; one pass builds
+  // the fine histogram of every candidate and that of the candidates below this chunk.
+  uint32_t off = 0;
+  auto take = [&](uint32_t bytes) {
+    uint8_t* at = stage + off;
+    off += (bytes + 15u) & ~15u;
+    return at;
+  };
+  uint32_t* fh = reinterpret_cast<uint32_t*>(take(kUBinsPadded * 4));   // all candidates
+  uint32_t* fb_lo = reinterpret_cast<uint32_t*>(take(kUBinsPadded * 4));  // those below k0
+  unsigned long long* bkey = reinterpret_cast<unsigned long long*>(take(kBandSmem * 8));
+  int* bpos = reinterpret_cast<int*>(take(kBandSmem * 4));
+  float* kf = reinterpret_cast<float*>(take((uint32_t)nwarps * kHeadDim * 4));
+  const int chunk_len = c_hi > k0 ? c_hi - k0 : 0;
+  const int nwords = (chunk_len + 31) / 32;
+  uint32_t* bm = reinterpret_cast<uint32_t*>(take((uint32_t)nwords * 4));
+  // This chunk's band keys, in the rest of the stages (a chunk's worth, or as many as fit).
+  int* own_band = reinterpret_cast<int*>(stage + off);
+  const uint32_t own_cap = min((uint32_t)max(chunk_len, 1), (stage_bytes > off ? stage_bytes - off : 0u) / 4u);
+  for (int e = tid; e < kUBinsPadded; e += nt) {
+    fh[e] = 0u;
+    fb_lo[e] = 0u;
+  }
+  for (int w = tid; w < nwords; w += nt) bm[w] = 0u;
+  if (tid == 0) {
+    ncand_s = min(__ldcg(rs + kRowNcand), (uint32_t)p.kv.max_len);
+    below_s = 0u;
+    slot_s = 0u;  // this chunk's band keys listed so far
+  }
+  constexpr int kRegCand = 16;
+  const uint32_t chunk_n = kRegCand * (uint32_t)nt;
+  // Loads of the first kRegCand x nt entries, issued before the count is known (entries
+  // past the count are ignored).
+  float rt[kRegCand];
+  int rj[kRegCand];
+  auto load_regs = [&](uint32_t c0) {
+#pragma unroll
+    for (int u = 0; u < kRegCand; ++u) {
+      const uint32_t e = c0 + (uint32_t)u * nt + tid;
+      const bool in = e < (uint32_t)p.kv.max_len;
+      rt[u] = in ? __ldcg(gct + e) : -INFINITY;
+      rj[u] = in ? __ldcg(gcj + e) : -1;
+    }
+  };
+  load_regs(0);
+  __syncthreads();
+  const uint32_t n = ncand_s;
+  const FineBins fb = fb_s;
+  auto add_hist = [&](uint32_t c0) {
+    uint32_t top = 0, bot = 0, top_lo = 0, bot_lo = 0;
+#pragma unroll
+    for (int u = 0; u < kRegCand; ++u) {
+      const uint32_t e = c0 + (uint32_t)u * nt + tid;
+      if (e >= n) continue;
+      const int bb = fb.bin(rt[u]);
+      const bool lo = rj[u] < k0;
+      if (bb == kUBins - 1) {
+        ++top;
+        top_lo += lo;
+      } else if (bb == 0) {
+        ++bot;
+        bot_lo += lo;
+      } else {
+        atomicAdd(&fh[ubin_slot(bb)], 1u);
+        if (lo) atomicAdd(&fb_lo[ubin_slot(bb)], 1u);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      top += __shfl_xor_sync(0xffffffffu, top, o);
+      bot += __shfl_xor_sync(0xffffffffu, bot, o);
+      top_lo += __shfl_xor_sync(0xffffffffu, top_lo, o);
+      bot_lo += __shfl_xor_sync(0xffffffffu, bot_lo, o);
+    }
+    if (lane == 0) {
+      if (top) atomicAdd(&fh[ubin_slot(kUBins - 1)], top);
+      if (bot) atomicAdd(&fh[ubin_slot(0)], bot);
+      if (top_lo) atomicAdd(&fb_lo[ubin_slot(kUBins - 1)], top_lo);
+      if (bot_lo) atomicAdd(&fb_lo[ubin_slot(0)], bot_lo);
+    }
+  };
+  add_hist(0);
+  for (uint32_t c0 = chunk_n; c0 < n; c0 += chunk_n) {  // long lists only
+    load_regs(c0);
+    add_hist(c0);
+  }
+  __syncthreads();
+  const int B = kth_bin_from_top(p.k_sel, fh);
+  const int mb = mb_s;
+  if (tid < 32) {
+    // Bins >= B + mb are in, bins [B - mb, B + mb) form the band: the totals, and the
+    // sure ones below this chunk.
+    uint32_t sure = 0, band = 0, sure_lo = 0;
+#pragma unroll 8
+    for (int e = lane; e < kUBins; e += 32) {
+      const uint32_t c = fh[ubin_slot(e)];
+      const bool in = e >= B + mb;
+      sure += in ? c : 0u;
+      band += (e >= B - mb && e < B + mb) ? c : 0u;
+      sure_lo += in ? fb_lo[ubin_slot(e)] : 0u;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sure += __shfl_xor_sync(0xffffffffu, sure, o);
+      band += __shfl_xor_sync(0xffffffffu, band, o);
+      sure_lo += __shfl_xor_sync(0xffffffffu, sure_lo, o);
+    }
+    if (lane == 0) {
+      sure_s = sure;
+      nband_s = band;
+      base_s = sure_lo;
+    }
+  }
+  __syncthreads();
+  const int need2 = p.k_sel - (int)sure_s;  // taken from the band: 1 <= need2 <= n_band
+  const int n_band = (int)nband_s;
+  const bool rank_band = need2 < n_band;
+  // This chunk's candidates: the sure ones into the bitmap; band keys listed for the
+  // float64 re-scoring (when every band key is taken they count as sure, below the chunk
+  // too).
+  auto classify = [&](uint32_t c0) {
+    uint32_t band_lo = 0;
+#pragma unroll
+    for (int u = 0; u < kRegCand; ++u) {
+      const uint32_t e = c0 + (uint32_t)u * nt + tid;
+      if (e >= n) continue;
+      const int bb = fb.bin(rt[u]);
+      const int j = rj[u];
+      const bool sure = bb >= B + mb;
+      const bool band = !sure && bb >= B - mb;
+      if (band && !rank_band && j < k0) ++band_lo;
+      if (j < k0 || j >= c_hi) continue;
+      if (sure || (band && !rank_band)) {
+        atomicOr(&bm[(j - k0) >> 5], 1u << ((j - k0) & 31));
+      } else if (band) {
+        const uint32_t slot = atomicAdd(&slot_s, 1u);
+        if (slot < own_cap) own_band[slot] = j;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) band_lo += __shfl_xor_sync(0xffffffffu, band_lo, o);
+    if (lane == 0 && band_lo) atomicAdd(&below_s, band_lo);
+  };
+  if (n <= chunk_n) {
+    classify(0);
+  } else {
+    for (uint32_t c0 = 0; c0 < n; c0 += chunk_n) {
+      load_regs(c0);
+      classify(c0);
+    }
+  }
+  __syncthreads();
+  if (rank_band) {
+    // This chunk's band keys: float64 keys (one warp each) appended to the row's band list.
+    const int nob = (int)min(slot_s, own_cap);
+    if (tid == 0 && slot_s > own_cap) set_status(p.status, HS2_ERR_UNSUPPORTED);
+    __shared__ uint32_t bbase_s;
+    if (tid == 0) bbase_s = nob ? atomicAdd(rs + kRowNBand, (uint32_t)nob) : 0u;
+    __syncthreads();
+    for (int e = warp; e < nob; e += nwarps) {
+      const int j = own_band[e];
+      const double v = rescore_f64<H, FP8>(p.kv, p.sm_scale, (size_t)b * p.kv.max_len + j, qv.base,
+                                           qv.hstride, qv.cstride, rl.dl, kf + warp * kHeadDim,
+                                           lane);
+      if (lane == 0) {
+        p.band_t[rowoff + bbase_s + e] = v;
+        p.band_j[rowoff + bbase_s + e] = j;
+      }
+    }
+    row_arrive(rs + kRowArrive3);
+    if (!row_wait(rs + kRowArrive3, (uint32_t)S)) ok = false;
+    // Every CTA ranks the whole band by (key desc, position asc): the top need2 are in.
+    const double* gbt = p.band_t + rowoff;
+    const int32_t* gbj = p.band_j + rowoff;
+    uint32_t band_lo = 0;
+    auto take_band = [&](int je) {
+      if (je < k0) ++band_lo;
+      else if (je < c_hi) atomicOr(&bm[(je - k0) >> 5], 1u << ((je - k0) & 31));
+    };
+    if (n_band <= kBandSmem) {
+      for (int e = tid; e < n_band; e += nt) {
+        bkey[e] = ordered_key64(__ldcg(gbt + e));
+        bpos[e] = __ldcg(gbj + e);
+      }
+      __syncthreads();
+      for (int e = tid; e < n_band; e += nt) {
+        const unsigned long long ke = bkey[e];
+        const int je = bpos[e];
+        int rank = 0;
+        for (int f = 0; f < n_band; ++f) {
+          const unsigned long long kf2 = bkey[f];
+          rank += (kf2 > ke) || (kf2 == ke && bpos[f] < je);
+        }
+        if (rank < need2) take_band(je);
+      }
+    } else {
+      // A large band (many equal keys): the boundary by radix select over the list.
+      __shared__ uint32_t gt_s;
+      const int nb = min(n_band, (int)p.kv.max_len);
+      const unsigned long long vb = block_kth_largest<unsigned long long, 64>(
+          nb, need2, [&](int e) { return ordered_key64(__ldcg(gbt + e)); },
+          [](int) { return true; }, &gt_s);
+      const int take_eq = need2 - (int)gt_s;
+      const uint32_t jb_inv = block_kth_largest<uint32_t, 32>(
+          nb, take_eq, [&](int e) { return ~(uint32_t)__ldcg(gbj + e); },
+          [&](int e) { return ordered_key64(__ldcg(gbt + e)) == vb; }, &gt_s);
+      const int jb = (int)~jb_inv;
+      for (int e = tid; e < nb; e += nt) {
+        const unsigned long long k = ordered_key64(__ldcg(gbt + e));
+        const int je = __ldcg(gbj + e);
+        if (k > vb || (k == vb && je <= jb)) take_band(je);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) band_lo += __shfl_xor_sync(0xffffffffu, band_lo, o);
+    if (lane == 0 && band_lo) atomicAdd(&below_s, band_lo);
+  }
+  __syncthreads();
+
+  // ---- 4. this chunk's positions in order, from the slot after the selected positions
+  // below the chunk
+  const int per = (nwords + nt - 1) / nt;
+  const int w0 = tid * per, w1 = min(w0 + per, nwords);
+  uint32_t cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
+  uint32_t incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  if (lane == 31) warp_cnt[warp] = incl;
+  __syncthreads();
+  uint32_t at = base_s + below_s + incl - cnt;
+  for (int k = 0; k < warp; ++k) at += warp_cnt[k];
+  for (int w = w0; w < w1; ++w) {
+    uint32_t bits = bm[w];
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      if (at < (uint32_t)p.k_sel) out_row[at] = k0 + w * 32 + bit;
+      ++at;
+    }
+  }
+  // The window and the padding after the k_sel selected positions.
+  if (split == 0)
+    for (int e = p.k_sel + tid; e < width; e += nt) {
+      const int v = n_c + (e - p.k_sel);
+      out_row[e] = v <= pos ? v : -1;
+    }
+  return ok;
+}
+
+// The whole tail (fuse 1 or 2), called by every thread of every CTA after the stream,
+// with the CTA's partial written and (fuse 2) its u histogram in `uhist_s`.  NW: warps of
+// the CTA.  The K/V stages (`stage`, `stage_bytes`) are idle; the first kTailTiles tiles
+// of `tile_bytes` take gathered K rows.  Returns false if a wait gave up.
+template <int H, bool FP8, int NW, typename Recompute>
+__device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, uint32_t stage_bytes,
+                                           uint32_t tile_bytes, const uint32_t* uhist_s, int bq,
+                                           int b, int split, int pos, int k0, int k1,
+                                           const QView& qv, Recompute&& recompute) {
+  __shared__ RowLse<H> rl;
+  const int S = p.splits1;
+  const int n_c = pos - p.window + 1;
+  const bool sel_row = p.fuse == 2 && n_c > p.k_sel;
+  const int width = p.window + p.k_sel;
+  uint32_t* rs = p.rowsync + (size_t)bq * 8;
+  uint32_t* gu = p.uhist + (size_t)bq * kHistBins;
+  const int c_hi = min(k1, n_c);
+  const int chunk_len = sel_row && c_hi > k0 ? c_hi - k0 : 0;
+  // Before the second barrier the stages hold: the gathered tiles, the row's u histogram,
+  // then this chunk's bounds (a piece at a time), its candidate positions and their keys.
+  const uint32_t tiles = kTailTiles * tile_bytes;
+  uint32_t* uh = reinterpret_cast<uint32_t*>(stage + tiles);
+  const uint32_t uoff = tiles + ((kUBinsPadded * 4u + 15u) & ~15u);
+  const int piece = (int)(((stage_bytes - uoff - kTailTiles * 128u * 4u) / 8u) & ~3u);
+  float* us = reinterpret_cast<float*>(stage + uoff);
+  int* cl = reinterpret_cast<int*>(stage + uoff + 4u * (uint32_t)piece);
+  float* t2s = reinterpret_cast<float*>(stage + uoff + 8u * (uint32_t)piece);
+  bool ok = true;
+  __syncthreads();
+  if (sel_row) {
+    // This chunk's first bounds on their way on chip (waited for after the barrier), and
+    // the bins at or above this CTA's own k_sel-th largest u published (the row's
+    // boundary bin is at least that high).
+    async_words(us, p.ubuf + (size_t)bq * p.ld_u + k0, min(piece, chunk_len));
+    const int low = kth_bin_from_top(p.k_sel, uhist_s);
+    add_bins(uhist_s, gu, low);
+  }
+  row_arrive(rs + kRowArrive1);
+  if (!row_wait(rs + kRowArrive1, (uint32_t)S)) ok = false;
+  if (sel_row) async_bins(uh, gu);  // in flight with the partials' loads of row_lse
+  row_lse<H>(p.part_ml + (size_t)bq * S * H * 2, S, rl);
+  if (p.fuse == 2 && !sel_row && split == 0)
+    write_all_positions(p.sel_idx + (size_t)bq * width, width, pos);
+  if (sel_row) {
+    sm100::cp_async_wait_all();
+    __syncthreads();
+    const int bk = kth_bin_from_top(p.k_sel, uh);
+    if (!row_select<H, FP8>(p, stage, stage_bytes, tile_bytes, us, cl, t2s, piece, bq, b, split,
+                            S, k0, c_hi, n_c, pos, bk, rl, qv, recompute))
+      ok = false;
+  }
+  // The index set is complete and visible: the next kernel (a sparse layer reads it
+  // without waiting for this grid to end) may start while this CTA merges its share.
+  sm100::fence_acq_rel_gpu();
+  __syncthreads();
+  griddep_launch_dependents();
+  row_merge<H>(p, bq, split, S, rl);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // The last CTA of the row to get here leaves the row's counters at zero.
+    __threadfence();
+    if (atomicAdd(rs + kRowDone, 1u) == (uint32_t)S - 1u) {
+      rs[kRowArrive1] = 0u;
+      rs[kRowArrive2] = 0u;
+      rs[kRowArrive3] = 0u;
+      rs[kRowNcand] = 0u;
+      rs[kRowNBand] = 0u;
+      rs[kRowDone] = 0u;
+      __threadfence();
+    }
+  }
+  return ok;
+}
+
+}  // namespace hs2

@@ -34,6 +34,7 @@
 #include "hs2_internal.cuh"
 #include "sm100.cuh"
 #include "tc_common.cuh"
+#include "decode_select.cuh"
 
 namespace hs2 {
 
@@ -58,10 +59,14 @@ struct Fp8Smem {
   static constexpr uint32_t kPBytes = 3 * H * kKeyTile;       // P_hi, P_lo, P_lo2
   static constexpr uint32_t kRedBytes = (4 * H + 8) * 4;      // [4 warps][H] + V-scale maxima
   static constexpr uint32_t kRefBytes = (2 * H + 8) * 4;      // mref, alpha, scalars
-  static constexpr uint32_t kMaxBars = 4 * 6 + 9;
-  // (+ 1024 for alignment, + 1024 for the static shared memory of the Q staging)
-  static constexpr uint32_t kFixed =
-      kQBytes + 2 * kPBytes + kRedBytes + kRefBytes + kMaxBars * 8 + 16 + 2048;
+  static constexpr uint32_t kMaxBars = 4 * 6 + 10;
+  // Full layer only: the histogram of the selection bounds u and the exchange of the two
+  // head halves' partial bounds ([2][128] floats).
+  static constexpr uint32_t kSelBytes = GATHER ? 0u : (uint32_t)kUBinsPadded * 4u + 2u * 128u * 4u;
+  // (+ 1024 for alignment, + 1024 for the static shared memory of the Q staging, + 7168
+  // for that of the fused tail)
+  static constexpr uint32_t kFixed = kQBytes + 2 * kPBytes + kRedBytes + kRefBytes +
+                                     kMaxBars * 8 + 16 + kSelBytes + 2048 + (GATHER ? 0 : 7168);
   // Raw stages (K and V each): as many as fit, up to six; gather mode keeps one (its
   // CTAs mostly take a single tile).
   static constexpr int kFit = (int)((227u * 1024u - kFixed) / (2 * kRawTile));
@@ -73,9 +78,11 @@ struct Fp8Smem {
   static constexpr uint32_t kRedOff = kPOff + 2 * kPBytes;
   static constexpr uint32_t kRefOff = kRedOff + kRedBytes;
   static constexpr uint32_t kBarOff = kRefOff + kRefBytes;
-  static constexpr uint32_t kBars = 4 * R + 9;
+  static constexpr uint32_t kBars = 4 * R + 10;
   static constexpr uint32_t kSlotOff = kBarOff + kBars * 8;
-  static constexpr uint32_t kBytes = kSlotOff + 16 + 1024;
+  static constexpr uint32_t kUHistOff = (kSlotOff + 16 + 15) / 16 * 16;  // 16-byte aligned
+  static constexpr uint32_t kUxOff = kUHistOff + (GATHER ? 0u : (uint32_t)kUBinsPadded * 4u);
+  static constexpr uint32_t kBytes = kUHistOff + kSelBytes + 1024;
   static constexpr uint32_t kTmemCols = tmem_cols_pow2(7 * H);  // S: 2 x 2H, O: 3H
   static_assert(R >= 1 && kBytes <= 227 * 1024, "shared memory budget");
   static_assert(kQOff + kQBytes >= kClusterMlOff + 2 * H * 4, "cluster partial fits");
@@ -127,10 +134,112 @@ __device__ __forceinline__ void block_max_group_f8(const float (&v)[HH], float* 
 
 }  // namespace
 
+// Fused tail of the full layer, as in the bf16 kernel (decode_select.cuh): a function of
+// its own whose indices are recomputed from the CTA's coordinates.  The candidates' E4M3 K
+// rows go through the stream's own kind::f8f6f4 MMA against [Q_hi | Q_lo] (S buffers of 2H
+// columns), and at 64 heads the two head halves combine their partial keys through ux_s.
+// The float64 re-scoring reads the bf16 query from global memory.
+template <int H>
+__device__ __noinline__ bool full_fp8_tail(const FullParams& p) {
+  using L = Fp8Smem<H, false>;
+  constexpr int R = L::R;
+  constexpr int NHALF = fp8_halves<H>();
+  constexpr int HH = H / NHALF;
+  constexpr int NSOFT = 128 * NHALF;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t k_addr = smem_u32(smem + L::kKRawOff);
+  const uint32_t q_addr = smem_u32(smem + L::kQOff);
+  const float* qsc_s = reinterpret_cast<const float*>(smem + L::kRefOff) + 2 * H;
+  uint64_t* post_bar = reinterpret_cast<uint64_t*>(smem + L::kBarOff) + 4 * R + 9;
+  const uint32_t* tmem_slot = reinterpret_cast<const uint32_t*>(smem + L::kSlotOff);
+  const uint32_t* uhist_s = reinterpret_cast<const uint32_t*>(smem + L::kUHistOff);
+  float* ux_s = reinterpret_cast<float*>(smem + L::kUxOff);
+  const int warp = threadIdx.x >> 5;
+  const int split = blockIdx.x, bq = blockIdx.y;
+  const int b = bq / p.n_q, qi = bq % p.n_q;
+  const int pos = seq_len(p.kv, b, p.n_q, p.status, false) - p.n_q + qi;
+  const int k0 = split * p.chunk1;
+  const int k1 = min(k0 + p.chunk1, pos + 1);
+  const size_t row_base = (size_t)b * p.kv.max_len;
+  const float c2 = p.sm_scale * kLog2eF8 * qsc_s[0];
+  auto recompute = [&](const int* list, int m, float* t2, uint32_t round, const float* D) -> bool {
+    bool rok = true;
+    const int ntile = (m + kKeyTile - 1) / kKeyTile;
+    for (int tl = 0; tl < ntile; ++tl)
+      gather_list_rows<8, kRawTile>(k_addr + tl * kRawTile, static_cast<const uint8_t*>(p.kv.k),
+                                    list + tl * kKeyTile, min(kKeyTile, m - tl * kKeyTile),
+                                    row_base, threadIdx.x, blockDim.x);
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    if (warp == 1) {
+      if (elect_one()) {
+        constexpr uint32_t id_qk = idesc_e4m3(128, 2 * H, false, false);
+        for (int tl = 0; tl < ntile; ++tl) {
+#pragma unroll
+          for (int kk = 0; kk < kHeadDim / 32; ++kk)
+            mma_e4m3_ss(tmem_base + tl * 2 * H, k_e4m3_desc(k_addr + tl * kRawTile, kk),
+                        q_e4m3_desc<2 * H>(q_addr, kk), id_qk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(post_bar);
+      }
+      __syncwarp();
+    } else if (warp >= 2) {
+      const int lg = warp & 3;
+      const int t = lg * 32 + (int)lane_id();
+      const int half = (warp - 2) >> 2;
+      const int hoff = half * HH;
+      const uint32_t lane_base = (uint32_t)(lg * 32) << 16;
+      if (!mbar_wait(post_bar, round & 1u)) rok = false;
+      tc_fence_after();
+      for (int tl = 0; tl < ntile; ++tl) {
+        uint32_t r[2 * HH];
+#pragma unroll
+        for (int c = 0; c < HH; c += 16) {
+          tmem_ld16(tmem_base + lane_base + tl * 2 * H + hoff + c,
+                    *reinterpret_cast<uint32_t(*)[16]>(r + c));
+          tmem_ld16(tmem_base + lane_base + tl * 2 * H + H + hoff + c,
+                    *reinterpret_cast<uint32_t(*)[16]>(r + HH + c));
+        }
+        tmem_wait_ld();
+        const int slot = tl * kKeyTile + t;
+        const int jj = slot < m ? list[slot] : -1;
+        const float cks = jj >= 0 ? c2 * __ldg(p.kv.k_scale + row_base + jj) : 0.f;
+        float v = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < HH; ++e)
+          v = fmaxf(v, fmaf(__uint_as_float(r[HH + e]), 0.0625f, __uint_as_float(r[e])) * cks -
+                           D[hoff + e]);
+        if (NHALF == 2) {
+          if (half == 1) ux_s[t] = v;
+          named_bar_sync(3, NSOFT);
+          if (half == 0) v = fmaxf(v, ux_s[t]);
+          named_bar_sync(3, NSOFT);  // ux_s is reused by the next tile
+        }
+        if (half == 0 && jj >= 0) t2[slot] = v;
+      }
+      tc_fence_before();
+    }
+    __syncthreads();
+    return rok;
+  };
+  QView qv;
+  qv.base = reinterpret_cast<const uint8_t*>(p.q + (size_t)bq * H * kHeadDim);
+  qv.hstride = kHeadDim * 2;  // bf16 rows [H][128] in global memory
+  qv.cstride = 16;
+  return fused_tail<H, true, fp8_threads<H>() / 32>(p, smem, 2u * R * kRawTile, kRawTile, uhist_s,
+                                                     bq, b, split, pos, k0, k1, qv, recompute);
+}
+
 template <int H, bool GATHER>
 __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     full_attn_fp8_kernel(const __grid_constant__ CUtensorMap tmap_k,
-                         const __grid_constant__ CUtensorMap tmap_v, FullParams p) {
+                         const __grid_constant__ CUtensorMap tmap_v,
+                         const __grid_constant__ FullParams p) {
   using L = Fp8Smem<H, GATHER>;
   constexpr int R = L::R;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -155,7 +264,10 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
   uint64_t* p_full = s_full + 4;    // [2]
   uint64_t* p_free = s_full + 6;    // [2]
   uint64_t* mma_done = s_full + 8;
+  uint64_t* post_bar = s_full + 9;  // MMAs of the selection tail
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
+  uint32_t* uhist_s = reinterpret_cast<uint32_t*>(smem + L::kUHistOff);
+  float* ux_s = reinterpret_cast<float*>(smem + L::kUxOff);  // [2][128]
 
   const int warp = threadIdx.x >> 5;
   const int split = blockIdx.x, bq = blockIdx.y;
@@ -178,8 +290,11 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
       beta_s[s] = 0.f;
     }
     mbar_init(mma_done, 1);
+    mbar_init(post_bar, 1);
     fence_mbar_init();
   }
+  if (!GATHER)
+    for (int e = threadIdx.x; e < kUBinsPadded; e += blockDim.x) uhist_s[e] = 0u;
   if (warp == 1) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
@@ -350,6 +465,19 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     const int hoff = half * HH;
     const uint32_t lane_base = (uint32_t)(lg * 32) << 16;
     const uint64_t keep_policy = policy_evict_last();
+    // Fused selection: keys [0, n_c) record their bound u_j = max_h x_hj and count it.  At
+    // 64 heads the two halves' partial maxima meet in ux_s one tile later (after the
+    // next tile's barrier 3), and half 0 records them.
+    const int n_c = pos - p.window + 1;
+    const bool sel_keys = !GATHER && p.fuse == 2 && n_c > p.k_sel;
+    float* urow = sel_keys ? p.ubuf + (size_t)bq * p.ld_u : nullptr;
+    float u_prev = -INFINITY;
+    int j_prev = 0;
+    bool rec_prev = false;
+    auto record_u = [&](int jj, float u) {
+      st_global_f32_hint(urow + jj, u, keep_policy);
+      atomicAdd(&uhist_s[ubin_slot(ubin(u))], 1u);
+    };
     // This group's references: in registers up to 16 heads per thread; above, read
     // from shared memory at each use (registers are the limit there).
     constexpr bool kRefRegs = HH <= 16;
@@ -427,6 +555,22 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
       const float cks = c2 * ks;  // one Q scale for every head: one multiplier per key
 #pragma unroll
       for (int e = 0; e < HH; ++e) x[e] = valid ? x[e] * cks : -INFINITY;
+      if (sel_keys) {
+        float u = x[0];
+#pragma unroll
+        for (int e = 1; e < HH; ++e) u = fmaxf(u, x[e]);
+        const bool rec = valid && j < n_c;
+        if (NHALF == 1) {
+          if (rec) record_u(j, u);
+        } else if (half == 1) {
+          ux_s[(i & 1) * 128 + t] = u;
+        } else {
+          if (rec_prev) record_u(j_prev, fmaxf(u_prev, ux_s[((i - 1) & 1) * 128 + t]));
+          u_prev = u;
+          j_prev = j;
+          rec_prev = rec;
+        }
+      }
       bool over = valid && fabsf(vs) > vlim;
 #pragma unroll
       for (int h = 0; h < HH; ++h) over |= x[h] - ref(h) > kRescaleAtF8;
@@ -535,7 +679,14 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
       fence_proxy_async_smem();
       mbar_arrive(p_full + sb);
     }
-    griddep_launch_dependents();  // the merge may be scheduled; it waits for this grid
+    if (NHALF == 2 && sel_keys) {
+      named_bar_sync(3, NSOFT);
+      if (half == 0 && rec_prev)
+        record_u(j_prev, fmaxf(u_prev, ux_s[((n_tiles - 1) & 1) * 128 + t]));
+    }
+    // The merge kernel may be scheduled (it waits for this grid); with the fused tail the
+    // next kernel starts only once the index set is written.
+    if (GATHER || !p.fuse) griddep_launch_dependents();
     const int last = n_tiles - 1;
     if (ok && !mbar_wait(p_free + (last & 1), (last >> 1) & 1)) ok = false;
     tc_fence_after();
@@ -579,6 +730,9 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     __syncwarp();
     cluster_sync();
   }
+  if constexpr (!GATHER) {
+    if (p.fuse && !full_fp8_tail<H>(p)) set_status(p.status, HS2_ERR_DEVICE_TIMEOUT);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -601,8 +755,8 @@ static cudaError_t launch_fp8_t(FullParams p, const CUtensorMap& tk, const CUten
     if (max_cluster < 1) return cudaErrorLaunchOutOfResources;
   }
   if (!GATHER)
-    return launch_pdl(kernel, dim3(p.splits1, bq), dim3(fp8_threads<H>()), L::kBytes, st, tk, tv,
-                      p);
+    return launch_pdl_coop(kernel, dim3(p.splits1, bq), dim3(fp8_threads<H>()), L::kBytes,
+                           p.fuse != 0 && p.splits1 > 1, st, tk, tv, p);
   plan_gather_cluster(p.idx_width, max_cluster, &p.splits1, &p.chunk1);
   return launch_pdl_cluster(kernel, dim3(p.splits1, bq), dim3(fp8_threads<H>()), L::kBytes, p.splits1,
                             st, tk, tv, p);

@@ -26,6 +26,7 @@
 #include "hs2_internal.cuh"
 #include "sm100.cuh"
 #include "tc_common.cuh"
+#include "decode_select.cuh"
 
 namespace hs2 {
 
@@ -49,9 +50,12 @@ struct FullSmem {
   static constexpr uint32_t kRedOff = kPOff + 4 * kPBytes;  // [4 warps][H] floats
   static constexpr uint32_t kRefOff = kRedOff + 4 * H * 4;  // [H] reference, [H] alpha
   static constexpr uint32_t kBarOff = kRefOff + 2 * H * 4;
-  static constexpr uint32_t kBars = 4 * kStages + 9;
+  static constexpr uint32_t kBars = 4 * kStages + 10;
   static constexpr uint32_t kSlotOff = kBarOff + kBars * 8;
-  static constexpr uint32_t kBytes = kSlotOff + 16 + 1024;
+  // Histogram of the selection bounds u (full layer only).
+  static constexpr uint32_t kUHistOff = (kSlotOff + 16 + 15) / 16 * 16;  // 16-byte aligned
+  static constexpr uint32_t kUHistBytes = GATHER ? 0u : (uint32_t)kUBinsPadded * 4u;
+  static constexpr uint32_t kBytes = kUHistOff + kUHistBytes + 1024;
   static constexpr uint32_t kTmemCols = tmem_cols_pow2(3 * H);
   static_assert(kBytes <= 227 * 1024, "shared memory budget");
 };
@@ -71,10 +75,95 @@ __device__ __forceinline__ void block_max_heads(const float (&v)[H], float* red,
   named_bar_sync(1, 128);
 }
 
+// Fused tail of the full layer (decode_select.cuh): the CTAs of a row merge their
+// partials and (fuse 2) select the row's tokens, in the K/V stages, idle by now.  A
+// function of its own, called after the stream: every index is recomputed here from the
+// CTA's coordinates and the parameters, so that nothing stays live in registers across
+// the stream for it.  Candidates' K rows are gathered into the first stages and go through
+// the stream's S^T = K . Q^T MMA (S buffers at TMEM columns [tile H, tile H + H)).
+template <int H>
+__device__ __noinline__ bool full_tc_tail(const FullParams& p) {
+  using L = FullSmem<H, false>;
+  constexpr int NS = L::kStages;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t k_addr = smem_u32(smem + L::kKOff);
+  const uint8_t* qs = smem + L::kQOff;
+  const uint32_t q_addr = smem_u32(qs);
+  uint64_t* post_bar = reinterpret_cast<uint64_t*>(smem + L::kBarOff) + 4 * NS + 9;
+  const uint32_t* tmem_slot = reinterpret_cast<const uint32_t*>(smem + L::kSlotOff);
+  const uint32_t* uhist_s = reinterpret_cast<const uint32_t*>(smem + L::kUHistOff);
+  const int warp = threadIdx.x >> 5;
+  const int split = blockIdx.x, bq = blockIdx.y;
+  const int b = bq / p.n_q, qi = bq % p.n_q;
+  const int pos = seq_len(p.kv, b, p.n_q, p.status, false) - p.n_q + qi;
+  const int k0 = split * p.chunk1;
+  const int k1 = min(k0 + p.chunk1, pos + 1);
+  const size_t row_base = (size_t)b * p.kv.max_len;
+  const float c2 = p.sm_scale * kLog2e;
+  auto recompute = [&](const int* list, int m, float* t2, uint32_t round, const float* D) -> bool {
+    bool rok = true;
+    const int ntile = (m + kKeyTile - 1) / kKeyTile;
+    for (int tl = 0; tl < ntile; ++tl)
+      gather_list_rows<16, kBoxBytes>(k_addr + tl * L::kTile, static_cast<const uint8_t*>(p.kv.k),
+                                      list + tl * kKeyTile, min(kKeyTile, m - tl * kKeyTile),
+                                      row_base, threadIdx.x, blockDim.x);
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    if (warp == 1) {
+      if (elect_one()) {
+        const uint32_t id_qk = idesc_f16(128, H, true, false, false);
+        for (int tl = 0; tl < ntile; ++tl) {
+#pragma unroll
+          for (int kk = 0; kk < kHeadDim / 16; ++kk)
+            mma_f16_ss(tmem_base + tl * H, kmajor_sw128_desc(k_addr + tl * L::kTile, kk),
+                       q_kmajor_desc<H>(q_addr, kk), id_qk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(post_bar);
+      }
+      __syncwarp();
+    } else if (warp >= 2) {
+      const int lg = warp & 3;
+      const int t = lg * 32 + (int)lane_id();
+      const uint32_t lane_base = (uint32_t)(lg * 32) << 16;
+      if (!mbar_wait(post_bar, round & 1u)) rok = false;
+      tc_fence_after();
+      for (int tl = 0; tl < ntile; ++tl) {
+        uint32_t r[H];
+#pragma unroll
+        for (int c = 0; c < H; c += 16)
+          tmem_ld16(tmem_base + lane_base + tl * H + c, *reinterpret_cast<uint32_t(*)[16]>(r + c));
+        tmem_wait_ld();
+        const int slot = tl * kKeyTile + t;
+        if (slot < m) {
+          float v = -INFINITY;
+#pragma unroll
+          for (int h = 0; h < H; ++h) v = fmaxf(v, __uint_as_float(r[h]) * c2 - D[h]);
+          t2[slot] = v;
+        }
+      }
+      tc_fence_before();
+    }
+    __syncthreads();
+    return rok;
+  };
+  QView qv;
+  qv.base = qs;         // Q as the MMA's K-major operand: chunk c of head h at
+  qv.hstride = 16;      // c * H * 16 + h * 16
+  qv.cstride = H * 16;
+  return fused_tail<H, false, 6>(p, smem, 2u * NS * L::kTile, L::kTile, uhist_s, bq, b, split, pos,
+                                 k0, k1, qv, recompute);
+}
+
 template <int H, bool GATHER>
 __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
     full_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
-                        const __grid_constant__ CUtensorMap tmap_v, FullParams p) {
+                        const __grid_constant__ CUtensorMap tmap_v,
+                        const __grid_constant__ FullParams p) {
   using L = FullSmem<H, GATHER>;
   constexpr int NS = L::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -96,7 +185,9 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
   uint64_t* p_full = s_full + 4;         // [2]
   uint64_t* p_free = s_full + 6;         // [2]
   uint64_t* mma_done = s_full + 8;
+  uint64_t* post_bar = s_full + 9;  // MMAs of the selection tail
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
+  uint32_t* uhist_s = reinterpret_cast<uint32_t*>(smem + L::kUHistOff);
 
   const int warp = threadIdx.x >> 5;
   const int split = blockIdx.x, bq = blockIdx.y;
@@ -117,8 +208,11 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
       mbar_init(p_free + s, 1);
     }
     mbar_init(mma_done, 1);
+    mbar_init(post_bar, 1);
     fence_mbar_init();
   }
+  if (!GATHER)
+    for (int e = threadIdx.x; e < kUBinsPadded; e += blockDim.x) uhist_s[e] = 0u;
   if (warp == 1) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
@@ -289,6 +383,10 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
       const uint32_t lane_base = (uint32_t)(lg * 32) << 16;
       const float c2 = p.sm_scale * kLog2e;
       const uint64_t keep_policy = policy_evict_last();
+      // Fused selection: keys [0, n_c) record their bound u_j = max_h x_hj and count it.
+      const int n_c = pos - p.window + 1;
+      const bool sel_keys = !GATHER && p.fuse == 2 && n_c > p.k_sel;
+      float* urow = sel_keys ? p.ubuf + (size_t)bq * p.ld_u : nullptr;
       float l[H];
 #pragma unroll
       for (int h = 0; h < H; ++h) l[h] = 0.f;
@@ -329,6 +427,13 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
         mbar_arrive(s_free + sb);
         const int j = k0 + i * kKeyTile + t;
         bool valid = j < k1;
+        if (sel_keys && valid && j < n_c) {
+          float u = x[0];
+#pragma unroll
+          for (int h = 1; h < H; ++h) u = fmaxf(u, x[h]);
+          st_global_f32_hint(urow + j, u, keep_policy);
+          atomicAdd(&uhist_s[ubin_slot(ubin(u))], 1u);
+        }
         if (GATHER && valid) {
           const int pj = __ldcg(idx_row + j);
           valid = pj >= 0 && pj < Lb;
@@ -407,7 +512,9 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
         fence_proxy_async_smem();
         mbar_arrive(p_full + sb);
       }
-      griddep_launch_dependents();  // the merge may be scheduled; it waits for this grid
+      // The merge kernel may be scheduled (it waits for this grid); with the fused tail the
+      // next kernel starts only once the index set is written.
+      if (GATHER || !p.fuse) griddep_launch_dependents();
       // Epilogue: O^T row t is dimension t of every head; l is reduced across threads.
       const int last = n_tiles - 1;
       if (ok && !mbar_wait(p_free + (last & 1), (last >> 1) & 1)) ok = false;
@@ -444,6 +551,9 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
     __syncwarp();
     cluster_sync();
   }
+  if constexpr (!GATHER) {
+    if (p.fuse && !full_tc_tail<H>(p)) set_status(p.status, HS2_ERR_DEVICE_TIMEOUT);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -465,7 +575,9 @@ static cudaError_t launch_full_tc_t(FullParams p, const CUtensorMap& tk, const C
     max_cluster = GATHER ? largest_cluster(kernel, dim3(192), L::kBytes) : 1;
     if (max_cluster < 1) return cudaErrorLaunchOutOfResources;
   }
-  if (!GATHER) return launch_pdl(kernel, dim3(p.splits1, bq), dim3(192), L::kBytes, st, tk, tv, p);
+  if (!GATHER)
+    return launch_pdl_coop(kernel, dim3(p.splits1, bq), dim3(192), L::kBytes,
+                           p.fuse != 0 && p.splits1 > 1, st, tk, tv, p);
   plan_gather_cluster(p.idx_width, max_cluster, &p.splits1, &p.chunk1);
   return launch_pdl_cluster(kernel, dim3(p.splits1, bq), dim3(192), L::kBytes, p.splits1, st, tk,
                             tv, p);

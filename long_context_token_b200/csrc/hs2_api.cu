@@ -78,10 +78,15 @@ bool make_layout(int batch, int n_q, int h, int max_len, int window, int k_sel, 
   w.use_sbuf = sbuf_eligible(n_q, h, dtype);
   w.sbuf = take(w.use_sbuf ? bq * ml * hh * sizeof(float) : 0);
   w.direct = take(bq * (size_t)k_sel * sizeof(int32_t));
-  w.cand_t = take(bq * ml * sizeof(float));
-  w.cand_j = take(bq * ml * sizeof(int32_t));
+  // (rows of ld_u entries for the fused tail, whose 16-byte copies need aligned rows)
+  const size_t ld_u = (ml + 31) / 32 * 32;
+  w.cand_t = take(bq * ld_u * sizeof(float));
+  w.cand_j = take(bq * ld_u * sizeof(int32_t));
   w.band_t = take(bq * ml * sizeof(double));
   w.band_j = take(bq * ml * sizeof(int32_t));
+  w.ld_u = (max_len + 31) / 32 * 32;
+  w.ubuf = take(bq * (size_t)w.ld_u * sizeof(float));
+  w.rowcnt = take(bq * (size_t)kSmCountBound * sizeof(uint32_t));
   w.total = off;
   *L = w;
   return true;
@@ -157,6 +162,7 @@ static void plan_decode_splits(const hs2_kv* kv, int n_q, const WsLayout& w, int
   const int bq = kv->batch * n_q;
   int splits = device_sm_count() / bq;
   if (splits > w.splits1) splits = w.splits1;
+  if (splits > kSmCountBound) splits = kSmCountBound;  // the fused tail's per-row bound
   if (splits < 1) splits = 1;
   int chunk = (kv->max_len + splits - 1) / splits;
   chunk = (chunk + 127) / 128 * 128;
@@ -164,9 +170,19 @@ static void plan_decode_splits(const hs2_kv* kv, int n_q, const WsLayout& w, int
   *chunk_out = chunk;
 }
 
+// Shapes whose full layer runs on the one-token tensor-core kernels, which merge their
+// split partials themselves and can select the row's tokens in the same launch.
+static bool fused_full_layer(const hs2_kv* kv, int n_q, int h) {
+  if (kv->dtype == HS2_KV_BF16) return h <= 64 && !mq_eligible(n_q, h);
+  return h <= 64;  // FP8: the E4M3 tensor-core kernel for any number of tokens
+}
+
+// The full layer.  On the fused shapes (fused_full_layer) the kernel merges its split
+// partials itself and, with `idx` non-null, also writes the token selection (then
+// run_select must not follow); elsewhere the split merge follows as its own kernel.
 static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int window,
                            int k_sel, float sm_scale, float* out, float* lse, void* ws,
-                           const WsLayout& w, cudaStream_t s) {
+                           const WsLayout& w, cudaStream_t s, int32_t* idx = nullptr) {
   FullParams p;
   p.q = static_cast<const uint16_t*>(q);
   p.kv = view_of(kv);
@@ -180,6 +196,22 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
   p.part_o = ws_ptr<float>(ws, w.part1_o);
   p.part_ml = ws_ptr<float>(ws, w.part1_ml);
   p.status = ws_ptr<uint32_t>(ws, w.status);
+  if (fused_full_layer(kv, n_q, h)) {
+    p.fuse = idx ? 2 : 1;
+    p.out = out;
+    p.lse_out = lse;
+    p.lse64 = ws_ptr<double>(ws, w.lse64);
+    p.ubuf = ws_ptr<float>(ws, w.ubuf);
+    p.ld_u = w.ld_u;
+    p.uhist = ws_ptr<uint32_t>(ws, w.hist);
+    p.rowsync = ws_ptr<uint32_t>(ws, w.counters);
+    p.cand_t = ws_ptr<float>(ws, w.cand_t);
+    p.cand_j = ws_ptr<int32_t>(ws, w.cand_j);
+    p.band_t = ws_ptr<double>(ws, w.band_t);
+    p.band_j = ws_ptr<int32_t>(ws, w.band_j);
+    p.rowcnt = ws_ptr<uint32_t>(ws, w.rowcnt);
+    p.sel_idx = idx;
+  }
   bool log2_partials = false;
   cudaError_t e;
   if (kv->dtype == HS2_KV_FP8_E4M3 && h <= 64) {
@@ -193,8 +225,11 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
       return cuda_fail(cudaErrorInvalidValue, "tensor maps of K/V");
     const int bq = kv->batch * n_q;
     plan_decode_splits(kv, n_q, w, &p.splits1, &p.chunk1);
-    p.sbuf = w.use_sbuf ? ws_ptr<float>(ws, w.sbuf) : nullptr;
+    // The stored logits serve a separate hs2_select call only.
+    p.sbuf = w.use_sbuf && p.fuse != 2 ? ws_ptr<float>(ws, w.sbuf) : nullptr;
     e = launch_full_attn_fp8(p, tk, tv, bq, s);
+    if (e != cudaSuccess) return cuda_fail(e, "full-attention launch");
+    if (p.fuse) return HS2_OK;
     log2_partials = true;
   } else if (kv->dtype == HS2_KV_BF16 && mq_eligible(n_q, h)) {
     // Several new tokens (or 128 heads): 128 query rows of one sequence per CTA, so
@@ -228,8 +263,11 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
       return cuda_fail(cudaErrorInvalidValue, "tensor maps of K/V");
     const int bq = kv->batch * n_q;
     plan_decode_splits(kv, n_q, w, &p.splits1, &p.chunk1);
-    p.sbuf = w.use_sbuf ? ws_ptr<float>(ws, w.sbuf) : nullptr;
+    // The stored logits serve a separate hs2_select call only.
+    p.sbuf = w.use_sbuf && p.fuse != 2 ? ws_ptr<float>(ws, w.sbuf) : nullptr;
     e = launch_full_attn_tc(p, tk, tv, bq, s);
+    if (e != cudaSuccess) return cuda_fail(e, "full-attention launch");
+    if (p.fuse) return HS2_OK;
     log2_partials = true;
   } else {
     e = launch_full_attn(p, kv->batch, s);
@@ -434,6 +472,9 @@ hs2_status hs2_full_attn_select(const void* q, int n_q, int h_q, const hs2_kv* k
   hs2_status st = prepare(q, n_q, h_q, kv, window, k_sel, workspace, ws_bytes, &P);
   if (st != HS2_OK) return st;
   if (!out || !aligned16(out) || !idx) return HS2_ERR_INVALID_ARGUMENT;
+  if (fused_full_layer(kv, n_q, h_q))  // one launch: full layer, merge and selection
+    return run_full(q, n_q, h_q, kv, window, k_sel, sm_scale, out, lse, workspace, P.w,
+                    (cudaStream_t)stream, idx);
   st = run_full(q, n_q, h_q, kv, window, k_sel, sm_scale, out, lse, workspace, P.w,
                 (cudaStream_t)stream);
   if (st != HS2_OK) return st;
@@ -577,6 +618,15 @@ const char* hs2_status_string(hs2_status s) {
 }
 
 const char* hs2_last_cuda_error(void) { return g_last_cuda_error; }
+
+int hs2_select_fused(int n_q, int h_q, int dtype) {
+  hs2_kv kv;
+  memset(&kv, 0, sizeof(kv));
+  kv.dtype = dtype;
+  if (dtype != HS2_KV_BF16 && dtype != HS2_KV_FP8_E4M3) return 0;
+  if (n_q < 1 || n_q > kMaxNq || h_q < 16 || h_q > kMaxHeads || h_q % 16 != 0) return 0;
+  return fused_full_layer(&kv, n_q, h_q) ? 1 : 0;
+}
 
 int hs2_abi_version(void) { return HS2_ABI_VERSION; }
 

@@ -41,10 +41,13 @@ struct WsLayout {
   size_t sbuf = 0;        // f32 [bq][max_len][h] raw logits (0 bytes when not used)
   bool use_sbuf = false;
   size_t direct = 0;      // i32 [bq][k_sel]
-  size_t cand_t = 0;      // f32 [bq][max_len]
-  size_t cand_j = 0;      // i32 [bq][max_len]
+  size_t cand_t = 0;      // f32 [bq][max_len rounded up to 32]
+  size_t cand_j = 0;      // i32 [bq][max_len rounded up to 32]
   size_t band_t = 0;      // f64 [bq][max_len]
   size_t band_j = 0;      // i32 [bq][max_len]
+  size_t ubuf = 0;        // f32 [bq][ld_u] per-key selection bounds of the fused tail
+  size_t rowcnt = 0;      // u32 [bq][kSmCountBound] per-CTA counts of the fused tail
+  int ld_u = 0;           // max_len rounded up to 32
   size_t part4_o = 0;     // f32 [bq][splits4][h][128]
   size_t part4_ml = 0;    // f32 [bq][splits4][h][2]
   size_t total = 0;
@@ -89,7 +92,25 @@ struct FullParams {
   // Gather mode only: if set, the splits1 CTAs of one row form a thread-block cluster,
   // merge their partials through distributed shared memory and write the normalised
   // output [bq][h][128] here (part_o / part_ml are then unused).
+  // Full layer with a fused tail (fuse >= 1): the merged output [bq][h][128].
   float* out = nullptr;
+  // Fused tail of the one-token tensor-core full layer (not gather mode):
+  //   fuse 1: the CTAs of a row merge their split partials themselves into out, lse_out
+  //           and lse64 (no separate merge kernel);
+  //   fuse 2: the same, plus the token selection of the row into sel_idx.
+  int fuse = 0;
+  float* lse_out = nullptr;      // [bq][h] or null
+  double* lse64 = nullptr;       // [bq][h]
+  float* ubuf = nullptr;         // [bq][ld_u]: per-key bound u_j = max_h x_hj (log2 units)
+  int ld_u = 0;
+  uint32_t* uhist = nullptr;     // [bq][kHistBins] (the first kUBins bins used)
+  uint32_t* rowsync = nullptr;   // [bq][8]: arrival counters and the candidate count
+  float* cand_t = nullptr;       // [bq][ld_u] the row's candidate list: keys ...
+  int32_t* cand_j = nullptr;     // [bq][ld_u] ... and positions
+  double* band_t = nullptr;      // [bq][max_len] the row's band list: float64 keys ...
+  int32_t* band_j = nullptr;     // [bq][max_len] ... and positions
+  uint32_t* rowcnt = nullptr;    // [bq][kSmCountBound] sure selections per CTA of a row
+  int32_t* sel_idx = nullptr;    // [bq][window + k_sel]
 };
 
 // Split merge (full layer: log2-domain partials; sparse layers: natural-log ones).
@@ -171,6 +192,26 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
+// The same, optionally as a cooperative launch (every CTA resident at once), for the
+// kernels whose CTAs of one row wait for one another.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl_coop(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                   bool cooperative, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = cooperative ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
 }
 

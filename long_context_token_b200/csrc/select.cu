@@ -21,6 +21,7 @@
 // eps = 1e-3 * max(1, |bin edges| + max_h delta_h).
 #include "tile_simt.cuh"
 #include "sm100.cuh"
+#include "select_common.cuh"
 
 namespace hs2 {
 
@@ -427,67 +428,6 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(SelectParams p
 }
 
 // ----------------------------------------------------------------------------
-// float64 selection key of one position, by one warp: max_h(sm_scale * q_h . k_j -
-// delta_h) from the stored inputs (K row widened exactly to float64 in the warp's
-// shared row kd -- FP8: code x scale -- then each lane takes heads lane, lane + 32, ...;
-// for H < 32 the lanes split each head's dot product into 32 / H parts, lane = part *
-// H + head).  q: the query's bf16 rows [H][kQLd] in shared memory; dlt: the float64
-// shifts.  Every lane returns the key.
-// ----------------------------------------------------------------------------
-constexpr int kQLd = kHeadDim + 8;  // padded q row (bf16) in shared memory
-
-template <int H, bool FP8>
-__device__ __forceinline__ double rescore_f64(const SelectParams& p, size_t row,
-                                              const uint16_t* qsm, const double* dlt,
-                                              double* kd, int lane) {
-  constexpr int kParts = H < 32 ? 32 / H : 1;
-  constexpr int kSpan = kHeadDim / kParts;
-  const int part = kParts > 1 ? lane / H : 0;
-  if (FP8) {
-    const uint32_t w4 = __ldg(reinterpret_cast<const uint32_t*>(
-                                  static_cast<const uint8_t*>(p.kv.k) + row * kHeadDim) + lane);
-    const double ksc = (double)__ldg(p.kv.k_scale + row);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) kd[4 * lane + u] = e4m3_to_f64((w4 >> (8 * u)) & 0xffu) * ksc;
-  } else {
-    const uint2 w4 = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.kv.k) +
-                                                          row * kHeadDim) + lane);
-    kd[4 * lane] = (double)bf16_bits_to_f32(w4.x & 0xffffu);
-    kd[4 * lane + 1] = (double)bf16_bits_to_f32(w4.x >> 16);
-    kd[4 * lane + 2] = (double)bf16_bits_to_f32(w4.y & 0xffffu);
-    kd[4 * lane + 3] = (double)bf16_bits_to_f32(w4.y >> 16);
-  }
-  __syncwarp();
-  const double scale = (double)p.sm_scale;
-  double best = -INFINITY;
-  for (int h0 = 0; h0 < H; h0 += 32 / kParts) {
-    const int h = h0 + (kParts > 1 ? lane % H : lane);
-    double dot = 0.0;
-    if (h < H) {
-      const uint16_t* qh = qsm + h * kQLd;
-#pragma unroll 4
-      for (int c = part * kSpan; c < (part + 1) * kSpan; c += 8) {
-        const uint4 qv = *reinterpret_cast<const uint4*>(qh + c);
-        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          dot = fma((double)bf16_bits_to_f32(qw[u] & 0xffffu), kd[c + 2 * u], dot);
-          dot = fma((double)bf16_bits_to_f32(qw[u] >> 16), kd[c + 2 * u + 1], dot);
-        }
-      }
-    }
-#pragma unroll
-    for (int o = 16; o >= 32 / kParts && kParts > 1; o >>= 1)
-      dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    if (h < H) best = fmax(best, scale * dot - dlt[h]);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) best = fmax(best, __shfl_xor_sync(0xffffffffu, best, o));
-  __syncwarp();  // the warp's next position reuses kd
-  return best;
-}
-
-// ----------------------------------------------------------------------------
 // 3. finish: exact select + float64 refinement + window merge + sort
 // ----------------------------------------------------------------------------
 constexpr int kFinThreads = 1024;
@@ -505,109 +445,6 @@ __host__ __device__ constexpr size_t finish_dyn_smem(int H) {
          (size_t)(kFinThreads / 32) * kHeadDim * sizeof(double);
 }
 
-// Warp-aggregated append to a shared-memory counter: one atomic per warp; returns the
-// lane's slot (only meaningful where pred holds).
-__device__ __forceinline__ uint32_t warp_slot(bool pred, uint32_t* counter) {
-  const unsigned m = __ballot_sync(0xffffffffu, pred);
-  const int lane = threadIdx.x & 31;
-  uint32_t base = 0;
-  if (m) {
-    const int leader = __ffs(m) - 1;
-    if (lane == leader) base = atomicAdd(counter, (uint32_t)__popc(m));
-    base = __shfl_sync(0xffffffffu, base, leader);
-  }
-  return base + __popc(m & ((1u << lane) - 1u));
-}
-
-// Radix select over the elements e in [0, n) with pred(e): the r-th largest
-// (1-based) of key(e), a KeyT of KBITS bits, 8 bits per pass.  Returns the key;
-// *n_gt receives how many selected elements are strictly greater.  Each pass builds a
-// 256-bin shared histogram of the current digit, then warp 0 finds the digit holding
-// the r-th element with a warp-wide prefix sum (lane l owns digits 255-8l .. 248-8l).
-// Keys known to lie in [lo, hi] share the bits above the highest bit where lo and hi
-// differ: those digits are skipped (pass lo = 0, hi = all ones when nothing is known).
-template <typename KeyT, int KBITS, typename KeyFn, typename PredFn>
-__device__ KeyT block_kth_largest(int n, int r, KeyFn key, PredFn pred, uint32_t* n_gt,
-                                  KeyT lo = KeyT(0), KeyT hi = ~KeyT(0)) {
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t sh_digit, sh_rem, sh_gt;
-  const KeyT diff = lo ^ hi;
-  if (diff == 0) {  // every key equals lo
-    if (threadIdx.x == 0) *n_gt = 0u;
-    __syncthreads();
-    return lo;
-  }
-  int top = KBITS - 1;
-  while (!((diff >> top) & 1)) --top;
-  const int start = (top / 8) * 8;  // lowest bit of the highest digit that varies
-  KeyT mask = start + 8 >= KBITS ? KeyT(0) : ~((KeyT(1) << (start + 8)) - 1);
-  KeyT prefix = lo & mask;
-  uint32_t rem = (uint32_t)r, gt = 0;
-  for (int shift = start; shift >= 0; shift -= 8) {
-    for (int e = threadIdx.x; e < 256; e += blockDim.x) hist[e] = 0u;
-    if (threadIdx.x == 0) {
-      sh_digit = 0u;
-      sh_rem = rem;
-      sh_gt = 0u;
-    }
-    __syncthreads();
-    // Keys of one pass share most of their digits (the candidates come from one bin),
-    // so lanes with the same digit are combined first: one shared atomic per distinct
-    // digit per warp instead of one per key on the same address.
-    const int n_r = (n + 31) & ~31;  // whole warps take part in the match
-    for (int e = threadIdx.x; e < n_r; e += blockDim.x) {
-      bool take = false;
-      uint32_t digit = 0;
-      if (e < n && pred(e)) {
-        const KeyT k = key(e);
-        take = (k & mask) == prefix;
-        digit = (uint32_t)(k >> shift) & 255u;
-      }
-      const uint32_t tag = take ? digit : 256u;
-      const unsigned same = __match_any_sync(0xffffffffu, tag);
-      if (take && (threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&hist[digit], __popc(same));
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      const int lane = threadIdx.x;
-      uint32_t c[8], s = 0;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        c[u] = hist[255 - 8 * lane - u];
-        s += c[u];
-      }
-      uint32_t incl = s;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const uint32_t excl = incl - s;
-      if (excl < rem && rem <= incl) {
-        uint32_t cum = excl;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          if (cum + c[u] >= rem) {
-            sh_digit = (uint32_t)(255 - 8 * lane - u);
-            sh_rem = rem - cum;
-            sh_gt = cum;
-            break;
-          }
-          cum += c[u];
-        }
-      }
-    }
-    __syncthreads();
-    prefix |= (KeyT)sh_digit << shift;
-    mask |= (KeyT)255 << shift;
-    rem = sh_rem;
-    gt += sh_gt;
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) *n_gt = gt;
-  __syncthreads();
-  return prefix;
-}
 
 template <int H, bool FP8>
 __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams p) {
@@ -623,7 +460,7 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
   uint16_t* qsm = reinterpret_cast<uint16_t*>(fin_dyn);  // [H][kQLd] bf16 q of this query
   float* cts = reinterpret_cast<float*>(fin_dyn + (size_t)H * kQLd * sizeof(uint16_t));
   int* cjs = reinterpret_cast<int*>(cts + kCandSmem);
-  double* kdsm = reinterpret_cast<double*>(cjs + kCandSmem);  // [warps][128] widened K rows
+  float* kdsm = reinterpret_cast<float*>(cjs + kCandSmem);  // [warps][128] widened K rows
   __shared__ double dlt[H];
   griddep_wait();
   const int bq = blockIdx.x;
@@ -730,11 +567,12 @@ __global__ void __launch_bounds__(kFinThreads) select_finish_kernel(SelectParams
   if (need2 > 0) {
     // float64 re-scoring of the band, one warp per key.
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    double* kd = kdsm + warp * kHeadDim;
+    float* kd = kdsm + warp * kHeadDim;
     for (int e = warp; e < n_band; e += blockDim.x / 32) {
       const int j = band_smem ? band_js[e] : __ldcg(bj + e);
       const double best =
-          rescore_f64<H, FP8>(p, (size_t)b * p.kv.max_len + j, qsm, dlt, kd, lane);
+          rescore_f64<H, FP8>(p.kv, p.sm_scale, (size_t)b * p.kv.max_len + j,
+                              reinterpret_cast<const uint8_t*>(qsm), kQLd * 2, 16, dlt, kd, lane);
       if (lane == 0) {
         if (band_smem) band_ts[e] = best;
         else bt[e] = best;
@@ -900,8 +738,9 @@ template <int H, bool FP8>
 __global__ void __launch_bounds__(kBlkThreads) select_blocks_kernel(SelectParams p) {
   extern __shared__ __align__(16) unsigned char blk_dyn[];
   uint16_t* qsm = reinterpret_cast<uint16_t*>(blk_dyn);  // [H][kQLd] bf16 q of this query
-  double* kdsm = reinterpret_cast<double*>(blk_dyn + (size_t)H * kQLd * sizeof(uint16_t));
-  float* bkey = reinterpret_cast<float*>(kdsm + (kBlkThreads / 32) * kHeadDim);  // [n_blk]
+  float* kdsm = reinterpret_cast<float*>(blk_dyn + (size_t)H * kQLd * sizeof(uint16_t));
+  float* bkey = reinterpret_cast<float*>(blk_dyn + (size_t)H * kQLd * sizeof(uint16_t) +
+                                         (size_t)(kBlkThreads / 32) * kHeadDim * sizeof(double));
   __shared__ double dlt[H];
   __shared__ unsigned long long band_key[kBlkSmallBand];  // exact scores, ordered keys
   __shared__ int band_blk[kBlkSmallBand];
@@ -984,7 +823,7 @@ __global__ void __launch_bounds__(kBlkThreads) select_blocks_kernel(SelectParams
     const int need2 = kb - (int)n_keep_s;  // >= 1: tau's own block is in the band
     // float64 re-scoring of the band blocks' positions, one warp per position; each
     // block's score is the maximum over its positions (atomic max on ordered keys).
-    double* kd = kdsm + warp * kHeadDim;
+    float* kd = kdsm + warp * kHeadDim;
     const long long n_pos = (long long)n_band * blk;
     for (long long f = warp; f < n_pos; f += kWarps) {
       const int e = (int)(f / blk);
@@ -995,7 +834,8 @@ __global__ void __launch_bounds__(kBlkThreads) select_blocks_kernel(SelectParams
       // is within eps / 2 of the exact one).  Both uniform over the warp.
       if (j >= n_c || __ldcg(trow + j) < bkey[c] - eps) continue;
       const double best =
-          rescore_f64<H, FP8>(p, (size_t)b * p.kv.max_len + j, qsm, dlt, kd, lane);
+          rescore_f64<H, FP8>(p.kv, p.sm_scale, (size_t)b * p.kv.max_len + j,
+                              reinterpret_cast<const uint8_t*>(qsm), kQLd * 2, 16, dlt, kd, lane);
       if (lane == 0) {
         if (band_smem) atomicMax(&band_key[e], ordered_key64(best));
         else atomicMax(bk + e, ordered_key64(best));

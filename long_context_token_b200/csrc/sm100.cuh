@@ -125,6 +125,26 @@ __device__ __forceinline__ void st_global_v4_hint(void* p, uint4 v, uint64_t pol
                "r"(v.y), "r"(v.z), "r"(v.w), "l"(policy)
                : "memory");
 }
+// 4-byte global store with an L2 eviction-priority policy.
+__device__ __forceinline__ void st_global_f32_hint(float* p, float v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(policy)
+               : "memory");
+}
+// Load with acquire semantics at GPU scope (pairs with a release or a fence + atomic of
+// another CTA).
+__device__ __forceinline__ uint32_t ld_acquire_gpu_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Reduction with release semantics at GPU scope: writes ordered before it (by this
+// thread, or by the threads of its CTA through a preceding block barrier) are visible to a
+// thread that observes it with an acquire load.
+__device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Acquire-release fence at GPU scope.
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 // 16-byte global load with an L2 eviction-priority policy.
 // The same through L2 only (no L1 allocation): coherent with writes made by a grid that
 // completed before this one started, even without a grid-dependency wait.

@@ -87,6 +87,23 @@ __device__ __forceinline__ void gather_tile_rows(uint32_t kdst, uint32_t vdst, c
   }
 }
 
+// Gather of up to 128 rows named by a list in shared memory (rows [0, m) of the tile;
+// the rest zero-filled) into the same 128-byte-swizzled layout (K only).  Every listed
+// position must lie inside its sequence.  Each thread still has to wait for its copies.
+template <int CHUNKS, uint32_t BOX>
+__device__ __forceinline__ void gather_list_rows(uint32_t kdst, const uint8_t* kb, const int* list,
+                                                 int m, size_t row_base, int tid, int nthreads) {
+  constexpr uint32_t kRowBytes = CHUNKS * 16;
+  for (int w = tid; w < kKeyTile * CHUNKS; w += nthreads) {
+    const int r = w / CHUNKS, c = w % CHUNKS;
+    const int j = r < m ? list[r] : -1;
+    const size_t off = j >= 0 ? (row_base + (size_t)j) * kRowBytes : 0;
+    const uint32_t at = (uint32_t)(c >> 3) * BOX + (uint32_t)r * 128u +
+                        ((uint32_t)((c & 7) ^ (r & 7)) << 4);
+    sm100::cp_async_16(kdst + at, kb + off + c * 16, j >= 0 ? 16u : 0u);
+  }
+}
+
 // 2^x with the hardware approximation (relative error about 2^-22), results below the
 // normal range flushed to zero; 2^-inf = 0.
 __device__ __forceinline__ float ex2_ftz(float x) {

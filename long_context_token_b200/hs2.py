@@ -37,7 +37,7 @@ EXPORTS = ("hs2_workspace_bytes", "hs2_full_attn_select", "hs2_full_attn", "hs2_
            "hs2_sparse_attn", "hs2_check_device_status", "hs2_status_string",
            "hs2_last_cuda_error", "hs2_abi_version", "hs2_sparse_attn_noalloc", "hs2_kv_append",
            "hs2_full_attn_select_blocks", "hs2_select_blocks", "hs2_prefill_workspace_bytes",
-           "hs2_prefill_attn")
+           "hs2_prefill_attn", "hs2_select_fused")
 
 
 class Hs2Error(RuntimeError):
@@ -106,6 +106,8 @@ def lib():
     L.hs2_last_cuda_error.restype = ctypes.c_char_p
     L.hs2_abi_version.argtypes = []
     L.hs2_abi_version.restype = i32
+    L.hs2_select_fused.argtypes = [i32, i32, i32]
+    L.hs2_select_fused.restype = i32
     _lib = L
     return L
 
@@ -193,6 +195,11 @@ def _check_q(q: torch.Tensor, cache: Cache) -> Tuple[int, int]:
 
 def default_scale() -> float:
     return float(torch.tensor(1.0 / math.sqrt(128.0), dtype=torch.float32))
+
+
+def select_fused(cache: "Cache", n_q: int, h_q: int) -> bool:
+    """True if full_attn_select runs as one kernel for these sizes (hs2_select_fused)."""
+    return bool(lib().hs2_select_fused(n_q, h_q, cache.dtype))
 
 
 def full_attn_select(q: torch.Tensor, cache: Cache, window: int = 128, k_sel: int = 1024,

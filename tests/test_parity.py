@@ -99,6 +99,12 @@ SMALL = [
     dict(id="append5-h48", batch=1, max_len=4321, n_q=5, h_q=48, kv="bf16", seed=114),
     dict(id="append3-h64-short", batch=2, max_len=700, n_q=3, h_q=64, kv="bf16", seed=115,
          lens=[700, 130]),
+    # several tokens on an FP8 cache whose rows are an odd number of keys long (the row
+    # buffers of the fused selection are padded to keep their 16-byte copies aligned)
+    dict(id="append3-fp8-odd-len", batch=2, max_len=1509, n_q=3, h_q=16, kv="fp8", seed=116,
+         lens=[1509, 1402]),
+    dict(id="append2-fp8-h64-odd", batch=3, max_len=2001, n_q=2, h_q=64, kv="fp8", seed=117,
+         lens=[2001, 1999, 1200]),
 ]
 
 
