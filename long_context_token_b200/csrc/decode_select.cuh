@@ -19,16 +19,17 @@
 //      u_j < lo - W - 2 eps can be among the top k_sel (the k_sel-th largest t, T, is at
 //      least lo - W), so only the other keys of its chunk -- the candidates, a few per
 //      thousand -- get their exact float32 t_j, from their K rows gathered again through
-//      the tensor cores, and go to the row's candidate list;
-//   3. after the second barrier every CTA reads the whole candidate list (a few thousand
-//      entries) and takes the same decisions from it: the fine histogram of t over
-//      [lo - W - 2 eps, hi] (which holds T) gives the bin B of the k_sel-th largest t; with
-//      m bins of width at least eps around it, keys of bins >= B + m are in, keys of bins
-//      < B - m are out, and the band between is re-scored in float64 and ranked by (key
-//      desc, position asc);
-//   4. each CTA writes the selected positions of its own chunk, in order, from the slot
-//      after the selected positions below its chunk; the first CTA appends the window.
-//      Then the CTA lets the next kernel start and merges its share of the row's output.
+//      the tensor cores.  Each CTA keeps its candidates (ascending positions) and counts
+//      them in the row's fine histogram of t over [lo - W - 2 eps, hi], which holds T;
+//   3. after the second barrier the fine histogram gives the bin B of the k_sel-th
+//      largest t; with m bins of width at least eps around it, keys of bins >= B + m are
+//      in, keys of bins < B - m are out.  Each CTA counts its own keys that are in, and
+//      re-scores its own keys of the band between in float64 into the row's band list;
+//   4. after the third barrier every CTA ranks the band by (key desc, position asc) and
+//      writes the selected positions of its own chunk, in order, from the slot after those
+//      of the lower chunks (their counts, and the band keys below its chunk that the
+//      ranking takes); the first CTA appends the window.  Then the CTA lets the next
+//      kernel start and merges its share of the row's output.
 // The float32 keys are within eps / 2 of the exact ones, eps = 1e-3 max(1, |bin edge| +
 // W) (as in the separate selection kernels), so the chosen set is the float64
 // definition's up to the tie band.
@@ -51,12 +52,11 @@ constexpr float kSelEps = 1e-3f;
 constexpr long long kRowSpinCycles = 4000000000ll;
 constexpr int kBandSmem = 512;       // bands up to this size are ranked pairwise on chip
 constexpr int kTailTiles = 2;        // candidate tiles (128 keys) gathered at a time
-static_assert(kUBins <= kHistBins, "the u histogram lives in the histogram region");
+static_assert(2 * kUBins <= kHistBins, "the u and fine histograms share a row's histogram region");
 
 // Slots of a row's synchronisation words (the first two belong to the separate selection
 // kernels).
-enum : int { kRowNBand = 2, kRowArrive1 = 3, kRowArrive2 = 4, kRowArrive3 = 5, kRowDone = 6,
-             kRowNcand = 7 };
+enum : int { kRowNBand = 2, kRowArrive1 = 3, kRowArrive2 = 4, kRowArrive3 = 5, kRowDone = 6 };
 
 // Histogram bin of a bound u: monotone in u, u below -64 + 1/16 in bin 0 and u at or above
 // 64 - 1/16 in the last bin (a NaN goes to bin 0).
@@ -259,12 +259,12 @@ __device__ __forceinline__ void async_words(void* dst, const void* src, int n) {
 }
 
 // Block-wide ordered compaction: the indices e of [0, m) with pred(e), in increasing
-// order, as val(e) into out[0, count); returns count to every thread.  Each thread takes a
+// order, each handed to emit(rank, e); returns the count to every thread.  Each thread takes a
 // contiguous run of up to 64 indices (independent loads, a bit mask), then one block-wide
 // exclusive scan of the counts places the runs: no atomics on a shared counter, whose
 // round trips would serialise a loop run by a handful of warps.  All threads call.
-template <typename Pred, typename Val>
-__device__ __forceinline__ int block_compact(int m, Pred pred, Val val, int* out) {
+template <typename Pred, typename Emit>
+__device__ __forceinline__ int block_compact(int m, Pred pred, Emit emit) {
   __shared__ uint32_t wsum[32];
   const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nw = nt >> 5;
@@ -296,7 +296,7 @@ __device__ __forceinline__ int block_compact(int m, Pred pred, Val val, int* out
     while (mask) {
       const int r = __ffsll(mask) - 1;
       mask &= mask - 1;
-      out[at++] = val(e0 + r);
+      emit((int)at++, e0 + r);
     }
     total += (int)all;
     __syncthreads();  // wsum is reused by the next chunk or call
@@ -449,35 +449,67 @@ struct QView {
   int hstride, cstride;
 };
 
+// Position of j in a CTA's ascending list of candidate positions oj[0, n) (an entry may
+// hold ~j once taken: the order of the plain values is kept).
+__device__ __forceinline__ int find_position(const int* oj, int n, int j) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    const int v = oj[mid];
+    if ((v < 0 ? ~v : v) < j) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
 // Steps 2 to 4 of the selection (see the top of this file), after the row's first barrier
-// and lse, with this CTA's first `first` bounds already in `us`.  All threads of every CTA
+// and lse, with this CTA's first `piece` bounds already in `us`.  All threads of every CTA
 // of the row call it.  `recompute(list, m, t2, round, D)` (all threads) gathers the K rows
 // of the positions list[0, m) (m <= kTailTiles * 128), runs them through the stream's S =
 // K Q^T MMA and stores t = max_h (x_h - D[h]) of each into t2[0, m), ending with a block
-// barrier; it returns false if a wait gave up.  Returns false if a wait gave up.
+// barrier; it returns false if a wait gave up.  `scratch` (the gathered tiles' space) is
+// free once the candidates are re-scored.  Returns false if a wait gave up.
 template <int H, bool FP8, typename Recompute>
-__device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* stage,
-                                           uint32_t stage_bytes, uint32_t tile_bytes, float* us,
+__device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* scratch, float* us,
                                            int* cl, float* t2s, int piece, int bq, int b,
                                            int split, int S, int k0, int c_hi, int n_c, int pos,
                                            int bk, const RowLse<H>& rl, const QView& qv,
                                            Recompute&& recompute) {
-  __shared__ uint32_t slot_s, ncand_s, nband_s, sure_s, below_s, base_s;
   __shared__ float eps_s;
   __shared__ FineBins fb_s;
   __shared__ int mb_s;
-  __shared__ unsigned long long vb_s;
-  __shared__ int jb_s;
-  __shared__ uint32_t warp_cnt[32];
+  __shared__ BinScan bs_s;
+  __shared__ uint32_t red_s[2][32];
   const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = nt >> 5;
   const int width = p.window + p.k_sel;
   int32_t* out_row = p.sel_idx + (size_t)bq * width;
   const size_t rowoff = (size_t)bq * p.kv.max_len;
   uint32_t* rs = p.rowsync + (size_t)bq * 8;
-  float* gct = p.cand_t + (size_t)bq * p.ld_u;  // the row's candidate list (16-byte aligned)
-  int32_t* gcj = p.cand_j + (size_t)bq * p.ld_u;
+  uint32_t* gfh = p.uhist + (size_t)bq * kHistBins + kUBins;  // the row's fine histogram
+  uint32_t* rowcnt = p.rowcnt + (size_t)bq * kSmCountBound;
   bool ok = true;
+
+  // Block-wide sums of two counters (all threads call; the result to every thread).
+  auto block_sum2 = [&](uint32_t& x, uint32_t& y) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      x += __shfl_xor_sync(0xffffffffu, x, o);
+      y += __shfl_xor_sync(0xffffffffu, y, o);
+    }
+    if (lane == 0) {
+      red_s[0][warp] = x;
+      red_s[1][warp] = y;
+    }
+    __syncthreads();
+    x = 0u;
+    y = 0u;
+    for (int w = 0; w < nwarps; ++w) {
+      x += red_s[0][w];
+      y += red_s[1][w];
+    }
+    __syncthreads();
+  };
 
   if (tid == 0) {
     const float edge = fmaxf(fabsf(ubin_edge(bk)), fabsf(ubin_edge(bk + 1)));
@@ -496,10 +528,18 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* stage,
   }
   __syncthreads();
   const float eps = eps_s;
+  const FineBins fb = fb_s;
+  const int mb = mb_s;
   const float theta = ubin_floor(bk) - rl.W - 2.f * eps;
 
   // ---- 2. this chunk's candidates, a piece at a time, through the tensor cores in rounds
-  // of kTailTiles tiles; their keys go to the row's candidate list.
+  // of kTailTiles tiles.  Their keys go to the row's fine histogram and to this CTA's list
+  // (ascending positions): on chip when the chunk is one piece, else in the row's
+  // candidate rows at the chunk's offset.
+  const bool one_piece = c_hi - k0 <= piece;
+  float* ot = one_piece ? us : p.cand_t + (size_t)bq * p.ld_u + k0;
+  int* oj = one_piece ? cl : p.cand_j + (size_t)bq * p.ld_u + k0;
+  int own_n = 0;
   uint32_t round = 0;
   for (int pc = k0; pc < c_hi; pc += piece) {
     const int m = min(piece, c_hi - pc);
@@ -510,21 +550,36 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* stage,
     }
     __syncthreads();
     const int ncl = block_compact(
-        m, [&](int e) { return us[e] >= theta; }, [&](int e) { return pc + e; }, cl);
-    uint32_t base = 0;
-    if (tid == 0 && ncl > 0) base = atomicAdd(rs + kRowNcand, (uint32_t)ncl);  // in flight
+        m, [&](int e) { return us[e] >= theta; }, [&](int at, int e) { cl[at] = pc + e; });
     for (int r0 = 0; r0 < ncl; r0 += kTailTiles * 128, ++round) {
       const int mm = min(kTailTiles * 128, ncl - r0);
       if (!recompute(cl + r0, mm, t2s, round, rl.D)) ok = false;
-      if (tid == 0 && r0 == 0) slot_s = base;
-      __syncthreads();
-      const uint32_t at = slot_s + (uint32_t)r0;
+      uint32_t top = 0, bot = 0;
       for (int e = tid; e < mm; e += nt) {
-        gct[at + e] = t2s[e];
-        gcj[at + e] = cl[r0 + e];
+        const float t = t2s[e];
+        const int bb = fb.bin(t);
+        if (bb == kUBins - 1) ++top;
+        else if (bb == 0) ++bot;
+        else atomicAdd(gfh + bb, 1u);
+        if (one_piece) {
+          us[r0 + e] = t;  // the bounds were consumed by the compaction
+        } else {
+          ot[own_n + r0 + e] = t;
+          oj[own_n + r0 + e] = cl[r0 + e];
+        }
       }
-      __syncthreads();
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        top += __shfl_xor_sync(0xffffffffu, top, o);
+        bot += __shfl_xor_sync(0xffffffffu, bot, o);
+      }
+      if (lane == 0) {
+        if (top) atomicAdd(gfh + kUBins - 1, top);
+        if (bot) atomicAdd(gfh, bot);
+      }
+      __syncthreads();  // t2s is refilled by the next round
     }
+    own_n += ncl;
   }
   row_arrive(rs + kRowArrive2);
   if (!row_wait(rs + kRowArrive2, (uint32_t)S)) ok = false;
@@ -533,206 +588,94 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* stage,
   uint32_t* gu = p.uhist + (size_t)bq * kHistBins;
   for (int e = split * nt + tid; e < kUBins; e += S * nt) gu[e] = 0u;
 
-  // ---- 3. every CTA reads the row's candidate list and takes the same decisions
-  // Each thread holds kRegCand entries of the list in registers per pass; one pass builds
-  // the fine histogram of every candidate and that of the candidates below this chunk.
-  uint32_t off = 0;
-  auto take = [&](uint32_t bytes) {
-    uint8_t* at = stage + off;
-    off += (bytes + 15u) & ~15u;
-    return at;
-  };
-  uint32_t* fh = reinterpret_cast<uint32_t*>(take(kUBinsPadded * 4));   // all candidates
-  uint32_t* fb_lo = reinterpret_cast<uint32_t*>(take(kUBinsPadded * 4));  // those below k0
-  unsigned long long* bkey = reinterpret_cast<unsigned long long*>(take(kBandSmem * 8));
-  int* bpos = reinterpret_cast<int*>(take(kBandSmem * 4));
-  float* kf = reinterpret_cast<float*>(take((uint32_t)nwarps * kHeadDim * 4));
-  const int chunk_len = c_hi > k0 ? c_hi - k0 : 0;
-  const int nwords = (chunk_len + 31) / 32;
-  uint32_t* bm = reinterpret_cast<uint32_t*>(take((uint32_t)nwords * 4));
-  // This chunk's band keys, in the rest of the stages (a chunk's worth, or as many as fit).
-  int* own_band = reinterpret_cast<int*>(stage + off);
-  const uint32_t own_cap = min((uint32_t)max(chunk_len, 1), (stage_bytes > off ? stage_bytes - off : 0u) / 4u);
-  for (int e = tid; e < kUBinsPadded; e += nt) {
-    fh[e] = 0u;
-    fb_lo[e] = 0u;
-  }
-  for (int w = tid; w < nwords; w += nt) bm[w] = 0u;
-  if (tid == 0) {
-    ncand_s = min(__ldcg(rs + kRowNcand), (uint32_t)p.kv.max_len);
-    below_s = 0u;
-    slot_s = 0u;  // this chunk's band keys listed so far
-  }
-  constexpr int kRegCand = 16;
-  const uint32_t chunk_n = kRegCand * (uint32_t)nt;
-  // Loads of the first kRegCand x nt entries, issued before the count is known (entries
-  // past the count are ignored).
-  float rt[kRegCand];
-  int rj[kRegCand];
-  auto load_regs = [&](uint32_t c0) {
-#pragma unroll
-    for (int u = 0; u < kRegCand; ++u) {
-      const uint32_t e = c0 + (uint32_t)u * nt + tid;
-      const bool in = e < (uint32_t)p.kv.max_len;
-      rt[u] = in ? __ldcg(gct + e) : -INFINITY;
-      rj[u] = in ? __ldcg(gcj + e) : -1;
-    }
-  };
-  load_regs(0);
-  __syncthreads();
-  const uint32_t n = ncand_s;
-  const FineBins fb = fb_s;
-  auto add_hist = [&](uint32_t c0) {
-    uint32_t top = 0, bot = 0, top_lo = 0, bot_lo = 0;
-#pragma unroll
-    for (int u = 0; u < kRegCand; ++u) {
-      const uint32_t e = c0 + (uint32_t)u * nt + tid;
-      if (e >= n) continue;
-      const int bb = fb.bin(rt[u]);
-      const bool lo = rj[u] < k0;
-      if (bb == kUBins - 1) {
-        ++top;
-        top_lo += lo;
-      } else if (bb == 0) {
-        ++bot;
-        bot_lo += lo;
-      } else {
-        atomicAdd(&fh[ubin_slot(bb)], 1u);
-        if (lo) atomicAdd(&fb_lo[ubin_slot(bb)], 1u);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      top += __shfl_xor_sync(0xffffffffu, top, o);
-      bot += __shfl_xor_sync(0xffffffffu, bot, o);
-      top_lo += __shfl_xor_sync(0xffffffffu, top_lo, o);
-      bot_lo += __shfl_xor_sync(0xffffffffu, bot_lo, o);
-    }
-    if (lane == 0) {
-      if (top) atomicAdd(&fh[ubin_slot(kUBins - 1)], top);
-      if (bot) atomicAdd(&fh[ubin_slot(0)], bot);
-      if (top_lo) atomicAdd(&fb_lo[ubin_slot(kUBins - 1)], top_lo);
-      if (bot_lo) atomicAdd(&fb_lo[ubin_slot(0)], bot_lo);
-    }
-  };
-  add_hist(0);
-  for (uint32_t c0 = chunk_n; c0 < n; c0 += chunk_n) {  // long lists only
-    load_regs(c0);
-    add_hist(c0);
+  // ---- 3. the row's fine histogram gives B, the bin of the k_sel-th largest t: keys of
+  // bins >= B + mb are in, keys of bins [B - mb, B + mb) form the band.
+  if (warp == 0) {
+    const BinScan r = scan_global_bins(gfh, p.k_sel, mb);
+    if (lane == 0) bs_s = r;
   }
   __syncthreads();
-  const int B = kth_bin_from_top(p.k_sel, fh);
-  const int mb = mb_s;
-  if (tid < 32) {
-    // Bins >= B + mb are in, bins [B - mb, B + mb) form the band: the totals, and the
-    // sure ones below this chunk.
-    uint32_t sure = 0, band = 0, sure_lo = 0;
-#pragma unroll 8
-    for (int e = lane; e < kUBins; e += 32) {
-      const uint32_t c = fh[ubin_slot(e)];
-      const bool in = e >= B + mb;
-      sure += in ? c : 0u;
-      band += (e >= B - mb && e < B + mb) ? c : 0u;
-      sure_lo += in ? fb_lo[ubin_slot(e)] : 0u;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      sure += __shfl_xor_sync(0xffffffffu, sure, o);
-      band += __shfl_xor_sync(0xffffffffu, band, o);
-      sure_lo += __shfl_xor_sync(0xffffffffu, sure_lo, o);
-    }
-    if (lane == 0) {
-      sure_s = sure;
-      nband_s = band;
-      base_s = sure_lo;
-    }
-  }
-  __syncthreads();
-  const int need2 = p.k_sel - (int)sure_s;  // taken from the band: 1 <= need2 <= n_band
-  const int n_band = (int)nband_s;
+  const int B = bs_s.bin;
+  const int n_band = (int)bs_s.near;
+  const int need2 = p.k_sel - (int)bs_s.above;  // taken from the band: 1 <= need2 <= n_band
   const bool rank_band = need2 < n_band;
-  // This chunk's candidates: the sure ones into the bitmap; band keys listed for the
-  // float64 re-scoring (when every band key is taken they count as sure, below the chunk
-  // too).
-  auto classify = [&](uint32_t c0) {
-    uint32_t band_lo = 0;
-#pragma unroll
-    for (int u = 0; u < kRegCand; ++u) {
-      const uint32_t e = c0 + (uint32_t)u * nt + tid;
-      if (e >= n) continue;
-      const int bb = fb.bin(rt[u]);
-      const int j = rj[u];
-      const bool sure = bb >= B + mb;
-      const bool band = !sure && bb >= B - mb;
-      if (band && !rank_band && j < k0) ++band_lo;
-      if (j < k0 || j >= c_hi) continue;
-      if (sure || (band && !rank_band)) {
-        atomicOr(&bm[(j - k0) >> 5], 1u << ((j - k0) & 31));
-      } else if (band) {
-        const uint32_t slot = atomicAdd(&slot_s, 1u);
-        if (slot < own_cap) own_band[slot] = j;
+  // When every band key is taken the band counts as in.
+  const int in_bin = rank_band ? B + mb : B - mb;
+  auto in_band = [&](int bb) { return bb >= B - mb && bb < B + mb; };
+  uint32_t cin = 0, cband = 0;
+  for (int e = tid; e < own_n; e += nt) {
+    const int bb = fb.bin(ot[e]);
+    cin += bb >= in_bin;
+    cband += rank_band && in_band(bb);
+  }
+  block_sum2(cin, cband);
+  if (tid == 0) rowcnt[split] = cin;  // read by the higher chunks after the third barrier
+  // The float64 keys of this chunk's band keys (one warp each) go to the row's band list.
+  float* kf = reinterpret_cast<float*>(scratch);
+  if (cband) {
+    for (int c = warp * 32; c < own_n; c += nwarps * 32) {
+      const int e = c + lane;
+      const bool isb = e < own_n && in_band(fb.bin(ot[e]));
+      unsigned mask = __ballot_sync(0xffffffffu, isb);
+      while (mask) {
+        const int ee = c + __ffs(mask) - 1;
+        mask &= mask - 1;
+        const int j = oj[ee];
+        uint32_t slot = 0;
+        if (lane == 0) slot = atomicAdd(rs + kRowNBand, 1u);  // in flight while re-scoring
+        const double v = rescore_f64<H, FP8>(p.kv, p.sm_scale, (size_t)b * p.kv.max_len + j,
+                                             qv.base, qv.hstride, qv.cstride, rl.dl,
+                                             kf + warp * kHeadDim, lane);
+        if (lane == 0 && slot < (uint32_t)p.kv.max_len) {
+          p.band_t[rowoff + slot] = v;
+          p.band_j[rowoff + slot] = j;
+        }
       }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) band_lo += __shfl_xor_sync(0xffffffffu, band_lo, o);
-    if (lane == 0 && band_lo) atomicAdd(&below_s, band_lo);
-  };
-  if (n <= chunk_n) {
-    classify(0);
-  } else {
-    for (uint32_t c0 = 0; c0 < n; c0 += chunk_n) {
-      load_regs(c0);
-      classify(c0);
     }
   }
-  __syncthreads();
+  row_arrive(rs + kRowArrive3);
+  if (!row_wait(rs + kRowArrive3, (uint32_t)S)) ok = false;
+  // Every CTA has read the fine histogram: clear this CTA's share for the next call.
+  for (int e = split * nt + tid; e < kUBins; e += S * nt) gfh[e] = 0u;
+
+  // ---- 4. the slot of this chunk's first selected position: the selections of the lower
+  // chunks (their counts, and the band keys below k0 that the ranking takes)
+  uint32_t below = 0, unused = 0;
+  for (int s2 = tid; s2 < split; s2 += nt) below += __ldcg(rowcnt + s2);
   if (rank_band) {
-    // This chunk's band keys: float64 keys (one warp each) appended to the row's band list.
-    const int nob = (int)min(slot_s, own_cap);
-    if (tid == 0 && slot_s > own_cap) set_status(p.status, HS2_ERR_UNSUPPORTED);
-    __shared__ uint32_t bbase_s;
-    if (tid == 0) bbase_s = nob ? atomicAdd(rs + kRowNBand, (uint32_t)nob) : 0u;
-    __syncthreads();
-    for (int e = warp; e < nob; e += nwarps) {
-      const int j = own_band[e];
-      const double v = rescore_f64<H, FP8>(p.kv, p.sm_scale, (size_t)b * p.kv.max_len + j, qv.base,
-                                           qv.hstride, qv.cstride, rl.dl, kf + warp * kHeadDim,
-                                           lane);
-      if (lane == 0) {
-        p.band_t[rowoff + bbase_s + e] = v;
-        p.band_j[rowoff + bbase_s + e] = j;
-      }
-    }
-    row_arrive(rs + kRowArrive3);
-    if (!row_wait(rs + kRowArrive3, (uint32_t)S)) ok = false;
     // Every CTA ranks the whole band by (key desc, position asc): the top need2 are in.
+    // Those of this chunk are marked (~j) in its list.
     const double* gbt = p.band_t + rowoff;
     const int32_t* gbj = p.band_j + rowoff;
-    uint32_t band_lo = 0;
-    auto take_band = [&](int je) {
-      if (je < k0) ++band_lo;
-      else if (je < c_hi) atomicOr(&bm[(je - k0) >> 5], 1u << ((je - k0) & 31));
+    auto take = [&](int je) {
+      if (je < k0) ++below;
+      else if (je < c_hi) {
+        const int e = find_position(oj, own_n, je);
+        if (e < own_n) oj[e] = ~je;
+      }
     };
-    if (n_band <= kBandSmem) {
-      for (int e = tid; e < n_band; e += nt) {
+    const int nb = min(n_band, (int)p.kv.max_len);
+    if (nb <= kBandSmem) {
+      unsigned long long* bkey = reinterpret_cast<unsigned long long*>(scratch);
+      int* bpos = reinterpret_cast<int*>(scratch + kBandSmem * 8);
+      for (int e = tid; e < nb; e += nt) {
         bkey[e] = ordered_key64(__ldcg(gbt + e));
         bpos[e] = __ldcg(gbj + e);
       }
       __syncthreads();
-      for (int e = tid; e < n_band; e += nt) {
+      for (int e = tid; e < nb; e += nt) {
         const unsigned long long ke = bkey[e];
         const int je = bpos[e];
         int rank = 0;
-        for (int f = 0; f < n_band; ++f) {
+        for (int f = 0; f < nb; ++f) {
           const unsigned long long kf2 = bkey[f];
           rank += (kf2 > ke) || (kf2 == ke && bpos[f] < je);
         }
-        if (rank < need2) take_band(je);
+        if (rank < need2) take(je);
       }
     } else {
       // A large band (many equal keys): the boundary by radix select over the list.
       __shared__ uint32_t gt_s;
-      const int nb = min(n_band, (int)p.kv.max_len);
       const unsigned long long vb = block_kth_largest<unsigned long long, 64>(
           nb, need2, [&](int e) { return ordered_key64(__ldcg(gbt + e)); },
           [](int) { return true; }, &gt_s);
@@ -744,40 +687,20 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* stage,
       for (int e = tid; e < nb; e += nt) {
         const unsigned long long k = ordered_key64(__ldcg(gbt + e));
         const int je = __ldcg(gbj + e);
-        if (k > vb || (k == vb && je <= jb)) take_band(je);
+        if (k > vb || (k == vb && je <= jb)) take(je);
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) band_lo += __shfl_xor_sync(0xffffffffu, band_lo, o);
-    if (lane == 0 && band_lo) atomicAdd(&below_s, band_lo);
   }
-  __syncthreads();
-
-  // ---- 4. this chunk's positions in order, from the slot after the selected positions
-  // below the chunk
-  const int per = (nwords + nt - 1) / nt;
-  const int w0 = tid * per, w1 = min(w0 + per, nwords);
-  uint32_t cnt = 0;
-  for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
-  uint32_t incl = cnt;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += x;
-  }
-  if (lane == 31) warp_cnt[warp] = incl;
-  __syncthreads();
-  uint32_t at = base_s + below_s + incl - cnt;
-  for (int k = 0; k < warp; ++k) at += warp_cnt[k];
-  for (int w = w0; w < w1; ++w) {
-    uint32_t bits = bm[w];
-    while (bits) {
-      const int bit = __ffs(bits) - 1;
-      bits &= bits - 1;
-      if (at < (uint32_t)p.k_sel) out_row[at] = k0 + w * 32 + bit;
-      ++at;
-    }
-  }
+  block_sum2(below, unused);  // also orders the marks before the compaction reads them
+  // This chunk's selected positions, in order, from slot `below`.
+  block_compact(
+      own_n,
+      [&](int e) { return oj[e] < 0 || fb.bin(ot[e]) >= in_bin; },
+      [&](int at, int e) {
+        const uint32_t slot = below + (uint32_t)at;
+        const int v = oj[e];
+        if (slot < (uint32_t)p.k_sel) out_row[slot] = v < 0 ? ~v : v;
+      });
   // The window and the padding after the k_sel selected positions.
   if (split == 0)
     for (int e = p.k_sel + tid; e < width; e += nt) {
@@ -834,8 +757,8 @@ __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, 
     sm100::cp_async_wait_all();
     __syncthreads();
     const int bk = kth_bin_from_top(p.k_sel, uh);
-    if (!row_select<H, FP8>(p, stage, stage_bytes, tile_bytes, us, cl, t2s, piece, bq, b, split,
-                            S, k0, c_hi, n_c, pos, bk, rl, qv, recompute))
+    if (!row_select<H, FP8>(p, stage, us, cl, t2s, piece, bq, b, split, S, k0, c_hi, n_c, pos,
+                            bk, rl, qv, recompute))
       ok = false;
   }
   // The index set is complete and visible: the next kernel (a sparse layer reads it
@@ -852,7 +775,6 @@ __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, 
       rs[kRowArrive1] = 0u;
       rs[kRowArrive2] = 0u;
       rs[kRowArrive3] = 0u;
-      rs[kRowNcand] = 0u;
       rs[kRowNBand] = 0u;
       rs[kRowDone] = 0u;
       __threadfence();

@@ -103,13 +103,13 @@ struct FullParams {
   double* lse64 = nullptr;       // [bq][h]
   float* ubuf = nullptr;         // [bq][ld_u]: per-key bound u_j = max_h x_hj (log2 units)
   int ld_u = 0;
-  uint32_t* uhist = nullptr;     // [bq][kHistBins] (the first kUBins bins used)
-  uint32_t* rowsync = nullptr;   // [bq][8]: arrival counters and the candidate count
-  float* cand_t = nullptr;       // [bq][ld_u] the row's candidate list: keys ...
+  uint32_t* uhist = nullptr;     // [bq][kHistBins]: the u histogram, then the fine one
+  uint32_t* rowsync = nullptr;   // [bq][8]: arrival counters and the band list's length
+  float* cand_t = nullptr;       // [bq][ld_u] candidates of long chunks, at the chunk's offset: keys ...
   int32_t* cand_j = nullptr;     // [bq][ld_u] ... and positions
   double* band_t = nullptr;      // [bq][max_len] the row's band list: float64 keys ...
   int32_t* band_j = nullptr;     // [bq][max_len] ... and positions
-  uint32_t* rowcnt = nullptr;    // [bq][kSmCountBound] sure selections per CTA of a row
+  uint32_t* rowcnt = nullptr;    // [bq][kSmCountBound] keys per CTA of a row in before the band ranking
   int32_t* sel_idx = nullptr;    // [bq][window + k_sel]
 };
 
