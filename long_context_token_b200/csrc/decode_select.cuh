@@ -85,7 +85,7 @@ struct FineBins {
 
 // Shared-memory histograms keep four padding words after every 64 bins: 16-byte chunks
 // stay aligned (cp.async copies them in), and the 32 lanes scanning 64 consecutive bins
-// each (kth_bin_from_top) meet at most 4-way bank conflicts.
+// each (scan_bins) meet at most 4-way bank conflicts.
 constexpr int kUBinsPadded = kUBins + kUBins / 16;
 __device__ __forceinline__ int ubin_slot(int b) { return b + ((b >> 6) << 2); }
 
@@ -118,125 +118,83 @@ static __device__ __noinline__ bool row_wait(uint32_t* counter, uint32_t target)
   return ok_s != 0;
 }
 
-// Warp 0 scans a padded shared-memory histogram (ubin_slot) from the top: lane l owns
-// bins [kUBins - 64(l + 1), kUBins - 64 l).  Returns (to every thread) the bin holding the
-// k-th largest element, or 0 if there are fewer than k.  All threads call.
-__device__ __forceinline__ int kth_bin_from_top(int k, const uint32_t* hs) {
-  static_assert(kUBins == 32 * 64, "64 bins per lane");
-  __shared__ int bin_s;
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    const int base = kUBins - 64 * (lane + 1);
-    const uint4* row = reinterpret_cast<const uint4*>(hs + ubin_slot(base));  // contiguous
-    uint4 c[16];
-    uint32_t sum = 0;
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      c[u] = row[u];
-      sum += c[u].x + c[u].y + c[u].z + c[u].w;
-    }
-    uint32_t incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += x;
-    }
-    if (lane == 0) bin_s = 0;
-    __syncwarp();
-    const uint32_t above = incl - sum;
-    if (above < (uint32_t)k && (uint32_t)k <= incl) {
-      uint32_t cum = above;
-      int bin = base;
-      bool found = false;
-#pragma unroll
-      for (int u = 15; u >= 0; --u) {
-        const uint32_t v[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
-#pragma unroll
-        for (int q = 3; q >= 0; --q) {
-          cum += v[q];
-          if (!found && cum >= (uint32_t)k) {
-            found = true;
-            bin = base + 4 * u + q;
-          }
-        }
-      }
-      bin_s = bin;
-    }
-  }
-  __syncthreads();
-  return bin_s;
-}
-
-// Warp 0 (all 32 lanes) reads a global kUBins histogram straight into registers (lane l
-// holds bins [kUBins - 64(l + 1), kUBins - 64 l)) and finds the bin B holding the k-th
-// largest element (0 if there are fewer than k).  With mb > 0 it also sums the bins >= B +
-// mb (`above`) and the bins [B - mb, B + mb) (`near`).  Results in lane 0.
+// The bin B holding the k-th largest element of a padded shared-memory histogram
+// (ubin_slot; 0 if there are fewer than k), and with mb > 0 the counts in the bins >= B +
+// mb (`above`) and in [B - mb, B + mb) (`near`).  Warp 0 scans (lane l owns the bins
+// [kUBins - 64(l + 1), kUBins - 64 l), contiguous in the padded layout); every thread
+// calls it and gets the result.  The tail runs this code once per launch, so it is one
+// out-of-line copy with rolled loops: fetching instructions that run once costs more
+// than executing them.
 struct BinScan {
   int bin;
   uint32_t above, near;
 };
-__device__ __forceinline__ BinScan scan_global_bins(const uint32_t* gh, int k, int mb) {
+static __device__ __noinline__ BinScan scan_bins(const uint32_t* hs, int k, int mb) {
   static_assert(kUBins == 32 * 64, "64 bins per lane");
-  const int lane = threadIdx.x & 31;
-  const int base = kUBins - 64 * (lane + 1);
-  uint4 c[16];
-#pragma unroll
-  for (int u = 0; u < 16; ++u) c[u] = __ldcg(reinterpret_cast<const uint4*>(gh + base) + u);
-  uint32_t sum = 0;
-#pragma unroll
-  for (int u = 0; u < 16; ++u) sum += c[u].x + c[u].y + c[u].z + c[u].w;
-  uint32_t incl = sum;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += x;
-  }
-  const uint32_t before = incl - sum;  // in the bins above this lane's
-  int bin = -1;
-  if (before < (uint32_t)k && (uint32_t)k <= incl) {
-    uint32_t cum = before;
-#pragma unroll
-    for (int u = 15; u >= 0; --u) {
-      const uint32_t v[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
-#pragma unroll
-      for (int q = 3; q >= 0; --q) {
-        cum += v[q];
-        if (bin < 0 && cum >= (uint32_t)k) bin = base + 4 * u + q;
-      }
-    }
-  }
-  const unsigned found = __ballot_sync(0xffffffffu, bin >= 0);
-  const int B = found ? __shfl_sync(0xffffffffu, bin, __ffs(found) - 1) : 0;
-  BinScan r;
-  r.bin = B;
-  r.above = 0;
-  r.near = 0;
-  if (mb > 0) {
-    uint32_t above = 0, near = 0;
-#pragma unroll
+  __shared__ BinScan out_s;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int base = kUBins - 64 * (lane + 1);
+    const uint4* row = reinterpret_cast<const uint4*>(hs + ubin_slot(base));
+    uint32_t sum = 0;
+#pragma unroll 1
     for (int u = 0; u < 16; ++u) {
-      const uint32_t v[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+      const uint4 c = row[u];
+      sum += (c.x + c.y) + (c.z + c.w);
+    }
+    uint32_t incl = sum;
+#pragma unroll 1
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += x;
+    }
+    const uint32_t before = incl - sum;  // in the bins above this lane's
+    int bin = -1;
+    if (before < (uint32_t)k && (uint32_t)k <= incl) {
+      uint32_t cum = before;
+#pragma unroll 1
+      for (int u = 15; u >= 0 && bin < 0; --u) {
+        const uint4 c = row[u];
+        const uint32_t v[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int e = base + 4 * u + q;
-        above += e >= B + mb ? v[q] : 0u;
-        near += (e >= B - mb && e < B + mb) ? v[q] : 0u;
+        for (int q = 3; q >= 0; --q) {
+          cum += v[q];
+          if (bin < 0 && cum >= (uint32_t)k) bin = base + 4 * u + q;
+        }
       }
     }
+    const unsigned found = __ballot_sync(0xffffffffu, bin >= 0);
+    const int B = found ? __shfl_sync(0xffffffffu, bin, __ffs(found) - 1) : 0;
+    uint32_t above = 0, near = 0;
+    if (mb > 0) {
+#pragma unroll 1
+      for (int u = 0; u < 16; ++u) {
+        const uint4 c = row[u];
+        const uint32_t v[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      above += __shfl_xor_sync(0xffffffffu, above, o);
-      near += __shfl_xor_sync(0xffffffffu, near, o);
+        for (int q = 0; q < 4; ++q) {
+          const int e = base + 4 * u + q;
+          above += e >= B + mb ? v[q] : 0u;
+          near += (e >= B - mb && e < B + mb) ? v[q] : 0u;
+        }
+      }
+      above = __reduce_add_sync(0xffffffffu, above);
+      near = __reduce_add_sync(0xffffffffu, near);
     }
-    r.above = above;
-    r.near = near;
+    if (lane == 0) {
+      out_s.bin = B;
+      out_s.above = above;
+      out_s.near = near;
+    }
   }
-  return r;
+  __syncthreads();
+  return out_s;
 }
 
 // Adds a padded shared-memory histogram to a global one: every non-empty bin at or above
 // `low`.  All threads call.
 __device__ __forceinline__ void add_bins(const uint32_t* hs, uint32_t* gh, int low) {
+#pragma unroll 1
   for (int e = low + (int)threadIdx.x; e < kUBins; e += blockDim.x) {
     const uint32_t c = hs[ubin_slot(e)];
     if (c) atomicAdd(gh + e, c);
@@ -307,7 +265,7 @@ __device__ __forceinline__ int block_compact(int m, Pred pred, Emit emit) {
 // The row's log-sum-exp per head, from its split partials.
 template <int H>
 struct RowLse {
-  float M[H];      // largest reference m over the non-empty splits (log2 units)
+  float M[H];      // largest m over the non-empty splits (log2 units)
   float invL[H];   // 1 / sum_s l_s 2^(m_s - M)
   double lse2[H];  // M + log2 sum_s l_s 2^(m_s - M)  (log2 units)
   double dl[H];    // (lse2 - min_h lse2) ln 2: the float64 shifts of the re-scoring
@@ -315,123 +273,149 @@ struct RowLse {
   float W;         // max_h D
 };
 
-// Every thread calls this; pml: the row's partials [S][H][2] (m in log2 units, l).  Head h
-// is taken by tph consecutive threads (the largest power of two, at most 32, with
-// H * tph <= blockDim), each over the splits sub, sub + tph, ...: the largest reference M
-// over the non-empty splits, then L = sum_s l_s 2^(m_s - M) with each weight in float32
-// (relative error below 2^-22, well under that of the partial sums l) summed without loss
-// (two-sum, also across the threads of the head).  log2 L is taken on the mantissa of its
+// Ordered 32-bit keys of float32 values for an unsigned atomicMax (key 0, the zero state,
+// is below every value).
+__device__ __forceinline__ uint32_t max_key(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float max_key_value(uint32_t k) {
+  return k == 0u ? -INFINITY : __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Every thread calls this; pml: the row's partials [S][H][2] (m in log2 units, l); rowmax:
+// the ordered keys of the row's largest m per head (every CTA of the row adds its own
+// before the first barrier); tmp: blockDim.x float2 of shared scratch.  M_h is that
+// largest m, and L_h = sum_s l_s 2^(m_s - M_h), each weight in float32 (relative error
+// below 2^-22, well under that of the partial sums l) summed without loss (two-sum).
+// Thread t takes head t % H and the splits t / H, t / H + G, ... (G = blockDim / H), so
+// consecutive threads read consecutive partials.  log2 L is taken on the mantissa of its
 // leading float (log2f of a value in [0.5, 1), absolute error about 2^-24) plus the
 // exponent and the first-order term of the trailing float, and assembled with M in
 // float64: lse2 carries about 2^-23 absolute, well inside the 1e-6 tie band of the
 // selection.  The shifts D and dl are taken from C, a common value just below the
-// smallest lse2 (the ranking does not depend on which).
+// smallest lse2 (the ranking does not depend on which).  Every CTA of the row reads the
+// same partials in the same order, so all get the same bits.
 template <int H>
-__device__ __forceinline__ void row_lse(const float* __restrict__ pml, int S, RowLse<H>& r) {
+static __device__ __noinline__ void row_lse(const float* __restrict__ pml,
+                                            const uint32_t* __restrict__ rowmax, int S,
+                                            RowLse<H>& r, float2* tmp) {
   const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31;
-  int tph = 1;
-  while (tph < 32 && 2 * tph * H <= nt) tph *= 2;
-  const int h = tid / tph, sub = tid % tph;
-  const bool mine = h < H;
-  float M = -INFINITY;
-  if (mine) {
-#pragma unroll 8
-    for (int s = sub; s < S; s += tph) {
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(pml + ((size_t)s * H + h) * 2));
-      if (v.y > 0.f) M = fmaxf(M, v.x);
-    }
-  }
-  for (int o = 1; o < tph; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const int G = nt / H;
+  const int h = tid % H, g = tid / H;
+  if (tid < H) r.M[tid] = max_key_value(__ldcg(rowmax + tid));
+  __syncthreads();
   float ls = 0.f, le = 0.f;
-  if (mine && M != -INFINITY) {
+  if (g < G) {
+    const float M = r.M[h];
+    const float2* src = reinterpret_cast<const float2*>(pml) + h;
 #pragma unroll 8
-    for (int s = sub; s < S; s += tph) {
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(pml + ((size_t)s * H + h) * 2));
+    for (int s = g; s < S; s += G) {
+      const float2 v = __ldcg(src + (size_t)s * H);
       if (v.y > 0.f) two_sum_acc(ls, le, v.y * exp2f(v.x - M));
     }
   }
-  for (int o = 1; o < tph; o <<= 1) {
-    const float os = __shfl_xor_sync(0xffffffffu, ls, o);
-    const float oe = __shfl_xor_sync(0xffffffffu, le, o);
-    le += oe;
-    two_sum_acc(ls, le, os);
-  }
-  if (mine && sub == 0) {
-    const float lh = ls + le;            // leading float of L
-    const float ll = (ls - lh) + le;     // and the rest
-    r.M[h] = M;
+  tmp[tid] = make_float2(ls, le);
+  __syncthreads();
+  if (tid < H) {
+    ls = 0.f;
+    le = 0.f;
+#pragma unroll 1
+    for (int g2 = 0; g2 < G; ++g2) {
+      const float2 v = tmp[g2 * H + tid];
+      le += v.y;
+      two_sum_acc(ls, le, v.x);
+    }
+    const float lh = ls + le;         // leading float of L
+    const float ll = (ls - lh) + le;  // and the rest
     if (lh > 0.f) {
       int ex;
       const float mant = frexpf(lh, &ex);  // lh = mant 2^ex, mant in [0.5, 1)
-      r.invL[h] = 1.f / lh;
-      r.lse2[h] = (double)M + (double)ex + (double)log2f(mant) +
-                  (double)(ll / lh * 1.4426950408889634f);
+      r.invL[tid] = 1.f / lh;
+      r.lse2[tid] = (double)r.M[tid] + (double)ex + (double)log2f(mant) +
+                    (double)(ll / lh * 1.4426950408889634f);
     } else {
-      r.invL[h] = 0.f;
-      r.lse2[h] = -INFINITY;
+      r.invL[tid] = 0.f;
+      r.lse2[tid] = -INFINITY;
     }
   }
   __syncthreads();
   if (tid < 32) {
-    float mn = INFINITY, mx = -INFINITY;
-    for (int hh = lane; hh < H; hh += 32) {
-      mn = fminf(mn, (float)r.lse2[hh]);
-      mx = fmaxf(mx, (float)r.lse2[hh]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    }
+    float mn = INFINITY;
+#pragma unroll 1
+    for (int hh = lane; hh < H; hh += 32) mn = fminf(mn, (float)r.lse2[hh]);
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 16));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 8));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 4));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
     const double c = (double)mn - 1e-5 * fmax(1.0, fabs((double)mn));  // at or below every lse2
     float w = 0.f;
+#pragma unroll 1
     for (int hh = lane; hh < H; hh += 32) {
       const double d = r.lse2[hh] - c;
       r.D[hh] = (float)d;
       r.dl[hh] = d * 0.69314718055994530942;
       w = fmaxf(w, (float)d);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, o));
+    w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, 16));
+    w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, 8));
+    w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, 4));
+    w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, 2));
+    w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, 1));
     if (lane == 0) r.W = w * (1.f + 1e-6f);  // covers the rounding of D to float
-    (void)mx;
   }
   __syncthreads();
 }
 
-// This CTA's share of the row's merged output: outputs (h, d) of the row taken in turn
-// by the row's S CTAs; out_h = sum_s 2^(m_s - M) o_s / L.  The thread holding d = 0 of a
-// head writes its lse (natural log) to lse64 and lse_out.
+// This CTA's share of the row's merged output, out_h = sum_s 2^(m_s - M) o_s / L: CTA r
+// of the row takes the outputs [r P, (r + 1) P), P = ceil(H kHeadDim / S); each output is
+// summed by G = blockDim / P threads over every G-th split (consecutive threads read
+// consecutive outputs of one split), and the G sums meet in shared memory (tmp: blockDim.x
+// floats).  The thread holding d = 0 of a head writes its lse (natural log) to lse64 and
+// lse_out.  Every thread calls it.
 template <int H>
-__device__ __forceinline__ void row_merge(const FullParams& p, int bq, int split, int S,
-                                          const RowLse<H>& r) {
+static __device__ __noinline__ void row_merge(const FullParams& p, int bq, int split, int S,
+                                              const RowLse<H>& r, float* tmp) {
   const float* po = p.part_o + (size_t)bq * S * H * kHeadDim;
-  const float* pml = p.part_ml + (size_t)bq * S * H * 2;
+  const float2* pml = reinterpret_cast<const float2*>(p.part_ml + (size_t)bq * S * H * 2);
   constexpr int kOut = H * kHeadDim;
-  constexpr int kB = 8;  // splits whose loads are in flight together
-  for (int o = split * (int)blockDim.x + (int)threadIdx.x; o < kOut; o += S * (int)blockDim.x) {
+  const int nt = blockDim.x, tid = threadIdx.x;
+  const int opc = (kOut + S - 1) / S;
+  const int o0 = split * opc, o1 = min(o0 + opc, kOut);
+  const int P = min(opc, nt);  // outputs per round
+  const int G = nt / P;        // threads per output
+  const int ol = tid % P, g = tid / P;
+#pragma unroll 1
+  for (int ob = o0; ob < o1; ob += P) {
+    const int o = ob + ol;
+    const bool mine = g < G && o < o1;
     const int h = o / kHeadDim, d = o % kHeadDim;
-    const float M = r.M[h], il = r.invL[h];
     float acc = 0.f;
-    for (int s0 = 0; s0 < S; s0 += kB) {
-      float2 ml[kB];
-      float v[kB];
-#pragma unroll
-      for (int u = 0; u < kB; ++u) {
-        const int s = s0 + u;
-        ml[u] = s < S ? __ldcg(reinterpret_cast<const float2*>(pml + ((size_t)s * H + h) * 2))
-                      : make_float2(0.f, 0.f);
-        v[u] = s < S ? __ldcg(po + ((size_t)s * H + h) * kHeadDim + d) : 0.f;
+    if (mine) {
+      const float M = r.M[h], il = r.invL[h];
+#pragma unroll 8
+      for (int s = g; s < S; s += G) {
+        const float2 ml = __ldcg(pml + (size_t)s * H + h);
+        const float v = __ldcg(po + ((size_t)s * H + h) * kHeadDim + d);
+        if (ml.y > 0.f) acc = fmaf(exp2f(ml.x - M) * il, v, acc);
       }
-#pragma unroll
-      for (int u = 0; u < kB; ++u)
-        if (ml[u].y > 0.f) acc = fmaf(exp2f(ml[u].x - M) * il, v[u], acc);
     }
-    p.out[(size_t)bq * kOut + o] = acc;
-    if (d == 0) {
-      const double lse = r.lse2[h] * 0.69314718055994530942;
-      if (p.lse64) p.lse64[(size_t)bq * H + h] = lse;
-      if (p.lse_out) p.lse_out[(size_t)bq * H + h] = (float)lse;
+    if (G > 1) {
+      tmp[tid] = acc;
+      __syncthreads();
+      if (mine && g == 0)
+#pragma unroll 1
+        for (int g2 = 1; g2 < G; ++g2) acc += tmp[g2 * P + ol];
+      __syncthreads();
+    }
+    if (mine && g == 0) {
+      p.out[(size_t)bq * kOut + o] = acc;
+      if (d == 0) {
+        const double lse = r.lse2[h] * 0.69314718055994530942;
+        if (p.lse64) p.lse64[(size_t)bq * H + h] = lse;
+        if (p.lse_out) p.lse_out[(size_t)bq * H + h] = (float)lse;
+      }
     }
   }
 }
@@ -478,7 +462,6 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* scratch
   __shared__ float eps_s;
   __shared__ FineBins fb_s;
   __shared__ int mb_s;
-  __shared__ BinScan bs_s;
   __shared__ uint32_t red_s[2][32];
   const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = nt >> 5;
@@ -589,20 +572,27 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* scratch
   for (int e = split * nt + tid; e < kUBins; e += S * nt) gu[e] = 0u;
 
   // ---- 3. the row's fine histogram gives B, the bin of the k_sel-th largest t: keys of
-  // bins >= B + mb are in, keys of bins [B - mb, B + mb) form the band.
-  if (warp == 0) {
-    const BinScan r = scan_global_bins(gfh, p.k_sel, mb);
-    if (lane == 0) bs_s = r;
-  }
+  // bins >= B + mb are in, keys of bins [B - mb, B + mb) form the band.  (The scratch
+  // holds a copy of the histogram, then the band keys being re-scored and the per-warp K
+  // rows, later the band list being ranked.)
+  uint32_t* fhs = reinterpret_cast<uint32_t*>(scratch);
+  uint8_t* bscr = scratch + kUBinsPadded * 4;
+  double* bval = reinterpret_cast<double*>(bscr);
+  int* bl = reinterpret_cast<int*>(bscr + kBandSmem * 8);
+  float* kf = reinterpret_cast<float*>(bscr + kBandSmem * 12);
+  async_bins(fhs, gfh);
+  sm100::cp_async_wait_all();
   __syncthreads();
-  const int B = bs_s.bin;
-  const int n_band = (int)bs_s.near;
-  const int need2 = p.k_sel - (int)bs_s.above;  // taken from the band: 1 <= need2 <= n_band
+  const BinScan bs = scan_bins(fhs, p.k_sel, mb);
+  const int B = bs.bin;
+  const int n_band = (int)bs.near;
+  const int need2 = p.k_sel - (int)bs.above;  // taken from the band: 1 <= need2 <= n_band
   const bool rank_band = need2 < n_band;
   // When every band key is taken the band counts as in.
   const int in_bin = rank_band ? B + mb : B - mb;
   auto in_band = [&](int bb) { return bb >= B - mb && bb < B + mb; };
   uint32_t cin = 0, cband = 0;
+#pragma unroll 1
   for (int e = tid; e < own_n; e += nt) {
     const int bb = fb.bin(ot[e]);
     cin += bb >= in_bin;
@@ -610,27 +600,42 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* scratch
   }
   block_sum2(cin, cband);
   if (tid == 0) rowcnt[split] = cin;  // read by the higher chunks after the third barrier
-  // The float64 keys of this chunk's band keys (one warp each) go to the row's band list.
-  float* kf = reinterpret_cast<float*>(scratch);
+  // The float64 keys of this chunk's band keys go to the row's band list: up to kBandSmem
+  // at a time are listed on chip and taken by the warps in turn (one key per warp).
   if (cband) {
-    for (int c = warp * 32; c < own_n; c += nwarps * 32) {
-      const int e = c + lane;
-      const bool isb = e < own_n && in_band(fb.bin(ot[e]));
-      unsigned mask = __ballot_sync(0xffffffffu, isb);
-      while (mask) {
-        const int ee = c + __ffs(mask) - 1;
-        mask &= mask - 1;
-        const int j = oj[ee];
-        uint32_t slot = 0;
-        if (lane == 0) slot = atomicAdd(rs + kRowNBand, 1u);  // in flight while re-scoring
+    uint32_t base = 0;
+    if (tid == 0) base = atomicAdd(rs + kRowNBand, cband);  // in flight while re-scoring
+#pragma unroll 1
+    for (uint32_t r0 = 0; r0 < cband; r0 += kBandSmem) {
+      const uint32_t rn = min(cband - r0, (uint32_t)kBandSmem);
+      block_compact(
+          own_n, [&](int e) { return in_band(fb.bin(ot[e])); },
+          [&](int at, int e) {
+            if ((uint32_t)at - r0 < rn) bl[at - r0] = e;
+          });
+#pragma unroll 1
+      for (int i = warp; i < (int)rn; i += nwarps) {
+        const int j = oj[bl[i]];
         const double v = rescore_f64<H, FP8>(p.kv, p.sm_scale, (size_t)b * p.kv.max_len + j,
                                              qv.base, qv.hstride, qv.cstride, rl.dl,
                                              kf + warp * kHeadDim, lane);
-        if (lane == 0 && slot < (uint32_t)p.kv.max_len) {
-          p.band_t[rowoff + slot] = v;
-          p.band_j[rowoff + slot] = j;
+        if (lane == 0) {
+          bval[i] = v;
+          bl[i] = j;
         }
       }
+      if (tid == 0) red_s[0][0] = base;
+      __syncthreads();
+      const uint32_t at0 = red_s[0][0] + r0;
+#pragma unroll 1
+      for (int i = tid; i < (int)rn; i += nt) {
+        const uint32_t slot = at0 + (uint32_t)i;
+        if (slot < (uint32_t)p.kv.max_len) {
+          p.band_t[rowoff + slot] = bval[i];
+          p.band_j[rowoff + slot] = bl[i];
+        }
+      }
+      __syncthreads();
     }
   }
   row_arrive(rs + kRowArrive3);
@@ -656,8 +661,8 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* scratch
     };
     const int nb = min(n_band, (int)p.kv.max_len);
     if (nb <= kBandSmem) {
-      unsigned long long* bkey = reinterpret_cast<unsigned long long*>(scratch);
-      int* bpos = reinterpret_cast<int*>(scratch + kBandSmem * 8);
+      unsigned long long* bkey = reinterpret_cast<unsigned long long*>(bval);
+      int* bpos = bl;
       for (int e = tid; e < nb; e += nt) {
         bkey[e] = ordered_key64(__ldcg(gbt + e));
         bpos[e] = __ldcg(gbj + e);
@@ -737,36 +742,43 @@ __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, 
   float* us = reinterpret_cast<float*>(stage + uoff);
   int* cl = reinterpret_cast<int*>(stage + uoff + 4u * (uint32_t)piece);
   float* t2s = reinterpret_cast<float*>(stage + uoff + 8u * (uint32_t)piece);
+  uint32_t* rowmax = p.rowmax + (size_t)bq * kMaxHeads;
+  static_assert(NW * 32 * 8 <= kTailTiles * 16384, "the tail's scratch fits the tiles' space");
   bool ok = true;
   __syncthreads();
+  if (threadIdx.x < H) {
+    // This CTA's m per head joins the row's maxima (the reference of the row's lse).
+    const float2 v = __ldcg(reinterpret_cast<const float2*>(p.part_ml) +
+                            ((size_t)bq * S + split) * H + threadIdx.x);
+    if (v.y > 0.f) atomicMax(rowmax + threadIdx.x, max_key(v.x));
+  }
   if (sel_row) {
     // This chunk's first bounds on their way on chip (waited for after the barrier), and
     // the bins at or above this CTA's own k_sel-th largest u published (the row's
     // boundary bin is at least that high).
     async_words(us, p.ubuf + (size_t)bq * p.ld_u + k0, min(piece, chunk_len));
-    const int low = kth_bin_from_top(p.k_sel, uhist_s);
+    const int low = scan_bins(uhist_s, p.k_sel, 0).bin;
     add_bins(uhist_s, gu, low);
   }
   row_arrive(rs + kRowArrive1);
   if (!row_wait(rs + kRowArrive1, (uint32_t)S)) ok = false;
   if (sel_row) async_bins(uh, gu);  // in flight with the partials' loads of row_lse
-  row_lse<H>(p.part_ml + (size_t)bq * S * H * 2, S, rl);
+  row_lse<H>(p.part_ml + (size_t)bq * S * H * 2, rowmax, S, rl, reinterpret_cast<float2*>(stage));
   if (p.fuse == 2 && !sel_row && split == 0)
     write_all_positions(p.sel_idx + (size_t)bq * width, width, pos);
   if (sel_row) {
     sm100::cp_async_wait_all();
     __syncthreads();
-    const int bk = kth_bin_from_top(p.k_sel, uh);
+    const int bk = scan_bins(uh, p.k_sel, 0).bin;
     if (!row_select<H, FP8>(p, stage, us, cl, t2s, piece, bq, b, split, S, k0, c_hi, n_c, pos,
                             bk, rl, qv, recompute))
       ok = false;
   }
-  // The index set is complete and visible: the next kernel (a sparse layer reads it
-  // without waiting for this grid to end) may start while this CTA merges its share.
-  sm100::fence_acq_rel_gpu();
+  // The next kernel (a sparse layer) may be scheduled while this CTA merges its share; it
+  // waits for this grid to finish before reading the index set.
   __syncthreads();
   griddep_launch_dependents();
-  row_merge<H>(p, bq, split, S, rl);
+  row_merge<H>(p, bq, split, S, rl, reinterpret_cast<float*>(stage));
   __syncthreads();
   if (threadIdx.x == 0) {
     // The last CTA of the row to get here leaves the row's counters at zero.
@@ -777,6 +789,8 @@ __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, 
       rs[kRowArrive3] = 0u;
       rs[kRowNBand] = 0u;
       rs[kRowDone] = 0u;
+#pragma unroll 1
+      for (int hh = 0; hh < H; ++hh) rowmax[hh] = 0u;
       __threadfence();
     }
   }

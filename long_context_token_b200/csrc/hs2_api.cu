@@ -68,6 +68,7 @@ bool make_layout(int batch, int n_q, int h, int max_len, int window, int k_sel, 
   // Regions of the full layer and the selection.
   w.clear_begin = off;
   w.hist = take(bq * kHistBins * sizeof(uint32_t));
+  w.rowmax = take(bq * kMaxHeads * sizeof(uint32_t));
   w.counters = take(bq * 8 * sizeof(uint32_t));
   w.clear_end = off;
   w.selmeta = take(bq * 4 * sizeof(uint32_t));
@@ -205,6 +206,7 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
     p.ld_u = w.ld_u;
     p.uhist = ws_ptr<uint32_t>(ws, w.hist);
     p.rowsync = ws_ptr<uint32_t>(ws, w.counters);
+    p.rowmax = ws_ptr<uint32_t>(ws, w.rowmax);
     p.cand_t = ws_ptr<float>(ws, w.cand_t);
     p.cand_j = ws_ptr<int32_t>(ws, w.cand_j);
     p.band_t = ws_ptr<double>(ws, w.band_t);

@@ -31,6 +31,7 @@ struct WsLayout {
   size_t status = 0;      // u32 status word; never cleared by a compute call
   size_t clear_begin = 0; // [clear_begin, clear_end) is zeroed by every full-layer call
   size_t hist = 0;        // u32 [bq][kHistBins]
+  size_t rowmax = 0;      // u32 [bq][kMaxHeads] per-head maxima of a row's split partials (fused tail)
   size_t counters = 0;    // u32 [bq][8]: 0 direct, 1 cand, 2 band
   size_t clear_end = 0;
   size_t selmeta = 0;     // u32 [bq][4]: bin, eps bits, k_eff, n_c
@@ -104,6 +105,7 @@ struct FullParams {
   float* ubuf = nullptr;         // [bq][ld_u]: per-key bound u_j = max_h x_hj (log2 units)
   int ld_u = 0;
   uint32_t* uhist = nullptr;     // [bq][kHistBins]: the u histogram, then the fine one
+  uint32_t* rowmax = nullptr;    // [bq][kMaxHeads]: ordered keys of the row's largest m per head
   uint32_t* rowsync = nullptr;   // [bq][8]: arrival counters and the band list's length
   float* cand_t = nullptr;       // [bq][ld_u] candidates of long chunks, at the chunk's offset: keys ...
   int32_t* cand_j = nullptr;     // [bq][ld_u] ... and positions
