@@ -107,6 +107,15 @@ typedef struct hs2_kv {
 HS2_API size_t hs2_workspace_bytes(int batch, int n_q, int h_q, int max_len, int window,
                            int k_sel, int dtype);
 
+/* Byte offset, within a workspace of these sizes, of the float64 log-sum-exp that the
+ * full layer leaves there: double [batch][n_q][h_q], natural log, the values the token
+ * selection shifts the heads' scores by.  Valid after hs2_full_attn or
+ * hs2_full_attn_select until the next call that uses the workspace.  (size_t)-1 if the
+ * sizes are unsupported.  A diagnostic: the `lse` output of those calls is the same
+ * value rounded to float32. */
+HS2_API size_t hs2_workspace_lse64_offset(int batch, int n_q, int h_q, int max_len,
+                                          int window, int k_sel, int dtype);
+
 /* Full-attention layer + token selection (steps 1 and 2).
  *   q        device bf16 [batch][n_q][h_q][128].
  *   sm_scale softmax scale applied to q.k (normally 1/sqrt(128) as float32).
@@ -197,25 +206,31 @@ HS2_API hs2_status hs2_prefill_attn(const void* q, int n_q, int h_q, const hs2_k
  * Overlap: the layer's kernel may start while the previous kernel on the stream is
  * still finishing when that kernel is this library's (programmatic dependent launch);
  * it reads q_layer, idx and the cache right away and waits for that kernel to end only
- * before writing `out`.  No library call writes those inputs except hs2_select /
- * hs2_full_attn_select, which complete the index set before the next kernel may start.
+ * before writing `out`.  The library calls that write those inputs (hs2_select and
+ * hs2_full_attn_select the index set, hs2_kv_append the cache rows and lengths) finish
+ * those writes before they let the next kernel start.
  * After any other kernel (not this library's) the layer starts when it has ended. */
 HS2_API hs2_status hs2_sparse_attn(const void* q_layer, int n_q, int h_q, const hs2_kv* kv,
                            const int32_t* idx, int idx_width, float sm_scale, float* out,
                            void* workspace, size_t ws_bytes, hs2_stream_t stream);
 
 /* One reusing sparse-attention layer for callers that cannot allocate device memory
- * (no counterpart in the paper; a deployment aid).  It computes exactly what
- * hs2_sparse_attn computes, with the same arguments except the workspace: its scratch
+ * (no counterpart in the paper; a deployment aid).  It computes the same layer as
+ * hs2_sparse_attn, within the same tolerances (for h_q <= 64 with a different kernel:
+ * CUDA-core gathers and a separate split merge), with the same arguments except the
+ * workspace: its scratch
  * (the split partials) lives in a fixed 4 MiB array inside the library,
  * which every GPU that loads the library keeps until the process exits.  Callers that
  * hand out all device memory from their own pool, or that must not call cudaMalloc
  * mid-step (it can synchronise the device), use this entry point.
  *   device_status  device uint32 into which the kernels OR (1 << code) for each
- *                  device-side error (HS2_ERR_INDEX_OUT_OF_RANGE, HS2_ERR_BAD_LENGTH);
- *                  may be NULL to discard them.  The caller clears it.
+ *                  device-side error (HS2_ERR_INDEX_OUT_OF_RANGE: an index outside
+ *                  [-1, lens[b]); lengths outside [n_q, max_len] are clamped without a
+ *                  report).  The caller clears it.  May be NULL: the errors then
+ *                  accumulate in a word of the library's array that nothing reads or
+ *                  clears.
  * Limit: 256 + B*n_q*ceil(idx_width/64)*h_q*520 bytes (two regions, each rounded up to
- * 256) must fit in 4 MiB, e.g. B*n_q*h_q <= 384 at idx_width 1152;
+ * 256) must fit in 4 MiB, e.g. B*n_q*h_q <= 448 at idx_width 1152;
  * larger sizes return HS2_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress)
  * and should come before any stream capture on that device.  All calls on a device
@@ -245,9 +260,25 @@ HS2_API hs2_status hs2_kv_append(const void* k_new, const void* v_new, int n_new
                                  const hs2_kv* kv, int32_t* lens, void* workspace,
                                  size_t ws_bytes, hs2_stream_t stream);
 
-/* Synchronises `stream`, returns the first error recorded by the kernels since the
- * last check (HS2_OK if none) and clears it. */
+/* Synchronises `stream` and returns an error the kernels recorded since the last check
+ * (HS2_OK if none), then clears them all.  Each kind of error sets its own bit of the
+ * workspace's status word, so when several kinds were recorded the call returns the
+ * lowest-numbered code among them (the order of hs2_status, not the order in time).
+ * After HS2_ERR_DEVICE_TIMEOUT the workspace's contents are undefined: zero-fill it again
+ * before the next call that uses it. */
 HS2_API hs2_status hs2_check_device_status(void* workspace, hs2_stream_t stream);
+
+/* Test hook for the error path of the bounded device-side waits; not for production.
+ *   mode 1: the bf16 one-token full-layer kernel issues no loads and no MMAs, so its
+ *           softmax warps' first wait on an MMA result runs out (after about 10 us);
+ *   mode 2: the fused selection tail's row barriers wait for one CTA more than the row
+ *           has, so each runs out (after about 10 us);
+ *   mode 0: normal operation (the default).
+ * A wait that runs out records HS2_ERR_DEVICE_TIMEOUT and the kernel finishes with no
+ * copy or MMA of its own in flight; outputs are then undefined and the workspace must be
+ * zero-filled again before its next use.  The setting is process-wide, applies to the
+ * launches that follow, and is not synchronised between host threads. */
+HS2_API void hs2_debug_stall_waits(int mode);
 
 /* Static description of a status code (never NULL). */
 HS2_API const char* hs2_status_string(hs2_status status);

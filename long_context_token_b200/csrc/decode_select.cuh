@@ -98,14 +98,17 @@ __device__ __forceinline__ void row_arrive(uint32_t* counter) {
   __syncthreads();
   if (threadIdx.x == 0) sm100::red_release_gpu_add(counter, 1u);
 }
-static __device__ __noinline__ bool row_wait(uint32_t* counter, uint32_t target) {
+// `stall` (the stall test) waits for one CTA more than the row has, with a short limit.
+static __device__ __noinline__ bool row_wait(uint32_t* counter, uint32_t target, bool stall) {
   __shared__ uint32_t ok_s;
   if (threadIdx.x == 0) {
     uint32_t ok = 1;
+    const long long limit = stall ? kStallTestCycles : kRowSpinCycles;
+    target += stall ? 1u : 0u;
     if (sm100::ld_acquire_gpu_u32(counter) < target) {
       const long long t0 = clock64();
       while (sm100::ld_acquire_gpu_u32(counter) < target) {
-        if (clock64() - t0 > kRowSpinCycles) {
+        if (clock64() - t0 > limit) {
           ok = 0;
           break;
         }
@@ -565,7 +568,7 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* scratch
     own_n += ncl;
   }
   row_arrive(rs + kRowArrive2);
-  if (!row_wait(rs + kRowArrive2, (uint32_t)S)) ok = false;
+  if (!row_wait(rs + kRowArrive2, (uint32_t)S, p.stall_test == 2)) ok = false;
   // Every CTA of the row has its copy of the u histogram by now (each copied it before
   // arriving): clear this CTA's share for the next call.
   uint32_t* gu = p.uhist + (size_t)bq * kHistBins;
@@ -639,7 +642,7 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* scratch
     }
   }
   row_arrive(rs + kRowArrive3);
-  if (!row_wait(rs + kRowArrive3, (uint32_t)S)) ok = false;
+  if (!row_wait(rs + kRowArrive3, (uint32_t)S, p.stall_test == 2)) ok = false;
   // Every CTA has read the fine histogram: clear this CTA's share for the next call.
   for (int e = split * nt + tid; e < kUBins; e += S * nt) gfh[e] = 0u;
 
@@ -761,7 +764,7 @@ __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, 
     add_bins(uhist_s, gu, low);
   }
   row_arrive(rs + kRowArrive1);
-  if (!row_wait(rs + kRowArrive1, (uint32_t)S)) ok = false;
+  if (!row_wait(rs + kRowArrive1, (uint32_t)S, p.stall_test == 2)) ok = false;
   if (sel_row) async_bins(uh, gu);  // in flight with the partials' loads of row_lse
   row_lse<H>(p.part_ml + (size_t)bq * S * H * 2, rowmax, S, rl, reinterpret_cast<float2*>(stage));
   if (p.fuse == 2 && !sel_row && split == 0)
@@ -774,8 +777,9 @@ __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, 
                             bk, rl, qv, recompute))
       ok = false;
   }
-  // The next kernel (a sparse layer) may be scheduled while this CTA merges its share; it
-  // waits for this grid to finish before reading the index set.
+  // The index set is complete and visible: the next kernel (a sparse layer, which reads
+  // it before waiting for this grid to end) may start while this CTA merges its share.
+  sm100::fence_acq_rel_gpu();
   __syncthreads();
   griddep_launch_dependents();
   row_merge<H>(p, bq, split, S, rl, reinterpret_cast<float*>(stage));

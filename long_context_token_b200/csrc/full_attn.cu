@@ -27,6 +27,7 @@ __global__ void __launch_bounds__(kThreads) full_attn_simt_kernel(FullParams p) 
   for (int hd = threadIdx.x; hd < H; hd += kThreads) {
     s.m_run[hd] = -INFINITY;
     s.l_run[hd] = 0.f;
+    s.l_err[hd] = 0.f;
   }
   float acc[H / 2];
 #pragma unroll

@@ -313,7 +313,8 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
         const uint64_t pol = policy_evict_first();
         const int row0 = b * p.kv.max_len + k0;
         int issued = 0;
-        for (int i = 0; i < n_tiles && ok; ++i) {
+        const bool stall = p.stall_test == 1;  // the stall test issues no load
+        for (int i = 0; i < n_tiles && ok && !stall; ++i) {
           const int s = i % NS;
           const uint32_t ph = ((i / NS) & 1) ^ 1;
           const int row = row0 + i * kKeyTile;
@@ -358,6 +359,7 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
           mma_commit(vempty + s);
           return true;
         };
+        if (!GATHER && p.stall_test == 1) ok = false;  // the stall test issues no MMA
         for (int i = 0; i < n_tiles && ok; ++i) {
           const int s = i % NS, sb = i & 1;
           if (!mbar_wait(kfull + s, (i / NS) & 1)) { ok = false; break; }
@@ -396,7 +398,8 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
         // A failed wait in any softmax thread stops the waits of all of them (they
         // keep taking part in the named barriers, so none is left behind).
         const int sb = i & 1;
-        if (ok && !mbar_wait(s_full + sb, (i >> 1) & 1)) ok = false;
+        const long long limit = !GATHER && p.stall_test == 1 ? kStallTestCycles : kWaitCycles;
+        if (ok && !mbar_wait(s_full + sb, (i >> 1) & 1, limit)) ok = false;
         if (named_bar_or(3, 128, !ok)) ok = false;
         tc_fence_after();
         float x[H];

@@ -24,6 +24,9 @@ constexpr int kTargetCtas = 4 * 148;
 constexpr int kMinChunk = 256;
 constexpr int kChunk4 = 64;
 
+// The bounded-wait test hook (hs2_debug_stall_waits): copied into every full-layer launch.
+static int g_stall_test = 0;
+
 // `row_ctas`: CTAs of one key chunk across the batch (one per (sequence, token) row,
 // or per group of G tokens in the several-token kernel).
 int plan_splits1(int row_ctas, int max_len, int /*num_sms*/) {
@@ -197,6 +200,7 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
   p.part_o = ws_ptr<float>(ws, w.part1_o);
   p.part_ml = ws_ptr<float>(ws, w.part1_ml);
   p.status = ws_ptr<uint32_t>(ws, w.status);
+  p.stall_test = g_stall_test;
   if (fused_full_layer(kv, n_q, h)) {
     p.fuse = idx ? 2 : 1;
     p.out = out;
@@ -442,6 +446,17 @@ size_t hs2_workspace_bytes(int batch, int n_q, int h_q, int max_len, int window,
   WsLayout w;
   make_layout(batch, n_q, h_q, max_len, window, k_sel, dtype, &w);
   return w.total;
+}
+
+void hs2_debug_stall_waits(int mode) { g_stall_test = mode == 1 || mode == 2 ? mode : 0; }
+
+size_t hs2_workspace_lse64_offset(int batch, int n_q, int h_q, int max_len, int window,
+                                  int k_sel, int dtype) {
+  if (hs2_workspace_bytes(batch, n_q, h_q, max_len, window, k_sel, dtype) == 0)
+    return ~(size_t)0;
+  WsLayout w;
+  make_layout(batch, n_q, h_q, max_len, window, k_sel, dtype, &w);
+  return w.lse64;
 }
 
 hs2_status hs2_full_attn(const void* q, int n_q, int h_q, const hs2_kv* kv, int window,

@@ -16,6 +16,7 @@ constexpr int kChunk3Keys = 8192;      // keys per CTA of the compaction pass
 constexpr int kMaxIdxWidth = 4096;      // window + k_sel
 constexpr int kMaxNq = 64;
 constexpr int kMaxHeads = 128;
+constexpr long long kStallTestCycles = 20000;  // the stall test's wait limit
 constexpr int kSmCountBound = 160;      // workspace sizing assumes at most this many SMs
 
 // Status bits kept in the workspace's status word (one bit per hs2_status code).
@@ -100,6 +101,11 @@ struct FullParams {
   //           and lse64 (no separate merge kernel);
   //   fuse 2: the same, plus the token selection of the row into sel_idx.
   int fuse = 0;
+  // Test hook for the bounded waits (hs2_debug_stall_waits): 1 = the bf16 one-token kernel
+  // issues no loads or MMAs and its softmax warps' first wait gives up after
+  // kStallTestCycles; 2 = the fused tail's row barriers wait for one CTA more than the row
+  // has, each giving up after kStallTestCycles.
+  int stall_test = 0;
   float* lse_out = nullptr;      // [bq][h] or null
   double* lse64 = nullptr;       // [bq][h]
   float* ubuf = nullptr;         // [bq][ld_u]: per-key bound u_j = max_h x_hj (log2 units)

@@ -5,7 +5,8 @@
 // row's E4M3 codes and its per-token scale s = amax / 448 (code = x / s rounded to
 // nearest even with saturation, both divisions IEEE float32; an all-zero row gets
 // s = 1).  The CTA reads the sequence's length once and grows it after every row is
-// written, so no other CTA reads or writes that length.
+// written, so no other CTA reads or writes that length.  The next kernel may start only
+// once every CTA has written its rows and length.
 #include <cuda_fp8.h>
 
 #include "hs2_internal.cuh"
@@ -16,14 +17,13 @@ constexpr int kAppendThreads = 256;
 
 __global__ void __launch_bounds__(kAppendThreads) kv_append_kernel(AppendParams p) {
   griddep_wait();  // earlier kernels may still read the lengths and the cache
-  griddep_launch_dependents();
   const int b = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int L = p.lens[b];
   const bool fits = L >= 0 && L + p.n_new <= p.max_len;
   if (!fits) {
     if (threadIdx.x == 0) set_status(p.status, HS2_ERR_BAD_LENGTH);
-    return;
+    return;  // (an exiting CTA counts as having let the next kernel start)
   }
   const int rows = 2 * p.n_new;  // K then V of each new token
   for (int r = warp; r < rows; r += kAppendThreads / 32) {
@@ -52,6 +52,11 @@ __global__ void __launch_bounds__(kAppendThreads) kv_append_kernel(AppendParams 
   }
   __syncthreads();
   if (threadIdx.x == 0) p.lens[b] = L + p.n_new;
+  // The next kernel may read the lengths and the cache before it waits for this one (the
+  // tensor-core sparse layer does): only the complete, visible rows and lengths let it start.
+  __threadfence();
+  __syncthreads();
+  griddep_launch_dependents();
 }
 
 cudaError_t launch_kv_append(const AppendParams& p, int batch, cudaStream_t st) {

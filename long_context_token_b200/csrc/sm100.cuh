@@ -59,8 +59,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Waits for the phase with the given parity to complete.  Gives up after about
 // `limit_cycles` SM clocks and returns false (the caller records a timeout and
 // winds down); never spins forever.
+constexpr long long kWaitCycles = 4000000000ll;  // about two seconds at the boost clock
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          long long limit_cycles = 4000000000ll) {
+                                          long long limit_cycles = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {

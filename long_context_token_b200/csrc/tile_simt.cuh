@@ -17,7 +17,7 @@ __host__ __device__ constexpr size_t simt_smem_bytes(int H) {
                           + kTile * kKsLd            // K tile
                           + kTile * kHeadDim         // V tile
                           + (size_t)H * kTile        // S / P tile
-                          + 3 * (size_t)H)           // m, l, alpha
+                          + 4 * (size_t)H)           // m, l (two floats), alpha
          + sizeof(int) * kTile;                      // row index of each tile row
 }
 
@@ -28,6 +28,7 @@ struct SimtSmem {
   float* S;
   float* m_run;
   float* l_run;
+  float* l_err;  // trailing float of l (l = l_run + l_err, summed without loss)
   float* alpha;
   int* rowidx;
 };
@@ -40,7 +41,8 @@ __device__ __forceinline__ SimtSmem carve_simt(float* sm, int H) {
   s.S = s.vs + kTile * kHeadDim;
   s.m_run = s.S + H * kTile;
   s.l_run = s.m_run + H;
-  s.alpha = s.l_run + H;
+  s.l_err = s.l_run + H;
+  s.alpha = s.l_err + H;
   s.rowidx = reinterpret_cast<int*>(s.alpha + H);
   return s;
 }
@@ -119,18 +121,25 @@ __device__ __forceinline__ void qk_tile(const SimtSmem& s) {
   for (int r = 0; r < R; ++r) s.S[(hg + 8 * r) * kTile + key] = valid ? acc[r] : -INFINITY;
 }
 
-// Online-softmax update of one tile: S <- exp(S - m_new), l and alpha updated.
+// Online-softmax update of one tile: S <- exp(S - m), l and alpha updated.  The
+// reference m moves only when a logit exceeds it by more than kLazyRescale (or on the
+// first key), so l and O are rescaled a handful of times per chunk, and l is summed
+// without loss (two-sum): the partial's l carries little more than the rounding of the
+// exponentials, which the float64 lse of the selection relies on.
+constexpr float kLazyRescale = 8.f;  // p <= e^8 between rescales
 template <int H>
 __device__ __forceinline__ void softmax_tile(const SimtSmem& s) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   for (int hd = w; hd < H; hd += kThreads / 32) {
     const float x = s.S[hd * kTile + lane];
     const float m_old = s.m_run[hd];
-    const float m_new = fmaxf(m_old, warp_max(x));
+    const float tmax = warp_max(x);
+    const float m_new = (m_old == -INFINITY || tmax > m_old + kLazyRescale) ? fmaxf(m_old, tmax)
+                                                                           : m_old;
     float pr = 0.f, al = 1.f;
     if (m_new != -INFINITY) {
       pr = expf(x - m_new);
-      al = expf(m_old - m_new);
+      if (m_new != m_old) al = expf(m_old - m_new);
     }
     const float sum = warp_sum(pr);
     s.S[hd * kTile + lane] = pr;
@@ -138,7 +147,11 @@ __device__ __forceinline__ void softmax_tile(const SimtSmem& s) {
     if (lane == 0) {
       s.alpha[hd] = al;
       s.m_run[hd] = m_new;
-      s.l_run[hd] = s.l_run[hd] * al + sum;
+      float l = s.l_run[hd] * al, e = s.l_err[hd] * al;
+      const float t = l + sum, bp = t - l;
+      e += (l - (t - bp)) + (sum - bp);
+      s.l_run[hd] = t;
+      s.l_err[hd] = e;
     }
   }
 }
@@ -196,7 +209,7 @@ __device__ __forceinline__ void write_partial(const SimtSmem& s, const float* ac
   for (int r = 0; r < H / 2; ++r) part_o[(hg2 + 2 * r) * kHeadDim + d] = acc[r];
   for (int hd = threadIdx.x; hd < H; hd += kThreads) {
     part_ml[2 * hd] = s.m_run[hd];
-    part_ml[2 * hd + 1] = s.l_run[hd];
+    part_ml[2 * hd + 1] = s.l_run[hd] + s.l_err[hd];
   }
 }
 

@@ -37,7 +37,8 @@ EXPORTS = ("hs2_workspace_bytes", "hs2_full_attn_select", "hs2_full_attn", "hs2_
            "hs2_sparse_attn", "hs2_check_device_status", "hs2_status_string",
            "hs2_last_cuda_error", "hs2_abi_version", "hs2_sparse_attn_noalloc", "hs2_kv_append",
            "hs2_full_attn_select_blocks", "hs2_select_blocks", "hs2_prefill_workspace_bytes",
-           "hs2_prefill_attn", "hs2_select_fused")
+           "hs2_prefill_attn", "hs2_select_fused", "hs2_workspace_lse64_offset",
+           "hs2_debug_stall_waits")
 
 
 class Hs2Error(RuntimeError):
@@ -108,6 +109,10 @@ def lib():
     L.hs2_abi_version.restype = i32
     L.hs2_select_fused.argtypes = [i32, i32, i32]
     L.hs2_select_fused.restype = i32
+    L.hs2_workspace_lse64_offset.argtypes = [i32] * 7
+    L.hs2_workspace_lse64_offset.restype = sz
+    L.hs2_debug_stall_waits.argtypes = [i32]
+    L.hs2_debug_stall_waits.restype = None
     _lib = L
     return L
 
@@ -200,6 +205,18 @@ def default_scale() -> float:
 def select_fused(cache: "Cache", n_q: int, h_q: int) -> bool:
     """True if full_attn_select runs as one kernel for these sizes (hs2_select_fused)."""
     return bool(lib().hs2_select_fused(n_q, h_q, cache.dtype))
+
+
+def workspace_lse64(workspace: torch.Tensor, cache: "Cache", n_q: int, h_q: int,
+                    window: int = 128, k_sel: int = 1024) -> torch.Tensor:
+    """The float64 lse [batch, n_q, h_q] that the last full layer left in `workspace`
+    (a view, not a copy; hs2_workspace_lse64_offset)."""
+    off = lib().hs2_workspace_lse64_offset(cache.batch, n_q, h_q, cache.max_len, window,
+                                           k_sel, cache.dtype)
+    if off == (1 << 64) - 1:
+        raise Hs2Error(2, "hs2_workspace_lse64_offset")
+    n = cache.batch * n_q * h_q * 8
+    return workspace[off:off + n].view(torch.float64).view(cache.batch, n_q, h_q)
 
 
 def full_attn_select(q: torch.Tensor, cache: Cache, window: int = 128, k_sel: int = 1024,

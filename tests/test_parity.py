@@ -2,7 +2,8 @@
 
 Index sets must equal the oracle's except inside the tie band (gap between the
 k-th and (k+1)-th importance below 1e-6 relative); outputs within max-abs 2e-3
-(bf16 cache) or 1e-2 (FP8 cache); lse within 1e-4.
+(bf16 cache) or 1e-2 (FP8 cache); lse within 1e-4, and the float64 lse that the
+selection uses within 1e-6.
 """
 from __future__ import annotations
 
@@ -18,6 +19,7 @@ pytestmark = [pytest.mark.gpu, pytest.mark.filterwarnings("ignore::RuntimeWarnin
 
 TOL = {"bf16": 2e-3, "fp8": 1e-2}
 LSE_TOL = 1e-4
+LSE64_TOL = 1e-6
 
 
 def run_gpu(inp: workloads.Inputs, twice: bool = False):
@@ -30,10 +32,12 @@ def run_gpu(inp: workloads.Inputs, twice: bool = False):
     runs = []
     for _ in range(2 if twice else 1):
         out, idx, lse = hs2.full_attn_select(q, cache, inp.window, inp.k_sel, inp.sm_scale, ws)
+        lse64 = hs2.workspace_lse64(ws, cache, inp.n_q, inp.h_q, inp.window, inp.k_sel)
+        lse64 = lse64.cpu().numpy()  # before the sparse layers reuse the workspace
         sp = [hs2.sparse_attn(ql.to(dev), cache, idx, ws, inp.sm_scale) for ql in inp.q_layers]
         torch.cuda.synchronize()
         runs.append(dict(out=out.cpu().numpy(), idx=idx.cpu().numpy(), lse=lse.cpu().numpy(),
-                         sparse=[s.cpu().numpy() for s in sp]))
+                         lse64=lse64, sparse=[s.cpu().numpy() for s in sp]))
     status = hs2.check_device_status(ws)
     return runs, status
 
@@ -50,6 +54,11 @@ def compare_bits(bits: dict, res: dict, sparse_full: bool = True):
     assert err < tol, f"full-layer output max-abs error {err}"
     lerr = np.abs(res["lse"] - ref["lse"]).max()
     assert lerr < LSE_TOL, f"lse error {lerr}"
+    if "lse64" in res:
+        # The float64 lse that the selection shifts each head's scores by: its error moves
+        # the ranking directly, so it is held to the selection's tie band.
+        l64 = np.abs(res["lse64"].reshape(ref["lse"].shape) - ref["lse"]).max()
+        assert l64 <= LSE64_TOL, f"float64 lse error {l64}"
     B, n_q = bits["q"].shape[:2]
     window, k_sel = bits["window"], bits["k_sel"]
     n_exact = 0
@@ -105,6 +114,15 @@ SMALL = [
          lens=[1509, 1402]),
     dict(id="append2-fp8-h64-odd", batch=3, max_len=2001, n_q=2, h_q=64, kv="fp8", seed=117,
          lens=[2001, 1999, 1200]),
+    # shapes served by the CUDA-core kernels: FP8 with more than 64 heads, one-token bf16
+    # with 80, 96 or 112 heads
+    dict(id="h128-fp8-cuda-core", batch=2, max_len=2500, n_q=1, h_q=128, kv="fp8", seed=118,
+         lens=[2500, 1777]),
+    dict(id="h96-fp8-append2-cuda-core", batch=1, max_len=1900, n_q=2, h_q=96, kv="fp8",
+         seed=119),
+    dict(id="h80-bf16-cuda-core", batch=2, max_len=3000, n_q=1, h_q=80, kv="bf16", seed=120,
+         lens=[3000, 2111]),
+    dict(id="h112-bf16-cuda-core", batch=1, max_len=2300, n_q=1, h_q=112, kv="bf16", seed=121),
 ]
 
 
