@@ -756,16 +756,19 @@ __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, 
     if (v.y > 0.f) atomicMax(rowmax + threadIdx.x, max_key(v.x));
   }
   if (sel_row) {
-    // This chunk's first bounds on their way on chip (waited for after the barrier), and
-    // the bins at or above this CTA's own k_sel-th largest u published (the row's
+    // The bins at or above this CTA's own k_sel-th largest u published (the row's
     // boundary bin is at least that high).
-    async_words(us, p.ubuf + (size_t)bq * p.ld_u + k0, min(piece, chunk_len));
     const int low = scan_bins(uhist_s, p.k_sel, 0).bin;
     add_bins(uhist_s, gu, low);
   }
   row_arrive(rs + kRowArrive1);
   if (!row_wait(rs + kRowArrive1, (uint32_t)S, p.stall_test == 2)) ok = false;
-  if (sel_row) async_bins(uh, gu);  // in flight with the partials' loads of row_lse
+  if (sel_row) {
+    // In flight with the partials' loads of row_lse: the row's u histogram and this
+    // chunk's first bounds (whichever CTA streamed those keys).
+    async_bins(uh, gu);
+    async_words(us, p.ubuf + (size_t)bq * p.ld_u + k0, min(piece, chunk_len));
+  }
   row_lse<H>(p.part_ml + (size_t)bq * S * H * 2, rowmax, S, rl, reinterpret_cast<float2*>(stage));
   if (p.fuse == 2 && !sel_row && split == 0)
     write_all_positions(p.sel_idx + (size_t)bq * width, width, pos);
@@ -793,6 +796,7 @@ __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, 
       rs[kRowArrive3] = 0u;
       rs[kRowNBand] = 0u;
       rs[kRowDone] = 0u;
+      rs[kRowTileSlot] = 0u;
 #pragma unroll 1
       for (int hh = 0; hh < H; ++hh) rowmax[hh] = 0u;
       __threadfence();

@@ -50,10 +50,11 @@ struct FullSmem {
   static constexpr uint32_t kRedOff = kPOff + 4 * kPBytes;  // [4 warps][H] floats
   static constexpr uint32_t kRefOff = kRedOff + 4 * H * 4;  // [H] reference, [H] alpha
   static constexpr uint32_t kBarOff = kRefOff + 2 * H * 4;
-  static constexpr uint32_t kBars = 4 * kStages + 10;
+  static constexpr uint32_t kBars = 4 * kStages + 10 + kTileRing;
   static constexpr uint32_t kSlotOff = kBarOff + kBars * 8;
+  static constexpr uint32_t kRingOff = kSlotOff + 16;  // [kTileRing] tile indices
   // Histogram of the selection bounds u (full layer only).
-  static constexpr uint32_t kUHistOff = (kSlotOff + 16 + 15) / 16 * 16;  // 16-byte aligned
+  static constexpr uint32_t kUHistOff = (kRingOff + 4 * kTileRing + 15) / 16 * 16;
   static constexpr uint32_t kUHistBytes = GATHER ? 0u : (uint32_t)kUBinsPadded * 4u;
   static constexpr uint32_t kBytes = kUHistOff + kUHistBytes + 1024;
   static constexpr uint32_t kTmemCols = tmem_cols_pow2(3 * H);
@@ -186,7 +187,9 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
   uint64_t* p_free = s_full + 6;         // [2]
   uint64_t* mma_done = s_full + 8;
   uint64_t* post_bar = s_full + 9;  // MMAs of the selection tail
+  uint64_t* idx_bar = s_full + 10;  // [kTileRing] one per slot of the tile-index ring
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
+  int* tile_ring = reinterpret_cast<int*>(smem + L::kRingOff);
   uint32_t* uhist_s = reinterpret_cast<uint32_t*>(smem + L::kUHistOff);
 
   const int warp = threadIdx.x >> 5;
@@ -209,6 +212,7 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
     }
     mbar_init(mma_done, 1);
     mbar_init(post_bar, 1);
+    for (int r = 0; r < kTileRing; ++r) mbar_init(idx_bar + r, 1);
     fence_mbar_init();
   }
   if (!GATHER)
@@ -240,7 +244,17 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
   const int k1 = GATHER ? min(k0 + p.chunk1, p.idx_width) : min(k0 + p.chunk1, pos + 1);
   const int32_t* idx_row = GATHER ? p.idx + (size_t)bq * p.idx_width : nullptr;
   const size_t row_base = (size_t)b * p.kv.max_len;
-  const int n_tiles = k0 < k1 ? (k1 - k0 + kKeyTile - 1) / kKeyTile : 0;
+  // Fused full layer with several CTAs a row: the row's tiles are shared out at run time
+  // (CTA r takes tiles r, r + S, ..., r + (NS - 1) S, then claims the next free tile
+  // from the row's counter until none is left), so that CTAs slowed by the memory
+  // system take fewer tiles and the row's CTAs reach its first barrier together.  The
+  // selection keeps its static ownership of positions (chunk r), whoever read them.
+  const int S = p.splits1;
+  const bool dyn = !GATHER && p.fuse != 0 && S > 1;
+  const int row_tiles = (pos + 1 + kKeyTile - 1) / kKeyTile;
+  const int n_tiles = dyn ? (split < row_tiles ? 1 : 0)  // (only whether any)
+                          : (k0 < k1 ? (k1 - k0 + kKeyTile - 1) / kKeyTile : 0);
+  const int k_end = dyn ? pos + 1 : k1;  // keys at or past this one are masked
   const size_t pidx = (size_t)bq * p.splits1 + split;
   // Cluster mode keeps the partial in this CTA's shared memory (the K stages, idle by
   // the time the partial is written) for the on-chip merge.
@@ -310,15 +324,28 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
     } else if (warp == 0) {
       // ------------------------------------------------------------ TMA producer
       if (elect_one()) {
+        // Tile i's index goes to slot i of the ring (its barrier arrived on) before the
+        // tile's loads; past the last tile an index of -1 ends the MMA warp's and the
+        // softmax warps' loops.  (The stage barriers see loads only: their phases stay in
+        // step with the tiles, which the wait for the last loads below relies on.)
         const uint64_t pol = policy_evict_first();
-        const int row0 = b * p.kv.max_len + k0;
+        const int row_b = b * p.kv.max_len;
+        uint32_t* row_counter = p.rowsync + (size_t)bq * 8 + kRowTileSlot;
+        uint32_t claimed = 0;
         int issued = 0;
         const bool stall = p.stall_test == 1;  // the stall test issues no load
-        for (int i = 0; i < n_tiles && ok && !stall; ++i) {
+        for (int i = 0; ok && !stall; ++i) {
           const int s = i % NS;
           const uint32_t ph = ((i / NS) & 1) ^ 1;
-          const int row = row0 + i * kKeyTile;
+          const int tile = dyn ? (i < NS ? split + i * S : NS * S + (int)claimed)
+                               : (i < n_tiles ? k0 / kKeyTile + i : -1);
+          const bool end = tile < 0 || tile >= row_tiles || (!dyn && i >= n_tiles);
           if (!mbar_wait(kempty + s, ph)) { ok = false; break; }
+          tile_ring[i % kTileRing] = end ? -1 : tile;
+          mbar_arrive(idx_bar + i % kTileRing);
+          if (end) break;
+          if (dyn && i + 1 >= NS) claimed = atomicAdd(row_counter, 1u);  // tile i + 1's
+          const int row = row_b + tile * kKeyTile;
           mbar_arrive_expect_tx(kfull + s, L::kTile);
           tma_load_2d(kst + s * L::kTile, &tmap_k, kfull + s, 0, row, pol);
           tma_load_2d(kst + s * L::kTile + kBoxBytes, &tmap_k, kfull + s, 64, row, pol);
@@ -360,9 +387,15 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
           return true;
         };
         if (!GATHER && p.stall_test == 1) ok = false;  // the stall test issues no MMA
-        for (int i = 0; i < n_tiles && ok; ++i) {
+        int n_done = 0;
+        for (int i = 0; (GATHER ? i < n_tiles : true) && ok; ++i) {
           const int s = i % NS, sb = i & 1;
+          if (!GATHER) {  // the tile's index first (-1: past the last tile)
+            if (!mbar_wait(idx_bar + i % kTileRing, (i / kTileRing) & 1)) { ok = false; break; }
+            if (tile_ring[i % kTileRing] < 0) break;
+          }
           if (!mbar_wait(kfull + s, (i / NS) & 1)) { ok = false; break; }
+          n_done = i + 1;
           if (!mbar_wait(s_free + sb, ((i >> 1) & 1) ^ 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t k_addr = smem_u32(kst + s * L::kTile);
@@ -374,7 +407,7 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
           mma_commit(kempty + s);
           if (i > 0 && !issue_pv(i - 1)) { ok = false; break; }
         }
-        if (ok && !issue_pv(n_tiles - 1)) ok = false;
+        if (ok && n_done > 0 && !issue_pv(n_done - 1)) ok = false;
         mma_commit(mma_done);
         if (!mbar_wait(mma_done, 0)) ok = false;
       }
@@ -394,12 +427,22 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
       for (int h = 0; h < H; ++h) l[h] = 0.f;
       if (t < H) mref_s[t] = -INFINITY;
       named_bar_sync(1, 128);
-      for (int i = 0; i < n_tiles; ++i) {
+      int n_done = 0;
+      for (int i = 0; GATHER ? i < n_tiles : true; ++i) {
         // A failed wait in any softmax thread stops the waits of all of them (they
-        // keep taking part in the named barriers, so none is left behind).
+        // keep taking part in the named barriers, so none is left behind).  Without
+        // gathers the tile comes from the producer's ring (-1: no more tiles).
         const int sb = i & 1;
-        const long long limit = !GATHER && p.stall_test == 1 ? kStallTestCycles : kWaitCycles;
-        if (ok && !mbar_wait(s_full + sb, (i >> 1) & 1, limit)) ok = false;
+        int tile = k0 / kKeyTile + i;
+        if (!GATHER) {
+          const long long limit = p.stall_test == 1 ? kStallTestCycles : kWaitCycles;
+          if (ok && !mbar_wait(idx_bar + i % kTileRing, (i / kTileRing) & 1, limit)) ok = false;
+          tile = ok ? tile_ring[i % kTileRing] : -1;
+          if (named_bar_or(3, 128, !ok)) ok = false;
+          if (!ok || tile < 0) break;  // the same for every softmax thread
+        }
+        n_done = i + 1;
+        if (ok && !mbar_wait(s_full + sb, (i >> 1) & 1)) ok = false;
         if (named_bar_or(3, 128, !ok)) ok = false;
         tc_fence_after();
         float x[H];
@@ -413,8 +456,8 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
           if (!GATHER && p.sbuf) {
             // Raw float32 logits of keys outside the window, for the selection (kept in
             // L2 with an evict-last policy; the selection reads them right after).
-            const int jj = k0 + i * kKeyTile + t;
-            if (jj < k1 && jj <= pos - p.window && pos - p.window + 1 > p.k_sel) {
+            const int jj = tile * kKeyTile + t;
+            if (jj < k_end && jj <= pos - p.window && pos - p.window + 1 > p.k_sel) {
               float* dst = p.sbuf + ((size_t)bq * p.kv.max_len + jj) * H;
 #pragma unroll
               for (int e = 0; e < H / 4; ++e)
@@ -428,8 +471,8 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
         }
         tc_fence_before();
         mbar_arrive(s_free + sb);
-        const int j = k0 + i * kKeyTile + t;
-        bool valid = j < k1;
+        const int j = tile * kKeyTile + t;
+        bool valid = j < k_end;
         if (sel_keys && valid && j < n_c) {
           float u = x[0];
 #pragma unroll
@@ -499,9 +542,10 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
           *reinterpret_cast<uint4*>(plo + c * (kKeyTile * 16) + t * 16) =
               make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
-        if (!GATHER && !valid && i == n_tiles - 1) {
-          // Rows past the chunk end may hold anything (NaN included); 0 * NaN would
-          // poison P.V, so zero this key's V row once its tile has landed.
+        if (!GATHER && !valid) {
+          // Rows past the row's end (only its last tile has them) may hold anything, NaN
+          // included; 0 * NaN would poison P.V, so zero this key's V row once its tile
+          // has landed.
           const int s = i % NS;
           if (ok && !mbar_wait(vfull + s, (i / NS) & 1)) ok = false;
           uint4* v0 = reinterpret_cast<uint4*>(vst + s * L::kTile + t * 128);
@@ -519,8 +563,8 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
       // next kernel starts only once the index set is written.
       if (GATHER || !p.fuse) griddep_launch_dependents();
       // Epilogue: O^T row t is dimension t of every head; l is reduced across threads.
-      const int last = n_tiles - 1;
-      if (ok && !mbar_wait(p_free + (last & 1), (last >> 1) & 1)) ok = false;
+      const int last = n_done - 1;
+      if (ok && n_done > 0 && !mbar_wait(p_free + (last & 1), (last >> 1) & 1)) ok = false;
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < H; c += 16) {

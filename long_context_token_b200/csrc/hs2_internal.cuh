@@ -17,6 +17,8 @@ constexpr int kMaxIdxWidth = 4096;      // window + k_sel
 constexpr int kMaxNq = 64;
 constexpr int kMaxHeads = 128;
 constexpr long long kStallTestCycles = 20000;  // the stall test's wait limit
+constexpr int kTileRing = 8;      // slots of a full-layer CTA's tile-index ring
+constexpr int kRowTileSlot = 7;   // rowsync word: the row's next free tile (fused full layer)
 constexpr int kSmCountBound = 160;      // workspace sizing assumes at most this many SMs
 
 // Status bits kept in the workspace's status word (one bit per hs2_status code).
@@ -112,7 +114,7 @@ struct FullParams {
   int ld_u = 0;
   uint32_t* uhist = nullptr;     // [bq][kHistBins]: the u histogram, then the fine one
   uint32_t* rowmax = nullptr;    // [bq][kMaxHeads]: ordered keys of the row's largest m per head
-  uint32_t* rowsync = nullptr;   // [bq][8]: arrival counters and the band list's length
+  uint32_t* rowsync = nullptr;   // [bq][8]: arrival counters, the band list's length, the next tile
   float* cand_t = nullptr;       // [bq][ld_u] candidates of long chunks, at the chunk's offset: keys ...
   int32_t* cand_j = nullptr;     // [bq][ld_u] ... and positions
   double* band_t = nullptr;      // [bq][max_len] the row's band list: float64 keys ...

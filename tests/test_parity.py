@@ -20,6 +20,16 @@ pytestmark = [pytest.mark.gpu, pytest.mark.filterwarnings("ignore::RuntimeWarnin
 TOL = {"bf16": 2e-3, "fp8": 1e-2}
 LSE_TOL = 1e-4
 LSE64_TOL = 1e-6
+# The CUDA-core full layer (shapes the tensor-core kernels do not take) sums each logit's
+# 128 products in float32 one after another: about 2^-24 x 128 of sum |q_c k_c| of
+# rounding, which over the 128 heads of a row reaches about 1.2e-6 in the lse.
+LSE64_TOL_CUDA_CORE = 2e-6
+
+
+def cuda_core_path(kv: str, n_q: int, h: int) -> bool:
+    """Shapes whose full layer runs on the CUDA-core kernel: FP8 with more than 64 heads,
+    bf16 with 80, 96 or 112 heads."""
+    return (kv == "fp8" and h > 64) or (kv == "bf16" and h in (80, 96, 112))
 
 
 def run_gpu(inp: workloads.Inputs, twice: bool = False):
@@ -57,8 +67,10 @@ def compare_bits(bits: dict, res: dict, sparse_full: bool = True):
     if "lse64" in res:
         # The float64 lse that the selection shifts each head's scores by: its error moves
         # the ranking directly, so it is held to the selection's tie band.
+        B, n_q, h = ref["lse"].shape
+        tol64 = LSE64_TOL_CUDA_CORE if cuda_core_path(bits["kv"], n_q, h) else LSE64_TOL
         l64 = np.abs(res["lse64"].reshape(ref["lse"].shape) - ref["lse"]).max()
-        assert l64 <= LSE64_TOL, f"float64 lse error {l64}"
+        assert l64 <= tol64, f"float64 lse error {l64}"
     B, n_q = bits["q"].shape[:2]
     window, k_sel = bits["window"], bits["k_sel"]
     n_exact = 0
@@ -114,8 +126,8 @@ SMALL = [
          lens=[1509, 1402]),
     dict(id="append2-fp8-h64-odd", batch=3, max_len=2001, n_q=2, h_q=64, kv="fp8", seed=117,
          lens=[2001, 1999, 1200]),
-    # shapes served by the CUDA-core kernels: FP8 with more than 64 heads, one-token bf16
-    # with 80, 96 or 112 heads
+    # shapes served by the CUDA-core kernels: FP8 with more than 64 heads, bf16 with 80,
+    # 96 or 112 heads
     dict(id="h128-fp8-cuda-core", batch=2, max_len=2500, n_q=1, h_q=128, kv="fp8", seed=118,
          lens=[2500, 1777]),
     dict(id="h96-fp8-append2-cuda-core", batch=1, max_len=1900, n_q=2, h_q=96, kv="fp8",
@@ -123,6 +135,8 @@ SMALL = [
     dict(id="h80-bf16-cuda-core", batch=2, max_len=3000, n_q=1, h_q=80, kv="bf16", seed=120,
          lens=[3000, 2111]),
     dict(id="h112-bf16-cuda-core", batch=1, max_len=2300, n_q=1, h_q=112, kv="bf16", seed=121),
+    dict(id="h96-bf16-append3-cuda-core", batch=2, max_len=1700, n_q=3, h_q=96, kv="bf16",
+         seed=122, lens=[1700, 1234]),
 ]
 
 
