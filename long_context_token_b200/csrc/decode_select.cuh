@@ -83,11 +83,9 @@ struct FineBins {
   }
 };
 
-// Shared-memory histograms keep four padding words after every 64 bins: 16-byte chunks
-// stay aligned (cp.async copies them in), and the 32 lanes scanning 64 consecutive bins
-// each (scan_bins) meet at most 4-way bank conflicts.
-constexpr int kUBinsPadded = kUBins + kUBins / 16;
-__device__ __forceinline__ int ubin_slot(int b) { return b + ((b >> 6) << 2); }
+// Shared-memory histograms are dense (bin b at word b), as in global memory, so that one
+// bulk reduction publishes a CTA's histogram and 16-byte copies bring the row's back.
+constexpr uint32_t kUHistBytes = kUBins * 4u;
 
 // ---- row barriers: every CTA of a row arrives once per counter and call, then waits
 // until `target` have.  Arrival: a block barrier, then a release reduction by thread 0
@@ -121,11 +119,12 @@ static __device__ __noinline__ bool row_wait(uint32_t* counter, uint32_t target,
   return ok_s != 0;
 }
 
-// The bin B holding the k-th largest element of a padded shared-memory histogram
-// (ubin_slot; 0 if there are fewer than k), and with mb > 0 the counts in the bins >= B +
-// mb (`above`) and in [B - mb, B + mb) (`near`).  Warp 0 scans (lane l owns the bins
-// [kUBins - 64(l + 1), kUBins - 64 l), contiguous in the padded layout); every thread
-// calls it and gets the result.  The tail runs this code once per launch, so it is one
+// The bin B holding the k-th largest element of a dense shared-memory histogram (0 if
+// there are fewer than k), and with mb > 0 the counts in the bins >= B + mb (`above`)
+// and in [B - mb, B + mb) (`near`).  Warp 0 scans: lane l owns the bins [kUBins - 64(l +
+// 1), kUBins - 64 l), 16 chunks of 4, which it sums starting at chunk l mod 16 so that the
+// lanes' 16-byte loads meet at most 4-way bank conflicts.  Every thread calls it and gets
+// the result.  The tail runs this code once per launch, so it is one
 // out-of-line copy with rolled loops: fetching instructions that run once costs more
 // than executing them.
 struct BinScan {
@@ -138,11 +137,11 @@ static __device__ __noinline__ BinScan scan_bins(const uint32_t* hs, int k, int 
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
     const int base = kUBins - 64 * (lane + 1);
-    const uint4* row = reinterpret_cast<const uint4*>(hs + ubin_slot(base));
+    const uint4* row = reinterpret_cast<const uint4*>(hs + base);
     uint32_t sum = 0;
 #pragma unroll 1
     for (int u = 0; u < 16; ++u) {
-      const uint4 c = row[u];
+      const uint4 c = row[(u + lane) & 15];
       sum += (c.x + c.y) + (c.z + c.w);
     }
     uint32_t incl = sum;
@@ -171,7 +170,8 @@ static __device__ __noinline__ BinScan scan_bins(const uint32_t* hs, int k, int 
     uint32_t above = 0, near = 0;
     if (mb > 0) {
 #pragma unroll 1
-      for (int u = 0; u < 16; ++u) {
+      for (int u0 = 0; u0 < 16; ++u0) {
+        const int u = (u0 + lane) & 15;
         const uint4 c = row[u];
         const uint32_t v[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
@@ -194,21 +194,11 @@ static __device__ __noinline__ BinScan scan_bins(const uint32_t* hs, int k, int 
   return out_s;
 }
 
-// Adds a padded shared-memory histogram to a global one: every non-empty bin at or above
-// `low`.  All threads call.
-__device__ __forceinline__ void add_bins(const uint32_t* hs, uint32_t* gh, int low) {
-#pragma unroll 1
-  for (int e = low + (int)threadIdx.x; e < kUBins; e += blockDim.x) {
-    const uint32_t c = hs[ubin_slot(e)];
-    if (c) atomicAdd(gh + e, c);
-  }
-}
-
 // Asynchronous copies (cp.async, waited for with cp_async_wait_all) by all threads:
-// a global histogram into a padded shared-memory copy, and n 4-byte words.
+// a global histogram into a dense shared-memory copy, and n 4-byte words.
 __device__ __forceinline__ void async_bins(uint32_t* hs, const uint32_t* gh) {
   for (int v = threadIdx.x; v < kUBins / 4; v += blockDim.x)
-    sm100::cp_async_16(sm100::smem_u32(hs + ubin_slot(4 * v)), gh + 4 * v, 16u);
+    sm100::cp_async_16(sm100::smem_u32(hs + 4 * v), gh + 4 * v, 16u);
 }
 __device__ __forceinline__ void async_words(void* dst, const void* src, int n) {
   const int nv = (n + 3) / 4;
@@ -371,37 +361,94 @@ static __device__ __noinline__ void row_lse(const float* __restrict__ pml,
   __syncthreads();
 }
 
-// This CTA's share of the row's merged output, out_h = sum_s 2^(m_s - M) o_s / L: CTA r
-// of the row takes the outputs [r P, (r + 1) P), P = ceil(H kHeadDim / S); each output is
-// summed by G = blockDim / P threads over every G-th split (consecutive threads read
-// consecutive outputs of one split), and the G sums meet in shared memory (tmp: blockDim.x
-// floats).  The thread holding d = 0 of a head writes its lse (natural log) to lse64 and
-// lse_out.  Every thread calls it.
+// The outputs (h, d) of a row that CTA r merges: [r P, (r + 1) P) with P = ceil(H
+// kHeadDim / S) rounded up to a multiple of 4 (so that each split's part of the share is
+// a 16-byte-aligned run); MergeShare also gives the heads the share spans.
+struct MergeShare {
+  int o0, o1, opc;
+  int h0, nh;  // heads [h0, h0 + nh), h0 even and nh even: whole 16-byte (m, l) pairs
+};
+template <int H>
+__device__ __forceinline__ MergeShare merge_share(int split, int S) {
+  constexpr int kOut = H * kHeadDim;
+  MergeShare m;
+  m.opc = (((kOut + S - 1) / S) + 3) & ~3;
+  m.o0 = min(split * m.opc, kOut);
+  m.o1 = min(m.o0 + m.opc, kOut);
+  m.h0 = (m.o0 / kHeadDim) & ~1;
+  m.nh = m.o1 > m.o0 ? (((m.o1 - 1) / kHeadDim + 2) & ~1) - m.h0 : 0;
+  return m;
+}
+
+// Bytes of shared memory that prefetch_merge fills (a multiple of 16).
+template <int H>
+__device__ __forceinline__ uint32_t merge_prefetch_bytes(int split, int S) {
+  const MergeShare m = merge_share<H>(split, S);
+  return (uint32_t)S * m.opc * 4u + (uint32_t)S * m.nh * 8u;
+}
+
+// The split partials this CTA's share of the merge reads, copied on chip (cp.async, all
+// threads): o of every split for the share's outputs ([S][opc] floats at mo), then (m, l)
+// of every split for the share's heads ([S][nh] float2 after it).
+template <int H>
+__device__ __forceinline__ void prefetch_merge(const FullParams& p, int bq, int split, int S,
+                                               float* mo) {
+  const MergeShare m = merge_share<H>(split, S);
+  const float* po = p.part_o + (size_t)bq * S * H * kHeadDim;
+  const float* pml = p.part_ml + (size_t)bq * S * H * 2;
+  const int n4 = (m.o1 - m.o0) / 4;  // 16-byte chunks of one split
+  for (int e = threadIdx.x; e < S * n4; e += blockDim.x) {
+    const int s = e / n4, c = e % n4;
+    sm100::cp_async_16(sm100::smem_u32(mo + s * m.opc + 4 * c),
+                       po + (size_t)s * H * kHeadDim + m.o0 + 4 * c, 16u);
+  }
+  float* ml = mo + S * m.opc;
+  const int n2 = m.nh / 2;  // 16-byte chunks (two heads) of one split
+  for (int e = threadIdx.x; e < S * n2; e += blockDim.x) {
+    const int s = e / n2, c = e % n2;
+    sm100::cp_async_16(sm100::smem_u32(ml + 4 * e), pml + ((size_t)s * H + m.h0 + 2 * c) * 2, 16u);
+  }
+}
+
+// This CTA's share of the row's merged output, out_h = sum_s 2^(m_s - M) o_s / L: each
+// output is summed by G = blockDim / P threads over every G-th split (consecutive
+// threads take consecutive outputs of one split), and the G sums meet in shared memory
+// (tmp: blockDim.x floats).  The partials come from `mo` (prefetch_merge, complete) or,
+// if null, from global memory.  The thread holding d = 0 of a head writes its lse
+// (natural log) to lse64 and lse_out.  Every thread calls it.
 template <int H>
 static __device__ __noinline__ void row_merge(const FullParams& p, int bq, int split, int S,
-                                              const RowLse<H>& r, float* tmp) {
+                                              const RowLse<H>& r, float* tmp, const float* mo) {
   const float* po = p.part_o + (size_t)bq * S * H * kHeadDim;
   const float2* pml = reinterpret_cast<const float2*>(p.part_ml + (size_t)bq * S * H * 2);
   constexpr int kOut = H * kHeadDim;
+  const MergeShare m = merge_share<H>(split, S);
+  const float2* mml = reinterpret_cast<const float2*>(mo + S * m.opc);
   const int nt = blockDim.x, tid = threadIdx.x;
-  const int opc = (kOut + S - 1) / S;
-  const int o0 = split * opc, o1 = min(o0 + opc, kOut);
-  const int P = min(opc, nt);  // outputs per round
-  const int G = nt / P;        // threads per output
+  const int P = min(m.opc, nt);  // outputs per round
+  const int G = nt / P;          // threads per output
   const int ol = tid % P, g = tid / P;
 #pragma unroll 1
-  for (int ob = o0; ob < o1; ob += P) {
+  for (int ob = m.o0; ob < m.o1; ob += P) {
     const int o = ob + ol;
-    const bool mine = g < G && o < o1;
+    const bool mine = g < G && o < m.o1;
     const int h = o / kHeadDim, d = o % kHeadDim;
     float acc = 0.f;
     if (mine) {
       const float M = r.M[h], il = r.invL[h];
-#pragma unroll 8
-      for (int s = g; s < S; s += G) {
-        const float2 ml = __ldcg(pml + (size_t)s * H + h);
-        const float v = __ldcg(po + ((size_t)s * H + h) * kHeadDim + d);
-        if (ml.y > 0.f) acc = fmaf(exp2f(ml.x - M) * il, v, acc);
+      if (mo) {
+#pragma unroll 4
+        for (int s = g; s < S; s += G) {
+          const float2 ml = mml[s * m.nh + h - m.h0];
+          if (ml.y > 0.f) acc = fmaf(exp2f(ml.x - M) * il, mo[s * m.opc + o - m.o0], acc);
+        }
+      } else {
+#pragma unroll 16
+        for (int s = g; s < S; s += G) {
+          const float2 ml = __ldcg(pml + (size_t)s * H + h);
+          const float v = __ldcg(po + ((size_t)s * H + h) * kHeadDim + d);
+          if (ml.y > 0.f) acc = fmaf(exp2f(ml.x - M) * il, v, acc);
+        }
       }
     }
     if (G > 1) {
@@ -579,7 +626,7 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* scratch
   // holds a copy of the histogram, then the band keys being re-scored and the per-warp K
   // rows, later the band list being ranked.)
   uint32_t* fhs = reinterpret_cast<uint32_t*>(scratch);
-  uint8_t* bscr = scratch + kUBinsPadded * 4;
+  uint8_t* bscr = scratch + kUHistBytes;
   double* bval = reinterpret_cast<double*>(bscr);
   int* bl = reinterpret_cast<int*>(bscr + kBandSmem * 8);
   float* kf = reinterpret_cast<float*>(bscr + kBandSmem * 12);
@@ -736,12 +783,18 @@ __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, 
   uint32_t* gu = p.uhist + (size_t)bq * kHistBins;
   const int c_hi = min(k1, n_c);
   const int chunk_len = sel_row && c_hi > k0 ? c_hi - k0 : 0;
-  // Before the second barrier the stages hold: the gathered tiles, the row's u histogram,
-  // then this chunk's bounds (a piece at a time), its candidate positions and their keys.
+  // The stages hold: the gathered tiles (later the tail's scratch), the row's u
+  // histogram, the merge's inputs (when they fit beside a one-piece chunk), then this
+  // chunk's bounds (a piece at a time), its candidate positions and their keys.
   const uint32_t tiles = kTailTiles * tile_bytes;
   uint32_t* uh = reinterpret_cast<uint32_t*>(stage + tiles);
-  const uint32_t uoff = tiles + ((kUBinsPadded * 4u + 15u) & ~15u);
-  const int piece = (int)(((stage_bytes - uoff - kTailTiles * 128u * 4u) / 8u) & ~3u);
+  const uint32_t moff = tiles + kUHistBytes;
+  const uint32_t fixed = moff + kTailTiles * 128u * 4u;
+  uint32_t mbytes = merge_prefetch_bytes<H>(split, S);
+  if (fixed + mbytes + 8u * (uint32_t)((chunk_len + 3) & ~3) > stage_bytes) mbytes = 0;
+  float* mo = mbytes ? reinterpret_cast<float*>(stage + moff) : nullptr;
+  const uint32_t uoff = moff + mbytes;
+  const int piece = (int)(((stage_bytes - fixed - mbytes) / 8u) & ~3u);
   float* us = reinterpret_cast<float*>(stage + uoff);
   int* cl = reinterpret_cast<int*>(stage + uoff + 4u * (uint32_t)piece);
   float* t2s = reinterpret_cast<float*>(stage + uoff + 8u * (uint32_t)piece);
@@ -756,10 +809,16 @@ __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, 
     if (v.y > 0.f) atomicMax(rowmax + threadIdx.x, max_key(v.x));
   }
   if (sel_row) {
-    // The bins at or above this CTA's own k_sel-th largest u published (the row's
-    // boundary bin is at least that high).
-    const int low = scan_bins(uhist_s, p.k_sel, 0).bin;
-    add_bins(uhist_s, gu, low);
+    // This CTA's u histogram added to the row's in one bulk reduction (its writes done
+    // and ordered before the barrier's release).
+    sm100::fence_proxy_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      sm100::bulk_reduce_add_u32(gu, uhist_s, kUHistBytes);
+      sm100::bulk_commit();
+      sm100::bulk_wait_all();
+      sm100::fence_proxy_async_global();
+    }
   }
   row_arrive(rs + kRowArrive1);
   if (!row_wait(rs + kRowArrive1, (uint32_t)S, p.stall_test == 2)) ok = false;
@@ -769,6 +828,7 @@ __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, 
     async_bins(uh, gu);
     async_words(us, p.ubuf + (size_t)bq * p.ld_u + k0, min(piece, chunk_len));
   }
+  if (mo) prefetch_merge<H>(p, bq, split, S, mo);  // read at the very end
   row_lse<H>(p.part_ml + (size_t)bq * S * H * 2, rowmax, S, rl, reinterpret_cast<float2*>(stage));
   if (p.fuse == 2 && !sel_row && split == 0)
     write_all_positions(p.sel_idx + (size_t)bq * width, width, pos);
@@ -785,7 +845,11 @@ __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, 
   sm100::fence_acq_rel_gpu();
   __syncthreads();
   griddep_launch_dependents();
-  row_merge<H>(p, bq, split, S, rl, reinterpret_cast<float*>(stage));
+  if (mo) {
+    sm100::cp_async_wait_all();
+    __syncthreads();
+  }
+  row_merge<H>(p, bq, split, S, rl, reinterpret_cast<float*>(stage), mo);
   __syncthreads();
   if (threadIdx.x == 0) {
     // The last CTA of the row to get here leaves the row's counters at zero.

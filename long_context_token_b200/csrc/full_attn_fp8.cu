@@ -62,7 +62,7 @@ struct Fp8Smem {
   static constexpr uint32_t kMaxBars = 4 * 6 + 10;
   // Full layer only: the histogram of the selection bounds u and the exchange of the two
   // head halves' partial bounds ([2][128] floats).
-  static constexpr uint32_t kSelBytes = GATHER ? 0u : (uint32_t)kUBinsPadded * 4u + 2u * 128u * 4u;
+  static constexpr uint32_t kSelBytes = GATHER ? 0u : kUHistBytes + 2u * 128u * 4u;
   // (+ 1024 for alignment, + 1024 for the static shared memory of the Q staging, + 7168
   // for that of the fused tail)
   static constexpr uint32_t kFixed = kQBytes + 2 * kPBytes + kRedBytes + kRefBytes +
@@ -81,7 +81,7 @@ struct Fp8Smem {
   static constexpr uint32_t kBars = 4 * R + 10;
   static constexpr uint32_t kSlotOff = kBarOff + kBars * 8;
   static constexpr uint32_t kUHistOff = (kSlotOff + 16 + 15) / 16 * 16;  // 16-byte aligned
-  static constexpr uint32_t kUxOff = kUHistOff + (GATHER ? 0u : (uint32_t)kUBinsPadded * 4u);
+  static constexpr uint32_t kUxOff = kUHistOff + (GATHER ? 0u : kUHistBytes);
   static constexpr uint32_t kBytes = kUHistOff + kSelBytes + 1024;
   static constexpr uint32_t kTmemCols = tmem_cols_pow2(7 * H);  // S: 2 x 2H, O: 3H
   static_assert(R >= 1 && kBytes <= 227 * 1024, "shared memory budget");
@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     fence_mbar_init();
   }
   if (!GATHER)
-    for (int e = threadIdx.x; e < kUBinsPadded; e += blockDim.x) uhist_s[e] = 0u;
+    for (int e = threadIdx.x; e < kUBins; e += blockDim.x) uhist_s[e] = 0u;
   if (warp == 1) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
@@ -476,7 +476,7 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     bool rec_prev = false;
     auto record_u = [&](int jj, float u) {
       st_global_f32_hint(urow + jj, u, keep_policy);
-      atomicAdd(&uhist_s[ubin_slot(ubin(u))], 1u);
+      atomicAdd(&uhist_s[ubin(u)], 1u);
     };
     // This group's references: in registers up to 16 heads per thread; above, read
     // from shared memory at each use (registers are the limit there).

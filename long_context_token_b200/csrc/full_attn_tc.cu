@@ -55,8 +55,8 @@ struct FullSmem {
   static constexpr uint32_t kRingOff = kSlotOff + 16;  // [kTileRing] tile indices
   // Histogram of the selection bounds u (full layer only).
   static constexpr uint32_t kUHistOff = (kRingOff + 4 * kTileRing + 15) / 16 * 16;
-  static constexpr uint32_t kUHistBytes = GATHER ? 0u : (uint32_t)kUBinsPadded * 4u;
-  static constexpr uint32_t kBytes = kUHistOff + kUHistBytes + 1024;
+  static constexpr uint32_t kUHistLen = GATHER ? 0u : hs2::kUHistBytes;
+  static constexpr uint32_t kBytes = kUHistOff + kUHistLen + 1024;
   static constexpr uint32_t kTmemCols = tmem_cols_pow2(3 * H);
   static_assert(kBytes <= 227 * 1024, "shared memory budget");
 };
@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
     fence_mbar_init();
   }
   if (!GATHER)
-    for (int e = threadIdx.x; e < kUBinsPadded; e += blockDim.x) uhist_s[e] = 0u;
+    for (int e = threadIdx.x; e < kUBins; e += blockDim.x) uhist_s[e] = 0u;
   if (warp == 1) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
@@ -478,7 +478,7 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
 #pragma unroll
           for (int h = 1; h < H; ++h) u = fmaxf(u, x[h]);
           st_global_f32_hint(urow + j, u, keep_policy);
-          atomicAdd(&uhist_s[ubin_slot(ubin(u))], 1u);
+          atomicAdd(&uhist_s[ubin(u)], 1u);
         }
         if (GATHER && valid) {
           const int pj = __ldcg(idx_row + j);
