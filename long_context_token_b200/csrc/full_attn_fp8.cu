@@ -59,14 +59,15 @@ struct Fp8Smem {
   static constexpr uint32_t kPBytes = 3 * H * kKeyTile;       // P_hi, P_lo, P_lo2
   static constexpr uint32_t kRedBytes = (4 * H + 8) * 4;      // [4 warps][H] + V-scale maxima
   static constexpr uint32_t kRefBytes = (2 * H + 8) * 4;      // mref, alpha, scalars
-  static constexpr uint32_t kMaxBars = 4 * 6 + 10;
+  static constexpr uint32_t kMaxBars = 4 * 6 + 10 + kTileRing;
   // Full layer only: the histogram of the selection bounds u and the exchange of the two
   // head halves' partial bounds ([2][128] floats).
   static constexpr uint32_t kSelBytes = GATHER ? 0u : kUHistBytes + 2u * 128u * 4u;
   // (+ 1024 for alignment, + 1024 for the static shared memory of the Q staging, + 7168
   // for that of the fused tail)
   static constexpr uint32_t kFixed = kQBytes + 2 * kPBytes + kRedBytes + kRefBytes +
-                                     kMaxBars * 8 + 16 + kSelBytes + 2048 + (GATHER ? 0 : 7168);
+                                     kMaxBars * 8 + 16 + 4 * kTileRing + kSelBytes + 2048 +
+                                     (GATHER ? 0 : 7168);
   // Raw stages (K and V each): as many as fit, up to six; gather mode keeps one (its
   // CTAs mostly take a single tile).
   static constexpr int kFit = (int)((227u * 1024u - kFixed) / (2 * kRawTile));
@@ -78,9 +79,10 @@ struct Fp8Smem {
   static constexpr uint32_t kRedOff = kPOff + 2 * kPBytes;
   static constexpr uint32_t kRefOff = kRedOff + kRedBytes;
   static constexpr uint32_t kBarOff = kRefOff + kRefBytes;
-  static constexpr uint32_t kBars = 4 * R + 10;
+  static constexpr uint32_t kBars = 4 * R + 10 + kTileRing;
   static constexpr uint32_t kSlotOff = kBarOff + kBars * 8;
-  static constexpr uint32_t kUHistOff = (kSlotOff + 16 + 15) / 16 * 16;  // 16-byte aligned
+  static constexpr uint32_t kRingOff = kSlotOff + 16;  // [kTileRing] tile indices
+  static constexpr uint32_t kUHistOff = (kRingOff + 4 * kTileRing + 15) / 16 * 16;
   static constexpr uint32_t kUxOff = kUHistOff + (GATHER ? 0u : kUHistBytes);
   static constexpr uint32_t kBytes = kUHistOff + kSelBytes + 1024;
   static constexpr uint32_t kTmemCols = tmem_cols_pow2(7 * H);  // S: 2 x 2H, O: 3H
@@ -265,7 +267,9 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
   uint64_t* p_free = s_full + 6;    // [2]
   uint64_t* mma_done = s_full + 8;
   uint64_t* post_bar = s_full + 9;  // MMAs of the selection tail
+  uint64_t* idx_bar = s_full + 10;  // [kTileRing] one per slot of the tile-index ring
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
+  int* tile_ring = reinterpret_cast<int*>(smem + L::kRingOff);
   uint32_t* uhist_s = reinterpret_cast<uint32_t*>(smem + L::kUHistOff);
   float* ux_s = reinterpret_cast<float*>(smem + L::kUxOff);  // [2][128]
 
@@ -291,6 +295,7 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     }
     mbar_init(mma_done, 1);
     mbar_init(post_bar, 1);
+    for (int r = 0; r < kTileRing; ++r) mbar_init(idx_bar + r, 1);
     fence_mbar_init();
   }
   if (!GATHER)
@@ -318,12 +323,20 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
   const int k1 = GATHER ? min(k0 + p.chunk1, p.idx_width) : min(k0 + p.chunk1, pos + 1);
   const int32_t* idx_row = GATHER ? p.idx + (size_t)bq * p.idx_width : nullptr;
   const size_t row_base = (size_t)b * p.kv.max_len;
-  const int n_tiles = k0 < k1 ? (k1 - k0 + kKeyTile - 1) / kKeyTile : 0;
+  // Fused full layer with several CTAs a row: the row's tiles are shared out at run time
+  // (CTA r takes tiles r, r + S, ..., r + (R - 1) S, then claims the next free tile from
+  // the row's counter), as in the bf16 kernel; the selection keeps its static chunks.
+  const int S = p.splits1;
+  const bool dyn = !GATHER && p.fuse != 0 && S > 1;
+  const int row_tiles = (pos + 1 + kKeyTile - 1) / kKeyTile;
+  const int n_tiles = dyn ? (split < row_tiles ? 1 : 0)  // (only whether any)
+                          : (k0 < k1 ? (k1 - k0 + kKeyTile - 1) / kKeyTile : 0);
+  const int k_end = dyn ? pos + 1 : k1;  // entries at or past this one are absent
   const size_t pidx = (size_t)bq * p.splits1 + split;
 
   // Row of the cache behind tile entry e (or -1 for an absent / past-the-end entry).
   auto entry_row = [&](int e) -> long long {
-    if (e >= k1) return -1;
+    if (e < 0 || e >= k_end) return -1;
     if (!GATHER) return (long long)(row_base + e);
     const int j = __ldcg(idx_row + e);  // through L2: may have been written by the previous grid
     return (j >= 0 && j < Lb) ? (long long)(row_base + j) : -1;
@@ -394,14 +407,25 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
       }
     } else if (elect_one()) {
       // ---------------------------------------------------------- TMA producer
+      // Tile i's index goes to slot i of the ring (its barrier arrived on) before the
+      // tile's loads; past the last tile an index of -1 ends the other warps' loops.
       const uint64_t pol = policy_evict_first();
-      const int row0 = b * p.kv.max_len + k0;
+      const int row_b = b * p.kv.max_len;
+      uint32_t* row_counter = p.rowsync + (size_t)bq * 8 + kRowTileSlot;
+      uint32_t claimed = 0;
       int issued = 0;
-      for (int i = 0; i < n_tiles && ok; ++i) {
+      for (int i = 0; ok; ++i) {
         const int s = i % R;
         const uint32_t ph = ((i / R) & 1) ^ 1;
-        const int row = row0 + i * kKeyTile;
+        const int tile = dyn ? (i < R ? split + i * S : R * S + (int)claimed)
+                             : (i < n_tiles ? k0 / kKeyTile + i : -1);
+        const bool end = tile < 0 || tile >= row_tiles || (!dyn && i >= n_tiles);
         if (!mbar_wait(kr_empty + s, ph)) { ok = false; break; }
+        tile_ring[i % kTileRing] = end ? -1 : tile;
+        mbar_arrive(idx_bar + i % kTileRing);
+        if (end) break;
+        if (dyn && i + 1 >= R) claimed = atomicAdd(row_counter, 1u);  // tile i + 1's
+        const int row = row_b + tile * kKeyTile;
         mbar_arrive_expect_tx(kr_full + s, kRawTile);
         tma_load_2d(kraw + s * kRawTile, &tmap_k, kr_full + s, 0, row, pol);
         if (!mbar_wait(vr_empty + s, ph)) { ok = false; break; }
@@ -435,9 +459,15 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
         mma_commit(vr_empty + s);
         return true;
       };
-      for (int i = 0; i < n_tiles && ok; ++i) {
+      int n_done = 0;
+      for (int i = 0; (GATHER ? i < n_tiles : true) && ok; ++i) {
         const int s = i % R, sb = i & 1;
+        if (!GATHER) {  // the tile's index first (-1: past the last tile)
+          if (!mbar_wait(idx_bar + i % kTileRing, (i / kTileRing) & 1)) { ok = false; break; }
+          if (tile_ring[i % kTileRing] < 0) break;
+        }
         if (!mbar_wait(kr_full + s, (i / R) & 1)) { ok = false; break; }
+        n_done = i + 1;
         if (!mbar_wait(s_free + sb, ((i >> 1) & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t k_addr = smem_u32(kraw + s * kRawTile);
@@ -449,7 +479,7 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
         mma_commit(kr_empty + s);
         if (i > 0 && !issue_pv(i - 1)) { ok = false; break; }
       }
-      if (ok && !issue_pv(n_tiles - 1)) ok = false;
+      if (ok && n_done > 0 && !issue_pv(n_done - 1)) ok = false;
       mma_commit(mma_done);
       if (!mbar_wait(mma_done, 0)) ok = false;
     }
@@ -495,27 +525,54 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     float vlim = 0.f, vmul = 0.f;
     // Per-key scales (and validity) are loaded two tiles ahead so that their memory
     // latency overlaps the tiles in between instead of stalling each tile.
-    auto scales_of = [&](int i, float& ks, float& vs, bool& ok_row) {
-      const long long row = i < n_tiles ? entry_row(k0 + i * kKeyTile + t) : -1;
+    // Tiles in the order this CTA takes them, by their first entry: k0 + 128 i in gather
+    // mode, else from the producer's ring (read in order, never past its -1).
+    int seen = 0;
+    bool ring_end = false;
+    auto next_base = [&]() -> int {
+      int v = -1;
+      if (GATHER) {
+        v = seen < n_tiles ? k0 + seen * kKeyTile : -1;
+      } else if (!ring_end) {
+        if (ok && !mbar_wait(idx_bar + seen % kTileRing, (seen / kTileRing) & 1)) ok = false;
+        const int tl = ok ? tile_ring[seen % kTileRing] : -1;
+        ring_end = tl < 0;
+        v = tl < 0 ? -1 : tl * kKeyTile;
+      }
+      ++seen;
+      return v;
+    };
+    auto scales_of = [&](int base, float& ks, float& vs, bool& ok_row) {
+      const long long row = base >= 0 ? entry_row(base + t) : -1;
       ok_row = row >= 0;
       ks = ok_row ? __ldg(p.kv.k_scale + row) : 0.f;
       vs = ok_row ? __ldg(p.kv.v_scale + row) : 0.f;
     };
+    int base_next = next_base();
+    int base_far = base_next >= 0 ? next_base() : -1;
     float ks_next, vs_next, ks_far, vs_far;
     bool val_next, val_far;
-    scales_of(0, ks_next, vs_next, val_next);
-    scales_of(1, ks_far, vs_far, val_far);
+    scales_of(base_next, ks_next, vs_next, val_next);
+    scales_of(base_far, ks_far, vs_far, val_far);
     const float qinv = qsc_s[0];
     const float c2 = p.sm_scale * kLog2eF8 * qinv;  // Q-scaled logit -> log2 units
-    for (int i = 0; i < n_tiles; ++i) {
+    int n_done = 0;
+    for (int i = 0;; ++i) {
       const int sb = i & 1;
-      const int j = k0 + i * kKeyTile + t;
+      // This tile, and the one two ahead (its scales' loads start now).
+      const int base = base_next;
+      base_next = base_far;
+      base_far = base_far >= 0 ? next_base() : -1;
+      if (named_bar_or(3, NSOFT, !ok)) ok = false;
+      if (!ok || base < 0) break;  // the same for every softmax thread
+      n_done = i + 1;
+      const int j = base + t;
       const float ks = ks_next, vs = vs_next;
       const bool valid = val_next;
       ks_next = ks_far;
       vs_next = vs_far;
       val_next = val_far;
-      scales_of(i + 2, ks_far, vs_far, val_far);
+      scales_of(base_far, ks_far, vs_far, val_far);
       if (ok && !mbar_wait(s_full + sb, (i >> 1) & 1)) ok = false;
       if (named_bar_or(3, NSOFT, !ok)) ok = false;
       tc_fence_after();
@@ -538,7 +595,7 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
       tc_fence_before();
       mbar_arrive(s_free + sb);
       if (!GATHER && p.sbuf) {
-        if (j < k1 && j <= pos - p.window && pos - p.window + 1 > p.k_sel) {
+        if (j < k_end && j <= pos - p.window && pos - p.window + 1 > p.k_sel) {
           const float qk = qinv * ks;  // the stored logit is q.k times the key's scale
           float* dst = p.sbuf + ((size_t)bq * p.kv.max_len + j) * H + hoff;
 #pragma unroll
@@ -667,9 +724,10 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
         *reinterpret_cast<uint4*>(pb + (ch0 + 2 * (H / 16)) * (kKeyTile * 16) + t * 16) =
             make_uint4(w2[0], w2[1], w2[2], w2[3]);
       }
-      if (!GATHER && !valid && half == 0 && i == n_tiles - 1) {
-        // Rows past the chunk end may hold anything (NaN codes included); 0 * NaN would
-        // poison P.V, so zero this key's V row once its tile has landed.
+      if (!GATHER && !valid && half == 0) {
+        // Rows past the row's end (only its last tile has them) may hold anything, NaN
+        // codes included; 0 * NaN would poison P.V, so zero this key's V row once its
+        // tile has landed.
         const int s = i % R;
         if (ok && !mbar_wait(vr_full + s, (i / R) & 1)) ok = false;
         uint4* v0 = reinterpret_cast<uint4*>(vraw + s * kRawTile + t * 128);
@@ -682,13 +740,13 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
     if (NHALF == 2 && sel_keys) {
       named_bar_sync(3, NSOFT);
       if (half == 0 && rec_prev)
-        record_u(j_prev, fmaxf(u_prev, ux_s[((n_tiles - 1) & 1) * 128 + t]));
+        record_u(j_prev, fmaxf(u_prev, ux_s[((n_done - 1) & 1) * 128 + t]));
     }
     // The merge kernel may be scheduled (it waits for this grid); with the fused tail the
     // next kernel starts only once the index set is written.
     if (GATHER || !p.fuse) griddep_launch_dependents();
-    const int last = n_tiles - 1;
-    if (ok && !mbar_wait(p_free + (last & 1), (last >> 1) & 1)) ok = false;
+    const int last = n_done - 1;
+    if (ok && n_done > 0 && !mbar_wait(p_free + (last & 1), (last >> 1) & 1)) ok = false;
     tc_fence_after();
     const float oscale = ev == kNoScale ? 0.f : ldexpf(1.f, ev);
 #pragma unroll
