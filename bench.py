@@ -43,17 +43,16 @@ LAUNCHES_PER_SPARSE = 1         # gather attention with the split merge on chip 
 
 
 # DRAM bytes (read + write) of one full-layer launch, from an ncu capture of the same
-# kernel (dram__bytes_read.sum + dram__bytes_write.sum) on the first 2 of the 8
-# sequences, scaled by sequences (the traffic is per sequence); see profiles/.
+# kernel (dram__bytes_read.sum + dram__bytes_write.sum): the one-launch full layer (stream,
+# split merge and token selection) where "fused"; the captures are summarised in profiles/.
 NCU_TRAFFIC = {
-    2: {"bytes": 4 * (134_288_128 + 786_304), "kernel": "full_attn_tc_kernel<16, 0>",
-        "capture": "2 x 131072 keys, scaled x4", "fused": False},
-    # first sequence of the ragged batch, scaled by the launch's algorithmic bytes
-    3: {"bytes": round((56_967_424 + 623_104) * 245_681_880 / 56_903_232),
-        "kernel": "full_attn_fp8_kernel<16, 0>",
-        "capture": "first sequence (56.9 MB of codes and scales), scaled to the 4-sequence launch",
-        "fused": False},
-    4: {"bytes": 276_918_528 + 5_604_608, "kernel": "full_attn_fp8_kernel<64, 0>",
+    2: {"bytes": 4 * (134_890_752 + 659_328), "kernel": "full_attn_tc_kernel<16, 0>",
+        "capture": "2 x 131072 keys (two launches averaged), scaled x4", "fused": True},
+    3: {"bytes": 246_885_888 + 3_051_008, "kernel": "full_attn_fp8_kernel<16, 0>",
+        "capture": "the whole launch", "fused": True},
+    4: {"bytes": 277_461_760 + 4_877_824, "kernel": "full_attn_fp8_kernel<64, 0>",
+        "capture": "the whole launch", "fused": True},
+    5: {"bytes": 67_430_656 + 3_554_816, "kernel": "full_attn_mq_kernel<16>",
         "capture": "the whole launch", "fused": False},
 }
 

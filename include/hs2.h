@@ -268,6 +268,16 @@ HS2_API hs2_status hs2_kv_append(const void* k_new, const void* v_new, int n_new
  * before the next call that uses it. */
 HS2_API hs2_status hs2_check_device_status(void* workspace, hs2_stream_t stream);
 
+/* Reproducibility switch (process-wide; 0 by default).  By default the one-launch full
+ * layer shares each row's key tiles out among its CTAs at run time (CTAs slowed by the
+ * memory system take fewer tiles), so the grouping of the float32 partial sums, and with
+ * it the last bits of the outputs and of the lse, can differ between two runs on the same
+ * inputs; the index set differs only where two keys' exact scores are within the lse's
+ * rounding (~1e-7).  With `on` nonzero every CTA takes a fixed chunk of keys and repeated
+ * runs are bitwise identical, at some cost in speed.  Applies to the launches that follow;
+ * not synchronised between host threads. */
+HS2_API void hs2_set_deterministic(int on);
+
 /* Test hook for the error path of the bounded device-side waits; not for production.
  *   mode 1: the bf16 one-token full-layer kernel issues no loads and no MMAs, so its
  *           softmax warps' first wait on an MMA result runs out (after about 10 us);

@@ -29,7 +29,8 @@
 //      writes the selected positions of its own chunk, in order, from the slot after those
 //      of the lower chunks (their counts, and the band keys below its chunk that the
 //      ranking takes); the first CTA appends the window.  Then the CTA lets the next
-//      kernel start and merges its share of the row's output.
+//      kernel start.  (Each CTA merges its share of the row's output between arriving at
+//      the second barrier and waiting there.)
 // The float32 keys are within eps / 2 of the exact ones, eps = 1e-3 max(1, |bin edge| +
 // W) (as in the separate selection kernels), so the chosen set is the float64
 // definition's up to the tie band.
@@ -296,14 +297,25 @@ static __device__ __noinline__ void row_lse(const float* __restrict__ pml,
   const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31;
   const int G = nt / H;
   const int h = tid % H, g = tid / H;
+  // The thread's first kFirst partials are requested with the maxima (one round trip).
+  constexpr int kFirst = 4;
+  const float2* src = reinterpret_cast<const float2*>(pml) + h;
+  float2 first[kFirst];
+#pragma unroll
+  for (int k = 0; k < kFirst; ++k) {
+    const int s = g + k * G;
+    first[k] = g < G && s < S ? __ldcg(src + (size_t)s * H) : make_float2(0.f, 0.f);
+  }
   if (tid < H) r.M[tid] = max_key_value(__ldcg(rowmax + tid));
   __syncthreads();
   float ls = 0.f, le = 0.f;
   if (g < G) {
     const float M = r.M[h];
-    const float2* src = reinterpret_cast<const float2*>(pml) + h;
+#pragma unroll
+    for (int k = 0; k < kFirst; ++k)
+      if (first[k].y > 0.f) two_sum_acc(ls, le, first[k].y * exp2f(first[k].x - M));
 #pragma unroll 8
-    for (int s = g; s < S; s += G) {
+    for (int s = g + kFirst * G; s < S; s += G) {
       const float2 v = __ldcg(src + (size_t)s * H);
       if (v.y > 0.f) two_sum_acc(ls, le, v.y * exp2f(v.x - M));
     }
@@ -503,12 +515,12 @@ __device__ __forceinline__ int find_position(const int* oj, int n, int j) {
 // K Q^T MMA and stores t = max_h (x_h - D[h]) of each into t2[0, m), ending with a block
 // barrier; it returns false if a wait gave up.  `scratch` (the gathered tiles' space) is
 // free once the candidates are re-scored.  Returns false if a wait gave up.
-template <int H, bool FP8, typename Recompute>
+template <int H, bool FP8, typename Recompute, typename Merge>
 __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* scratch, float* us,
                                            int* cl, float* t2s, int piece, int bq, int b,
                                            int split, int S, int k0, int c_hi, int n_c, int pos,
                                            int bk, const RowLse<H>& rl, const QView& qv,
-                                           Recompute&& recompute) {
+                                           Recompute&& recompute, Merge&& merge) {
   __shared__ float eps_s;
   __shared__ FineBins fb_s;
   __shared__ int mb_s;
@@ -615,6 +627,7 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* scratch
     own_n += ncl;
   }
   row_arrive(rs + kRowArrive2);
+  merge();  // this CTA's share of the outputs, while the row's other CTAs arrive
   if (!row_wait(rs + kRowArrive2, (uint32_t)S, p.stall_test == 2)) ok = false;
   // Every CTA of the row has its copy of the u histogram by now (each copied it before
   // arriving): clear this CTA's share for the next call.
@@ -832,12 +845,19 @@ __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, 
   row_lse<H>(p.part_ml + (size_t)bq * S * H * 2, rowmax, S, rl, reinterpret_cast<float2*>(stage));
   if (p.fuse == 2 && !sel_row && split == 0)
     write_all_positions(p.sel_idx + (size_t)bq * width, width, pos);
+  // The merge needs only the lse and the partials: with a selection it runs while the
+  // CTA waits at the row's second barrier, else at the end.
+  bool merged = false;
+  auto merge = [&]() {
+    row_merge<H>(p, bq, split, S, rl, reinterpret_cast<float*>(stage), mo);
+    merged = true;
+  };
   if (sel_row) {
-    sm100::cp_async_wait_all();
+    sm100::cp_async_wait_all();  // (the merge's partials too)
     __syncthreads();
     const int bk = scan_bins(uh, p.k_sel, 0).bin;
     if (!row_select<H, FP8>(p, stage, us, cl, t2s, piece, bq, b, split, S, k0, c_hi, n_c, pos,
-                            bk, rl, qv, recompute))
+                            bk, rl, qv, recompute, merge))
       ok = false;
   }
   // The index set is complete and visible: the next kernel (a sparse layer, which reads
@@ -845,11 +865,13 @@ __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, 
   sm100::fence_acq_rel_gpu();
   __syncthreads();
   griddep_launch_dependents();
-  if (mo) {
-    sm100::cp_async_wait_all();
-    __syncthreads();
+  if (!merged) {
+    if (mo) {
+      sm100::cp_async_wait_all();
+      __syncthreads();
+    }
+    merge();
   }
-  row_merge<H>(p, bq, split, S, rl, reinterpret_cast<float*>(stage), mo);
   __syncthreads();
   if (threadIdx.x == 0) {
     // The last CTA of the row to get here leaves the row's counters at zero.

@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(fp8_threads<H>(), 1)
   // (CTA r takes tiles r, r + S, ..., r + (R - 1) S, then claims the next free tile from
   // the row's counter), as in the bf16 kernel; the selection keeps its static chunks.
   const int S = p.splits1;
-  const bool dyn = !GATHER && p.fuse != 0 && S > 1;
+  const bool dyn = !GATHER && p.fuse != 0 && S > 1 && !p.deterministic;
   const int row_tiles = (pos + 1 + kKeyTile - 1) / kKeyTile;
   const int n_tiles = dyn ? (split < row_tiles ? 1 : 0)  // (only whether any)
                           : (k0 < k1 ? (k1 - k0 + kKeyTile - 1) / kKeyTile : 0);

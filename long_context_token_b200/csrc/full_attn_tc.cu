@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(192, (GATHER && H <= 16) ? 2 : 1)
   // system take fewer tiles and the row's CTAs reach its first barrier together.  The
   // selection keeps its static ownership of positions (chunk r), whoever read them.
   const int S = p.splits1;
-  const bool dyn = !GATHER && p.fuse != 0 && S > 1;
+  const bool dyn = !GATHER && p.fuse != 0 && S > 1 && !p.deterministic;
   const int row_tiles = (pos + 1 + kKeyTile - 1) / kKeyTile;
   const int n_tiles = dyn ? (split < row_tiles ? 1 : 0)  // (only whether any)
                           : (k0 < k1 ? (k1 - k0 + kKeyTile - 1) / kKeyTile : 0);

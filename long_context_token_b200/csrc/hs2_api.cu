@@ -26,6 +26,8 @@ constexpr int kChunk4 = 64;
 
 // The bounded-wait test hook (hs2_debug_stall_waits): copied into every full-layer launch.
 static int g_stall_test = 0;
+// hs2_set_deterministic: static key chunks in the full layer (no run-time tile sharing).
+static int g_deterministic = 0;
 
 // `row_ctas`: CTAs of one key chunk across the batch (one per (sequence, token) row,
 // or per group of G tokens in the several-token kernel).
@@ -201,6 +203,7 @@ static hs2_status run_full(const void* q, int n_q, int h, const hs2_kv* kv, int 
   p.part_ml = ws_ptr<float>(ws, w.part1_ml);
   p.status = ws_ptr<uint32_t>(ws, w.status);
   p.stall_test = g_stall_test;
+  p.deterministic = g_deterministic;
   if (fused_full_layer(kv, n_q, h)) {
     p.fuse = idx ? 2 : 1;
     p.out = out;
@@ -449,6 +452,8 @@ size_t hs2_workspace_bytes(int batch, int n_q, int h_q, int max_len, int window,
 }
 
 void hs2_debug_stall_waits(int mode) { g_stall_test = mode == 1 || mode == 2 ? mode : 0; }
+
+void hs2_set_deterministic(int on) { g_deterministic = on ? 1 : 0; }
 
 size_t hs2_workspace_lse64_offset(int batch, int n_q, int h_q, int max_len, int window,
                                   int k_sel, int dtype) {

@@ -108,6 +108,9 @@ struct FullParams {
   // kStallTestCycles; 2 = the fused tail's row barriers wait for one CTA more than the row
   // has, each giving up after kStallTestCycles.
   int stall_test = 0;
+  // Static key chunks per CTA (hs2_set_deterministic): results bitwise-reproducible across
+  // runs, at the cost of the run-time balancing of the row's tiles.
+  int deterministic = 0;
   float* lse_out = nullptr;      // [bq][h] or null
   double* lse64 = nullptr;       // [bq][h]
   float* ubuf = nullptr;         // [bq][ld_u]: per-key bound u_j = max_h x_hj (log2 units)

@@ -38,7 +38,7 @@ EXPORTS = ("hs2_workspace_bytes", "hs2_full_attn_select", "hs2_full_attn", "hs2_
            "hs2_last_cuda_error", "hs2_abi_version", "hs2_sparse_attn_noalloc", "hs2_kv_append",
            "hs2_full_attn_select_blocks", "hs2_select_blocks", "hs2_prefill_workspace_bytes",
            "hs2_prefill_attn", "hs2_select_fused", "hs2_workspace_lse64_offset",
-           "hs2_debug_stall_waits")
+           "hs2_debug_stall_waits", "hs2_set_deterministic")
 
 
 class Hs2Error(RuntimeError):
@@ -113,6 +113,8 @@ def lib():
     L.hs2_workspace_lse64_offset.restype = sz
     L.hs2_debug_stall_waits.argtypes = [i32]
     L.hs2_debug_stall_waits.restype = None
+    L.hs2_set_deterministic.argtypes = [i32]
+    L.hs2_set_deterministic.restype = None
     _lib = L
     return L
 
@@ -205,6 +207,11 @@ def default_scale() -> float:
 def select_fused(cache: "Cache", n_q: int, h_q: int) -> bool:
     """True if full_attn_select runs as one kernel for these sizes (hs2_select_fused)."""
     return bool(lib().hs2_select_fused(n_q, h_q, cache.dtype))
+
+
+def set_deterministic(on: bool) -> None:
+    """Static key chunks in the full layer: bitwise-reproducible runs (hs2_set_deterministic)."""
+    lib().hs2_set_deterministic(1 if on else 0)
 
 
 def workspace_lse64(workspace: torch.Tensor, cache: "Cache", n_q: int, h_q: int,
