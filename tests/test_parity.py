@@ -198,16 +198,20 @@ def test_repeat_runs_are_bitwise_identical_in_deterministic_mode(case):
 def test_repeat_runs_agree_within_rounding_by_default(case):
     """Run-time tile sharing regroups the float32 partial sums between runs: the index set
     stays the same (no key of these inputs sits within the lse's rounding of another) and
-    the outputs differ by rounding only."""
+    the outputs differ by rounding only -- for an FP8 cache also by the E4M3 split of P,
+    whose power-of-two scale follows the largest V scale among the tiles a CTA took
+    (values of P v_scale below 2^-6 of it are kept to 2^-18): far inside the 1e-2
+    tolerance, above float32 rounding."""
+    out_tol = 1e-6 if case["kv"] == "bf16" else 1e-4
     inp = workloads.make_inputs(2, 60000, n_q=1, h_q=16, kv=case["kv"], seed=case["seed"],
                                 n_sparse=1, lens=[60000, 47111])
     runs = [r for _ in range(3) for r in run_gpu(inp, twice=True)[0]]
     a = runs[0]
     for b in runs[1:]:
         assert np.array_equal(a["idx"], b["idx"])
-        assert np.abs(a["out"] - b["out"]).max() <= 1e-6
+        assert np.abs(a["out"] - b["out"]).max() <= out_tol
         assert np.abs(a["lse64"] - b["lse64"]).max() <= 1e-6
-        assert np.abs(a["sparse"][0] - b["sparse"][0]).max() <= 1e-6
+        assert np.abs(a["sparse"][0] - b["sparse"][0]).max() <= out_tol
     compare(inp, a)
 
 
