@@ -709,7 +709,13 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* scratch
   // ---- 4. the slot of this chunk's first selected position: the selections of the lower
   // chunks (their counts, and the band keys below k0 that the ranking takes)
   uint32_t below = 0, unused = 0;
-  for (int s2 = tid; s2 < split; s2 += nt) below += __ldcg(rowcnt + s2);
+  // (each count is only added once the band list's loads are also on their way)
+  uint32_t lower_cnt[(kSmCountBound + 127) / 128];
+#pragma unroll
+  for (int u = 0; u < (kSmCountBound + 127) / 128; ++u) {
+    const int s2 = tid + u * 128;
+    lower_cnt[u] = s2 < split && tid < 128 ? __ldcg(rowcnt + s2) : 0u;
+  }
   if (rank_band) {
     // Every CTA ranks the whole band by (key desc, position asc): the top need2 are in.
     // Those of this chunk are marked (~j) in its list.
@@ -731,15 +737,24 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* scratch
         bpos[e] = __ldcg(gbj + e);
       }
       __syncthreads();
-      for (int e = tid; e < nb; e += nt) {
+      // One warp per band key: its rank is the number of keys ahead of it (key desc,
+      // position asc), counted 32 at a time with a ballot.
+#pragma unroll 1
+      for (int e = warp; e < nb; e += nwarps) {
         const unsigned long long ke = bkey[e];
         const int je = bpos[e];
         int rank = 0;
-        for (int f = 0; f < nb; ++f) {
-          const unsigned long long kf2 = bkey[f];
-          rank += (kf2 > ke) || (kf2 == ke && bpos[f] < je);
+#pragma unroll 1
+        for (int f0 = 0; f0 < nb; f0 += 32) {
+          const int f = f0 + lane;
+          bool ahead = false;
+          if (f < nb) {
+            const unsigned long long kf2 = bkey[f];
+            ahead = (kf2 > ke) || (kf2 == ke && bpos[f] < je);
+          }
+          rank += __popc(__ballot_sync(0xffffffffu, ahead));
         }
-        if (rank < need2) take(je);
+        if (lane == 0 && rank < need2) take(je);
       }
     } else {
       // A large band (many equal keys): the boundary by radix select over the list.
@@ -759,6 +774,8 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* scratch
       }
     }
   }
+#pragma unroll
+  for (int u = 0; u < (kSmCountBound + 127) / 128; ++u) below += lower_cnt[u];
   block_sum2(below, unused);  // also orders the marks before the compaction reads them
   // This chunk's selected positions, in order, from slot `below`.
   block_compact(
@@ -779,14 +796,15 @@ __device__ __forceinline__ bool row_select(const FullParams& p, uint8_t* scratch
 }
 
 // The whole tail (fuse 1 or 2), called by every thread of every CTA after the stream,
-// with the CTA's partial written and (fuse 2) its u histogram in `uhist_s`.  NW: warps of
+// with the CTA's partial written, its m per head in `own_m` (shared memory; null for a
+// CTA that took no tile) and (fuse 2) its u histogram in `uhist_s`.  NW: warps of
 // the CTA.  The K/V stages (`stage`, `stage_bytes`) are idle; the first kTailTiles tiles
 // of `tile_bytes` take gathered K rows.  Returns false if a wait gave up.
 template <int H, bool FP8, int NW, typename Recompute>
 __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, uint32_t stage_bytes,
-                                           uint32_t tile_bytes, const uint32_t* uhist_s, int bq,
-                                           int b, int split, int pos, int k0, int k1,
-                                           const QView& qv, Recompute&& recompute) {
+                                           uint32_t tile_bytes, const uint32_t* uhist_s,
+                                           const float* own_m, int bq, int b, int split, int pos,
+                                           int k0, int k1, const QView& qv, Recompute&& recompute) {
   __shared__ RowLse<H> rl;
   const int S = p.splits1;
   const int n_c = pos - p.window + 1;
@@ -815,11 +833,11 @@ __device__ __forceinline__ bool fused_tail(const FullParams& p, uint8_t* stage, 
   static_assert(NW * 32 * 8 <= kTailTiles * 16384, "the tail's scratch fits the tiles' space");
   bool ok = true;
   __syncthreads();
-  if (threadIdx.x < H) {
-    // This CTA's m per head joins the row's maxima (the reference of the row's lse).
-    const float2 v = __ldcg(reinterpret_cast<const float2*>(p.part_ml) +
-                            ((size_t)bq * S + split) * H + threadIdx.x);
-    if (v.y > 0.f) atomicMax(rowmax + threadIdx.x, max_key(v.x));
+  if (threadIdx.x < H && own_m) {
+    // This CTA's m per head (the value of its partial, still on chip) joins the row's
+    // maxima, the reference of the row's lse.
+    const float m = own_m[threadIdx.x];
+    if (m > -INFINITY) atomicMax(rowmax + threadIdx.x, max_key(m));
   }
   if (sel_row) {
     // This CTA's u histogram added to the row's in one bulk reduction (its writes done

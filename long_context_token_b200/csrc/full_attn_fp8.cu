@@ -233,8 +233,14 @@ __device__ __noinline__ bool full_fp8_tail(const FullParams& p) {
   qv.base = reinterpret_cast<const uint8_t*>(p.q + (size_t)bq * H * kHeadDim);
   qv.hstride = kHeadDim * 2;  // bf16 rows [H][128] in global memory
   qv.cstride = 16;
+  // The partial's m per head is still in the softmax warps' reference array, unless the
+  // CTA took no tile (the same rule as the stream's).
+  const bool dyn = p.splits1 > 1 && !p.deterministic;
+  const bool took = dyn ? split < (pos + kKeyTile) / kKeyTile : k0 < k1;
+  const float* own_m = took ? reinterpret_cast<const float*>(smem + L::kRefOff) : nullptr;
   return fused_tail<H, true, fp8_threads<H>() / 32>(p, smem, 2u * R * kRawTile, kRawTile, uhist_s,
-                                                     bq, b, split, pos, k0, k1, qv, recompute);
+                                                     own_m, bq, b, split, pos, k0, k1, qv,
+                                                     recompute);
 }
 
 template <int H, bool GATHER>

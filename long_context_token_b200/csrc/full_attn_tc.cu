@@ -156,8 +156,13 @@ __device__ __noinline__ bool full_tc_tail(const FullParams& p) {
   qv.base = qs;         // Q as the MMA's K-major operand: chunk c of head h at
   qv.hstride = 16;      // c * H * 16 + h * 16
   qv.cstride = H * 16;
-  return fused_tail<H, false, 6>(p, smem, 2u * NS * L::kTile, L::kTile, uhist_s, bq, b, split, pos,
-                                 k0, k1, qv, recompute);
+  // The partial's m per head is still in the softmax warps' reference array, unless the
+  // CTA took no tile (the same rule as the stream's).
+  const bool dyn = p.splits1 > 1 && !p.deterministic;
+  const bool took = dyn ? split < (pos + kKeyTile) / kKeyTile : k0 < k1;
+  const float* own_m = took ? reinterpret_cast<const float*>(smem + L::kRefOff) : nullptr;
+  return fused_tail<H, false, 6>(p, smem, 2u * NS * L::kTile, L::kTile, uhist_s, own_m, bq, b,
+                                 split, pos, k0, k1, qv, recompute);
 }
 
 template <int H, bool GATHER>
