@@ -122,77 +122,101 @@ static __device__ __noinline__ bool row_wait(uint32_t* counter, uint32_t target,
 
 // The bin B holding the k-th largest element of a dense shared-memory histogram (0 if
 // there are fewer than k), and with mb > 0 the counts in the bins >= B + mb (`above`)
-// and in [B - mb, B + mb) (`near`).  Warp 0 scans: lane l owns the bins [kUBins - 64(l +
-// 1), kUBins - 64 l), 16 chunks of 4, which it sums starting at chunk l mod 16 so that the
-// lanes' 16-byte loads meet at most 4-way bank conflicts.  Every thread calls it and gets
-// the result.  The tail runs this code once per launch, so it is one
-// out-of-line copy with rolled loops: fetching instructions that run once costs more
-// than executing them.
+// and in [B - mb, B + mb) (`near`).  Threads t < 128 own the bins [kUBins - 16(t + 1),
+// kUBins - 16 t) (thread 0 the top ones), read as four 16-byte chunks starting at chunk
+// t mod 4 so that a warp's loads meet at most 4-way bank conflicts; one block-wide scan
+// from the top finds the owner of the k-th element, which walks its 16 bins.  Every
+// thread calls it (blockDim >= 128) and gets the result.  The tail runs this code once
+// per launch and histogram, so it is one out-of-line copy.
 struct BinScan {
   int bin;
   uint32_t above, near;
 };
 static __device__ __noinline__ BinScan scan_bins(const uint32_t* hs, int k, int mb) {
-  static_assert(kUBins == 32 * 64, "64 bins per lane");
+  static_assert(kUBins == 128 * 16, "16 bins per scanning thread");
+  __shared__ uint32_t wtot[4];
+  __shared__ uint32_t wsum2[2][4];
   __shared__ BinScan out_s;
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    const int base = kUBins - 64 * (lane + 1);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool own = tid < 128;
+  const int base = kUBins - 16 * (tid + 1);
+  uint32_t v[16];  // v[4c + q]: bin base + 4c + q
+  uint32_t sum = 0;
+  if (own) {
     const uint4* row = reinterpret_cast<const uint4*>(hs + base);
-    uint32_t sum = 0;
-#pragma unroll 1
-    for (int u = 0; u < 16; ++u) {
-      const uint4 c = row[(u + lane) & 15];
-      sum += (c.x + c.y) + (c.z + c.w);
-    }
-    uint32_t incl = sum;
-#pragma unroll 1
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += x;
-    }
-    const uint32_t before = incl - sum;  // in the bins above this lane's
-    int bin = -1;
-    if (before < (uint32_t)k && (uint32_t)k <= incl) {
-      uint32_t cum = before;
-#pragma unroll 1
-      for (int u = 15; u >= 0 && bin < 0; --u) {
-        const uint4 c = row[u];
-        const uint32_t v[4] = {c.x, c.y, c.z, c.w};
+    uint4 c[4];
 #pragma unroll
-        for (int q = 3; q >= 0; --q) {
-          cum += v[q];
-          if (bin < 0 && cum >= (uint32_t)k) bin = base + 4 * u + q;
+    for (int u = 0; u < 4; ++u) c[u] = row[(u + tid) & 3];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int ch = (u + tid) & 3;
+#pragma unroll
+      for (int ch2 = 0; ch2 < 4; ++ch2)
+        if (ch == ch2) {
+          v[4 * ch2] = c[u].x;
+          v[4 * ch2 + 1] = c[u].y;
+          v[4 * ch2 + 2] = c[u].z;
+          v[4 * ch2 + 3] = c[u].w;
         }
+    }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) sum += v[e];
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] = 0u;
+  }
+  uint32_t incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  if (own && lane == 31) wtot[warp] = incl;
+  if (tid == 0) out_s.bin = 0;
+  __syncthreads();
+  uint32_t before = incl - sum;  // in the bins above this thread's
+  for (int w = 0; w < warp && w < 4; ++w) before += wtot[w];
+  if (own && before < (uint32_t)k && (uint32_t)k <= before + sum) {
+    uint32_t cum = before;
+    int bin = base;
+#pragma unroll
+    for (int e = 15; e >= 0; --e) {
+      cum += v[e];
+      if (cum >= (uint32_t)k) {
+        bin = base + e;
+        break;
       }
     }
-    const unsigned found = __ballot_sync(0xffffffffu, bin >= 0);
-    const int B = found ? __shfl_sync(0xffffffffu, bin, __ffs(found) - 1) : 0;
-    uint32_t above = 0, near = 0;
-    if (mb > 0) {
-#pragma unroll 1
-      for (int u0 = 0; u0 < 16; ++u0) {
-        const int u = (u0 + lane) & 15;
-        const uint4 c = row[u];
-        const uint32_t v[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int e = base + 4 * u + q;
-          above += e >= B + mb ? v[q] : 0u;
-          near += (e >= B - mb && e < B + mb) ? v[q] : 0u;
-        }
-      }
-      above = __reduce_add_sync(0xffffffffu, above);
-      near = __reduce_add_sync(0xffffffffu, near);
-    }
-    if (lane == 0) {
-      out_s.bin = B;
-      out_s.above = above;
-      out_s.near = near;
-    }
+    out_s.bin = bin;
   }
   __syncthreads();
-  return out_s;
+  BinScan r;
+  r.bin = out_s.bin;
+  r.above = 0u;
+  r.near = 0u;
+  if (mb > 0) {
+    const int B = r.bin;
+    uint32_t above = 0, near = 0;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int bb = base + e;
+      above += bb >= B + mb ? v[e] : 0u;
+      near += (bb >= B - mb && bb < B + mb) ? v[e] : 0u;
+    }
+    above = __reduce_add_sync(0xffffffffu, above);
+    near = __reduce_add_sync(0xffffffffu, near);
+    if (own && lane == 0) {
+      wsum2[0][warp] = above;
+      wsum2[1][warp] = near;
+    }
+    __syncthreads();
+    r.above = (wsum2[0][0] + wsum2[0][1]) + (wsum2[0][2] + wsum2[0][3]);
+    r.near = (wsum2[1][0] + wsum2[1][1]) + (wsum2[1][2] + wsum2[1][3]);
+    __syncthreads();  // wsum2 and out_s are reused by the next call
+  } else {
+    __syncthreads();
+  }
+  return r;
 }
 
 // Asynchronous copies (cp.async, waited for with cp_async_wait_all) by all threads:
