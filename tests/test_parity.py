@@ -140,6 +140,30 @@ SMALL = [
 ]
 
 
+def test_long_chunks_in_several_pieces_match_oracle():
+    """74 sequences of up to 32768 keys: two CTAs a row, so each CTA's chunk (16384 keys)
+    is longer than the on-chip piece of the fused selection's bounds, and the candidates
+    of a chunk are kept in the row's candidate buffer instead of on chip."""
+    lens = [32768 - 37 * i for i in range(74)]
+    inp = workloads.make_inputs(74, 32768, n_q=1, h_q=16, kv="bf16", seed=125, lens=lens,
+                                n_sparse=1)
+    runs, status = run_gpu(inp)
+    assert status == 0
+    compare(inp, runs[0])
+
+
+def test_long_chunks_with_all_keys_tied_match_oracle():
+    """A zero query over long chunks: every key of a row ties, so the whole row is the band
+    -- each CTA re-scores its ~16000 band keys in rounds of at most 512 on chip, and the
+    band is ranked by the radix fallback; the lowest positions win the ties."""
+    lens = [32768 - 37 * i for i in range(74)]
+    inp = workloads.make_inputs(74, 32768, n_q=1, h_q=16, kv="bf16", seed=126, lens=lens,
+                                n_sparse=1, q_zero=True)
+    runs, status = run_gpu(inp)
+    assert status == 0
+    compare(inp, runs[0])
+
+
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: c["id"])
 def test_small_cases_match_oracle(case):
     kw = {k: v for k, v in case.items() if k != "id"}
