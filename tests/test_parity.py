@@ -482,6 +482,27 @@ def test_block_selection_zero_query_keeps_lowest_blocks(kv):
     assert res["idx"][0, 0].tolist() == want.tolist()
 
 
+@pytest.mark.parametrize("kv,h_q", [("bf16", 16), ("fp8", 64)])
+def test_separate_full_layer_and_selection_match_oracle(kv, h_q):
+    """hs2_full_attn then hs2_select (the two halves of hs2_full_attn_select) on one
+    60000-key row: the full layer's CTAs share the row's tiles out at run time (the stored
+    logits of the 16-head step are indexed by position, whoever computed them)."""
+    dev = torch.device("cuda:0")
+    inp = workloads.make_inputs(1, 60000, n_q=1, h_q=h_q, kv=kv, seed=213, n_sparse=1)
+    cache = hs2.Cache(inp.k.to(dev), inp.v.to(dev), inp.lens.to(dev),
+                      None if inp.k_scale is None else inp.k_scale.to(dev),
+                      None if inp.v_scale is None else inp.v_scale.to(dev))
+    ws = hs2.alloc_workspace(cache, 1, h_q)
+    q = inp.q.to(dev)
+    lse = torch.empty(1, 1, h_q, dtype=torch.float32, device=dev)
+    out = hs2.full_attn(q, cache, 128, 1024, inp.sm_scale, ws, lse=lse)
+    idx = hs2.select(q, cache, ws, 128, 1024, inp.sm_scale)
+    sp = [hs2.sparse_attn(inp.q_layers[0].to(dev), cache, idx, ws, inp.sm_scale)]
+    assert hs2.check_device_status(ws) == 0
+    compare(inp, dict(out=out.cpu().numpy(), idx=idx.cpu().numpy(), lse=lse.cpu().numpy(),
+                      sparse=[x.cpu().numpy() for x in sp]))
+
+
 def test_block_then_token_selection_share_a_workspace():
     """Block mode leaves the selection state clean: a token-level call on the same
     workspace right after it still matches the oracle."""
