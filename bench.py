@@ -238,7 +238,7 @@ def run_reference(args, w):
                 "value = sequences/s / batch",
         "sequences_timed": seqs, "seconds_timed": secs,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_of(w, args.block),
+        "data": "synthetic", "config": config_of(w, args.block, args.deterministic),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
                          "sample": f"{seqs} whole sequences of the batch, one per step, "
                                    "full layer + selection + every sparse layer in float64"},
@@ -382,11 +382,17 @@ def run_prefill(args, w):
     print(json.dumps(line), flush=True)
 
 
-def config_of(w, block: int = 1):
+def config_of(w, block: int = 1, deterministic: bool = False):
+    # The one-launch full layer (one token per row, up to 64 heads; any FP8 shape up to 64
+    # heads) shares each row's key tiles out at run time unless asked for fixed chunks.
+    one_launch = w.h_q <= 64 and (w.kv == "fp8" or w.n_q == 1)
+    shared = one_launch and not deterministic
     return {"workload": w.name, "batch": w.batch, "context": w.max_len,
             "selection": "token" if block == 1 else f"blocks of {block} positions",
             "ragged_from": w.len_lo, "n_q": w.n_q, "h_q": w.h_q, "h_kv": 1, "head_dim": 128,
             "kv_cache": w.kv, "window": w.window, "k_sel": w.k_sel, "sparse_layers": w.n_sparse,
+            "key_tiles": ("shared out among a row's CTAs at run time" if shared
+                          else "fixed chunks per CTA (bitwise-reproducible runs)"),
             "l2": "flushed before every timed step (256 MiB write, then 256 MiB read of "
                   "another buffer)"}
 
@@ -402,6 +408,8 @@ def main():
                     help="seconds of oracle time for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="fixed key chunks per CTA in the full layer (hs2_set_deterministic)")
     ap.add_argument("--block", type=int, default=1,
                     help="1: token-level selection (the method); N > 1: whole blocks of N "
                          "positions (the first-generation comparator)")
@@ -440,6 +448,7 @@ def main():
     n_layers = len(inp.q_layers)
     ws = hs2.alloc_workspace(cache, n_q, h, w.window, w.k_sel)
     fused = args.block == 1 and hs2.select_fused(cache, n_q, h)
+    hs2.set_deterministic(args.deterministic)
     # Every input of a step (the full layer's queries, then each sparse layer's) sits in
     # one device buffer, and every result (the full layer's output, each sparse layer's
     # output, then the index set) in another, so that the end-to-end leg moves each with
@@ -651,7 +660,7 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.kv == "bf16" else "fp8-e4m3",
-        "data": "synthetic", "config": config_of(w, args.block),
+        "data": "synthetic", "config": config_of(w, args.block, args.deterministic),
         "hbm_gbs": ab["step"] / (total_ms / args.steps / 1e3) / 1e9,
         "alg_bytes_per_step": ab["step"],
         "phase_ms": phases | {"sparse_layers": statistics.mean(sp_ms),

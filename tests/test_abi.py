@@ -50,6 +50,19 @@ def test_workspace_sizes_for_every_workload(L, n):
     assert w.batch * w.n_q * w.max_len * 4 < b < 2 ** 30
 
 
+@pytest.mark.parametrize("n", sorted(workloads.WORKLOADS))
+def test_lse64_offset_lies_inside_the_workspace(L, n):
+    """The float64 lse the selection uses: 8-byte aligned, [batch][n_q][h_q] doubles inside
+    the workspace, and (size_t)-1 for unsupported sizes."""
+    w = workloads.WORKLOADS[n]
+    args = (w.batch, w.n_q, w.h_q, w.max_len, 128, 1024, int(w.kv == "fp8"))
+    total = L.hs2_workspace_bytes(*args)
+    off = L.hs2_workspace_lse64_offset(*args)
+    assert off % 8 == 0
+    assert off + w.batch * w.n_q * w.h_q * 8 <= total
+    assert L.hs2_workspace_lse64_offset(1, 1, 24, 4096, 128, 1024, 0) == 2 ** 64 - 1
+
+
 @pytest.mark.parametrize("args", [
     (1, 1, 24, 4096, 128, 1024, 0),    # h_q not a multiple of 16
     (1, 1, 144, 4096, 128, 1024, 0),   # h_q > 128
