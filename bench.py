@@ -298,9 +298,11 @@ def run_prefill(args, w):
     with ClockSampler(dev) as clk:
         for k in range(args.steps):
             flush_l2(k)
+            torch.cuda.nvtx.range_push("hs2 step")
             start.record(stream)
             graph.replay()
             end.record(stream)
+            torch.cuda.nvtx.range_pop()
             end.synchronize()
             replay_ms.append(start.elapsed_time(end))
     wall = time.perf_counter() - wall0
@@ -349,9 +351,11 @@ def run_prefill(args, w):
         e_ms = 0.0
         for k in range(args.steps):
             flush_l2(k)
+            torch.cuda.nvtx.range_push("hs2 step end to end")
             start.record(stream)
             g2.replay()
             end.record(stream)
+            torch.cuda.nvtx.range_pop()
             end.synchronize()
             e_ms += start.elapsed_time(end)
         line["e2e"] = {"value": tokens * args.steps / (e_ms / 1e3), "unit": "tokens/s",
@@ -564,9 +568,11 @@ def main():
     with ClockSampler(dev) as clk:
         for k in range(args.steps):
             flush_l2(k)
+            torch.cuda.nvtx.range_push("hs2 step")
             start.record(stream)
             graph.replay()
             end.record(stream)
+            torch.cuda.nvtx.range_pop()
             end.synchronize()
             replay_ms.append(start.elapsed_time(end))
         if world > 1:
@@ -574,7 +580,9 @@ def main():
         wall = time.perf_counter() - wall0
         for k in range(args.steps):
             flush_l2(k)
+            torch.cuda.nvtx.range_push("hs2 step with phase marks")
             graph_marked.replay()
+            torch.cuda.nvtx.range_pop()
             end.record(stream)
             end.synchronize()
             step_ms.append(elapsed(0, 3))
@@ -620,9 +628,11 @@ def main():
         e_ms = 0.0
         for k in range(args.steps):
             flush_l2(k)
+            torch.cuda.nvtx.range_push("hs2 step end to end")
             start.record(stream)
             g2.replay()
             end.record(stream)
+            torch.cuda.nvtx.range_pop()
             end.synchronize()
             e_ms += start.elapsed_time(end)
         e_ms = max_over_ranks(e_ms, dev)
