@@ -11,10 +11,11 @@
 // stream each key records only the bound
 //     u_j = max_h x_hj,     u_j - W <= t_j <= u_j,     W = max_h D_h,
 // and counts u_j in a shared-memory histogram, linear in u.  Then, per row (CTA r of the
-// row owns the positions [r chunk, (r + 1) chunk) for the selection):
-//   1. every CTA publishes its histogram and arrives at the row's first barrier (its own
-//      bounds already on their way into shared memory), then computes the row's lse from
-//      the split partials;
+// row owns the positions [r chunk, (r + 1) chunk) for the selection, whichever CTA
+// streamed them):
+//   1. every CTA publishes its m per head and its histogram and arrives at the row's first
+//      barrier, then copies its chunk's bounds and the row's histogram on chip and computes
+//      the row's lse from the split partials;
 //   2. the bin holding the k_sel-th largest u gives a lower edge lo; no key with
 //      u_j < lo - W - 2 eps can be among the top k_sel (the k_sel-th largest t, T, is at
 //      least lo - W), so only the other keys of its chunk -- the candidates, a few per
