@@ -126,7 +126,14 @@ HS2_API size_t hs2_workspace_lse64_offset(int batch, int n_q, int h_q, int max_l
  *            all of [0, p]; unused slots are -1.
  *   lse      device float32 [batch][n_q][h_q] natural-log sum-exp of the logits,
  *            or NULL.
- * Equivalent to hs2_full_attn followed by hs2_select on the same workspace. */
+ * Equivalent to hs2_full_attn followed by hs2_select on the same workspace.  For one new
+ * token per sequence on a bf16 cache and for an FP8 cache, with h_q <= 64
+ * (hs2_select_fused), it is a single cooperative kernel: the full layer's CTAs merge
+ * their split partials and select the tokens in its tail, re-scoring only the keys whose
+ * bound u_j = max_h s_hj can reach the top k_sel, so K is read once.  The index set is
+ * the same either way outside the tie band (keys whose exact importances differ by less
+ * than the lse's rounding); outputs can differ between runs in their last bits unless
+ * hs2_set_deterministic is on. */
 HS2_API hs2_status hs2_full_attn_select(const void* q, int n_q, int h_q, const hs2_kv* kv,
                                 int window, int k_sel, float sm_scale, float* out,
                                 int32_t* idx, float* lse, void* workspace,
